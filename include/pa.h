@@ -1,0 +1,171 @@
+/*
+ * pa.h -- C ABI of libpa, the B200 (sm_100a) paged decode-attention library.
+ *
+ * The operations follow the pages on vLLM's PagedAttention:
+ *  - "vllm源码剖析" (jsqmd.com/news/690568) §一.2 "为什么要reshape": the KV
+ *    cache is [num_blocks, block_size, num_kv_heads, head_size], addressed per
+ *    token through the flat view [num_blocks*block_size, num_kv_heads,
+ *    head_size]; §一.3 "token和请求块的映射": a token's slot is its block id
+ *    times block_size plus its offset (index mod block_size).
+ *  - "vLLM PagedAttention 原理与源码深度解析" (toukenai.cn) §3.1: a per-sequence
+ *    block table maps logical blocks to physical blocks; §5.3 "注意力计算":
+ *    forward(q, kv_cache, block_tables, context_lens) gathers K/V through the
+ *    block tables and returns softmax(q.k * scale) . v per query head.
+ *  - "vllm源码分析：…PagedAttention核心实现" (vergex.cn/9743.html) §第三讲:
+ *    logical block i of a sequence is read from physical block block_table[i].
+ *
+ * Conventions shared by every entry point:
+ *  - Every buffer argument is a DEVICE pointer owned by the caller.  The
+ *    library allocates no memory, never synchronises (except
+ *    pa_check_error), and keeps no per-call state.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously; the returned status covers argument
+ *    validation and launch errors only.
+ *  - 16-bit element type `dtype`: PA_F16 (IEEE binary16) or PA_BF16.  Query,
+ *    caches, new K/V and the output all share it.
+ *  - All tensors are dense row-major with the layouts stated per call; every
+ *    pointer to 16-bit data must be 16-byte aligned and head_dim a multiple of 8.
+ *  - Query head h reads KV head h / (num_heads / num_kv_heads) (consecutive
+ *    grouping, as in Llama-style GQA).
+ *  - context_lens[s] counts the tokens sequence s attends to, including a
+ *    token written this step by pa_reshape_and_cache (call it first, on the
+ *    same stream).  context_lens[s] == 0 yields an all-zero output row.
+ *  - Only block_tables[s][0 .. ceil(context_lens[s]/block_size)-1] are read.
+ *  - Kernels check every block id, slot and context length they read.  An
+ *    out-of-range value never causes an out-of-bounds access: the access is
+ *    skipped (reads return zeros), and the first such event is recorded in a
+ *    per-device error word that pa_check_error reports.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_NULL = 1,        /* a required pointer is NULL */
+    PA_ERR_SHAPE = 2,       /* a size is out of range or sizes disagree */
+    PA_ERR_DTYPE = 3,       /* unknown element type */
+    PA_ERR_ALIGN = 4,       /* a pointer or row stride is not 16-byte aligned */
+    PA_ERR_UNSUPPORTED = 5, /* valid, but not built: head_dim, block_size, partition size */
+    PA_ERR_CUDA = 6,        /* a CUDA call failed (no device, launch, tensor map) */
+    PA_ERR_BOUNDS = 7       /* pa_check_error: a kernel met an out-of-range index */
+} pa_status;
+
+typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Codes stored in the top 8 bits of the detail word of pa_check_error;
+ * the low 56 bits hold the offending index (see each code). */
+enum {
+    PA_CHECK_SLOT = 1,          /* slot_mapping[t] >= num_blocks*block_size; index = t */
+    PA_CHECK_BLOCK_ID = 2,      /* block id outside [0, num_blocks); index = s*max_blocks_per_seq + i */
+    PA_CHECK_CONTEXT_LEN = 3,   /* context_lens[s] < 0 or > max_blocks_per_seq*block_size; index = s */
+    PA_CHECK_PARTITIONS = 4,    /* ceil(context_lens[s]/partition_size) > max_partitions; index = s */
+    PA_CHECK_WAIT_TIMEOUT = 5   /* a shared-memory barrier wait gave up; index = CTA id */
+};
+
+/* Short English name of a status code (static string, never NULL). */
+const char *pa_status_string(pa_status status);
+
+/* ABI version of this header: (major << 16) | minor. */
+int32_t pa_abi_version(void);
+
+/*
+ * pa_reshape_and_cache -- write this step's new K/V rows into the paged caches.
+ * ("vllm源码剖析" §一.2 and §一.3.)
+ *   key, value     [num_tokens, num_kv_heads, head_dim], consecutive tokens
+ *                  key_stride / value_stride ELEMENTS apart (>= num_kv_heads*head_dim,
+ *                  a multiple of 8); inside a token row the layout is dense.
+ *   key_cache, value_cache
+ *                  [num_blocks, block_size, num_kv_heads, head_dim] (dense).
+ *   slot_mapping   [num_tokens] int64: flat slot = block_id*block_size + offset;
+ *                  a negative slot marks a padding token and is skipped.
+ * For every token t with slot >= 0: key_cache_flat[slot] = key[t] and
+ * value_cache_flat[slot] = value[t], bit for bit.  Slots must be distinct.
+ * block_size may be any positive value here.  num_tokens == 0 is a no-op.
+ */
+pa_status pa_reshape_and_cache(const void *key, const void *value,
+                               int64_t key_stride, int64_t value_stride,
+                               void *key_cache, void *value_cache,
+                               const int64_t *slot_mapping, int64_t num_tokens,
+                               int64_t num_kv_heads, int64_t head_dim,
+                               int64_t num_blocks, int64_t block_size,
+                               pa_dtype dtype, void *stream);
+
+/*
+ * pa_decode -- single-pass paged decode attention, one query token per sequence.
+ * ("vLLM PagedAttention 原理与源码深度解析" §5.3.)
+ *   out            [num_seqs, num_heads, head_dim]       (written)
+ *   query          [num_seqs, num_heads, head_dim]
+ *   key_cache, value_cache  [num_blocks, block_size, num_kv_heads, head_dim]
+ *   block_tables   [num_seqs, max_blocks_per_seq] int32
+ *   context_lens   [num_seqs] int32
+ *   scale          multiplies q.k before the softmax (1/sqrt(head_dim) on the page)
+ * out[s,h,:] = sum_j softmax_j(scale * q[s,h,:] . k_j) v_j over the first
+ * context_lens[s] tokens of sequence s, computed with fp32 accumulation and
+ * rounded to dtype (nearest even).
+ * Built for head_dim in {64, 128}, block_size == 16, num_heads % num_kv_heads == 0.
+ */
+pa_status pa_decode(void *out, const void *query,
+                    const void *key_cache, const void *value_cache,
+                    const int32_t *block_tables, const int32_t *context_lens,
+                    float scale, int64_t num_seqs, int64_t num_heads,
+                    int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                    int64_t block_size, int64_t max_blocks_per_seq,
+                    pa_dtype dtype, void *stream);
+
+/*
+ * pa_decode_split -- the same attention cut into partitions of partition_size
+ * logical tokens (partition p covers tokens [p*P, (p+1)*P) of [0, ctx)), for
+ * long contexts.  The pages do not describe this split; its merge is the
+ * log-sum-exp identity applied by pa_reduce.
+ *   tmp_out     [num_seqs, num_heads, max_partitions, head_dim] fp32 (written)
+ *   max_logits  [num_seqs, num_heads, max_partitions] fp32 (written)
+ *   exp_sums    [num_seqs, num_heads, max_partitions] fp32 (written)
+ * For every partition p < ceil(ctx/partition_size), with z_j = scale*q.k_j:
+ *   max_logits = max_j z_j,  exp_sums = sum_j exp(z_j - max),
+ *   tmp_out    = sum_j exp(z_j - max) v_j        (not normalised).
+ * Entries of partitions >= ceil(ctx/partition_size) are not written.
+ * partition_size must be a positive multiple of block_size; the caller
+ * guarantees ceil(ctx/partition_size) <= max_partitions (checked on device).
+ * The three fp32 buffers are caller-owned scratch that pa_reduce consumes.
+ */
+pa_status pa_decode_split(float *tmp_out, float *max_logits, float *exp_sums,
+                          const void *query, const void *key_cache,
+                          const void *value_cache, const int32_t *block_tables,
+                          const int32_t *context_lens, float scale,
+                          int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads,
+                          int64_t head_dim, int64_t num_blocks, int64_t block_size,
+                          int64_t max_blocks_per_seq, int64_t partition_size,
+                          int64_t max_partitions, pa_dtype dtype, void *stream);
+
+/*
+ * pa_reduce -- merge the partitions written by pa_decode_split:
+ *   M = max_p max_logits[p],  w_p = exp(max_logits[p] - M),
+ *   out = (sum_p w_p tmp_out[p]) / (sum_p w_p exp_sums[p])
+ * over p < ceil(context_lens[s]/partition_size); ctx == 0 gives zeros.
+ *   out  [num_seqs, num_heads, head_dim] dtype (written)
+ */
+pa_status pa_reduce(void *out, const float *tmp_out, const float *max_logits,
+                    const float *exp_sums, const int32_t *context_lens,
+                    int64_t num_seqs, int64_t num_heads, int64_t head_dim,
+                    int64_t partition_size, int64_t max_partitions,
+                    pa_dtype dtype, void *stream);
+
+/*
+ * pa_check_error -- synchronise `stream`, read and clear the current device's
+ * error word.  Returns PA_OK if no kernel recorded a problem since the last
+ * call, PA_ERR_BOUNDS otherwise (then *detail, if not NULL, receives
+ * (code << 56) | index with a PA_CHECK_* code), or PA_ERR_CUDA.
+ */
+pa_status pa_check_error(void *stream, int64_t *detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,210 @@
+"""ctypes binding of libpa (include/pa.h): argument marshalling only.
+
+Every function here takes torch CUDA tensors, checks that their dtype,
+device and layout match what the C entry point expects, and passes raw
+pointers, sizes and the current CUDA stream.  All arithmetic runs in the
+library's kernels; there is no fallback.  If libpa.so is missing the first
+call raises ``PagedAttentionError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import re
+from pathlib import Path
+
+import torch
+
+from . import build as _build
+
+LIBRARY = _build.LIBRARY
+HEADER = _build.INCLUDE / "pa.h"
+
+PA_OK = 0
+STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_NULL", 2: "PA_ERR_SHAPE", 3: "PA_ERR_DTYPE",
+                4: "PA_ERR_ALIGN", 5: "PA_ERR_UNSUPPORTED", 6: "PA_ERR_CUDA",
+                7: "PA_ERR_BOUNDS"}
+CHECK_CODES = {1: "slot", 2: "block_id", 3: "context_len", 4: "partitions", 5: "wait_timeout"}
+DTYPE_CODES = {torch.float16: 0, torch.bfloat16: 1}
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, status: int, what: str, detail: int | None = None):
+        self.status = status
+        self.detail = detail
+        msg = f"{what}: {STATUS_NAMES.get(status, status)}"
+        if detail:
+            msg += (f" (device check {CHECK_CODES.get(detail >> 56, detail >> 56)}, "
+                    f"index {detail & ((1 << 56) - 1)})")
+        super().__init__(msg)
+
+
+_i64 = ctypes.c_int64
+_p = ctypes.c_void_p
+_f = ctypes.c_float
+_i = ctypes.c_int
+
+# name -> (restype, argtypes); the order is the header's.
+SIGNATURES = {
+    "pa_status_string": (ctypes.c_char_p, [_i]),
+    "pa_abi_version": (ctypes.c_int32, []),
+    "pa_reshape_and_cache": (_i, [_p, _p, _i64, _i64, _p, _p, _p, _i64, _i64, _i64, _i64, _i64,
+                                  _i, _p]),
+    "pa_decode": (_i, [_p, _p, _p, _p, _p, _p, _f, _i64, _i64, _i64, _i64, _i64, _i64, _i64,
+                       _i, _p]),
+    "pa_decode_split": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _f, _i64, _i64, _i64, _i64, _i64,
+                             _i64, _i64, _i64, _i64, _i, _p]),
+    "pa_reduce": (_i, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i, _p]),
+    "pa_check_error": (_i, [_p, ctypes.POINTER(_i64)]),
+}
+
+_lib: ctypes.CDLL | None = None
+
+
+def load(path: Path | str | None = None) -> ctypes.CDLL:
+    """Load libpa.so (built in-tree by ``build.build()``) and bind signatures."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = Path(path) if path else LIBRARY
+    if not p.exists():
+        raise PagedAttentionError(6, f"libpa.so not found at {p}; run "
+                                     "`python -m paged_kv_cache_444_b200.build`")
+    lib = ctypes.CDLL(str(p))
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/pa.h declares."""
+    text = HEADER.read_text(encoding="utf-8")
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return load().pa_status_string(status).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != PA_OK:
+        raise PagedAttentionError(status, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in DTYPE_CODES:
+        raise TypeError(f"expected float16 or bfloat16, got {t.dtype}")
+    return DTYPE_CODES[t.dtype]
+
+
+def _need(cond: bool, msg: str) -> None:
+    if not cond:
+        raise ValueError(msg)
+
+
+# ---------------------------------------------------------------------------
+# One wrapper per C entry point, same names
+# ---------------------------------------------------------------------------
+def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
+                         value_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                         stream=None) -> None:
+    """key/value [T, Hk, D] (token rows may be strided), caches
+    [NB, bs, Hk, D] contiguous, slot_mapping [T] int64 on the device."""
+    T, Hk, D = key.shape
+    NB, bs = key_cache.shape[0], key_cache.shape[1]
+    _need(value.shape == key.shape, "key/value shapes differ")
+    _need(key_cache.shape == (NB, bs, Hk, D) and value_cache.shape == key_cache.shape,
+          "cache shape must be [num_blocks, block_size, num_kv_heads, head_dim]")
+    _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
+    _need(key.stride()[1:] == (D, 1) and value.stride()[1:] == (D, 1),
+          "key/value token rows must be dense")
+    _need(slot_mapping.dtype == torch.int64 and slot_mapping.shape == (T,), "slot_mapping [T] int64")
+    dt = _dtype_code(key)
+    _need(value.dtype == key.dtype == key_cache.dtype == value_cache.dtype, "dtype mismatch")
+    st = load().pa_reshape_and_cache(
+        key.data_ptr(), value.data_ptr(), key.stride(0) if T else Hk * D,
+        value.stride(0) if T else Hk * D, key_cache.data_ptr(), value_cache.data_ptr(),
+        slot_mapping.data_ptr(), T, Hk, D, NB, bs, dt, _stream(stream))
+    _check(st, "pa_reshape_and_cache")
+
+
+def _attention_common(query, key_cache, value_cache, block_tables, context_lens):
+    S, H, D = query.shape
+    NB, bs, Hk, D2 = key_cache.shape
+    _need(D2 == D, "head_dim of query and cache differ")
+    _need(value_cache.shape == key_cache.shape, "key/value cache shapes differ")
+    _need(query.is_contiguous() and key_cache.is_contiguous() and value_cache.is_contiguous(),
+          "query and caches must be contiguous")
+    _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
+          block_tables.shape[0] == S and block_tables.is_contiguous(),
+          "block_tables must be [num_seqs, max_blocks] int32 contiguous")
+    _need(context_lens.dtype == torch.int32 and context_lens.shape == (S,),
+          "context_lens must be [num_seqs] int32")
+    _need(query.dtype == key_cache.dtype == value_cache.dtype, "dtype mismatch")
+    return S, H, D, NB, bs, Hk, block_tables.shape[1], _dtype_code(query)
+
+
+def pa_decode(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+              value_cache: torch.Tensor, block_tables: torch.Tensor,
+              context_lens: torch.Tensor, scale: float, stream=None) -> None:
+    S, H, D, NB, bs, Hk, MB, dt = _attention_common(query, key_cache, value_cache,
+                                                    block_tables, context_lens)
+    _need(out.shape == query.shape and out.dtype == query.dtype and out.is_contiguous(),
+          "out must match query")
+    st = load().pa_decode(out.data_ptr(), query.data_ptr(), key_cache.data_ptr(),
+                          value_cache.data_ptr(), block_tables.data_ptr(),
+                          context_lens.data_ptr(), float(scale), S, H, Hk, D, NB, bs, MB, dt,
+                          _stream(stream))
+    _check(st, "pa_decode")
+
+
+def pa_decode_split(tmp_out: torch.Tensor, max_logits: torch.Tensor, exp_sums: torch.Tensor,
+                    query: torch.Tensor, key_cache: torch.Tensor, value_cache: torch.Tensor,
+                    block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                    partition_size: int, stream=None) -> None:
+    S, H, D, NB, bs, Hk, MB, dt = _attention_common(query, key_cache, value_cache,
+                                                    block_tables, context_lens)
+    P = max_logits.shape[-1]
+    _need(tmp_out.shape == (S, H, P, D) and tmp_out.dtype == torch.float32
+          and tmp_out.is_contiguous(), "tmp_out must be [S, H, P, D] float32")
+    _need(max_logits.shape == (S, H, P) and exp_sums.shape == (S, H, P) and
+          max_logits.dtype == exp_sums.dtype == torch.float32, "max_logits/exp_sums [S, H, P] f32")
+    st = load().pa_decode_split(tmp_out.data_ptr(), max_logits.data_ptr(), exp_sums.data_ptr(),
+                                query.data_ptr(), key_cache.data_ptr(), value_cache.data_ptr(),
+                                block_tables.data_ptr(), context_lens.data_ptr(), float(scale),
+                                S, H, Hk, D, NB, bs, MB, int(partition_size), P, dt,
+                                _stream(stream))
+    _check(st, "pa_decode_split")
+
+
+def pa_reduce(out: torch.Tensor, tmp_out: torch.Tensor, max_logits: torch.Tensor,
+              exp_sums: torch.Tensor, context_lens: torch.Tensor, partition_size: int,
+              stream=None) -> None:
+    S, H, P, D = tmp_out.shape
+    _need(out.shape == (S, H, D) and out.is_contiguous(), "out must be [S, H, D]")
+    _need(max_logits.shape == (S, H, P) and exp_sums.shape == (S, H, P), "partials shape")
+    _need(context_lens.dtype == torch.int32 and context_lens.shape == (S,), "context_lens")
+    st = load().pa_reduce(out.data_ptr(), tmp_out.data_ptr(), max_logits.data_ptr(),
+                          exp_sums.data_ptr(), context_lens.data_ptr(), S, H, D,
+                          int(partition_size), P, _dtype_code(out), _stream(stream))
+    _check(st, "pa_reduce")
+
+
+def pa_check_error(stream=None) -> int:
+    """Synchronise the stream; raise PagedAttentionError if a kernel met an
+    out-of-range index since the last check; return 0 otherwise."""
+    detail = _i64(0)
+    st = load().pa_check_error(_stream(stream), ctypes.byref(detail))
+    if st != PA_OK:
+        raise PagedAttentionError(st, "pa_check_error", int(detail.value))
+    return 0

@@ -1,0 +1,323 @@
+// pa_api.cu -- the extern "C" entry points of libpa (declared in include/pa.h):
+// host-side argument validation, TMA tensor-map encoding, kernel selection
+// and launch on the caller's stream.  The library allocates nothing and keeps
+// no state beyond the per-device error word and per-device kernel attributes.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "pa.h"
+#include "pa_cache_reduce.cuh"
+#include "pa_decode.cuh"
+
+namespace {
+
+using namespace pa;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// cuTensorMapEncodeTiled, fetched once through the runtime (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4-D view of a cache [num_blocks, 16, Hk, D] for 16 x 64-element page boxes:
+//   dim0: 64 elements (128 B, contiguous)
+//   dim1: D/64 column boxes of a row      stride 128 B
+//   dim2: Hk KV heads                      stride D*2 B
+//   dim3: num_blocks*16 token rows         stride Hk*D*2 B
+// box {64, 1, 1, 16}, 128-byte swizzle, zero fill out of range.
+bool encode_cache_map(CUtensorMap* map, const void* cache, pa_dtype dtype, int64_t num_blocks,
+                      int64_t num_kv_heads, int64_t head_dim) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(head_dim / 64),
+                              static_cast<cuuint64_t>(num_kv_heads),
+                              static_cast<cuuint64_t>(num_blocks * kPage)};
+  const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(head_dim * 2),
+                                 static_cast<cuuint64_t>(num_kv_heads * head_dim * 2)};
+  const cuuint32_t box[4] = {64, 1, 1, kPage};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        4, const_cast<void*>(cache), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+template <class K>
+bool ensure_smem(K kernel, int bytes, std::atomic<uint64_t>* done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  const uint64_t bit = 1ull << dev;
+  if (done_mask->load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  done_mask->fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+
+pa_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// Pipeline depth per head_dim: stages of (K page + V page) per warp.
+template <int D>
+struct Stages { static constexpr int value = D == 64 ? 4 : 3; };
+
+template <int D, bool BF16, class Warp>
+pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, const DecodeArgs& a,
+                          long long grid, cudaStream_t stream) {
+  constexpr int NST = Stages<D>::value;
+  using L = DecodeSmem<D, NST>;
+  auto kernel = paged_decode_kernel<D, NST, BF16, Warp>;
+  static std::atomic<uint64_t> done{0};
+  if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
+  kernel<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(km, vm, a);
+  return launch_status();
+}
+
+template <int D, bool BF16>
+pa_status launch_decode_d(const CUtensorMap& km, const CUtensorMap& vm, const DecodeArgs& a,
+                          long long grid, cudaStream_t stream) {
+  if (a.group == 1) return launch_decode_t<D, BF16, SimtWarp<D, BF16>>(km, vm, a, grid, stream);
+  if (a.group <= 8)
+    return launch_decode_t<D, BF16, MmaWarp<D, BF16, false>>(km, vm, a, grid, stream);
+  return launch_decode_t<D, BF16, MmaWarp<D, BF16, true>>(km, vm, a, grid, stream);
+}
+
+// Shared validation of the attention arguments (host only, no CUDA calls).
+pa_status check_attention_args(const void* query, const void* key_cache, const void* value_cache,
+                               const int32_t* block_tables, const int32_t* context_lens,
+                               float scale, int64_t num_seqs, int64_t num_heads,
+                               int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                               int64_t block_size, int64_t max_blocks_per_seq, pa_dtype dtype) {
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_DTYPE;
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 ||
+      block_size <= 0 || max_blocks_per_seq <= 0)
+    return PA_ERR_SHAPE;
+  if (num_heads % num_kv_heads != 0) return PA_ERR_SHAPE;
+  if (!std::isfinite(scale)) return PA_ERR_SHAPE;
+  if (num_seqs > 0 && (!query || !key_cache || !value_cache || !block_tables || !context_lens))
+    return PA_ERR_NULL;
+  if (head_dim % 8 != 0) return PA_ERR_ALIGN;
+  if (num_seqs > 0 && (!aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache)))
+    return PA_ERR_ALIGN;
+  if (num_seqs > 0 && ((reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+                        (reinterpret_cast<uintptr_t>(context_lens) & 3u)))
+    return PA_ERR_ALIGN;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != kPage) return PA_ERR_UNSUPPORTED;
+  if (num_heads / num_kv_heads > 16) return PA_ERR_UNSUPPORTED;
+  // index ranges the kernels address with 32-bit ints
+  if (num_blocks * kPage > INT32_MAX || max_blocks_per_seq * kPage > INT32_MAX ||
+      num_heads > 65535 || num_seqs * num_heads > INT32_MAX)
+    return PA_ERR_SHAPE;
+  return PA_OK;
+}
+
+pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cache,
+                     int64_t num_seqs, int64_t head_dim, int64_t num_blocks, pa_dtype dtype,
+                     cudaStream_t stream) {
+  CUtensorMap km, vm;
+  if (!encode_cache_map(&km, key_cache, dtype, num_blocks, a.num_kv_heads, head_dim) ||
+      !encode_cache_map(&vm, value_cache, dtype, num_blocks, a.num_kv_heads, head_dim))
+    return PA_ERR_CUDA;
+  const long long grid = num_seqs * a.num_kv_heads * static_cast<long long>(a.parts_per_head);
+  if (grid > INT32_MAX) return PA_ERR_SHAPE;
+  const bool bf16 = dtype == PA_BF16;
+  if (head_dim == 64)
+    return bf16 ? launch_decode_d<64, true>(km, vm, a, grid, stream)
+                : launch_decode_d<64, false>(km, vm, a, grid, stream);
+  return bf16 ? launch_decode_d<128, true>(km, vm, a, grid, stream)
+              : launch_decode_d<128, false>(km, vm, a, grid, stream);
+}
+
+DecodeArgs make_args(const void* query, const int32_t* block_tables, const int32_t* context_lens,
+                     float scale, int64_t num_heads, int64_t num_kv_heads,
+                     int64_t max_blocks_per_seq, int64_t num_blocks) {
+  DecodeArgs a{};
+  a.query = static_cast<const uint16_t*>(query);
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.scale_log2 = scale * kLog2e;
+  a.num_heads = static_cast<int>(num_heads);
+  a.num_kv_heads = static_cast<int>(num_kv_heads);
+  a.group = static_cast<int>(num_heads / num_kv_heads);
+  a.max_blocks_per_seq = static_cast<int>(max_blocks_per_seq);
+  a.num_blocks = static_cast<int>(num_blocks);
+  a.partition_size = 0;
+  a.parts_per_head = 1;
+  a.max_partitions = 1;
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(pa_status status) {
+  switch (status) {
+    case PA_OK: return "ok";
+    case PA_ERR_NULL: return "null pointer";
+    case PA_ERR_SHAPE: return "bad shape or size";
+    case PA_ERR_DTYPE: return "unknown dtype";
+    case PA_ERR_ALIGN: return "misaligned pointer or stride";
+    case PA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_BOUNDS: return "out-of-range index met on the device";
+  }
+  return "unknown status";
+}
+
+int32_t pa_abi_version(void) { return (1 << 16) | 0; }
+
+pa_status pa_reshape_and_cache(const void* key, const void* value, int64_t key_stride,
+                               int64_t value_stride, void* key_cache, void* value_cache,
+                               const int64_t* slot_mapping, int64_t num_tokens,
+                               int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                               int64_t block_size, pa_dtype dtype, void* stream) {
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_DTYPE;
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 || block_size <= 0)
+    return PA_ERR_SHAPE;
+  const int64_t row = num_kv_heads * head_dim;
+  if (key_stride < row || value_stride < row) return PA_ERR_SHAPE;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_NULL;
+  if (head_dim % 8 != 0 || key_stride % 8 != 0 || value_stride % 8 != 0) return PA_ERR_ALIGN;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache) ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return PA_ERR_ALIGN;
+  const int64_t chunks = row / 8;
+  if (chunks > INT32_MAX) return PA_ERR_SHAPE;
+  const int64_t total = num_tokens * chunks;
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  if (blocks > 148 * 32) blocks = 148 * 32;  // grid-stride beyond 32 CTAs per SM
+  reshape_and_cache_kernel<<<static_cast<unsigned>(blocks), threads, 0, as_stream(stream)>>>(
+      static_cast<const uint16_t*>(key), static_cast<const uint16_t*>(value), key_stride,
+      value_stride, static_cast<uint16_t*>(key_cache), static_cast<uint16_t*>(value_cache),
+      slot_mapping, num_tokens, static_cast<int>(chunks), num_blocks * block_size);
+  return launch_status();
+}
+
+pa_status pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, float scale,
+                    int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads, int64_t head_dim,
+                    int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq,
+                    pa_dtype dtype, void* stream) {
+  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
+                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
+                                      num_blocks, block_size, max_blocks_per_seq, dtype);
+  if (st != PA_OK) return st;
+  if (num_seqs == 0) return PA_OK;
+  if (!out) return PA_ERR_NULL;
+  if (!aligned16(out)) return PA_ERR_ALIGN;
+  DecodeArgs a = make_args(query, block_tables, context_lens, scale, num_heads, num_kv_heads,
+                           max_blocks_per_seq, num_blocks);
+  a.out = static_cast<uint16_t*>(out);
+  return run_decode(a, key_cache, value_cache, num_seqs, head_dim, num_blocks, dtype,
+                    as_stream(stream));
+}
+
+pa_status pa_decode_split(float* tmp_out, float* max_logits, float* exp_sums, const void* query,
+                          const void* key_cache, const void* value_cache,
+                          const int32_t* block_tables, const int32_t* context_lens, float scale,
+                          int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads,
+                          int64_t head_dim, int64_t num_blocks, int64_t block_size,
+                          int64_t max_blocks_per_seq, int64_t partition_size,
+                          int64_t max_partitions, pa_dtype dtype, void* stream) {
+  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
+                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
+                                      num_blocks, block_size, max_blocks_per_seq, dtype);
+  if (st != PA_OK) return st;
+  if (partition_size <= 0 || max_partitions <= 0) return PA_ERR_SHAPE;
+  if (partition_size % kPage != 0) return PA_ERR_UNSUPPORTED;
+  if (partition_size > INT32_MAX || max_partitions > INT32_MAX) return PA_ERR_SHAPE;
+  if (num_seqs == 0) return PA_OK;
+  if (!tmp_out || !max_logits || !exp_sums) return PA_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(tmp_out) & 7u) || (reinterpret_cast<uintptr_t>(max_logits) & 3u) ||
+      (reinterpret_cast<uintptr_t>(exp_sums) & 3u))
+    return PA_ERR_ALIGN;
+  DecodeArgs a = make_args(query, block_tables, context_lens, scale, num_heads, num_kv_heads,
+                           max_blocks_per_seq, num_blocks);
+  a.tmp_out = tmp_out;
+  a.max_logits = max_logits;
+  a.exp_sums = exp_sums;
+  a.partition_size = static_cast<int>(partition_size);
+  a.parts_per_head = static_cast<int>(max_partitions);
+  a.max_partitions = static_cast<int>(max_partitions);
+  return run_decode(a, key_cache, value_cache, num_seqs, head_dim, num_blocks, dtype,
+                    as_stream(stream));
+}
+
+pa_status pa_reduce(void* out, const float* tmp_out, const float* max_logits,
+                    const float* exp_sums, const int32_t* context_lens, int64_t num_seqs,
+                    int64_t num_heads, int64_t head_dim, int64_t partition_size,
+                    int64_t max_partitions, pa_dtype dtype, void* stream) {
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_DTYPE;
+  if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || partition_size <= 0 ||
+      max_partitions <= 0)
+    return PA_ERR_SHAPE;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !tmp_out || !max_logits || !exp_sums || !context_lens) return PA_ERR_NULL;
+  if (head_dim % 2 != 0 || head_dim > 2 * kReduceThreads) return PA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(out) & 3u) || (reinterpret_cast<uintptr_t>(tmp_out) & 7u))
+    return PA_ERR_ALIGN;
+  if (num_seqs * num_heads > INT32_MAX || partition_size > INT32_MAX ||
+      max_partitions > INT32_MAX)
+    return PA_ERR_SHAPE;
+  const unsigned grid = static_cast<unsigned>(num_seqs * num_heads);
+  cudaStream_t s = as_stream(stream);
+  if (dtype == PA_BF16)
+    lse_reduce_kernel<true><<<grid, kReduceThreads, 0, s>>>(
+        static_cast<uint16_t*>(out), tmp_out, max_logits, exp_sums, context_lens,
+        static_cast<int>(num_heads), static_cast<int>(head_dim), static_cast<int>(partition_size),
+        static_cast<int>(max_partitions));
+  else
+    lse_reduce_kernel<false><<<grid, kReduceThreads, 0, s>>>(
+        static_cast<uint16_t*>(out), tmp_out, max_logits, exp_sums, context_lens,
+        static_cast<int>(num_heads), static_cast<int>(head_dim), static_cast<int>(partition_size),
+        static_cast<int>(max_partitions));
+  return launch_status();
+}
+
+pa_status pa_check_error(void* stream, int64_t* detail) {
+  cudaStream_t s = as_stream(stream);
+  unsigned long long word = 0;
+  const unsigned long long zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&word, pa::g_error_word, sizeof word, 0, cudaMemcpyDeviceToHost,
+                                s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemcpyToSymbolAsync(pa::g_error_word, &zero, sizeof zero, 0, cudaMemcpyHostToDevice,
+                                s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+  if (detail) *detail = static_cast<int64_t>(word);
+  return word ? PA_ERR_BOUNDS : PA_OK;
+}
+
+}  // extern "C"

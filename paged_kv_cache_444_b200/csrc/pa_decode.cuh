@@ -1,0 +1,514 @@
+// pa_decode.cuh -- paged decode attention on sm_100a.
+//
+// What it computes ("vLLM PagedAttention 原理与源码深度解析" §5.3; "vllm源码分析"
+// §第三讲): for one query token per sequence, out = softmax(scale * q K^T) V
+// over the sequence's first context_lens[s] tokens, whose K/V rows live in
+// 16-token physical blocks named by the sequence's block table ("vllm源码剖析"
+// §一.2: cache [num_blocks, block_size, num_kv_heads, head_dim]).
+//
+// Work decomposition.  One CTA owns one (sequence, KV head, partition) item:
+// the whole sequence for pa_decode, `partition_size` tokens for
+// pa_decode_split.  The CTA's four warps take the item's pages round-robin;
+// each warp streams its pages through its own ring of NST shared-memory
+// stages, keeps its own online-softmax state, and the four states are merged
+// through shared memory at the end (the log-sum-exp identity, exact up to
+// rounding).  No warp ever waits for another until that merge.
+//
+// Gather.  A page of one KV head is 16 rows of head_dim 16-bit values,
+// num_kv_heads*head_dim elements apart.  One TMA tensor-tile load moves a
+// 16 x 64-element box (2 KB) of it into shared memory, 128-byte swizzled so
+// that both the row-wise reads of the CUDA-core path and the 8-row ldmatrix
+// reads of the tensor-core path are bank-conflict free.  Lane 0 of the warp
+// issues the loads for a page NST pages ahead, right after the page that last
+// used the stage has been consumed.  The block id of every page comes from a
+// window of 32 ids held one per lane (a second window is prefetched).
+//
+// Math.  fp32 throughout.  For one query head per KV head (MHA) the dot
+// products and the P.V accumulation run on the CUDA cores with packed fp32
+// FMA (FFMA2).  For a GQA group (2..16 query heads per KV head) the group is
+// a small dense contraction: S = Q K^T and O += P V run as mma.sync m16n8k16
+// with fp32 accumulators (Q rows padded to 16, P rounded to the cache dtype
+// for the second product).  The softmax is online, in base 2 with
+// scale*log2(e) folded into the logits, with warp-shuffle max reductions.
+#pragma once
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+constexpr int kPage = 16;       // tokens per physical block (block_size)
+constexpr int kWarps = 4;       // warps per CTA
+constexpr int kThreads = kWarps * 32;
+constexpr int kBoxBytes = kPage * 128;  // one 16 x 64-element TMA box
+
+struct DecodeArgs {
+  const uint16_t* query;      // [S, H, D]
+  uint16_t* out;              // [S, H, D]            (single-pass mode)
+  float* tmp_out;             // [S, H, P, D]         (split mode, else null)
+  float* max_logits;          // [S, H, P]
+  float* exp_sums;            // [S, H, P]
+  const int32_t* block_tables;  // [S, MB]
+  const int32_t* context_lens;  // [S]
+  float scale_log2;           // scale * log2(e)
+  int num_heads;
+  int num_kv_heads;
+  int group;                  // num_heads / num_kv_heads
+  int max_blocks_per_seq;
+  int num_blocks;
+  int partition_size;         // tokens per item in split mode (multiple of 16)
+  int parts_per_head;         // grid items per (seq, kv head): max_partitions or 1
+  int max_partitions;
+};
+
+template <int D, int NST>
+struct DecodeSmem {
+  static constexpr int kPageBytes = kPage * D * 2;       // one tensor, one page, one head
+  static constexpr int kStageBytes = 2 * kPageBytes;      // K page + V page
+  static constexpr int kStagesBytes = kWarps * NST * kStageBytes;
+  static constexpr int kBarOffset = kStagesBytes;
+  static constexpr int kProbOffset = kBarOffset + kWarps * NST * 8;
+  static constexpr int kRedMOffset = kProbOffset + kWarps * kPage * 4;
+  static constexpr int kRedLOffset = kRedMOffset + kWarps * 16 * 4;
+  static constexpr int kBytes = kRedLOffset + kWarps * 16 * 4;
+  static constexpr int kAlloc = kBytes + 1024;            // + alignment slack
+  // the merge buffer (kWarps x group x D floats) reuses the stage area
+  static_assert(kWarps * 16 * D * 4 <= kStagesBytes, "merge buffer must fit in the stages");
+  static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
+};
+
+// Address of 16-byte chunk `c` (0 .. D/8-1) of row `r` in a swizzled page.
+template <int D>
+__device__ __forceinline__ uint32_t page_chunk(uint32_t base, int r, int c) {
+  return base + (c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+
+// ---------------------------------------------------------------------------
+// Per-warp state and page step: tensor-core path (GQA groups)
+// ---------------------------------------------------------------------------
+template <int D, bool BF16, bool TWO_ROWS>
+struct MmaWarp {
+  static constexpr int KSTEPS = D / 16;  // k-steps of 16 over head_dim
+  static constexpr int NTILES = D / 8;   // 8-wide n-tiles of the output
+  uint32_t qa[KSTEPS][4];                // Q as mma A fragments (rows = query heads of the group)
+  float acc[NTILES][4];                  // O fragments (rows r0 / r1)
+  float m[2], l[2];                      // running max (log2 domain) and lane-partial sums
+
+  __device__ __forceinline__ void init(const uint16_t* q_group, int group, int lane) {
+    const int r0 = lane >> 2, r1 = r0 + 8, tig = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      const int klo = kk * 16 + tig * 2, khi = klo + 8;
+      const uint32_t* q0 = reinterpret_cast<const uint32_t*>(q_group + r0 * D);
+      const uint32_t* q1 = reinterpret_cast<const uint32_t*>(q_group + r1 * D);
+      qa[kk][0] = r0 < group ? q0[klo >> 1] : 0u;
+      qa[kk][1] = (TWO_ROWS && r1 < group) ? q1[klo >> 1] : 0u;
+      qa[kk][2] = r0 < group ? q0[khi >> 1] : 0u;
+      qa[kk][3] = (TWO_ROWS && r1 < group) ? q1[khi >> 1] : 0u;
+    }
+#pragma unroll
+    for (int n = 0; n < NTILES; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.f;
+  }
+
+  __device__ __forceinline__ void page(uint32_t kbase, uint32_t vbase, int tok0, int t_end,
+                                       float scale_log2, int lane, float*) {
+    const int tig = lane & 3;
+    // ---- S = Q K^T for the page's 16 tokens (two 8-token n-tiles) ----
+    float sc[2][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sc[0][i] = sc[1][i] = 0.f;
+    const int ktok = ((lane >> 4) << 3) + (lane & 7);
+    const int kchk = (lane >> 3) & 1;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(page_chunk<D>(kbase, ktok, kk * 2 + kchk), b0, b1, b2, b3);
+      mma_16816<BF16>(sc[0], qa[kk], b0, b1);
+      mma_16816<BF16>(sc[1], qa[kk], b2, b3);
+    }
+    // ---- scale, mask the tail, row max over the page ----
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = tok0 + nt * 8 + tig * 2 + (i & 1);
+        const float x = t < t_end ? sc[nt][i] * scale_log2 : -INFINITY;
+        sc[nt][i] = x;
+        if (i < 2) mx0 = fmaxf(mx0, x); else mx1 = fmaxf(mx1, x);
+      }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    const float mn0 = fmaxf(m[0], mx0);
+    const float al0 = ex2(m[0] - mn0);
+    m[0] = mn0;
+    float mn1 = 0.f, al1 = 1.f;
+    if constexpr (TWO_ROWS) {
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      mn1 = fmaxf(m[1], mx1);
+      al1 = ex2(m[1] - mn1);
+      m[1] = mn1;
+    }
+    // ---- P = 2^(x - m), rounded to the cache dtype as the A operand of P V ----
+    uint32_t pa[4];
+    pa[0] = pack2<BF16>(ex2(sc[0][0] - mn0), ex2(sc[0][1] - mn0));
+    pa[2] = pack2<BF16>(ex2(sc[1][0] - mn0), ex2(sc[1][1] - mn0));
+    {
+      const float2 u = unpack2<BF16>(pa[0]), v = unpack2<BF16>(pa[2]);
+      l[0] = l[0] * al0 + ((u.x + u.y) + (v.x + v.y));
+    }
+    if constexpr (TWO_ROWS) {
+      pa[1] = pack2<BF16>(ex2(sc[0][2] - mn1), ex2(sc[0][3] - mn1));
+      pa[3] = pack2<BF16>(ex2(sc[1][2] - mn1), ex2(sc[1][3] - mn1));
+      const float2 u = unpack2<BF16>(pa[1]), v = unpack2<BF16>(pa[3]);
+      l[1] = l[1] * al1 + ((u.x + u.y) + (v.x + v.y));
+    } else {
+      pa[1] = pa[3] = 0u;
+    }
+    // ---- rescale O, then O += P V ----
+#pragma unroll
+    for (int n = 0; n < NTILES; ++n) {
+      acc[n][0] *= al0;
+      acc[n][1] *= al0;
+      if constexpr (TWO_ROWS) {
+        acc[n][2] *= al1;
+        acc[n][3] *= al1;
+      }
+    }
+    const int vtok = ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int vchk = lane >> 4;
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_trans(page_chunk<D>(vbase, vtok, 2 * j + vchk), b0, b1, b2, b3);
+      mma_16816<BF16>(acc[2 * j], pa, b0, b1);
+      mma_16816<BF16>(acc[2 * j + 1], pa, b2, b3);
+    }
+  }
+
+  // Write this warp's (m, l, O) rows < group into the merge buffers.
+  __device__ __forceinline__ void publish(float* red_acc, float* red_m, float* red_l, int group,
+                                          int lane) {
+    const int r0 = lane >> 2, r1 = r0 + 8, tig = lane & 3;
+    float l0 = l[0];
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    float l1 = l[1];
+    if constexpr (TWO_ROWS) {
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    }
+    if (r0 < group) {
+#pragma unroll
+      for (int n = 0; n < NTILES; ++n)
+        *reinterpret_cast<float2*>(red_acc + r0 * D + n * 8 + tig * 2) =
+            make_float2(acc[n][0], acc[n][1]);
+      if (tig == 0) {
+        red_m[r0] = m[0];
+        red_l[r0] = l0;
+      }
+    }
+    if constexpr (TWO_ROWS) {
+      if (r1 < group) {
+#pragma unroll
+        for (int n = 0; n < NTILES; ++n)
+          *reinterpret_cast<float2*>(red_acc + r1 * D + n * 8 + tig * 2) =
+              make_float2(acc[n][2], acc[n][3]);
+        if (tig == 0) {
+          red_m[r1] = m[1];
+          red_l[r1] = l1;
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Per-warp state and page step: CUDA-core path (one query head per KV head)
+// ---------------------------------------------------------------------------
+template <int D, bool BF16>
+struct SimtWarp {
+  static_assert(D == 64 || D == 128, "CUDA-core path is built for head_dim 64 and 128");
+  static constexpr int QCH = D / 16;     // 16-byte chunks per lane in Q.K (half a row)
+  static constexpr int VCH = D / 8;      // 16-byte chunks per row
+  static constexpr int TG = 32 / VCH;    // token groups in P.V
+  static constexpr int TPL = kPage / TG; // tokens per lane in P.V
+  float2 qf[QCH * 4];                    // this lane's half of q, in its read order
+  float2 acc[4];                         // 8 output dims of one token group
+  float m, l;
+  uint32_t kxor;                         // per-lane chunk swizzle for Q.K reads
+  int kbox;                              // box offset (bytes) of this lane's half row
+
+  __device__ __forceinline__ void init(const uint16_t* q_row, int, int lane) {
+    const int tok = lane >> 1, hf = lane & 1;
+    kxor = static_cast<uint32_t>(((hf * 4) ^ (tok & 7)) << 4);
+    kbox = (D == 128 ? hf * kBoxBytes : 0) + tok * 128;
+#pragma unroll
+    for (int k = 0; k < QCH; ++k) {
+      // step k reads logical chunk (D==128 ? 8*hf : 0) + (k ^ 4*hf) of the row
+      const int c = (D == 128 ? hf * 8 : 0) + (k ^ (hf * 4));
+      const uint4 raw = *reinterpret_cast<const uint4*>(q_row + c * 8);
+      qf[k * 4 + 0] = unpack2<BF16>(raw.x);
+      qf[k * 4 + 1] = unpack2<BF16>(raw.y);
+      qf[k * 4 + 2] = unpack2<BF16>(raw.z);
+      qf[k * 4 + 3] = unpack2<BF16>(raw.w);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
+    m = -INFINITY;
+    l = 0.f;
+  }
+
+  __device__ __forceinline__ void page(uint32_t kbase, uint32_t vbase, int tok0, int t_end,
+                                       float scale_log2, int lane, float* probs) {
+    const int tok = lane >> 1, hf = lane & 1;
+    // ---- q . k for token `tok`, this lane's half of the row ----
+    float2 d2 = make_float2(0.f, 0.f);
+    const uint32_t krow = kbase + kbox;
+#pragma unroll
+    for (int k = 0; k < QCH; ++k) {
+      const uint4 raw = lds128(krow + ((static_cast<uint32_t>(k) << 4) ^ kxor));
+      d2 = ffma2(qf[k * 4 + 0], unpack2<BF16>(raw.x), d2);
+      d2 = ffma2(qf[k * 4 + 1], unpack2<BF16>(raw.y), d2);
+      d2 = ffma2(qf[k * 4 + 2], unpack2<BF16>(raw.z), d2);
+      d2 = ffma2(qf[k * 4 + 3], unpack2<BF16>(raw.w), d2);
+    }
+    float dot = d2.x + d2.y;
+    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+    const float x = (tok0 + tok) < t_end ? dot * scale_log2 : -INFINITY;
+    float mx = x;
+#pragma unroll
+    for (int o = 2; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float mn = fmaxf(m, mx);
+    const float al = ex2(m - mn);
+    m = mn;
+    const float p = ex2(x - mn);
+    l = l * al + (hf ? 0.f : p);
+    if (hf == 0) probs[tok] = p;
+    __syncwarp();
+    // ---- O = O * alpha + sum_j p_j v_j over this lane's tokens and 8 dims ----
+    const int cc = lane % VCH, tg = lane / VCH;
+    const float2 al2 = make_float2(al, al);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = fmul2(acc[i], al2);
+    float pj[TPL];
+#pragma unroll
+    for (int i = 0; i < TPL; i += 4) {
+      const float4 p4 = *reinterpret_cast<const float4*>(probs + tg * TPL + i);
+      pj[i] = p4.x; pj[i + 1] = p4.y; pj[i + 2] = p4.z; pj[i + 3] = p4.w;
+    }
+    const uint32_t vrow = vbase + (cc >> 3) * kBoxBytes + tg * TPL * 128;
+    const uint32_t vx = static_cast<uint32_t>((cc & 7) ^ ((tg * TPL) & 7));
+#pragma unroll
+    for (int i = 0; i < TPL; ++i) {
+      const uint4 raw = lds128(vrow + i * 128 + ((vx ^ static_cast<uint32_t>(i)) << 4));
+      const float2 pp = make_float2(pj[i], pj[i]);
+      acc[0] = ffma2(pp, unpack2<BF16>(raw.x), acc[0]);
+      acc[1] = ffma2(pp, unpack2<BF16>(raw.y), acc[1]);
+      acc[2] = ffma2(pp, unpack2<BF16>(raw.z), acc[2]);
+      acc[3] = ffma2(pp, unpack2<BF16>(raw.w), acc[3]);
+    }
+  }
+
+  __device__ __forceinline__ void publish(float* red_acc, float* red_m, float* red_l, int,
+                                          int lane) {
+    float lt = l;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
+#pragma unroll
+    for (int o = VCH; o < 32; o <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[i].x += __shfl_xor_sync(0xffffffffu, acc[i].x, o);
+        acc[i].y += __shfl_xor_sync(0xffffffffu, acc[i].y, o);
+      }
+    }
+    if (lane < VCH) {
+      float4* dst = reinterpret_cast<float4*>(red_acc + lane * 8);
+      dst[0] = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
+      dst[1] = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
+    }
+    if (lane == 0) {
+      red_m[0] = m;
+      red_l[0] = lt;
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// The kernel: one (sequence, KV head, partition) item per CTA.
+// ---------------------------------------------------------------------------
+template <int D, int NST, bool BF16, class Warp>
+__global__ void __launch_bounds__(kThreads)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                        const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
+  using L = DecodeSmem<D, NST>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  int item = blockIdx.x;
+  const int part = item % a.parts_per_head;
+  item /= a.parts_per_head;
+  const int kvh = item % a.num_kv_heads;
+  const int s = item / a.num_kv_heads;
+  const int group = a.group;
+  const bool split = a.tmp_out != nullptr;
+
+  // ---- context length and this item's token range ----
+  int ctx = a.context_lens[s];
+  const int cap = a.max_blocks_per_seq * kPage;
+  if (ctx < 0 || ctx > cap) {
+    if (threadIdx.x == 0 && part == 0 && kvh == 0) record_error(kErrContextLen, s);
+    ctx = ctx < 0 ? 0 : cap;
+  }
+  int t_begin = 0, t_end = ctx;
+  if (split) {
+    if (threadIdx.x == 0 && part == 0 && kvh == 0 &&
+        (ctx + a.partition_size - 1) / a.partition_size > a.max_partitions)
+      record_error(kErrPartitions, s);
+    t_begin = part * a.partition_size;
+    t_end = min(t_begin + a.partition_size, ctx);
+    if (t_begin >= t_end) return;  // partition past the end: nothing to write
+  } else if (ctx == 0) {
+    // empty sequence: zero output rows
+    uint16_t* o = a.out + (static_cast<size_t>(s) * a.num_heads + kvh * group) * D;
+    for (int i = threadIdx.x; i < group * D; i += kThreads) o[i] = 0;
+    return;
+  }
+
+  const int first_page = t_begin / kPage;
+  const int n_pages = (t_end - first_page * kPage + kPage - 1) / kPage;
+  const int my_pages = n_pages > warp ? (n_pages - warp + kWarps - 1) / kWarps : 0;
+  const int32_t* bt = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + first_page;
+
+  const uint32_t stage0 = smem_addr(smem) + warp * NST * L::kStageBytes;
+  const uint32_t bar0 = smem_addr(smem + L::kBarOffset) + warp * NST * 8;
+  float* probs = reinterpret_cast<float*>(smem + L::kProbOffset) + warp * kPage;
+
+  if (lane == 0) {
+    for (int i = 0; i < NST; ++i) mbar_init(bar0 + i * 8, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+
+  // ---- block ids: lane j holds the id of this warp's page (win*32 + j) ----
+  const size_t row_base = static_cast<size_t>(s) * a.max_blocks_per_seq + first_page;
+  auto load_ids = [&](int win) -> int {
+    const int k = win * 32 + lane;
+    if (k >= my_pages) return -1;
+    const int idx = warp + k * kWarps;
+    int id = bt[idx];
+    if (id < 0 || id >= a.num_blocks) {
+      record_error(kErrBlockId, static_cast<long long>(row_base + idx));
+      id = -1;  // TMA zero-fills a box at a negative row: no out-of-range read
+    }
+    return id;
+  };
+  int win = 0;
+  int ids_cur = load_ids(0);
+  int ids_next = my_pages > 32 ? load_ids(1) : -1;
+
+  auto issue = [&](int k) {  // whole warp; lane 0 issues the TMA for page k
+    const int src = ((k >> 5) == win) ? ids_cur : ids_next;
+    const int id = __shfl_sync(0xffffffffu, src, k & 31);
+    if (lane == 0) {
+      const int st = k % NST;
+      const uint32_t bar = bar0 + st * 8;
+      const uint32_t dk = stage0 + st * L::kStageBytes;
+      const uint32_t dv = dk + L::kPageBytes;
+      const int row = id * kPage;
+      mbar_arrive_expect_tx(bar, L::kStageBytes);
+#pragma unroll
+      for (int b = 0; b < D / 64; ++b) tma_load_4d(dk + b * kBoxBytes, &kmap, bar, 0, b, kvh, row);
+#pragma unroll
+      for (int b = 0; b < D / 64; ++b) tma_load_4d(dv + b * kBoxBytes, &vmap, bar, 0, b, kvh, row);
+    }
+  };
+
+  const int pre = my_pages < NST ? my_pages : NST;
+  for (int k = 0; k < pre; ++k) issue(k);
+
+  // ---- this warp's query rows ----
+  Warp st;
+  const uint16_t* q_group =
+      a.query + (static_cast<size_t>(s) * a.num_heads + static_cast<size_t>(kvh) * group) * D;
+  st.init(q_group, group, lane);
+
+  // ---- main loop over this warp's pages ----
+  bool ok = true;
+  for (int k = 0; k < my_pages; ++k) {
+    if (k > 0 && (k & 31) == 0) {
+      ++win;
+      ids_cur = ids_next;
+      ids_next = my_pages > (win + 1) * 32 ? load_ids(win + 1) : -1;
+    }
+    const int stg = k % NST;
+    if (!mbar_wait_bounded(bar0 + stg * 8, (k / NST) & 1)) {
+      if (lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
+      ok = false;
+      break;
+    }
+    const uint32_t kb = stage0 + stg * L::kStageBytes;
+    const int tok0 = (first_page + warp + k * kWarps) * kPage;
+    st.page(kb, kb + L::kPageBytes, tok0, t_end, a.scale_log2, lane, probs);
+    __syncwarp();
+    if (k + NST < my_pages) issue(k + NST);
+  }
+
+  // ---- merge the four warps (the stage area is reused as the merge buffer) ----
+  __syncthreads();
+  float* red_acc = reinterpret_cast<float*>(smem);
+  float* red_m = reinterpret_cast<float*>(smem + L::kRedMOffset);
+  float* red_l = reinterpret_cast<float*>(smem + L::kRedLOffset);
+  if (ok) {
+    st.publish(red_acc + warp * group * D, red_m + warp * 16, red_l + warp * 16, group, lane);
+  } else {
+    for (int g = lane; g < group; g += 32) {
+      red_m[warp * 16 + g] = -INFINITY;
+      red_l[warp * 16 + g] = 0.f;
+    }
+  }
+  __syncthreads();
+
+  const int h0 = kvh * group;
+  for (int o = threadIdx.x * 2; o < group * D; o += kThreads * 2) {
+    const int g = o / D, d = o % D;
+    float mw[kWarps];
+    float big_m = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      mw[w] = red_m[w * 16 + g];
+      big_m = fmaxf(big_m, mw[w]);
+    }
+    float big_l = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float e = (mw[w] == -INFINITY) ? 0.f : ex2(mw[w] - big_m);
+      big_l += e * red_l[w * 16 + g];
+      if (e != 0.f) {
+        const float2 v = *reinterpret_cast<const float2*>(red_acc + (w * group + g) * D + d);
+        o0 += e * v.x;
+        o1 += e * v.y;
+      }
+    }
+    const size_t hrow = static_cast<size_t>(s) * a.num_heads + h0 + g;
+    if (split) {
+      const size_t pidx = hrow * a.max_partitions + part;
+      *reinterpret_cast<float2*>(a.tmp_out + pidx * D + d) = make_float2(o0, o1);
+      if (d == 0) {
+        a.max_logits[pidx] = big_m * kLn2;
+        a.exp_sums[pidx] = big_l;
+      }
+    } else {
+      const float inv = big_l > 0.f ? 1.f / big_l : 0.f;
+      *reinterpret_cast<uint32_t*>(a.out + hrow * D + d) = pack2<BF16>(o0 * inv, o1 * inv);
+    }
+  }
+}
+
+}  // namespace pa

@@ -1,0 +1,90 @@
+"""Shared plumbing of the GPU parity tests: move a seeded batch between the
+CUDA path (through the C-ABI binding) and the fp64 oracle (on host copies
+taken BEFORE the GPU touches anything).  No attention arithmetic here."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as oracle_mod
+from paged_kv_cache_444_b200 import workloads
+
+TOL = {"f16": 2e-3, "bf16": 8e-3}   # max-abs vs the fp64 oracle
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def ocode(cfg: workloads.DecodeConfig) -> int:
+    return oracle_mod.BF16 if cfg.dtype == "bf16" else oracle_mod.F16
+
+
+class HostCopy:
+    """Host snapshot of a batch (16-bit data as uint16 bits)."""
+
+    def __init__(self, batch: workloads.DecodeBatch):
+        self.cfg = batch.cfg
+        self.context_lens = batch.context_lens.cpu().numpy().astype(np.int32)
+        self.block_tables = batch.block_tables.cpu().numpy().astype(np.int32)
+        self.slot_mapping = batch.slot_mapping.cpu().numpy().astype(np.int64)
+        self.key_cache = bits(batch.key_cache)
+        self.value_cache = bits(batch.value_cache)
+        self.query = bits(batch.query)
+        self.key = bits(batch.key)
+        self.value = bits(batch.value)
+
+
+def oracle_step(orc, host: HostCopy, write: bool = True):
+    """Oracle cache write (on copies) then oracle decode; returns
+    (out float64 [S,H,D], key_cache_after, value_cache_after)."""
+    cfg = host.cfg
+    kc = host.key_cache.copy()
+    vc = host.value_cache.copy()
+    if write:
+        rc = orc.reshape_and_cache(host.key, host.value, kc, vc, host.slot_mapping,
+                                   cfg.num_blocks, cfg.block_size)
+        assert rc == oracle_mod.OK
+    out = orc.decode(host.query, kc, vc, host.block_tables, host.context_lens, cfg.scale,
+                     ocode(cfg))
+    return out, kc, vc
+
+
+def gpu_step(batch: workloads.DecodeBatch, write: bool = True, partition_size: int = 0,
+             max_partitions: int | None = None):
+    """The CUDA path: pa_reshape_and_cache, then pa_decode or
+    pa_decode_split + pa_reduce.  Returns (out, partials or None)."""
+    from paged_kv_cache_444_b200 import (SplitWorkspace, pa_decode, pa_decode_split, pa_reduce,
+                                         pa_reshape_and_cache)
+    cfg = batch.cfg
+    if write:
+        pa_reshape_and_cache(batch.key, batch.value, batch.key_cache, batch.value_cache,
+                             batch.slot_mapping)
+    out = torch.full_like(batch.query, float("nan"))
+    parts = None
+    if partition_size:
+        P = max_partitions or (batch.block_tables.shape[1] * cfg.block_size + partition_size - 1) \
+            // partition_size
+        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, batch.query.device)
+        ws.tmp_out.fill_(float("nan"))
+        ws.max_logits.fill_(float("nan"))
+        ws.exp_sums.fill_(float("nan"))
+        pa_decode_split(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query, batch.key_cache,
+                        batch.value_cache, batch.block_tables, batch.context_lens, cfg.scale,
+                        partition_size)
+        pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, batch.context_lens,
+                  partition_size)
+        parts = ws
+    else:
+        pa_decode(out, batch.query, batch.key_cache, batch.value_cache, batch.block_tables,
+                  batch.context_lens, cfg.scale)
+    torch.cuda.synchronize()
+    return out, parts
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def max_err(gpu_out: torch.Tensor, ref: np.ndarray) -> float:
+    return float(np.max(np.abs(to_f64(gpu_out) - ref))) if ref.size else 0.0

@@ -1,0 +1,266 @@
+"""CUDA path vs the fp64 oracle, element by element, on seeded batches small
+enough for the oracle to finish in seconds but spanning many pages, warps and
+ragged tails (GPU).  Tolerances: max-abs 2e-3 (fp16), 8e-3 (bf16); the cache
+write is compared bit for bit over the whole buffer."""
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_444_b200 import PagedAttentionError, pa_check_error, workloads
+from parity_helpers import TOL, HostCopy, bits, gpu_step, max_err, oracle_step, to_f64
+
+pytestmark = pytest.mark.gpu
+
+C = workloads.CONFIGS
+
+# Scaled-down versions of the five workloads (same dtype / head layout).
+SMALL = {
+    "tiny": C["tiny"],
+    "mha_small": C["mha_llama2_7b"].scaled(name="mha_small", num_seqs=6, num_heads=8,
+                                             num_kv_heads=8, num_blocks=256,
+                                             ctx=("uniform", 1, 300), seed=11),
+    "gqa_small": C["gqa_llama3_8b"].scaled(name="gqa_small", num_seqs=8, num_heads=32,
+                                             num_kv_heads=8, num_blocks=512,
+                                             ctx=("uniform", 1, 700), seed=12),
+    "long_small": C["long_context_split"].scaled(name="long_small", num_seqs=2, num_heads=8,
+                                                   num_kv_heads=2, num_blocks=512,
+                                                   ctx=("uniform", 1500, 3000), seed=13),
+    "shared_small": C["shared_prefix_beam"].scaled(name="shared_small", num_seqs=8,
+                                                     num_heads=8, num_kv_heads=2,
+                                                     num_blocks=256, shared_prefix_blocks=4,
+                                                     ctx=("lognormal", 150.0, 0.6, 65, 400),
+                                                     seed=14),
+    # other head layouts the kernels are built for
+    "d64_gqa2": C["tiny"].scaled(name="d64_gqa2", num_seqs=5, num_heads=8, num_kv_heads=4,
+                                 dtype="bf16", num_blocks=128, ctx=("uniform", 1, 200), seed=15),
+    "gqa3_f16": C["gqa_llama3_8b"].scaled(name="gqa3_f16", num_seqs=4, num_heads=12,
+                                            num_kv_heads=4, dtype="f16", num_blocks=128,
+                                            ctx=("uniform", 1, 300), seed=16),
+    "gqa8": C["gqa_llama3_8b"].scaled(name="gqa8", num_seqs=3, num_heads=16, num_kv_heads=2,
+                                        num_blocks=128, ctx=("uniform", 30, 400), seed=17),
+    "gqa16_two_rows": C["gqa_llama3_8b"].scaled(name="gqa16_two_rows", num_seqs=3,
+                                                  num_heads=32, num_kv_heads=2, num_blocks=128,
+                                                  ctx=("uniform", 30, 400), seed=18),
+    "gqa16_d64_f16": C["tiny"].scaled(name="gqa16_d64_f16", num_seqs=3, num_heads=32,
+                                        num_kv_heads=2, num_blocks=128,
+                                        ctx=("uniform", 1, 300), seed=19),
+    "mha_bf16": C["mha_llama2_7b"].scaled(name="mha_bf16", num_seqs=4, num_heads=4,
+                                            num_kv_heads=4, dtype="bf16", num_blocks=128,
+                                            ctx=("uniform", 1, 400), seed=20),
+}
+
+
+@pytest.fixture(scope="module")
+def dev(cuda_device):
+    from paged_kv_cache_444_b200 import load
+    load()
+    return cuda_device
+
+
+def _check_close(gpu_out, ref, cfg, what):
+    err = max_err(gpu_out, ref)
+    assert np.isfinite(to_f64(gpu_out)).all(), f"{what}: non-finite output"
+    assert err <= TOL[cfg.dtype], f"{what}: max-abs error {err:.3e} > {TOL[cfg.dtype]}"
+    return err
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_decode_matches_oracle(name, dev, oracle_lib):
+    cfg = SMALL[name]
+    batch = workloads.make_batch(cfg, dev)
+    host = HostCopy(batch)
+    ref, kc_ref, vc_ref = oracle_step(oracle_lib, host)
+    out, _ = gpu_step(batch)
+    pa_check_error()
+    # cache write: bit-exact over the whole buffers
+    assert np.array_equal(bits(batch.key_cache), kc_ref)
+    assert np.array_equal(bits(batch.value_cache), vc_ref)
+    _check_close(out, ref, cfg, name)
+
+
+@pytest.mark.parametrize("name", ["long_small", "gqa_small", "mha_small", "d64_gqa2",
+                                  "gqa16_two_rows"])
+@pytest.mark.parametrize("ps", [16, 64, 512])
+def test_split_matches_oracle(name, ps, dev, oracle_lib):
+    cfg = SMALL[name]
+    batch = workloads.make_batch(cfg, dev)
+    host = HostCopy(batch)
+    ref, kc_ref, vc_ref = oracle_step(oracle_lib, host)
+    out, ws = gpu_step(batch, partition_size=ps)
+    pa_check_error()
+    _check_close(out, ref, cfg, f"{name} split {ps}")
+    # the partial statistics themselves, against the oracle's partitions
+    P = ws.max_partitions
+    acc, pmax, psum = oracle_lib.decode_partitioned(host.query, kc_ref, vc_ref,
+                                                    host.block_tables, host.context_lens,
+                                                    cfg.scale, 1 if cfg.dtype == "bf16" else 0,
+                                                    ps, P)
+    gm = ws.max_logits.cpu().numpy().astype(np.float64)
+    gs = ws.exp_sums.cpu().numpy().astype(np.float64)
+    ga = ws.tmp_out.cpu().numpy().astype(np.float64)
+    valid = ~np.isnan(pmax)
+    assert np.array_equal(valid, ~np.isnan(gm)), "partitions written differ from ceil(ctx/P)"
+    assert np.max(np.abs(gm[valid] - pmax[valid])) <= 1e-4
+    rel = np.abs(gs[valid] - psum[valid]) / psum[valid]
+    assert np.max(rel) <= 1e-2
+    na = acc / psum[..., None]
+    ng = ga / gs[..., None]
+    assert np.nanmax(np.abs(na - ng)) <= TOL[cfg.dtype]
+
+
+def test_split_single_partition_equals_single_pass(dev):
+    cfg = SMALL["gqa_small"]
+    batch = workloads.make_batch(cfg, dev)
+    one, _ = gpu_step(batch)
+    batch2 = workloads.make_batch(cfg, dev)
+    big = 16 * batch.block_tables.shape[1]
+    two, _ = gpu_step(batch2, partition_size=big)
+    assert (to_f64(one) - to_f64(two)).__abs__().max() <= 2 * TOL[cfg.dtype]
+
+
+@pytest.mark.parametrize("name", ["tiny", "gqa_small", "mha_bf16"])
+def test_context_len_one_returns_v_exactly(name, dev):
+    cfg = SMALL[name]
+    batch = workloads.make_batch(cfg, dev)
+    batch.context_lens.fill_(1)
+    out, _ = gpu_step(batch, write=False)
+    G = cfg.group_size
+    bt0 = batch.block_tables[:, 0].long()
+    v0 = batch.value_cache[bt0, 0]                     # [S, Hk, D]
+    want = v0.repeat_interleave(G, dim=1)
+    assert torch.equal(out, want)
+
+
+def test_permutation_invariance_bitwise(dev):
+    cfg = SMALL["gqa_small"]
+    batch = workloads.make_batch(cfg, dev)
+    base, _ = gpu_step(batch, write=False)
+    g = torch.Generator().manual_seed(5)
+    pi = torch.randperm(cfg.num_blocks, generator=g).to(dev)
+    kc = torch.empty_like(batch.key_cache)
+    vc = torch.empty_like(batch.value_cache)
+    kc[pi] = batch.key_cache
+    vc[pi] = batch.value_cache
+    bt = torch.where(batch.block_tables >= 0, pi[batch.block_tables.clamp(min=0).long()],
+                     torch.full_like(batch.block_tables, -1)).to(torch.int32)
+    batch.key_cache, batch.value_cache, batch.block_tables = kc, vc, bt
+    moved, _ = gpu_step(batch, write=False)
+    assert torch.equal(base, moved)
+
+
+def test_shared_prefix_equals_private_copies_bitwise(dev):
+    cfg = SMALL["shared_small"]
+    batch = workloads.make_batch(cfg, dev)
+    shared, _ = gpu_step(batch, write=False)
+    bt = batch.block_tables.clone()
+    used = set(int(x) for x in bt.flatten().tolist() if x >= 0)
+    free = [b for b in range(cfg.num_blocks) if b not in used]
+    for s in range(cfg.num_seqs):
+        if s % cfg.share_group == 0:
+            continue
+        for i in range(cfg.shared_prefix_blocks):
+            nb = free.pop()
+            batch.key_cache[nb] = batch.key_cache[int(bt[s, i])]
+            batch.value_cache[nb] = batch.value_cache[int(bt[s, i])]
+            bt[s, i] = nb
+    batch.block_tables = bt
+    private, _ = gpu_step(batch, write=False)
+    assert torch.equal(shared, private)
+
+
+def test_zero_and_ragged_context_lengths(dev, oracle_lib):
+    cfg = SMALL["gqa_small"].scaled(ctx=("fixed", (0, 1, 15, 16, 17, 31, 32, 33)), num_seqs=8)
+    batch = workloads.make_batch(cfg, dev)
+    host = HostCopy(batch)
+    ref, _, _ = oracle_step(oracle_lib, host)
+    out, _ = gpu_step(batch)
+    assert (to_f64(out[0]) == 0).all()
+    _check_close(out, ref, cfg, "ragged")
+    b2 = workloads.make_batch(cfg, dev)
+    out2, _ = gpu_step(b2, partition_size=16)
+    assert (to_f64(out2[0]) == 0).all()
+    _check_close(out2, ref, cfg, "ragged split")
+
+
+def test_long_sequence_many_pages_per_warp(dev, oracle_lib):
+    # > 32 pages per warp exercises the second block-id window
+    cfg = SMALL["mha_small"].scaled(num_seqs=2, num_heads=2, num_kv_heads=2, num_blocks=1024,
+                                    ctx=("fixed", (3000, 2049)))
+    batch = workloads.make_batch(cfg, dev)
+    host = HostCopy(batch)
+    ref, _, _ = oracle_step(oracle_lib, host)
+    out, _ = gpu_step(batch)
+    _check_close(out, ref, cfg, "long single pass")
+
+
+def test_write_padding_and_strided_rows(dev, oracle_lib):
+    cfg = SMALL["gqa_small"]
+    batch = workloads.make_batch(cfg, dev)
+    T = cfg.num_seqs
+    big = torch.randn((T, 3, cfg.num_kv_heads, cfg.head_dim), device=dev).to(cfg.torch_dtype)
+    batch.key = big[:, 0]
+    batch.value = big[:, 2]
+    batch.slot_mapping[1] = -1
+    batch.slot_mapping[5] = -3
+    host = HostCopy(batch)
+    host.key = bits(batch.key).reshape(T, cfg.num_kv_heads, cfg.head_dim)
+    host.value = bits(batch.value).reshape(T, cfg.num_kv_heads, cfg.head_dim)
+    kc, vc = host.key_cache.copy(), host.value_cache.copy()
+    assert oracle_lib.reshape_and_cache(host.key, host.value, kc, vc, host.slot_mapping,
+                                        cfg.num_blocks, cfg.block_size) == 0
+    from paged_kv_cache_444_b200 import pa_reshape_and_cache
+    pa_reshape_and_cache(batch.key, batch.value, batch.key_cache, batch.value_cache,
+                         batch.slot_mapping)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(batch.key_cache), kc)
+    assert np.array_equal(bits(batch.value_cache), vc)
+
+
+def test_bounds_checks_report_and_skip(dev):
+    cfg = SMALL["gqa_small"]
+    pa_check_error()
+    batch = workloads.make_batch(cfg, dev)
+    # a slot past the end: skipped, reported with its token index
+    batch.slot_mapping[3] = cfg.num_blocks * cfg.block_size + 5
+    before = batch.key_cache.clone()
+    from paged_kv_cache_444_b200 import pa_reshape_and_cache
+    pa_reshape_and_cache(batch.key, batch.value, batch.key_cache, batch.value_cache,
+                         batch.slot_mapping)
+    with pytest.raises(PagedAttentionError) as e:
+        pa_check_error()
+    assert e.value.detail >> 56 == 1 and e.value.detail & 0xffff == 3
+    changed = (batch.key_cache != before).flatten(1).any(1).nonzero().flatten().tolist()
+    assert len(changed) <= cfg.num_seqs - 1
+    pa_check_error()  # cleared
+    # a block id past the pool: read as zeros, reported
+    b = workloads.make_batch(cfg, dev)
+    b.block_tables[2, 0] = cfg.num_blocks + 7
+    out, _ = gpu_step(b, write=False)
+    with pytest.raises(PagedAttentionError) as e:
+        pa_check_error()
+    assert e.value.detail >> 56 == 2
+    assert np.isfinite(to_f64(out)).all()
+    # a context length beyond the table: clamped, reported
+    b = workloads.make_batch(cfg, dev)
+    b.context_lens[4] = b.block_tables.shape[1] * cfg.block_size + 100
+    out, _ = gpu_step(b, write=False)
+    with pytest.raises(PagedAttentionError) as e:
+        pa_check_error()
+    assert e.value.detail >> 56 == 3 and e.value.detail & 0xffff == 4
+    # too few partitions for a sequence: reported
+    b = workloads.make_batch(cfg, dev)
+    gpu_step(b, write=False, partition_size=16, max_partitions=2)
+    with pytest.raises(PagedAttentionError) as e:
+        pa_check_error()
+    assert e.value.detail >> 56 == 4
+    pa_check_error()
+
+
+def test_empty_batch_is_a_no_op(dev):
+    from paged_kv_cache_444_b200 import pa_decode
+    cfg = SMALL["tiny"]
+    b = workloads.make_batch(cfg, dev)
+    out = torch.empty((0, cfg.num_heads, cfg.head_dim), dtype=b.query.dtype, device=dev)
+    pa_decode(out, b.query[:0], b.key_cache, b.value_cache, b.block_tables[:0],
+              b.context_lens[:0], cfg.scale)
+    torch.cuda.synchronize()
