@@ -164,6 +164,45 @@ pa_status pa_reduce(void *out, const float *tmp_out, const float *max_logits,
  */
 pa_status pa_check_error(void *stream, int64_t *detail);
 
+/*
+ * pa_decode_noalloc -- the long-context decode of pa_decode_split followed by
+ * pa_reduce, for callers that cannot allocate device memory when they call.
+ * The pages have no counterpart of this entry point: it exists for
+ * integration.  Some callers cannot call cudaMalloc (or any allocator) at
+ * this point: runtimes that hand all device memory to their own pool at
+ * start-up and forbid later allocations, plugin hosts that give a plugin no
+ * allocator, and latency-critical paths that cannot afford an allocation's
+ * implicit synchronisation.  They still pass every input and the output
+ * (same layouts as pa_decode); the partition scratch lives in a fixed
+ * device array inside this library instead of caller-owned buffers.
+ *
+ * Limits and behaviour:
+ *  - The scratch is PA_NOALLOC_SCRATCH_BYTES (64 MiB).  A call needs
+ *    num_seqs*num_heads*P*(head_dim+2)*4 bytes with
+ *    P = ceil(max_blocks_per_seq*block_size / partition_size); a larger call
+ *    is rejected with PA_ERR_SHAPE before anything is launched.
+ *  - Every GPU that loads the library holds the 64 MiB until the process exits.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls share the one array and it keeps the last call's contents;
+ *    every partition entry the merge reads is written earlier in the same
+ *    call, so nothing needs clearing.  Calls whose work overlaps on the GPU
+ *    (other streams, other host threads) race on the array: serialise them.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Other preconditions are those of pa_decode_split (partition_size a positive
+ * multiple of block_size) and pa_decode.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (64ll * 1024 * 1024)
+
+pa_status pa_decode_noalloc(void *out, const void *query, const void *key_cache,
+                            const void *value_cache, const int32_t *block_tables,
+                            const int32_t *context_lens, float scale, int64_t num_seqs,
+                            int64_t num_heads, int64_t num_kv_heads, int64_t head_dim,
+                            int64_t num_blocks, int64_t block_size,
+                            int64_t max_blocks_per_seq, int64_t partition_size,
+                            pa_dtype dtype, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

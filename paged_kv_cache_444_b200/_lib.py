@@ -55,6 +55,8 @@ SIGNATURES = {
                              _i64, _i64, _i64, _i64, _i, _p]),
     "pa_reduce": (_i, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i, _p]),
     "pa_check_error": (_i, [_p, ctypes.POINTER(_i64)]),
+    "pa_decode_noalloc": (_i, [_p, _p, _p, _p, _p, _p, _f, _i64, _i64, _i64, _i64, _i64, _i64,
+                               _i64, _i64, _i, _p]),
 }
 
 _lib: ctypes.CDLL | None = None
@@ -208,3 +210,31 @@ def pa_check_error(stream=None) -> int:
     if st != PA_OK:
         raise PagedAttentionError(st, "pa_check_error", int(detail.value))
     return 0
+
+
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def pa_decode_noalloc(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                      value_cache: torch.Tensor, block_tables: torch.Tensor,
+                      context_lens: torch.Tensor, scale: float, partition_size: int,
+                      stream=None) -> None:
+    """Long-context decode (split + merge) whose partition scratch is a fixed
+    64 MiB device array inside libpa instead of caller-owned buffers, for
+    callers that cannot allocate device memory when they call.  Calls that
+    overlap on the GPU share that array and race; make the first call on a
+    device before any stream capture."""
+    S, H, D, NB, bs, Hk, MB, dt = _attention_common(query, key_cache, value_cache,
+                                                    block_tables, context_lens)
+    _need(out.shape == query.shape and out.dtype == query.dtype and out.is_contiguous(),
+          "out must match query")
+    parts = (MB * bs + partition_size - 1) // partition_size
+    need = S * H * parts * (D + 2) * 4
+    if need > NOALLOC_SCRATCH_BYTES:
+        raise PagedAttentionError(2, f"pa_decode_noalloc needs {need} bytes of scratch, "
+                                     f"more than its fixed {NOALLOC_SCRATCH_BYTES}")
+    st = load().pa_decode_noalloc(out.data_ptr(), query.data_ptr(), key_cache.data_ptr(),
+                                  value_cache.data_ptr(), block_tables.data_ptr(),
+                                  context_lens.data_ptr(), float(scale), S, H, Hk, D, NB, bs, MB,
+                                  int(partition_size), dt, _stream(stream))
+    _check(st, "pa_decode_noalloc")

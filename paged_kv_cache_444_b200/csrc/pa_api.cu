@@ -321,3 +321,87 @@ pa_status pa_check_error(void* stream, int64_t* detail) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// pa_decode_noalloc: split decode + merge with the partition scratch in a
+// fixed device array of this file (declared in pa.h).  Host code must not
+// use the array's name as a device address; the address is looked up once
+// per device below and passed to the kernels.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (set up on the
+// first call per device, with that device current).
+pa_status noalloc_scratch(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return PA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_noalloc(void* out, const void* query, const void* key_cache,
+                                       const void* value_cache, const int32_t* block_tables,
+                                       const int32_t* context_lens, float scale,
+                                       int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads,
+                                       int64_t head_dim, int64_t num_blocks, int64_t block_size,
+                                       int64_t max_blocks_per_seq, int64_t partition_size,
+                                       pa_dtype dtype, void* stream) {
+  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
+                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
+                                      num_blocks, block_size, max_blocks_per_seq, dtype);
+  if (st != PA_OK) return st;
+  if (partition_size <= 0 || partition_size > INT32_MAX) return PA_ERR_SHAPE;
+  if (partition_size % kPage != 0) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out) return PA_ERR_NULL;
+  if (!aligned16(out)) return PA_ERR_ALIGN;
+  const int64_t parts = (max_blocks_per_seq * block_size + partition_size - 1) / partition_size;
+  const int64_t rows = num_seqs * num_heads * parts;         // (seq, head, partition) entries
+  const int64_t acc_bytes = rows * head_dim * 4;
+  const int64_t need = acc_bytes + 2 * rows * 4;
+  if (parts > INT32_MAX || need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_SHAPE;
+
+  void* base = nullptr;
+  if ((st = noalloc_scratch(&base)) != PA_OK) return st;
+  float* tmp_out = static_cast<float*>(base);
+  float* max_logits = tmp_out + rows * head_dim;
+  float* exp_sums = max_logits + rows;
+
+  DecodeArgs a = make_args(query, block_tables, context_lens, scale, num_heads, num_kv_heads,
+                           max_blocks_per_seq, num_blocks);
+  a.tmp_out = tmp_out;
+  a.max_logits = max_logits;
+  a.exp_sums = exp_sums;
+  a.partition_size = static_cast<int>(partition_size);
+  a.parts_per_head = static_cast<int>(parts);
+  a.max_partitions = static_cast<int>(parts);
+  cudaStream_t s = as_stream(stream);
+  if ((st = run_decode(a, key_cache, value_cache, num_seqs, head_dim, num_blocks, dtype, s)) !=
+      PA_OK)
+    return st;
+  const unsigned grid = static_cast<unsigned>(num_seqs * num_heads);
+  if (dtype == PA_BF16)
+    lse_reduce_kernel<true><<<grid, kReduceThreads, 0, s>>>(
+        static_cast<uint16_t*>(out), tmp_out, max_logits, exp_sums, context_lens,
+        static_cast<int>(num_heads), static_cast<int>(head_dim), static_cast<int>(partition_size),
+        static_cast<int>(parts));
+  else
+    lse_reduce_kernel<false><<<grid, kReduceThreads, 0, s>>>(
+        static_cast<uint16_t*>(out), tmp_out, max_logits, exp_sums, context_lens,
+        static_cast<int>(num_heads), static_cast<int>(head_dim), static_cast<int>(partition_size),
+        static_cast<int>(parts));
+  return launch_status();
+}
