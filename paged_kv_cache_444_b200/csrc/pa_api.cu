@@ -85,25 +85,93 @@ pa_status launch_status() {
 template <int D>
 struct Stages { static constexpr int value = D == 64 ? 4 : 3; };
 
+#ifndef PA_CLUSTER_PAGES
+#define PA_CLUSTER_PAGES 256  // an item with more pages is spread over its cluster
+#endif
+#ifndef PA_CLUSTER_TABLE_PAGES
+#define PA_CLUSTER_TABLE_PAGES 512  // clusters only when a table can hold more pages
+#endif
+
+// Cluster size for a single-pass launch.  Clusters are used only when the
+// block table admits very long sequences (more than PA_CLUSTER_TABLE_PAGES
+// pages): then every item longer than PA_CLUSTER_PAGES pages is spread so that
+// the longest possible one gives each CTA about PA_CLUSTER_TABLE_PAGES pages.
+// A power of two, at most kMaxCluster, and no more than the device can
+// co-schedule for this kernel.
+template <class K>
+int pick_cluster(K kernel, int smem_bytes, int64_t max_pages, int* cache) {
+  int want = 1;
+  while (want < kMaxCluster && static_cast<int64_t>(want) * PA_CLUSTER_TABLE_PAGES < max_pages)
+    want *= 2;
+  int dev = 0;
+  if (want == 1 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
+  if (cache[dev] == 0) {  // largest schedulable cluster size for this kernel on this device
+    int best = 1;
+    for (int c = kMaxCluster; c > 1; c /= 2) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(c, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem_bytes;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = c;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n > 0) {
+        best = c;
+        break;
+      }
+      cudaGetLastError();
+    }
+    cache[dev] = best;
+  }
+  return want < cache[dev] ? want : cache[dev];
+}
+
 template <int D, bool BF16, class Warp>
-pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, const DecodeArgs& a,
-                          long long grid, cudaStream_t stream) {
+pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeArgs a,
+                          long long grid, int64_t max_pages, cudaStream_t stream) {
   constexpr int NST = Stages<D>::value;
   using L = DecodeSmem<D, NST>;
   auto kernel = paged_decode_kernel<D, NST, BF16, Warp>;
   static std::atomic<uint64_t> done{0};
+  static int cluster_cache[kMaxDevices] = {};
   if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
-  kernel<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(km, vm, a);
+  const bool split = a.tmp_out != nullptr;
+  const int c = split ? 1 : pick_cluster(kernel, L::kAlloc, max_pages, cluster_cache);
+  a.cluster_pages = PA_CLUSTER_PAGES;
+  if (c == 1) {
+    kernel<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(km, vm, a);
+    return launch_status();
+  }
+  if (grid * c > INT32_MAX) return PA_ERR_SHAPE;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid * c), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = c;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, km, vm, a) != cudaSuccess) return PA_ERR_CUDA;
   return launch_status();
 }
 
 template <int D, bool BF16>
 pa_status launch_decode_d(const CUtensorMap& km, const CUtensorMap& vm, const DecodeArgs& a,
-                          long long grid, cudaStream_t stream) {
-  if (a.group == 1) return launch_decode_t<D, BF16, SimtWarp<D, BF16>>(km, vm, a, grid, stream);
+                          long long grid, int64_t max_pages, cudaStream_t stream) {
+  if (a.group == 1)
+    return launch_decode_t<D, BF16, SimtWarp<D, BF16>>(km, vm, a, grid, max_pages, stream);
   if (a.group <= 8)
-    return launch_decode_t<D, BF16, MmaWarp<D, BF16, false>>(km, vm, a, grid, stream);
-  return launch_decode_t<D, BF16, MmaWarp<D, BF16, true>>(km, vm, a, grid, stream);
+    return launch_decode_t<D, BF16, MmaWarp<D, BF16, false>>(km, vm, a, grid, max_pages, stream);
+  return launch_decode_t<D, BF16, MmaWarp<D, BF16, true>>(km, vm, a, grid, max_pages, stream);
 }
 
 // Shared validation of the attention arguments (host only, no CUDA calls).
@@ -146,11 +214,12 @@ pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cach
   const long long grid = num_seqs * a.num_kv_heads * static_cast<long long>(a.parts_per_head);
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
   const bool bf16 = dtype == PA_BF16;
+  const int64_t max_pages = a.max_blocks_per_seq;  // block_size == 16 == one page
   if (head_dim == 64)
-    return bf16 ? launch_decode_d<64, true>(km, vm, a, grid, stream)
-                : launch_decode_d<64, false>(km, vm, a, grid, stream);
-  return bf16 ? launch_decode_d<128, true>(km, vm, a, grid, stream)
-              : launch_decode_d<128, false>(km, vm, a, grid, stream);
+    return bf16 ? launch_decode_d<64, true>(km, vm, a, grid, max_pages, stream)
+                : launch_decode_d<64, false>(km, vm, a, grid, max_pages, stream);
+  return bf16 ? launch_decode_d<128, true>(km, vm, a, grid, max_pages, stream)
+              : launch_decode_d<128, false>(km, vm, a, grid, max_pages, stream);
 }
 
 DecodeArgs make_args(const void* query, const int32_t* block_tables, const int32_t* context_lens,
@@ -169,6 +238,8 @@ DecodeArgs make_args(const void* query, const int32_t* block_tables, const int32
   a.partition_size = 0;
   a.parts_per_head = 1;
   a.max_partitions = 1;
+  a.num_seqs = 0;
+  a.longest_first = 0;
   return a;
 }
 
@@ -236,6 +307,8 @@ pa_status pa_decode(void* out, const void* query, const void* key_cache, const v
   DecodeArgs a = make_args(query, block_tables, context_lens, scale, num_heads, num_kv_heads,
                            max_blocks_per_seq, num_blocks);
   a.out = static_cast<uint16_t*>(out);
+  a.num_seqs = static_cast<int>(num_seqs);
+  a.longest_first = num_seqs > 1 && num_seqs <= kLptMaxSeqs;
   return run_decode(a, key_cache, value_cache, num_seqs, head_dim, num_blocks, dtype,
                     as_stream(stream));
 }
@@ -281,8 +354,8 @@ pa_status pa_reduce(void* out, const float* tmp_out, const float* max_logits,
     return PA_ERR_SHAPE;
   if (num_seqs == 0) return PA_OK;
   if (!out || !tmp_out || !max_logits || !exp_sums || !context_lens) return PA_ERR_NULL;
-  if (head_dim % 2 != 0 || head_dim > 2 * kReduceThreads) return PA_ERR_UNSUPPORTED;
-  if ((reinterpret_cast<uintptr_t>(out) & 3u) || (reinterpret_cast<uintptr_t>(tmp_out) & 7u))
+  if (head_dim % 4 != 0 || head_dim > 4 * kReduceThreads) return PA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(out) & 7u) || (reinterpret_cast<uintptr_t>(tmp_out) & 15u))
     return PA_ERR_ALIGN;
   if (num_seqs * num_heads > INT32_MAX || partition_size > INT32_MAX ||
       max_partitions > INT32_MAX)

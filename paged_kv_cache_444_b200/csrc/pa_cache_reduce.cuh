@@ -40,12 +40,14 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 // Log-sum-exp merge of split partitions.  One CTA per (sequence, query head):
 //   M = max_p m_p;  w_p = exp(m_p - M);  out = sum_p w_p acc_p / sum_p w_p l_p.
-// The weights are computed once per partition into shared memory (in chunks
-// of kReduceChunk partitions); each thread then owns two output dims and
-// walks the partitions with coalesced loads.
+// The weights go to shared memory (kReduceChunk partitions at a time).  The
+// partial accumulators are read as float4: thread t owns dims 4*(t % (D/4))
+// of every kReduceThreads/(D/4)-th partition, with kReduceUnroll independent
+// loads in flight, and the partition groups are summed through shared memory.
 // ---------------------------------------------------------------------------
 constexpr int kReduceThreads = 128;
 constexpr int kReduceChunk = 1024;
+constexpr int kReduceUnroll = 4;
 
 template <bool BF16>
 __global__ void __launch_bounds__(kReduceThreads)
@@ -55,6 +57,7 @@ __global__ void __launch_bounds__(kReduceThreads)
                       int partition_size, int max_partitions) {
   __shared__ float w_sh[kReduceChunk];
   __shared__ float red[kReduceThreads / 32];
+  __shared__ float4 part_sh[kReduceThreads];
   const int sh = blockIdx.x;  // s * num_heads + h
   const int s = sh / num_heads;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -65,9 +68,9 @@ __global__ void __launch_bounds__(kReduceThreads)
   if (nparts > max_partitions) nparts = max_partitions;  // flagged by the split kernel
   const size_t base = static_cast<size_t>(sh) * max_partitions;
   uint16_t* o = out + static_cast<size_t>(sh) * head_dim;
-  const int d = tid * 2;
   if (nparts == 0) {
-    if (d < head_dim) *reinterpret_cast<uint32_t*>(o + d) = 0u;
+    for (int d = tid * 2; d < head_dim; d += kReduceThreads * 2)
+      *reinterpret_cast<uint32_t*>(o + d) = 0u;
     return;
   }
 
@@ -83,8 +86,12 @@ __global__ void __launch_bounds__(kReduceThreads)
   for (int w = 1; w < kReduceThreads / 32; ++w) big_m = fmaxf(big_m, red[w]);
   __syncthreads();
 
+  const int quads = head_dim >> 2;                 // float4 columns per row
+  const int groups = kReduceThreads / quads;       // partition groups (head_dim <= 4*threads)
+  const int q = tid % quads, grp = tid / quads;
+  const bool active = grp < groups;
   float lsum = 0.f;
-  float2 acc = make_float2(0.f, 0.f);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int c0 = 0; c0 < nparts; c0 += kReduceChunk) {
     const int n = min(kReduceChunk, nparts - c0);
     for (int p = tid; p < n; p += kReduceThreads) {
@@ -93,12 +100,24 @@ __global__ void __launch_bounds__(kReduceThreads)
       lsum += w * exp_sums[base + c0 + p];
     }
     __syncthreads();
-    if (d < head_dim) {
-      const float* src = tmp_out + (base + c0) * head_dim + d;
-      for (int p = 0; p < n; ++p) {
-        const float2 v = *reinterpret_cast<const float2*>(src + static_cast<size_t>(p) * head_dim);
-        acc.x += w_sh[p] * v.x;
-        acc.y += w_sh[p] * v.y;
+    if (active) {
+      const float4* src = reinterpret_cast<const float4*>(tmp_out + (base + c0) * head_dim) + q;
+      int p = grp;
+      for (; p + (kReduceUnroll - 1) * groups < n; p += kReduceUnroll * groups) {
+        float4 v[kReduceUnroll];
+#pragma unroll
+        for (int u = 0; u < kReduceUnroll; ++u)
+          v[u] = __ldg(src + static_cast<size_t>(p + u * groups) * quads);
+#pragma unroll
+        for (int u = 0; u < kReduceUnroll; ++u) {
+          const float w = w_sh[p + u * groups];
+          acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+        }
+      }
+      for (; p < n; p += groups) {
+        const float4 v = __ldg(src + static_cast<size_t>(p) * quads);
+        const float w = w_sh[p];
+        acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
       }
     }
     __syncthreads();
@@ -106,13 +125,22 @@ __global__ void __launch_bounds__(kReduceThreads)
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
   if (lane == 0) red[warp] = lsum;
+  part_sh[tid] = acc;
   __syncthreads();
   float big_l = 0.f;
 #pragma unroll
   for (int w = 0; w < kReduceThreads / 32; ++w) big_l += red[w];
-  if (d < head_dim) {
-    const float inv = big_l > 0.f ? 1.f / big_l : 0.f;
-    *reinterpret_cast<uint32_t*>(o + d) = pack2<BF16>(acc.x * inv, acc.y * inv);
+  const float inv = big_l > 0.f ? 1.f / big_l : 0.f;
+  if (tid < quads) {
+    float4 t = part_sh[tid];
+    for (int g = 1; g < groups; ++g) {
+      const float4 u = part_sh[g * quads + tid];
+      t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+    }
+    uint2 packed;
+    packed.x = pack2<BF16>(t.x * inv, t.y * inv);
+    packed.y = pack2<BF16>(t.z * inv, t.w * inv);
+    *reinterpret_cast<uint2*>(o + tid * 4) = packed;
   }
 }
 

@@ -40,6 +40,8 @@ constexpr int kPage = 16;       // tokens per physical block (block_size)
 constexpr int kWarps = 4;       // warps per CTA
 constexpr int kThreads = kWarps * 32;
 constexpr int kBoxBytes = kPage * 128;  // one 16 x 64-element TMA box
+constexpr int kMaxCluster = 8;          // CTAs per item at most (portable cluster size)
+constexpr int kLptMaxSeqs = 256;        // longest-first ordering for batches up to this size
 
 struct DecodeArgs {
   const uint16_t* query;      // [S, H, D]
@@ -58,7 +60,11 @@ struct DecodeArgs {
   int partition_size;         // tokens per item in split mode (multiple of 16)
   int parts_per_head;         // grid items per (seq, kv head): max_partitions or 1
   int max_partitions;
+  int cluster_pages;          // an item with more pages than this is spread over its cluster
+  int num_seqs;
+  int longest_first;          // order single-pass items by descending context length
 };
+
 
 template <int D, int NST>
 struct DecodeSmem {
@@ -69,11 +75,16 @@ struct DecodeSmem {
   static constexpr int kProbOffset = kBarOffset + kWarps * NST * 8;
   static constexpr int kRedMOffset = kProbOffset + kWarps * kPage * 4;
   static constexpr int kRedLOffset = kRedMOffset + kWarps * 16 * 4;
-  static constexpr int kBytes = kRedLOffset + kWarps * 16 * 4;
+  static constexpr int kPartMOffset = kRedLOffset + kWarps * 16 * 4;
+  static constexpr int kPartLOffset = kPartMOffset + 16 * 4;
+  static constexpr int kBytes = kPartLOffset + 16 * 4;
   static constexpr int kAlloc = kBytes + 1024;            // + alignment slack
-  // the merge buffer (kWarps x group x D floats) reuses the stage area
-  static_assert(kWarps * 16 * D * 4 <= kStagesBytes, "merge buffer must fit in the stages");
+  // the merge buffers reuse the stage area: per-warp rows (kWarps x group x D
+  // floats) and, for an item spread over a cluster, this CTA's merged rows
+  static constexpr int kPartAccOffset = kWarps * 16 * D * 4;
+  static_assert(kPartAccOffset + 16 * D * 4 <= kStagesBytes, "merge buffers must fit in the stages");
   static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
+  static_assert((kLptMaxSeqs + 1) * 4 <= kStagesBytes, "length table must fit in the stages");
 };
 
 // Address of 16-byte chunk `c` (0 .. D/8-1) of row `r` in a swizzled page.
@@ -339,7 +350,18 @@ struct SimtWarp {
 };
 
 // ---------------------------------------------------------------------------
-// The kernel: one (sequence, KV head, partition) item per CTA.
+// The kernel: one (sequence, KV head, partition) item per cluster.
+//
+// Launched without a cluster attribute, every CTA is a cluster of one and
+// owns one item.  Launched with clusters of C CTAs (pa_decode only), an item
+// longer than cluster_pages pages is spread over all C CTAs of its cluster
+// (page i goes to CTA i % C, then to warp (i / C) % 4); each CTA merges its
+// four warps in shared memory, then the CTAs merge their partial rows through
+// distributed shared memory, each CTA finishing a slice of the outputs.  A
+// shorter item stays on CTA 0 and the other CTAs of its cluster exit at once;
+// the choice depends only on the item's length, so every CTA of a cluster
+// takes the same branch and either all of them reach both cluster barriers
+// or none does.
 // ---------------------------------------------------------------------------
 template <int D, int NST, bool BF16, class Warp>
 __global__ void __launch_bounds__(kThreads)
@@ -350,40 +372,78 @@ __global__ void __launch_bounds__(kThreads)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int csize = static_cast<int>(cluster_nctarank());
+  const int crank = static_cast<int>(cluster_ctarank());
 
-  int item = blockIdx.x;
+  int item = blockIdx.x / csize;
   const int part = item % a.parts_per_head;
   item /= a.parts_per_head;
   const int kvh = item % a.num_kv_heads;
-  const int s = item / a.num_kv_heads;
+  int s = item / a.num_kv_heads;
   const int group = a.group;
   const bool split = a.tmp_out != nullptr;
+  const bool reporter = threadIdx.x == 0 && crank == 0 && part == 0 && kvh == 0;
+
+  // ---- longest-first order: grid slot s takes the s-th longest sequence
+  // (ties by index), so that long items start first and short ones fill the
+  // tail.  The rank of every sequence is counted against all others. ----
+  if (a.longest_first) {
+    int* lens = reinterpret_cast<int*>(smem);      // stage area, not in use yet
+    int* chosen = lens + kLptMaxSeqs;
+    const int n4 = (a.num_seqs + 3) >> 2;
+    for (int i = threadIdx.x; i < n4 * 4; i += kThreads)
+      lens[i] = i < a.num_seqs ? max(a.context_lens[i], 0) : -1;  // -1 pads: never counted
+    __syncthreads();
+    const int4* lens4 = reinterpret_cast<const int4*>(lens);
+    for (int t = threadIdx.x; t < a.num_seqs; t += kThreads) {
+      const int lt = lens[t];
+      int rank = 0;
+      for (int j4 = 0; j4 < n4; ++j4) {
+        const int4 v = lens4[j4];
+        const int j = j4 * 4;
+        rank += (v.x > lt) | ((v.x == lt) & (j < t));
+        rank += (v.y > lt) | ((v.y == lt) & (j + 1 < t));
+        rank += (v.z > lt) | ((v.z == lt) & (j + 2 < t));
+        rank += (v.w > lt) | ((v.w == lt) & (j + 3 < t));
+      }
+      if (rank == s) *chosen = t;
+    }
+    __syncthreads();
+    s = *chosen;
+    __syncthreads();  // the stage area is about to be reused
+  }
 
   // ---- context length and this item's token range ----
   int ctx = a.context_lens[s];
   const int cap = a.max_blocks_per_seq * kPage;
   if (ctx < 0 || ctx > cap) {
-    if (threadIdx.x == 0 && part == 0 && kvh == 0) record_error(kErrContextLen, s);
+    if (reporter) record_error(kErrContextLen, s);
     ctx = ctx < 0 ? 0 : cap;
   }
   int t_begin = 0, t_end = ctx;
   if (split) {
-    if (threadIdx.x == 0 && part == 0 && kvh == 0 &&
-        (ctx + a.partition_size - 1) / a.partition_size > a.max_partitions)
+    if (reporter && (ctx + a.partition_size - 1) / a.partition_size > a.max_partitions)
       record_error(kErrPartitions, s);
     t_begin = part * a.partition_size;
     t_end = min(t_begin + a.partition_size, ctx);
     if (t_begin >= t_end) return;  // partition past the end: nothing to write
   } else if (ctx == 0) {
     // empty sequence: zero output rows
-    uint16_t* o = a.out + (static_cast<size_t>(s) * a.num_heads + kvh * group) * D;
-    for (int i = threadIdx.x; i < group * D; i += kThreads) o[i] = 0;
+    if (crank == 0) {
+      uint16_t* o = a.out + (static_cast<size_t>(s) * a.num_heads + kvh * group) * D;
+      for (int i = threadIdx.x; i < group * D; i += kThreads) o[i] = 0;
+    }
     return;
   }
 
   const int first_page = t_begin / kPage;
   const int n_pages = (t_end - first_page * kPage + kPage - 1) / kPage;
-  const int my_pages = n_pages > warp ? (n_pages - warp + kWarps - 1) / kWarps : 0;
+  const bool spread = csize > 1 && n_pages > a.cluster_pages;
+  if (csize > 1 && !spread && crank != 0) return;  // short item: CTA 0 alone
+  const int ctas = spread ? csize : 1;             // CTAs sharing this item
+  const int page0 = (spread ? crank : 0) + ctas * warp;  // this warp's first page
+  const int pstride = ctas * kWarps;                      // and its page stride
+  const int my_pages = n_pages > page0 ? (n_pages - page0 + pstride - 1) / pstride : 0;
   const int32_t* bt = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + first_page;
 
   const uint32_t stage0 = smem_addr(smem) + warp * NST * L::kStageBytes;
@@ -401,7 +461,7 @@ __global__ void __launch_bounds__(kThreads)
   auto load_ids = [&](int win) -> int {
     const int k = win * 32 + lane;
     if (k >= my_pages) return -1;
-    const int idx = warp + k * kWarps;
+    const int idx = page0 + k * pstride;
     int id = bt[idx];
     if (id < 0 || id >= a.num_blocks) {
       record_error(kErrBlockId, static_cast<long long>(row_base + idx));
@@ -454,7 +514,7 @@ __global__ void __launch_bounds__(kThreads)
       break;
     }
     const uint32_t kb = stage0 + stg * L::kStageBytes;
-    const int tok0 = (first_page + warp + k * kWarps) * kPage;
+    const int tok0 = (first_page + page0 + k * pstride) * kPage;
     st.page(kb, kb + L::kPageBytes, tok0, t_end, a.scale_log2, lane, probs);
     __syncwarp();
     if (k + NST < my_pages) issue(k + NST);
@@ -476,6 +536,9 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
 
   const int h0 = kvh * group;
+  float* part_acc = reinterpret_cast<float*>(smem + L::kPartAccOffset);
+  float* part_m = reinterpret_cast<float*>(smem + L::kPartMOffset);
+  float* part_l = reinterpret_cast<float*>(smem + L::kPartLOffset);
   for (int o = threadIdx.x * 2; o < group * D; o += kThreads * 2) {
     const int g = o / D, d = o % D;
     float mw[kWarps];
@@ -497,7 +560,14 @@ __global__ void __launch_bounds__(kThreads)
       }
     }
     const size_t hrow = static_cast<size_t>(s) * a.num_heads + h0 + g;
-    if (split) {
+    if (spread) {
+      // this CTA's merged rows, for the cluster-wide merge below
+      *reinterpret_cast<float2*>(part_acc + g * D + d) = make_float2(o0, o1);
+      if (d == 0) {
+        part_m[g] = big_m;
+        part_l[g] = big_l;
+      }
+    } else if (split) {
       const size_t pidx = hrow * a.max_partitions + part;
       *reinterpret_cast<float2*>(a.tmp_out + pidx * D + d) = make_float2(o0, o1);
       if (d == 0) {
@@ -509,6 +579,42 @@ __global__ void __launch_bounds__(kThreads)
       *reinterpret_cast<uint32_t*>(a.out + hrow * D + d) = pack2<BF16>(o0 * inv, o1 * inv);
     }
   }
+  if (!spread) return;
+
+  // ---- cluster-wide merge through distributed shared memory ----
+  cluster_sync();  // every CTA's part_* rows are complete and visible
+  {
+    const int pairs = group * D / 2;
+    const int per = (pairs + ctas - 1) / ctas;
+    const int lo = crank * per, hi = min(pairs, lo + per);
+    const uint32_t acc_base = smem_addr(part_acc), m_base = smem_addr(part_m),
+                   l_base = smem_addr(part_l);
+    for (int pr = lo + threadIdx.x; pr < hi; pr += kThreads) {
+      const int o = pr * 2, g = o / D, d = o % D;
+      float mc[kMaxCluster];
+      float big_m = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kMaxCluster; ++c) {
+        mc[c] = c < ctas ? ld_cluster_f32(map_cluster(m_base + g * 4, c)) : -INFINITY;
+        big_m = fmaxf(big_m, mc[c]);
+      }
+      float big_l = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < kMaxCluster; ++c) {
+        const float e = (mc[c] == -INFINITY) ? 0.f : ex2(mc[c] - big_m);
+        if (e != 0.f) {
+          big_l += e * ld_cluster_f32(map_cluster(l_base + g * 4, c));
+          const float2 v = ld_cluster_f32x2(map_cluster(acc_base + (g * D + d) * 4, c));
+          o0 += e * v.x;
+          o1 += e * v.y;
+        }
+      }
+      const size_t hrow = static_cast<size_t>(s) * a.num_heads + h0 + g;
+      const float inv = big_l > 0.f ? 1.f / big_l : 0.f;
+      *reinterpret_cast<uint32_t*>(a.out + hrow * D + d) = pack2<BF16>(o0 * inv, o1 * inv);
+    }
+  }
+  cluster_sync();  // no CTA leaves while another may still read its shared memory
 }
 
 }  // namespace pa

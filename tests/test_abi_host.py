@@ -77,7 +77,8 @@ def test_split_and_reduce_validation(lib):
     r = lib.pa_reduce
     assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 128, 0, 1, 0, None) == SHAPE
     assert r(None, FAKE, FAKE, FAKE, FAKE, 4, 8, 128, 512, 1, 0, None) == NULL
-    assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 512, 512, 1, 0, None) == UNSUP
+    assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 130, 512, 1, 0, None) == UNSUP
+    assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 516, 512, 1, 0, None) == UNSUP
     assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 128, 512, 1, 0, None) == OK
 
 

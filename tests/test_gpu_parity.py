@@ -193,6 +193,44 @@ def test_long_sequence_many_pages_per_warp(dev, oracle_lib):
     _check_close(out, ref, cfg, "long single pass")
 
 
+@pytest.mark.parametrize("name,ctx", [
+    # long and short items in one launch, with a block table wide enough
+    # (> 512 pages) that single-pass decode runs in thread-block clusters:
+    # items over 256 pages are spread over the CTAs of their cluster (merged
+    # through distributed shared memory), shorter ones stay on one CTA
+    ("gqa_small", (1, 40, 4097, 5000, 17000)),
+    ("gqa16_two_rows", (17, 9000, 4200)),
+    ("d64_gqa2", (5, 12000, 4100)),
+    ("mha_bf16", (4300, 1, 8200)),
+])
+def test_cluster_spread_items_match_oracle(name, ctx, dev, oracle_lib):
+    base = SMALL[name]
+    need = sum((c + 15) // 16 for c in ctx)
+    cfg = base.scaled(num_seqs=len(ctx), ctx=("fixed", ctx), num_blocks=need + 64)
+    batch = workloads.make_batch(cfg, dev)
+    width = 1100  # table columns past each sequence's pages are never read
+    pad = torch.full((cfg.num_seqs, width - batch.block_tables.shape[1]), -1,
+                     dtype=torch.int32, device=dev)
+    batch.block_tables = torch.cat([batch.block_tables, pad], dim=1).contiguous()
+    host = HostCopy(batch)
+    ref, _, _ = oracle_step(oracle_lib, host)
+    out, _ = gpu_step(batch)
+    pa_check_error()
+    _check_close(out, ref, cfg, f"{name} spread")
+
+
+def test_many_sequences_natural_order(dev, oracle_lib):
+    # more sequences than the longest-first ordering handles
+    cfg = SMALL["mha_small"].scaled(num_seqs=300, num_heads=2, num_kv_heads=2, num_blocks=2048,
+                                    ctx=("uniform", 0, 90), seed=21)
+    batch = workloads.make_batch(cfg, dev)
+    host = HostCopy(batch)
+    ref, _, _ = oracle_step(oracle_lib, host)
+    out, _ = gpu_step(batch)
+    pa_check_error()
+    _check_close(out, ref, cfg, "natural order")
+
+
 def test_write_padding_and_strided_rows(dev, oracle_lib):
     cfg = SMALL["gqa_small"]
     batch = workloads.make_batch(cfg, dev)
