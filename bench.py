@@ -200,24 +200,65 @@ class Step:
                 ev[2].record()
 
 
-def time_steps(step: Step, steps: int, warmup: int, world: int, device, clocks=None):
+def time_steps(step: Step, steps: int, warmup: int, world: int, device, clocks=None,
+               kernel_steps: int = 200):
+    """Warm up, then time `steps` steps back to back (CUDA events at the two
+    ends only, so consecutive launches may overlap as they would in use), then
+    time `kernel_steps` more with an event between every two kernels for the
+    per-kernel durations.  Returns (ms per step, [ms per kernel])."""
     for _ in range(warmup):
         step.run()
     torch.cuda.synchronize()
     barrier(world, device)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(step.launches + 1)]
-           for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ctx = clocks if clocks is not None else _Null()
     with ctx:
         torch.cuda.synchronize()
-        for k in range(steps):
-            step.run(evs[k])
+        start.record()
+        for _ in range(steps):
+            step.run()
+        end.record()
         torch.cuda.synchronize()
     barrier(world, device)
-    total_ms = evs[0][0].elapsed_time(evs[-1][-1])
-    per_kernel = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps
+    ms = start.elapsed_time(end) / steps
+    ks = max(1, min(steps, kernel_steps))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(step.launches + 1)]
+           for _ in range(ks)]
+    for k in range(ks):
+        step.run(evs[k])
+    torch.cuda.synchronize()
+    per_kernel = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / ks
                   for i in range(step.launches)]
-    return total_ms / steps, per_kernel
+    return ms, per_kernel
+
+
+def graph_steps(step: Step, steps: int, warmup: int) -> float | None:
+    """The same step captured once in a CUDA graph and replayed `steps` times
+    (ms per step), or None if capture is not possible here."""
+    try:
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for _ in range(3):
+                step.run()
+        torch.cuda.current_stream().wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step.run()
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(steps):
+            g.replay()
+        end.record()
+        torch.cuda.synchronize()
+        del g
+        return start.elapsed_time(end) / steps
+    except Exception as e:  # pragma: no cover - depends on the box
+        print(f"graph capture unavailable: {e!r}", file=sys.stderr)
+        return None
 
 
 class _Null:
@@ -391,6 +432,7 @@ def run_native(args, world, rank, local):
         step = Step(batch)
         ms, per_kernel = time_steps(step, steps, warmup, world, device, clocks)
         ms_max = max_over_ranks(ms, world, device)
+        gms = graph_steps(step, steps, warmup) if args.graph else None
         ctx = batch.context_lens.cpu().tolist()
         by = workloads.algorithmic_bytes(cfg, ctx)
         attn_ms = per_kernel[1] + (per_kernel[2] if step.ps else 0.0)
@@ -407,6 +449,7 @@ def run_native(args, world, rank, local):
             "kernel_bytes": kern_bytes,
             "bytes": by,
             "tokens_per_s": sum_over_ranks(cfg.num_seqs, world, device) / (ms_max / 1e3),
+            "graph_ms_per_step": gms,
         }
         return cfg, batch, step, res
 
@@ -466,6 +509,8 @@ def run_native(args, world, rank, local):
                    "l2": "inputs larger than L2 (K/V read per step >> 126 MB), no flush",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "decode_tokens_per_s": round(main["tokens_per_s"], 1),
+        "graph_ms_per_step": (round(main["graph_ms_per_step"], 5)
+                              if main["graph_ms_per_step"] else None),
         "attention_gbs": round(main["attention_gbs"], 1),
         "per_kernel_ms": {n: round(v, 5) for n, v in zip(
             ["pa_reshape_and_cache", kname] + (["pa_reduce"] if step.ps else []),
@@ -486,6 +531,8 @@ def run_native(args, world, rank, local):
                 "kernel_frac_of_peak": round(r["kernel_gbs"] / peak, 4),
                 "attention_frac_of_peak": round(r["attention_gbs"] / peak, 4),
                 "decode_tokens_per_s": round(r["tokens_per_s"], 1),
+                "graph_ms_per_step": (round(r["graph_ms_per_step"], 5)
+                                      if r["graph_ms_per_step"] else None),
                 "per_kernel_ms": [round(x, 5) for x in r["per_kernel_ms"]]}
             for n, r in results.items()}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -566,6 +613,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of oracle work for the CPU baseline")
+    ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time the step replayed from a CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

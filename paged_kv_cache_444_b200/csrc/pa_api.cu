@@ -81,6 +81,40 @@ pa_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialisation (the kernel may start while
+// the previous kernel of the stream drains; every kernel here waits for it
+// with griddepcontrol.wait before reading inputs) and, if cluster > 1, as
+// clusters of `cluster` CTAs along x.
+template <class K, class... Args>
+pa_status launch_ex(K kernel, unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                    int cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[2];
+  int n = 0;
+  if (cluster > 1) {
+    attrs[n].id = cudaLaunchAttributeClusterDimension;
+    attrs[n].val.clusterDim.x = cluster;
+    attrs[n].val.clusterDim.y = 1;
+    attrs[n].val.clusterDim.z = 1;
+    ++n;
+  } else {
+    attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attrs;
+  cfg.numAttrs = n;
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
 // Pipeline depth per head_dim: stages of (K page + V page) per warp.
 template <int D>
 struct Stages { static constexpr int value = D == 64 ? 4 : 3; };
@@ -143,25 +177,9 @@ pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeAr
   const bool split = a.tmp_out != nullptr;
   const int c = split ? 1 : pick_cluster(kernel, L::kAlloc, max_pages, cluster_cache);
   a.cluster_pages = PA_CLUSTER_PAGES;
-  if (c == 1) {
-    kernel<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(km, vm, a);
-    return launch_status();
-  }
   if (grid * c > INT32_MAX) return PA_ERR_SHAPE;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid * c), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = L::kAlloc;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = c;
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kernel, km, vm, a) != cudaSuccess) return PA_ERR_CUDA;
-  return launch_status();
+  return launch_ex(kernel, static_cast<unsigned>(grid * c), kThreads, L::kAlloc, stream, c, km,
+                   vm, a);
 }
 
 template <int D, bool BF16>
@@ -285,11 +303,13 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, int64_t key_s
   const int threads = 256;
   int64_t blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 32) blocks = 148 * 32;  // grid-stride beyond 32 CTAs per SM
-  reshape_and_cache_kernel<<<static_cast<unsigned>(blocks), threads, 0, as_stream(stream)>>>(
-      static_cast<const uint16_t*>(key), static_cast<const uint16_t*>(value), key_stride,
-      value_stride, static_cast<uint16_t*>(key_cache), static_cast<uint16_t*>(value_cache),
-      slot_mapping, num_tokens, static_cast<int>(chunks), num_blocks * block_size);
-  return launch_status();
+  return launch_ex(reshape_and_cache_kernel, static_cast<unsigned>(blocks), threads, 0,
+                   as_stream(stream), 1, static_cast<const uint16_t*>(key),
+                   static_cast<const uint16_t*>(value), static_cast<long long>(key_stride),
+                   static_cast<long long>(value_stride), static_cast<uint16_t*>(key_cache),
+                   static_cast<uint16_t*>(value_cache), slot_mapping,
+                   static_cast<long long>(num_tokens), static_cast<int>(chunks),
+                   static_cast<long long>(num_blocks * block_size));
 }
 
 pa_status pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
@@ -361,18 +381,11 @@ pa_status pa_reduce(void* out, const float* tmp_out, const float* max_logits,
       max_partitions > INT32_MAX)
     return PA_ERR_SHAPE;
   const unsigned grid = static_cast<unsigned>(num_seqs * num_heads);
-  cudaStream_t s = as_stream(stream);
-  if (dtype == PA_BF16)
-    lse_reduce_kernel<true><<<grid, kReduceThreads, 0, s>>>(
-        static_cast<uint16_t*>(out), tmp_out, max_logits, exp_sums, context_lens,
-        static_cast<int>(num_heads), static_cast<int>(head_dim), static_cast<int>(partition_size),
-        static_cast<int>(max_partitions));
-  else
-    lse_reduce_kernel<false><<<grid, kReduceThreads, 0, s>>>(
-        static_cast<uint16_t*>(out), tmp_out, max_logits, exp_sums, context_lens,
-        static_cast<int>(num_heads), static_cast<int>(head_dim), static_cast<int>(partition_size),
-        static_cast<int>(max_partitions));
-  return launch_status();
+  auto kernel = dtype == PA_BF16 ? lse_reduce_kernel<true> : lse_reduce_kernel<false>;
+  return launch_ex(kernel, grid, kReduceThreads, 0, as_stream(stream), 1,
+                   static_cast<uint16_t*>(out), tmp_out, max_logits, exp_sums, context_lens,
+                   static_cast<int>(num_heads), static_cast<int>(head_dim),
+                   static_cast<int>(partition_size), static_cast<int>(max_partitions));
 }
 
 pa_status pa_check_error(void* stream, int64_t* detail) {

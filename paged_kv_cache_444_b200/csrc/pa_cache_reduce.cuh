@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(256)
                              uint16_t* __restrict__ key_cache, uint16_t* __restrict__ value_cache,
                              const int64_t* __restrict__ slot_mapping, long long num_tokens,
                              int chunks_per_token, long long num_slots) {
+  pdl_launch_dependents();
+  pdl_wait();
   const long long total = num_tokens * chunks_per_token;
   const long long row = static_cast<long long>(chunks_per_token) * 8;  // elements per token row
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
@@ -40,14 +42,14 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 // Log-sum-exp merge of split partitions.  One CTA per (sequence, query head):
 //   M = max_p m_p;  w_p = exp(m_p - M);  out = sum_p w_p acc_p / sum_p w_p l_p.
-// The weights go to shared memory (kReduceChunk partitions at a time).  The
-// partial accumulators are read as float4: thread t owns dims 4*(t % (D/4))
-// of every kReduceThreads/(D/4)-th partition, with kReduceUnroll independent
-// loads in flight, and the partition groups are summed through shared memory.
+// Single pass: thread t owns the float4 column t % (D/4) of every
+// (threads/(D/4))-th partition and merges them online (running max, with the
+// partial sum and accumulator rescaled when the max grows), loading
+// kReduceBatch partitions before using any so that the loads overlap.  The
+// partition groups are then merged through shared memory the same way.
 // ---------------------------------------------------------------------------
-constexpr int kReduceThreads = 128;
-constexpr int kReduceChunk = 1024;
-constexpr int kReduceUnroll = 4;
+constexpr int kReduceThreads = 256;
+constexpr int kReduceBatch = 8;
 
 template <bool BF16>
 __global__ void __launch_bounds__(kReduceThreads)
@@ -55,12 +57,14 @@ __global__ void __launch_bounds__(kReduceThreads)
                       const float* __restrict__ max_logits, const float* __restrict__ exp_sums,
                       const int32_t* __restrict__ context_lens, int num_heads, int head_dim,
                       int partition_size, int max_partitions) {
-  __shared__ float w_sh[kReduceChunk];
-  __shared__ float red[kReduceThreads / 32];
-  __shared__ float4 part_sh[kReduceThreads];
+  __shared__ float4 acc_sh[kReduceThreads];
+  __shared__ float m_sh[kReduceThreads];
+  __shared__ float l_sh[kReduceThreads];
+  pdl_launch_dependents();
+  pdl_wait();
   const int sh = blockIdx.x;  // s * num_heads + h
   const int s = sh / num_heads;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
 
   int ctx = context_lens[s];
   if (ctx < 0) ctx = 0;
@@ -74,69 +78,59 @@ __global__ void __launch_bounds__(kReduceThreads)
     return;
   }
 
-  // M = max over partitions
-  float mloc = -INFINITY;
-  for (int p = tid; p < nparts; p += kReduceThreads) mloc = fmaxf(mloc, max_logits[base + p]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, off));
-  if (lane == 0) red[warp] = mloc;
-  __syncthreads();
-  float big_m = red[0];
-#pragma unroll
-  for (int w = 1; w < kReduceThreads / 32; ++w) big_m = fmaxf(big_m, red[w]);
-  __syncthreads();
-
   const int quads = head_dim >> 2;                 // float4 columns per row
   const int groups = kReduceThreads / quads;       // partition groups (head_dim <= 4*threads)
   const int q = tid % quads, grp = tid / quads;
-  const bool active = grp < groups;
-  float lsum = 0.f;
+  float m = -INFINITY, l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c0 = 0; c0 < nparts; c0 += kReduceChunk) {
-    const int n = min(kReduceChunk, nparts - c0);
-    for (int p = tid; p < n; p += kReduceThreads) {
-      const float w = ex2((max_logits[base + c0 + p] - big_m) * kLog2e);
-      w_sh[p] = w;
-      lsum += w * exp_sums[base + c0 + p];
-    }
-    __syncthreads();
-    if (active) {
-      const float4* src = reinterpret_cast<const float4*>(tmp_out + (base + c0) * head_dim) + q;
-      int p = grp;
-      for (; p + (kReduceUnroll - 1) * groups < n; p += kReduceUnroll * groups) {
-        float4 v[kReduceUnroll];
+  if (grp < groups) {
+    const float4* rows = reinterpret_cast<const float4*>(tmp_out + base * head_dim) + q;
+    for (int p0 = grp; p0 < nparts; p0 += groups * kReduceBatch) {
+      float mp[kReduceBatch], lp[kReduceBatch];
+      float4 v[kReduceBatch];
 #pragma unroll
-        for (int u = 0; u < kReduceUnroll; ++u)
-          v[u] = __ldg(src + static_cast<size_t>(p + u * groups) * quads);
-#pragma unroll
-        for (int u = 0; u < kReduceUnroll; ++u) {
-          const float w = w_sh[p + u * groups];
-          acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
+      for (int u = 0; u < kReduceBatch; ++u) {
+        const int p = p0 + u * groups;
+        if (p < nparts) {
+          mp[u] = __ldg(max_logits + base + p);
+          lp[u] = __ldg(exp_sums + base + p);
+          v[u] = __ldg(rows + static_cast<size_t>(p) * quads);
         }
       }
-      for (; p < n; p += groups) {
-        const float4 v = __ldg(src + static_cast<size_t>(p) * quads);
-        const float w = w_sh[p];
-        acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+#pragma unroll
+      for (int u = 0; u < kReduceBatch; ++u) {
+        if (p0 + u * groups < nparts) {
+          const float mn = fmaxf(m, mp[u]);
+          const float sc = ex2((m - mn) * kLog2e);     // 0 while m is still -inf
+          const float e = ex2((mp[u] - mn) * kLog2e);
+          acc.x = acc.x * sc + e * v[u].x;
+          acc.y = acc.y * sc + e * v[u].y;
+          acc.z = acc.z * sc + e * v[u].z;
+          acc.w = acc.w * sc + e * v[u].w;
+          l = l * sc + e * lp[u];
+          m = mn;
+        }
       }
     }
-    __syncthreads();
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-  if (lane == 0) red[warp] = lsum;
-  part_sh[tid] = acc;
+  acc_sh[tid] = acc;
+  m_sh[tid] = m;
+  l_sh[tid] = l;
   __syncthreads();
-  float big_l = 0.f;
-#pragma unroll
-  for (int w = 0; w < kReduceThreads / 32; ++w) big_l += red[w];
-  const float inv = big_l > 0.f ? 1.f / big_l : 0.f;
   if (tid < quads) {
-    float4 t = part_sh[tid];
-    for (int g = 1; g < groups; ++g) {
-      const float4 u = part_sh[g * quads + tid];
-      t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+    float big_m = -INFINITY;
+    for (int g = 0; g < groups; ++g) big_m = fmaxf(big_m, m_sh[g * quads + tid]);
+    float big_l = 0.f;
+    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int g = 0; g < groups; ++g) {
+      const float mg = m_sh[g * quads + tid];
+      if (mg == -INFINITY) continue;                 // a group without partitions
+      const float e = ex2((mg - big_m) * kLog2e);
+      const float4 u = acc_sh[g * quads + tid];
+      t.x += e * u.x; t.y += e * u.y; t.z += e * u.z; t.w += e * u.w;
+      big_l += e * l_sh[g * quads + tid];
     }
+    const float inv = big_l > 0.f ? 1.f / big_l : 0.f;
     uint2 packed;
     packed.x = pack2<BF16>(t.x * inv, t.y * inv);
     packed.y = pack2<BF16>(t.z * inv, t.w * inv);

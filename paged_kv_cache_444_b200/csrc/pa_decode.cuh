@@ -374,6 +374,10 @@ __global__ void __launch_bounds__(kThreads)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int csize = static_cast<int>(cluster_nctarank());
   const int crank = static_cast<int>(cluster_ctarank());
+  prefetch_tensormap(&kmap);
+  prefetch_tensormap(&vmap);
+  pdl_launch_dependents();
+  pdl_wait();  // inputs may come from the previous kernel of the stream
 
   int item = blockIdx.x / csize;
   const int part = item % a.parts_per_head;

@@ -146,6 +146,22 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialisation may start while the previous kernel of its stream is still
+// running; pdl_wait() blocks until that kernel has completed and its writes
+// are visible (a no-op for a normal launch).  Every kernel here calls it
+// before its first read of any input, and calls pdl_launch_dependents() early
+// so that the next kernel can be scheduled during its own tail.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Thread-block clusters: rank, size, barrier, distributed shared memory.
 // Without a cluster launch a CTA is a cluster of one (rank 0, size 1).
 // ---------------------------------------------------------------------------
