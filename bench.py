@@ -428,6 +428,11 @@ def run_native(args, world, rank, local):
     def bench_config(name, steps, warmup, clocks=None):
         cfg = workloads.CONFIGS[name]
         cfg = cfg.scaled(seed=cfg.seed + 1000 * rank)
+        if name == args.config and (args.num_seqs or args.num_blocks):
+            # a smaller batch of the same workload (profiling captures only)
+            cfg = cfg.scaled(num_seqs=args.num_seqs or cfg.num_seqs,
+                             num_blocks=args.num_blocks or cfg.num_blocks,
+                             name=f"{cfg.name}[seqs={args.num_seqs or cfg.num_seqs}]")
         batch = workloads.make_batch(cfg, device)
         step = Step(batch)
         ms, per_kernel = time_steps(step, steps, warmup, world, device, clocks)
@@ -450,6 +455,8 @@ def run_native(args, world, rank, local):
             "bytes": by,
             "tokens_per_s": sum_over_ranks(cfg.num_seqs, world, device) / (ms_max / 1e3),
             "graph_ms_per_step": gms,
+            "kernel": "pa_decode_split" if step.ps else "pa_decode",
+            "context_tokens": int(sum(ctx)),
         }
         return cfg, batch, step, res
 
@@ -478,14 +485,7 @@ def run_native(args, world, rank, local):
             "frac": round(main["kernel_gbs"] / peak, 4), "peak_kind": peak_kind,
             "algorithmic_bytes_per_launch": main["kernel_bytes"],
             "traffic": None}
-    tp = ROOT / "profiles" / "traffic.json"
-    if tp.exists():
-        try:
-            t = json.loads(tp.read_text()).get(args.config, {}).get(kname)
-            if t and t.get("source_sha") == kernel_source_digest():
-                roof["traffic"] = t["bytes_per_launch"]
-        except Exception:
-            pass
+    roof["traffic"] = recorded_traffic(args.config, kname, sum(ctx_main))
 
     line = {
         "metric": METRIC,
@@ -529,6 +529,8 @@ def run_native(args, world, rank, local):
                 "attention_gbs": round(r["attention_gbs"], 1),
                 "kernel_gbs": round(r["kernel_gbs"], 1),
                 "kernel_frac_of_peak": round(r["kernel_gbs"] / peak, 4),
+                "kernel_traffic": recorded_traffic(n, r["kernel"], r["context_tokens"]),
+                "kernel_algorithmic_bytes": r["kernel_bytes"],
                 "attention_frac_of_peak": round(r["attention_gbs"] / peak, 4),
                 "decode_tokens_per_s": round(r["tokens_per_s"], 1),
                 "graph_ms_per_step": (round(r["graph_ms_per_step"], 5)
@@ -543,6 +545,26 @@ def run_native(args, world, rank, local):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def recorded_traffic(config: str, kernel: str, context_tokens: int):
+    """DRAM bytes per launch of `kernel` on `config` from the committed ncu
+    capture (profiles/traffic.json), or None if there is none or the kernel
+    sources changed since it was taken."""
+    tp = ROOT / "profiles" / "traffic.json"
+    if not tp.exists():
+        return None
+    try:
+        t = json.loads(tp.read_text()).get(config, {}).get(kernel)
+    except Exception:
+        return None
+    if not t or t.get("source_sha") != kernel_source_digest():
+        return None
+    if t.get("bytes_per_launch"):
+        return int(t["bytes_per_launch"])
+    if t.get("bytes_per_context_token"):
+        return int(t["bytes_per_context_token"] * context_tokens)
+    return None
 
 
 def kernel_source_digest() -> str:
@@ -615,6 +637,10 @@ def main(argv=None):
                     help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="also time the step replayed from a CUDA graph")
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="override the workload's batch size (small profiling captures)")
+    ap.add_argument("--num-blocks", type=int, default=0,
+                    help="override the workload's block pool size (small profiling captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
