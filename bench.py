@@ -232,6 +232,30 @@ def time_steps(step: Step, steps: int, warmup: int, world: int, device, clocks=N
     return ms, per_kernel
 
 
+def shared_prefix_kernel_ms(batch, warmup: int, reps: int = 100) -> float:
+    """CUDA-event time of pa_decode_shared_prefix on a batch with prefix groups
+    (the same attention as pa_decode, reading each shared page once per group)."""
+    from paged_kv_cache_444_b200 import pa_decode_shared_prefix
+    cfg = batch.cfg
+    out = torch.empty_like(batch.query)
+    sizes = (batch.group_starts[1:] - batch.group_starts[:-1]).tolist()
+
+    def run():
+        pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
+                                batch.block_tables, batch.context_lens, batch.group_starts,
+                                batch.prefix_blocks, cfg.scale, max(sizes))
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(reps):
+        run()
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / reps
+
+
 def graph_steps(step: Step, steps: int, warmup: int) -> float | None:
     """The same step captured once in a CUDA graph and replayed `steps` times
     (ms per step), or None if capture is not possible here."""
@@ -438,6 +462,8 @@ def run_native(args, world, rank, local):
         ms, per_kernel = time_steps(step, steps, warmup, world, device, clocks)
         ms_max = max_over_ranks(ms, world, device)
         gms = graph_steps(step, steps, warmup) if args.graph else None
+        shared_ms = shared_prefix_kernel_ms(batch, warmup) if batch.group_starts is not None \
+            else None
         ctx = batch.context_lens.cpu().tolist()
         by = workloads.algorithmic_bytes(cfg, ctx)
         attn_ms = per_kernel[1] + (per_kernel[2] if step.ps else 0.0)
@@ -455,6 +481,7 @@ def run_native(args, world, rank, local):
             "bytes": by,
             "tokens_per_s": sum_over_ranks(cfg.num_seqs, world, device) / (ms_max / 1e3),
             "graph_ms_per_step": gms,
+            "shared_prefix_kernel_ms": shared_ms,
             "kernel": "pa_decode_split" if step.ps else "pa_decode",
             "context_tokens": int(sum(ctx)),
         }
@@ -535,7 +562,9 @@ def run_native(args, world, rank, local):
                 "decode_tokens_per_s": round(r["tokens_per_s"], 1),
                 "graph_ms_per_step": (round(r["graph_ms_per_step"], 5)
                                       if r["graph_ms_per_step"] else None),
-                "per_kernel_ms": [round(x, 5) for x in r["per_kernel_ms"]]}
+                "per_kernel_ms": [round(x, 5) for x in r["per_kernel_ms"]],
+                **({"pa_decode_shared_prefix_ms": round(r["shared_prefix_kernel_ms"], 5)}
+                   if r["shared_prefix_kernel_ms"] else {})}
             for n, r in results.items()}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, ctx_main, bt_main, batch,

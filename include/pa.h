@@ -65,7 +65,8 @@ enum {
     PA_CHECK_BLOCK_ID = 2,      /* block id outside [0, num_blocks); index = s*max_blocks_per_seq + i */
     PA_CHECK_CONTEXT_LEN = 3,   /* context_lens[s] < 0 or > max_blocks_per_seq*block_size; index = s */
     PA_CHECK_PARTITIONS = 4,    /* ceil(context_lens[s]/partition_size) > max_partitions; index = s */
-    PA_CHECK_WAIT_TIMEOUT = 5   /* a shared-memory barrier wait gave up; index = CTA id */
+    PA_CHECK_WAIT_TIMEOUT = 5,  /* a shared-memory barrier wait gave up; index = CTA id */
+    PA_CHECK_GROUP = 6          /* malformed group bounds or prefix length; index = group */
 };
 
 /* Short English name of a status code (static string, never NULL). */
@@ -155,6 +156,33 @@ pa_status pa_reduce(void *out, const float *tmp_out, const float *max_logits,
                     int64_t num_seqs, int64_t num_heads, int64_t head_dim,
                     int64_t partition_size, int64_t max_partitions,
                     pa_dtype dtype, void *stream);
+
+/*
+ * pa_decode_shared_prefix -- pa_decode for a batch whose sequences come in
+ * groups that share the first blocks of their tables (beam candidates, a
+ * common prompt prefix): "vLLM PagedAttention 原理与源码深度解析" §3.3 (beams
+ * share prefix blocks through ref_count) and "读一个真实 serving 系统 · vLLM
+ * 架构巡礼" §2 (KVCacheBlock.ref_cnt).  The output equals pa_decode's (same
+ * formula, fp32 accumulation, another summation order), but each shared
+ * page is read once per group instead of once per member.
+ *   group_starts   [num_groups + 1] int32: group g is sequences
+ *                  [group_starts[g], group_starts[g+1]); 0 = starts[0] <= ... <= starts[G] = num_seqs
+ *   prefix_blocks  [num_groups] int32: entries 0 .. prefix_blocks[g]-1 of every
+ *                  member's block table are the same ids (read from the first member)
+ *   max_group_size host-side upper bound of any group's size
+ * Other arguments and layouts as pa_decode.  A group larger than
+ * max_group_size or malformed group bounds are reported by pa_check_error
+ * (PA_CHECK_GROUP).  Members are processed 16 / (num_heads/num_kv_heads) at a
+ * time, so a group wider than that re-reads its prefix once per chunk.
+ */
+pa_status pa_decode_shared_prefix(void *out, const void *query, const void *key_cache,
+                                  const void *value_cache, const int32_t *block_tables,
+                                  const int32_t *context_lens, const int32_t *group_starts,
+                                  const int32_t *prefix_blocks, float scale, int64_t num_seqs,
+                                  int64_t num_groups, int64_t max_group_size, int64_t num_heads,
+                                  int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                                  int64_t block_size, int64_t max_blocks_per_seq,
+                                  pa_dtype dtype, void *stream);
 
 /*
  * pa_check_error -- synchronise `stream`, read and clear the current device's

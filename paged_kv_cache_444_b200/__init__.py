@@ -11,11 +11,12 @@ from __future__ import annotations
 import torch
 
 from ._lib import (PagedAttentionError, load, pa_check_error, pa_decode, pa_decode_noalloc,
-                   pa_decode_split, pa_reduce, pa_reshape_and_cache)
+                   pa_decode_shared_prefix, pa_decode_split, pa_reduce, pa_reshape_and_cache)
 
 __all__ = [
     "PagedAttentionError", "load", "pa_reshape_and_cache", "pa_decode", "pa_decode_split",
-    "pa_reduce", "pa_check_error", "pa_decode_noalloc", "SplitWorkspace", "decode_step",
+    "pa_reduce", "pa_check_error", "pa_decode_noalloc", "pa_decode_shared_prefix",
+    "SplitWorkspace", "decode_step",
 ]
 
 

@@ -23,7 +23,8 @@ PA_OK = 0
 STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_NULL", 2: "PA_ERR_SHAPE", 3: "PA_ERR_DTYPE",
                 4: "PA_ERR_ALIGN", 5: "PA_ERR_UNSUPPORTED", 6: "PA_ERR_CUDA",
                 7: "PA_ERR_BOUNDS"}
-CHECK_CODES = {1: "slot", 2: "block_id", 3: "context_len", 4: "partitions", 5: "wait_timeout"}
+CHECK_CODES = {1: "slot", 2: "block_id", 3: "context_len", 4: "partitions", 5: "wait_timeout",
+               6: "group"}
 DTYPE_CODES = {torch.float16: 0, torch.bfloat16: 1}
 
 
@@ -57,6 +58,8 @@ SIGNATURES = {
     "pa_check_error": (_i, [_p, ctypes.POINTER(_i64)]),
     "pa_decode_noalloc": (_i, [_p, _p, _p, _p, _p, _p, _f, _i64, _i64, _i64, _i64, _i64, _i64,
                                _i64, _i64, _i, _p]),
+    "pa_decode_shared_prefix": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _f, _i64, _i64, _i64, _i64,
+                                     _i64, _i64, _i64, _i64, _i64, _i, _p]),
 }
 
 _lib: ctypes.CDLL | None = None
@@ -200,6 +203,30 @@ def pa_reduce(out: torch.Tensor, tmp_out: torch.Tensor, max_logits: torch.Tensor
                           exp_sums.data_ptr(), context_lens.data_ptr(), S, H, D,
                           int(partition_size), P, _dtype_code(out), _stream(stream))
     _check(st, "pa_reduce")
+
+
+def pa_decode_shared_prefix(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                            value_cache: torch.Tensor, block_tables: torch.Tensor,
+                            context_lens: torch.Tensor, group_starts: torch.Tensor,
+                            prefix_blocks: torch.Tensor, scale: float, max_group_size: int,
+                            stream=None) -> None:
+    """pa_decode for sequences grouped by a shared table prefix: group g is
+    sequences group_starts[g] .. group_starts[g+1]-1, whose first
+    prefix_blocks[g] table entries are the same ids (read once per group)."""
+    S, H, D, NB, bs, Hk, MB, dt = _attention_common(query, key_cache, value_cache,
+                                                    block_tables, context_lens)
+    _need(out.shape == query.shape and out.dtype == query.dtype and out.is_contiguous(),
+          "out must match query")
+    n_groups = prefix_blocks.shape[0]
+    _need(group_starts.dtype == torch.int32 and group_starts.shape == (n_groups + 1,),
+          "group_starts must be [num_groups + 1] int32")
+    _need(prefix_blocks.dtype == torch.int32, "prefix_blocks must be int32")
+    st = load().pa_decode_shared_prefix(
+        out.data_ptr(), query.data_ptr(), key_cache.data_ptr(), value_cache.data_ptr(),
+        block_tables.data_ptr(), context_lens.data_ptr(), group_starts.data_ptr(),
+        prefix_blocks.data_ptr(), float(scale), S, n_groups, int(max_group_size), H, Hk, D, NB,
+        bs, MB, dt, _stream(stream))
+    _check(st, "pa_decode_shared_prefix")
 
 
 def pa_check_error(stream=None) -> int:

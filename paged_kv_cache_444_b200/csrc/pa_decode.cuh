@@ -123,7 +123,16 @@ struct MmaWarp {
   }
 
   __device__ __forceinline__ void page(uint32_t kbase, uint32_t vbase, int tok0, int t_end,
-                                       float scale_log2, int lane, float*) {
+                                       float scale_log2, int lane, float* probs) {
+    page_rows(kbase, vbase, tok0, t_end, t_end, scale_log2, lane);
+    (void)probs;
+  }
+
+  // One page with a token limit per row: row r0 (lane/4) sees tokens < lim0,
+  // row r1 (lane/4 + 8) tokens < lim1.  A row whose tokens are all masked so
+  // far keeps m = -inf, l = 0, O = 0 (exp of -inf against a zero reference).
+  __device__ __forceinline__ void page_rows(uint32_t kbase, uint32_t vbase, int tok0, int lim0,
+                                            int lim1, float scale_log2, int lane) {
     const int tig = lane & 3;
     // ---- S = Q K^T for the page's 16 tokens (two 8-token n-tiles) ----
     float sc[2][4];
@@ -145,39 +154,66 @@ struct MmaWarp {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int t = tok0 + nt * 8 + tig * 2 + (i & 1);
-        const float x = t < t_end ? sc[nt][i] * scale_log2 : -INFINITY;
+        const float x = t < (i < 2 ? lim0 : lim1) ? sc[nt][i] * scale_log2 : -INFINITY;
         sc[nt][i] = x;
         if (i < 2) mx0 = fmaxf(mx0, x); else mx1 = fmaxf(mx1, x);
       }
     }
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    const float mn0 = fmaxf(m[0], mx0);
+    // reference max: the running max, or 0 while a row has seen no token
+    // (then every exponent below is of -inf and gives 0, never NaN)
+    const float mn0r = fmaxf(m[0], mx0);
+    const float mn0 = mn0r == -INFINITY ? 0.f : mn0r;
     const float al0 = ex2(m[0] - mn0);
-    m[0] = mn0;
+    m[0] = mn0r;
     float mn1 = 0.f, al1 = 1.f;
     if constexpr (TWO_ROWS) {
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      mn1 = fmaxf(m[1], mx1);
+      const float mn1r = fmaxf(m[1], mx1);
+      mn1 = mn1r == -INFINITY ? 0.f : mn1r;
       al1 = ex2(m[1] - mn1);
-      m[1] = mn1;
+      m[1] = mn1r;
     }
-    // ---- P = 2^(x - m), rounded to the cache dtype as the A operand of P V ----
-    uint32_t pa[4];
-    pa[0] = pack2<BF16>(ex2(sc[0][0] - mn0), ex2(sc[0][1] - mn0));
-    pa[2] = pack2<BF16>(ex2(sc[1][0] - mn0), ex2(sc[1][1] - mn0));
-    {
+    // ---- P = 2^(x - m) as the A operand of P V.  bf16 keeps 8 mantissa
+    // bits, so P goes in as a hi + lo pair of bf16 (about 16 bits, two mma
+    // per tile) and l sums the unrounded fp32 p; fp16 (11 bits) goes in once
+    // and l sums the rounded values, so that O / l stays a convex combination.
+    float p0[4], p1[4];
+    p0[0] = ex2(sc[0][0] - mn0); p0[1] = ex2(sc[0][1] - mn0);
+    p0[2] = ex2(sc[1][0] - mn0); p0[3] = ex2(sc[1][1] - mn0);
+    if constexpr (TWO_ROWS) {
+      p1[0] = ex2(sc[0][2] - mn1); p1[1] = ex2(sc[0][3] - mn1);
+      p1[2] = ex2(sc[1][2] - mn1); p1[3] = ex2(sc[1][3] - mn1);
+    } else {
+      p1[0] = p1[1] = p1[2] = p1[3] = 0.f;
+    }
+    uint32_t pa[4], pl[4];
+    pa[0] = pack2<BF16>(p0[0], p0[1]);
+    pa[2] = pack2<BF16>(p0[2], p0[3]);
+    pa[1] = TWO_ROWS ? pack2<BF16>(p1[0], p1[1]) : 0u;
+    pa[3] = TWO_ROWS ? pack2<BF16>(p1[2], p1[3]) : 0u;
+    if constexpr (BF16) {
+      const float2 h0 = unpack2<BF16>(pa[0]), h2 = unpack2<BF16>(pa[2]);
+      pl[0] = pack2<BF16>(p0[0] - h0.x, p0[1] - h0.y);
+      pl[2] = pack2<BF16>(p0[2] - h2.x, p0[3] - h2.y);
+      if constexpr (TWO_ROWS) {
+        const float2 h1 = unpack2<BF16>(pa[1]), h3 = unpack2<BF16>(pa[3]);
+        pl[1] = pack2<BF16>(p1[0] - h1.x, p1[1] - h1.y);
+        pl[3] = pack2<BF16>(p1[2] - h3.x, p1[3] - h3.y);
+      } else {
+        pl[1] = pl[3] = 0u;
+      }
+      l[0] = l[0] * al0 + ((p0[0] + p0[1]) + (p0[2] + p0[3]));
+      if constexpr (TWO_ROWS) l[1] = l[1] * al1 + ((p1[0] + p1[1]) + (p1[2] + p1[3]));
+    } else {
       const float2 u = unpack2<BF16>(pa[0]), v = unpack2<BF16>(pa[2]);
       l[0] = l[0] * al0 + ((u.x + u.y) + (v.x + v.y));
-    }
-    if constexpr (TWO_ROWS) {
-      pa[1] = pack2<BF16>(ex2(sc[0][2] - mn1), ex2(sc[0][3] - mn1));
-      pa[3] = pack2<BF16>(ex2(sc[1][2] - mn1), ex2(sc[1][3] - mn1));
-      const float2 u = unpack2<BF16>(pa[1]), v = unpack2<BF16>(pa[3]);
-      l[1] = l[1] * al1 + ((u.x + u.y) + (v.x + v.y));
-    } else {
-      pa[1] = pa[3] = 0u;
+      if constexpr (TWO_ROWS) {
+        const float2 w = unpack2<BF16>(pa[1]), z = unpack2<BF16>(pa[3]);
+        l[1] = l[1] * al1 + ((w.x + w.y) + (z.x + z.y));
+      }
     }
     // ---- rescale O, then O += P V ----
 #pragma unroll
@@ -197,6 +233,10 @@ struct MmaWarp {
       ldsm_x4_trans(page_chunk<D>(vbase, vtok, 2 * j + vchk), b0, b1, b2, b3);
       mma_16816<BF16>(acc[2 * j], pa, b0, b1);
       mma_16816<BF16>(acc[2 * j + 1], pa, b2, b3);
+      if constexpr (BF16) {
+        mma_16816<BF16>(acc[2 * j], pl, b0, b1);
+        mma_16816<BF16>(acc[2 * j + 1], pl, b2, b3);
+      }
     }
   }
 
@@ -348,6 +388,87 @@ struct SimtWarp {
     }
   }
 };
+
+// ---------------------------------------------------------------------------
+// End of an item: merge the four warps' rows (already published into the
+// red_* buffers) and, for an item spread over a cluster, the CTAs' rows
+// through distributed shared memory.  emit(row, d, o0, o1, m, l) receives
+// each finished pair of output dims: the unnormalised sums o0, o1, the row
+// max m (log2 domain) and the row sum l.  With `spread`, every CTA of the
+// cluster must call this (it holds two cluster barriers); each emits a slice.
+// ---------------------------------------------------------------------------
+template <int D, int NST, class Emit>
+__device__ __forceinline__ void merge_and_emit(uint8_t* smem, int nrows, bool spread, int ctas,
+                                               int crank, Emit&& emit) {
+  using L = DecodeSmem<D, NST>;
+  const float* red_acc = reinterpret_cast<const float*>(smem);
+  const float* red_m = reinterpret_cast<const float*>(smem + L::kRedMOffset);
+  const float* red_l = reinterpret_cast<const float*>(smem + L::kRedLOffset);
+  float* part_acc = reinterpret_cast<float*>(smem + L::kPartAccOffset);
+  float* part_m = reinterpret_cast<float*>(smem + L::kPartMOffset);
+  float* part_l = reinterpret_cast<float*>(smem + L::kPartLOffset);
+  for (int o = threadIdx.x * 2; o < nrows * D; o += kThreads * 2) {
+    const int g = o / D, d = o % D;
+    float mw[kWarps];
+    float big_m = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      mw[w] = red_m[w * 16 + g];
+      big_m = fmaxf(big_m, mw[w]);
+    }
+    float big_l = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float e = (mw[w] == -INFINITY) ? 0.f : ex2(mw[w] - big_m);
+      big_l += e * red_l[w * 16 + g];
+      if (e != 0.f) {
+        const float2 v = *reinterpret_cast<const float2*>(red_acc + (w * nrows + g) * D + d);
+        o0 += e * v.x;
+        o1 += e * v.y;
+      }
+    }
+    if (spread) {
+      *reinterpret_cast<float2*>(part_acc + g * D + d) = make_float2(o0, o1);
+      if (d == 0) {
+        part_m[g] = big_m;
+        part_l[g] = big_l;
+      }
+    } else {
+      emit(g, d, o0, o1, big_m, big_l);
+    }
+  }
+  if (!spread) return;
+
+  cluster_sync();  // every CTA's part_* rows are complete and visible
+  const int pairs = nrows * D / 2;
+  const int per = (pairs + ctas - 1) / ctas;
+  const int lo = crank * per, hi = min(pairs, lo + per);
+  const uint32_t acc_base = smem_addr(part_acc), m_base = smem_addr(part_m),
+                 l_base = smem_addr(part_l);
+  for (int pr = lo + static_cast<int>(threadIdx.x); pr < hi; pr += kThreads) {
+    const int o = pr * 2, g = o / D, d = o % D;
+    float mc[kMaxCluster];
+    float big_m = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c) {
+      mc[c] = c < ctas ? ld_cluster_f32(map_cluster(m_base + g * 4, c)) : -INFINITY;
+      big_m = fmaxf(big_m, mc[c]);
+    }
+    float big_l = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c) {
+      const float e = (mc[c] == -INFINITY) ? 0.f : ex2(mc[c] - big_m);
+      if (e != 0.f) {
+        big_l += e * ld_cluster_f32(map_cluster(l_base + g * 4, c));
+        const float2 v = ld_cluster_f32x2(map_cluster(acc_base + (g * D + d) * 4, c));
+        o0 += e * v.x;
+        o1 += e * v.y;
+      }
+    }
+    emit(g, d, o0, o1, big_m, big_l);
+  }
+  cluster_sync();  // no CTA leaves while another may still read its shared memory
+}
 
 // ---------------------------------------------------------------------------
 // The kernel: one (sequence, KV head, partition) item per cluster.
@@ -512,7 +633,8 @@ __global__ void __launch_bounds__(kThreads)
       ids_next = my_pages > (win + 1) * 32 ? load_ids(win + 1) : -1;
     }
     const int stg = k % NST;
-    if (!mbar_wait_bounded(bar0 + stg * 8, (k / NST) & 1)) {
+    // the whole warp takes the same branch, whatever each lane's wait saw
+    if (!__all_sync(~0u, mbar_wait_bounded(bar0 + stg * 8, (k / NST) & 1))) {
       if (lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
       ok = false;
       break;
@@ -539,39 +661,11 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
 
-  const int h0 = kvh * group;
-  float* part_acc = reinterpret_cast<float*>(smem + L::kPartAccOffset);
-  float* part_m = reinterpret_cast<float*>(smem + L::kPartMOffset);
-  float* part_l = reinterpret_cast<float*>(smem + L::kPartLOffset);
-  for (int o = threadIdx.x * 2; o < group * D; o += kThreads * 2) {
-    const int g = o / D, d = o % D;
-    float mw[kWarps];
-    float big_m = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      mw[w] = red_m[w * 16 + g];
-      big_m = fmaxf(big_m, mw[w]);
-    }
-    float big_l = 0.f, o0 = 0.f, o1 = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float e = (mw[w] == -INFINITY) ? 0.f : ex2(mw[w] - big_m);
-      big_l += e * red_l[w * 16 + g];
-      if (e != 0.f) {
-        const float2 v = *reinterpret_cast<const float2*>(red_acc + (w * group + g) * D + d);
-        o0 += e * v.x;
-        o1 += e * v.y;
-      }
-    }
-    const size_t hrow = static_cast<size_t>(s) * a.num_heads + h0 + g;
-    if (spread) {
-      // this CTA's merged rows, for the cluster-wide merge below
-      *reinterpret_cast<float2*>(part_acc + g * D + d) = make_float2(o0, o1);
-      if (d == 0) {
-        part_m[g] = big_m;
-        part_l[g] = big_l;
-      }
-    } else if (split) {
+  const size_t hrow0 = static_cast<size_t>(s) * a.num_heads + static_cast<size_t>(kvh) * group;
+  merge_and_emit<D, NST>(smem, group, spread, ctas, crank,
+                         [&](int g, int d, float o0, float o1, float big_m, float big_l) {
+    const size_t hrow = hrow0 + g;
+    if (split) {
       const size_t pidx = hrow * a.max_partitions + part;
       *reinterpret_cast<float2*>(a.tmp_out + pidx * D + d) = make_float2(o0, o1);
       if (d == 0) {
@@ -582,43 +676,7 @@ __global__ void __launch_bounds__(kThreads)
       const float inv = big_l > 0.f ? 1.f / big_l : 0.f;
       *reinterpret_cast<uint32_t*>(a.out + hrow * D + d) = pack2<BF16>(o0 * inv, o1 * inv);
     }
-  }
-  if (!spread) return;
-
-  // ---- cluster-wide merge through distributed shared memory ----
-  cluster_sync();  // every CTA's part_* rows are complete and visible
-  {
-    const int pairs = group * D / 2;
-    const int per = (pairs + ctas - 1) / ctas;
-    const int lo = crank * per, hi = min(pairs, lo + per);
-    const uint32_t acc_base = smem_addr(part_acc), m_base = smem_addr(part_m),
-                   l_base = smem_addr(part_l);
-    for (int pr = lo + threadIdx.x; pr < hi; pr += kThreads) {
-      const int o = pr * 2, g = o / D, d = o % D;
-      float mc[kMaxCluster];
-      float big_m = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kMaxCluster; ++c) {
-        mc[c] = c < ctas ? ld_cluster_f32(map_cluster(m_base + g * 4, c)) : -INFINITY;
-        big_m = fmaxf(big_m, mc[c]);
-      }
-      float big_l = 0.f, o0 = 0.f, o1 = 0.f;
-#pragma unroll
-      for (int c = 0; c < kMaxCluster; ++c) {
-        const float e = (mc[c] == -INFINITY) ? 0.f : ex2(mc[c] - big_m);
-        if (e != 0.f) {
-          big_l += e * ld_cluster_f32(map_cluster(l_base + g * 4, c));
-          const float2 v = ld_cluster_f32x2(map_cluster(acc_base + (g * D + d) * 4, c));
-          o0 += e * v.x;
-          o1 += e * v.y;
-        }
-      }
-      const size_t hrow = static_cast<size_t>(s) * a.num_heads + h0 + g;
-      const float inv = big_l > 0.f ? 1.f / big_l : 0.f;
-      *reinterpret_cast<uint32_t*>(a.out + hrow * D + d) = pack2<BF16>(o0 * inv, o1 * inv);
-    }
-  }
-  cluster_sync();  // no CTA leaves while another may still read its shared memory
+  });
 }
 
 }  // namespace pa

@@ -124,7 +124,7 @@ def build_block_tables(cfg: DecodeConfig, context_lens: torch.Tensor,
     sequences in order; sharing groups reuse the first shared_prefix_blocks
     ids of their group.  Unused entries are -1."""
     blocks_needed = [(int(c) + cfg.block_size - 1) // cfg.block_size for c in context_lens]
-    max_blocks = max(1, max(blocks_needed))
+    max_blocks = max(1, max(blocks_needed), cfg.shared_prefix_blocks)
     tables = torch.full((cfg.num_seqs, max_blocks), -1, dtype=torch.int32)
     perm = torch.randperm(cfg.num_blocks, generator=gen).to(torch.int32)
     cursor = 0
@@ -132,12 +132,13 @@ def build_block_tables(cfg: DecodeConfig, context_lens: torch.Tensor,
     for s, nb in enumerate(blocks_needed):
         row: list[int] = []
         if cfg.shared_prefix_blocks > 0:
+            # every member's table starts with the group's shared ids (entries
+            # past its own context are never read for that member)
             if s % cfg.share_group == 0:
                 shared = perm[cursor:cursor + cfg.shared_prefix_blocks].tolist()
                 cursor += cfg.shared_prefix_blocks
-            take = min(nb, cfg.shared_prefix_blocks)
-            row.extend(shared[:take])
-            nb -= take
+            row.extend(shared)
+            nb = max(0, nb - cfg.shared_prefix_blocks)
         row.extend(perm[cursor:cursor + nb].tolist())
         cursor += nb
         if cursor > cfg.num_blocks:
@@ -181,6 +182,8 @@ class DecodeBatch:
     query: torch.Tensor
     key: torch.Tensor
     value: torch.Tensor
+    group_starts: torch.Tensor | None = None    # shared-prefix groups (int32 [G+1])
+    prefix_blocks: torch.Tensor | None = None   # shared table entries per group (int32 [G])
     meta: dict = field(default_factory=dict)
 
     @property
@@ -214,8 +217,15 @@ def make_batch(cfg: DecodeConfig, device: str | torch.device = "cpu") -> DecodeB
                                    dtype=dt, device=device), vgen)
     value = _fill_normal(torch.empty((cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim),
                                      dtype=dt, device=device), vgen)
+    group_starts = prefix_blocks = None
+    if cfg.shared_prefix_blocks > 0:
+        starts = list(range(0, cfg.num_seqs, cfg.share_group)) + [cfg.num_seqs]
+        group_starts = torch.tensor(starts, dtype=torch.int32, device=device)
+        prefix_blocks = torch.full((len(starts) - 1,), cfg.shared_prefix_blocks,
+                                   dtype=torch.int32, device=device)
     return DecodeBatch(cfg, context_lens.to(device), block_tables.to(device),
-                       slot_mapping.to(device), key_cache, value_cache, query, key, value)
+                       slot_mapping.to(device), key_cache, value_cache, query, key, value,
+                       group_starts, prefix_blocks)
 
 
 def algorithmic_bytes(cfg: DecodeConfig, context_lens) -> dict:

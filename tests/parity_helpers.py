@@ -51,18 +51,24 @@ def oracle_step(orc, host: HostCopy, write: bool = True):
 
 
 def gpu_step(batch: workloads.DecodeBatch, write: bool = True, partition_size: int = 0,
-             max_partitions: int | None = None):
-    """The CUDA path: pa_reshape_and_cache, then pa_decode or
-    pa_decode_split + pa_reduce.  Returns (out, partials or None)."""
-    from paged_kv_cache_444_b200 import (SplitWorkspace, pa_decode, pa_decode_split, pa_reduce,
-                                         pa_reshape_and_cache)
+             max_partitions: int | None = None, shared_prefix: bool = False,
+             max_group_size: int | None = None):
+    """The CUDA path: pa_reshape_and_cache, then pa_decode, pa_decode_split +
+    pa_reduce, or pa_decode_shared_prefix.  Returns (out, partials or None)."""
+    from paged_kv_cache_444_b200 import (SplitWorkspace, pa_decode, pa_decode_shared_prefix,
+                                         pa_decode_split, pa_reduce, pa_reshape_and_cache)
     cfg = batch.cfg
     if write:
         pa_reshape_and_cache(batch.key, batch.value, batch.key_cache, batch.value_cache,
                              batch.slot_mapping)
     out = torch.full_like(batch.query, float("nan"))
     parts = None
-    if partition_size:
+    if shared_prefix:
+        sizes = (batch.group_starts[1:] - batch.group_starts[:-1]).tolist()
+        pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
+                                batch.block_tables, batch.context_lens, batch.group_starts,
+                                batch.prefix_blocks, cfg.scale, max_group_size or max(sizes))
+    elif partition_size:
         P = max_partitions or (batch.block_tables.shape[1] * cfg.block_size + partition_size - 1) \
             // partition_size
         ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, batch.query.device)

@@ -11,6 +11,12 @@ from paged_kv_cache_444_b200 import build as pa_build
 OK, NULL, SHAPE, DTYPE, ALIGN, UNSUP, CUDA, BOUNDS = range(8)
 FAKE = 0x10000          # 16-byte aligned stand-in pointer; never dereferenced on these paths
 
+# Calls with stand-in pointers must be rejected before any launch.  They run
+# only where no GPU is visible, so that a validation gap can never turn into
+# a launch on stand-in pointers.
+host_only = pytest.mark.skipif(torch.cuda.is_available(),
+                               reason="stand-in pointers: host-only validation test")
+
 
 @pytest.fixture(scope="module")
 def lib():
@@ -46,6 +52,7 @@ def _decode(lib, **kw):
                          args["NB"], args["bs"], args["MB"], args["dt"], None)
 
 
+@host_only
 def test_decode_validation(lib):
     assert _decode(lib, dt=5) == DTYPE
     assert _decode(lib, query=None) == NULL
@@ -66,6 +73,7 @@ def test_decode_validation(lib):
     assert _decode(lib, S=0, out=None, query=None) == OK  # empty batch: nothing to do
 
 
+@host_only
 def test_split_and_reduce_validation(lib):
     f = lib.pa_decode_split
     base = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, 4, 8, 2, 128, 64, 16, 8]
@@ -78,10 +86,11 @@ def test_split_and_reduce_validation(lib):
     assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 128, 0, 1, 0, None) == SHAPE
     assert r(None, FAKE, FAKE, FAKE, FAKE, 4, 8, 128, 512, 1, 0, None) == NULL
     assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 130, 512, 1, 0, None) == UNSUP
-    assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 516, 512, 1, 0, None) == UNSUP
+    assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 1028, 512, 1, 0, None) == UNSUP
     assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 128, 512, 1, 0, None) == OK
 
 
+@host_only
 def test_reshape_validation(lib):
     f = lib.pa_reshape_and_cache
     good = [FAKE, FAKE, 256, 256, FAKE, FAKE, FAKE, 4, 2, 128, 64, 16, 0, None]
@@ -113,3 +122,20 @@ def test_valid_call_without_gpu_reports_cuda_error(lib):
 def test_binding_raises_without_library(tmp_path):
     with pytest.raises(_lib.PagedAttentionError):
         _lib.load(tmp_path / "missing.so")
+
+
+@host_only
+def test_shared_prefix_validation(lib):
+    f = lib.pa_decode_shared_prefix
+    base = [FAKE] * 8 + [0.1, 8]            # out .. prefix_blocks, scale, num_seqs
+    sizes = [2, 4, 8, 2, 128, 64, 16, 8, 0, None]  # groups, max size, H, Hk, D, NB, bs, MB, dt
+    assert f(*base, *sizes[:1], 0, *sizes[2:]) == SHAPE          # max_group_size 0
+    assert f(*base, -1, *sizes[1:]) == SHAPE                      # negative group count
+    assert f(*base, 0, *sizes[1:]) == OK                          # no groups: nothing to do
+    b = list(base)
+    b[6] = None
+    assert f(*b, *sizes) == NULL                                  # group_starts
+    b = list(base)
+    b[7] = FAKE + 2
+    assert f(*b, *sizes) == ALIGN                                 # prefix_blocks
+    assert f(*base, 2, 4, 64, 2, 128, 64, 16, 8, 0, None) == UNSUP  # 32 query heads per KV head

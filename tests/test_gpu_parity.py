@@ -231,6 +231,79 @@ def test_many_sequences_natural_order(dev, oracle_lib):
     _check_close(out, ref, cfg, "natural order")
 
 
+def _regroup(batch, starts, prefix):
+    """Make sequences [starts[g], starts[g+1]) share their first prefix[g]
+    table entries -- the ids of the group's longest member (clamped to its
+    block count) -- and attach the group arrays."""
+    bt = batch.block_tables.clone()
+    ctx = batch.context_lens.tolist()
+    prefix = list(prefix)
+    for g in range(len(starts) - 1):
+        members = list(range(starts[g], starts[g + 1]))
+        donor = max(members, key=lambda s: ctx[s])
+        prefix[g] = min(prefix[g], (ctx[donor] + 15) // 16)
+        for s in members:
+            bt[s, :prefix[g]] = bt[donor, :prefix[g]]
+    batch.block_tables = bt
+    dev = bt.device
+    batch.group_starts = torch.tensor(starts, dtype=torch.int32, device=dev)
+    batch.prefix_blocks = torch.tensor(prefix, dtype=torch.int32, device=dev)
+    return batch
+
+
+SHARED_CASES = {
+    # name: (base config, overrides, group starts, prefix blocks per group)
+    "beam4_gqa4": ("shared_small", {}, None, None),
+    "mha_16_members": ("mha_small", dict(num_seqs=20, num_heads=2, num_kv_heads=2, num_blocks=600,
+                                         ctx=("uniform", 40, 300), seed=41),
+                       [0, 16, 20], [2, 1]),
+    "gqa8_chunked": ("gqa8", dict(num_seqs=7, num_blocks=300, ctx=("uniform", 1, 400), seed=42),
+                     [0, 5, 7], [3, 0]),
+    "gqa2_ragged_bf16": ("d64_gqa2", dict(num_seqs=9, num_blocks=400, ctx=("uniform", 1, 600),
+                                          seed=43), [0, 1, 4, 9], [1, 5, 2]),
+    "short_members": ("gqa_small", dict(num_seqs=4, num_blocks=200,
+                                        ctx=("fixed", (20, 300, 5, 0)), seed=44),
+                      [0, 4], [8]),
+    "long_prefix_spread": ("gqa_small", dict(num_seqs=4, num_blocks=900,
+                                             ctx=("fixed", (3000, 2900, 3100, 4000)), seed=45),
+                           [0, 4], [150]),
+}
+
+
+@pytest.mark.parametrize("name", list(SHARED_CASES))
+def test_shared_prefix_matches_oracle(name, dev, oracle_lib):
+    base, over, starts, prefix = SHARED_CASES[name]
+    cfg = SMALL[base].scaled(**over) if over else SMALL[base]
+    batch = workloads.make_batch(cfg, dev)
+    if starts is not None:
+        batch = _regroup(batch, starts, prefix)
+    host = HostCopy(batch)
+    ref, kc_ref, vc_ref = oracle_step(oracle_lib, host)
+    out, _ = gpu_step(batch, shared_prefix=True)
+    pa_check_error()
+    assert np.array_equal(bits(batch.key_cache), kc_ref)
+    _check_close(out, ref, cfg, f"shared prefix {name}")
+    plain, _ = gpu_step(batch, write=False)
+    assert np.max(np.abs(to_f64(plain) - to_f64(out))) <= TOL[cfg.dtype]
+
+
+def test_shared_prefix_reports_bad_groups(dev):
+    cfg = SMALL["shared_small"]
+    batch = workloads.make_batch(cfg, dev)
+    batch.group_starts[1] = batch.group_starts[2] + 1       # not monotone
+    gpu_step(batch, write=False, shared_prefix=True, max_group_size=cfg.share_group)
+    with pytest.raises(PagedAttentionError) as e:
+        pa_check_error()
+    assert e.value.detail >> 56 == 6
+    batch = _regroup(workloads.make_batch(cfg, dev), [0, 8], [4])
+    # one group of 8 members, but room for 4 (one chunk of 16 rows / 4 heads)
+    gpu_step(batch, write=False, shared_prefix=True, max_group_size=4)
+    with pytest.raises(PagedAttentionError) as e:
+        pa_check_error()
+    assert e.value.detail >> 56 == 6
+    pa_check_error()
+
+
 def test_write_padding_and_strided_rows(dev, oracle_lib):
     cfg = SMALL["gqa_small"]
     batch = workloads.make_batch(cfg, dev)
@@ -281,6 +354,7 @@ def test_bounds_checks_report_and_skip(dev):
     # a context length beyond the table: clamped, reported
     b = workloads.make_batch(cfg, dev)
     b.context_lens[4] = b.block_tables.shape[1] * cfg.block_size + 100
+    b.block_tables[4, :] = b.block_tables[4, 0]   # every entry valid: only the length is wrong
     out, _ = gpu_step(b, write=False)
     with pytest.raises(PagedAttentionError) as e:
         pa_check_error()
