@@ -87,6 +87,18 @@ class Oracle:
         lib.oracle_decode_partitioned.restype = ctypes.c_int
         lib.oracle_lse_merge.argtypes = [_p] * 5 + [_i64] * 5
         lib.oracle_lse_merge.restype = ctypes.c_int
+        lib.oracle_copy_blocks.argtypes = [_p] * 3 + [_i64] * 6
+        lib.oracle_copy_blocks.restype = ctypes.c_int
+        lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_f64.restype = ctypes.c_double
+        lib.oracle_f64_to_e4m3.argtypes = [ctypes.c_double]
+        lib.oracle_f64_to_e4m3.restype = ctypes.c_uint8
+        lib.oracle_reshape_and_cache_fp8.argtypes = ([_p] * 5 + [_i64] * 7 +
+                                                     [ctypes.c_float, ctypes.c_float, ctypes.c_int])
+        lib.oracle_reshape_and_cache_fp8.restype = ctypes.c_int
+        lib.oracle_decode_fp8.argtypes = ([_p] * 6 + [_i64] * 7 +
+                                          [ctypes.c_double] * 3 + [ctypes.c_int])
+        lib.oracle_decode_fp8.restype = ctypes.c_int
 
     # ---- scalar helpers -------------------------------------------------
     def f16_to_f64(self, bits: int) -> float:
@@ -146,6 +158,57 @@ class Oracle:
             key.ctypes.data, value.ctypes.data, key_cache.ctypes.data,
             value_cache.ctypes.data, slots.ctypes.data, T, Hk, D, num_blocks,
             block_size, key_stride, value_stride))
+
+    def e4m3_to_f64(self, bits: int) -> float:
+        return self._lib.oracle_e4m3_to_f64(int(bits))
+
+    def f64_to_e4m3(self, x: float) -> int:
+        return int(self._lib.oracle_f64_to_e4m3(float(x)))
+
+    def reshape_and_cache_fp8(self, key, value, key_cache, value_cache, slot_mapping,
+                              num_blocks: int, block_size: int, k_scale: float, v_scale: float,
+                              dtype: int) -> int:
+        """Quantising write of 16-bit key/value [T, Hk, D] into uint8 E4M3
+        caches [NB, bs, Hk, D] (in place)."""
+        assert key_cache.dtype == np.uint8 and key_cache.flags.c_contiguous
+        assert value_cache.dtype == np.uint8 and value_cache.flags.c_contiguous
+        T, Hk, D = key.shape
+        key_stride = key.strides[0] // 2 if T > 0 else Hk * D
+        value_stride = value.strides[0] // 2 if T > 0 else Hk * D
+        slots = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+        return int(self._lib.oracle_reshape_and_cache_fp8(
+            key.ctypes.data, value.ctypes.data, key_cache.ctypes.data, value_cache.ctypes.data,
+            slots.ctypes.data, T, Hk, D, num_blocks, block_size, key_stride, value_stride,
+            float(k_scale), float(v_scale), dtype))
+
+    def decode_fp8(self, query, key_cache, value_cache, block_tables, context_lens,
+                   scale: float, k_scale: float, v_scale: float, dtype: int) -> np.ndarray:
+        """softmax(scale q K^T) V with K = code * k_scale, V = code * v_scale."""
+        q = np.ascontiguousarray(query, dtype=np.uint16)
+        kc = np.ascontiguousarray(key_cache, dtype=np.uint8)
+        vc = np.ascontiguousarray(value_cache, dtype=np.uint8)
+        bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+        cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+        S, H, D = q.shape
+        NB, bs, Hk, _ = kc.shape
+        out = np.zeros((S, H, D), dtype=np.float64)
+        rc = self._lib.oracle_decode_fp8(out.ctypes.data, q.ctypes.data, kc.ctypes.data,
+                                         vc.ctypes.data, bt.ctypes.data, cl.ctypes.data,
+                                         S, H, Hk, D, NB, bs, bt.shape[1], float(scale),
+                                         float(k_scale), float(v_scale), dtype)
+        if rc != OK:
+            raise ValueError(f"oracle_decode_fp8 failed with code {rc}")
+        return out
+
+    def copy_blocks(self, key_cache, value_cache, block_mapping) -> int:
+        """In-place copy of whole blocks src -> dst (pairs [n, 2] int64) in
+        both caches [NB, bs, Hk, D] (any fixed-size element, contiguous)."""
+        assert key_cache.flags.c_contiguous and value_cache.flags.c_contiguous
+        NB, bs, Hk, D = key_cache.shape
+        pairs = np.ascontiguousarray(block_mapping, dtype=np.int64).reshape(-1, 2)
+        return int(self._lib.oracle_copy_blocks(key_cache.ctypes.data, value_cache.ctypes.data,
+                                                pairs.ctypes.data, pairs.shape[0], NB, bs, Hk,
+                                                D, key_cache.itemsize))
 
     def decode(self, query, key_cache, value_cache, block_tables, context_lens,
                scale: float, dtype: int) -> np.ndarray:

@@ -135,6 +135,43 @@ uint16_t oracle_f64_to_bf16(double x)
     return sign | (uint16_t)(biased << 7) | frac;
 }
 
+/* OCP FP8 E4M3 ("fn" variant): 1 sign bit, 4 exponent bits (bias 7), 3
+ * fraction bits, no infinities; S.1111.111 is NaN; max finite 448. */
+double oracle_e4m3_to_f64(uint8_t bits)
+{
+    int sign = (bits >> 7) & 1;
+    int expo = (bits >> 3) & 0xf;
+    int frac = bits & 0x7;
+    double mag;
+    if (expo == 0xf && frac == 0x7) {
+        mag = NAN;
+    } else if (expo == 0) {
+        mag = ldexp((double)frac, -9);                 /* subnormal: frac/8 * 2^-6 */
+    } else {
+        mag = ldexp((double)(8 + frac), expo - 10);    /* (1 + frac/8) * 2^(e-7) */
+    }
+    return sign ? -mag : mag;
+}
+
+/* double -> E4M3, round to nearest even, saturating finite values to +-448. */
+uint8_t oracle_f64_to_e4m3(double x)
+{
+    uint8_t sign = signbit(x) ? 0x80 : 0;
+    if (isnan(x)) return 0x7f;
+    double r = round_to_format(x, 3, -6);
+    double a = fabs(r);
+    if (a > 448.0 || isinf(a)) a = 448.0;              /* saturate */
+    if (a == 0.0) return sign;
+    if (a < ldexp(1.0, -6)) {                          /* subnormal */
+        return sign | (uint8_t)(a / ldexp(1.0, -9));
+    }
+    int e;
+    double f = frexp(a, &e);
+    int biased = e - 1 + 7;
+    uint8_t frac = (uint8_t)((f * 2.0 - 1.0) * 8.0);
+    return sign | (uint8_t)(biased << 3) | frac;
+}
+
 static double decode16(uint16_t bits, int dtype)
 {
     return dtype == ORACLE_BF16 ? oracle_bf16_to_f64(bits) : oracle_f16_to_f64(bits);
@@ -209,6 +246,37 @@ int oracle_reshape_and_cache(const uint16_t *key, const uint16_t *value,
         if (slot >= num_blocks * block_size) { rc = ORACLE_BAD_SLOT; continue; }
         memcpy(key_cache + slot * row, key + t * key_stride, (size_t)row * 2);
         memcpy(value_cache + slot * row, value + t * value_stride, (size_t)row * 2);
+    }
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Block copy for copy-on-write: [P1] §第一讲, [P2] §3.3                      */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Copy-on-write: before a sequence writes into a block it shares (ref_count
+ * > 1), the block is copied to a private one.  For each pair i, copy the whole
+ * block block_mapping[2i] (source) of both caches onto block block_mapping[2i+1]
+ * (destination), byte for byte: block_size * num_kv_heads * head_dim
+ * elements of elem_bytes each.  Pairs are applied in order.  Returns
+ * ORACLE_BAD_BLOCK (after skipping the pair) if an id is out of range.
+ */
+int oracle_copy_blocks(uint8_t *key_cache, uint8_t *value_cache,
+                       const int64_t *block_mapping, int64_t num_pairs,
+                       int64_t num_blocks, int64_t block_size, int64_t num_kv_heads,
+                       int64_t head_dim, int64_t elem_bytes)
+{
+    int rc = ORACLE_OK;
+    size_t block_bytes = (size_t)(block_size * num_kv_heads * head_dim * elem_bytes);
+    for (int64_t i = 0; i < num_pairs; ++i) {
+        int64_t src = block_mapping[2 * i], dst = block_mapping[2 * i + 1];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+            rc = ORACLE_BAD_BLOCK;
+            continue;
+        }
+        memmove(key_cache + dst * block_bytes, key_cache + src * block_bytes, block_bytes);
+        memmove(value_cache + dst * block_bytes, value_cache + src * block_bytes, block_bytes);
     }
     return rc;
 }
@@ -415,6 +483,102 @@ int oracle_lse_merge(double *out, const double *part_acc, const double *part_max
             }
             for (int64_t d = 0; d < head_dim; ++d) o[d] /= big_l;
         }
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP8 KV cache ("vLLM PagedAttention 原理与源码深度解析" §8.4: --kv-cache-dtype fp8) */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Quantising cache write: like oracle_reshape_and_cache, but each element x
+ * of key (value) is stored as E4M3 of the float product x * inv_k (x * inv_v),
+ * where inv = 1.0f / scale is computed in float and the product is a float
+ * multiplication -- the same two roundings a GPU takes -- then rounded to
+ * E4M3 nearest-even with saturation.  The stored code dequantises as
+ * code * scale.
+ */
+int oracle_reshape_and_cache_fp8(const uint16_t *key, const uint16_t *value,
+                                 uint8_t *key_cache, uint8_t *value_cache,
+                                 const int64_t *slot_mapping, int64_t num_tokens,
+                                 int64_t num_kv_heads, int64_t head_dim,
+                                 int64_t num_blocks, int64_t block_size,
+                                 int64_t key_stride, int64_t value_stride,
+                                 float k_scale, float v_scale, int dtype)
+{
+    int rc = ORACLE_OK;
+    int64_t row = num_kv_heads * head_dim;
+    float inv_k = 1.0f / k_scale, inv_v = 1.0f / v_scale;
+    for (int64_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= num_blocks * block_size) { rc = ORACLE_BAD_SLOT; continue; }
+        for (int64_t e = 0; e < row; ++e) {
+            float kx = (float)decode16(key[t * key_stride + e], dtype);
+            float vx = (float)decode16(value[t * value_stride + e], dtype);
+            key_cache[slot * row + e] = oracle_f64_to_e4m3((double)(kx * inv_k));
+            value_cache[slot * row + e] = oracle_f64_to_e4m3((double)(vx * inv_v));
+        }
+    }
+    return rc;
+}
+
+/*
+ * Decode over an E4M3 cache: exactly oracle_decode with every cached K (V)
+ * element replaced by its dequantised value code * k_scale (code * v_scale),
+ * in double.  query is 16-bit (dtype).
+ */
+int oracle_decode_fp8(double *out, const uint16_t *query,
+                      const uint8_t *key_cache, const uint8_t *value_cache,
+                      const int32_t *block_tables, const int32_t *context_lens,
+                      int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads,
+                      int64_t head_dim, int64_t num_blocks, int64_t block_size,
+                      int64_t max_blocks_per_seq, double scale, double k_scale,
+                      double v_scale, int dtype)
+{
+    if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || block_size <= 0)
+        return ORACLE_BAD_ARG;
+    int64_t group = num_heads / num_kv_heads;
+    for (int64_t s = 0; s < num_seqs; ++s) {
+        int64_t ctx = context_lens[s];
+        double *o = out + s * num_heads * head_dim;
+        if (ctx <= 0) {
+            for (int64_t e = 0; e < num_heads * head_dim; ++e) o[e] = 0.0;
+            continue;
+        }
+        if (ctx > max_blocks_per_seq * block_size) return ORACLE_BAD_ARG;
+        double *kc = malloc(sizeof(double) * (size_t)(ctx * head_dim));
+        double *vc = malloc(sizeof(double) * (size_t)(ctx * head_dim));
+        double *z = malloc(sizeof(double) * (size_t)ctx);
+        double *q = malloc(sizeof(double) * (size_t)head_dim);
+        if (!kc || !vc || !z || !q) { free(kc); free(vc); free(z); free(q); return ORACLE_NO_MEMORY; }
+        const int32_t *bt = block_tables + s * max_blocks_per_seq;
+        for (int64_t h = 0; h < num_heads; ++h) {
+            int64_t kvh = h / group;
+            if (h % group == 0) {
+                for (int64_t j = 0; j < ctx; ++j) {
+                    int64_t block = bt[j / block_size];
+                    int64_t r = j % block_size;
+                    if (block < 0 || block >= num_blocks) {
+                        free(kc); free(vc); free(z); free(q);
+                        return ORACLE_BAD_BLOCK;
+                    }
+                    int64_t base = ((block * block_size + r) * num_kv_heads + kvh) * head_dim;
+                    for (int64_t d = 0; d < head_dim; ++d) {
+                        kc[j * head_dim + d] = oracle_e4m3_to_f64(key_cache[base + d]) * k_scale;
+                        vc[j * head_dim + d] = oracle_e4m3_to_f64(value_cache[base + d]) * v_scale;
+                    }
+                }
+            }
+            const uint16_t *qs = query + (s * num_heads + h) * head_dim;
+            for (int64_t d = 0; d < head_dim; ++d) q[d] = decode16(qs[d], dtype);
+            double m, l;
+            double *acc = o + h * head_dim;
+            attend_range(q, kc, vc, head_dim, 0, ctx, scale, z, &m, &l, acc);
+            for (int64_t d = 0; d < head_dim; ++d) acc[d] /= l;
+        }
+        free(kc); free(vc); free(z); free(q);
     }
     return ORACLE_OK;
 }

@@ -353,6 +353,141 @@ def pin_partition_merge(orc):
     assert np.max(np.abs(acc[:, :, 0] / psum[:, :, 0, None] - single)) <= 1e-14
 
 
+def pin_copy_on_write_blocks(orc):
+    """Copy-on-write ("vllm源码分析" 第一讲; "vLLM PagedAttention 原理与源码深度解析"
+    §3.3): after copying a shared block to a private one, the private block
+    holds the same bytes, the source is untouched, and every other block keeps
+    its canary; attention of a sequence re-pointed at the copy is unchanged."""
+    rng = np.random.default_rng(23)
+    NB, bs, Hk, D = 10, 4, 2, 8
+    kc = rng.integers(0, 65535, (NB, bs, Hk, D), dtype=np.uint16)
+    vc = rng.integers(0, 65535, (NB, bs, Hk, D), dtype=np.uint16)
+    kc = np.where(np.isnan(kc.view(np.float16)), 0x3c00, kc).astype(np.uint16)
+    vc = np.where(np.isnan(vc.view(np.float16)), 0x3c00, vc).astype(np.uint16)
+    kc = np.where(np.isinf(kc.view(np.float16)), 0x3c00, kc).astype(np.uint16)
+    vc = np.where(np.isinf(vc.view(np.float16)), 0x3c00, vc).astype(np.uint16)
+    k0, v0 = kc.copy(), vc.copy()
+    pairs = np.array([[3, 7], [0, 9]], dtype=np.int64)
+    assert orc.copy_blocks(kc, vc, pairs) == oracle_mod.OK
+    for b in range(NB):
+        src = {7: 3, 9: 0}.get(b, b)
+        assert np.array_equal(kc[b], k0[src]) and np.array_equal(vc[b], v0[src])
+    # a sequence reading block 3 reads the same values from its private copy 7
+    q = rng.integers(0x3000, 0x3c00, (1, Hk, D), dtype=np.uint16)
+    bt_shared = np.array([[1, 3]], dtype=np.int32)
+    bt_private = np.array([[1, 7]], dtype=np.int32)
+    cl = np.array([6], dtype=np.int32)
+    a = orc.decode(q, kc, vc, bt_shared, cl, 0.3, F16)
+    b = orc.decode(q, kc, vc, bt_private, cl, 0.3, F16)
+    assert np.array_equal(a, b)
+    bad = np.array([[2, NB]], dtype=np.int64)
+    assert orc.copy_blocks(kc, vc, bad) == oracle_mod.BAD_BLOCK
+
+
+def _e4m3_torch(codes: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.asarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn) \
+        .to(torch.float64).numpy()
+
+
+def pin_e4m3_decode_all_codes(orc):
+    """E4M3 decode equals torch's float8_e4m3fn -> float64 cast on all 256 codes."""
+    codes = np.arange(256, dtype=np.uint8)
+    got = np.array([orc.e4m3_to_f64(c) for c in codes])
+    want = _e4m3_torch(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert np.array_equal(got[ok], want[ok])
+
+
+def pin_e4m3_rounding(orc):
+    """double -> E4M3 nearest-even equals torch's float32 -> float8_e4m3fn cast
+    inside +-464 (ties included); beyond, finite values saturate to +-448."""
+    rng = np.random.default_rng(29)
+    xs = (rng.standard_normal(3000) * np.exp2(rng.integers(-12, 9, 3000))).astype(np.float32)
+    xs = xs[np.abs(xs) < 464]
+    grid = _e4m3_torch(np.arange(0, 127, dtype=np.uint8))
+    ties = (grid[:-1] + grid[1:]) / 2                      # midpoints between neighbours
+    xs = np.concatenate([xs.astype(np.float64), ties, -ties])
+    want = torch.from_numpy(xs.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([orc.f64_to_e4m3(float(x)) for x in xs], dtype=np.uint8)
+    assert np.array_equal(got, want)
+    for x, code in [(464.0, 0x7e), (1e30, 0x7e), (float("inf"), 0x7e), (-500.0, 0xfe),
+                    (float("nan"), 0x7f)]:
+        assert orc.f64_to_e4m3(x) == code, x
+
+
+def pin_fp8_write_worked_example(orc):
+    """The quantising write puts token n of the worked example (block_size 4)
+    at block (n-1) div 4, offset (n-1) mod 4, as E4M3 of x * (1/scale) taken
+    in float (torch's float32 product and float8 cast), saturated; nothing
+    else changes."""
+    rows = read_golden("slot_mapping_example.txt")
+    bs = int(rows[0][1])
+    NB, Hk, D = 3, 2, 8
+    rng = np.random.default_rng(31)
+    key_f = (rng.standard_normal((9, Hk, D)) * 3).astype(np.float16)
+    val_f = (rng.standard_normal((9, Hk, D)) * 3).astype(np.float16)
+    key_f[0, 0, 0] = 1000.0                                 # saturates at 448 * scale
+    key, value = key_f.view(np.uint16), val_f.view(np.uint16)
+    kc = np.full((NB, bs, Hk, D), 0xaa, dtype=np.uint8)
+    vc = np.full((NB, bs, Hk, D), 0x55, dtype=np.uint8)
+    table = np.array([0, 1, 2], dtype=np.int32)
+    slots = np.array([orc.slot(table, i, bs) for i in range(9)], dtype=np.int64)
+    ks, vs = 0.75, 1.5
+    assert orc.reshape_and_cache_fp8(key, value, kc, vc, slots, NB, bs, ks, vs, F16) == 0
+    inv_k, inv_v = np.float32(1) / np.float32(ks), np.float32(1) / np.float32(vs)
+
+    def q8(x16, inv):
+        prod = torch.from_numpy(x16.astype(np.float32)) * torch.tensor(inv)
+        prod = prod.clamp(-448, 448)                       # the write saturates
+        return prod.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+    ek = np.full_like(kc, 0xaa)
+    ev = np.full_like(vc, 0x55)
+    for token, index, block, offset in [tuple(map(int, r)) for r in rows[1:]]:
+        ek[block, offset] = q8(key_f[index], inv_k)
+        ev[block, offset] = q8(val_f[index], inv_v)
+    assert np.array_equal(kc, ek) and np.array_equal(vc, ev)
+    assert orc.e4m3_to_f64(kc[0, 0, 0, 0]) == 448.0
+
+
+def pin_fp8_decode_sdpa(orc):
+    """Decode over an E4M3 cache == torch SDPA (float64) over the dequantised
+    K = code * k_scale, V = code * v_scale, gathered contiguously."""
+    rng = np.random.default_rng(37)
+    for S, H, Hk, D, bs, ctx, dt in [(3, 8, 2, 32, 4, [5, 13, 1], F16),
+                                     (2, 4, 4, 16, 16, [40, 17], BF16)]:
+        NB = sum((c + bs - 1) // bs for c in ctx) + 3
+        kc = rng.integers(0, 255, (NB, bs, Hk, D), dtype=np.uint8)
+        vc = rng.integers(0, 255, (NB, bs, Hk, D), dtype=np.uint8)
+        kc[(kc & 0x7f) == 0x7f] = 0x30                      # no NaN codes
+        vc[(vc & 0x7f) == 0x7f] = 0x31
+        tdt = torch.bfloat16 if dt == BF16 else torch.float16
+        q = _bits(torch.randn((S, H, D), generator=torch.Generator().manual_seed(S)).to(tdt))
+        perm = rng.permutation(NB).astype(np.int32)
+        MB = max((c + bs - 1) // bs for c in ctx)
+        bt = np.full((S, MB), -1, dtype=np.int32)
+        cur = 0
+        for s_, c in enumerate(ctx):
+            nb = (c + bs - 1) // bs
+            bt[s_, :nb] = perm[cur:cur + nb]
+            cur += nb
+        cl = np.asarray(ctx, dtype=np.int32)
+        ks, vs = 0.02, 0.05
+        got = orc.decode_fp8(q, kc, vc, bt, cl, 0.2, ks, vs, dt)
+        kd = torch.from_numpy(_e4m3_torch(kc) * ks)
+        vd = torch.from_numpy(_e4m3_torch(vc) * vs)
+        qd = torch.from_numpy(q.view(np.int16)).view(tdt).to(torch.float64)
+        for s_ in range(S):
+            nb = (ctx[s_] + bs - 1) // bs
+            idx = torch.from_numpy(bt[s_, :nb].astype(np.int64))
+            k = kd[idx].reshape(nb * bs, Hk, D)[:ctx[s_]].permute(1, 0, 2)[None]
+            v = vd[idx].reshape(nb * bs, Hk, D)[:ctx[s_]].permute(1, 0, 2)[None]
+            o = F.scaled_dot_product_attention(qd[s_][None, :, None, :], k, v, scale=0.2,
+                                               enable_gqa=True)[0, :, 0, :]
+            assert np.max(np.abs(got[s_] - o.numpy())) <= 1e-12
+
+
 ALL_PINS = [
     pin_f16_decode_all_patterns,
     pin_bf16_decode_all_patterns,
@@ -369,4 +504,9 @@ ALL_PINS = [
     pin_closed_forms,
     pin_context_mask,
     pin_partition_merge,
+    pin_copy_on_write_blocks,
+    pin_e4m3_decode_all_codes,
+    pin_e4m3_rounding,
+    pin_fp8_write_worked_example,
+    pin_fp8_decode_sdpa,
 ]

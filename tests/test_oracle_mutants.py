@@ -69,6 +69,18 @@ MUTATIONS = [
      "attend_range(q, kc, vc, head_dim, 0, ctx > 1 ? ctx - 1 : ctx, scale, z, &m, &l, acc);"),
     ("merge: partition weight dropped", "double w = exp(part_max[base + p] - big_m);", "double w = 1.0;"),
     ("merge: sum not weighted", "big_l += w * part_sum[base + p];", "big_l += part_sum[base + p];"),
+    ("copy: destination and source swapped",
+     "memmove(key_cache + dst * block_bytes, key_cache + src * block_bytes, block_bytes);",
+     "memmove(key_cache + src * block_bytes, key_cache + dst * block_bytes, block_bytes);"),
+    ("copy: half a block", "size_t block_bytes = (size_t)(block_size * num_kv_heads * head_dim * elem_bytes);",
+     "size_t block_bytes = (size_t)(block_size * num_kv_heads * head_dim * elem_bytes / 2);"),
+    ("e4m3 decode: exponent bias", "mag = ldexp((double)(8 + frac), expo - 10);",
+     "mag = ldexp((double)(8 + frac), expo - 11);"),
+    ("e4m3 encode: no saturation", "if (a > 448.0 || isinf(a)) a = 448.0;", "if (isinf(a)) a = 448.0;"),
+    ("e4m3 encode: scale not applied", "key_cache[slot * row + e] = oracle_f64_to_e4m3((double)(kx * inv_k));",
+     "key_cache[slot * row + e] = oracle_f64_to_e4m3((double)kx);"),
+    ("fp8 decode: v scale dropped", "vc[j * head_dim + d] = oracle_e4m3_to_f64(value_cache[base + d]) * v_scale;",
+     "vc[j * head_dim + d] = oracle_e4m3_to_f64(value_cache[base + d]);"),
     ("partition: end not clipped to ctx",
      "int64_t t1 = t0 + partition_size < ctx ? t0 + partition_size : ctx;",
      "int64_t t1 = t0 + partition_size < ctx ? t0 + partition_size : ctx - 1;"),
