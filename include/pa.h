@@ -98,6 +98,25 @@ pa_status pa_reshape_and_cache(const void *key, const void *value,
                                pa_dtype dtype, void *stream);
 
 /*
+ * pa_copy_blocks -- the device half of copy-on-write: before a sequence
+ * writes into a block it shares with others (ref_count > 1), the block is
+ * copied to a private one ("vllm源码分析" 第一讲; "vLLM PagedAttention 原理与源码
+ * 深度解析" §3.3).
+ *   key_cache, value_cache  [num_blocks, block_size, num_kv_heads, head_dim],
+ *                           elem_bytes per element (2 for fp16/bf16, 1 for fp8)
+ *   block_mapping           [num_pairs, 2] int64 (device): (source, destination)
+ * Copies every byte of block source onto block destination, in both caches.
+ * Destinations must be distinct and must not be the source of another pair in
+ * the same call.  An id outside [0, num_blocks) skips its pair and is reported
+ * by pa_check_error (PA_CHECK_BLOCK_ID, index = pair).  A block must be a
+ * multiple of 16 bytes and both caches 16-byte aligned.
+ */
+pa_status pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *block_mapping,
+                         int64_t num_pairs, int64_t num_blocks, int64_t block_size,
+                         int64_t num_kv_heads, int64_t head_dim, int64_t elem_bytes,
+                         void *stream);
+
+/*
  * pa_decode -- single-pass paged decode attention, one query token per sequence.
  * ("vLLM PagedAttention 原理与源码深度解析" §5.3.)
  *   out            [num_seqs, num_heads, head_dim]       (written)
@@ -183,6 +202,50 @@ pa_status pa_decode_shared_prefix(void *out, const void *query, const void *key_
                                   int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
                                   int64_t block_size, int64_t max_blocks_per_seq,
                                   pa_dtype dtype, void *stream);
+
+/*
+ * FP8 KV cache ("vLLM PagedAttention 原理与源码深度解析" §8.4: --kv-cache-dtype
+ * fp8).  The caches hold one byte per element, an OCP E4M3 code c; with one
+ * scale per cache tensor, c stands for c * k_scale in the key cache and
+ * c * v_scale in the value cache (k_scale, v_scale finite and > 0).  Query,
+ * new K/V rows and outputs stay 16-bit (dtype).  head_dim must be 128 for the
+ * decode calls.
+ *
+ * pa_reshape_and_cache_fp8 -- as pa_reshape_and_cache, but element x of key
+ * (value) is stored as E4M3(x * (1.0f / k_scale)) (resp. v_scale): the
+ * reciprocal and the product in float, then nearest-even to E4M3 with
+ * saturation to +-448 (NaN stays NaN).  Caches are [num_blocks, block_size,
+ * num_kv_heads, head_dim] bytes; head_dim must be a multiple of 16.
+ */
+pa_status pa_reshape_and_cache_fp8(const void *key, const void *value,
+                                   int64_t key_stride, int64_t value_stride,
+                                   void *key_cache, void *value_cache,
+                                   const int64_t *slot_mapping, int64_t num_tokens,
+                                   int64_t num_kv_heads, int64_t head_dim,
+                                   int64_t num_blocks, int64_t block_size,
+                                   float k_scale, float v_scale, pa_dtype dtype,
+                                   void *stream);
+
+/* pa_decode over E4M3 caches: out = softmax(scale * q . (c_k * k_scale)) . (c_v * v_scale). */
+pa_status pa_decode_fp8(void *out, const void *query, const void *key_cache,
+                        const void *value_cache, const int32_t *block_tables,
+                        const int32_t *context_lens, float scale, float k_scale,
+                        float v_scale, int64_t num_seqs, int64_t num_heads,
+                        int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                        int64_t block_size, int64_t max_blocks_per_seq, pa_dtype dtype,
+                        void *stream);
+
+/* pa_decode_split over E4M3 caches (partials as pa_decode_split, in dequantised
+ * units); merge them with pa_reduce. */
+pa_status pa_decode_split_fp8(float *tmp_out, float *max_logits, float *exp_sums,
+                              const void *query, const void *key_cache,
+                              const void *value_cache, const int32_t *block_tables,
+                              const int32_t *context_lens, float scale, float k_scale,
+                              float v_scale, int64_t num_seqs, int64_t num_heads,
+                              int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                              int64_t block_size, int64_t max_blocks_per_seq,
+                              int64_t partition_size, int64_t max_partitions,
+                              pa_dtype dtype, void *stream);
 
 /*
  * pa_check_error -- synchronise `stream`, read and clear the current device's

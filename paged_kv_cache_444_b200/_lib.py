@@ -60,6 +60,13 @@ SIGNATURES = {
                                _i64, _i64, _i, _p]),
     "pa_decode_shared_prefix": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _f, _i64, _i64, _i64, _i64,
                                      _i64, _i64, _i64, _i64, _i64, _i, _p]),
+    "pa_copy_blocks": (_i, [_p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p]),
+    "pa_reshape_and_cache_fp8": (_i, [_p, _p, _i64, _i64, _p, _p, _p, _i64, _i64, _i64, _i64,
+                                      _i64, _f, _f, _i, _p]),
+    "pa_decode_fp8": (_i, [_p, _p, _p, _p, _p, _p, _f, _f, _f, _i64, _i64, _i64, _i64, _i64,
+                           _i64, _i64, _i, _p]),
+    "pa_decode_split_fp8": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _f, _f, _f, _i64, _i64, _i64,
+                                 _i64, _i64, _i64, _i64, _i64, _i64, _i, _p]),
 }
 
 _lib: ctypes.CDLL | None = None
@@ -227,6 +234,90 @@ def pa_decode_shared_prefix(out: torch.Tensor, query: torch.Tensor, key_cache: t
         prefix_blocks.data_ptr(), float(scale), S, n_groups, int(max_group_size), H, Hk, D, NB,
         bs, MB, dt, _stream(stream))
     _check(st, "pa_decode_shared_prefix")
+
+
+def pa_copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor,
+                   block_mapping: torch.Tensor, stream=None) -> None:
+    """Copy whole blocks (copy-on-write): block_mapping [n, 2] int64 holds
+    (source, destination) pairs; caches [NB, bs, Hk, D] contiguous."""
+    NB, bs, Hk, D = key_cache.shape
+    _need(value_cache.shape == key_cache.shape and key_cache.dtype == value_cache.dtype,
+          "key/value caches differ")
+    _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
+    _need(block_mapping.dtype == torch.int64 and block_mapping.dim() == 2 and
+          block_mapping.shape[1] == 2 and block_mapping.is_contiguous(),
+          "block_mapping must be [n, 2] int64")
+    st = load().pa_copy_blocks(key_cache.data_ptr(), value_cache.data_ptr(),
+                               block_mapping.data_ptr(), block_mapping.shape[0], NB, bs, Hk, D,
+                               key_cache.element_size(), _stream(stream))
+    _check(st, "pa_copy_blocks")
+
+
+def _fp8_caches(key_cache, value_cache):
+    _need(key_cache.dtype == torch.uint8 and value_cache.dtype == torch.uint8,
+          "fp8 caches are uint8 tensors of E4M3 codes")
+    _need(key_cache.shape == value_cache.shape and key_cache.dim() == 4, "cache shapes")
+    _need(key_cache.is_contiguous() and value_cache.is_contiguous(), "caches must be contiguous")
+    return key_cache.shape
+
+
+def pa_reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
+                             value_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                             k_scale: float, v_scale: float, stream=None) -> None:
+    """Quantising write of 16-bit key/value [T, Hk, D] into uint8 E4M3 caches."""
+    T, Hk, D = key.shape
+    NB, bs, _, _ = _fp8_caches(key_cache, value_cache)
+    _need(value.shape == key.shape and key.dtype == value.dtype, "key/value differ")
+    _need(key.stride()[1:] == (D, 1) and value.stride()[1:] == (D, 1), "rows must be dense")
+    _need(slot_mapping.dtype == torch.int64 and slot_mapping.shape == (T,), "slot_mapping")
+    st = load().pa_reshape_and_cache_fp8(
+        key.data_ptr(), value.data_ptr(), key.stride(0) if T else Hk * D,
+        value.stride(0) if T else Hk * D, key_cache.data_ptr(), value_cache.data_ptr(),
+        slot_mapping.data_ptr(), T, Hk, D, NB, bs, float(k_scale), float(v_scale),
+        _dtype_code(key), _stream(stream))
+    _check(st, "pa_reshape_and_cache_fp8")
+
+
+def _fp8_attention_common(query, key_cache, value_cache, block_tables, context_lens):
+    S, H, D = query.shape
+    NB, bs, Hk, D2 = _fp8_caches(key_cache, value_cache)
+    _need(D2 == D, "head_dim of query and cache differ")
+    _need(query.is_contiguous(), "query must be contiguous")
+    _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
+          block_tables.shape[0] == S and block_tables.is_contiguous(), "block_tables")
+    _need(context_lens.dtype == torch.int32 and context_lens.shape == (S,), "context_lens")
+    return S, H, D, NB, bs, Hk, block_tables.shape[1], _dtype_code(query)
+
+
+def pa_decode_fp8(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                  value_cache: torch.Tensor, block_tables: torch.Tensor,
+                  context_lens: torch.Tensor, scale: float, k_scale: float, v_scale: float,
+                  stream=None) -> None:
+    S, H, D, NB, bs, Hk, MB, dt = _fp8_attention_common(query, key_cache, value_cache,
+                                                        block_tables, context_lens)
+    _need(out.shape == query.shape and out.dtype == query.dtype and out.is_contiguous(), "out")
+    st = load().pa_decode_fp8(out.data_ptr(), query.data_ptr(), key_cache.data_ptr(),
+                              value_cache.data_ptr(), block_tables.data_ptr(),
+                              context_lens.data_ptr(), float(scale), float(k_scale),
+                              float(v_scale), S, H, Hk, D, NB, bs, MB, dt, _stream(stream))
+    _check(st, "pa_decode_fp8")
+
+
+def pa_decode_split_fp8(tmp_out, max_logits, exp_sums, query, key_cache, value_cache,
+                        block_tables, context_lens, scale: float, k_scale: float,
+                        v_scale: float, partition_size: int, stream=None) -> None:
+    S, H, D, NB, bs, Hk, MB, dt = _fp8_attention_common(query, key_cache, value_cache,
+                                                        block_tables, context_lens)
+    P = max_logits.shape[-1]
+    _need(tmp_out.shape == (S, H, P, D) and tmp_out.dtype == torch.float32, "tmp_out")
+    _need(max_logits.shape == (S, H, P) and exp_sums.shape == (S, H, P), "partials")
+    st = load().pa_decode_split_fp8(tmp_out.data_ptr(), max_logits.data_ptr(),
+                                    exp_sums.data_ptr(), query.data_ptr(), key_cache.data_ptr(),
+                                    value_cache.data_ptr(), block_tables.data_ptr(),
+                                    context_lens.data_ptr(), float(scale), float(k_scale),
+                                    float(v_scale), S, H, Hk, D, NB, bs, MB, int(partition_size),
+                                    P, dt, _stream(stream))
+    _check(st, "pa_decode_split_fp8")
 
 
 def pa_check_error(stream=None) -> int:

@@ -12,6 +12,7 @@
 #include "pa.h"
 #include "pa_cache_reduce.cuh"
 #include "pa_decode.cuh"
+#include "pa_decode_fp8.cuh"
 #include "pa_shared_prefix.cuh"
 
 namespace {
@@ -46,18 +47,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 //   dim3: num_blocks*16 token rows         stride Hk*D*2 B
 // box {64, 1, 1, 16}, 128-byte swizzle, zero fill out of range.
 bool encode_cache_map(CUtensorMap* map, const void* cache, pa_dtype dtype, int64_t num_blocks,
-                      int64_t num_kv_heads, int64_t head_dim) {
+                      int64_t num_kv_heads, int64_t head_dim, int elem_bytes = 2) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(head_dim / 64),
+  const cuuint64_t per_box = 128 / elem_bytes;   // elements in one 128-byte box row
+  const cuuint64_t dims[4] = {per_box, static_cast<cuuint64_t>(head_dim * elem_bytes / 128),
                               static_cast<cuuint64_t>(num_kv_heads),
                               static_cast<cuuint64_t>(num_blocks * kPage)};
-  const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(head_dim * 2),
-                                 static_cast<cuuint64_t>(num_kv_heads * head_dim * 2)};
-  const cuuint32_t box[4] = {64, 1, 1, kPage};
+  const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(head_dim * elem_bytes),
+                                 static_cast<cuuint64_t>(num_kv_heads * head_dim * elem_bytes)};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(per_box), 1, 1, kPage};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = fn(map, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+  const CUtensorMapDataType type = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUresult r = fn(map, type,
                         4, const_cast<void*>(cache), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -123,6 +127,9 @@ pa_status launch_ex(K kernel, unsigned grid, unsigned block, size_t smem, cudaSt
 #ifndef PA_STAGES_D64
 #define PA_STAGES_D64 4
 #endif
+#ifndef PA_STAGES_FP8
+#define PA_STAGES_FP8 4  // fp8 pages are half the bytes: twice the stages in the same space
+#endif
 template <int D>
 struct Stages { static constexpr int value = D == 64 ? PA_STAGES_D64 : PA_STAGES_D128; };
 
@@ -172,12 +179,12 @@ int pick_cluster(K kernel, int smem_bytes, int64_t max_pages, int* cache) {
   return want < cache[dev] ? want : cache[dev];
 }
 
-template <int D, bool BF16, class Warp>
+template <int D, bool BF16, class Warp, int EB = 2>
 pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeArgs a,
                           long long grid, int64_t max_pages, cudaStream_t stream) {
-  constexpr int NST = Stages<D>::value;
-  using L = DecodeSmem<D, NST>;
-  auto kernel = paged_decode_kernel<D, NST, BF16, Warp>;
+  constexpr int NST = EB == 1 ? PA_STAGES_FP8 : Stages<D>::value;
+  using L = DecodeSmem<D, NST, EB>;
+  auto kernel = paged_decode_kernel<D, NST, BF16, Warp, EB>;
   static std::atomic<uint64_t> done{0};
   static int cluster_cache[kMaxDevices] = {};
   if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
@@ -279,6 +286,43 @@ pa_status launch_shared_prefix_t(const CUtensorMap& km, const CUtensorMap& vm,
                    vm, a);
 }
 
+// Decode over E4M3 caches (head_dim 128): same kernel, fp8 page steps.
+pa_status run_decode_fp8(DecodeArgs a, const void* key_cache, const void* value_cache,
+                         int64_t num_seqs, int64_t num_blocks, pa_dtype dtype,
+                         cudaStream_t stream) {
+  CUtensorMap km, vm;
+  if (!encode_cache_map(&km, key_cache, dtype, num_blocks, a.num_kv_heads, 128, 1) ||
+      !encode_cache_map(&vm, value_cache, dtype, num_blocks, a.num_kv_heads, 128, 1))
+    return PA_ERR_CUDA;
+  const long long grid = num_seqs * a.num_kv_heads * static_cast<long long>(a.parts_per_head);
+  if (grid > INT32_MAX) return PA_ERR_SHAPE;
+  const int64_t max_pages = a.max_blocks_per_seq;
+  if (dtype == PA_BF16) {
+    if (a.group == 1)
+      return launch_decode_t<128, true, SimtFp8Warp<128, true>, 1>(km, vm, a, grid, max_pages,
+                                                                  stream);
+    if (a.group <= 8)
+      return launch_decode_t<128, true, MmaFp8Warp<128, true, false>, 1>(km, vm, a, grid,
+                                                                        max_pages, stream);
+    return launch_decode_t<128, true, MmaFp8Warp<128, true, true>, 1>(km, vm, a, grid, max_pages,
+                                                                     stream);
+  }
+  if (a.group == 1)
+    return launch_decode_t<128, false, SimtFp8Warp<128, false>, 1>(km, vm, a, grid, max_pages,
+                                                                  stream);
+  if (a.group <= 8)
+    return launch_decode_t<128, false, MmaFp8Warp<128, false, false>, 1>(km, vm, a, grid,
+                                                                        max_pages, stream);
+  return launch_decode_t<128, false, MmaFp8Warp<128, false, true>, 1>(km, vm, a, grid, max_pages,
+                                                                     stream);
+}
+
+pa_status check_fp8_scales(float k_scale, float v_scale) {
+  if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f))
+    return PA_ERR_SHAPE;
+  return PA_OK;
+}
+
 DecodeArgs make_args(const void* query, const int32_t* block_tables, const int32_t* context_lens,
                      float scale, int64_t num_heads, int64_t num_kv_heads,
                      int64_t max_blocks_per_seq, int64_t num_blocks) {
@@ -287,6 +331,7 @@ DecodeArgs make_args(const void* query, const int32_t* block_tables, const int32
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.scale_log2 = scale * kLog2e;
+  a.v_scale = 1.0f;
   a.num_heads = static_cast<int>(num_heads);
   a.num_kv_heads = static_cast<int>(num_kv_heads);
   a.group = static_cast<int>(num_heads / num_kv_heads);
@@ -349,6 +394,31 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, int64_t key_s
                    static_cast<uint16_t*>(value_cache), slot_mapping,
                    static_cast<long long>(num_tokens), static_cast<int>(chunks),
                    static_cast<long long>(num_blocks * block_size));
+}
+
+pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_mapping,
+                         int64_t num_pairs, int64_t num_blocks, int64_t block_size,
+                         int64_t num_kv_heads, int64_t head_dim, int64_t elem_bytes,
+                         void* stream) {
+  if (num_pairs < 0 || num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 ||
+      head_dim <= 0 || (elem_bytes != 1 && elem_bytes != 2))
+    return PA_ERR_SHAPE;
+  if (num_pairs == 0) return PA_OK;
+  if (!key_cache || !value_cache || !block_mapping) return PA_ERR_NULL;
+  const int64_t block_bytes = block_size * num_kv_heads * head_dim * elem_bytes;
+  if (block_bytes % 16 != 0 || !aligned16(key_cache) || !aligned16(value_cache) ||
+      (reinterpret_cast<uintptr_t>(block_mapping) & 7u))
+    return PA_ERR_ALIGN;
+  const int64_t units = block_bytes / 16;
+  const int64_t total = num_pairs * units;
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  if (blocks > 148 * 32) blocks = 148 * 32;
+  return launch_ex(copy_blocks_kernel, static_cast<unsigned>(blocks), threads, 0,
+                   as_stream(stream), 1, static_cast<uint4*>(key_cache),
+                   static_cast<uint4*>(value_cache), block_mapping,
+                   static_cast<long long>(num_pairs), static_cast<long long>(units),
+                   static_cast<long long>(num_blocks));
 }
 
 pa_status pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
@@ -478,6 +548,102 @@ pa_status pa_decode_shared_prefix(void* out, const void* query, const void* key_
                 : launch_shared_prefix_t<64, false>(km, vm, a, items, s);
   return bf16 ? launch_shared_prefix_t<128, true>(km, vm, a, items, s)
               : launch_shared_prefix_t<128, false>(km, vm, a, items, s);
+}
+
+pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, int64_t key_stride,
+                                   int64_t value_stride, void* key_cache, void* value_cache,
+                                   const int64_t* slot_mapping, int64_t num_tokens,
+                                   int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                                   int64_t block_size, float k_scale, float v_scale,
+                                   pa_dtype dtype, void* stream) {
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_DTYPE;
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 || block_size <= 0)
+    return PA_ERR_SHAPE;
+  pa_status st = check_fp8_scales(k_scale, v_scale);
+  if (st != PA_OK) return st;
+  const int64_t row = num_kv_heads * head_dim;
+  if (key_stride < row || value_stride < row) return PA_ERR_SHAPE;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_NULL;
+  if (head_dim % 16 != 0 || key_stride % 8 != 0 || value_stride % 8 != 0) return PA_ERR_ALIGN;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache) ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return PA_ERR_ALIGN;
+  const int64_t chunks = row / 16;
+  if (chunks > INT32_MAX) return PA_ERR_SHAPE;
+  const int64_t total = num_tokens * chunks;
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  if (blocks > 148 * 32) blocks = 148 * 32;
+  const float inv_k = 1.0f / k_scale, inv_v = 1.0f / v_scale;
+  auto kernel = dtype == PA_BF16 ? reshape_and_cache_fp8_kernel<true>
+                                 : reshape_and_cache_fp8_kernel<false>;
+  return launch_ex(kernel, static_cast<unsigned>(blocks), threads, 0, as_stream(stream), 1,
+                   static_cast<const uint16_t*>(key), static_cast<const uint16_t*>(value),
+                   static_cast<long long>(key_stride), static_cast<long long>(value_stride),
+                   static_cast<uint8_t*>(key_cache), static_cast<uint8_t*>(value_cache),
+                   slot_mapping, static_cast<long long>(num_tokens), static_cast<int>(chunks),
+                   static_cast<long long>(num_blocks * block_size), inv_k, inv_v);
+}
+
+pa_status pa_decode_fp8(void* out, const void* query, const void* key_cache,
+                        const void* value_cache, const int32_t* block_tables,
+                        const int32_t* context_lens, float scale, float k_scale, float v_scale,
+                        int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads,
+                        int64_t head_dim, int64_t num_blocks, int64_t block_size,
+                        int64_t max_blocks_per_seq, pa_dtype dtype, void* stream) {
+  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
+                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
+                                      num_blocks, block_size, max_blocks_per_seq, dtype);
+  if (st != PA_OK) return st;
+  if ((st = check_fp8_scales(k_scale, v_scale)) != PA_OK) return st;
+  if (head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out) return PA_ERR_NULL;
+  if (!aligned16(out)) return PA_ERR_ALIGN;
+  DecodeArgs a = make_args(query, block_tables, context_lens, scale * k_scale, num_heads,
+                           num_kv_heads, max_blocks_per_seq, num_blocks);
+  a.v_scale = v_scale;
+  a.out = static_cast<uint16_t*>(out);
+  a.num_seqs = static_cast<int>(num_seqs);
+  a.longest_first = num_seqs > 1 && num_seqs <= kLptMaxSeqs;
+  return run_decode_fp8(a, key_cache, value_cache, num_seqs, num_blocks, dtype,
+                        as_stream(stream));
+}
+
+pa_status pa_decode_split_fp8(float* tmp_out, float* max_logits, float* exp_sums,
+                              const void* query, const void* key_cache, const void* value_cache,
+                              const int32_t* block_tables, const int32_t* context_lens,
+                              float scale, float k_scale, float v_scale, int64_t num_seqs,
+                              int64_t num_heads, int64_t num_kv_heads, int64_t head_dim,
+                              int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq,
+                              int64_t partition_size, int64_t max_partitions, pa_dtype dtype,
+                              void* stream) {
+  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
+                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
+                                      num_blocks, block_size, max_blocks_per_seq, dtype);
+  if (st != PA_OK) return st;
+  if ((st = check_fp8_scales(k_scale, v_scale)) != PA_OK) return st;
+  if (head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (partition_size <= 0 || max_partitions <= 0) return PA_ERR_SHAPE;
+  if (partition_size % kPage != 0) return PA_ERR_UNSUPPORTED;
+  if (partition_size > INT32_MAX || max_partitions > INT32_MAX) return PA_ERR_SHAPE;
+  if (num_seqs == 0) return PA_OK;
+  if (!tmp_out || !max_logits || !exp_sums) return PA_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(tmp_out) & 7u) || (reinterpret_cast<uintptr_t>(max_logits) & 3u) ||
+      (reinterpret_cast<uintptr_t>(exp_sums) & 3u))
+    return PA_ERR_ALIGN;
+  DecodeArgs a = make_args(query, block_tables, context_lens, scale * k_scale, num_heads,
+                           num_kv_heads, max_blocks_per_seq, num_blocks);
+  a.v_scale = v_scale;
+  a.tmp_out = tmp_out;
+  a.max_logits = max_logits;
+  a.exp_sums = exp_sums;
+  a.partition_size = static_cast<int>(partition_size);
+  a.parts_per_head = static_cast<int>(max_partitions);
+  a.max_partitions = static_cast<int>(max_partitions);
+  return run_decode_fp8(a, key_cache, value_cache, num_seqs, num_blocks, dtype,
+                        as_stream(stream));
 }
 
 pa_status pa_check_error(void* stream, int64_t* detail) {

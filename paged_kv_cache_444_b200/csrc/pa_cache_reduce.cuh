@@ -40,6 +40,34 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
+// Block copy for copy-on-write ("vllm源码分析" 第一讲, "vLLM PagedAttention
+// 原理与源码深度解析" §3.3): before a sequence writes into a block it shares,
+// the block is copied to a private one.  Pair i copies block mapping[2i] onto
+// block mapping[2i+1] in both caches; one thread moves one 16-byte unit of K
+// and the same unit of V, consecutive threads walk a block.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    copy_blocks_kernel(uint4* __restrict__ key_cache, uint4* __restrict__ value_cache,
+                       const int64_t* __restrict__ mapping, long long num_pairs,
+                       long long units_per_block, long long num_blocks) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const long long total = num_pairs * units_per_block;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long pair = i / units_per_block;
+    const long long u = i - pair * units_per_block;
+    const long long src = mapping[2 * pair], dst = mapping[2 * pair + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+      if (u == 0) record_error(kErrBlockId, pair);
+      continue;
+    }
+    key_cache[dst * units_per_block + u] = key_cache[src * units_per_block + u];
+    value_cache[dst * units_per_block + u] = value_cache[src * units_per_block + u];
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Log-sum-exp merge of split partitions.  One CTA per (sequence, query head):
 //   M = max_p m_p;  w_p = exp(m_p - M);  out = sum_p w_p acc_p / sum_p w_p l_p.
 // Single pass: thread t owns the float4 column t % (D/4) of every

@@ -51,7 +51,8 @@ struct DecodeArgs {
   float* exp_sums;            // [S, H, P]
   const int32_t* block_tables;  // [S, MB]
   const int32_t* context_lens;  // [S]
-  float scale_log2;           // scale * log2(e)
+  float scale_log2;           // scale * log2(e) (* k_scale for an fp8 cache)
+  float v_scale;              // multiplies every output (1, or v_scale for an fp8 cache)
   int num_heads;
   int num_kv_heads;
   int group;                  // num_heads / num_kv_heads
@@ -66,9 +67,10 @@ struct DecodeArgs {
 };
 
 
-template <int D, int NST>
+template <int D, int NST, int EB = 2>   // EB: bytes per cache element (2, or 1 for fp8)
 struct DecodeSmem {
-  static constexpr int kPageBytes = kPage * D * 2;       // one tensor, one page, one head
+  static constexpr int kPageBytes = kPage * D * EB;      // one tensor, one page, one head
+  static constexpr int kBoxesPerRow = D * EB / 128;       // 128-byte TMA boxes per row
   static constexpr int kStageBytes = 2 * kPageBytes;      // K page + V page
   static constexpr int kStagesBytes = kWarps * NST * kStageBytes;
   static constexpr int kBarOffset = kStagesBytes;
@@ -83,7 +85,7 @@ struct DecodeSmem {
   // floats) and, for an item spread over a cluster, this CTA's merged rows
   static constexpr int kPartAccOffset = kWarps * 16 * D * 4;
   static_assert(kPartAccOffset + 16 * D * 4 <= kStagesBytes, "merge buffers must fit in the stages");
-  static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
+  static_assert((D * EB) % 128 == 0, "a cache row must be a whole number of 128-byte boxes");
   static_assert((kLptMaxSeqs + 1) * 4 <= kStagesBytes, "length table must fit in the stages");
 };
 
@@ -397,10 +399,10 @@ struct SimtWarp {
 // max m (log2 domain) and the row sum l.  With `spread`, every CTA of the
 // cluster must call this (it holds two cluster barriers); each emits a slice.
 // ---------------------------------------------------------------------------
-template <int D, int NST, class Emit>
+template <int D, int NST, int EB = 2, class Emit>
 __device__ __forceinline__ void merge_and_emit(uint8_t* smem, int nrows, bool spread, int ctas,
                                                int crank, Emit&& emit) {
-  using L = DecodeSmem<D, NST>;
+  using L = DecodeSmem<D, NST, EB>;
   const float* red_acc = reinterpret_cast<const float*>(smem);
   const float* red_m = reinterpret_cast<const float*>(smem + L::kRedMOffset);
   const float* red_l = reinterpret_cast<const float*>(smem + L::kRedLOffset);
@@ -484,11 +486,11 @@ __device__ __forceinline__ void merge_and_emit(uint8_t* smem, int nrows, bool sp
 // takes the same branch and either all of them reach both cluster barriers
 // or none does.
 // ---------------------------------------------------------------------------
-template <int D, int NST, bool BF16, class Warp>
+template <int D, int NST, bool BF16, class Warp, int EB = 2>
 __global__ void __launch_bounds__(kThreads)
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
-  using L = DecodeSmem<D, NST>;
+  using L = DecodeSmem<D, NST, EB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -609,9 +611,11 @@ __global__ void __launch_bounds__(kThreads)
       const int row = id * kPage;
       mbar_arrive_expect_tx(bar, L::kStageBytes);
 #pragma unroll
-      for (int b = 0; b < D / 64; ++b) tma_load_4d(dk + b * kBoxBytes, &kmap, bar, 0, b, kvh, row);
+      for (int b = 0; b < L::kBoxesPerRow; ++b)
+        tma_load_4d(dk + b * kBoxBytes, &kmap, bar, 0, b, kvh, row);
 #pragma unroll
-      for (int b = 0; b < D / 64; ++b) tma_load_4d(dv + b * kBoxBytes, &vmap, bar, 0, b, kvh, row);
+      for (int b = 0; b < L::kBoxesPerRow; ++b)
+        tma_load_4d(dv + b * kBoxBytes, &vmap, bar, 0, b, kvh, row);
     }
   };
 
@@ -662,9 +666,11 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
 
   const size_t hrow0 = static_cast<size_t>(s) * a.num_heads + static_cast<size_t>(kvh) * group;
-  merge_and_emit<D, NST>(smem, group, spread, ctas, crank,
-                         [&](int g, int d, float o0, float o1, float big_m, float big_l) {
+  merge_and_emit<D, NST, EB>(smem, group, spread, ctas, crank,
+                             [&](int g, int d, float o0, float o1, float big_m, float big_l) {
     const size_t hrow = hrow0 + g;
+    o0 *= a.v_scale;
+    o1 *= a.v_scale;
     if (split) {
       const size_t pidx = hrow * a.max_partitions + part;
       *reinterpret_cast<float2*>(a.tmp_out + pidx * D + d) = make_float2(o0, o1);

@@ -1,0 +1,374 @@
+// pa_decode_fp8.cuh -- page steps of paged decode attention over an E4M3
+// (fp8) KV cache ("vLLM PagedAttention 原理与源码深度解析" §8.4 names the
+// --kv-cache-dtype fp8 option; the scheme here is one scale per cache tensor:
+// a stored code c means c * k_scale for K and c * v_scale for V).
+//
+// A cached row of head_dim 128 is 128 bytes: one 128-byte-swizzled TMA box
+// per page and tensor, so a page of one head is 2 KB instead of 4 KB.  The
+// query stays 16-bit; k_scale is folded into the logit scale and v_scale into
+// the output, so the page steps below work on the raw codes:
+//  - SimtFp8Warp (one query head per KV head): codes -> fp16 -> fp32 with
+//    cvt.rn.f16x2.e4m3x2, then packed fp32 FMA as in the 16-bit path.
+//  - MmaFp8Warp (GQA group): the page is read with the same b16 ldmatrix as
+//    the 16-bit path, which hands each lane 4 consecutive codes of a row
+//    where the 16-bit fragment layout expects 2 + 2 codes 8 apart.  Inside
+//    one 16-element k-step that is a fixed permutation of the head dims, so
+//    Q's A fragments are loaded with the same permutation and S = Q K^T is
+//    unchanged.  For P.V the transposed ldmatrix hands each lane 2 tokens x
+//    2 dims; a byte permute splits them into the even-dim and odd-dim
+//    fragments of two n-tiles, and the output dims are put back in order
+//    when the warp publishes its rows.
+#pragma once
+
+#include "pa_decode.cuh"
+
+namespace pa {
+
+// ---------------------------------------------------------------------------
+// CUDA-core path, head_dim 128
+// ---------------------------------------------------------------------------
+template <int D, bool BF16>
+struct SimtFp8Warp {
+  static_assert(D == 128, "fp8 CUDA-core path is built for head_dim 128");
+  static constexpr int QCH = 4;   // 16-byte chunks (16 dims) per lane in Q.K: half a row
+  static constexpr int TPL = 4;   // tokens per lane in P.V (4 token groups x 8 chunks)
+  float2 qf[QCH * 8];             // this lane's 64 query dims, in its read order
+  float2 acc[8];                  // 16 output dims of one token group
+  float m, l;
+  uint32_t kxor;
+  int krow;
+
+  __device__ __forceinline__ void init(const uint16_t* q_row, int, int lane) {
+    const int tok = lane >> 1, hf = lane & 1;
+    kxor = static_cast<uint32_t>(((hf * 4) ^ (tok & 7)) << 4);
+    krow = tok * 128;
+#pragma unroll
+    for (int k = 0; k < QCH; ++k) {
+      const int c = hf * 4 + k;   // logical chunk read at step k (physical k ^ kxor)
+      const uint4 r0 = *reinterpret_cast<const uint4*>(q_row + c * 16);
+      const uint4 r1 = *reinterpret_cast<const uint4*>(q_row + c * 16 + 8);
+      qf[k * 8 + 0] = unpack2<BF16>(r0.x);
+      qf[k * 8 + 1] = unpack2<BF16>(r0.y);
+      qf[k * 8 + 2] = unpack2<BF16>(r0.z);
+      qf[k * 8 + 3] = unpack2<BF16>(r0.w);
+      qf[k * 8 + 4] = unpack2<BF16>(r1.x);
+      qf[k * 8 + 5] = unpack2<BF16>(r1.y);
+      qf[k * 8 + 6] = unpack2<BF16>(r1.z);
+      qf[k * 8 + 7] = unpack2<BF16>(r1.w);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = make_float2(0.f, 0.f);
+    m = -INFINITY;
+    l = 0.f;
+  }
+
+  __device__ __forceinline__ void page(uint32_t kbase, uint32_t vbase, int tok0, int t_end,
+                                       float scale_log2, int lane, float* probs) {
+    const int tok = lane >> 1, hf = lane & 1;
+    float2 d2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < QCH; ++k) {
+      const uint4 raw = lds128(kbase + krow + ((static_cast<uint32_t>(k) << 4) ^ kxor));
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        d2 = ffma2(qf[k * 8 + 2 * i], e4m3x2_to_f2(w[i]), d2);
+        d2 = ffma2(qf[k * 8 + 2 * i + 1], e4m3x2_to_f2(w[i] >> 16), d2);
+      }
+    }
+    float dot = d2.x + d2.y;
+    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+    const float x = (tok0 + tok) < t_end ? dot * scale_log2 : -INFINITY;
+    float mx = x;
+#pragma unroll
+    for (int o = 2; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float mn = fmaxf(m, mx);
+    const float al = ex2(m - mn);
+    m = mn;
+    const float p = ex2(x - mn);
+    l = l * al + (hf ? 0.f : p);
+    if (hf == 0) probs[tok] = p;
+    __syncwarp();
+    const int cc = lane & 7, tg = lane >> 3;
+    const float2 al2 = make_float2(al, al);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = fmul2(acc[i], al2);
+    const float4 p4 = *reinterpret_cast<const float4*>(probs + tg * TPL);
+    const float pj[TPL] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+    for (int i = 0; i < TPL; ++i) {
+      const int j = tg * TPL + i;
+      const uint4 raw = lds128(vbase + j * 128 + ((cc ^ (j & 7)) << 4));
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      const float2 pp = make_float2(pj[i], pj[i]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] = ffma2(pp, e4m3x2_to_f2(w[q]), acc[2 * q]);
+        acc[2 * q + 1] = ffma2(pp, e4m3x2_to_f2(w[q] >> 16), acc[2 * q + 1]);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void publish(float* red_acc, float* red_m, float* red_l, int,
+                                          int lane) {
+    float lt = l;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
+#pragma unroll
+    for (int o = 8; o < 32; o <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        acc[i].x += __shfl_xor_sync(0xffffffffu, acc[i].x, o);
+        acc[i].y += __shfl_xor_sync(0xffffffffu, acc[i].y, o);
+      }
+    }
+    if (lane < 8) {
+      float4* dst = reinterpret_cast<float4*>(red_acc + lane * 16);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dst[i] = make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x, acc[2 * i + 1].y);
+    }
+    if (lane == 0) {
+      red_m[0] = m;
+      red_l[0] = lt;
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Tensor-core path (GQA groups of 2..16), head_dim 128
+// ---------------------------------------------------------------------------
+template <int D, bool BF16, bool TWO_ROWS>
+struct MmaFp8Warp {
+  static_assert(D == 128, "fp8 tensor-core path is built for head_dim 128");
+  static constexpr int KSTEPS = D / 16;
+  static constexpr int NTILES = D / 8;
+  uint32_t qa[KSTEPS][4];   // Q fragments, head dims permuted as the fp8 K fragments
+  float acc[NTILES][4];     // n-tile 2c: even dims of 16-dim chunk c; 2c+1: odd dims
+  float m[2], l[2];
+
+  __device__ __forceinline__ void init(const uint16_t* q_group, int group, int lane) {
+    const int r0 = lane >> 2, r1 = r0 + 8, tig = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      // k positions tig*2+{0,1} hold dims 4*tig+{0,1}; positions tig*2+8+{0,1}
+      // hold dims 4*tig+{2,3} of this 16-dim step
+      const int d0 = kk * 16 + tig * 4;
+      const uint32_t* q0 = reinterpret_cast<const uint32_t*>(q_group + r0 * D);
+      const uint32_t* q1 = reinterpret_cast<const uint32_t*>(q_group + r1 * D);
+      qa[kk][0] = r0 < group ? q0[d0 >> 1] : 0u;
+      qa[kk][1] = (TWO_ROWS && r1 < group) ? q1[d0 >> 1] : 0u;
+      qa[kk][2] = r0 < group ? q0[(d0 >> 1) + 1] : 0u;
+      qa[kk][3] = (TWO_ROWS && r1 < group) ? q1[(d0 >> 1) + 1] : 0u;
+    }
+#pragma unroll
+    for (int n = 0; n < NTILES; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.f;
+  }
+
+  __device__ __forceinline__ void page(uint32_t kbase, uint32_t vbase, int tok0, int t_end,
+                                       float scale_log2, int lane, float*) {
+    const int tig = lane & 3;
+    // ---- S = Q K^T: one x4 ldmatrix covers two k-steps for both 8-token n-tiles ----
+    float sc[2][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sc[0][i] = sc[1][i] = 0.f;
+    const int mtok = ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int mchk = lane >> 4;
+#pragma unroll
+    for (int kp = 0; kp < KSTEPS / 2; ++kp) {
+      const int c = 2 * kp + mchk;
+      uint32_t r0, r1, r2, r3;  // (tok 0-7, chunk 2kp) (8-15, 2kp) (0-7, 2kp+1) (8-15, 2kp+1)
+      ldsm_x4(kbase + mtok * 128 + ((c ^ (mtok & 7)) << 4), r0, r1, r2, r3);
+      mma_16816<BF16>(sc[0], qa[2 * kp], e4m3x2_to_op2<BF16>(r0), e4m3x2_to_op2<BF16>(r0 >> 16));
+      mma_16816<BF16>(sc[1], qa[2 * kp], e4m3x2_to_op2<BF16>(r1), e4m3x2_to_op2<BF16>(r1 >> 16));
+      mma_16816<BF16>(sc[0], qa[2 * kp + 1], e4m3x2_to_op2<BF16>(r2),
+                      e4m3x2_to_op2<BF16>(r2 >> 16));
+      mma_16816<BF16>(sc[1], qa[2 * kp + 1], e4m3x2_to_op2<BF16>(r3),
+                      e4m3x2_to_op2<BF16>(r3 >> 16));
+    }
+    // ---- scale, mask, online softmax (as in the 16-bit path) ----
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = tok0 + nt * 8 + tig * 2 + (i & 1);
+        const float x = t < t_end ? sc[nt][i] * scale_log2 : -INFINITY;
+        sc[nt][i] = x;
+        if (i < 2) mx0 = fmaxf(mx0, x); else mx1 = fmaxf(mx1, x);
+      }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    const float mn0 = fmaxf(m[0], mx0);
+    const float al0 = ex2(m[0] - mn0);
+    m[0] = mn0;
+    float mn1 = 0.f, al1 = 1.f;
+    if constexpr (TWO_ROWS) {
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      mn1 = fmaxf(m[1], mx1);
+      al1 = ex2(m[1] - mn1);
+      m[1] = mn1;
+    }
+    float p0[4], p1[4];
+    p0[0] = ex2(sc[0][0] - mn0); p0[1] = ex2(sc[0][1] - mn0);
+    p0[2] = ex2(sc[1][0] - mn0); p0[3] = ex2(sc[1][1] - mn0);
+    if constexpr (TWO_ROWS) {
+      p1[0] = ex2(sc[0][2] - mn1); p1[1] = ex2(sc[0][3] - mn1);
+      p1[2] = ex2(sc[1][2] - mn1); p1[3] = ex2(sc[1][3] - mn1);
+    } else {
+      p1[0] = p1[1] = p1[2] = p1[3] = 0.f;
+    }
+    uint32_t pa[4], pl[4];
+    pa[0] = pack2<BF16>(p0[0], p0[1]);
+    pa[2] = pack2<BF16>(p0[2], p0[3]);
+    pa[1] = TWO_ROWS ? pack2<BF16>(p1[0], p1[1]) : 0u;
+    pa[3] = TWO_ROWS ? pack2<BF16>(p1[2], p1[3]) : 0u;
+    if constexpr (BF16) {
+      const float2 h0 = unpack2<BF16>(pa[0]), h2 = unpack2<BF16>(pa[2]);
+      pl[0] = pack2<BF16>(p0[0] - h0.x, p0[1] - h0.y);
+      pl[2] = pack2<BF16>(p0[2] - h2.x, p0[3] - h2.y);
+      if constexpr (TWO_ROWS) {
+        const float2 h1 = unpack2<BF16>(pa[1]), h3 = unpack2<BF16>(pa[3]);
+        pl[1] = pack2<BF16>(p1[0] - h1.x, p1[1] - h1.y);
+        pl[3] = pack2<BF16>(p1[2] - h3.x, p1[3] - h3.y);
+      } else {
+        pl[1] = pl[3] = 0u;
+      }
+      l[0] = l[0] * al0 + ((p0[0] + p0[1]) + (p0[2] + p0[3]));
+      if constexpr (TWO_ROWS) l[1] = l[1] * al1 + ((p1[0] + p1[1]) + (p1[2] + p1[3]));
+    } else {
+      const float2 u = unpack2<BF16>(pa[0]), v = unpack2<BF16>(pa[2]);
+      l[0] = l[0] * al0 + ((u.x + u.y) + (v.x + v.y));
+      if constexpr (TWO_ROWS) {
+        const float2 w = unpack2<BF16>(pa[1]), z = unpack2<BF16>(pa[3]);
+        l[1] = l[1] * al1 + ((w.x + w.y) + (z.x + z.y));
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < NTILES; ++n) {
+      acc[n][0] *= al0;
+      acc[n][1] *= al0;
+      if constexpr (TWO_ROWS) {
+        acc[n][2] *= al1;
+        acc[n][3] *= al1;
+      }
+    }
+    // ---- O += P V: one transposed x4 ldmatrix covers two 16-dim chunks.  Each
+    // register holds codes [t0: d, d+1][t1: d, d+1] (t0 = 2*tig, d = 2*(lane/4));
+    // bytes {0, 2} feed the even-dim n-tile, bytes {1, 3} the odd-dim one. ----
+#pragma unroll
+    for (int cp = 0; cp < D / 32; ++cp) {
+      const int c = 2 * cp + mchk;
+      uint32_t r0, r1, r2, r3;  // (tok 0-7, chunk 2cp) (8-15, 2cp) (0-7, 2cp+1) (8-15, 2cp+1)
+      ldsm_x4_trans(vbase + mtok * 128 + ((c ^ (mtok & 7)) << 4), r0, r1, r2, r3);
+      const uint32_t e0 = e4m3x2_to_op2<BF16>(__byte_perm(r0, 0, 0x0020));
+      const uint32_t o0 = e4m3x2_to_op2<BF16>(__byte_perm(r0, 0, 0x0031));
+      const uint32_t e1 = e4m3x2_to_op2<BF16>(__byte_perm(r1, 0, 0x0020));
+      const uint32_t o1 = e4m3x2_to_op2<BF16>(__byte_perm(r1, 0, 0x0031));
+      const uint32_t e2 = e4m3x2_to_op2<BF16>(__byte_perm(r2, 0, 0x0020));
+      const uint32_t o2 = e4m3x2_to_op2<BF16>(__byte_perm(r2, 0, 0x0031));
+      const uint32_t e3 = e4m3x2_to_op2<BF16>(__byte_perm(r3, 0, 0x0020));
+      const uint32_t o3 = e4m3x2_to_op2<BF16>(__byte_perm(r3, 0, 0x0031));
+      mma_16816<BF16>(acc[4 * cp + 0], pa, e0, e1);
+      mma_16816<BF16>(acc[4 * cp + 1], pa, o0, o1);
+      mma_16816<BF16>(acc[4 * cp + 2], pa, e2, e3);
+      mma_16816<BF16>(acc[4 * cp + 3], pa, o2, o3);
+      if constexpr (BF16) {
+        mma_16816<BF16>(acc[4 * cp + 0], pl, e0, e1);
+        mma_16816<BF16>(acc[4 * cp + 1], pl, o0, o1);
+        mma_16816<BF16>(acc[4 * cp + 2], pl, e2, e3);
+        mma_16816<BF16>(acc[4 * cp + 3], pl, o2, o3);
+      }
+    }
+  }
+
+  // Rows < group into the merge buffers, head dims back in order: chunk c's
+  // dims 4*tig .. 4*tig+3 are (even c0, odd c0, even c1, odd c1).
+  __device__ __forceinline__ void publish(float* red_acc, float* red_m, float* red_l, int group,
+                                          int lane) {
+    const int r0 = lane >> 2, r1 = r0 + 8, tig = lane & 3;
+    float l0 = l[0];
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    float l1 = l[1];
+    if constexpr (TWO_ROWS) {
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    }
+    if (r0 < group) {
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c)
+        *reinterpret_cast<float4*>(red_acc + r0 * D + c * 16 + tig * 4) =
+            make_float4(acc[2 * c][0], acc[2 * c + 1][0], acc[2 * c][1], acc[2 * c + 1][1]);
+      if (tig == 0) {
+        red_m[r0] = m[0];
+        red_l[r0] = l0;
+      }
+    }
+    if constexpr (TWO_ROWS) {
+      if (r1 < group) {
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c)
+          *reinterpret_cast<float4*>(red_acc + r1 * D + c * 16 + tig * 4) =
+              make_float4(acc[2 * c][2], acc[2 * c + 1][2], acc[2 * c][3], acc[2 * c + 1][3]);
+        if (tig == 0) {
+          red_m[r1] = m[1];
+          red_l[r1] = l1;
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Quantising cache write: key/value rows (16-bit) -> E4M3 codes of x * inv_scale
+// (float product, nearest even, saturating).  One thread makes one 16-byte
+// chunk (16 elements) of K and the same chunk of V.
+// ---------------------------------------------------------------------------
+template <bool BF16>
+__global__ void __launch_bounds__(256)
+    reshape_and_cache_fp8_kernel(const uint16_t* __restrict__ key,
+                                 const uint16_t* __restrict__ value, long long key_stride,
+                                 long long value_stride, uint8_t* __restrict__ key_cache,
+                                 uint8_t* __restrict__ value_cache,
+                                 const int64_t* __restrict__ slot_mapping, long long num_tokens,
+                                 int chunks_per_token, long long num_slots, float inv_k,
+                                 float inv_v) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const long long total = num_tokens * chunks_per_token;
+  const long long row = static_cast<long long>(chunks_per_token) * 16;  // bytes per cache row
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long t = i / chunks_per_token;
+    const int c = static_cast<int>(i - t * chunks_per_token);
+    const long long slot = slot_mapping[t];
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (c == 0) record_error(kErrSlot, t);
+      continue;
+    }
+    auto quantise = [](const uint16_t* src, float inv) {
+      const uint4 a = *reinterpret_cast<const uint4*>(src);
+      const uint4 b = *reinterpret_cast<const uint4*>(src + 8);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      uint32_t out[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 u = unpack2<BF16>(w[2 * k]), v = unpack2<BF16>(w[2 * k + 1]);
+        out[k] = f2_to_e4m3x2(u.x * inv, u.y * inv) | (f2_to_e4m3x2(v.x * inv, v.y * inv) << 16);
+      }
+      return make_uint4(out[0], out[1], out[2], out[3]);
+    };
+    *reinterpret_cast<uint4*>(key_cache + slot * row + c * 16) =
+        quantise(key + t * key_stride + c * 16, inv_k);
+    *reinterpret_cast<uint4*>(value_cache + slot * row + c * 16) =
+        quantise(value + t * value_stride + c * 16, inv_v);
+  }
+}
+
+}  // namespace pa

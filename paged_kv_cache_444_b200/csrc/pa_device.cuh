@@ -241,6 +241,41 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   }
 }
 
+// Two E4M3 values (low byte first) -> half2, exactly (E4M3 is a subset of fp16).
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t pair16) {
+  uint32_t h;
+  const unsigned short p = static_cast<unsigned short>(pair16 & 0xffffu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(p));
+  return h;
+}
+
+// Two E4M3 values -> the packed 16-bit operand type of the mma (fp16 or bf16),
+// exactly: E4M3 -> fp16 is exact, and fp16 values of E4M3 range are exact in bf16.
+template <bool BF16>
+__device__ __forceinline__ uint32_t e4m3x2_to_op2(uint32_t pair16) {
+  const uint32_t h = e4m3x2_to_h2(pair16);
+  if constexpr (BF16) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+    __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+    return *reinterpret_cast<uint32_t*>(&b);
+  } else {
+    return h;
+  }
+}
+
+// Two E4M3 values -> two floats, exactly.
+__device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t pair16) {
+  const uint32_t h = e4m3x2_to_h2(pair16);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// Two floats -> two E4M3 (low byte = lo), nearest even, saturating to +-448.
+__device__ __forceinline__ uint32_t f2_to_e4m3x2(float lo, float hi) {
+  unsigned short r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -194,9 +194,11 @@ __global__ void __launch_bounds__(kThreads)
       const int row = id * kPage;
       mbar_arrive_expect_tx(bar, L::kStageBytes);
 #pragma unroll
-      for (int b = 0; b < D / 64; ++b) tma_load_4d(dk + b * kBoxBytes, &kmap, bar, 0, b, kvh, row);
+      for (int b = 0; b < L::kBoxesPerRow; ++b)
+        tma_load_4d(dk + b * kBoxBytes, &kmap, bar, 0, b, kvh, row);
 #pragma unroll
-      for (int b = 0; b < D / 64; ++b) tma_load_4d(dv + b * kBoxBytes, &vmap, bar, 0, b, kvh, row);
+      for (int b = 0; b < L::kBoxesPerRow; ++b)
+        tma_load_4d(dv + b * kBoxBytes, &vmap, bar, 0, b, kvh, row);
     }
   };
   const int pre = my_count < NST ? my_count : NST;

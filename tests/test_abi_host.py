@@ -139,3 +139,37 @@ def test_shared_prefix_validation(lib):
     b[7] = FAKE + 2
     assert f(*b, *sizes) == ALIGN                                 # prefix_blocks
     assert f(*base, 2, 4, 64, 2, 128, 64, 16, 8, 0, None) == UNSUP  # 32 query heads per KV head
+
+
+@host_only
+def test_copy_blocks_validation(lib):
+    f = lib.pa_copy_blocks
+    assert f(FAKE, FAKE, FAKE, 0, 64, 16, 2, 128, 2, None) == OK        # no pairs
+    assert f(FAKE, FAKE, FAKE, 3, 64, 16, 2, 128, 4, None) == SHAPE     # element size
+    assert f(None, FAKE, FAKE, 3, 64, 16, 2, 128, 2, None) == NULL
+    assert f(FAKE + 8, FAKE, FAKE, 3, 64, 16, 2, 128, 2, None) == ALIGN
+    assert f(FAKE, FAKE, FAKE + 4, 3, 64, 16, 2, 128, 2, None) == ALIGN
+    assert f(FAKE, FAKE, FAKE, 3, 64, 1, 1, 4, 2, None) == ALIGN        # 8-byte blocks
+
+
+@host_only
+def test_fp8_validation(lib):
+    f = lib.pa_decode_fp8
+    base = [FAKE] * 6 + [0.1]
+    ok_sizes = [4, 8, 2, 128, 64, 16, 8, 0, None]
+    assert f(*base, 0.0, 1.0, *ok_sizes) == SHAPE                     # k_scale must be > 0
+    assert f(*base, 1.0, float("inf"), *ok_sizes) == SHAPE
+    assert f(*base, 1.0, 1.0, 4, 8, 2, 64, 64, 16, 8, 0, None) == UNSUP   # head_dim 64
+    assert f(*base, 1.0, 1.0, 0, 8, 2, 128, 64, 16, 8, 0, None) == OK     # empty batch
+    w = lib.pa_reshape_and_cache_fp8
+    good = [FAKE, FAKE, 256, 256, FAKE, FAKE, FAKE, 4, 2, 128, 64, 16, 0.5, 0.5, 0, None]
+    bad = list(good)
+    bad[12] = -1.0
+    assert w(*bad) == SHAPE
+    bad = list(good)
+    bad[9] = 72                                                        # not a multiple of 16
+    bad[2] = bad[3] = 144
+    assert w(*bad) == ALIGN
+    bad = list(good)
+    bad[7] = 0
+    assert w(*bad) == OK

@@ -1,0 +1,144 @@
+"""E4M3 (fp8) KV cache on the GPU vs the fp64 oracle (GPU).
+
+The fp8 caches start from seeded N(0,1) values quantised by torch's own
+float8_e4m3fn cast (x * 64, so the codes span the E4M3 range, scale 1/64);
+the step's new rows are written by pa_reshape_and_cache_fp8 and compared bit
+for bit with the oracle's quantising write, then decode is compared with the
+oracle's fp8 decode (same tolerances as the 16-bit path, which they inherit
+from the 16-bit query and output)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as oracle_mod
+from paged_kv_cache_444_b200 import (SplitWorkspace, pa_check_error, pa_decode_fp8,
+                                     pa_decode_split_fp8, pa_reduce, pa_reshape_and_cache_fp8,
+                                     workloads)
+from parity_helpers import TOL, bits, ocode, to_f64
+
+pytestmark = pytest.mark.gpu
+
+K_SCALE, V_SCALE = 1.0 / 64, 1.0 / 32
+C = workloads.CONFIGS
+CASES = {
+    "mha_f16": C["mha_llama2_7b"].scaled(num_seqs=5, num_heads=4, num_kv_heads=4, num_blocks=256,
+                                         ctx=("uniform", 1, 500), seed=51),
+    "gqa_bf16": C["gqa_llama3_8b"].scaled(num_seqs=6, num_blocks=400, ctx=("uniform", 1, 700),
+                                          seed=52),
+    "gqa_f16": C["shared_prefix_beam"].scaled(num_seqs=4, num_blocks=300, shared_prefix_blocks=0,
+                                              share_group=1, ctx=("uniform", 1, 600), seed=53),
+    "gqa16_bf16": C["gqa_llama3_8b"].scaled(num_seqs=3, num_heads=32, num_kv_heads=2,
+                                            num_blocks=200, ctx=("uniform", 30, 900), seed=54),
+    "ragged_bf16": C["gqa_llama3_8b"].scaled(num_seqs=8, num_blocks=100,
+                                             ctx=("fixed", (0, 1, 15, 16, 17, 31, 32, 33)),
+                                             seed=55),
+}
+
+
+def _fp8_batch(cfg, dev):
+    b = workloads.make_batch(cfg, dev)
+    q8 = lambda t, s: (t.float() * (1.0 / s)).clamp(-448, 448).to(torch.float8_e4m3fn) \
+        .view(torch.uint8)
+    kc = q8(b.key_cache, K_SCALE).contiguous()
+    vc = q8(b.value_cache, V_SCALE).contiguous()
+    return b, kc, vc
+
+
+def _oracle(orc, b, kc, vc):
+    cfg = b.cfg
+    kh = kc.cpu().numpy().copy()
+    vh = vc.cpu().numpy().copy()
+    assert orc.reshape_and_cache_fp8(bits(b.key), bits(b.value), kh, vh,
+                                     b.slot_mapping.cpu().numpy(), cfg.num_blocks,
+                                     cfg.block_size, K_SCALE, V_SCALE, ocode(cfg)) == 0
+    ref = orc.decode_fp8(bits(b.query), kh, vh, b.block_tables.cpu().numpy(),
+                         b.context_lens.cpu().numpy(), cfg.scale, K_SCALE, V_SCALE, ocode(cfg))
+    return ref, kh, vh
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_fp8_write_and_decode_match_oracle(name, cuda_device, oracle_lib):
+    cfg = CASES[name]
+    b, kc, vc = _fp8_batch(cfg, cuda_device)
+    ref, kh, vh = _oracle(oracle_lib, b, kc, vc)
+    pa_reshape_and_cache_fp8(b.key, b.value, kc, vc, b.slot_mapping, K_SCALE, V_SCALE)
+    out = torch.full_like(b.query, float("nan"))
+    pa_decode_fp8(out, b.query, kc, vc, b.block_tables, b.context_lens, cfg.scale, K_SCALE,
+                  V_SCALE)
+    torch.cuda.synchronize()
+    pa_check_error()
+    assert np.array_equal(kc.cpu().numpy(), kh) and np.array_equal(vc.cpu().numpy(), vh)
+    g = to_f64(out)
+    assert np.isfinite(g).all()
+    err = np.max(np.abs(g - ref))
+    assert err <= TOL[cfg.dtype], f"{name}: {err:.3e}"
+
+
+@pytest.mark.parametrize("name", ["gqa_bf16", "mha_f16"])
+@pytest.mark.parametrize("ps", [16, 256])
+def test_fp8_split_matches_oracle(name, ps, cuda_device, oracle_lib):
+    cfg = CASES[name]
+    b, kc, vc = _fp8_batch(cfg, cuda_device)
+    ref, _, _ = _oracle(oracle_lib, b, kc, vc)
+    pa_reshape_and_cache_fp8(b.key, b.value, kc, vc, b.slot_mapping, K_SCALE, V_SCALE)
+    P = (b.block_tables.shape[1] * 16 + ps - 1) // ps
+    ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, cuda_device)
+    out = torch.full_like(b.query, float("nan"))
+    pa_decode_split_fp8(ws.tmp_out, ws.max_logits, ws.exp_sums, b.query, kc, vc, b.block_tables,
+                        b.context_lens, cfg.scale, K_SCALE, V_SCALE, ps)
+    pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, b.context_lens, ps)
+    torch.cuda.synchronize()
+    pa_check_error()
+    err = np.max(np.abs(to_f64(out) - ref))
+    assert err <= TOL[cfg.dtype], f"{name} split {ps}: {err:.3e}"
+
+
+@pytest.mark.parametrize("name", ["mha_f16", "gqa_bf16"])
+def test_fp8_context_len_one_is_exact(name, cuda_device):
+    # p = 1, and code * 2^-5 is exact in fp32 and in the 16-bit output
+    cfg = CASES[name]
+    b, kc, vc = _fp8_batch(cfg, cuda_device)
+    b.context_lens.fill_(1)
+    out = torch.empty_like(b.query)
+    pa_decode_fp8(out, b.query, kc, vc, b.block_tables, b.context_lens, cfg.scale, K_SCALE,
+                  V_SCALE)
+    torch.cuda.synchronize()
+    v0 = vc[b.block_tables[:, 0].long(), 0].view(torch.float8_e4m3fn).to(torch.float32) * V_SCALE
+    want = v0.to(b.query.dtype).repeat_interleave(cfg.group_size, dim=1)
+    assert torch.equal(out, want)
+
+
+def test_fp8_full_size_gqa_sampled(cuda_device, oracle_lib):
+    """The Llama-3-8B GQA batch at full size with an fp8 cache (half the
+    bytes of the bf16 one), checked on sampled sequences."""
+    cfg = C["gqa_llama3_8b"]
+    b, kc, vc = _fp8_batch(cfg, cuda_device)
+    seqs = [0, 37, 127]
+    # host snapshot of the sampled sequences' blocks before the write
+    bt = b.block_tables[seqs].cpu().numpy()
+    ctx = b.context_lens[seqs].cpu().numpy().astype(np.int32)
+    used = sorted({int(x) for i in range(len(seqs))
+                   for x in bt[i, :(int(ctx[i]) + 15) // 16]})
+    remap = {blk: n for n, blk in enumerate(used)}
+    bt_new = np.full_like(bt, -1)
+    for i in range(len(seqs)):
+        for j in range((int(ctx[i]) + 15) // 16):
+            bt_new[i, j] = remap[int(bt[i, j])]
+    ids = torch.tensor(used, dtype=torch.long, device=cuda_device)
+    kh = kc.index_select(0, ids).cpu().numpy().copy()
+    vh = vc.index_select(0, ids).cpu().numpy().copy()
+    slots = b.slot_mapping[seqs].cpu().numpy()
+    slots = np.array([remap[int(x) // 16] * 16 + int(x) % 16 for x in slots], dtype=np.int64)
+    assert oracle_lib.reshape_and_cache_fp8(bits(b.key[seqs]), bits(b.value[seqs]), kh, vh, slots,
+                                            len(used), 16, K_SCALE, V_SCALE, oracle_mod.BF16) == 0
+    ref = oracle_lib.decode_fp8(bits(b.query[seqs]), kh, vh, bt_new, ctx, cfg.scale, K_SCALE,
+                                V_SCALE, oracle_mod.BF16)
+    pa_reshape_and_cache_fp8(b.key, b.value, kc, vc, b.slot_mapping, K_SCALE, V_SCALE)
+    out = torch.empty_like(b.query)
+    pa_decode_fp8(out, b.query, kc, vc, b.block_tables, b.context_lens, cfg.scale, K_SCALE,
+                  V_SCALE)
+    torch.cuda.synchronize()
+    pa_check_error()
+    assert np.array_equal(kc.index_select(0, ids).cpu().numpy(), kh)
+    err = np.max(np.abs(to_f64(out[seqs]) - ref))
+    assert err <= TOL["bf16"], err

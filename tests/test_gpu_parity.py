@@ -304,6 +304,29 @@ def test_shared_prefix_reports_bad_groups(dev):
     pa_check_error()
 
 
+@pytest.mark.parametrize("name", ["gqa_small", "tiny"])
+def test_copy_blocks_bit_exact(name, dev, oracle_lib):
+    cfg = SMALL[name]
+    batch = workloads.make_batch(cfg, dev)
+    g = torch.Generator().manual_seed(7)
+    perm = torch.randperm(cfg.num_blocks, generator=g)
+    pairs = torch.stack([perm[:20], perm[20:40]], dim=1).contiguous()  # distinct, disjoint
+    kc, vc = bits(batch.key_cache), bits(batch.value_cache)
+    assert oracle_lib.copy_blocks(kc, vc, pairs.numpy()) == 0
+    from paged_kv_cache_444_b200 import pa_copy_blocks
+    pa_copy_blocks(batch.key_cache, batch.value_cache, pairs.to(dev))
+    torch.cuda.synchronize()
+    pa_check_error()
+    assert np.array_equal(bits(batch.key_cache), kc)
+    assert np.array_equal(bits(batch.value_cache), vc)
+    # an id past the pool is skipped and reported with its pair index
+    bad = torch.tensor([[0, 1], [2, cfg.num_blocks]], dtype=torch.int64, device=dev)
+    pa_copy_blocks(batch.key_cache, batch.value_cache, bad)
+    with pytest.raises(PagedAttentionError) as e:
+        pa_check_error()
+    assert e.value.detail >> 56 == 2 and e.value.detail & 0xffff == 1
+
+
 def test_write_padding_and_strided_rows(dev, oracle_lib):
     cfg = SMALL["gqa_small"]
     batch = workloads.make_batch(cfg, dev)
