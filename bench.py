@@ -256,6 +256,34 @@ def shared_prefix_kernel_ms(batch, warmup: int, reps: int = 100) -> float:
     return start.elapsed_time(end) / reps
 
 
+def fp8_decode_ms(batch, warmup: int, reps: int = 100) -> float | None:
+    """CUDA-event time of pa_decode_fp8 on the same batch with its caches held
+    as E4M3 codes (x * 64 quantised by torch, scale 1/64); None where the
+    fp8 path is not built (head_dim != 128) or the batch uses the split path."""
+    from paged_kv_cache_444_b200 import pa_decode_fp8
+    cfg = batch.cfg
+    if cfg.head_dim != 128 or cfg.partition_size:
+        return None
+    q8 = lambda t: (t.float() * 64.0).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    kc, vc = q8(batch.key_cache), q8(batch.value_cache)
+    out = torch.empty_like(batch.query)
+
+    def run():
+        pa_decode_fp8(out, batch.query, kc, vc, batch.block_tables, batch.context_lens,
+                      cfg.scale, 1.0 / 64, 1.0 / 64)
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(reps):
+        run()
+    end.record()
+    torch.cuda.synchronize()
+    del kc, vc
+    return start.elapsed_time(end) / reps
+
+
 def graph_steps(step: Step, steps: int, warmup: int) -> float | None:
     """The same step captured once in a CUDA graph and replayed `steps` times
     (ms per step), or None if capture is not possible here."""
@@ -294,37 +322,27 @@ class _Null:
 
 
 def e2e_steps(step: Step, steps: int, warmup: int, world: int, device):
-    """Same step through the public API with this step's inputs copied in
-    from pinned host memory and the output read back, all inside the timing."""
-    from paged_kv_cache_444_b200 import decode_step
+    """The same step through the C ABI from host buffers (pa_decode_step_host):
+    every step copies its inputs in from pinned host memory, writes the cache,
+    attends, and copies the output back, all inside the timing."""
+    from paged_kv_cache_444_b200 import HostStep
     b, cfg = step.b, step.cfg
-    host = {n: getattr(b, n).cpu().pin_memory() for n in
-            ("query", "key", "value", "slot_mapping", "block_tables", "context_lens")}
-    dev = {n: torch.empty_like(getattr(b, n)) for n in host}
-    out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_host.numel() * out_host.element_size()
-
-    def one():
-        for n, t in host.items():
-            dev[n].copy_(t, non_blocking=True)
-        decode_step(dev["query"], dev["key"], dev["value"], b.key_cache, b.value_cache,
-                    dev["slot_mapping"], dev["block_tables"], dev["context_lens"], cfg.scale,
-                    out=step.out, partition_size=step.ps, workspace=step.ws)
-        out_host.copy_(step.out, non_blocking=True)
-
+    hs = HostStep(b.key_cache, b.value_cache, cfg.num_seqs, cfg.num_heads,
+                  b.block_tables.shape[1], cfg.scale, step.ps, cfg.torch_dtype)
+    for n in ("query", "key", "value", "slot_mapping", "block_tables", "context_lens"):
+        getattr(hs, n).copy_(getattr(b, n).cpu())
     for _ in range(warmup):
-        one()
+        hs.run()
     torch.cuda.synchronize()
     barrier(world, device)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
     for _ in range(steps):
-        one()
+        hs.run()
     end.record()
     torch.cuda.synchronize()
     barrier(world, device)
-    return start.elapsed_time(end) / steps, h2d, d2h
+    return start.elapsed_time(end) / steps, hs.h2d_bytes, hs.d2h_bytes
 
 
 # ---------------------------------------------------------------------------
@@ -464,6 +482,7 @@ def run_native(args, world, rank, local):
         gms = graph_steps(step, steps, warmup) if args.graph else None
         shared_ms = shared_prefix_kernel_ms(batch, warmup) if batch.group_starts is not None \
             else None
+        f8_ms = fp8_decode_ms(batch, warmup) if args.fp8 else None
         ctx = batch.context_lens.cpu().tolist()
         by = workloads.algorithmic_bytes(cfg, ctx)
         attn_ms = per_kernel[1] + (per_kernel[2] if step.ps else 0.0)
@@ -482,6 +501,7 @@ def run_native(args, world, rank, local):
             "tokens_per_s": sum_over_ranks(cfg.num_seqs, world, device) / (ms_max / 1e3),
             "graph_ms_per_step": gms,
             "shared_prefix_kernel_ms": shared_ms,
+            "fp8_ms": f8_ms,
             "kernel": "pa_decode_split" if step.ps else "pa_decode",
             "context_tokens": int(sum(ctx)),
         }
@@ -547,7 +567,7 @@ def run_native(args, world, rank, local):
         "e2e": {"value": round(total_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "api": "paged_kv_cache_444_b200.decode_step with pinned host inputs"},
+                "api": "pa_decode_step_host (C ABI, pinned host buffers in and out)"},
         "clocks": clocks.summary(),
     }
     if results:
@@ -564,7 +584,8 @@ def run_native(args, world, rank, local):
                                       if r["graph_ms_per_step"] else None),
                 "per_kernel_ms": [round(x, 5) for x in r["per_kernel_ms"]],
                 **({"pa_decode_shared_prefix_ms": round(r["shared_prefix_kernel_ms"], 5)}
-                   if r["shared_prefix_kernel_ms"] else {})}
+                   if r["shared_prefix_kernel_ms"] else {}),
+                **(fp8_entry(r, peak) if r["fp8_ms"] else {})}
             for n, r in results.items()}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, ctx_main, bt_main, batch,
@@ -574,6 +595,18 @@ def run_native(args, world, rank, local):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def fp8_entry(r: dict, peak: float) -> dict:
+    """pa_decode_fp8 on the same batch: time, algorithmic GB/s (K/V at one
+    byte per element) and the speed-up over the 16-bit decode kernel."""
+    by = r["bytes"]
+    fp8_bytes = by["kv"] // 2 + by["block_table"] + by["query"] + by["out"] + by["context_lens"]
+    gbs = fp8_bytes / (r["fp8_ms"] / 1e3) / 1e9
+    return {"pa_decode_fp8": {"ms": round(r["fp8_ms"], 5), "gbs": round(gbs, 1),
+                              "frac_of_peak": round(gbs / peak, 4),
+                              "speedup_vs_16bit_kernel": round(r["per_kernel_ms"][1] /
+                                                               r["fp8_ms"], 3)}}
 
 
 def recorded_traffic(config: str, kernel: str, context_tokens: int):
@@ -666,6 +699,8 @@ def main(argv=None):
                     help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="also time the step replayed from a CUDA graph")
+    ap.add_argument("--fp8", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time pa_decode_fp8 on each batch (E4M3 copy of its caches)")
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="override the workload's batch size (small profiling captures)")
     ap.add_argument("--num-blocks", type=int, default=0,

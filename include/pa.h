@@ -248,6 +248,40 @@ pa_status pa_decode_split_fp8(float *tmp_out, float *max_logits, float *exp_sums
                               pa_dtype dtype, void *stream);
 
 /*
+ * pa_decode_step_host -- one whole decode step of one attention layer for a
+ * caller whose per-step inputs are in HOST memory (pinned memory makes the
+ * copies asynchronous; pageable memory works but the copies then block).
+ * Enqueues on `stream`: host->device copies of query [S,H,D], key and value
+ * [S,Hk,D] (one new token per sequence), slot_mapping [S] int64,
+ * block_tables [S,MB] int32 and context_lens [S] int32 into `workspace`; the
+ * cache write (pa_reshape_and_cache); attention (pa_decode, or
+ * pa_decode_split + pa_reduce when partition_size > 0); and the copy of the
+ * output [S,H,D] back to out_host.  Returns without waiting: out_host is
+ * valid once the stream has reached this point.
+ *   key_cache, value_cache   device caches as for pa_decode (stay resident)
+ *   workspace                caller-owned device memory, 256-byte aligned, of
+ *                            pa_decode_step_host_workspace_bytes(...) bytes
+ * If the six host inputs sit in one host buffer at the same offsets as in
+ * the workspace (each part in the order above, starting 256-byte aligned
+ * after the previous one), they are copied with a single transfer.
+ * Errors as for the calls it makes; PA_ERR_SHAPE if the workspace is small.
+ */
+int64_t pa_decode_step_host_workspace_bytes(int64_t num_seqs, int64_t num_heads,
+                                            int64_t num_kv_heads, int64_t head_dim,
+                                            int64_t max_blocks_per_seq, int64_t block_size,
+                                            int64_t partition_size);
+
+pa_status pa_decode_step_host(void *out_host, const void *query_host, const void *key_host,
+                              const void *value_host, const int64_t *slot_mapping_host,
+                              const int32_t *block_tables_host,
+                              const int32_t *context_lens_host, void *key_cache,
+                              void *value_cache, void *workspace, int64_t workspace_bytes,
+                              float scale, int64_t num_seqs, int64_t num_heads,
+                              int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                              int64_t block_size, int64_t max_blocks_per_seq,
+                              int64_t partition_size, pa_dtype dtype, void *stream);
+
+/*
  * pa_check_error -- synchronise `stream`, read and clear the current device's
  * error word.  Returns PA_OK if no kernel recorded a problem since the last
  * call, PA_ERR_BOUNDS otherwise (then *detail, if not NULL, receives

@@ -67,6 +67,8 @@ SIGNATURES = {
                            _i64, _i64, _i, _p]),
     "pa_decode_split_fp8": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _f, _f, _f, _i64, _i64, _i64,
                                  _i64, _i64, _i64, _i64, _i64, _i64, _i, _p]),
+    "pa_decode_step_host_workspace_bytes": (_i64, [_i64] * 7),
+    "pa_decode_step_host": (_i, [_p] * 10 + [_i64, _f] + [_i64] * 8 + [_i, _p]),
 }
 
 _lib: ctypes.CDLL | None = None
@@ -96,6 +98,25 @@ def header_functions() -> list[str]:
     text = HEADER.read_text(encoding="utf-8")
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+def header_signatures() -> dict[str, list[str]]:
+    """Parameter type of every function include/pa.h declares, as C text
+    (pointers collapse to 'ptr')."""
+    text = HEADER.read_text(encoding="utf-8")
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(?:pa_status|int64_t|int32_t|const char\s*\*)\s*(pa_[a-z0-9_]+)"
+                         r"\s*\(([^)]*)\)\s*;", text):
+        params = [p.strip() for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+        kinds = []
+        for p_ in params:
+            if "*" in p_:
+                kinds.append("ptr")
+            else:
+                kinds.append(p_.rsplit(None, 1)[0].replace("const ", ""))
+        out[m.group(1)] = kinds
+    return out
 
 
 def status_string(status: int) -> str:
@@ -318,6 +339,61 @@ def pa_decode_split_fp8(tmp_out, max_logits, exp_sums, query, key_cache, value_c
                                     float(v_scale), S, H, Hk, D, NB, bs, MB, int(partition_size),
                                     P, dt, _stream(stream))
     _check(st, "pa_decode_split_fp8")
+
+
+class HostStep:
+    """pa_decode_step_host for one layer: per-step inputs live in (pinned)
+    host tensors, the caches and a device workspace stay resident.  `run()`
+    enqueues copies in, the cache write, attention and the copy out."""
+
+    def __init__(self, key_cache, value_cache, num_seqs, num_heads, max_blocks_per_seq,
+                 scale: float, partition_size: int = 0, dtype=torch.float16):
+        NB, bs, Hk, D = key_cache.shape
+        self.key_cache, self.value_cache = key_cache, value_cache
+        self.dims = (num_seqs, num_heads, Hk, D, NB, bs, max_blocks_per_seq)
+        self.scale, self.partition_size, self.dtype = float(scale), int(partition_size), dtype
+        n = load().pa_decode_step_host_workspace_bytes(num_seqs, num_heads, Hk, D,
+                                                       max_blocks_per_seq, bs, partition_size)
+        _need(n >= 0, "bad step sizes")
+        self.workspace = torch.empty(n, dtype=torch.uint8, device=key_cache.device)
+        # one pinned host buffer laid out like the workspace, so the six
+        # inputs travel in a single copy
+        S, H, D_ = num_seqs, num_heads, D
+        parts = [((S, H, D_), dtype), ((S, Hk, D_), dtype), ((S, Hk, D_), dtype),
+                 ((S,), torch.int64), ((S, max_blocks_per_seq), torch.int32), ((S,), torch.int32)]
+        offs, at = [], 0
+        for shape, dt in parts:
+            offs.append(at)
+            nbytes = int(torch.Size(shape).numel()) * torch.tensor([], dtype=dt).element_size()
+            at = (at + nbytes + 255) // 256 * 256
+        self.staging = torch.empty(at, dtype=torch.uint8).pin_memory()
+        views = []
+        for (shape, dt), o in zip(parts, offs):
+            nbytes = int(torch.Size(shape).numel()) * torch.tensor([], dtype=dt).element_size()
+            views.append(self.staging[o:o + nbytes].view(dt).view(shape))
+        (self.query, self.key, self.value, self.slot_mapping, self.block_tables,
+         self.context_lens) = views
+        self.out = torch.empty((S, H, D_), dtype=dtype).pin_memory()
+
+    @property
+    def h2d_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in
+                   (self.query, self.key, self.value, self.slot_mapping, self.block_tables,
+                    self.context_lens))
+
+    @property
+    def d2h_bytes(self) -> int:
+        return self.out.numel() * self.out.element_size()
+
+    def run(self, stream=None) -> None:
+        S, H, Hk, D, NB, bs, MB = self.dims
+        st = load().pa_decode_step_host(
+            self.out.data_ptr(), self.query.data_ptr(), self.key.data_ptr(),
+            self.value.data_ptr(), self.slot_mapping.data_ptr(), self.block_tables.data_ptr(),
+            self.context_lens.data_ptr(), self.key_cache.data_ptr(), self.value_cache.data_ptr(),
+            self.workspace.data_ptr(), self.workspace.numel(), self.scale, S, H, Hk, D, NB, bs,
+            MB, self.partition_size, DTYPE_CODES[self.dtype], _stream(stream))
+        _check(st, "pa_decode_step_host")
 
 
 def pa_check_error(stream=None) -> int:

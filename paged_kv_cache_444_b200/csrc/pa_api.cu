@@ -646,6 +646,130 @@ pa_status pa_decode_split_fp8(float* tmp_out, float* max_logits, float* exp_sums
                         as_stream(stream));
 }
 
+// ---------------------------------------------------------------------------
+// One decode step from host buffers.  Workspace layout (each part 256-byte
+// aligned): query, key, value, slot_mapping, block_tables, context_lens, out,
+// then for the split path tmp_out, max_logits, exp_sums.
+// ---------------------------------------------------------------------------
+namespace {
+struct StepLayout {
+  int64_t off[10];
+  int64_t total;
+};
+
+int64_t align256(int64_t x) { return (x + 255) & ~static_cast<int64_t>(255); }
+
+StepLayout step_layout(int64_t S, int64_t H, int64_t Hk, int64_t D, int64_t MB, int64_t bs,
+                       int64_t partition_size) {
+  const int64_t parts = partition_size > 0 ? (MB * bs + partition_size - 1) / partition_size : 0;
+  const int64_t sizes[10] = {S * H * D * 2, S * Hk * D * 2, S * Hk * D * 2, S * 8, S * MB * 4,
+                             S * 4, S * H * D * 2, S * H * parts * D * 4, S * H * parts * 4,
+                             S * H * parts * 4};
+  StepLayout l{};
+  int64_t at = 0;
+  for (int i = 0; i < 10; ++i) {
+    l.off[i] = at;
+    at = align256(at + sizes[i]);
+  }
+  l.total = at;
+  return l;
+}
+}  // namespace
+
+int64_t pa_decode_step_host_workspace_bytes(int64_t num_seqs, int64_t num_heads,
+                                            int64_t num_kv_heads, int64_t head_dim,
+                                            int64_t max_blocks_per_seq, int64_t block_size,
+                                            int64_t partition_size) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      max_blocks_per_seq <= 0 || block_size <= 0 || partition_size < 0)
+    return -1;
+  return step_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                     block_size, partition_size)
+      .total;
+}
+
+pa_status pa_decode_step_host(void* out_host, const void* query_host, const void* key_host,
+                              const void* value_host, const int64_t* slot_mapping_host,
+                              const int32_t* block_tables_host,
+                              const int32_t* context_lens_host, void* key_cache,
+                              void* value_cache, void* workspace, int64_t workspace_bytes,
+                              float scale, int64_t num_seqs, int64_t num_heads,
+                              int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                              int64_t block_size, int64_t max_blocks_per_seq,
+                              int64_t partition_size, pa_dtype dtype, void* stream) {
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_DTYPE;
+  if (num_seqs < 0 || partition_size < 0) return PA_ERR_SHAPE;
+  if (num_seqs == 0) return PA_OK;
+  if (!out_host || !query_host || !key_host || !value_host || !slot_mapping_host ||
+      !block_tables_host || !context_lens_host || !key_cache || !value_cache || !workspace)
+    return PA_ERR_NULL;
+  const int64_t need = pa_decode_step_host_workspace_bytes(num_seqs, num_heads, num_kv_heads,
+                                                           head_dim, max_blocks_per_seq,
+                                                           block_size, partition_size);
+  if (need < 0) return PA_ERR_SHAPE;
+  if (workspace_bytes < need) return PA_ERR_SHAPE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PA_ERR_ALIGN;
+  const StepLayout l = step_layout(num_seqs, num_heads, num_kv_heads, head_dim,
+                                   max_blocks_per_seq, block_size, partition_size);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  void* d_query = w + l.off[0];
+  void* d_key = w + l.off[1];
+  void* d_value = w + l.off[2];
+  int64_t* d_slots = reinterpret_cast<int64_t*>(w + l.off[3]);
+  int32_t* d_tables = reinterpret_cast<int32_t*>(w + l.off[4]);
+  int32_t* d_lens = reinterpret_cast<int32_t*>(w + l.off[5]);
+  void* d_out = w + l.off[6];
+  cudaStream_t s = as_stream(stream);
+  const int64_t q_bytes = num_seqs * num_heads * head_dim * 2;
+  const int64_t kv_bytes = num_seqs * num_kv_heads * head_dim * 2;
+  struct Copy { void* dst; const void* src; int64_t bytes; };
+  const Copy ins[6] = {{d_query, query_host, q_bytes}, {d_key, key_host, kv_bytes},
+                       {d_value, value_host, kv_bytes}, {d_slots, slot_mapping_host, num_seqs * 8},
+                       {d_tables, block_tables_host, num_seqs * max_blocks_per_seq * 4},
+                       {d_lens, context_lens_host, num_seqs * 4}};
+  // Inputs laid out in host memory exactly as in the workspace (one pinned
+  // buffer with the same offsets) go over in one copy; otherwise one each.
+  const uint8_t* hbase = static_cast<const uint8_t*>(query_host);
+  bool packed = true;
+  for (int i = 1; i < 6; ++i) packed = packed && ins[i].src == hbase + l.off[i];
+  if (packed) {
+    if (cudaMemcpyAsync(w, hbase, static_cast<size_t>(l.off[5] + num_seqs * 4),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return PA_ERR_CUDA;
+  } else {
+    for (const Copy& c : ins)
+      if (cudaMemcpyAsync(c.dst, c.src, static_cast<size_t>(c.bytes), cudaMemcpyHostToDevice,
+                          s) != cudaSuccess)
+        return PA_ERR_CUDA;
+  }
+  pa_status st = pa_reshape_and_cache(d_key, d_value, num_kv_heads * head_dim,
+                                      num_kv_heads * head_dim, key_cache, value_cache, d_slots,
+                                      num_seqs, num_kv_heads, head_dim, num_blocks, block_size,
+                                      dtype, stream);
+  if (st != PA_OK) return st;
+  if (partition_size > 0) {
+    const int64_t parts = (max_blocks_per_seq * block_size + partition_size - 1) / partition_size;
+    float* tmp = reinterpret_cast<float*>(w + l.off[7]);
+    float* mx = reinterpret_cast<float*>(w + l.off[8]);
+    float* es = reinterpret_cast<float*>(w + l.off[9]);
+    st = pa_decode_split(tmp, mx, es, d_query, key_cache, value_cache, d_tables, d_lens, scale,
+                         num_seqs, num_heads, num_kv_heads, head_dim, num_blocks, block_size,
+                         max_blocks_per_seq, partition_size, parts, dtype, stream);
+    if (st != PA_OK) return st;
+    st = pa_reduce(d_out, tmp, mx, es, d_lens, num_seqs, num_heads, head_dim, partition_size,
+                   parts, dtype, stream);
+  } else {
+    st = pa_decode(d_out, d_query, key_cache, value_cache, d_tables, d_lens, scale, num_seqs,
+                   num_heads, num_kv_heads, head_dim, num_blocks, block_size, max_blocks_per_seq,
+                   dtype, stream);
+  }
+  if (st != PA_OK) return st;
+  if (cudaMemcpyAsync(out_host, d_out, static_cast<size_t>(q_bytes), cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  return PA_OK;
+}
+
 pa_status pa_check_error(void* stream, int64_t* detail) {
   cudaStream_t s = as_stream(stream);
   unsigned long long word = 0;

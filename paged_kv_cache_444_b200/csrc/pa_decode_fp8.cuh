@@ -9,7 +9,7 @@
 // the output, so the page steps below work on the raw codes:
 //  - SimtFp8Warp (one query head per KV head): codes -> fp16 -> fp32 with
 //    cvt.rn.f16x2.e4m3x2, then packed fp32 FMA as in the 16-bit path.
-//  - MmaFp8Warp (GQA group): the page is read with the same b16 ldmatrix as
+//  - MmaFp8Warp (GQA group, fp16 mma): the page is read with the same b16 ldmatrix as
 //    the 16-bit path, which hands each lane 4 consecutive codes of a row
 //    where the 16-bit fragment layout expects 2 + 2 codes 8 apart.  Inside
 //    one 16-element k-step that is a fixed permutation of the head dims, so
@@ -136,19 +136,40 @@ struct SimtFp8Warp {
 };
 
 // ---------------------------------------------------------------------------
-// Tensor-core path (GQA groups of 2..16), head_dim 128
+// Tensor-core path (GQA groups of 2..16), head_dim 128.
+//
+// Both products run as fp16 mma whatever the query dtype: E4M3 -> fp16 is one
+// exact conversion, and P in fp16 keeps 11 bits.  A bf16 (or fp16) query row
+// is brought into fp16 range exactly by a power of two 2^s chosen from its
+// largest element (that element lands in [2^13, 2^14)); 2^-s is folded into
+// the row's logit scale.  Only elements more than 2^27 below the row's
+// largest can lose bits, and they cannot move a logit.
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool TWO_ROWS>
 struct MmaFp8Warp {
   static_assert(D == 128, "fp8 tensor-core path is built for head_dim 128");
   static constexpr int KSTEPS = D / 16;
   static constexpr int NTILES = D / 8;
-  uint32_t qa[KSTEPS][4];   // Q fragments, head dims permuted as the fp8 K fragments
+  uint32_t qa[KSTEPS][4];   // fp16 Q fragments, head dims permuted as the fp8 K fragments
   float acc[NTILES][4];     // n-tile 2c: even dims of 16-dim chunk c; 2c+1: odd dims
   float m[2], l[2];
+  float rs[2];              // 2^-s of rows r0, r1 (undo the query prescale)
+
+  __device__ __forceinline__ static float pow2(int e) {
+    return __int_as_float((e + 127) << 23);  // e in [-126, 127]
+  }
+
+  // 2^s that brings a row whose largest |element| is mx into [2^13, 2^14)
+  __device__ __forceinline__ static int prescale_exp(float mx) {
+    if (!(mx > 0.f)) return 0;
+    const int e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 127;  // floor(log2 mx)
+    return max(-100, min(100, 13 - e));
+  }
 
   __device__ __forceinline__ void init(const uint16_t* q_group, int group, int lane) {
     const int r0 = lane >> 2, r1 = r0 + 8, tig = lane & 3;
+    float2 v0[KSTEPS][2], v1[KSTEPS][2];
+    float mx0 = 0.f, mx1 = 0.f;
 #pragma unroll
     for (int kk = 0; kk < KSTEPS; ++kk) {
       // k positions tig*2+{0,1} hold dims 4*tig+{0,1}; positions tig*2+8+{0,1}
@@ -156,10 +177,30 @@ struct MmaFp8Warp {
       const int d0 = kk * 16 + tig * 4;
       const uint32_t* q0 = reinterpret_cast<const uint32_t*>(q_group + r0 * D);
       const uint32_t* q1 = reinterpret_cast<const uint32_t*>(q_group + r1 * D);
-      qa[kk][0] = r0 < group ? q0[d0 >> 1] : 0u;
-      qa[kk][1] = (TWO_ROWS && r1 < group) ? q1[d0 >> 1] : 0u;
-      qa[kk][2] = r0 < group ? q0[(d0 >> 1) + 1] : 0u;
-      qa[kk][3] = (TWO_ROWS && r1 < group) ? q1[(d0 >> 1) + 1] : 0u;
+      v0[kk][0] = unpack2<BF16>(r0 < group ? q0[d0 >> 1] : 0u);
+      v0[kk][1] = unpack2<BF16>(r0 < group ? q0[(d0 >> 1) + 1] : 0u);
+      v1[kk][0] = unpack2<BF16>((TWO_ROWS && r1 < group) ? q1[d0 >> 1] : 0u);
+      v1[kk][1] = unpack2<BF16>((TWO_ROWS && r1 < group) ? q1[(d0 >> 1) + 1] : 0u);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        mx0 = fmaxf(mx0, fmaxf(fabsf(v0[kk][h].x), fabsf(v0[kk][h].y)));
+        mx1 = fmaxf(mx1, fmaxf(fabsf(v1[kk][h].x), fabsf(v1[kk][h].y)));
+      }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const int s0 = prescale_exp(mx0), s1 = prescale_exp(mx1);
+    const float f0 = pow2(s0), f1 = pow2(s1);
+    rs[0] = pow2(-s0);
+    rs[1] = pow2(-s1);
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      qa[kk][0] = pack2<false>(v0[kk][0].x * f0, v0[kk][0].y * f0);
+      qa[kk][2] = pack2<false>(v0[kk][1].x * f0, v0[kk][1].y * f0);
+      qa[kk][1] = pack2<false>(v1[kk][0].x * f1, v1[kk][0].y * f1);
+      qa[kk][3] = pack2<false>(v1[kk][1].x * f1, v1[kk][1].y * f1);
     }
 #pragma unroll
     for (int n = 0; n < NTILES; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
@@ -181,21 +222,20 @@ struct MmaFp8Warp {
       const int c = 2 * kp + mchk;
       uint32_t r0, r1, r2, r3;  // (tok 0-7, chunk 2kp) (8-15, 2kp) (0-7, 2kp+1) (8-15, 2kp+1)
       ldsm_x4(kbase + mtok * 128 + ((c ^ (mtok & 7)) << 4), r0, r1, r2, r3);
-      mma_16816<BF16>(sc[0], qa[2 * kp], e4m3x2_to_op2<BF16>(r0), e4m3x2_to_op2<BF16>(r0 >> 16));
-      mma_16816<BF16>(sc[1], qa[2 * kp], e4m3x2_to_op2<BF16>(r1), e4m3x2_to_op2<BF16>(r1 >> 16));
-      mma_16816<BF16>(sc[0], qa[2 * kp + 1], e4m3x2_to_op2<BF16>(r2),
-                      e4m3x2_to_op2<BF16>(r2 >> 16));
-      mma_16816<BF16>(sc[1], qa[2 * kp + 1], e4m3x2_to_op2<BF16>(r3),
-                      e4m3x2_to_op2<BF16>(r3 >> 16));
+      mma_16816<false>(sc[0], qa[2 * kp], e4m3x2_to_h2(r0), e4m3x2_to_h2(r0 >> 16));
+      mma_16816<false>(sc[1], qa[2 * kp], e4m3x2_to_h2(r1), e4m3x2_to_h2(r1 >> 16));
+      mma_16816<false>(sc[0], qa[2 * kp + 1], e4m3x2_to_h2(r2), e4m3x2_to_h2(r2 >> 16));
+      mma_16816<false>(sc[1], qa[2 * kp + 1], e4m3x2_to_h2(r3), e4m3x2_to_h2(r3 >> 16));
     }
-    // ---- scale, mask, online softmax (as in the 16-bit path) ----
+    // ---- scale (with each row's 2^-s), mask, online softmax ----
+    const float sl0 = scale_log2 * rs[0], sl1 = scale_log2 * rs[1];
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int t = tok0 + nt * 8 + tig * 2 + (i & 1);
-        const float x = t < t_end ? sc[nt][i] * scale_log2 : -INFINITY;
+        const float x = t < t_end ? sc[nt][i] * (i < 2 ? sl0 : sl1) : -INFINITY;
         sc[nt][i] = x;
         if (i < 2) mx0 = fmaxf(mx0, x); else mx1 = fmaxf(mx1, x);
       }
@@ -213,40 +253,21 @@ struct MmaFp8Warp {
       al1 = ex2(m[1] - mn1);
       m[1] = mn1;
     }
-    float p0[4], p1[4];
-    p0[0] = ex2(sc[0][0] - mn0); p0[1] = ex2(sc[0][1] - mn0);
-    p0[2] = ex2(sc[1][0] - mn0); p0[3] = ex2(sc[1][1] - mn0);
-    if constexpr (TWO_ROWS) {
-      p1[0] = ex2(sc[0][2] - mn1); p1[1] = ex2(sc[0][3] - mn1);
-      p1[2] = ex2(sc[1][2] - mn1); p1[3] = ex2(sc[1][3] - mn1);
-    } else {
-      p1[0] = p1[1] = p1[2] = p1[3] = 0.f;
-    }
-    uint32_t pa[4], pl[4];
-    pa[0] = pack2<BF16>(p0[0], p0[1]);
-    pa[2] = pack2<BF16>(p0[2], p0[3]);
-    pa[1] = TWO_ROWS ? pack2<BF16>(p1[0], p1[1]) : 0u;
-    pa[3] = TWO_ROWS ? pack2<BF16>(p1[2], p1[3]) : 0u;
-    if constexpr (BF16) {
-      const float2 h0 = unpack2<BF16>(pa[0]), h2 = unpack2<BF16>(pa[2]);
-      pl[0] = pack2<BF16>(p0[0] - h0.x, p0[1] - h0.y);
-      pl[2] = pack2<BF16>(p0[2] - h2.x, p0[3] - h2.y);
-      if constexpr (TWO_ROWS) {
-        const float2 h1 = unpack2<BF16>(pa[1]), h3 = unpack2<BF16>(pa[3]);
-        pl[1] = pack2<BF16>(p1[0] - h1.x, p1[1] - h1.y);
-        pl[3] = pack2<BF16>(p1[2] - h3.x, p1[3] - h3.y);
-      } else {
-        pl[1] = pl[3] = 0u;
-      }
-      l[0] = l[0] * al0 + ((p0[0] + p0[1]) + (p0[2] + p0[3]));
-      if constexpr (TWO_ROWS) l[1] = l[1] * al1 + ((p1[0] + p1[1]) + (p1[2] + p1[3]));
-    } else {
-      const float2 u = unpack2<BF16>(pa[0]), v = unpack2<BF16>(pa[2]);
+    // ---- P in fp16; l sums the same rounded values ----
+    uint32_t pa[4];
+    pa[0] = pack2<false>(ex2(sc[0][0] - mn0), ex2(sc[0][1] - mn0));
+    pa[2] = pack2<false>(ex2(sc[1][0] - mn0), ex2(sc[1][1] - mn0));
+    {
+      const float2 u = unpack2<false>(pa[0]), v = unpack2<false>(pa[2]);
       l[0] = l[0] * al0 + ((u.x + u.y) + (v.x + v.y));
-      if constexpr (TWO_ROWS) {
-        const float2 w = unpack2<BF16>(pa[1]), z = unpack2<BF16>(pa[3]);
-        l[1] = l[1] * al1 + ((w.x + w.y) + (z.x + z.y));
-      }
+    }
+    if constexpr (TWO_ROWS) {
+      pa[1] = pack2<false>(ex2(sc[0][2] - mn1), ex2(sc[0][3] - mn1));
+      pa[3] = pack2<false>(ex2(sc[1][2] - mn1), ex2(sc[1][3] - mn1));
+      const float2 u = unpack2<false>(pa[1]), v = unpack2<false>(pa[3]);
+      l[1] = l[1] * al1 + ((u.x + u.y) + (v.x + v.y));
+    } else {
+      pa[1] = pa[3] = 0u;
     }
 #pragma unroll
     for (int n = 0; n < NTILES; ++n) {
@@ -265,24 +286,14 @@ struct MmaFp8Warp {
       const int c = 2 * cp + mchk;
       uint32_t r0, r1, r2, r3;  // (tok 0-7, chunk 2cp) (8-15, 2cp) (0-7, 2cp+1) (8-15, 2cp+1)
       ldsm_x4_trans(vbase + mtok * 128 + ((c ^ (mtok & 7)) << 4), r0, r1, r2, r3);
-      const uint32_t e0 = e4m3x2_to_op2<BF16>(__byte_perm(r0, 0, 0x0020));
-      const uint32_t o0 = e4m3x2_to_op2<BF16>(__byte_perm(r0, 0, 0x0031));
-      const uint32_t e1 = e4m3x2_to_op2<BF16>(__byte_perm(r1, 0, 0x0020));
-      const uint32_t o1 = e4m3x2_to_op2<BF16>(__byte_perm(r1, 0, 0x0031));
-      const uint32_t e2 = e4m3x2_to_op2<BF16>(__byte_perm(r2, 0, 0x0020));
-      const uint32_t o2 = e4m3x2_to_op2<BF16>(__byte_perm(r2, 0, 0x0031));
-      const uint32_t e3 = e4m3x2_to_op2<BF16>(__byte_perm(r3, 0, 0x0020));
-      const uint32_t o3 = e4m3x2_to_op2<BF16>(__byte_perm(r3, 0, 0x0031));
-      mma_16816<BF16>(acc[4 * cp + 0], pa, e0, e1);
-      mma_16816<BF16>(acc[4 * cp + 1], pa, o0, o1);
-      mma_16816<BF16>(acc[4 * cp + 2], pa, e2, e3);
-      mma_16816<BF16>(acc[4 * cp + 3], pa, o2, o3);
-      if constexpr (BF16) {
-        mma_16816<BF16>(acc[4 * cp + 0], pl, e0, e1);
-        mma_16816<BF16>(acc[4 * cp + 1], pl, o0, o1);
-        mma_16816<BF16>(acc[4 * cp + 2], pl, e2, e3);
-        mma_16816<BF16>(acc[4 * cp + 3], pl, o2, o3);
-      }
+      mma_16816<false>(acc[4 * cp + 0], pa, e4m3x2_to_h2(__byte_perm(r0, 0, 0x0020)),
+                       e4m3x2_to_h2(__byte_perm(r1, 0, 0x0020)));
+      mma_16816<false>(acc[4 * cp + 1], pa, e4m3x2_to_h2(__byte_perm(r0, 0, 0x0031)),
+                       e4m3x2_to_h2(__byte_perm(r1, 0, 0x0031)));
+      mma_16816<false>(acc[4 * cp + 2], pa, e4m3x2_to_h2(__byte_perm(r2, 0, 0x0020)),
+                       e4m3x2_to_h2(__byte_perm(r3, 0, 0x0020)));
+      mma_16816<false>(acc[4 * cp + 3], pa, e4m3x2_to_h2(__byte_perm(r2, 0, 0x0031)),
+                       e4m3x2_to_h2(__byte_perm(r3, 0, 0x0031)));
     }
   }
 

@@ -36,6 +36,24 @@ def test_exports_every_header_symbol(lib):
         assert hasattr(lib, n), n
 
 
+def test_binding_signatures_match_header():
+    """Every ctypes signature has the header's parameter count and kinds."""
+    import ctypes
+    kind = {"ptr": ctypes.c_void_p, "int64_t": ctypes.c_int64, "float": ctypes.c_float,
+            "pa_status": ctypes.c_int, "pa_dtype": ctypes.c_int, "int32_t": ctypes.c_int32}
+    decl = _lib.header_signatures()
+    assert set(decl) == set(_lib.SIGNATURES)
+    for name, params in decl.items():
+        args = _lib.SIGNATURES[name][1]
+        assert len(args) == len(params), (name, len(args), len(params))
+        for a, p in zip(args, params):
+            want = kind[p]
+            ok = (a is want or (p == "ptr" and a in (ctypes.c_void_p, ctypes.c_char_p) or
+                                (p == "ptr" and hasattr(a, "_type_"))) or
+                  (p in ("pa_status", "pa_dtype") and a is ctypes.c_int))
+            assert ok, (name, p, a)
+
+
 def test_status_strings_and_version(lib):
     assert lib.pa_abi_version() >> 16 == 1
     for code in range(8):

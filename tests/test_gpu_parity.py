@@ -327,6 +327,27 @@ def test_copy_blocks_bit_exact(name, dev, oracle_lib):
     assert e.value.detail >> 56 == 2 and e.value.detail & 0xffff == 1
 
 
+@pytest.mark.parametrize("name,ps", [("gqa_small", 0), ("mha_small", 0), ("long_small", 512)])
+def test_host_step_matches_oracle(name, ps, dev, oracle_lib):
+    """pa_decode_step_host: inputs in pinned host memory, copied in, written,
+    attended and copied back by one C call."""
+    from paged_kv_cache_444_b200 import HostStep
+    cfg = SMALL[name]
+    batch = workloads.make_batch(cfg, dev)
+    host = HostCopy(batch)
+    ref, kc_ref, _ = oracle_step(oracle_lib, host)
+    step = HostStep(batch.key_cache, batch.value_cache, cfg.num_seqs, cfg.num_heads,
+                    batch.block_tables.shape[1], cfg.scale, ps, cfg.torch_dtype)
+    for name_ in ("query", "key", "value", "slot_mapping", "block_tables", "context_lens"):
+        getattr(step, name_).copy_(getattr(batch, name_).cpu())
+    step.out.fill_(float("nan"))
+    step.run()
+    torch.cuda.synchronize()
+    pa_check_error()
+    assert np.array_equal(bits(batch.key_cache), kc_ref)
+    _check_close(step.out, ref, cfg, f"host step {name}")
+
+
 def test_write_padding_and_strided_rows(dev, oracle_lib):
     cfg = SMALL["gqa_small"]
     batch = workloads.make_batch(cfg, dev)
