@@ -541,6 +541,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* query, const void* key_
   a.num_groups = static_cast<int>(num_groups);
   a.members_per_chunk = static_cast<int>(per_chunk);
   a.chunks_per_group = static_cast<int>(chunks);
+  a.longest_first = num_groups * chunks <= kLptMaxSeqs;
   cudaStream_t s = as_stream(stream);
   const bool bf16 = dtype == PA_BF16;
   if (head_dim == 64)

@@ -41,6 +41,7 @@ struct SharedPrefixArgs {
   int members_per_chunk;          // 16 / G
   int chunks_per_group;           // ceil(max_group_size / members_per_chunk)
   int cluster_pages;              // items with more pages are spread over the cluster
+  int longest_first;              // order (group, chunk) slots by descending page count
 };
 
 template <int D, int NST, bool BF16>
@@ -61,12 +62,49 @@ __global__ void __launch_bounds__(kThreads)
   pdl_launch_dependents();
   pdl_wait();
 
-  int item = blockIdx.x / csize;
-  const int chunk = item % a.chunks_per_group;
-  item /= a.chunks_per_group;
+  // grid slot -> (group, chunk) and KV head; KV heads of one slot are adjacent
+  const int item = blockIdx.x / csize;
   const int kvh = item % a.num_kv_heads;
-  const int grp = item / a.num_kv_heads;
+  int slot = item / a.num_kv_heads;
   const int G = a.group;
+  if (a.longest_first) {
+    // rank every (group, chunk) slot by its page count, longest first (ties
+    // by index), and take the one whose rank is this grid slot
+    const int U = a.num_groups * a.chunks_per_group;
+    int* pages = reinterpret_cast<int*>(smem);       // stage area, not in use yet
+    int* chosen = pages + kLptMaxSeqs;
+    for (int u = threadIdx.x; u < U; u += kThreads) {
+      const int g = u / a.chunks_per_group, c = u % a.chunks_per_group;
+      const int b0 = a.group_starts[g], b1 = a.group_starts[g + 1];
+      const int p = a.prefix_blocks[g];
+      int tail = 0, most = 0;
+      const int first_m = b0 + c * a.members_per_chunk;
+      const int last_m = min(b1, first_m + a.members_per_chunk);
+      if (b0 >= 0 && b1 <= a.num_seqs && p >= 0) {
+        for (int sq = first_m; sq < last_m; ++sq) {
+          const int np = (max(a.context_lens[sq], 0) + kPage - 1) / kPage;
+          most = max(most, np);
+          tail += max(0, np - p);
+        }
+      }
+      pages[u] = min(p, most) + tail;
+    }
+    __syncthreads();
+    for (int u = threadIdx.x; u < U; u += kThreads) {
+      const int pu = pages[u];
+      int rank = 0;
+      for (int v = 0; v < U; ++v) {
+        const int pv = pages[v];
+        rank += (pv > pu) | ((pv == pu) & (v < u));
+      }
+      if (rank == slot) *chosen = u;
+    }
+    __syncthreads();
+    slot = *chosen;
+    __syncthreads();  // the stage area is about to be reused
+  }
+  const int chunk = slot % a.chunks_per_group;
+  const int grp = slot / a.chunks_per_group;
   const bool reporter = threadIdx.x == 0 && crank == 0 && kvh == 0 && chunk == 0;
 
   // ---- the group and this chunk's members ----
