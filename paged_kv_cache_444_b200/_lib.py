@@ -341,6 +341,65 @@ def pa_decode_split_fp8(tmp_out, max_logits, exp_sums, query, key_cache, value_c
     _check(st, "pa_decode_split_fp8")
 
 
+class DecodePlan:
+    """One decode step (cache write, then attention) over fixed tensors,
+    validated once: the argument lists of its C calls are built here, and
+    run() only adds the stream.  Tensors are held by reference, so their
+    contents may change between runs but not their storage.  The calls can
+    be captured in a CUDA graph (run() inside torch.cuda.graph)."""
+
+    def __init__(self, query, key, value, key_cache, value_cache, slot_mapping, block_tables,
+                 context_lens, scale: float, out=None, partition_size: int = 0, workspace=None):
+        S, H, D, NB, bs, Hk, MB, dt = _attention_common(query, key_cache, value_cache,
+                                                        block_tables, context_lens)
+        self.out = torch.empty_like(query) if out is None else out
+        _need(self.out.shape == query.shape and self.out.dtype == query.dtype and
+              self.out.is_contiguous(), "out must match query")
+        self._keep = [query, key, value, key_cache, value_cache, slot_mapping, block_tables,
+                      context_lens, self.out]
+        self.calls = []
+        if key is not None and key.shape[0] > 0:
+            T = key.shape[0]
+            _need(key.shape == (T, Hk, D) and value.shape == key.shape, "key/value shape")
+            _need(key.stride()[1:] == (D, 1) and value.stride()[1:] == (D, 1), "rows dense")
+            _need(slot_mapping.dtype == torch.int64 and slot_mapping.shape == (T,), "slots")
+            self.calls.append(("pa_reshape_and_cache", (
+                key.data_ptr(), value.data_ptr(), key.stride(0), value.stride(0),
+                key_cache.data_ptr(), value_cache.data_ptr(), slot_mapping.data_ptr(), T, Hk, D,
+                NB, bs, dt)))
+        if partition_size > 0:
+            if workspace is None:
+                P = (MB * bs + partition_size - 1) // partition_size
+                from . import SplitWorkspace
+                workspace = SplitWorkspace(S, H, D, P, query.device)
+            self._keep.append(workspace)
+            P = workspace.max_partitions
+            self.calls.append(("pa_decode_split", (
+                workspace.tmp_out.data_ptr(), workspace.max_logits.data_ptr(),
+                workspace.exp_sums.data_ptr(), query.data_ptr(), key_cache.data_ptr(),
+                value_cache.data_ptr(), block_tables.data_ptr(), context_lens.data_ptr(),
+                float(scale), S, H, Hk, D, NB, bs, MB, int(partition_size), P, dt)))
+            self.calls.append(("pa_reduce", (
+                self.out.data_ptr(), workspace.tmp_out.data_ptr(),
+                workspace.max_logits.data_ptr(), workspace.exp_sums.data_ptr(),
+                context_lens.data_ptr(), S, H, D, int(partition_size), P, dt)))
+        else:
+            self.calls.append(("pa_decode", (
+                self.out.data_ptr(), query.data_ptr(), key_cache.data_ptr(),
+                value_cache.data_ptr(), block_tables.data_ptr(), context_lens.data_ptr(),
+                float(scale), S, H, Hk, D, NB, bs, MB, dt)))
+        lib = load()
+        self._bound = [(getattr(lib, name), args, name) for name, args in self.calls]
+
+    def run(self, stream=None) -> torch.Tensor:
+        s = _stream(stream)
+        for fn, args, name in self._bound:
+            st = fn(*args, s)
+            if st != PA_OK:
+                raise PagedAttentionError(st, name)
+        return self.out
+
+
 class HostStep:
     """pa_decode_step_host for one layer: per-step inputs live in (pinned)
     host tensors, the caches and a device workspace stay resident.  `run()`

@@ -348,6 +348,36 @@ def test_host_step_matches_oracle(name, ps, dev, oracle_lib):
     _check_close(step.out, ref, cfg, f"host step {name}")
 
 
+@pytest.mark.parametrize("name,ps", [("gqa_small", 0), ("long_small", 64), ("tiny", 0)])
+def test_plan_replays_from_a_cuda_graph(name, ps, dev, oracle_lib):
+    """A DecodePlan run eagerly, and the same plan captured once in a CUDA
+    graph and replayed, both match the oracle; replay equals eager bit for bit."""
+    from paged_kv_cache_444_b200 import DecodePlan
+    cfg = SMALL[name]
+    batch = workloads.make_batch(cfg, dev)
+    host = HostCopy(batch)
+    ref, _, _ = oracle_step(oracle_lib, host)
+    plan = DecodePlan(batch.query, batch.key, batch.value, batch.key_cache, batch.value_cache,
+                      batch.slot_mapping, batch.block_tables, batch.context_lens, cfg.scale,
+                      partition_size=ps)
+    eager = plan.run().clone()
+    torch.cuda.synchronize()
+    _check_close(eager, ref, cfg, f"plan {name}")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        plan.run()                      # warm-up on the side stream
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        plan.run()
+    plan.out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    pa_check_error()
+    assert torch.equal(plan.out, eager)
+
+
 def test_write_padding_and_strided_rows(dev, oracle_lib):
     cfg = SMALL["gqa_small"]
     batch = workloads.make_batch(cfg, dev)
