@@ -66,7 +66,8 @@ enum {
     PA_CHECK_CONTEXT_LEN = 3,   /* context_lens[s] < 0 or > max_blocks_per_seq*block_size; index = s */
     PA_CHECK_PARTITIONS = 4,    /* ceil(context_lens[s]/partition_size) > max_partitions; index = s */
     PA_CHECK_WAIT_TIMEOUT = 5,  /* a shared-memory barrier wait gave up; index = CTA id */
-    PA_CHECK_GROUP = 6          /* malformed group bounds or prefix length; index = group */
+    PA_CHECK_GROUP = 6,         /* malformed group bounds or prefix length; index = group */
+    PA_CHECK_QUERY = 7          /* prefill: q_len < 0, q_len > context_lens[s] or context too long; index = s */
 };
 
 /* Short English name of a status code (static string, never NULL). */
@@ -280,6 +281,31 @@ pa_status pa_decode_step_host(void *out_host, const void *query_host, const void
                               int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
                               int64_t block_size, int64_t max_blocks_per_seq,
                               int64_t partition_size, pa_dtype dtype, void *stream);
+
+/*
+ * pa_prefill -- paged (chunked) prefill attention ("vLLM PagedAttention 原理与
+ * 源码深度解析" §8.1 Chunked Prefill: a prompt is processed a chunk of tokens
+ * per step).  Sequence s has q_len = query_starts[s+1] - query_starts[s] new
+ * query tokens, the LAST q_len of its context_lens[s] tokens, whose K/V are
+ * already in the caches (pa_reshape_and_cache first, on the same stream).
+ * Query token i (row query_starts[s] + i) sits at position
+ * pos = context_lens[s] - q_len + i and attends causally to tokens 0..pos:
+ *   out[t,h,:] = sum_{j<=pos} softmax_j(scale * q[t,h,:] . k_j) v_j.
+ *   query, out     [num_query_tokens, num_heads, head_dim], rows grouped by sequence
+ *   query_starts   [num_seqs + 1] int32, query_starts[0] = 0, nondecreasing,
+ *                  query_starts[num_seqs] = num_query_tokens
+ *   max_query_len  host-side upper bound of every q_len (sizes the grid)
+ * Other arguments as pa_decode.  A sequence with q_len > context_lens[s] is
+ * skipped and reported (PA_CHECK_QUERY).  fp32 accumulation; P enters the
+ * P.V product in the cache dtype (bf16 as a hi + lo pair).
+ */
+pa_status pa_prefill(void *out, const void *query, const void *key_cache,
+                     const void *value_cache, const int32_t *block_tables,
+                     const int32_t *context_lens, const int32_t *query_starts, float scale,
+                     int64_t num_seqs, int64_t num_query_tokens, int64_t max_query_len,
+                     int64_t num_heads, int64_t num_kv_heads, int64_t head_dim,
+                     int64_t num_blocks, int64_t block_size, int64_t max_blocks_per_seq,
+                     pa_dtype dtype, void *stream);
 
 /*
  * pa_check_error -- synchronise `stream`, read and clear the current device's

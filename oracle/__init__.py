@@ -99,6 +99,8 @@ class Oracle:
         lib.oracle_decode_fp8.argtypes = ([_p] * 6 + [_i64] * 7 +
                                           [ctypes.c_double] * 3 + [ctypes.c_int])
         lib.oracle_decode_fp8.restype = ctypes.c_int
+        lib.oracle_prefill.argtypes = [_p] * 7 + [_i64] * 7 + [ctypes.c_double, ctypes.c_int]
+        lib.oracle_prefill.restype = ctypes.c_int
 
     # ---- scalar helpers -------------------------------------------------
     def f16_to_f64(self, bits: int) -> float:
@@ -198,6 +200,29 @@ class Oracle:
                                          float(k_scale), float(v_scale), dtype)
         if rc != OK:
             raise ValueError(f"oracle_decode_fp8 failed with code {rc}")
+        return out
+
+    def prefill(self, query, key_cache, value_cache, block_tables, context_lens, query_starts,
+                scale: float, dtype: int) -> np.ndarray:
+        """Causal attention of each sequence's last q_len positions (query
+        [T, H, D], T = query_starts[-1]) over its paged context; float64 [T, H, D]."""
+        q = np.ascontiguousarray(query, dtype=np.uint16)
+        kc = np.ascontiguousarray(key_cache, dtype=np.uint16)
+        vc = np.ascontiguousarray(value_cache, dtype=np.uint16)
+        bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+        cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+        qs = np.ascontiguousarray(query_starts, dtype=np.int32)
+        T, H, D = q.shape
+        NB, bs, Hk, _ = kc.shape
+        S = cl.shape[0]
+        assert qs.shape == (S + 1,) and qs[-1] == T
+        out = np.zeros((T, H, D), dtype=np.float64)
+        rc = self._lib.oracle_prefill(out.ctypes.data, q.ctypes.data, kc.ctypes.data,
+                                      vc.ctypes.data, bt.ctypes.data, cl.ctypes.data,
+                                      qs.ctypes.data, S, H, Hk, D, NB, bs, bt.shape[1],
+                                      float(scale), dtype)
+        if rc != OK:
+            raise ValueError(f"oracle_prefill failed with code {rc}")
         return out
 
     def copy_blocks(self, key_cache, value_cache, block_mapping) -> int:

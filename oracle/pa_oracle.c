@@ -582,3 +582,62 @@ int oracle_decode_fp8(double *out, const uint16_t *query,
     }
     return ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Paged (chunked) prefill: "vLLM PagedAttention 原理与源码深度解析" §8.1       */
+/* (Chunked Prefill: a long prompt is processed a chunk of tokens at a time)  */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Sequence s contributes q_len = query_starts[s+1] - query_starts[s] query
+ * tokens: the LAST q_len positions of its context_lens[s] tokens (their K/V
+ * already in the cache).  Query token i sits at position
+ * pos = context_lens[s] - q_len + i and attends causally to tokens 0..pos:
+ *   out[t, h, :] = softmax_j<=pos(scale * q[t,h,:] . k_j) . v_j,
+ * t = query_starts[s] + i, query head h reading KV head h / (H / Hk).
+ *   query, out  [T, num_heads, head_dim] (T = query_starts[num_seqs])
+ * Requires q_len <= context_lens[s].
+ */
+int oracle_prefill(double *out, const uint16_t *query,
+                   const uint16_t *key_cache, const uint16_t *value_cache,
+                   const int32_t *block_tables, const int32_t *context_lens,
+                   const int32_t *query_starts, int64_t num_seqs, int64_t num_heads,
+                   int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                   int64_t block_size, int64_t max_blocks_per_seq, double scale, int dtype)
+{
+    if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || block_size <= 0)
+        return ORACLE_BAD_ARG;
+    int64_t group = num_heads / num_kv_heads;
+    for (int64_t s = 0; s < num_seqs; ++s) {
+        int64_t ctx = context_lens[s];
+        int64_t q0 = query_starts[s], q_len = query_starts[s + 1] - q0;
+        if (q_len <= 0) continue;
+        if (q_len > ctx || ctx > max_blocks_per_seq * block_size) return ORACLE_BAD_ARG;
+        double *kc = malloc(sizeof(double) * (size_t)(ctx * head_dim));
+        double *vc = malloc(sizeof(double) * (size_t)(ctx * head_dim));
+        double *z = malloc(sizeof(double) * (size_t)ctx);
+        double *q = malloc(sizeof(double) * (size_t)head_dim);
+        if (!kc || !vc || !z || !q) { free(kc); free(vc); free(z); free(q); return ORACLE_NO_MEMORY; }
+        for (int64_t h = 0; h < num_heads; ++h) {
+            int64_t kvh = h / group;
+            if (h % group == 0) {
+                int rc = gather_head(kc, vc, key_cache, value_cache,
+                                     block_tables + s * max_blocks_per_seq, ctx, kvh,
+                                     num_kv_heads, head_dim, num_blocks, block_size, dtype);
+                if (rc != ORACLE_OK) { free(kc); free(vc); free(z); free(q); return rc; }
+            }
+            for (int64_t i = 0; i < q_len; ++i) {
+                int64_t t = q0 + i;
+                int64_t pos = ctx - q_len + i;
+                const uint16_t *qs = query + (t * num_heads + h) * head_dim;
+                for (int64_t d = 0; d < head_dim; ++d) q[d] = decode16(qs[d], dtype);
+                double m, l;
+                double *acc = out + (t * num_heads + h) * head_dim;
+                attend_range(q, kc, vc, head_dim, 0, pos + 1, scale, z, &m, &l, acc);
+                for (int64_t d = 0; d < head_dim; ++d) acc[d] /= l;
+            }
+        }
+        free(kc); free(vc); free(z); free(q);
+    }
+    return ORACLE_OK;
+}

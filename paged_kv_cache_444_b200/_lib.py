@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_NULL", 2: "PA_ERR_SHAPE", 3: "PA_ERR_DTYP
                 4: "PA_ERR_ALIGN", 5: "PA_ERR_UNSUPPORTED", 6: "PA_ERR_CUDA",
                 7: "PA_ERR_BOUNDS"}
 CHECK_CODES = {1: "slot", 2: "block_id", 3: "context_len", 4: "partitions", 5: "wait_timeout",
-               6: "group"}
+               6: "group", 7: "query"}
 DTYPE_CODES = {torch.float16: 0, torch.bfloat16: 1}
 
 
@@ -69,6 +69,7 @@ SIGNATURES = {
                                  _i64, _i64, _i64, _i64, _i64, _i64, _i, _p]),
     "pa_decode_step_host_workspace_bytes": (_i64, [_i64] * 7),
     "pa_decode_step_host": (_i, [_p] * 10 + [_i64, _f] + [_i64] * 8 + [_i, _p]),
+    "pa_prefill": (_i, [_p] * 7 + [_f] + [_i64] * 9 + [_i, _p]),
 }
 
 _lib: ctypes.CDLL | None = None
@@ -339,6 +340,34 @@ def pa_decode_split_fp8(tmp_out, max_logits, exp_sums, query, key_cache, value_c
                                     float(v_scale), S, H, Hk, D, NB, bs, MB, int(partition_size),
                                     P, dt, _stream(stream))
     _check(st, "pa_decode_split_fp8")
+
+
+def pa_prefill(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+               value_cache: torch.Tensor, block_tables: torch.Tensor,
+               context_lens: torch.Tensor, query_starts: torch.Tensor, scale: float,
+               max_query_len: int, stream=None) -> None:
+    """Chunked prefill: query [T, H, D] rows grouped by sequence
+    (query_starts [S + 1] int32); each sequence's rows are the last q_len
+    positions of its context and attend causally over the paged cache."""
+    T, H, D = query.shape
+    NB, bs, Hk, D2 = key_cache.shape
+    S = context_lens.shape[0]
+    _need(D2 == D and value_cache.shape == key_cache.shape, "cache shapes")
+    _need(query.is_contiguous() and key_cache.is_contiguous() and value_cache.is_contiguous(),
+          "query and caches must be contiguous")
+    _need(block_tables.dtype == torch.int32 and block_tables.shape[0] == S and
+          block_tables.is_contiguous(), "block_tables must be [S, MB] int32")
+    _need(context_lens.dtype == torch.int32, "context_lens must be int32")
+    _need(query_starts.dtype == torch.int32 and query_starts.shape == (S + 1,),
+          "query_starts must be [S + 1] int32")
+    _need(out.shape == query.shape and out.dtype == query.dtype and out.is_contiguous(), "out")
+    _need(query.dtype == key_cache.dtype == value_cache.dtype, "dtype mismatch")
+    st = load().pa_prefill(out.data_ptr(), query.data_ptr(), key_cache.data_ptr(),
+                           value_cache.data_ptr(), block_tables.data_ptr(),
+                           context_lens.data_ptr(), query_starts.data_ptr(), float(scale), S, T,
+                           int(max_query_len), H, Hk, D, NB, bs, block_tables.shape[1],
+                           _dtype_code(query), _stream(stream))
+    _check(st, "pa_prefill")
 
 
 class DecodePlan:

@@ -13,6 +13,7 @@
 #include "pa_cache_reduce.cuh"
 #include "pa_decode.cuh"
 #include "pa_decode_fp8.cuh"
+#include "pa_prefill.cuh"
 #include "pa_shared_prefix.cuh"
 
 namespace {
@@ -321,6 +322,22 @@ pa_status check_fp8_scales(float k_scale, float v_scale) {
   if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f))
     return PA_ERR_SHAPE;
   return PA_OK;
+}
+
+#ifndef PA_PREFILL_STAGES
+#define PA_PREFILL_STAGES 4
+#endif
+
+template <int D, bool BF16>
+pa_status launch_prefill_t(const CUtensorMap& km, const CUtensorMap& vm, const PrefillArgs& a,
+                           long long grid, cudaStream_t stream) {
+  constexpr int NST = PA_PREFILL_STAGES;
+  using L = PrefillSmem<D, NST>;
+  auto kernel = paged_prefill_kernel<D, NST, BF16>;
+  static std::atomic<uint64_t> done{0};
+  if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
+  return launch_ex(kernel, static_cast<unsigned>(grid), kThreads, L::kAlloc, stream, 1, km, vm,
+                   a);
 }
 
 DecodeArgs make_args(const void* query, const int32_t* block_tables, const int32_t* context_lens,
@@ -769,6 +786,54 @@ pa_status pa_decode_step_host(void* out_host, const void* query_host, const void
       cudaSuccess)
     return PA_ERR_CUDA;
   return PA_OK;
+}
+
+pa_status pa_prefill(void* out, const void* query, const void* key_cache, const void* value_cache,
+                     const int32_t* block_tables, const int32_t* context_lens,
+                     const int32_t* query_starts, float scale, int64_t num_seqs,
+                     int64_t num_query_tokens, int64_t max_query_len, int64_t num_heads,
+                     int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                     int64_t block_size, int64_t max_blocks_per_seq, pa_dtype dtype,
+                     void* stream) {
+  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
+                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
+                                      num_blocks, block_size, max_blocks_per_seq, dtype);
+  if (st != PA_OK) return st;
+  if (num_query_tokens < 0 || max_query_len < 0) return PA_ERR_SHAPE;
+  if (num_seqs == 0 || num_query_tokens == 0 || max_query_len == 0) return PA_OK;
+  if (!out || !query_starts) return PA_ERR_NULL;
+  if (!aligned16(out) || (reinterpret_cast<uintptr_t>(query_starts) & 3u)) return PA_ERR_ALIGN;
+  if (num_query_tokens * num_heads > INT32_MAX || max_query_len > INT32_MAX) return PA_ERR_SHAPE;
+  const int64_t G = num_heads / num_kv_heads;
+  const int64_t tile = 64 / G;                            // G <= 16 checked above
+  const int64_t tiles = (max_query_len + tile - 1) / tile;
+  const long long grid = num_seqs * num_kv_heads * tiles;
+  if (grid > INT32_MAX) return PA_ERR_SHAPE;
+  CUtensorMap km, vm;
+  if (!encode_cache_map(&km, key_cache, dtype, num_blocks, num_kv_heads, head_dim) ||
+      !encode_cache_map(&vm, value_cache, dtype, num_blocks, num_kv_heads, head_dim))
+    return PA_ERR_CUDA;
+  PrefillArgs a{};
+  a.query = static_cast<const uint16_t*>(query);
+  a.out = static_cast<uint16_t*>(out);
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_starts = query_starts;
+  a.scale_log2 = scale * kLog2e;
+  a.num_heads = static_cast<int>(num_heads);
+  a.num_kv_heads = static_cast<int>(num_kv_heads);
+  a.group = static_cast<int>(G);
+  a.max_blocks_per_seq = static_cast<int>(max_blocks_per_seq);
+  a.num_blocks = static_cast<int>(num_blocks);
+  a.tile_tokens = static_cast<int>(tile);
+  a.tiles_per_seq = static_cast<int>(tiles);
+  cudaStream_t s = as_stream(stream);
+  const bool bf16 = dtype == PA_BF16;
+  if (head_dim == 64)
+    return bf16 ? launch_prefill_t<64, true>(km, vm, a, grid, s)
+                : launch_prefill_t<64, false>(km, vm, a, grid, s);
+  return bf16 ? launch_prefill_t<128, true>(km, vm, a, grid, s)
+              : launch_prefill_t<128, false>(km, vm, a, grid, s);
 }
 
 pa_status pa_check_error(void* stream, int64_t* detail) {

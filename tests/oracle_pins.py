@@ -488,6 +488,44 @@ def pin_fp8_decode_sdpa(orc):
             assert np.max(np.abs(got[s_] - o.numpy())) <= 1e-12
 
 
+def pin_prefill_causal_sdpa(orc):
+    """Chunked prefill: the last q_len positions of each sequence attend
+    causally over their context.  Equals torch SDPA (float64) with an
+    explicit mask j <= position on contiguously gathered K/V; q_len = 1
+    equals decode."""
+    rng = np.random.default_rng(41)
+    for S, H, Hk, D, bs, ctx, qlen, dt in [(3, 4, 2, 16, 4, [9, 17, 5], [3, 17, 1], F16),
+                                           (2, 8, 8, 8, 16, [40, 33], [12, 1], BF16)]:
+        NB = sum((c + bs - 1) // bs for c in ctx) + 2
+        q, kc, vc, bt, cl = _random_case(rng, S, H, Hk, D, bs, NB, ctx, dt)
+        tdt = torch.bfloat16 if dt == BF16 else torch.float16
+        T = sum(qlen)
+        gq = torch.Generator().manual_seed(T)
+        qt = _bits(torch.randn((T, H, D), generator=gq).to(tdt))
+        starts = np.concatenate([[0], np.cumsum(qlen)]).astype(np.int32)
+        got = orc.prefill(qt, kc, vc, bt, cl, starts, 0.3, dt)
+        to64 = lambda b: torch.from_numpy(b.view(np.int16)).view(tdt).to(torch.float64)
+        kd, vd, qd = to64(kc), to64(vc), to64(qt)
+        for s_ in range(S):
+            c, ql = ctx[s_], qlen[s_]
+            nb = (c + bs - 1) // bs
+            idx = torch.from_numpy(bt[s_, :nb].astype(np.int64))
+            k = kd[idx].reshape(nb * bs, Hk, D)[:c].permute(1, 0, 2)[None]
+            v = vd[idx].reshape(nb * bs, Hk, D)[:c].permute(1, 0, 2)[None]
+            pos = torch.arange(c - ql, c)
+            mask = (torch.arange(c)[None, :] <= pos[:, None])[None, None]
+            qq = qd[starts[s_]:starts[s_ + 1]].permute(1, 0, 2)[None]
+            o = F.scaled_dot_product_attention(qq, k, v, attn_mask=mask, scale=0.3,
+                                               enable_gqa=True)[0].permute(1, 0, 2)
+            assert np.max(np.abs(got[starts[s_]:starts[s_ + 1]] - o.numpy())) <= 1e-12
+        # one query per sequence at its last position is decode
+        ones = np.arange(S + 1, dtype=np.int32)
+        last = np.stack([qt[starts[i + 1] - 1] for i in range(S)])
+        dec = orc.decode(last, kc, vc, bt, cl, 0.3, dt)
+        pre = orc.prefill(last, kc, vc, bt, cl, ones, 0.3, dt)
+        assert np.array_equal(dec, pre)
+
+
 ALL_PINS = [
     pin_f16_decode_all_patterns,
     pin_bf16_decode_all_patterns,
@@ -509,4 +547,5 @@ ALL_PINS = [
     pin_e4m3_rounding,
     pin_fp8_write_worked_example,
     pin_fp8_decode_sdpa,
+    pin_prefill_causal_sdpa,
 ]

@@ -81,6 +81,10 @@ MUTATIONS = [
      "key_cache[slot * row + e] = oracle_f64_to_e4m3((double)kx);"),
     ("fp8 decode: v scale dropped", "vc[j * head_dim + d] = oracle_e4m3_to_f64(value_cache[base + d]) * v_scale;",
      "vc[j * head_dim + d] = oracle_e4m3_to_f64(value_cache[base + d]);"),
+    ("prefill: query position off by one", "int64_t pos = ctx - q_len + i;",
+     "int64_t pos = ctx - q_len + i - 1;"),
+    ("prefill: not causal", "attend_range(q, kc, vc, head_dim, 0, pos + 1, scale, z, &m, &l, acc);",
+     "attend_range(q, kc, vc, head_dim, 0, ctx, scale, z, &m, &l, acc);"),
     ("partition: end not clipped to ctx",
      "int64_t t1 = t0 + partition_size < ctx ? t0 + partition_size : ctx;",
      "int64_t t1 = t0 + partition_size < ctx ? t0 + partition_size : ctx - 1;"),
