@@ -292,6 +292,52 @@ def fp8_decode_ms(batch, warmup: int, reps: int = 100) -> float | None:
     return start.elapsed_time(end) / reps
 
 
+def prefill_measure(device, warmup: int, reps: int = 20, peak_tflops: float = 0.0,
+                    peak_kind: str = "") -> dict:
+    """Chunked prefill on a Llama-3-8B-shaped GQA layer: 8 sequences each
+    bringing a 512-token chunk at the end of a context drawn U[512, 4096]
+    (32/8 heads, d=128, bf16, 16-token blocks).  Compute-bound: reported in
+    TFLOP/s against the measured dense bf16 peak, with the CPU oracle's
+    count of flops: 4 * D * H * sum over queries of (position + 1)."""
+    from paged_kv_cache_444_b200 import pa_prefill
+    cfg = workloads.CONFIGS["gqa_llama3_8b"].scaled(
+        name="chunked_prefill_gqa", num_seqs=8, num_blocks=4096, ctx=("uniform", 512, 4096),
+        seed=444_006)
+    b = workloads.make_batch(cfg, device)
+    chunk = 512
+    T = cfg.num_seqs * chunk
+    g = torch.Generator(device=device).manual_seed(cfg.seed + 1)
+    query = torch.randn((T, cfg.num_heads, cfg.head_dim), generator=g, device=device).to(
+        cfg.torch_dtype)
+    starts = torch.arange(0, T + 1, chunk, dtype=torch.int32, device=device)
+    out = torch.empty_like(query)
+
+    def run():
+        pa_prefill(out, query, b.key_cache, b.value_cache, b.block_tables, b.context_lens,
+                   starts, cfg.scale, chunk)
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(reps):
+        run()
+    end.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / reps
+    ctx = b.context_lens.cpu().tolist()
+    pairs = sum(sum(c - chunk + i + 1 for i in range(chunk)) for c in ctx)
+    flops = 4 * cfg.head_dim * cfg.num_heads * pairs
+    tf = flops / (ms / 1e3) / 1e12
+    return {"workload": "chunked_prefill_gqa: 8 seqs x 512-token chunks at ctx U[512,4096], "
+                        "32/8 heads, d=128, bf16", "kernel": "pa_prefill",
+            "ms": round(ms, 5), "tflops": round(tf, 1),
+            "query_tokens_per_s": round(T / (ms / 1e3), 1),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak_tflops,
+                         "unit": "TFLOP/s", "frac": round(tf / peak_tflops, 4) if peak_tflops else None,
+                         "peak_kind": peak_kind, "algorithmic_flops": flops}}
+
+
 def graph_steps(step: Step, steps: int, warmup: int) -> float | None:
     """The same step captured once in a CUDA graph and replayed `steps` times
     (ms per step), or None if capture is not possible here."""
@@ -365,6 +411,17 @@ def measured_peak():
         except Exception:
             pass
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s: the burst figure (a kernel timed alone)."""
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        try:
+            return float(json.loads(p.read_text())["bf16_tflops"]), "measured (burst)"
+        except Exception:
+            pass
+    return 1590.0, "fallback (burst)"
 
 
 def attention_kernel_bytes(cfg, context_lens, split: bool) -> int:
@@ -595,6 +652,9 @@ def run_native(args, world, rank, local):
                    if r["shared_prefix_kernel_ms"] else {}),
                 **(fp8_entry(r, peak) if r["fp8_ms"] else {})}
             for n, r in results.items()}
+    if args.prefill and not args.only_main:
+        tp, tk = measured_tensor_peak()
+        line["prefill"] = prefill_measure(device, args.warmup, peak_tflops=tp, peak_kind=tk)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, ctx_main, bt_main, batch,
                                             budget_s=args.cpu_budget)
@@ -709,6 +769,8 @@ def main(argv=None):
                     help="also time the step replayed from a CUDA graph")
     ap.add_argument("--fp8", action=argparse.BooleanOptionalAction, default=True,
                     help="also time pa_decode_fp8 on each batch (E4M3 copy of its caches)")
+    ap.add_argument("--prefill", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time pa_prefill on a chunked-prefill GQA layer")
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="override the workload's batch size (small profiling captures)")
     ap.add_argument("--num-blocks", type=int, default=0,
