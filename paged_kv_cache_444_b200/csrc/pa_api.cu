@@ -324,20 +324,37 @@ pa_status check_fp8_scales(float k_scale, float v_scale) {
   return PA_OK;
 }
 
-#ifndef PA_PREFILL_STAGES
-#define PA_PREFILL_STAGES 4
-#endif
+// 4-D view of the query [T, H, D] for boxes of G heads x tile tokens x 64
+// elements (128-byte swizzle): rows land token-major, row = token * G + head.
+bool encode_query_map(CUtensorMap* map, const void* query, pa_dtype dtype, int64_t num_tokens,
+                      int64_t num_heads, int64_t head_dim, int64_t group, int64_t tile_tokens) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(head_dim / 64),
+                              static_cast<cuuint64_t>(num_heads),
+                              static_cast<cuuint64_t>(num_tokens)};
+  const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(head_dim * 2),
+                                 static_cast<cuuint64_t>(num_heads * head_dim * 2)};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(group),
+                             static_cast<cuuint32_t>(tile_tokens)};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        4, const_cast<void*>(query), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 template <int D, bool BF16>
-pa_status launch_prefill_t(const CUtensorMap& km, const CUtensorMap& vm, const PrefillArgs& a,
-                           long long grid, cudaStream_t stream) {
-  constexpr int NST = PA_PREFILL_STAGES;
-  using L = PrefillSmem<D, NST>;
-  auto kernel = paged_prefill_kernel<D, NST, BF16>;
+pa_status launch_prefill_t(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
+                           const PrefillArgs& a, long long grid, cudaStream_t stream) {
+  using L = PrefillSmem<D, BF16>;
+  auto kernel = paged_prefill_kernel<D, BF16>;
   static std::atomic<uint64_t> done{0};
   if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
-  return launch_ex(kernel, static_cast<unsigned>(grid), kThreads, L::kAlloc, stream, 1, km, vm,
-                   a);
+  return launch_ex(kernel, static_cast<unsigned>(grid), kPrefillThreads, L::kAlloc, stream, 1, qm,
+                   km, vm, a);
 }
 
 DecodeArgs make_args(const void* query, const int32_t* block_tables, const int32_t* context_lens,
@@ -805,21 +822,23 @@ pa_status pa_prefill(void* out, const void* query, const void* key_cache, const 
   if (!aligned16(out) || (reinterpret_cast<uintptr_t>(query_starts) & 3u)) return PA_ERR_ALIGN;
   if (num_query_tokens * num_heads > INT32_MAX || max_query_len > INT32_MAX) return PA_ERR_SHAPE;
   const int64_t G = num_heads / num_kv_heads;
-  const int64_t tile = 64 / G;                            // G <= 16 checked above
+  const int64_t tile = kPrefillRows / G;                  // G <= 16 checked above
   const int64_t tiles = (max_query_len + tile - 1) / tile;
   const long long grid = num_seqs * num_kv_heads * tiles;
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
-  CUtensorMap km, vm;
-  if (!encode_cache_map(&km, key_cache, dtype, num_blocks, num_kv_heads, head_dim) ||
+  CUtensorMap qm, km, vm;
+  if (!encode_query_map(&qm, query, dtype, num_query_tokens, num_heads, head_dim, G, tile) ||
+      !encode_cache_map(&km, key_cache, dtype, num_blocks, num_kv_heads, head_dim) ||
       !encode_cache_map(&vm, value_cache, dtype, num_blocks, num_kv_heads, head_dim))
     return PA_ERR_CUDA;
   PrefillArgs a{};
-  a.query = static_cast<const uint16_t*>(query);
   a.out = static_cast<uint16_t*>(out);
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.query_starts = query_starts;
   a.scale_log2 = scale * kLog2e;
+  a.num_seqs = static_cast<int>(num_seqs);
+  a.num_tokens = static_cast<int>(num_query_tokens);
   a.num_heads = static_cast<int>(num_heads);
   a.num_kv_heads = static_cast<int>(num_kv_heads);
   a.group = static_cast<int>(G);
@@ -830,10 +849,10 @@ pa_status pa_prefill(void* out, const void* query, const void* key_cache, const 
   cudaStream_t s = as_stream(stream);
   const bool bf16 = dtype == PA_BF16;
   if (head_dim == 64)
-    return bf16 ? launch_prefill_t<64, true>(km, vm, a, grid, s)
-                : launch_prefill_t<64, false>(km, vm, a, grid, s);
-  return bf16 ? launch_prefill_t<128, true>(km, vm, a, grid, s)
-              : launch_prefill_t<128, false>(km, vm, a, grid, s);
+    return bf16 ? launch_prefill_t<64, true>(qm, km, vm, a, grid, s)
+                : launch_prefill_t<64, false>(qm, km, vm, a, grid, s);
+  return bf16 ? launch_prefill_t<128, true>(qm, km, vm, a, grid, s)
+              : launch_prefill_t<128, false>(qm, km, vm, a, grid, s);
 }
 
 pa_status pa_check_error(void* stream, int64_t* detail) {

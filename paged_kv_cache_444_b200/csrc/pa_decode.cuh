@@ -645,6 +645,7 @@ __global__ void __launch_bounds__(kThreads)
     }
     const uint32_t kb = stage0 + stg * L::kStageBytes;
     const int tok0 = (first_page + page0 + k * pstride) * kPage;
+    if (tok0 + kPage > ctx) zero_page_tail<L::kBoxesPerRow>(kb + L::kPageBytes, ctx - tok0, lane);
     st.page(kb, kb + L::kPageBytes, tok0, t_end, a.scale_log2, lane, probs);
     __syncwarp();
     if (k + NST < my_pages) issue(k + NST);

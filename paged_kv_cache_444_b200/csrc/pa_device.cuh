@@ -59,6 +59,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                ::"r"(bar), "r"(bytes) : "memory");
 }
 
+// Plain arrival (one count) on a barrier.
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
@@ -97,6 +102,34 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (TMA, tensor-core operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// Zero rows [row0, 16) of a staged page (BOXES boxes of 16 rows x 128 B, whole
+// warp).  Cache rows past a sequence's context were never written and may
+// hold anything; their probability is 0, and 0 * NaN must not reach O.  The
+// proxy fence orders these writes before a later TMA refill of the stage.
+template <int BOXES>
+__device__ __forceinline__ void zero_page_tail(uint32_t page, int row0, int lane) {
+  const int chunks = (16 - row0) * 8;
+  for (int i = lane; i < chunks * BOXES; i += 32) {
+    const int b = i / chunks, c = i % chunks;
+    sts128(page + b * 2048 + row0 * 128 + c * 16, 0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------------------

@@ -1,4 +1,5 @@
-// pa_prefill.cuh -- paged (chunked) prefill attention on sm_100a.
+// pa_prefill.cuh -- paged (chunked) prefill attention on the sm_100a tensor
+// cores (tcgen05, accumulators in tensor memory).
 //
 // "vLLM PagedAttention 原理与源码深度解析" §8.1 (Chunked Prefill): a long prompt
 // is processed a chunk of tokens per step, so a step holds sequences with
@@ -7,76 +8,133 @@
 // already in the paged cache) sits at position ctx - q_len + i and attends
 // causally to tokens 0..pos.
 //
-// Work item: (sequence, KV head, tile of query tokens).  Its rows are the
-// tile's tokens x the G query heads of the KV head, token-major, at most 64:
-// warp w owns rows 16w..16w+15 as one mma tile, so -- unlike decode -- every
-// warp reads every page and no merge between warps is needed.  The pages go
-// through one ring of NST stages shared by the CTA: warp 0 holds the block
-// ids (32 per window, one per lane) and its lane 0 issues the TMA loads; each
-// page is released by a CTA barrier once all warps have used it.  The page
-// step is the GQA tensor-core step with a token limit per row (pos + 1), so
-// the causal mask costs nothing extra; a warp skips pages past all its rows.
+// Work item: (sequence, KV head, tile of 128/G query tokens).  Its 128 rows are
+// the tile's tokens x the G query heads of the KV head, token-major -- the M of
+// one 128-row MMA.  Keys go in blocks of 128 (8 pages of 16):
+//   S  = Q K^T      128 x 128, fp32 in tensor memory (two buffers)
+//   P  = 2^(S*scale*log2 e - m)   by four softmax warps, thread r = row r,
+//                                 written to shared memory as the next A operand
+//   O += P V        128 x D,   fp32 in tensor memory
+// Warp roles: warps 0-3 softmax and epilogue, warp 4 TMA (Q once; the K and V
+// pages of each block through rings of NST stages), warp 5 issues the MMAs.
+// The causal mask is a per-row key limit (pos + 1) applied to S; blocks past
+// the tile's last key are never loaded.  O is rescaled only when a row's
+// running maximum grows by more than 2^8 (the reference maximum may lag the
+// true one by that much: P <= 2^8 stays exact in the 16-bit operand and the
+// final 1/l uses the same reference).  bf16 P enters P V as a hi + lo pair of
+// bf16 products (16 bits of P); fp16 P is rounded once and l sums the rounded
+// values.
 #pragma once
 
 #include "pa_decode.cuh"
+#include "pa_umma.cuh"
 
 namespace pa {
 
 constexpr unsigned kErrQuery = 7;
+constexpr int kPrefillRows = 128;                   // query rows per CTA = MMA M
+constexpr int kPrefillKeys = 128;                   // keys per block = S tile N
+constexpr int kPrefillPages = kPrefillKeys / kPage; // 8 pages per block
+constexpr int kPrefillThreads = 192;                // 4 softmax warps, TMA warp, MMA warp
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 0;                      // O: columns [0, D)
+constexpr uint32_t kTmemS = 128;                    // S buffers: [128, 256) and [256, 384)
+constexpr float kRescaleSlack = 8.f;                // log2 units
 
 struct PrefillArgs {
-  const uint16_t* query;        // [T, H, D]
   uint16_t* out;                // [T, H, D]
   const int32_t* block_tables;  // [S, MB]
   const int32_t* context_lens;  // [S]
   const int32_t* query_starts;  // [S + 1]
   float scale_log2;
+  int num_seqs;
+  int num_tokens;               // T
   int num_heads;
   int num_kv_heads;
   int group;
   int max_blocks_per_seq;
   int num_blocks;
-  int tile_tokens;              // query tokens per CTA (64 / group)
+  int tile_tokens;              // query tokens per CTA (128 / group, rounded down)
   int tiles_per_seq;            // ceil(max_query_len / tile_tokens)
 };
 
-template <int D, int NST>
+template <int D, bool BF16>
 struct PrefillSmem {
-  static constexpr int kPageBytes = kPage * D * 2;
-  static constexpr int kStageBytes = 2 * kPageBytes;
-  static constexpr int kBoxesPerRow = D * 2 / 128;
-  static constexpr int kBarOffset = NST * kStageBytes;
-  static constexpr int kBytes = kBarOffset + NST * 8;
+  static constexpr int NST = D == 64 ? 4 : 2;       // K (and V) blocks in flight
+  static constexpr int kSlabs = D / 64;             // 64-element column slabs
+  static constexpr int kSlab = 128 * 128;           // 128 rows x 128 B
+  static constexpr int kQ = 0;
+  static constexpr int kP = kQ + kSlabs * kSlab;    // P (hi): 128 rows x 128 keys
+  static constexpr int kPlo = kP + 2 * kSlab;       // P lo (bf16 only)
+  static constexpr int kStage = kSlabs * kSlab;     // one block of K (or V)
+  static constexpr int kK = kPlo + (BF16 ? 2 * kSlab : 0);
+  static constexpr int kV = kK + NST * kStage;
+  static constexpr int kBarQ = kV + NST * kStage;
+  static constexpr int kBarKFull = kBarQ + 8;
+  static constexpr int kBarKEmpty = kBarKFull + 8 * NST;
+  static constexpr int kBarVFull = kBarKEmpty + 8 * NST;
+  static constexpr int kBarVEmpty = kBarVFull + 8 * NST;
+  static constexpr int kBarS = kBarVEmpty + 8 * NST;   // two
+  static constexpr int kBarP = kBarS + 16;
+  static constexpr int kBarO = kBarP + 8;
+  static constexpr int kBarDrain = kBarO + 8;
+  static constexpr int kTmemSlot = kBarDrain + 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kBytes = kAbort + 4;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-template <int D, int NST, bool BF16>
-__global__ void __launch_bounds__(kThreads)
-    paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
+// Bounded barrier wait that also gives up as soon as another role of the CTA
+// has given up (the shared abort flag); the first to time out records it.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
+                                              volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      record_error(kErrWaitTimeout, blockIdx.x);
+      return false;
+    }
+  }
+  return true;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    paged_prefill_kernel(const __grid_constant__ CUtensorMap qmap,
+                         const __grid_constant__ CUtensorMap kmap,
                          const __grid_constant__ CUtensorMap vmap, const PrefillArgs a) {
-  using L = PrefillSmem<D, NST>;
-  using Warp = MmaWarp<D, BF16, true>;
+  using L = PrefillSmem<D, BF16>;
+  constexpr int NST = L::NST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_addr(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  prefetch_tensormap(&kmap);
-  prefetch_tensormap(&vmap);
+  if (warp == 4 && lane == 0) {
+    prefetch_tensormap(&qmap);
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+  }
   pdl_launch_dependents();
   pdl_wait();
 
+  // ---- work item: the last tiles of every sequence (most keys) start first ----
+  const int per_tile = a.num_seqs * a.num_kv_heads;
   int item = blockIdx.x;
-  const int tile = item % a.tiles_per_seq;
-  item /= a.tiles_per_seq;
+  const int tile = a.tiles_per_seq - 1 - item / per_tile;
+  item %= per_tile;
   const int kvh = item % a.num_kv_heads;
   const int s = item / a.num_kv_heads;
   const int G = a.group;
 
   const int q0 = a.query_starts[s];
   const int q_len = a.query_starts[s + 1] - q0;
-  int ctx = a.context_lens[s];
+  const int ctx = a.context_lens[s];
   const int cap = a.max_blocks_per_seq * kPage;
-  if (q_len < 0 || q_len > ctx || ctx > cap) {
+  if (q0 < 0 || q_len < 0 || q0 > a.num_tokens - q_len || q_len > ctx || ctx > cap) {
     if (threadIdx.x == 0 && kvh == 0 && tile == 0) record_error(kErrQuery, s);
     return;
   }
@@ -84,133 +142,301 @@ __global__ void __launch_bounds__(kThreads)
   if (t_begin >= q_len) return;
   const int t_end = min(t_begin + a.tile_tokens, q_len);
   const int nrows = (t_end - t_begin) * G;
-  const int pos_base = ctx - q_len + t_begin;   // position of the tile's first token
-  const int n_pages = (pos_base + (t_end - t_begin) - 1) / kPage + 1;
+  const int pos_base = ctx - q_len + t_begin;     // position of the tile's first token
+  const int lim_max = pos_base + (t_end - t_begin);
+  const int n_pages = (lim_max + kPage - 1) / kPage;
+  const int nkb = (n_pages + kPrefillPages - 1) / kPrefillPages;
+  const int q_rows = a.tile_tokens * G;           // rows the Q box fills
 
-  const uint32_t stage0 = smem_addr(smem);
-  const uint32_t bar0 = smem_addr(smem + L::kBarOffset);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NST; ++i) mbar_init(bar0 + i * 8, 1);
+    mbar_init(sb + L::kBarQ, 1);
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(sb + L::kBarKFull + 8 * i, 1);
+      mbar_init(sb + L::kBarKEmpty + 8 * i, 1);
+      mbar_init(sb + L::kBarVFull + 8 * i, 1);
+      mbar_init(sb + L::kBarVEmpty + 8 * i, 1);
+    }
+    mbar_init(sb + L::kBarS, 1);
+    mbar_init(sb + L::kBarS + 8, 1);
+    mbar_init(sb + L::kBarP, 4 * 32);
+    mbar_init(sb + L::kBarO, 1);
+    mbar_init(sb + L::kBarDrain, 1);
+    *abort_flag = 0;
     fence_barrier_init();
   }
+  if (warp == 5) tmem_alloc(sb + L::kTmemSlot, kTmemCols);
+  if (warp < 4 && q_rows < kPrefillRows) {
+    // rows no Q box covers are zero (they are masked, but must not be NaN)
+    const int chunks = (kPrefillRows - q_rows) * 8;
+    for (int i = threadIdx.x; i < chunks * L::kSlabs; i += 128) {
+      const int b = i / chunks, c = i % chunks;
+      sts128(sb + L::kQ + b * L::kSlab + q_rows * 128 + c * 16, 0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
+  tmem_fence_before_sync();
   __syncthreads();
+  tmem_fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlot);
 
-  // ---- block ids (warp 0): lane j holds page win*32 + j ----
-  const int32_t* bt = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
-  auto load_ids = [&](int w) -> int {
-    const int k = w * 32 + lane;
-    if (k >= n_pages) return -1;
-    int id = bt[k];
-    if (id < 0 || id >= a.num_blocks) {
-      record_error(kErrBlockId, static_cast<long long>(s) * a.max_blocks_per_seq + k);
-      id = -1;
-    }
-    return id;
-  };
-  int win = 0, ids_cur = -1, ids_next = -1;
-  auto issue = [&](int k) {  // warp 0 only
-    const int src = ((k >> 5) == win) ? ids_cur : ids_next;
-    const int id = __shfl_sync(0xffffffffu, src, k & 31);
+  if (warp == 4) {
+    // ================= TMA producer =================
     if (lane == 0) {
-      const int st = k % NST;
-      const uint32_t bar = bar0 + st * 8;
-      const uint32_t dk = stage0 + st * L::kStageBytes;
-      const uint32_t dv = dk + L::kPageBytes;
-      mbar_arrive_expect_tx(bar, L::kStageBytes);
+      mbar_arrive_expect_tx(sb + L::kBarQ, L::kSlabs * q_rows * 128);
 #pragma unroll
-      for (int b = 0; b < L::kBoxesPerRow; ++b)
-        tma_load_4d(dk + b * kBoxBytes, &kmap, bar, 0, b, kvh, id * kPage);
-#pragma unroll
-      for (int b = 0; b < L::kBoxesPerRow; ++b)
-        tma_load_4d(dv + b * kBoxBytes, &vmap, bar, 0, b, kvh, id * kPage);
+      for (int b = 0; b < L::kSlabs; ++b)
+        tma_load_4d(sb + L::kQ + b * L::kSlab, &qmap, sb + L::kBarQ, 0, b, kvh * G,
+                    q0 + t_begin);
     }
-  };
-  if (warp == 0) {
-    ids_cur = load_ids(0);
-    ids_next = n_pages > 32 ? load_ids(1) : -1;
-    const int pre = n_pages < NST ? n_pages : NST;
-    for (int k = 0; k < pre; ++k) issue(k);
-  }
-
-  // ---- this warp's rows: r = token * G + head; lane rows r0, r1 = r0 + 8 ----
-  Warp st;
-  const int r0 = warp * 16 + (lane >> 2), r1 = r0 + 8, tig = lane & 3;
-  {
-    const uint16_t* qa0 = a.query + (static_cast<size_t>(q0 + t_begin + r0 / G) * a.num_heads +
-                                     kvh * G + r0 % G) * D;
-    const uint16_t* qa1 = a.query + (static_cast<size_t>(q0 + t_begin + r1 / G) * a.num_heads +
-                                     kvh * G + r1 % G) * D;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const int klo = kk * 16 + tig * 2, khi = klo + 8;
-      st.qa[kk][0] = r0 < nrows ? *reinterpret_cast<const uint32_t*>(qa0 + klo) : 0u;
-      st.qa[kk][1] = r1 < nrows ? *reinterpret_cast<const uint32_t*>(qa1 + klo) : 0u;
-      st.qa[kk][2] = r0 < nrows ? *reinterpret_cast<const uint32_t*>(qa0 + khi) : 0u;
-      st.qa[kk][3] = r1 < nrows ? *reinterpret_cast<const uint32_t*>(qa1 + khi) : 0u;
-    }
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) st.acc[n][0] = st.acc[n][1] = st.acc[n][2] = st.acc[n][3] = 0.f;
-    st.m[0] = st.m[1] = -INFINITY;
-    st.l[0] = st.l[1] = 0.f;
-  }
-  // keys j < lim take part: lim = position + 1 (0 for a padding row)
-  const int lim0 = r0 < nrows ? pos_base + r0 / G + 1 : 0;
-  const int lim1 = r1 < nrows ? pos_base + r1 / G + 1 : 0;
-  int warp_lim = max(lim0, lim1);
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) warp_lim = max(warp_lim, __shfl_xor_sync(0xffffffffu, warp_lim, o));
-
-  // ---- every warp walks every page ----
-  bool ok = true;
-  for (int k = 0; k < n_pages; ++k) {
-    const int stg = k % NST;
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar0 + stg * 8, (k / NST) & 1))) {
-      if (lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
-      ok = false;
-    }
-    if (__syncthreads_or(!ok)) {
-      ok = false;
-      break;  // every thread leaves the loop together
-    }
-    if (k * kPage < warp_lim) {
-      const uint32_t kb = stage0 + stg * L::kStageBytes;
-      st.page_rows(kb, kb + L::kPageBytes, k * kPage, lim0, lim1, a.scale_log2, lane);
-    }
-    __syncthreads();  // the stage is free again
-    if (warp == 0 && k + NST < n_pages) {
-      const int nk = k + NST;
-      if ((nk & 31) == 0 && (nk >> 5) != win) {
-        ++win;
-        ids_cur = ids_next;
-        ids_next = n_pages > (win + 1) * 32 ? load_ids(win + 1) : -1;
+    const int32_t* bt = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
+    int k_issued = 0, v_issued = 0;
+    bool ok = true;
+    for (int j = 0; j < nkb; ++j) {
+      const int st = j % NST;
+      const uint32_t par = ((j / NST) & 1) ^ 1;
+      int id = -1;
+      if (lane < kPrefillPages) {
+        const int pg = j * kPrefillPages + lane;
+        if (pg < n_pages) {
+          id = bt[pg];
+          if (id < 0 || id >= a.num_blocks) {
+            record_error(kErrBlockId, static_cast<long long>(s) * a.max_blocks_per_seq + pg);
+            id = -1;   // a fully out-of-range box: zeros
+          }
+        }
       }
-      issue(nk);
+      if (j >= NST) ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarKEmpty + 8 * st, par,
+                                                               abort_flag));
+      if (!ok) break;
+      const uint32_t kst = sb + L::kK + st * L::kStage;
+      if (lane == 0) mbar_arrive_expect_tx(sb + L::kBarKFull + 8 * st, L::kStage);
+#pragma unroll
+      for (int p = 0; p < kPrefillPages; ++p) {
+        const int idp = __shfl_sync(0xffffffffu, id, p);
+        if (lane == 0) {
+#pragma unroll
+          for (int b = 0; b < L::kSlabs; ++b)
+            tma_load_4d(kst + b * L::kSlab + p * 2048, &kmap, sb + L::kBarKFull + 8 * st, 0, b,
+                        kvh, idp * kPage);
+        }
+      }
+      k_issued = j + 1;
+      if (j >= NST) ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarVEmpty + 8 * st, par,
+                                                               abort_flag));
+      if (!ok) break;
+      const uint32_t vst = sb + L::kV + st * L::kStage;
+      if (lane == 0) mbar_arrive_expect_tx(sb + L::kBarVFull + 8 * st, L::kStage);
+#pragma unroll
+      for (int p = 0; p < kPrefillPages; ++p) {
+        const int idp = __shfl_sync(0xffffffffu, id, p);
+        if (lane == 0) {
+#pragma unroll
+          for (int b = 0; b < L::kSlabs; ++b)
+            tma_load_4d(vst + b * L::kSlab + p * 2048, &vmap, sb + L::kBarVFull + 8 * st, 0, b,
+                        kvh, idp * kPage);
+        }
+      }
+      v_issued = j + 1;
+    }
+    // every load issued lands before the CTA can exit (after an abort some were
+    // never consumed); in the normal path these phases have long completed
+    if (!mbar_wait_bounded(sb + L::kBarQ, 0) && lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
+    for (int j = max(0, k_issued - NST); j < k_issued; ++j)
+      mbar_wait_bounded(sb + L::kBarKFull + 8 * (j % NST), (j / NST) & 1);
+    for (int j = max(0, v_issued - NST); j < v_issued; ++j)
+      mbar_wait_bounded(sb + L::kBarVFull + 8 * (j % NST), (j / NST) & 1);
+  } else if (warp == 5) {
+    // ================= MMA issuer =================
+    constexpr uint32_t kIdS = umma_idesc_f16(BF16, kPrefillRows, kPrefillKeys, false);
+    constexpr uint32_t kIdO = umma_idesc_f16(BF16, kPrefillRows, D, true);
+    auto issue_s = [&](int j) {   // S_j = Q K_j^T into buffer j & 1
+      const uint32_t kst = sb + L::kK + (j % NST) * L::kStage;
+      const uint32_t d = tmem + kTmemS + static_cast<uint32_t>(j & 1) * kPrefillKeys;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * L::kSlab + (kk & 3) * 32;
+        umma_f16_ss(d, umma_desc_sw128(sb + L::kQ + off, 16, 1024),
+                    umma_desc_sw128(kst + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(sb + L::kBarS + 8 * (j & 1));
+      umma_commit(sb + L::kBarKEmpty + 8 * (j % NST));
+    };
+    bool ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarQ, 0, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarKFull, 0, abort_flag));
+    if (ok) {
+      tmem_fence_after_sync();
+      if (lane == 0) issue_s(0);
+      __syncwarp();
+    }
+    const int last_page = (ctx - 1) / kPage;
+    const int tail_row = ctx % kPage;          // first row past the context in the last page
+    for (int j = 0; ok && j < nkb; ++j) {
+      if (j + 1 < nkb) {
+        const int st1 = (j + 1) % NST;
+        ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarKFull + 8 * st1,
+                                                   ((j + 1) / NST) & 1, abort_flag));
+        if (!ok) break;
+        tmem_fence_after_sync();
+        if (lane == 0) issue_s(j + 1);
+        __syncwarp();
+      }
+      const int st = j % NST;
+      ok = __all_sync(0xffffffffu,
+                      wait_or_abort(sb + L::kBarVFull + 8 * st, (j / NST) & 1, abort_flag));
+      if (!ok) break;
+      const uint32_t vst = sb + L::kV + st * L::kStage;
+      const int pages_here = min(kPrefillPages, n_pages - j * kPrefillPages);
+      const int lp = last_page - j * kPrefillPages;
+      if (tail_row != 0 && lp >= 0 && lp < pages_here) {
+        // V rows past the context may hold anything; P is 0 there, and 0 * NaN
+        // must not reach O
+        const int chunks = (kPage - tail_row) * 8;
+        for (int i = lane; i < chunks * L::kSlabs; i += 32) {
+          const int b = i / chunks, c = i % chunks;
+          sts128(vst + b * L::kSlab + lp * 2048 + tail_row * 128 + c * 16, 0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarP, j & 1, abort_flag));
+      if (!ok) break;
+      tmem_fence_after_sync();
+      if (lane == 0) {
+        for (int k = 0; k < pages_here; ++k) {
+          const uint32_t poff = (k >> 2) * L::kSlab + (k & 3) * 32;
+          const uint64_t bd = umma_desc_sw128(vst + k * 2048, L::kSlab, 1024);
+          umma_f16_ss(tmem + kTmemO, umma_desc_sw128(sb + L::kP + poff, 16, 1024), bd, kIdO,
+                      (j > 0 || k > 0) ? 1u : 0u);
+          if constexpr (BF16)
+            umma_f16_ss(tmem + kTmemO, umma_desc_sw128(sb + L::kPlo + poff, 16, 1024), bd, kIdO,
+                        1u);
+        }
+        umma_commit(sb + L::kBarO);
+        umma_commit(sb + L::kBarVEmpty + 8 * st);
+      }
+      __syncwarp();
+    }
+    // every MMA issued has completed before tensor memory is freed
+    if (lane == 0) umma_commit(sb + L::kBarDrain);
+    __syncwarp();
+    if (!mbar_wait_bounded(sb + L::kBarDrain, 0) && lane == 0)
+      record_error(kErrWaitTimeout, blockIdx.x);
+  } else {
+    // ================= softmax (row = threadIdx.x = TMEM lane) =================
+    const int row = threadIdx.x;
+    const int lim = row < nrows ? pos_base + row / G + 1 : 0;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float sl2 = a.scale_log2;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkb; ++j) {
+      ok = __all_sync(0xffffffffu,
+                      wait_or_abort(sb + L::kBarS + 8 * (j & 1), (j >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tmem_fence_after_sync();
+      float p[kPrefillKeys];
+#pragma unroll
+      for (int c = 0; c < kPrefillKeys / 32; ++c)
+        tmem_ld32(t_lane + kTmemS + static_cast<uint32_t>(j & 1) * kPrefillKeys + 32 * c,
+                  *reinterpret_cast<float(*)[32]>(&p[32 * c]));
+      const int kbase = j * kPrefillKeys;
+      float mx = -INFINITY;
+      if (kbase + kPrefillKeys <= lim) {
+#pragma unroll
+        for (int c = 0; c < kPrefillKeys; ++c) {
+          p[c] *= sl2;
+          mx = fmaxf(mx, p[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kPrefillKeys; ++c) {
+          p[c] = kbase + c < lim ? p[c] * sl2 : -INFINITY;
+          mx = fmaxf(mx, p[c]);
+        }
+      }
+      const float m_new = fmaxf(m_ref, mx);
+      const bool need = m_new > m_ref + kRescaleSlack;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2(m_ref - m_new);   // 0 when m_ref is still -inf
+        m_ref = m_new;
+      }
+      l *= alpha;
+      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+#pragma unroll
+      for (int c = 0; c < kPrefillKeys; ++c) p[c] = ex2(p[c] - m_use);
+
+      if (j > 0) {
+        // P V of the previous block is done: O holds it and the P buffers are free
+        ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarO, (j - 1) & 1, abort_flag));
+        if (!ok) break;
+        tmem_fence_after_sync();
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(t_lane + kTmemO + 32 * c, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(t_lane + kTmemO + 32 * c, o);
+          }
+        }
+      }
+      // P (and l) -> shared memory, 16-byte chunk c of the row at c ^ (row % 8)
+#pragma unroll
+      for (int c = 0; c < kPrefillKeys / 8; ++c) {
+        uint32_t h[4], lo[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float x0 = p[8 * c + 2 * i], x1 = p[8 * c + 2 * i + 1];
+          h[i] = pack2<BF16>(x0, x1);
+          const float2 hf = unpack2<BF16>(h[i]);
+          if constexpr (BF16) {
+            lo[i] = pack2<true>(x0 - hf.x, x1 - hf.y);
+            l += x0 + x1;
+          } else {
+            l += hf.x + hf.y;
+          }
+        }
+        const uint32_t off = (c >> 3) * L::kSlab + row * 128 + (((c & 7) ^ (row & 7)) << 4);
+        sts128(sb + L::kP + off, h[0], h[1], h[2], h[3]);
+        if constexpr (BF16) sts128(sb + L::kPlo + off, lo[0], lo[1], lo[2], lo[3]);
+      }
+      fence_proxy_async_smem();
+      tmem_fence_before_sync();
+      mbar_arrive(sb + L::kBarP);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarO, (nkb - 1) & 1, abort_flag));
+    if (ok) {
+      tmem_fence_after_sync();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint16_t* o_row = a.out + (static_cast<size_t>(q0 + t_begin + row / G) * a.num_heads +
+                                 kvh * G + row % G) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tmem_ld32(t_lane + kTmemO + 32 * c, o);
+        if (row < nrows) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 v;
+            v.x = pack2<BF16>(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+            v.y = pack2<BF16>(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+            v.z = pack2<BF16>(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+            v.w = pack2<BF16>(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+            *reinterpret_cast<uint4*>(o_row + 32 * c + 8 * q) = v;
+          }
+        }
+      }
     }
   }
 
-  // ---- finish this warp's rows ----
-  float l0 = st.l[0], l1 = st.l[1];
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  const float inv0 = (ok && l0 > 0.f) ? 1.f / l0 : 0.f;
-  const float inv1 = (ok && l1 > 0.f) ? 1.f / l1 : 0.f;
-  if (r0 < nrows) {
-    uint16_t* o = a.out + (static_cast<size_t>(q0 + t_begin + r0 / G) * a.num_heads + kvh * G +
-                           r0 % G) * D;
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n)
-      *reinterpret_cast<uint32_t*>(o + n * 8 + tig * 2) =
-          pack2<BF16>(st.acc[n][0] * inv0, st.acc[n][1] * inv0);
-  }
-  if (r1 < nrows) {
-    uint16_t* o = a.out + (static_cast<size_t>(q0 + t_begin + r1 / G) * a.num_heads + kvh * G +
-                           r1 % G) * D;
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n)
-      *reinterpret_cast<uint32_t*>(o + n * 8 + tig * 2) =
-          pack2<BF16>(st.acc[n][2] * inv1, st.acc[n][3] * inv1);
+  tmem_fence_before_sync();
+  __syncthreads();
+  if (warp == 5) {
+    tmem_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 

@@ -142,6 +142,9 @@ __global__ void __launch_bounds__(kThreads)
   int most_pages = my_pages;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) most_pages = max(most_pages, __shfl_xor_sync(~0u, most_pages, o));
+  int most_ctx = my_ctx;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) most_ctx = max(most_ctx, __shfl_xor_sync(~0u, most_ctx, o));
   const int Pn = min(P, most_pages);                 // prefix pages anyone needs
   const int my_tail = lane < members ? max(0, my_pages - P) : 0;
   int incl = my_tail;                                // inclusive prefix sum of tails
@@ -288,6 +291,11 @@ __global__ void __launch_bounds__(kThreads)
     const int lim0 = (live0 && (member < 0 || member == mem0)) ? ctx0 : 0;
     const int lim1 = (live1 && (member < 0 || member == mem1)) ? ctx1 : 0;
     const uint32_t kb = stage0 + stg * L::kStageBytes;
+    // rows of this page no row of the item reads: past the owner's context
+    // (a tail page) or past every member's (the prefix)
+    const int page_lim = member >= 0 ? __shfl_sync(~0u, my_ctx, member) : most_ctx;
+    if (entry * kPage + kPage > page_lim && page_lim > entry * kPage)
+      zero_page_tail<L::kBoxesPerRow>(kb + L::kPageBytes, page_lim - entry * kPage, lane);
     st.page_rows(kb, kb + L::kPageBytes, entry * kPage, lim0, lim1, a.scale_log2, lane);
     __syncwarp();
     if (k + NST < my_count) issue(k + NST);

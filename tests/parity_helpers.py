@@ -88,6 +88,26 @@ def gpu_step(batch: workloads.DecodeBatch, write: bool = True, partition_size: i
     return out, parts
 
 
+def poison_past_context(batch: workloads.DecodeBatch, key_cache=None, value_cache=None,
+                        fill=float("nan")) -> int:
+    """Fill the cache rows past each sequence's context in its last block with
+    `fill` (NaN, or an E4M3 NaN code for fp8 caches).  Those rows were never
+    written: the oracle never reads them, and the kernels must not let a
+    probability of 0 times a NaN reach the output.  Returns the rows filled."""
+    cfg = batch.cfg
+    kc = batch.key_cache if key_cache is None else key_cache
+    vc = batch.value_cache if value_cache is None else value_cache
+    bt = batch.block_tables.cpu().numpy()
+    n = 0
+    for s, c in enumerate(batch.context_lens.cpu().tolist()):
+        if c % cfg.block_size:
+            blk = int(bt[s, (c - 1) // cfg.block_size])
+            kc[blk, c % cfg.block_size:] = fill
+            vc[blk, c % cfg.block_size:] = fill
+            n += cfg.block_size - c % cfg.block_size
+    return n
+
+
 def to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 

@@ -14,7 +14,7 @@ import oracle as oracle_mod
 from paged_kv_cache_444_b200 import (SplitWorkspace, pa_check_error, pa_decode_fp8,
                                      pa_decode_split_fp8, pa_reduce, pa_reshape_and_cache_fp8,
                                      workloads)
-from parity_helpers import TOL, bits, ocode, to_f64
+from parity_helpers import TOL, bits, ocode, poison_past_context, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -91,6 +91,32 @@ def test_fp8_split_matches_oracle(name, ps, cuda_device, oracle_lib):
     pa_check_error()
     err = np.max(np.abs(to_f64(out) - ref))
     assert err <= TOL[cfg.dtype], f"{name} split {ps}: {err:.3e}"
+
+
+@pytest.mark.parametrize("split", [0, 64])
+@pytest.mark.parametrize("name", ["mha_f16", "gqa_bf16", "gqa16_bf16"])
+def test_fp8_nan_codes_past_context_do_not_leak(name, split, cuda_device, oracle_lib):
+    """E4M3 NaN codes (0x7f) in the never-written rows past each context."""
+    cfg = CASES[name]
+    b, kc, vc = _fp8_batch(cfg, cuda_device)
+    assert poison_past_context(b, kc, vc, fill=0x7F) > 0
+    ref, _, _ = _oracle(oracle_lib, b, kc, vc)
+    pa_reshape_and_cache_fp8(b.key, b.value, kc, vc, b.slot_mapping, K_SCALE, V_SCALE)
+    out = torch.full_like(b.query, float("nan"))
+    if split:
+        P = (b.block_tables.shape[1] * 16 + split - 1) // split
+        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, cuda_device)
+        pa_decode_split_fp8(ws.tmp_out, ws.max_logits, ws.exp_sums, b.query, kc, vc,
+                            b.block_tables, b.context_lens, cfg.scale, K_SCALE, V_SCALE, split)
+        pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, b.context_lens, split)
+    else:
+        pa_decode_fp8(out, b.query, kc, vc, b.block_tables, b.context_lens, cfg.scale, K_SCALE,
+                      V_SCALE)
+    torch.cuda.synchronize()
+    pa_check_error()
+    g = to_f64(out)
+    assert np.isfinite(g).all()
+    assert np.max(np.abs(g - ref)) <= TOL[cfg.dtype]
 
 
 @pytest.mark.parametrize("name", ["mha_f16", "gqa_bf16"])

@@ -7,7 +7,8 @@ import pytest
 import torch
 
 from paged_kv_cache_444_b200 import PagedAttentionError, pa_check_error, workloads
-from parity_helpers import TOL, HostCopy, bits, gpu_step, max_err, oracle_step, to_f64
+from parity_helpers import (TOL, HostCopy, bits, gpu_step, max_err, oracle_step,
+                            poison_past_context, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -229,6 +230,25 @@ def test_many_sequences_natural_order(dev, oracle_lib):
     out, _ = gpu_step(batch)
     pa_check_error()
     _check_close(out, ref, cfg, "natural order")
+
+
+@pytest.mark.parametrize("mode", ["single", "split64", "shared"])
+@pytest.mark.parametrize("name", ["mha_small", "gqa_small", "gqa16_two_rows", "d64_gqa2",
+                                  "shared_small"])
+def test_nan_rows_past_context_do_not_leak(name, mode, dev, oracle_lib):
+    """Cache rows past a sequence's context (never written) hold NaN: the
+    output still matches the oracle, which never reads them."""
+    if mode == "shared" and name != "shared_small":
+        pytest.skip("shared-prefix layout only")
+    cfg = SMALL[name]
+    batch = workloads.make_batch(cfg, dev)
+    assert poison_past_context(batch) > 0
+    host = HostCopy(batch)
+    ref, _, _ = oracle_step(oracle_lib, host)
+    out, _ = gpu_step(batch, partition_size=64 if mode == "split64" else 0,
+                      shared_prefix=mode == "shared")
+    pa_check_error()
+    _check_close(out, ref, cfg, f"{name} {mode} with NaN past the context")
 
 
 def _regroup(batch, starts, prefix):
