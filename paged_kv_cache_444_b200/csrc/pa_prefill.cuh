@@ -11,19 +11,22 @@
 // Work item: (sequence, KV head, tile of 128/G query tokens).  Its 128 rows are
 // the tile's tokens x the G query heads of the KV head, token-major -- the M of
 // one 128-row MMA.  Keys go in blocks of 128 (8 pages of 16):
-//   S  = Q K^T      128 x 128, fp32 in tensor memory (two buffers)
+//   S  = Q K^T      128 x 128 fp32 in tensor memory (three buffers), Q and K
+//                   from shared memory
 //   P  = 2^(S*scale*log2 e - m)   by four softmax warps, thread r = row r,
-//                                 written to shared memory as the next A operand
-//   O += P V        128 x D,   fp32 in tensor memory
-// Warp roles: warps 0-3 softmax and epilogue, warp 4 TMA (Q once; the K and V
-// pages of each block through rings of NST stages), warp 5 issues the MMAs.
-// The causal mask is a per-row key limit (pos + 1) applied to S; blocks past
-// the tile's last key are never loaded.  O is rescaled only when a row's
-// running maximum grows by more than 2^8 (the reference maximum may lag the
-// true one by that much: P <= 2^8 stays exact in the 16-bit operand and the
-// final 1/l uses the same reference).  bf16 P enters P V as a hi + lo pair of
-// bf16 products (16 bits of P); fp16 P is rounded once and l sums the rounded
-// values.
+//                   written back over S in tensor memory as 16-bit pairs
+//   O += P V        128 x D fp32 in tensor memory, P from tensor memory and V
+//                   from shared memory
+// Keeping P in tensor memory leaves shared-memory bandwidth to the K and V
+// operands.  Warp roles: warps 0-3 softmax and epilogue, warp 4 TMA (Q once;
+// the K and V pages of each block through rings of NST stages), warp 5 issues
+// the MMAs.  The causal mask is a per-row key limit (pos + 1) applied to S;
+// blocks past the tile's last key are never loaded.  O is rescaled only when
+// a row's running maximum grows by more than 2^8 (the reference maximum may
+// lag the true one by that much: P <= 2^8 stays exact in the 16-bit operand
+// and the final 1/l uses the same reference).  bf16 P enters P V as a hi + lo
+// pair of bf16 products (16 bits of P); fp16 P is rounded once and l sums the
+// rounded values.
 #pragma once
 
 #include "pa_decode.cuh"
@@ -38,7 +41,8 @@ constexpr int kPrefillPages = kPrefillKeys / kPage; // 8 pages per block
 constexpr int kPrefillThreads = 192;                // 4 softmax warps, TMA warp, MMA warp
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;                      // O: columns [0, D)
-constexpr uint32_t kTmemS = 128;                    // S buffers: [128, 256) and [256, 384)
+constexpr uint32_t kTmemS = 128;                    // S / P buffers at 128, 256, 384
+constexpr int kSBufs = 3;
 constexpr float kRescaleSlack = 8.f;                // log2 units
 
 struct PrefillArgs {
@@ -60,22 +64,20 @@ struct PrefillArgs {
 
 template <int D, bool BF16>
 struct PrefillSmem {
-  static constexpr int NST = D == 64 ? 4 : 2;       // K (and V) blocks in flight
+  static constexpr int NST = D == 64 ? 4 : 3;       // K (and V) blocks in flight
   static constexpr int kSlabs = D / 64;             // 64-element column slabs
   static constexpr int kSlab = 128 * 128;           // 128 rows x 128 B
   static constexpr int kQ = 0;
-  static constexpr int kP = kQ + kSlabs * kSlab;    // P (hi): 128 rows x 128 keys
-  static constexpr int kPlo = kP + 2 * kSlab;       // P lo (bf16 only)
   static constexpr int kStage = kSlabs * kSlab;     // one block of K (or V)
-  static constexpr int kK = kPlo + (BF16 ? 2 * kSlab : 0);
+  static constexpr int kK = kQ + kSlabs * kSlab;
   static constexpr int kV = kK + NST * kStage;
   static constexpr int kBarQ = kV + NST * kStage;
   static constexpr int kBarKFull = kBarQ + 8;
   static constexpr int kBarKEmpty = kBarKFull + 8 * NST;
   static constexpr int kBarVFull = kBarKEmpty + 8 * NST;
   static constexpr int kBarVEmpty = kBarVFull + 8 * NST;
-  static constexpr int kBarS = kBarVEmpty + 8 * NST;   // two
-  static constexpr int kBarP = kBarS + 16;
+  static constexpr int kBarS = kBarVEmpty + 8 * NST;   // one per S / P buffer
+  static constexpr int kBarP = kBarS + 8 * kSBufs;
   static constexpr int kBarO = kBarP + 8;
   static constexpr int kBarDrain = kBarO + 8;
   static constexpr int kTmemSlot = kBarDrain + 8;
@@ -157,8 +159,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(sb + L::kBarVFull + 8 * i, 1);
       mbar_init(sb + L::kBarVEmpty + 8 * i, 1);
     }
-    mbar_init(sb + L::kBarS, 1);
-    mbar_init(sb + L::kBarS + 8, 1);
+    for (int i = 0; i < kSBufs; ++i) mbar_init(sb + L::kBarS + 8 * i, 1);
     mbar_init(sb + L::kBarP, 4 * 32);
     mbar_init(sb + L::kBarO, 1);
     mbar_init(sb + L::kBarDrain, 1);
@@ -250,16 +251,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // ================= MMA issuer =================
     constexpr uint32_t kIdS = umma_idesc_f16(BF16, kPrefillRows, kPrefillKeys, false);
     constexpr uint32_t kIdO = umma_idesc_f16(BF16, kPrefillRows, D, true);
-    auto issue_s = [&](int j) {   // S_j = Q K_j^T into buffer j & 1
+    auto issue_s = [&](int j) {   // S_j = Q K_j^T into buffer j % 3
       const uint32_t kst = sb + L::kK + (j % NST) * L::kStage;
-      const uint32_t d = tmem + kTmemS + static_cast<uint32_t>(j & 1) * kPrefillKeys;
+      const uint32_t d = tmem + kTmemS + static_cast<uint32_t>(j % kSBufs) * kPrefillKeys;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * L::kSlab + (kk & 3) * 32;
         umma_f16_ss(d, umma_desc_sw128(sb + L::kQ + off, 16, 1024),
                     umma_desc_sw128(kst + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
       }
-      umma_commit(sb + L::kBarS + 8 * (j & 1));
+      umma_commit(sb + L::kBarS + 8 * (j % kSBufs));
       umma_commit(sb + L::kBarKEmpty + 8 * (j % NST));
     };
     bool ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarQ, 0, abort_flag));
@@ -303,14 +304,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (!ok) break;
       tmem_fence_after_sync();
       if (lane == 0) {
+        // P_j sits in S_j's buffer: hi in its first 64 columns, lo in the next 64
+        const uint32_t pcol = tmem + kTmemS + static_cast<uint32_t>(j % kSBufs) * kPrefillKeys;
         for (int k = 0; k < pages_here; ++k) {
-          const uint32_t poff = (k >> 2) * L::kSlab + (k & 3) * 32;
           const uint64_t bd = umma_desc_sw128(vst + k * 2048, L::kSlab, 1024);
-          umma_f16_ss(tmem + kTmemO, umma_desc_sw128(sb + L::kP + poff, 16, 1024), bd, kIdO,
-                      (j > 0 || k > 0) ? 1u : 0u);
-          if constexpr (BF16)
-            umma_f16_ss(tmem + kTmemO, umma_desc_sw128(sb + L::kPlo + poff, 16, 1024), bd, kIdO,
-                        1u);
+          umma_f16_ts(tmem + kTmemO, pcol + 8 * k, bd, kIdO, (j > 0 || k > 0) ? 1u : 0u);
+          if constexpr (BF16) umma_f16_ts(tmem + kTmemO, pcol + 64 + 8 * k, bd, kIdO, 1u);
         }
         umma_commit(sb + L::kBarO);
         umma_commit(sb + L::kBarVEmpty + 8 * st);
@@ -331,30 +330,34 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkb; ++j) {
+      const uint32_t buf = kTmemS + static_cast<uint32_t>(j % kSBufs) * kPrefillKeys;
       ok = __all_sync(0xffffffffu,
-                      wait_or_abort(sb + L::kBarS + 8 * (j & 1), (j >> 1) & 1, abort_flag));
+                      wait_or_abort(sb + L::kBarS + 8 * (j % kSBufs), (j / kSBufs) & 1, abort_flag));
       if (!ok) break;
       tmem_fence_after_sync();
       float p[kPrefillKeys];
-#pragma unroll
-      for (int c = 0; c < kPrefillKeys / 32; ++c)
-        tmem_ld32(t_lane + kTmemS + static_cast<uint32_t>(j & 1) * kPrefillKeys + 32 * c,
-                  *reinterpret_cast<float(*)[32]>(&p[32 * c]));
+      tmem_ld128(t_lane + buf, p);
+      // logits in log2 units; keys at or past this row's limit are -inf
       const int kbase = j * kPrefillKeys;
-      float mx = -INFINITY;
+      const float2 sl2x2 = make_float2(sl2, sl2);
       if (kbase + kPrefillKeys <= lim) {
 #pragma unroll
-        for (int c = 0; c < kPrefillKeys; ++c) {
-          p[c] *= sl2;
-          mx = fmaxf(mx, p[c]);
+        for (int c = 0; c < kPrefillKeys; c += 2) {
+          const float2 x = fmul2(make_float2(p[c], p[c + 1]), sl2x2);
+          p[c] = x.x;
+          p[c + 1] = x.y;
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < kPrefillKeys; ++c) {
-          p[c] = kbase + c < lim ? p[c] * sl2 : -INFINITY;
-          mx = fmaxf(mx, p[c]);
-        }
+        for (int c = 0; c < kPrefillKeys; ++c) p[c] = kbase + c < lim ? p[c] * sl2 : -INFINITY;
       }
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = p[i];
+#pragma unroll
+      for (int c = 8; c < kPrefillKeys; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], p[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_new = fmaxf(m_ref, mx);
       const bool need = m_new > m_ref + kRescaleSlack;
       float alpha = 1.f;
@@ -364,8 +367,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       l *= alpha;
       const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+      const float2 negm = make_float2(-m_use, -m_use), one2 = make_float2(1.f, 1.f);
 #pragma unroll
-      for (int c = 0; c < kPrefillKeys; ++c) p[c] = ex2(p[c] - m_use);
+      for (int c = 0; c < kPrefillKeys; c += 2) {
+        const float2 x = ffma2(make_float2(p[c], p[c + 1]), one2, negm);
+        p[c] = ex2(x.x);
+        p[c + 1] = ex2(x.y);
+      }
 
       if (j > 0) {
         // P V of the previous block is done: O holds it and the P buffers are free
@@ -383,27 +391,34 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
         }
       }
-      // P (and l) -> shared memory, 16-byte chunk c of the row at c ^ (row % 8)
+      // P (and l) -> this S buffer: keys 2i, 2i+1 packed in column i (hi), and
+      // for bf16 the remainder p - hi in column 64 + i (lo)
+      float2 lsum[4];
 #pragma unroll
-      for (int c = 0; c < kPrefillKeys / 8; ++c) {
-        uint32_t h[4], lo[4];
+      for (int i = 0; i < 4; ++i) lsum[i] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float x0 = p[8 * c + 2 * i], x1 = p[8 * c + 2 * i + 1];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t h[32], lo[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float x0 = p[64 * half + 2 * i], x1 = p[64 * half + 2 * i + 1];
           h[i] = pack2<BF16>(x0, x1);
           const float2 hf = unpack2<BF16>(h[i]);
           if constexpr (BF16) {
-            lo[i] = pack2<true>(x0 - hf.x, x1 - hf.y);
-            l += x0 + x1;
+            const float2 r = ffma2(hf, make_float2(-1.f, -1.f), make_float2(x0, x1));
+            lo[i] = pack2<true>(r.x, r.y);
+            lsum[i & 3].x += x0;
+            lsum[i & 3].y += x1;
           } else {
-            l += hf.x + hf.y;
+            lsum[i & 3].x += hf.x;
+            lsum[i & 3].y += hf.y;
           }
         }
-        const uint32_t off = (c >> 3) * L::kSlab + row * 128 + (((c & 7) ^ (row & 7)) << 4);
-        sts128(sb + L::kP + off, h[0], h[1], h[2], h[3]);
-        if constexpr (BF16) sts128(sb + L::kPlo + off, lo[0], lo[1], lo[2], lo[3]);
+        tmem_st32u(t_lane + buf + 32 * half, h);
+        if constexpr (BF16) tmem_st32u(t_lane + buf + 64 + 32 * half, lo);
       }
-      fence_proxy_async_smem();
+      l += ((lsum[0].x + lsum[0].y) + (lsum[1].x + lsum[1].y)) +
+           ((lsum[2].x + lsum[2].y) + (lsum[3].x + lsum[3].y));
       tmem_fence_before_sync();
       mbar_arrive(sb + L::kBarP);
     }
