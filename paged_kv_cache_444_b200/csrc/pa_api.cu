@@ -824,7 +824,8 @@ pa_status pa_prefill(void* out, const void* query, const void* key_cache, const 
   const int64_t G = num_heads / num_kv_heads;
   const int64_t tile = kPrefillRows / G;                  // G <= 16 checked above
   const int64_t tiles = (max_query_len + tile - 1) / tile;
-  const long long grid = num_seqs * num_kv_heads * tiles;
+  const int64_t pairs = (tiles + 1) / 2;                  // two query tiles per CTA
+  const long long grid = num_seqs * num_kv_heads * pairs;
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
   CUtensorMap qm, km, vm;
   if (!encode_query_map(&qm, query, dtype, num_query_tokens, num_heads, head_dim, G, tile) ||
@@ -845,7 +846,7 @@ pa_status pa_prefill(void* out, const void* query, const void* key_cache, const 
   a.max_blocks_per_seq = static_cast<int>(max_blocks_per_seq);
   a.num_blocks = static_cast<int>(num_blocks);
   a.tile_tokens = static_cast<int>(tile);
-  a.tiles_per_seq = static_cast<int>(tiles);
+  a.pairs_per_seq = static_cast<int>(pairs);
   cudaStream_t s = as_stream(stream);
   const bool bf16 = dtype == PA_BF16;
   if (head_dim == 64)

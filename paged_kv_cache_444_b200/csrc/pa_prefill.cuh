@@ -8,25 +8,32 @@
 // already in the paged cache) sits at position ctx - q_len + i and attends
 // causally to tokens 0..pos.
 //
-// Work item: (sequence, KV head, tile of 128/G query tokens).  Its 128 rows are
-// the tile's tokens x the G query heads of the KV head, token-major -- the M of
-// one 128-row MMA.  Keys go in blocks of 128 (8 pages of 16):
-//   S  = Q K^T      128 x 128 fp32 in tensor memory (three buffers), Q and K
-//                   from shared memory
-//   P  = 2^(S*scale*log2 e - m)   by four softmax warps, thread r = row r,
-//                   written back over S in tensor memory as 16-bit pairs
-//   O += P V        128 x D fp32 in tensor memory, P from tensor memory and V
-//                   from shared memory
-// Keeping P in tensor memory leaves shared-memory bandwidth to the K and V
-// operands.  Warp roles: warps 0-3 softmax and epilogue, warp 4 TMA (Q once;
-// the K and V pages of each block through rings of NST stages), warp 5 issues
-// the MMAs.  The causal mask is a per-row key limit (pos + 1) applied to S;
-// blocks past the tile's last key are never loaded.  O is rescaled only when
-// a row's running maximum grows by more than 2^8 (the reference maximum may
-// lag the true one by that much: P <= 2^8 stays exact in the 16-bit operand
-// and the final 1/l uses the same reference).  bf16 P enters P V as a hi + lo
-// pair of bf16 products (16 bits of P); fp16 P is rounded once and l sums the
-// rounded values.
+// Work item: (sequence, KV head, pair of query tiles A and B).  A tile is
+// 128/G consecutive query tokens x the G query heads of the KV head,
+// token-major: 128 rows, the M of one MMA.  Both tiles walk the same keys in
+// blocks of 128 (8 pages of 16), so every K/V block gathered into shared
+// memory feeds 256 query rows.  Per tile t and block j:
+//   S_t  = Q_t K_j^T    128 x 128 fp32 in tensor memory; Q and K from shared
+//   P_t  = 2^(S_t*scale*log2 e - m)   by the tile's softmax warpgroup (thread
+//                       r = row r), written back over S_t as 16-bit pairs
+//   O_t += P_t V_j      128 x D fp32 in tensor memory; P from tensor memory,
+//                       V from shared memory
+// One warp issues every MMA in the order S_A(j), P_B(j-1) V, S_B(j), P_A(j) V,
+// so each warpgroup's softmax overlaps the other tile's MMAs.  MMAs from one
+// thread run in issue order: S_t(j+1) may overwrite P_t(j) as soon as it is
+// issued after the P V that reads it, and the commit that reports S_t(j+1)
+// also reports that P V done (the softmax may then rescale O_t).  Another warp
+// loads Q once and the K and V pages with TMA through rings of NST stages.
+//
+// The causal mask is a per-row key limit (pos + 1) applied to S; blocks past
+// the pair's last key are never loaded, and V rows past the context are
+// zeroed before use (never written, they may hold anything).  O is rescaled
+// only when a row's running maximum grows by more than 2^8 (the reference
+// maximum may lag the true one by that much: P <= 2^8 stays exact in the
+// 16-bit operand and the final 1/l uses the same reference).  bf16 P enters
+// P V as a hi + lo pair of bf16 products (about 17 bits of P, split with
+// integer rounding so the conversion unit stays free for 2^x); fp16 P is
+// rounded once and l sums the rounded values.
 #pragma once
 
 #include "pa_decode.cuh"
@@ -35,14 +42,15 @@
 namespace pa {
 
 constexpr unsigned kErrQuery = 7;
-constexpr int kPrefillRows = 128;                   // query rows per CTA = MMA M
+constexpr int kPrefillRows = 128;                   // query rows per tile = MMA M
 constexpr int kPrefillKeys = 128;                   // keys per block = S tile N
 constexpr int kPrefillPages = kPrefillKeys / kPage; // 8 pages per block
-constexpr int kPrefillThreads = 192;                // 4 softmax warps, TMA warp, MMA warp
+constexpr int kWarpMma = 8;                         // issues every MMA, owns tensor memory
+constexpr int kWarpTma = 9;                         // Q, K and V loads
+constexpr int kPrefillThreads = 10 * 32;            // + two softmax warpgroups (warps 0-7)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 0;                      // O: columns [0, D)
-constexpr uint32_t kTmemS = 128;                    // S / P buffers at 128, 256, 384
-constexpr int kSBufs = 3;
+constexpr uint32_t kTmemO = 0;                      // O_t: columns [128 t, 128 t + D)
+constexpr uint32_t kTmemS = 256;                    // S_t / P_t: [256 + 128 t, +128)
 constexpr float kRescaleSlack = 8.f;                // log2 units
 
 struct PrefillArgs {
@@ -58,29 +66,29 @@ struct PrefillArgs {
   int group;
   int max_blocks_per_seq;
   int num_blocks;
-  int tile_tokens;              // query tokens per CTA (128 / group, rounded down)
-  int tiles_per_seq;            // ceil(max_query_len / tile_tokens)
+  int tile_tokens;              // query tokens per tile (128 / group, rounded down)
+  int pairs_per_seq;            // ceil(ceil(max_query_len / tile_tokens) / 2)
 };
 
 template <int D, bool BF16>
 struct PrefillSmem {
-  static constexpr int NST = D == 64 ? 4 : 3;       // K (and V) blocks in flight
+  static constexpr int NST = D == 64 ? 4 : 2;       // K (and V) blocks in flight
   static constexpr int kSlabs = D / 64;             // 64-element column slabs
   static constexpr int kSlab = 128 * 128;           // 128 rows x 128 B
-  static constexpr int kQ = 0;
+  static constexpr int kQTile = kSlabs * kSlab;     // one tile of Q
+  static constexpr int kQ = 0;                      // Q_A, then Q_B
   static constexpr int kStage = kSlabs * kSlab;     // one block of K (or V)
-  static constexpr int kK = kQ + kSlabs * kSlab;
+  static constexpr int kK = kQ + 2 * kQTile;
   static constexpr int kV = kK + NST * kStage;
   static constexpr int kBarQ = kV + NST * kStage;
   static constexpr int kBarKFull = kBarQ + 8;
   static constexpr int kBarKEmpty = kBarKFull + 8 * NST;
   static constexpr int kBarVFull = kBarKEmpty + 8 * NST;
   static constexpr int kBarVEmpty = kBarVFull + 8 * NST;
-  static constexpr int kBarS = kBarVEmpty + 8 * NST;   // one per S / P buffer
-  static constexpr int kBarP = kBarS + 8 * kSBufs;
-  static constexpr int kBarO = kBarP + 8;
-  static constexpr int kBarDrain = kBarO + 8;
-  static constexpr int kTmemSlot = kBarDrain + 8;
+  static constexpr int kBarS = kBarVEmpty + 8 * NST;   // per tile: S_t(j) (and P_t(j-1) V) done
+  static constexpr int kBarP = kBarS + 16;             // per tile: P_t(j) written
+  static constexpr int kBarO = kBarP + 16;             // every MMA done
+  static constexpr int kTmemSlot = kBarO + 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
   static constexpr int kAlloc = kBytes + 1024;
@@ -115,7 +123,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sb = smem_addr(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp == 4 && lane == 0) {
+  if (warp == kWarpTma && lane == 0) {
     prefetch_tensormap(&qmap);
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&vmap);
@@ -123,11 +131,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   pdl_launch_dependents();
   pdl_wait();
 
-  // ---- work item: the last tiles of every sequence (most keys) start first ----
-  const int per_tile = a.num_seqs * a.num_kv_heads;
+  // ---- work item: the last tile pairs of every sequence (most keys) first ----
+  const int per_pair = a.num_seqs * a.num_kv_heads;
   int item = blockIdx.x;
-  const int tile = a.tiles_per_seq - 1 - item / per_tile;
-  item %= per_tile;
+  const int pair = a.pairs_per_seq - 1 - item / per_pair;
+  item %= per_pair;
   const int kvh = item % a.num_kv_heads;
   const int s = item / a.num_kv_heads;
   const int G = a.group;
@@ -137,18 +145,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int ctx = a.context_lens[s];
   const int cap = a.max_blocks_per_seq * kPage;
   if (q0 < 0 || q_len < 0 || q0 > a.num_tokens - q_len || q_len > ctx || ctx > cap) {
-    if (threadIdx.x == 0 && kvh == 0 && tile == 0) record_error(kErrQuery, s);
+    if (threadIdx.x == 0 && kvh == 0 && pair == 0) record_error(kErrQuery, s);
     return;
   }
-  const int t_begin = tile * a.tile_tokens;
-  if (t_begin >= q_len) return;
-  const int t_end = min(t_begin + a.tile_tokens, q_len);
-  const int nrows = (t_end - t_begin) * G;
-  const int pos_base = ctx - q_len + t_begin;     // position of the tile's first token
-  const int lim_max = pos_base + (t_end - t_begin);
+  const int tile_a = 2 * pair * a.tile_tokens, tile_b = tile_a + a.tile_tokens;
+  if (tile_a >= q_len) return;
+  const bool has_b = tile_b < q_len;
+  const int last_tok = min((has_b ? tile_b : tile_a) + a.tile_tokens, q_len);  // exclusive
+  const int lim_max = ctx - q_len + last_tok;      // keys the pair's last token sees
   const int n_pages = (lim_max + kPage - 1) / kPage;
   const int nkb = (n_pages + kPrefillPages - 1) / kPrefillPages;
-  const int q_rows = a.tile_tokens * G;           // rows the Q box fills
+  const int q_rows = a.tile_tokens * G;           // rows a Q box fills
 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
   if (threadIdx.x == 0) {
@@ -159,20 +166,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(sb + L::kBarVFull + 8 * i, 1);
       mbar_init(sb + L::kBarVEmpty + 8 * i, 1);
     }
-    for (int i = 0; i < kSBufs; ++i) mbar_init(sb + L::kBarS + 8 * i, 1);
-    mbar_init(sb + L::kBarP, 4 * 32);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(sb + L::kBarS + 8 * t, 1);
+      mbar_init(sb + L::kBarP + 8 * t, 4 * 32);
+    }
     mbar_init(sb + L::kBarO, 1);
-    mbar_init(sb + L::kBarDrain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) tmem_alloc(sb + L::kTmemSlot, kTmemCols);
-  if (warp < 4 && q_rows < kPrefillRows) {
+  if (warp == kWarpMma) tmem_alloc(sb + L::kTmemSlot, kTmemCols);
+  if (warp < 8 && q_rows < kPrefillRows) {
     // rows no Q box covers are zero (they are masked, but must not be NaN)
-    const int chunks = (kPrefillRows - q_rows) * 8;
-    for (int i = threadIdx.x; i < chunks * L::kSlabs; i += 128) {
+    const int t = warp >> 2, chunks = (kPrefillRows - q_rows) * 8;
+    for (int i = threadIdx.x & 127; i < chunks * L::kSlabs; i += 128) {
       const int b = i / chunks, c = i % chunks;
-      sts128(sb + L::kQ + b * L::kSlab + q_rows * 128 + c * 16, 0u, 0u, 0u, 0u);
+      sts128(sb + L::kQ + t * L::kQTile + b * L::kSlab + q_rows * 128 + c * 16, 0u, 0u, 0u, 0u);
     }
     fence_proxy_async_smem();
   }
@@ -181,14 +189,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   tmem_fence_after_sync();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlot);
 
-  if (warp == 4) {
+  if (warp == kWarpTma) {
     // ================= TMA producer =================
     if (lane == 0) {
-      mbar_arrive_expect_tx(sb + L::kBarQ, L::kSlabs * q_rows * 128);
+      const int tiles = has_b ? 2 : 1;
+      mbar_arrive_expect_tx(sb + L::kBarQ, tiles * L::kSlabs * q_rows * 128);
+      for (int t = 0; t < tiles; ++t) {
 #pragma unroll
-      for (int b = 0; b < L::kSlabs; ++b)
-        tma_load_4d(sb + L::kQ + b * L::kSlab, &qmap, sb + L::kBarQ, 0, b, kvh * G,
-                    q0 + t_begin);
+        for (int b = 0; b < L::kSlabs; ++b)
+          tma_load_4d(sb + L::kQ + t * L::kQTile + b * L::kSlab, &qmap, sb + L::kBarQ, 0, b,
+                      kvh * G, q0 + (t == 0 ? tile_a : tile_b));
+      }
     }
     const int32_t* bt = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
     int k_issued = 0, v_issued = 0;
@@ -247,51 +258,44 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_wait_bounded(sb + L::kBarKFull + 8 * (j % NST), (j / NST) & 1);
     for (int j = max(0, v_issued - NST); j < v_issued; ++j)
       mbar_wait_bounded(sb + L::kBarVFull + 8 * (j % NST), (j / NST) & 1);
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     // ================= MMA issuer =================
     constexpr uint32_t kIdS = umma_idesc_f16(BF16, kPrefillRows, kPrefillKeys, false);
     constexpr uint32_t kIdO = umma_idesc_f16(BF16, kPrefillRows, D, true);
-    auto issue_s = [&](int j) {   // S_j = Q K_j^T into buffer j % 3
+    auto issue_s = [&](int t, int j) {   // S_t(j) = Q_t K_j^T, then report it
       const uint32_t kst = sb + L::kK + (j % NST) * L::kStage;
-      const uint32_t d = tmem + kTmemS + static_cast<uint32_t>(j % kSBufs) * kPrefillKeys;
+      const uint32_t qt = sb + L::kQ + t * L::kQTile;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * L::kSlab + (kk & 3) * 32;
-        umma_f16_ss(d, umma_desc_sw128(sb + L::kQ + off, 16, 1024),
+        umma_f16_ss(tmem + kTmemS + 128 * t, umma_desc_sw128(qt + off, 16, 1024),
                     umma_desc_sw128(kst + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
       }
-      umma_commit(sb + L::kBarS + 8 * (j % kSBufs));
-      umma_commit(sb + L::kBarKEmpty + 8 * (j % NST));
+      umma_commit(sb + L::kBarS + 8 * t);
     };
-    bool ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarQ, 0, abort_flag));
-    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarKFull, 0, abort_flag));
-    if (ok) {
+    auto issue_pv = [&](int t, int j) {  // O_t += P_t(j) V_j over the block's pages
+      const uint32_t vst = sb + L::kV + (j % NST) * L::kStage;
+      const uint32_t pcol = tmem + kTmemS + 128 * t;  // hi in 64 columns, lo in the next 64
+      const int pages_here = min(kPrefillPages, n_pages - j * kPrefillPages);
+      for (int k = 0; k < pages_here; ++k) {
+        const uint64_t bd = umma_desc_sw128(vst + k * 2048, L::kSlab, 1024);
+        umma_f16_ts(tmem + kTmemO + 128 * t, pcol + 8 * k, bd, kIdO, (j > 0 || k > 0) ? 1u : 0u);
+        if constexpr (BF16) umma_f16_ts(tmem + kTmemO + 128 * t, pcol + 64 + 8 * k, bd, kIdO, 1u);
+      }
+    };
+    // whole-warp waits; lane 0 issues
+    auto wait = [&](uint32_t bar, uint32_t parity) {
+      const bool r = __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag));
       tmem_fence_after_sync();
-      if (lane == 0) issue_s(0);
-      __syncwarp();
-    }
+      return r;
+    };
     const int last_page = (ctx - 1) / kPage;
     const int tail_row = ctx % kPage;          // first row past the context in the last page
-    for (int j = 0; ok && j < nkb; ++j) {
-      if (j + 1 < nkb) {
-        const int st1 = (j + 1) % NST;
-        ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarKFull + 8 * st1,
-                                                   ((j + 1) / NST) & 1, abort_flag));
-        if (!ok) break;
-        tmem_fence_after_sync();
-        if (lane == 0) issue_s(j + 1);
-        __syncwarp();
-      }
-      const int st = j % NST;
-      ok = __all_sync(0xffffffffu,
-                      wait_or_abort(sb + L::kBarVFull + 8 * st, (j / NST) & 1, abort_flag));
-      if (!ok) break;
-      const uint32_t vst = sb + L::kV + st * L::kStage;
-      const int pages_here = min(kPrefillPages, n_pages - j * kPrefillPages);
+    auto v_ready = [&](int j) {                // V_j landed; clear its rows past the context
+      if (!wait(sb + L::kBarVFull + 8 * (j % NST), (j / NST) & 1)) return false;
       const int lp = last_page - j * kPrefillPages;
-      if (tail_row != 0 && lp >= 0 && lp < pages_here) {
-        // V rows past the context may hold anything; P is 0 there, and 0 * NaN
-        // must not reach O
+      if (tail_row != 0 && lp >= 0 && lp < kPrefillPages) {
+        const uint32_t vst = sb + L::kV + (j % NST) * L::kStage;
         const int chunks = (kPage - tail_row) * 8;
         for (int i = lane; i < chunks * L::kSlabs; i += 32) {
           const int b = i / chunks, c = i % chunks;
@@ -300,43 +304,69 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
       }
-      ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarP, j & 1, abort_flag));
-      if (!ok) break;
-      tmem_fence_after_sync();
+      return true;
+    };
+    bool ok = wait(sb + L::kBarQ, 0) && wait(sb + L::kBarKFull, 0);
+    if (ok) {
       if (lane == 0) {
-        // P_j sits in S_j's buffer: hi in its first 64 columns, lo in the next 64
-        const uint32_t pcol = tmem + kTmemS + static_cast<uint32_t>(j % kSBufs) * kPrefillKeys;
-        for (int k = 0; k < pages_here; ++k) {
-          const uint64_t bd = umma_desc_sw128(vst + k * 2048, L::kSlab, 1024);
-          umma_f16_ts(tmem + kTmemO, pcol + 8 * k, bd, kIdO, (j > 0 || k > 0) ? 1u : 0u);
-          if constexpr (BF16) umma_f16_ts(tmem + kTmemO, pcol + 64 + 8 * k, bd, kIdO, 1u);
-        }
-        umma_commit(sb + L::kBarO);
-        umma_commit(sb + L::kBarVEmpty + 8 * st);
+        issue_s(0, 0);
+        if (has_b) issue_s(1, 0);
+        umma_commit(sb + L::kBarKEmpty);
       }
       __syncwarp();
+      ok = v_ready(0) && wait(sb + L::kBarP, 0);
+      if (ok && lane == 0) issue_pv(0, 0);
+      __syncwarp();
     }
-    // every MMA issued has completed before tensor memory is freed
-    if (lane == 0) umma_commit(sb + L::kBarDrain);
+    for (int j = 1; ok && j < nkb; ++j) {
+      const int st = j % NST;
+      if (!(ok = wait(sb + L::kBarKFull + 8 * st, (j / NST) & 1))) break;
+      if (lane == 0) issue_s(0, j);                      // after P_A(j-1) V in issue order
+      __syncwarp();
+      if (has_b) {
+        if (!(ok = wait(sb + L::kBarP + 8, (j - 1) & 1))) break;
+        if (lane == 0) issue_pv(1, j - 1);
+        __syncwarp();
+      }
+      if (lane == 0) {
+        umma_commit(sb + L::kBarVEmpty + 8 * ((j - 1) % NST));   // V_{j-1} used by both tiles
+        if (has_b) issue_s(1, j);
+        umma_commit(sb + L::kBarKEmpty + 8 * st);                 // K_j used by both tiles
+      }
+      __syncwarp();
+      if (!(ok = v_ready(j) && wait(sb + L::kBarP, j & 1))) break;
+      if (lane == 0) issue_pv(0, j);
+      __syncwarp();
+    }
+    if (ok && has_b) {
+      ok = wait(sb + L::kBarP + 8, (nkb - 1) & 1);
+      if (ok && lane == 0) issue_pv(1, nkb - 1);
+      __syncwarp();
+    }
+    // every MMA issued has completed before the epilogue reads O and before
+    // tensor memory is freed (also after an abort)
+    if (lane == 0) umma_commit(sb + L::kBarO);
     __syncwarp();
-    if (!mbar_wait_bounded(sb + L::kBarDrain, 0) && lane == 0)
-      record_error(kErrWaitTimeout, blockIdx.x);
-  } else {
-    // ================= softmax (row = threadIdx.x = TMEM lane) =================
-    const int row = threadIdx.x;
-    const int lim = row < nrows ? pos_base + row / G + 1 : 0;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    if (!mbar_wait_bounded(sb + L::kBarO, 0) && lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
+  } else if (warp < 4 || has_b) {
+    // ================= softmax: tile t = warp / 4, row = TMEM lane =================
+    const int t = warp >> 2;
+    const int row = threadIdx.x & 127;
+    const int t_begin = t == 0 ? tile_a : tile_b;
+    const int nrows = (min(t_begin + a.tile_tokens, q_len) - t_begin) * G;
+    const int lim = row < nrows ? ctx - q_len + t_begin + row / G + 1 : 0;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t s_col = kTmemS + 128 * t, o_col = kTmemO + 128 * t;
     const float sl2 = a.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkb; ++j) {
-      const uint32_t buf = kTmemS + static_cast<uint32_t>(j % kSBufs) * kPrefillKeys;
-      ok = __all_sync(0xffffffffu,
-                      wait_or_abort(sb + L::kBarS + 8 * (j % kSBufs), (j / kSBufs) & 1, abort_flag));
+      // S_t(j) is in, and with it every earlier P_t V: O_t is current
+      ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarS + 8 * t, j & 1, abort_flag));
       if (!ok) break;
       tmem_fence_after_sync();
       float p[kPrefillKeys];
-      tmem_ld128(t_lane + buf, p);
+      tmem_ld128(t_lane + s_col, p);
       // logits in log2 units; keys at or past this row's limit are -inf
       const int kbase = j * kPrefillKeys;
       const float2 sl2x2 = make_float2(sl2, sl2);
@@ -374,25 +404,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         p[c] = ex2(x.x);
         p[c + 1] = ex2(x.y);
       }
-
-      if (j > 0) {
-        // P V of the previous block is done: O holds it and the P buffers are free
-        ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarO, (j - 1) & 1, abort_flag));
-        if (!ok) break;
-        tmem_fence_after_sync();
-        if (__any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tmem_ld32(t_lane + kTmemO + 32 * c, o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(t_lane + kTmemO + 32 * c, o);
-          }
-        }
-      }
-      // P (and l) -> this S buffer: keys 2i, 2i+1 packed in column i (hi), and
-      // for bf16 the remainder p - hi in column 64 + i (lo)
+      // P (and l) over S_t: keys 2i, 2i+1 packed in column i (hi); for bf16 the
+      // remainder p - hi in column 64 + i (lo)
       float2 lsum[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) lsum[i] = make_float2(0.f, 0.f);
@@ -402,27 +415,44 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float x0 = p[64 * half + 2 * i], x1 = p[64 * half + 2 * i + 1];
-          h[i] = pack2<BF16>(x0, x1);
-          const float2 hf = unpack2<BF16>(h[i]);
           if constexpr (BF16) {
-            const float2 r = ffma2(hf, make_float2(-1.f, -1.f), make_float2(x0, x1));
-            lo[i] = pack2<true>(r.x, r.y);
+            // hi = p rounded to bf16 by an integer add on the bit pattern (ties
+            // away from zero), lo = the exact fp32 remainder rounded the same way
+            const uint32_t b0 = __float_as_uint(x0) + 0x8000u, b1 = __float_as_uint(x1) + 0x8000u;
+            h[i] = __byte_perm(b0, b1, 0x7632);
+            const float2 r = ffma2(make_float2(__uint_as_float(b0 & 0xffff0000u),
+                                               __uint_as_float(b1 & 0xffff0000u)),
+                                   make_float2(-1.f, -1.f), make_float2(x0, x1));
+            lo[i] = __byte_perm(__float_as_uint(r.x) + 0x8000u, __float_as_uint(r.y) + 0x8000u,
+                                0x7632);
             lsum[i & 3].x += x0;
             lsum[i & 3].y += x1;
           } else {
+            h[i] = pack2<false>(x0, x1);
+            const float2 hf = unpack2<false>(h[i]);
             lsum[i & 3].x += hf.x;
             lsum[i & 3].y += hf.y;
           }
         }
-        tmem_st32u(t_lane + buf + 32 * half, h);
-        if constexpr (BF16) tmem_st32u(t_lane + buf + 64 + 32 * half, lo);
+        tmem_st32u(t_lane + s_col + 32 * half, h);
+        if constexpr (BF16) tmem_st32u(t_lane + s_col + 64 + 32 * half, lo);
       }
       l += ((lsum[0].x + lsum[0].y) + (lsum[1].x + lsum[1].y)) +
            ((lsum[2].x + lsum[2].y) + (lsum[3].x + lsum[3].y));
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(t_lane + o_col + 32 * c, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(t_lane + o_col + 32 * c, o);
+        }
+      }
       tmem_fence_before_sync();
-      mbar_arrive(sb + L::kBarP);
+      mbar_arrive(sb + L::kBarP + 8 * t);
     }
-    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarO, (nkb - 1) & 1, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarO, 0, abort_flag));
     if (ok) {
       tmem_fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -431,7 +461,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
-        tmem_ld32(t_lane + kTmemO + 32 * c, o);
+        tmem_ld32(t_lane + o_col + 32 * c, o);
         if (row < nrows) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -449,7 +479,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   tmem_fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tmem_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
