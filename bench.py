@@ -697,11 +697,25 @@ def recorded_traffic(config: str, kernel: str, context_tokens: int):
     return None
 
 
+# the chunked-prefill kernel and its tensor-core helpers are not on the decode
+# path whose traffic profiles/traffic.json records
+PREFILL_ONLY_SOURCES = ("pa_prefill.cuh", "pa_umma.cuh")
+
+
 def kernel_source_digest() -> str:
+    """Hash of the decode path's sources: every csrc file but the prefill-only
+    ones, with the marked prefill region of pa_api.cu left out."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for p in sorted((ROOT / "paged_kv_cache_444_b200" / "csrc").glob("*")):
-        h.update(p.read_bytes())
+        if p.name in PREFILL_ONLY_SOURCES:
+            continue
+        data = p.read_bytes()
+        if p.name == "pa_api.cu":
+            data = re.sub(rb"// >>> chunked prefill.*?// <<< chunked prefill", b"", data,
+                          flags=re.S)
+        h.update(data)
     return h.hexdigest()[:16]
 
 

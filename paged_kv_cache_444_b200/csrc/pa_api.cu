@@ -13,7 +13,6 @@
 #include "pa_cache_reduce.cuh"
 #include "pa_decode.cuh"
 #include "pa_decode_fp8.cuh"
-#include "pa_prefill.cuh"
 #include "pa_shared_prefix.cuh"
 
 namespace {
@@ -322,39 +321,6 @@ pa_status check_fp8_scales(float k_scale, float v_scale) {
   if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f))
     return PA_ERR_SHAPE;
   return PA_OK;
-}
-
-// 4-D view of the query [T, H, D] for boxes of G heads x tile tokens x 64
-// elements (128-byte swizzle): rows land token-major, row = token * G + head.
-bool encode_query_map(CUtensorMap* map, const void* query, pa_dtype dtype, int64_t num_tokens,
-                      int64_t num_heads, int64_t head_dim, int64_t group, int64_t tile_tokens) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(head_dim / 64),
-                              static_cast<cuuint64_t>(num_heads),
-                              static_cast<cuuint64_t>(num_tokens)};
-  const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(head_dim * 2),
-                                 static_cast<cuuint64_t>(num_heads * head_dim * 2)};
-  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(group),
-                             static_cast<cuuint32_t>(tile_tokens)};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = fn(map, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                        4, const_cast<void*>(query), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-template <int D, bool BF16>
-pa_status launch_prefill_t(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
-                           const PrefillArgs& a, long long grid, cudaStream_t stream) {
-  using L = PrefillSmem<D, BF16>;
-  auto kernel = paged_prefill_kernel<D, BF16>;
-  static std::atomic<uint64_t> done{0};
-  if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
-  return launch_ex(kernel, static_cast<unsigned>(grid), kPrefillThreads, L::kAlloc, stream, 1, qm,
-                   km, vm, a);
 }
 
 DecodeArgs make_args(const void* query, const int32_t* block_tables, const int32_t* context_lens,
@@ -805,57 +771,6 @@ pa_status pa_decode_step_host(void* out_host, const void* query_host, const void
   return PA_OK;
 }
 
-pa_status pa_prefill(void* out, const void* query, const void* key_cache, const void* value_cache,
-                     const int32_t* block_tables, const int32_t* context_lens,
-                     const int32_t* query_starts, float scale, int64_t num_seqs,
-                     int64_t num_query_tokens, int64_t max_query_len, int64_t num_heads,
-                     int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
-                     int64_t block_size, int64_t max_blocks_per_seq, pa_dtype dtype,
-                     void* stream) {
-  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
-                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
-                                      num_blocks, block_size, max_blocks_per_seq, dtype);
-  if (st != PA_OK) return st;
-  if (num_query_tokens < 0 || max_query_len < 0) return PA_ERR_SHAPE;
-  if (num_seqs == 0 || num_query_tokens == 0 || max_query_len == 0) return PA_OK;
-  if (!out || !query_starts) return PA_ERR_NULL;
-  if (!aligned16(out) || (reinterpret_cast<uintptr_t>(query_starts) & 3u)) return PA_ERR_ALIGN;
-  if (num_query_tokens * num_heads > INT32_MAX || max_query_len > INT32_MAX) return PA_ERR_SHAPE;
-  const int64_t G = num_heads / num_kv_heads;
-  const int64_t tile = kPrefillRows / G;                  // G <= 16 checked above
-  const int64_t tiles = (max_query_len + tile - 1) / tile;
-  const int64_t pairs = (tiles + 1) / 2;                  // two query tiles per CTA
-  const long long grid = num_seqs * num_kv_heads * pairs;
-  if (grid > INT32_MAX) return PA_ERR_SHAPE;
-  CUtensorMap qm, km, vm;
-  if (!encode_query_map(&qm, query, dtype, num_query_tokens, num_heads, head_dim, G, tile) ||
-      !encode_cache_map(&km, key_cache, dtype, num_blocks, num_kv_heads, head_dim) ||
-      !encode_cache_map(&vm, value_cache, dtype, num_blocks, num_kv_heads, head_dim))
-    return PA_ERR_CUDA;
-  PrefillArgs a{};
-  a.out = static_cast<uint16_t*>(out);
-  a.block_tables = block_tables;
-  a.context_lens = context_lens;
-  a.query_starts = query_starts;
-  a.scale_log2 = scale * kLog2e;
-  a.num_seqs = static_cast<int>(num_seqs);
-  a.num_tokens = static_cast<int>(num_query_tokens);
-  a.num_heads = static_cast<int>(num_heads);
-  a.num_kv_heads = static_cast<int>(num_kv_heads);
-  a.group = static_cast<int>(G);
-  a.max_blocks_per_seq = static_cast<int>(max_blocks_per_seq);
-  a.num_blocks = static_cast<int>(num_blocks);
-  a.tile_tokens = static_cast<int>(tile);
-  a.pairs_per_seq = static_cast<int>(pairs);
-  cudaStream_t s = as_stream(stream);
-  const bool bf16 = dtype == PA_BF16;
-  if (head_dim == 64)
-    return bf16 ? launch_prefill_t<64, true>(qm, km, vm, a, grid, s)
-                : launch_prefill_t<64, false>(qm, km, vm, a, grid, s);
-  return bf16 ? launch_prefill_t<128, true>(qm, km, vm, a, grid, s)
-              : launch_prefill_t<128, false>(qm, km, vm, a, grid, s);
-}
-
 pa_status pa_check_error(void* stream, int64_t* detail) {
   cudaStream_t s = as_stream(stream);
   unsigned long long word = 0;
@@ -959,3 +874,96 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* query, const void*
         static_cast<int>(parts));
   return launch_status();
 }
+
+// >>> chunked prefill (pa_prefill): host side.  Kept in one region, apart from
+// the decode path's code, so that the two can be versioned separately.
+#include "pa_prefill.cuh"
+
+namespace {
+// 4-D view of the query [T, H, D] for boxes of G heads x tile tokens x 64
+// elements (128-byte swizzle): rows land token-major, row = token * G + head.
+bool encode_query_map(CUtensorMap* map, const void* query, pa_dtype dtype, int64_t num_tokens,
+                      int64_t num_heads, int64_t head_dim, int64_t group, int64_t tile_tokens) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(head_dim / 64),
+                              static_cast<cuuint64_t>(num_heads),
+                              static_cast<cuuint64_t>(num_tokens)};
+  const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(head_dim * 2),
+                                 static_cast<cuuint64_t>(num_heads * head_dim * 2)};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(group),
+                             static_cast<cuuint32_t>(tile_tokens)};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        4, const_cast<void*>(query), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool BF16>
+pa_status launch_prefill_t(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
+                           const PrefillArgs& a, long long grid, cudaStream_t stream) {
+  using L = PrefillSmem<D, BF16>;
+  auto kernel = paged_prefill_kernel<D, BF16>;
+  static std::atomic<uint64_t> done{0};
+  if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
+  return launch_ex(kernel, static_cast<unsigned>(grid), kPrefillThreads, L::kAlloc, stream, 1, qm,
+                   km, vm, a);
+}
+
+
+}  // namespace
+
+extern "C" pa_status pa_prefill(void* out, const void* query, const void* key_cache, const void* value_cache,
+                     const int32_t* block_tables, const int32_t* context_lens,
+                     const int32_t* query_starts, float scale, int64_t num_seqs,
+                     int64_t num_query_tokens, int64_t max_query_len, int64_t num_heads,
+                     int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                     int64_t block_size, int64_t max_blocks_per_seq, pa_dtype dtype,
+                     void* stream) {
+  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
+                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
+                                      num_blocks, block_size, max_blocks_per_seq, dtype);
+  if (st != PA_OK) return st;
+  if (num_query_tokens < 0 || max_query_len < 0) return PA_ERR_SHAPE;
+  if (num_seqs == 0 || num_query_tokens == 0 || max_query_len == 0) return PA_OK;
+  if (!out || !query_starts) return PA_ERR_NULL;
+  if (!aligned16(out) || (reinterpret_cast<uintptr_t>(query_starts) & 3u)) return PA_ERR_ALIGN;
+  if (num_query_tokens * num_heads > INT32_MAX || max_query_len > INT32_MAX) return PA_ERR_SHAPE;
+  const int64_t G = num_heads / num_kv_heads;
+  const int64_t tile = kPrefillRows / G;                  // G <= 16 checked above
+  const int64_t tiles = (max_query_len + tile - 1) / tile;
+  const int64_t pairs = (tiles + 1) / 2;                  // two query tiles per CTA
+  const long long grid = num_seqs * num_kv_heads * pairs;
+  if (grid > INT32_MAX) return PA_ERR_SHAPE;
+  CUtensorMap qm, km, vm;
+  if (!encode_query_map(&qm, query, dtype, num_query_tokens, num_heads, head_dim, G, tile) ||
+      !encode_cache_map(&km, key_cache, dtype, num_blocks, num_kv_heads, head_dim) ||
+      !encode_cache_map(&vm, value_cache, dtype, num_blocks, num_kv_heads, head_dim))
+    return PA_ERR_CUDA;
+  PrefillArgs a{};
+  a.out = static_cast<uint16_t*>(out);
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_starts = query_starts;
+  a.scale_log2 = scale * kLog2e;
+  a.num_seqs = static_cast<int>(num_seqs);
+  a.num_tokens = static_cast<int>(num_query_tokens);
+  a.num_heads = static_cast<int>(num_heads);
+  a.num_kv_heads = static_cast<int>(num_kv_heads);
+  a.group = static_cast<int>(G);
+  a.max_blocks_per_seq = static_cast<int>(max_blocks_per_seq);
+  a.num_blocks = static_cast<int>(num_blocks);
+  a.tile_tokens = static_cast<int>(tile);
+  a.pairs_per_seq = static_cast<int>(pairs);
+  cudaStream_t s = as_stream(stream);
+  const bool bf16 = dtype == PA_BF16;
+  if (head_dim == 64)
+    return bf16 ? launch_prefill_t<64, true>(qm, km, vm, a, grid, s)
+                : launch_prefill_t<64, false>(qm, km, vm, a, grid, s);
+  return bf16 ? launch_prefill_t<128, true>(qm, km, vm, a, grid, s)
+              : launch_prefill_t<128, false>(qm, km, vm, a, grid, s);
+}
+// <<< chunked prefill
