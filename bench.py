@@ -654,7 +654,8 @@ def run_native(args, world, rank, local):
             for n, r in results.items()}
     if args.prefill and not args.only_main:
         tp, tk = measured_tensor_peak()
-        line["prefill"] = prefill_measure(device, args.warmup, peak_tflops=tp, peak_kind=tk)
+        line["prefill"] = prefill_measure(device, args.warmup, reps=args.prefill_reps,
+                                          peak_tflops=tp, peak_kind=tk)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, ctx_main, bt_main, batch,
                                             budget_s=args.cpu_budget)
@@ -785,6 +786,9 @@ def main(argv=None):
                     help="also time pa_decode_fp8 on each batch (E4M3 copy of its caches)")
     ap.add_argument("--prefill", action=argparse.BooleanOptionalAction, default=True,
                     help="also time pa_prefill on a chunked-prefill GQA layer")
+    ap.add_argument("--only-prefill", action="store_true",
+                    help="time only pa_prefill (its own JSON object; for profiling captures)")
+    ap.add_argument("--prefill-reps", type=int, default=20)
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="override the workload's batch size (small profiling captures)")
     ap.add_argument("--num-blocks", type=int, default=0,
@@ -797,6 +801,13 @@ def main(argv=None):
         ap.error("--gpus N > 1 must be launched with torch.distributed.run (one rank per GPU)")
     if args.impl == "reference":
         run_reference(args, world, rank, local)
+    elif args.only_prefill:
+        import torch
+        device = torch.device("cuda", local)
+        torch.cuda.set_device(device)
+        tp, tk = measured_tensor_peak()
+        print(json.dumps(prefill_measure(device, args.warmup, reps=args.prefill_reps,
+                                         peak_tflops=tp, peak_kind=tk)))
     else:
         run_native(args, world, rank, local)
 
