@@ -698,24 +698,24 @@ def recorded_traffic(config: str, kernel: str, context_tokens: int):
     return None
 
 
-# the chunked-prefill kernel and its tensor-core helpers are not on the decode
-# path whose traffic profiles/traffic.json records
-PREFILL_ONLY_SOURCES = ("pa_prefill.cuh", "pa_umma.cuh")
+# sources off the decode path whose traffic profiles/traffic.json records: the
+# chunked-prefill kernel, its tensor-core helpers and the shared-prefix kernel
+OFF_DECODE_PATH = ("pa_prefill.cuh", "pa_umma.cuh", "pa_shared_prefix.cuh")
 
 
-def kernel_source_digest() -> str:
-    """Hash of the decode path's sources: every csrc file but the prefill-only
-    ones, with the marked prefill region of pa_api.cu left out."""
+def kernel_source_digest(csrc: Path | None = None) -> str:
+    """Hash of the decode path's sources: every csrc file but those off the
+    path, with the marked host-side regions of pa_api.cu that serve other
+    kernels ("// >>> ..." to "// <<< ...") left out."""
     import hashlib
     import re
     h = hashlib.sha256()
-    for p in sorted((ROOT / "paged_kv_cache_444_b200" / "csrc").glob("*")):
-        if p.name in PREFILL_ONLY_SOURCES:
+    for p in sorted((csrc or ROOT / "paged_kv_cache_444_b200" / "csrc").glob("*")):
+        if p.name in OFF_DECODE_PATH:
             continue
         data = p.read_bytes()
         if p.name == "pa_api.cu":
-            data = re.sub(rb"// >>> chunked prefill.*?// <<< chunked prefill", b"", data,
-                          flags=re.S)
+            data = re.sub(rb"\n// >>> .*?\n// <<< [^\n]*", b"", data, flags=re.S)
         h.update(data)
     return h.hexdigest()[:16]
 

@@ -13,7 +13,6 @@
 #include "pa_cache_reduce.cuh"
 #include "pa_decode.cuh"
 #include "pa_decode_fp8.cuh"
-#include "pa_shared_prefix.cuh"
 
 namespace {
 
@@ -254,38 +253,6 @@ pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cach
               : launch_decode_d<128, false>(km, vm, a, grid, max_pages, stream);
 }
 
-#ifndef PA_SHARED_CLUSTER
-#define PA_SHARED_CLUSTER 2        // CTAs per shared-prefix item
-#endif
-#ifndef PA_SHARED_CLUSTER_PAGES
-#define PA_SHARED_CLUSTER_PAGES 64  // items with more pages are spread over the cluster
-#endif
-
-template <int D, bool BF16>
-pa_status launch_shared_prefix_t(const CUtensorMap& km, const CUtensorMap& vm,
-                                 SharedPrefixArgs a, long long items, cudaStream_t stream) {
-  constexpr int NST = Stages<D>::value;
-  using L = DecodeSmem<D, NST>;
-  auto kernel = shared_prefix_decode_kernel<D, NST, BF16>;
-  static std::atomic<uint64_t> done{0};
-  static int cluster_cache[kMaxDevices] = {};
-  if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
-  // one cluster size for the launch: as large as PA_SHARED_CLUSTER if the
-  // device can co-schedule it, and 1 when no item can exceed the threshold
-  const int64_t max_item_pages =
-      static_cast<int64_t>(a.members_per_chunk) * a.max_blocks_per_seq;
-  int c = 1;
-  if (max_item_pages > PA_SHARED_CLUSTER_PAGES) {
-    c = pick_cluster(kernel, L::kAlloc, static_cast<int64_t>(PA_SHARED_CLUSTER) *
-                                            PA_CLUSTER_TABLE_PAGES, cluster_cache);
-    if (c > PA_SHARED_CLUSTER) c = PA_SHARED_CLUSTER;
-  }
-  a.cluster_pages = PA_SHARED_CLUSTER_PAGES;
-  if (items * c > INT32_MAX) return PA_ERR_SHAPE;
-  return launch_ex(kernel, static_cast<unsigned>(items * c), kThreads, L::kAlloc, stream, c, km,
-                   vm, a);
-}
-
 // Decode over E4M3 caches (head_dim 128): same kernel, fp8 page steps.
 pa_status run_decode_fp8(DecodeArgs a, const void* key_cache, const void* value_cache,
                          int64_t num_seqs, int64_t num_blocks, pa_dtype dtype,
@@ -495,60 +462,6 @@ pa_status pa_reduce(void* out, const float* tmp_out, const float* max_logits,
                    static_cast<uint16_t*>(out), tmp_out, max_logits, exp_sums, context_lens,
                    static_cast<int>(num_heads), static_cast<int>(head_dim),
                    static_cast<int>(partition_size), static_cast<int>(max_partitions));
-}
-
-pa_status pa_decode_shared_prefix(void* out, const void* query, const void* key_cache,
-                                  const void* value_cache, const int32_t* block_tables,
-                                  const int32_t* context_lens, const int32_t* group_starts,
-                                  const int32_t* prefix_blocks, float scale, int64_t num_seqs,
-                                  int64_t num_groups, int64_t max_group_size, int64_t num_heads,
-                                  int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
-                                  int64_t block_size, int64_t max_blocks_per_seq, pa_dtype dtype,
-                                  void* stream) {
-  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
-                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
-                                      num_blocks, block_size, max_blocks_per_seq, dtype);
-  if (st != PA_OK) return st;
-  if (num_groups < 0 || max_group_size <= 0) return PA_ERR_SHAPE;
-  if (num_seqs == 0 || num_groups == 0) return PA_OK;
-  if (!out || !group_starts || !prefix_blocks) return PA_ERR_NULL;
-  if (!aligned16(out) || (reinterpret_cast<uintptr_t>(group_starts) & 3u) ||
-      (reinterpret_cast<uintptr_t>(prefix_blocks) & 3u))
-    return PA_ERR_ALIGN;
-  const int64_t G = num_heads / num_kv_heads;
-  const int64_t per_chunk = 16 / G;                       // G <= 16 checked above
-  const int64_t chunks = (max_group_size + per_chunk - 1) / per_chunk;
-  const int64_t items = num_groups * num_kv_heads * chunks;
-  if (num_groups > INT32_MAX || chunks > INT32_MAX || items > INT32_MAX) return PA_ERR_SHAPE;
-  CUtensorMap km, vm;
-  if (!encode_cache_map(&km, key_cache, dtype, num_blocks, num_kv_heads, head_dim) ||
-      !encode_cache_map(&vm, value_cache, dtype, num_blocks, num_kv_heads, head_dim))
-    return PA_ERR_CUDA;
-  SharedPrefixArgs a{};
-  a.query = static_cast<const uint16_t*>(query);
-  a.out = static_cast<uint16_t*>(out);
-  a.block_tables = block_tables;
-  a.context_lens = context_lens;
-  a.group_starts = group_starts;
-  a.prefix_blocks = prefix_blocks;
-  a.scale_log2 = scale * kLog2e;
-  a.num_seqs = static_cast<int>(num_seqs);
-  a.num_heads = static_cast<int>(num_heads);
-  a.num_kv_heads = static_cast<int>(num_kv_heads);
-  a.group = static_cast<int>(G);
-  a.max_blocks_per_seq = static_cast<int>(max_blocks_per_seq);
-  a.num_blocks = static_cast<int>(num_blocks);
-  a.num_groups = static_cast<int>(num_groups);
-  a.members_per_chunk = static_cast<int>(per_chunk);
-  a.chunks_per_group = static_cast<int>(chunks);
-  a.longest_first = num_groups * chunks <= kLptMaxSeqs;
-  cudaStream_t s = as_stream(stream);
-  const bool bf16 = dtype == PA_BF16;
-  if (head_dim == 64)
-    return bf16 ? launch_shared_prefix_t<64, true>(km, vm, a, items, s)
-                : launch_shared_prefix_t<64, false>(km, vm, a, items, s);
-  return bf16 ? launch_shared_prefix_t<128, true>(km, vm, a, items, s)
-              : launch_shared_prefix_t<128, false>(km, vm, a, items, s);
 }
 
 pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, int64_t key_stride,
@@ -874,6 +787,100 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* query, const void*
         static_cast<int>(parts));
   return launch_status();
 }
+
+
+// >>> shared-prefix decode (pa_decode_shared_prefix): host side, one region.
+#include "pa_shared_prefix.cuh"
+
+namespace {
+#ifndef PA_SHARED_CLUSTER
+#define PA_SHARED_CLUSTER 4        // CTAs per shared-prefix item (2: 69.6 µs, 4: 63.5, 8: 75.7 on the beam batch)
+#endif
+#ifndef PA_SHARED_CLUSTER_PAGES
+#define PA_SHARED_CLUSTER_PAGES 64  // items with more pages are spread over the cluster
+#endif
+
+template <int D, bool BF16>
+pa_status launch_shared_prefix_t(const CUtensorMap& km, const CUtensorMap& vm,
+                                 SharedPrefixArgs a, long long items, cudaStream_t stream) {
+  constexpr int NST = Stages<D>::value;
+  using L = DecodeSmem<D, NST>;
+  auto kernel = shared_prefix_decode_kernel<D, NST, BF16>;
+  static std::atomic<uint64_t> done{0};
+  static int cluster_cache[kMaxDevices] = {};
+  if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
+  // one cluster size for the launch: as large as PA_SHARED_CLUSTER if the
+  // device can co-schedule it, and 1 when no item can exceed the threshold
+  const int64_t max_item_pages =
+      static_cast<int64_t>(a.members_per_chunk) * a.max_blocks_per_seq;
+  int c = 1;
+  if (max_item_pages > PA_SHARED_CLUSTER_PAGES) {
+    c = pick_cluster(kernel, L::kAlloc, static_cast<int64_t>(PA_SHARED_CLUSTER) *
+                                            PA_CLUSTER_TABLE_PAGES, cluster_cache);
+    if (c > PA_SHARED_CLUSTER) c = PA_SHARED_CLUSTER;
+  }
+  a.cluster_pages = PA_SHARED_CLUSTER_PAGES;
+  if (items * c > INT32_MAX) return PA_ERR_SHAPE;
+  return launch_ex(kernel, static_cast<unsigned>(items * c), kThreads, L::kAlloc, stream, c, km,
+                   vm, a);
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_shared_prefix(void* out, const void* query, const void* key_cache,
+                                  const void* value_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, const int32_t* group_starts,
+                                  const int32_t* prefix_blocks, float scale, int64_t num_seqs,
+                                  int64_t num_groups, int64_t max_group_size, int64_t num_heads,
+                                  int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
+                                  int64_t block_size, int64_t max_blocks_per_seq, pa_dtype dtype,
+                                  void* stream) {
+  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
+                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
+                                      num_blocks, block_size, max_blocks_per_seq, dtype);
+  if (st != PA_OK) return st;
+  if (num_groups < 0 || max_group_size <= 0) return PA_ERR_SHAPE;
+  if (num_seqs == 0 || num_groups == 0) return PA_OK;
+  if (!out || !group_starts || !prefix_blocks) return PA_ERR_NULL;
+  if (!aligned16(out) || (reinterpret_cast<uintptr_t>(group_starts) & 3u) ||
+      (reinterpret_cast<uintptr_t>(prefix_blocks) & 3u))
+    return PA_ERR_ALIGN;
+  const int64_t G = num_heads / num_kv_heads;
+  const int64_t per_chunk = 16 / G;                       // G <= 16 checked above
+  const int64_t chunks = (max_group_size + per_chunk - 1) / per_chunk;
+  const int64_t items = num_groups * num_kv_heads * chunks;
+  if (num_groups > INT32_MAX || chunks > INT32_MAX || items > INT32_MAX) return PA_ERR_SHAPE;
+  CUtensorMap km, vm;
+  if (!encode_cache_map(&km, key_cache, dtype, num_blocks, num_kv_heads, head_dim) ||
+      !encode_cache_map(&vm, value_cache, dtype, num_blocks, num_kv_heads, head_dim))
+    return PA_ERR_CUDA;
+  SharedPrefixArgs a{};
+  a.query = static_cast<const uint16_t*>(query);
+  a.out = static_cast<uint16_t*>(out);
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.group_starts = group_starts;
+  a.prefix_blocks = prefix_blocks;
+  a.scale_log2 = scale * kLog2e;
+  a.num_seqs = static_cast<int>(num_seqs);
+  a.num_heads = static_cast<int>(num_heads);
+  a.num_kv_heads = static_cast<int>(num_kv_heads);
+  a.group = static_cast<int>(G);
+  a.max_blocks_per_seq = static_cast<int>(max_blocks_per_seq);
+  a.num_blocks = static_cast<int>(num_blocks);
+  a.num_groups = static_cast<int>(num_groups);
+  a.members_per_chunk = static_cast<int>(per_chunk);
+  a.chunks_per_group = static_cast<int>(chunks);
+  a.longest_first = num_groups * chunks <= kLptMaxSeqs;
+  cudaStream_t s = as_stream(stream);
+  const bool bf16 = dtype == PA_BF16;
+  if (head_dim == 64)
+    return bf16 ? launch_shared_prefix_t<64, true>(km, vm, a, items, s)
+                : launch_shared_prefix_t<64, false>(km, vm, a, items, s);
+  return bf16 ? launch_shared_prefix_t<128, true>(km, vm, a, items, s)
+              : launch_shared_prefix_t<128, false>(km, vm, a, items, s);
+}
+// <<< shared-prefix decode
 
 // >>> chunked prefill (pa_prefill): host side.  Kept in one region, apart from
 // the decode path's code, so that the two can be versioned separately.
