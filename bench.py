@@ -300,16 +300,9 @@ def prefill_measure(device, warmup: int, reps: int = 20, peak_tflops: float = 0.
     TFLOP/s against the measured dense bf16 peak, with the CPU oracle's
     count of flops: 4 * D * H * sum over queries of (position + 1)."""
     from paged_kv_cache_444_b200 import pa_prefill
-    cfg = workloads.CONFIGS["gqa_llama3_8b"].scaled(
-        name="chunked_prefill_gqa", num_seqs=8, num_blocks=4096, ctx=("uniform", 512, 4096),
-        seed=444_006)
-    b = workloads.make_batch(cfg, device)
-    chunk = 512
-    T = cfg.num_seqs * chunk
-    g = torch.Generator(device=device).manual_seed(cfg.seed + 1)
-    query = torch.randn((T, cfg.num_heads, cfg.head_dim), generator=g, device=device).to(
-        cfg.torch_dtype)
-    starts = torch.arange(0, T + 1, chunk, dtype=torch.int32, device=device)
+    pb = workloads.make_prefill_batch(device=device)
+    b, cfg, chunk, query, starts = pb.cache, pb.cache.cfg, pb.chunk, pb.query, pb.query_starts
+    T = query.shape[0]
     out = torch.empty_like(query)
 
     def run():

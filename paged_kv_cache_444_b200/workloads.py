@@ -228,6 +228,36 @@ def make_batch(cfg: DecodeConfig, device: str | torch.device = "cpu") -> DecodeB
                        group_starts, prefix_blocks)
 
 
+@dataclass
+class PrefillBatch:
+    """A chunked-prefill step: each sequence's `chunk` newest tokens are the
+    queries (packed [T, H, D], offsets query_starts), their K/V already in the
+    paged cache of `cache`."""
+    cache: DecodeBatch
+    query: torch.Tensor
+    query_starts: torch.Tensor
+    chunk: int
+
+
+PREFILL_CONFIG = CONFIGS["gqa_llama3_8b"].scaled(
+    name="chunked_prefill_gqa", num_seqs=8, num_blocks=4096, ctx=("uniform", 512, 4096),
+    seed=444_006)
+
+
+def make_prefill_batch(cfg: DecodeConfig = PREFILL_CONFIG, chunk: int = 512,
+                       device: str | torch.device = "cpu") -> PrefillBatch:
+    """The chunked-prefill workload: cfg's caches and contexts (every context
+    >= chunk), queries N(0,1) in the cache dtype from a generator seeded
+    seed + 1, chunk query tokens per sequence."""
+    b = make_batch(cfg, device)
+    T = cfg.num_seqs * chunk
+    g = torch.Generator(device=device).manual_seed(cfg.seed + 1)
+    query = torch.randn((T, cfg.num_heads, cfg.head_dim), generator=g, device=device).to(
+        cfg.torch_dtype)
+    starts = torch.arange(0, T + 1, chunk, dtype=torch.int32, device=device)
+    return PrefillBatch(b, query, starts, chunk)
+
+
 def algorithmic_bytes(cfg: DecodeConfig, context_lens) -> dict:
     """Bytes the decode step must move at least once, by part:
     K+V of every context token of every KV head, the block-table entries

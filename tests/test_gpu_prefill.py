@@ -129,3 +129,35 @@ def test_prefill_reports_query_longer_than_context(cuda_device):
     with pytest.raises(PagedAttentionError) as e:
         pa_check_error()
     assert e.value.detail >> 56 == 7 and e.value.detail & 0xffff == 1
+
+
+def test_prefill_full_size_sampled(cuda_device, oracle_lib):
+    """The chunked-prefill layer bench.py times (8 sequences x 512-token chunks,
+    32/8 heads, bf16), in the same launch, checked on samples the oracle
+    computes in seconds: the whole chunk of the shortest-context sequence, and
+    the last 64 query tokens of the longest (their positions are those of the
+    full chunk when they are given as a 64-token chunk of the same context)."""
+    pb = workloads.make_prefill_batch(device=cuda_device)
+    b, cfg, chunk = pb.cache, pb.cache.cfg, pb.chunk
+    out = torch.full_like(pb.query, float("nan"))
+    pa_prefill(out, pb.query, b.key_cache, b.value_cache, b.block_tables, b.context_lens,
+               pb.query_starts, cfg.scale, chunk)
+    torch.cuda.synchronize()
+    pa_check_error()
+    g = to_f64(out)
+    assert np.isfinite(g).all()
+    ctx = b.context_lens.cpu().numpy()
+    bt = b.block_tables.cpu().numpy()
+    for s, t0 in ((int(np.argmin(ctx)), 0), (int(np.argmax(ctx)), chunk - 64)):
+        n = (int(ctx[s]) + 15) // 16
+        ids = torch.tensor(bt[s, :n], dtype=torch.long, device=cuda_device)
+        kc = bits(b.key_cache.index_select(0, ids))
+        vc = bits(b.value_cache.index_select(0, ids))
+        rows = slice(s * chunk + t0, (s + 1) * chunk)
+        ref = oracle_lib.prefill(bits(pb.query[rows]), kc, vc,
+                                 np.arange(n, dtype=np.int32)[None, :],
+                                 ctx[s:s + 1].astype(np.int32),
+                                 np.array([0, chunk - t0], dtype=np.int32), cfg.scale,
+                                 ocode(cfg))
+        err = np.max(np.abs(g[rows] - ref))
+        assert err <= TOL[cfg.dtype], f"seq {s} tokens {t0}..{chunk}: {err:.3e}"
