@@ -444,11 +444,12 @@ class HostStep:
                                                        max_blocks_per_seq, bs, partition_size)
         _need(n >= 0, "bad step sizes")
         self.workspace = torch.empty(n, dtype=torch.uint8, device=key_cache.device)
-        # one pinned host buffer laid out like the workspace, so the six
-        # inputs travel in a single copy
+        # one pinned host buffer laid out like the workspace (key, value,
+        # slot_mapping, then query, block_tables, context_lens), so each of the
+        # step's two input stages travels in a single copy
         S, H, D_ = num_seqs, num_heads, D
-        parts = [((S, H, D_), dtype), ((S, Hk, D_), dtype), ((S, Hk, D_), dtype),
-                 ((S,), torch.int64), ((S, max_blocks_per_seq), torch.int32), ((S,), torch.int32)]
+        parts = [((S, Hk, D_), dtype), ((S, Hk, D_), dtype), ((S,), torch.int64),
+                 ((S, H, D_), dtype), ((S, max_blocks_per_seq), torch.int32), ((S,), torch.int32)]
         offs, at = [], 0
         for shape, dt in parts:
             offs.append(at)
@@ -459,8 +460,9 @@ class HostStep:
         for (shape, dt), o in zip(parts, offs):
             nbytes = int(torch.Size(shape).numel()) * torch.tensor([], dtype=dt).element_size()
             views.append(self.staging[o:o + nbytes].view(dt).view(shape))
-        (self.query, self.key, self.value, self.slot_mapping, self.block_tables,
+        (self.key, self.value, self.slot_mapping, self.query, self.block_tables,
          self.context_lens) = views
+        # pinned, so the attention writes its output straight into it
         self.out = torch.empty((S, H, D_), dtype=dtype).pin_memory()
 
     @property
@@ -475,10 +477,18 @@ class HostStep:
 
     def run(self, stream=None) -> None:
         S, H, Hk, D, NB, bs, MB = self.dims
+        # parts still in the staging buffer go as packed (NULL): one copy per stage
+        packed = self.staging.data_ptr()
+        inside = lambda t: packed <= t.data_ptr() < packed + self.staging.numel()
+        kv_packed = all(inside(t) for t in (self.key, self.value, self.slot_mapping))
+        q_packed = all(inside(t) for t in (self.query, self.block_tables, self.context_lens))
         st = load().pa_decode_step_host(
             self.out.data_ptr(), self.query.data_ptr(), self.key.data_ptr(),
-            self.value.data_ptr(), self.slot_mapping.data_ptr(), self.block_tables.data_ptr(),
-            self.context_lens.data_ptr(), self.key_cache.data_ptr(), self.value_cache.data_ptr(),
+            None if kv_packed else self.value.data_ptr(),
+            None if kv_packed else self.slot_mapping.data_ptr(),
+            None if q_packed else self.block_tables.data_ptr(),
+            None if q_packed else self.context_lens.data_ptr(),
+            self.key_cache.data_ptr(), self.value_cache.data_ptr(),
             self.workspace.data_ptr(), self.workspace.numel(), self.scale, S, H, Hk, D, NB, bs,
             MB, self.partition_size, DTYPE_CODES[self.dtype], _stream(stream))
         _check(st, "pa_decode_step_host")

@@ -7,7 +7,9 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "pa.h"
 #include "pa_cache_reduce.cuh"
@@ -576,7 +578,9 @@ int64_t align256(int64_t x) { return (x + 255) & ~static_cast<int64_t>(255); }
 StepLayout step_layout(int64_t S, int64_t H, int64_t Hk, int64_t D, int64_t MB, int64_t bs,
                        int64_t partition_size) {
   const int64_t parts = partition_size > 0 ? (MB * bs + partition_size - 1) / partition_size : 0;
-  const int64_t sizes[10] = {S * H * D * 2, S * Hk * D * 2, S * Hk * D * 2, S * 8, S * MB * 4,
+  // key, value, slot_mapping (what the cache write needs), then query,
+  // block_tables, context_lens, then out and the split partials
+  const int64_t sizes[10] = {S * Hk * D * 2, S * Hk * D * 2, S * 8, S * H * D * 2, S * MB * 4,
                              S * 4, S * H * D * 2, S * H * parts * D * 4, S * H * parts * 4,
                              S * H * parts * 4};
   StepLayout l{};
@@ -587,6 +591,45 @@ StepLayout step_layout(int64_t S, int64_t H, int64_t Hk, int64_t D, int64_t MB, 
   }
   l.total = at;
   return l;
+}
+
+// A side stream and two events per (device, caller stream): the step's query
+// and table copies run on the side stream while the cache write runs on the
+// caller's stream (fork after the caller's earlier work, join before the
+// attention).  Created once; calls on one stream are ordered, so reusing the
+// events is safe.
+struct StepFork {
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+const StepFork* step_fork(cudaStream_t s) {
+  static std::mutex mu;
+  static std::map<std::pair<int, cudaStream_t>, StepFork> forks;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = forks.find({dev, s});
+  if (it != forks.end()) return &it->second;
+  StepFork f;
+  if (cudaStreamCreateWithFlags(&f.side, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&f.fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&f.join, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return &forks.emplace(std::make_pair(dev, s), f).first->second;
+}
+
+// The device address of page-locked host memory the GPU can write directly,
+// or nullptr (pageable memory).
+void* device_view_of_host(void* p) {
+  cudaPointerAttributes attr{};
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return attr.type == cudaMemoryTypeHost ? attr.devicePointer : nullptr;
 }
 }  // namespace
 
@@ -614,8 +657,11 @@ pa_status pa_decode_step_host(void* out_host, const void* query_host, const void
   if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_DTYPE;
   if (num_seqs < 0 || partition_size < 0) return PA_ERR_SHAPE;
   if (num_seqs == 0) return PA_OK;
-  if (!out_host || !query_host || !key_host || !value_host || !slot_mapping_host ||
-      !block_tables_host || !context_lens_host || !key_cache || !value_cache || !workspace)
+  // value and slot_mapping: both given, or both NULL to say they follow
+  // key_host in one buffer at the workspace's offsets; the same for
+  // block_tables and context_lens after query_host
+  if (!out_host || !query_host || !key_host || !key_cache || !value_cache || !workspace ||
+      (!value_host != !slot_mapping_host) || (!block_tables_host != !context_lens_host))
     return PA_ERR_NULL;
   const int64_t need = pa_decode_step_host_workspace_bytes(num_seqs, num_heads, num_kv_heads,
                                                            head_dim, max_blocks_per_seq,
@@ -626,41 +672,57 @@ pa_status pa_decode_step_host(void* out_host, const void* query_host, const void
   const StepLayout l = step_layout(num_seqs, num_heads, num_kv_heads, head_dim,
                                    max_blocks_per_seq, block_size, partition_size);
   uint8_t* w = static_cast<uint8_t*>(workspace);
-  void* d_query = w + l.off[0];
-  void* d_key = w + l.off[1];
-  void* d_value = w + l.off[2];
-  int64_t* d_slots = reinterpret_cast<int64_t*>(w + l.off[3]);
+  void* d_key = w + l.off[0];
+  void* d_value = w + l.off[1];
+  int64_t* d_slots = reinterpret_cast<int64_t*>(w + l.off[2]);
+  void* d_query = w + l.off[3];
   int32_t* d_tables = reinterpret_cast<int32_t*>(w + l.off[4]);
   int32_t* d_lens = reinterpret_cast<int32_t*>(w + l.off[5]);
-  void* d_out = w + l.off[6];
   cudaStream_t s = as_stream(stream);
+  const StepFork* fork = step_fork(s);
+  if (!fork) return PA_ERR_CUDA;
   const int64_t q_bytes = num_seqs * num_heads * head_dim * 2;
   const int64_t kv_bytes = num_seqs * num_kv_heads * head_dim * 2;
   struct Copy { void* dst; const void* src; int64_t bytes; };
-  const Copy ins[6] = {{d_query, query_host, q_bytes}, {d_key, key_host, kv_bytes},
-                       {d_value, value_host, kv_bytes}, {d_slots, slot_mapping_host, num_seqs * 8},
-                       {d_tables, block_tables_host, num_seqs * max_blocks_per_seq * 4},
-                       {d_lens, context_lens_host, num_seqs * 4}};
-  // Inputs laid out in host memory exactly as in the workspace (one pinned
-  // buffer with the same offsets) go over in one copy; otherwise one each.
-  const uint8_t* hbase = static_cast<const uint8_t*>(query_host);
-  bool packed = true;
-  for (int i = 1; i < 6; ++i) packed = packed && ins[i].src == hbase + l.off[i];
-  if (packed) {
-    if (cudaMemcpyAsync(w, hbase, static_cast<size_t>(l.off[5] + num_seqs * 4),
-                        cudaMemcpyHostToDevice, s) != cudaSuccess)
-      return PA_ERR_CUDA;
-  } else {
-    for (const Copy& c : ins)
-      if (cudaMemcpyAsync(c.dst, c.src, static_cast<size_t>(c.bytes), cudaMemcpyHostToDevice,
-                          s) != cudaSuccess)
-        return PA_ERR_CUDA;
-  }
+  // A stage whose later parts the caller marked as packed (NULL) goes over in
+  // one copy from its first part's address, else one copy per part.
+  auto copy_in = [&](const Copy* c, int n, int first, cudaStream_t on) {
+    if (!c[1].src) {
+      const int64_t bytes = l.off[first + n - 1] - l.off[first] + c[n - 1].bytes;
+      return cudaMemcpyAsync(c[0].dst, c[0].src, static_cast<size_t>(bytes),
+                             cudaMemcpyHostToDevice, on) == cudaSuccess;
+    }
+    for (int i = 0; i < n; ++i)
+      if (cudaMemcpyAsync(c[i].dst, c[i].src, static_cast<size_t>(c[i].bytes),
+                          cudaMemcpyHostToDevice, on) != cudaSuccess)
+        return false;
+    return true;
+  };
+  const Copy write_in[3] = {{d_key, key_host, kv_bytes}, {d_value, value_host, kv_bytes},
+                            {d_slots, slot_mapping_host, num_seqs * 8}};
+  const Copy attend_in[3] = {{d_query, query_host, q_bytes},
+                             {d_tables, block_tables_host, num_seqs * max_blocks_per_seq * 4},
+                             {d_lens, context_lens_host, num_seqs * 4}};
+  // The new rows go first; then (fork) the side stream copies the query and
+  // tables while this stream writes the rows into the caches.  The fork comes
+  // after all earlier work on this stream, so nothing still reads the
+  // workspace the side stream overwrites.
+  if (!copy_in(write_in, 3, 0, s) || cudaEventRecord(fork->fork, s) != cudaSuccess ||
+      cudaStreamWaitEvent(fork->side, fork->fork, 0) != cudaSuccess ||
+      !copy_in(attend_in, 3, 3, fork->side) ||
+      cudaEventRecord(fork->join, fork->side) != cudaSuccess)
+    return PA_ERR_CUDA;
   pa_status st = pa_reshape_and_cache(d_key, d_value, num_kv_heads * head_dim,
                                       num_kv_heads * head_dim, key_cache, value_cache, d_slots,
                                       num_seqs, num_kv_heads, head_dim, num_blocks, block_size,
                                       dtype, stream);
   if (st != PA_OK) return st;
+  // join, then attend; the output goes straight into out_host when that is
+  // page-locked memory the device can address, else through the workspace
+  if (cudaStreamWaitEvent(s, fork->join, 0) != cudaSuccess) return PA_ERR_CUDA;
+  void* direct = device_view_of_host(out_host);
+  if (direct && !aligned16(direct)) direct = nullptr;
+  void* d_out = direct ? direct : static_cast<void*>(w + l.off[6]);
   if (partition_size > 0) {
     const int64_t parts = (max_blocks_per_seq * block_size + partition_size - 1) / partition_size;
     float* tmp = reinterpret_cast<float*>(w + l.off[7]);
@@ -678,8 +740,8 @@ pa_status pa_decode_step_host(void* out_host, const void* query_host, const void
                    dtype, stream);
   }
   if (st != PA_OK) return st;
-  if (cudaMemcpyAsync(out_host, d_out, static_cast<size_t>(q_bytes), cudaMemcpyDeviceToHost, s) !=
-      cudaSuccess)
+  if (!direct && cudaMemcpyAsync(out_host, d_out, static_cast<size_t>(q_bytes),
+                                 cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return PA_ERR_CUDA;
   return PA_OK;
 }

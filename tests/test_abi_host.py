@@ -191,3 +191,21 @@ def test_fp8_validation(lib):
     bad = list(good)
     bad[7] = 0
     assert w(*bad) == OK
+
+
+@host_only
+def test_step_host_packed_pairs_validation(lib):
+    """pa_decode_step_host: value/slot_mapping (and block_tables/context_lens)
+    are both given or both NULL (packed after key/query); one NULL alone is
+    PA_ERR_NULL, found before any CUDA call.  An empty batch is a no-op."""
+    f = lib.pa_decode_step_host
+    W = FAKE
+
+    def call(value, slots, tables, lens, S=4):
+        return f(W, W, W, value, slots, tables, lens, W, W, W, 1 << 30, 0.125, S, 8, 2, 128, 64,
+                 16, 8, 0, 0, None)
+    assert call(None, W, W, W) == NULL
+    assert call(W, None, W, W) == NULL
+    assert call(W, W, None, W) == NULL
+    assert call(W, W, W, None) == NULL
+    assert call(None, W, None, W, S=0) == OK

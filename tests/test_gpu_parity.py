@@ -368,6 +368,30 @@ def test_host_step_matches_oracle(name, ps, dev, oracle_lib):
     _check_close(step.out, ref, cfg, f"host step {name}")
 
 
+@pytest.mark.parametrize("name,ps", [("gqa_small", 0), ("long_small", 64)])
+def test_host_step_unpacked_inputs_pageable_output(name, ps, dev, oracle_lib):
+    """pa_decode_step_host with each input in its own pinned tensor (one copy
+    each) and a pageable output (written to the workspace, then copied back),
+    run twice in a row on one stream."""
+    from paged_kv_cache_444_b200 import HostStep
+    cfg = SMALL[name]
+    batch = workloads.make_batch(cfg, dev)
+    host = HostCopy(batch)
+    ref, kc_ref, _ = oracle_step(oracle_lib, host)
+    step = HostStep(batch.key_cache, batch.value_cache, cfg.num_seqs, cfg.num_heads,
+                    batch.block_tables.shape[1], cfg.scale, ps, cfg.torch_dtype)
+    for name_ in ("query", "key", "value", "slot_mapping", "block_tables", "context_lens"):
+        setattr(step, name_, getattr(batch, name_).cpu().clone().pin_memory())
+    step.out = torch.full(tuple(batch.query.shape), float("nan"), dtype=cfg.torch_dtype)
+    assert not step.out.is_pinned()
+    for _ in range(2):
+        step.run()
+    torch.cuda.synchronize()
+    pa_check_error()
+    assert np.array_equal(bits(batch.key_cache), kc_ref)
+    _check_close(step.out, ref, cfg, f"host step {name}, unpacked inputs, pageable output")
+
+
 @pytest.mark.parametrize("name,ps", [("gqa_small", 0), ("long_small", 64), ("tiny", 0)])
 def test_plan_replays_from_a_cuda_graph(name, ps, dev, oracle_lib):
     """A DecodePlan run eagerly, and the same plan captured once in a CUDA
