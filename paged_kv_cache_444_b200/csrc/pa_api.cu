@@ -562,11 +562,10 @@ pa_status pa_decode_split_fp8(float* tmp_out, float* max_logits, float* exp_sums
                         as_stream(stream));
 }
 
-// ---------------------------------------------------------------------------
-// One decode step from host buffers.  Workspace layout (each part 256-byte
-// aligned): query, key, value, slot_mapping, block_tables, context_lens, out,
-// then for the split path tmp_out, max_logits, exp_sums.
-// ---------------------------------------------------------------------------
+// >>> host-buffer step (pa_decode_step_host): one decode step from host
+// buffers.  Workspace layout (each part 256-byte aligned): key, value,
+// slot_mapping, query, block_tables, context_lens, out, then for the split
+// path tmp_out, max_logits, exp_sums.
 namespace {
 struct StepLayout {
   int64_t off[10];
@@ -745,6 +744,7 @@ pa_status pa_decode_step_host(void* out_host, const void* query_host, const void
     return PA_ERR_CUDA;
   return PA_OK;
 }
+// <<< host-buffer step
 
 pa_status pa_check_error(void* stream, int64_t* detail) {
   cudaStream_t s = as_stream(stream);
