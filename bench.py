@@ -559,6 +559,9 @@ def run_native(args, world, rank, local):
             "tokens_per_s": sum_over_ranks(cfg.num_seqs, world, device) / (ms_max / 1e3),
             "graph_ms_per_step": gms,
             "shared_prefix_kernel_ms": shared_ms,
+            "unique_kv_bytes": (workloads.unique_kv_bytes(cfg, batch.block_tables.cpu().tolist(),
+                                                          batch.context_lens.cpu().tolist())
+                                if shared_ms else None),
             "fp8_ms": f8_ms,
             "kernel": "pa_decode_split" if step.ps else "pa_decode",
             "context_tokens": int(sum(ctx)),
@@ -641,7 +644,14 @@ def run_native(args, world, rank, local):
                 "graph_ms_per_step": (round(r["graph_ms_per_step"], 5)
                                       if r["graph_ms_per_step"] else None),
                 "per_kernel_ms": [round(x, 5) for x in r["per_kernel_ms"]],
-                **({"pa_decode_shared_prefix_ms": round(r["shared_prefix_kernel_ms"], 5)}
+                **({"pa_decode_shared_prefix_ms": round(r["shared_prefix_kernel_ms"], 5),
+                    # the shared-prefix kernel reads each shared page once:
+                    # its rate on the unique K/V bytes, against the copy peak
+                    "pa_decode_shared_prefix_unique_gbs": round(
+                        r["unique_kv_bytes"] / (r["shared_prefix_kernel_ms"] / 1e3) / 1e9, 1),
+                    "pa_decode_shared_prefix_unique_frac_of_peak": round(
+                        r["unique_kv_bytes"] / (r["shared_prefix_kernel_ms"] / 1e3) / 1e9 / peak,
+                        4)}
                    if r["shared_prefix_kernel_ms"] else {}),
                 **(fp8_entry(r, peak) if r["fp8_ms"] else {})}
             for n, r in results.items()}
