@@ -83,10 +83,6 @@ bool ensure_smem(K kernel, int bytes, std::atomic<uint64_t>* done_mask) {
   return true;
 }
 
-pa_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
-}
-
 // Launch with programmatic stream serialisation (the kernel may start while
 // the previous kernel of the stream drains; every kernel here waits for it
 // with griddepcontrol.wait before reading inputs) and, if cluster > 1, as
@@ -766,12 +762,10 @@ pa_status pa_check_error(void* stream, int64_t* detail) {
 
 }  // extern "C"
 
-// ---------------------------------------------------------------------------
-// pa_decode_noalloc: split decode + merge with the partition scratch in a
-// fixed device array of this file (declared in pa.h).  Host code must not
-// use the array's name as a device address; the address is looked up once
-// per device below and passed to the kernels.
-// ---------------------------------------------------------------------------
+// >>> no-allocation entry point (pa_decode_noalloc): split decode + merge
+// with the partition scratch in a fixed device array of this file (declared
+// in pa.h).  Host code must not use the array's name as a device address; the
+// address is looked up once per device below and passed to the kernels.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
@@ -837,18 +831,13 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* query, const void*
       PA_OK)
     return st;
   const unsigned grid = static_cast<unsigned>(num_seqs * num_heads);
-  if (dtype == PA_BF16)
-    lse_reduce_kernel<true><<<grid, kReduceThreads, 0, s>>>(
-        static_cast<uint16_t*>(out), tmp_out, max_logits, exp_sums, context_lens,
-        static_cast<int>(num_heads), static_cast<int>(head_dim), static_cast<int>(partition_size),
-        static_cast<int>(parts));
-  else
-    lse_reduce_kernel<false><<<grid, kReduceThreads, 0, s>>>(
-        static_cast<uint16_t*>(out), tmp_out, max_logits, exp_sums, context_lens,
-        static_cast<int>(num_heads), static_cast<int>(head_dim), static_cast<int>(partition_size),
-        static_cast<int>(parts));
-  return launch_status();
+  auto kernel = dtype == PA_BF16 ? lse_reduce_kernel<true> : lse_reduce_kernel<false>;
+  return launch_ex(kernel, grid, kReduceThreads, 0, s, 1, static_cast<uint16_t*>(out), tmp_out,
+                   max_logits, exp_sums, context_lens, static_cast<int>(num_heads),
+                   static_cast<int>(head_dim), static_cast<int>(partition_size),
+                   static_cast<int>(parts));
 }
+// <<< no-allocation entry point
 
 
 // >>> shared-prefix decode (pa_decode_shared_prefix): host side, one region.
