@@ -31,8 +31,8 @@
 // only when a row's running maximum grows by more than 2^8 (the reference
 // maximum may lag the true one by that much: P <= 2^8 stays exact in the
 // 16-bit operand and the final 1/l uses the same reference).  bf16 P enters
-// P V as a hi + lo pair of bf16 products (about 17 bits of P, split with
-// integer rounding so the conversion unit stays free for 2^x); fp16 P is
+// P V as a hi + lo pair of bf16 products (at least 14 bits of P, split by
+// bit truncation so the conversion unit stays free for 2^x); fp16 P is
 // rounded once and l sums the rounded values.
 #pragma once
 
@@ -93,6 +93,13 @@ struct PrefillSmem {
   static constexpr int kBytes = kAbort + 4;
   static constexpr int kAlloc = kBytes + 1024;
 };
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 
 // Bounded barrier wait that also gives up as soon as another role of the CTA
 // has given up (the shared abort flag); the first to time out records it.
@@ -367,27 +374,33 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       tmem_fence_after_sync();
       float p[kPrefillKeys];
       tmem_ld128(t_lane + s_col, p);
-      // logits in log2 units; keys at or past this row's limit are -inf
+      // keys at or past this row's limit are -inf
       const int kbase = j * kPrefillKeys;
-      const float2 sl2x2 = make_float2(sl2, sl2);
-      if (kbase + kPrefillKeys <= lim) {
+      if (kbase + kPrefillKeys > lim) {
 #pragma unroll
-        for (int c = 0; c < kPrefillKeys; c += 2) {
-          const float2 x = fmul2(make_float2(p[c], p[c + 1]), sl2x2);
-          p[c] = x.x;
-          p[c + 1] = x.y;
-        }
-      } else {
+        for (int c = 0; c < kPrefillKeys; ++c) p[c] = kbase + c < lim ? p[c] : -INFINITY;
+      }
+      // the block's largest logit in log2 units: for scale > 0 the maximum of
+      // the raw S (three-input max), scaled once; otherwise S is scaled first
+      float mul = sl2;
+      if (!(sl2 > 0.f)) {
 #pragma unroll
-        for (int c = 0; c < kPrefillKeys; ++c) p[c] = kbase + c < lim ? p[c] * sl2 : -INFINITY;
+        for (int c = 0; c < kPrefillKeys; ++c) p[c] = p[c] == -INFINITY ? -INFINITY : p[c] * sl2;
+        mul = 1.f;
       }
       float mx8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = p[i];
+      static_assert((kPrefillKeys - 8) % 16 == 8, "the key loop below leaves 8 keys for the tail");
 #pragma unroll
-      for (int c = 8; c < kPrefillKeys; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], p[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      for (int c = 8; c + 16 <= kPrefillKeys; c += 16) {   // keys 8 .. 119
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], p[c + i], p[c + 8 + i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], p[kPrefillKeys - 8 + i]);   // 120 .. 127
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7])) * mul;
       const float m_new = fmaxf(m_ref, mx);
       const bool need = m_new > m_ref + kRescaleSlack;
       float alpha = 1.f;
@@ -397,10 +410,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       l *= alpha;
       const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-      const float2 negm = make_float2(-m_use, -m_use), one2 = make_float2(1.f, 1.f);
+      const float2 negm = make_float2(-m_use, -m_use), mul2 = make_float2(mul, mul);
 #pragma unroll
       for (int c = 0; c < kPrefillKeys; c += 2) {
-        const float2 x = ffma2(make_float2(p[c], p[c + 1]), one2, negm);
+        const float2 x = ffma2(make_float2(p[c], p[c + 1]), mul2, negm);   // S * scale - m
         p[c] = ex2(x.x);
         p[c + 1] = ex2(x.y);
       }
@@ -416,22 +429,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         for (int i = 0; i < 32; ++i) {
           const float x0 = p[64 * half + 2 * i], x1 = p[64 * half + 2 * i + 1];
           if constexpr (BF16) {
-            // hi = p rounded to bf16 by an integer add on the bit pattern (ties
-            // away from zero), lo = the exact fp32 remainder rounded the same way
-            const uint32_t b0 = __float_as_uint(x0) + 0x8000u, b1 = __float_as_uint(x1) + 0x8000u;
+            // hi = the top 16 bits of p (p truncated to bf16, remainder below
+            // 2^-7 p), lo = the exact fp32 remainder p - hi >= 0 truncated the
+            // same way: P keeps at least 14 significant bits (error < 2^-14 p),
+            // with no rounding arithmetic and no conversion-unit work
+            const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
             h[i] = __byte_perm(b0, b1, 0x7632);
             const float2 r = ffma2(make_float2(__uint_as_float(b0 & 0xffff0000u),
                                                __uint_as_float(b1 & 0xffff0000u)),
                                    make_float2(-1.f, -1.f), make_float2(x0, x1));
-            lo[i] = __byte_perm(__float_as_uint(r.x) + 0x8000u, __float_as_uint(r.y) + 0x8000u,
-                                0x7632);
-            lsum[i & 3].x += x0;
-            lsum[i & 3].y += x1;
+            lo[i] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
+            lsum[i & 3] = ffma2(make_float2(x0, x1), make_float2(1.f, 1.f), lsum[i & 3]);
           } else {
             h[i] = pack2<false>(x0, x1);
-            const float2 hf = unpack2<false>(h[i]);
-            lsum[i & 3].x += hf.x;
-            lsum[i & 3].y += hf.y;
+            lsum[i & 3] = ffma2(unpack2<false>(h[i]), make_float2(1.f, 1.f), lsum[i & 3]);
           }
         }
         tmem_st32u(t_lane + s_col + 32 * half, h);
