@@ -701,9 +701,10 @@ def recorded_traffic(config: str, kernel: str, context_tokens: int):
     return None
 
 
-# sources off the decode path whose traffic profiles/traffic.json records: the
-# chunked-prefill kernel, its tensor-core helpers and the shared-prefix kernel
-OFF_DECODE_PATH = ("pa_prefill.cuh", "pa_umma.cuh", "pa_shared_prefix.cuh")
+# sources off the 16-bit decode path whose traffic profiles/traffic.json
+# records: the chunked-prefill kernel, its tensor-core helpers, the
+# shared-prefix kernel and the fp8 page steps
+OFF_DECODE_PATH = ("pa_prefill.cuh", "pa_umma.cuh", "pa_shared_prefix.cuh", "pa_decode_fp8.cuh")
 
 
 def kernel_source_digest(csrc: Path | None = None) -> str:

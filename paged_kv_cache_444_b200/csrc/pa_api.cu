@@ -251,7 +251,8 @@ pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cach
               : launch_decode_d<128, false>(km, vm, a, grid, max_pages, stream);
 }
 
-// Decode over E4M3 caches (head_dim 128): same kernel, fp8 page steps.
+// >>> fp8 KV cache launch: decode over E4M3 caches (head_dim 128), same
+// kernel, fp8 page steps.
 pa_status run_decode_fp8(DecodeArgs a, const void* key_cache, const void* value_cache,
                          int64_t num_seqs, int64_t num_blocks, pa_dtype dtype,
                          cudaStream_t stream) {
@@ -263,24 +264,19 @@ pa_status run_decode_fp8(DecodeArgs a, const void* key_cache, const void* value_
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
   const int64_t max_pages = a.max_blocks_per_seq;
   if (dtype == PA_BF16) {
-    if (a.group == 1)
-      return launch_decode_t<128, true, SimtFp8Warp<128, true>, 1>(km, vm, a, grid, max_pages,
-                                                                  stream);
     if (a.group <= 8)
       return launch_decode_t<128, true, MmaFp8Warp<128, true, false>, 1>(km, vm, a, grid,
                                                                         max_pages, stream);
     return launch_decode_t<128, true, MmaFp8Warp<128, true, true>, 1>(km, vm, a, grid, max_pages,
                                                                      stream);
   }
-  if (a.group == 1)
-    return launch_decode_t<128, false, SimtFp8Warp<128, false>, 1>(km, vm, a, grid, max_pages,
-                                                                  stream);
   if (a.group <= 8)
     return launch_decode_t<128, false, MmaFp8Warp<128, false, false>, 1>(km, vm, a, grid,
                                                                         max_pages, stream);
   return launch_decode_t<128, false, MmaFp8Warp<128, false, true>, 1>(km, vm, a, grid, max_pages,
                                                                      stream);
 }
+// <<< fp8 KV cache launch
 
 pa_status check_fp8_scales(float k_scale, float v_scale) {
   if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f))
@@ -462,6 +458,7 @@ pa_status pa_reduce(void* out, const float* tmp_out, const float* max_logits,
                    static_cast<int>(partition_size), static_cast<int>(max_partitions));
 }
 
+// >>> fp8 KV cache entry points
 pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, int64_t key_stride,
                                    int64_t value_stride, void* key_cache, void* value_cache,
                                    const int64_t* slot_mapping, int64_t num_tokens,
@@ -557,6 +554,7 @@ pa_status pa_decode_split_fp8(float* tmp_out, float* max_logits, float* exp_sums
   return run_decode_fp8(a, key_cache, value_cache, num_seqs, num_blocks, dtype,
                         as_stream(stream));
 }
+// <<< fp8 KV cache entry points
 
 // >>> host-buffer step (pa_decode_step_host): one decode step from host
 // buffers.  Workspace layout (each part 256-byte aligned): key, value,
