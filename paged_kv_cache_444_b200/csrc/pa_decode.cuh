@@ -17,19 +17,19 @@
 // Gather.  A page of one KV head is 16 rows of head_dim 16-bit values,
 // num_kv_heads*head_dim elements apart.  One TMA tensor-tile load moves a
 // 16 x 64-element box (2 KB) of it into shared memory, 128-byte swizzled so
-// that both the row-wise reads of the CUDA-core path and the 8-row ldmatrix
-// reads of the tensor-core path are bank-conflict free.  Lane 0 of the warp
+// that the 8-row ldmatrix reads of the page step are bank-conflict free.  Lane 0 of the warp
 // issues the loads for a page NST pages ahead, right after the page that last
 // used the stage has been consumed.  The block id of every page comes from a
 // window of 32 ids held one per lane (a second window is prefetched).
 //
-// Math.  fp32 throughout.  For one query head per KV head (MHA) the dot
-// products and the P.V accumulation run on the CUDA cores with packed fp32
-// FMA (FFMA2).  For a GQA group (2..16 query heads per KV head) the group is
-// a small dense contraction: S = Q K^T and O += P V run as mma.sync m16n8k16
-// with fp32 accumulators (Q rows padded to 16, P rounded to the cache dtype
-// for the second product).  The softmax is online, in base 2 with
-// scale*log2(e) folded into the logits, with warp-shuffle max reductions.
+// Math.  fp32 throughout.  The G query heads of a KV head (1 for MHA, up to
+// 16 for GQA) form a small dense contraction: S = Q K^T and O += P V run as
+// mma.sync m16n8k16 with fp32 accumulators (Q rows padded to 16, P in the
+// cache dtype for the second product, bf16 as a hi + lo pair).  For one head
+// the tile has a single live row: the tensor cores take the products off the
+// issue path, which measured faster than packed fp32 FMA on the CUDA cores.
+// The softmax is online, in base 2 with scale*log2(e) folded into the logits,
+// with warp-shuffle max reductions.
 #pragma once
 
 #include "pa_device.cuh"
@@ -74,8 +74,7 @@ struct DecodeSmem {
   static constexpr int kStageBytes = 2 * kPageBytes;      // K page + V page
   static constexpr int kStagesBytes = kWarps * NST * kStageBytes;
   static constexpr int kBarOffset = kStagesBytes;
-  static constexpr int kProbOffset = kBarOffset + kWarps * NST * 8;
-  static constexpr int kRedMOffset = kProbOffset + kWarps * kPage * 4;
+  static constexpr int kRedMOffset = kBarOffset + kWarps * NST * 8;
   static constexpr int kRedLOffset = kRedMOffset + kWarps * 16 * 4;
   static constexpr int kPartMOffset = kRedLOffset + kWarps * 16 * 4;
   static constexpr int kPartLOffset = kPartMOffset + 16 * 4;
@@ -96,7 +95,7 @@ __device__ __forceinline__ uint32_t page_chunk(uint32_t base, int r, int c) {
 }
 
 // ---------------------------------------------------------------------------
-// Per-warp state and page step: tensor-core path (GQA groups)
+// Per-warp state and page step (tensor cores, every group size)
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool TWO_ROWS>
 struct MmaWarp {
@@ -125,9 +124,8 @@ struct MmaWarp {
   }
 
   __device__ __forceinline__ void page(uint32_t kbase, uint32_t vbase, int tok0, int t_end,
-                                       float scale_log2, int lane, float* probs) {
+                                       float scale_log2, int lane) {
     page_rows(kbase, vbase, tok0, t_end, t_end, scale_log2, lane);
-    (void)probs;
   }
 
   // One page with a token limit per row: row r0 (lane/4) sees tokens < lim0,
@@ -275,118 +273,6 @@ struct MmaWarp {
           red_l[r1] = l1;
         }
       }
-    }
-  }
-};
-
-// ---------------------------------------------------------------------------
-// Per-warp state and page step: CUDA-core path (one query head per KV head)
-// ---------------------------------------------------------------------------
-template <int D, bool BF16>
-struct SimtWarp {
-  static_assert(D == 64 || D == 128, "CUDA-core path is built for head_dim 64 and 128");
-  static constexpr int QCH = D / 16;     // 16-byte chunks per lane in Q.K (half a row)
-  static constexpr int VCH = D / 8;      // 16-byte chunks per row
-  static constexpr int TG = 32 / VCH;    // token groups in P.V
-  static constexpr int TPL = kPage / TG; // tokens per lane in P.V
-  float2 qf[QCH * 4];                    // this lane's half of q, in its read order
-  float2 acc[4];                         // 8 output dims of one token group
-  float m, l;
-  uint32_t kxor;                         // per-lane chunk swizzle for Q.K reads
-  int kbox;                              // box offset (bytes) of this lane's half row
-
-  __device__ __forceinline__ void init(const uint16_t* q_row, int, int lane) {
-    const int tok = lane >> 1, hf = lane & 1;
-    kxor = static_cast<uint32_t>(((hf * 4) ^ (tok & 7)) << 4);
-    kbox = (D == 128 ? hf * kBoxBytes : 0) + tok * 128;
-#pragma unroll
-    for (int k = 0; k < QCH; ++k) {
-      // step k reads logical chunk (D==128 ? 8*hf : 0) + (k ^ 4*hf) of the row
-      const int c = (D == 128 ? hf * 8 : 0) + (k ^ (hf * 4));
-      const uint4 raw = *reinterpret_cast<const uint4*>(q_row + c * 8);
-      qf[k * 4 + 0] = unpack2<BF16>(raw.x);
-      qf[k * 4 + 1] = unpack2<BF16>(raw.y);
-      qf[k * 4 + 2] = unpack2<BF16>(raw.z);
-      qf[k * 4 + 3] = unpack2<BF16>(raw.w);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
-    m = -INFINITY;
-    l = 0.f;
-  }
-
-  __device__ __forceinline__ void page(uint32_t kbase, uint32_t vbase, int tok0, int t_end,
-                                       float scale_log2, int lane, float* probs) {
-    const int tok = lane >> 1, hf = lane & 1;
-    // ---- q . k for token `tok`, this lane's half of the row ----
-    float2 d2 = make_float2(0.f, 0.f);
-    const uint32_t krow = kbase + kbox;
-#pragma unroll
-    for (int k = 0; k < QCH; ++k) {
-      const uint4 raw = lds128(krow + ((static_cast<uint32_t>(k) << 4) ^ kxor));
-      d2 = ffma2(qf[k * 4 + 0], unpack2<BF16>(raw.x), d2);
-      d2 = ffma2(qf[k * 4 + 1], unpack2<BF16>(raw.y), d2);
-      d2 = ffma2(qf[k * 4 + 2], unpack2<BF16>(raw.z), d2);
-      d2 = ffma2(qf[k * 4 + 3], unpack2<BF16>(raw.w), d2);
-    }
-    float dot = d2.x + d2.y;
-    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-    const float x = (tok0 + tok) < t_end ? dot * scale_log2 : -INFINITY;
-    float mx = x;
-#pragma unroll
-    for (int o = 2; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float mn = fmaxf(m, mx);
-    const float al = ex2(m - mn);
-    m = mn;
-    const float p = ex2(x - mn);
-    l = l * al + (hf ? 0.f : p);
-    if (hf == 0) probs[tok] = p;
-    __syncwarp();
-    // ---- O = O * alpha + sum_j p_j v_j over this lane's tokens and 8 dims ----
-    const int cc = lane % VCH, tg = lane / VCH;
-    const float2 al2 = make_float2(al, al);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] = fmul2(acc[i], al2);
-    float pj[TPL];
-#pragma unroll
-    for (int i = 0; i < TPL; i += 4) {
-      const float4 p4 = *reinterpret_cast<const float4*>(probs + tg * TPL + i);
-      pj[i] = p4.x; pj[i + 1] = p4.y; pj[i + 2] = p4.z; pj[i + 3] = p4.w;
-    }
-    const uint32_t vrow = vbase + (cc >> 3) * kBoxBytes + tg * TPL * 128;
-    const uint32_t vx = static_cast<uint32_t>((cc & 7) ^ ((tg * TPL) & 7));
-#pragma unroll
-    for (int i = 0; i < TPL; ++i) {
-      const uint4 raw = lds128(vrow + i * 128 + ((vx ^ static_cast<uint32_t>(i)) << 4));
-      const float2 pp = make_float2(pj[i], pj[i]);
-      acc[0] = ffma2(pp, unpack2<BF16>(raw.x), acc[0]);
-      acc[1] = ffma2(pp, unpack2<BF16>(raw.y), acc[1]);
-      acc[2] = ffma2(pp, unpack2<BF16>(raw.z), acc[2]);
-      acc[3] = ffma2(pp, unpack2<BF16>(raw.w), acc[3]);
-    }
-  }
-
-  __device__ __forceinline__ void publish(float* red_acc, float* red_m, float* red_l, int,
-                                          int lane) {
-    float lt = l;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
-#pragma unroll
-    for (int o = VCH; o < 32; o <<= 1) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[i].x += __shfl_xor_sync(0xffffffffu, acc[i].x, o);
-        acc[i].y += __shfl_xor_sync(0xffffffffu, acc[i].y, o);
-      }
-    }
-    if (lane < VCH) {
-      float4* dst = reinterpret_cast<float4*>(red_acc + lane * 8);
-      dst[0] = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
-      dst[1] = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
-    }
-    if (lane == 0) {
-      red_m[0] = m;
-      red_l[0] = lt;
     }
   }
 };
@@ -575,7 +461,6 @@ __global__ void __launch_bounds__(kThreads)
 
   const uint32_t stage0 = smem_addr(smem) + warp * NST * L::kStageBytes;
   const uint32_t bar0 = smem_addr(smem + L::kBarOffset) + warp * NST * 8;
-  float* probs = reinterpret_cast<float*>(smem + L::kProbOffset) + warp * kPage;
 
   if (lane == 0) {
     for (int i = 0; i < NST; ++i) mbar_init(bar0 + i * 8, 1);
@@ -646,7 +531,7 @@ __global__ void __launch_bounds__(kThreads)
     const uint32_t kb = stage0 + stg * L::kStageBytes;
     const int tok0 = (first_page + page0 + k * pstride) * kPage;
     if (tok0 + kPage > ctx) zero_page_tail<L::kBoxesPerRow>(kb + L::kPageBytes, ctx - tok0, lane);
-    st.page(kb, kb + L::kPageBytes, tok0, t_end, a.scale_log2, lane, probs);
+    st.page(kb, kb + L::kPageBytes, tok0, t_end, a.scale_log2, lane);
     __syncwarp();
     if (k + NST < my_pages) issue(k + NST);
   }

@@ -99,7 +99,7 @@ struct MmaFp8Warp {
   }
 
   __device__ __forceinline__ void page(uint32_t kbase, uint32_t vbase, int tok0, int t_end,
-                                       float scale_log2, int lane, float*) {
+                                       float scale_log2, int lane) {
     const int tig = lane & 3;
     // ---- S = Q K^T: one x4 ldmatrix covers two k-steps for both 8-token n-tiles ----
     float sc[2][4];
