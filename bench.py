@@ -368,6 +368,31 @@ class _Null:
         return False
 
 
+def bind_to_gpu_local_cpus(device_index: int) -> str:
+    """Restrict this process to the CPUs on the GPU's own NUMA node, before any
+    pinned host buffer is allocated, so that the staging memory of the
+    host-buffer step is first touched (and so placed) on that node and the PCIe
+    copies do not cross the socket link.  Reads sysfs only; changes nothing
+    outside this process.  Returns a short description for the JSON line."""
+    try:
+        p = torch.cuda.get_device_properties(device_index)
+        dev = Path("/sys/bus/pci/devices") / (
+            f"{p.pci_domain_id:04x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0")
+        spec = (dev / "local_cpulist").read_text().strip()
+        node = (dev / "numa_node").read_text().strip()
+        cpus: set[int] = set()
+        for part in spec.split(","):
+            lo, _, hi = part.partition("-")
+            cpus.update(range(int(lo), int(hi or lo) + 1))
+        cpus &= os.sched_getaffinity(0)
+        if not cpus:
+            return "unbound (no GPU-local CPU available to this process)"
+        os.sched_setaffinity(0, cpus)
+        return f"{len(cpus)} GPU-local CPUs (NUMA node {node})"
+    except Exception as e:  # pragma: no cover - depends on the box
+        return f"unbound ({type(e).__name__})"
+
+
 def e2e_steps(step: Step, steps: int, warmup: int, world: int, device):
     """The same step through the C ABI from host buffers (pa_decode_step_host):
     every step copies its inputs in from pinned host memory, writes the cache,
@@ -520,6 +545,7 @@ def cpu_baseline(cfg, context_lens, block_tables, batch, budget_s: float = 12.0)
 def run_native(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    host_cpus = bind_to_gpu_local_cpus(local)
     init_dist(world, "nccl")
     from paged_kv_cache_444_b200 import load
     load()
@@ -628,7 +654,8 @@ def run_native(args, world, rank, local):
         "e2e": {"value": round(total_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "api": "pa_decode_step_host (C ABI, pinned host buffers in and out)"},
+                "api": "pa_decode_step_host (C ABI, pinned host buffers in and out)",
+                "host_cpus": host_cpus},
         "clocks": clocks.summary(),
     }
     if results:
