@@ -118,6 +118,89 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
   return true;
 }
 
+// ---------------------------------------------------------------------------
+// Longest-first item order.  A unit is (sequence, tile pair); its cost grows
+// with the keys its last query token sees, hist + min(T2 (p + 1), q_len)
+// (hist = context - q_len, T2 = query tokens of a tile pair).  CTAs start in
+// grid order, so handing out units by descending key count (ties by
+// sequence, then pair) starts the long ones first and fills the tail with
+// short ones; the K/V a sequence's pairs share is read again from L2.
+// ---------------------------------------------------------------------------
+constexpr int kLptSeqsPerLane = 8;  // one warp ranks up to 256 sequences
+
+// floor(x / d) for x >= 0 and d >= 2 from a float reciprocal: below 2^24 both
+// are exact floats and the quotient (< 2^23) comes out within 1 of its floor,
+// which one correction step fixes.
+__device__ __forceinline__ int div_floor(int x, int d, float inv_d) {
+  if (x >= (1 << 24)) return x / d;
+  int q = __float2int_rz(__int2float_rn(x) * inv_d);
+  if (q * d > x) --q;
+  else if ((q + 1) * d <= x) ++q;
+  return q;
+}
+
+// One sequence as the ranking sees it: hist = context - q_len, its tile
+// pairs, and q_len (-1 marks an invalid sequence, which has no units).
+struct LptSeq {
+  int hist[kLptSeqsPerLane], q_len[kLptSeqsPerLane], pairs[kLptSeqsPerLane];
+};
+
+// Pairs of sequence i whose key count exceeds K.
+__device__ __forceinline__ int pairs_above(const LptSeq& q, int i, int t2, float inv_t2, int K) {
+  if (q.q_len[i] <= 0) return 0;
+  const int x = K - q.hist[i];
+  if (x >= q.q_len[i]) return 0;
+  return x < 0 ? q.pairs[i] : q.pairs[i] - div_floor(x, t2, inv_t2);  // T2 (p + 1) <= x fall short
+}
+
+// The unit of rank j (0 = most keys), found by one warp: a binary search for
+// its key count K (the least K with at most j units above it), then its place
+// among the units with exactly K keys in (sequence, pair) order.  Returns
+// false when fewer than j + 1 units exist.
+__device__ __forceinline__ bool prefill_unit_of_rank(const LptSeq& q, int max_keys, int t2, int j,
+                                                     int lane, int& s_out, int& p_out) {
+  const float inv_t2 = 1.f / static_cast<float>(t2);
+  auto above = [&](int K) {
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < kLptSeqsPerLane; ++i) c += pairs_above(q, i, t2, inv_t2, K);
+    return static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)));
+  };
+  if (above(-1) <= j) return false;
+  int lo = -1, hi = max_keys;  // above(lo) > j >= above(hi) = 0
+  while (hi - lo > 1) {
+    const int mid = lo + (hi - lo) / 2;
+    if (above(mid) <= j) hi = mid;
+    else lo = mid;
+  }
+  const int K = hi;
+  int t = j - above(K);  // index among the units with exactly K keys
+  bool found = false;
+#pragma unroll
+  for (int i = 0; i < kLptSeqsPerLane; ++i) {
+    const int below = pairs_above(q, i, t2, inv_t2, K - 1);
+    const int e = below - pairs_above(q, i, t2, inv_t2, K);
+    int inc = e;  // inclusive scan over the lanes (sequences i*32 + lane)
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, d);
+      if (lane >= d) inc += v;
+    }
+    const int total = __shfl_sync(0xffffffffu, inc, 31);
+    if (!found && t < total) {
+      const int src = __ffs(__ballot_sync(0xffffffffu, t < inc)) - 1;
+      const int before = __shfl_sync(0xffffffffu, inc - e, src);
+      // the pairs with exactly K keys follow the pairs - below with fewer
+      const int first = __shfl_sync(0xffffffffu, q.pairs[i] - below, src);
+      s_out = i * 32 + src;
+      p_out = first + (t - before);
+      found = true;
+    }
+    if (!found) t -= total;
+  }
+  return found;
+}
+
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap qmap,
@@ -138,20 +221,68 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   pdl_launch_dependents();
   pdl_wait();
 
-  // ---- work item: the last tile pairs of every sequence (most keys) first ----
-  const int per_pair = a.num_seqs * a.num_kv_heads;
-  int item = blockIdx.x;
-  const int pair = a.pairs_per_seq - 1 - item / per_pair;
-  item %= per_pair;
-  const int kvh = item % a.num_kv_heads;
-  const int s = item / a.num_kv_heads;
+  // ---- work item ----
+  const int cap = a.max_blocks_per_seq * kPage;
+  auto seq_valid = [&](int q0, int q_len, int ctx) {
+    return !(q0 < 0 || q_len < 0 || q0 > a.num_tokens - q_len || q_len > ctx || ctx > cap);
+  };
   const int G = a.group;
+  int s, pair, kvh;
+  if (a.num_seqs <= 32 * kLptSeqsPerLane) {
+    // longest first: CTA b takes unit b / Hk, KV head b % Hk
+    int* slot = reinterpret_cast<int*>(smem);  // stage area, not in use yet
+    if (warp == 0) {
+      LptSeq q;
+      int max_keys = 0;
+      const int t2 = 2 * a.tile_tokens;
+#pragma unroll
+      for (int i = 0; i < kLptSeqsPerLane; ++i) {
+        const int t = i * 32 + lane;
+        q.hist[i] = 0;
+        q.q_len[i] = -1;
+        q.pairs[i] = 0;
+        if (t < a.num_seqs) {
+          const int q0 = a.query_starts[t], ql = a.query_starts[t + 1] - q0;
+          const int ctx = a.context_lens[t];
+          if (seq_valid(q0, ql, ctx)) {
+            q.hist[i] = ctx - ql;
+            q.q_len[i] = ql;
+            q.pairs[i] = ql / t2 + (ql % t2 != 0);
+            max_keys = max(max_keys, ctx);
+          } else if (t == static_cast<int>(blockIdx.x)) {
+            record_error(kErrQuery, t);  // each sequence is checked by one CTA
+          }
+        }
+      }
+      max_keys = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(max_keys)));
+      int us = -1, up = 0;
+      const bool found = prefill_unit_of_rank(
+          q, max_keys, t2, static_cast<int>(blockIdx.x) / a.num_kv_heads, lane, us, up);
+      if (lane == 0) {
+        slot[0] = found ? us : -1;
+        slot[1] = up;
+      }
+    }
+    __syncthreads();
+    s = slot[0];
+    pair = slot[1];
+    kvh = static_cast<int>(blockIdx.x) % a.num_kv_heads;
+    __syncthreads();  // the stage area is about to be reused
+    if (s < 0) return;  // more CTAs than units: nothing to do
+  } else {
+    // the last tile pairs of every sequence (most keys) first
+    const int per_pair = a.num_seqs * a.num_kv_heads;
+    int item = blockIdx.x;
+    pair = a.pairs_per_seq - 1 - item / per_pair;
+    item %= per_pair;
+    kvh = item % a.num_kv_heads;
+    s = item / a.num_kv_heads;
+  }
 
   const int q0 = a.query_starts[s];
   const int q_len = a.query_starts[s + 1] - q0;
   const int ctx = a.context_lens[s];
-  const int cap = a.max_blocks_per_seq * kPage;
-  if (q0 < 0 || q_len < 0 || q0 > a.num_tokens - q_len || q_len > ctx || ctx > cap) {
+  if (!seq_valid(q0, q_len, ctx)) {
     if (threadIdx.x == 0 && kvh == 0 && pair == 0) record_error(kErrQuery, s);
     return;
   }

@@ -35,6 +35,29 @@ CASES = {
     "long_mha_f16_d64": (C["tiny"], dict(num_seqs=2, num_heads=2, num_kv_heads=2, num_blocks=300,
                                          ctx=("fixed", (2500, 1100)), seed=68), (300, 1100)),
 }
+
+
+def _mixed(seed, n, ctx_hi, q_hi):
+    """n contexts U[1, ctx_hi) and query lengths U[0, q_hi] capped by them
+    (some sequences bring no query tokens)."""
+    rng = np.random.default_rng(seed)
+    ctx = [int(c) for c in rng.integers(1, ctx_hi, n)]
+    q = [0 if rng.random() < 0.15 else int(min(c, rng.integers(1, q_hi + 1))) for c in ctx]
+    return tuple(ctx), tuple(q)
+
+
+# 40 sequences: the longest-first order ranks units across several 32-sequence
+# chunks, with many equal key counts and empty sequences among them
+_ctx, _q = _mixed(444_071, 40, 300, 70)
+CASES["many_seqs_gqa4_bf16"] = (C["gqa_llama3_8b"], dict(num_seqs=40, num_heads=8,
+                                                          num_kv_heads=2, num_blocks=1000,
+                                                          ctx=("fixed", _ctx), seed=71), _q)
+# more sequences than the longest-first order ranks: the fixed order instead
+_ctx, _q = _mixed(444_072, 300, 48, 6)
+CASES["fixed_order_300_seqs_f16"] = (C["gqa_llama3_8b"], dict(num_seqs=300, num_heads=4,
+                                                               num_kv_heads=2, dtype="f16",
+                                                               num_blocks=1200,
+                                                               ctx=("fixed", _ctx), seed=72), _q)
 # scale 1 instead of 1/sqrt(D): peaked rows whose running maximum jumps by more
 # than 2^8 between key blocks, so the output accumulator is rescaled
 SCALE = {"peaky_bf16": 1.0, "peaky_f16": 1.0}
@@ -129,6 +152,20 @@ def test_prefill_reports_query_longer_than_context(cuda_device):
     with pytest.raises(PagedAttentionError) as e:
         pa_check_error()
     assert e.value.detail >> 56 == 7 and e.value.detail & 0xffff == 1
+
+
+def test_prefill_reports_invalid_sequence_in_fixed_order(cuda_device):
+    """Past 256 sequences the units go out in the fixed order; an invalid
+    sequence is still skipped and reported, and the others are written."""
+    cfg, b, query, starts, qlens = _case("fixed_order_300_seqs_f16", cuda_device)
+    bad = next(i for i, q in enumerate(qlens) if q > 0 and i > 200)
+    b.context_lens[bad] = qlens[bad] - 1                    # q_len > context
+    out = torch.zeros_like(query)
+    pa_prefill(out, query, b.key_cache, b.value_cache, b.block_tables, b.context_lens, starts,
+               cfg.scale, max(qlens))
+    with pytest.raises(PagedAttentionError) as e:
+        pa_check_error()
+    assert e.value.detail >> 56 == 7 and e.value.detail & 0xffff == bad
 
 
 def test_prefill_full_size_sampled(cuda_device, oracle_lib):
