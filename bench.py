@@ -368,6 +368,17 @@ class _Null:
         return False
 
 
+def parse_cpulist(spec: str) -> set[int]:
+    """The CPUs of a sysfs cpulist such as "0-15,32-47" (an empty list: none)."""
+    cpus: set[int] = set()
+    for part in spec.strip().split(","):
+        if not part:
+            continue
+        lo, _, hi = part.partition("-")
+        cpus.update(range(int(lo), int(hi or lo) + 1))
+    return cpus
+
+
 def bind_to_gpu_local_cpus(device_index: int) -> str:
     """Restrict this process to the CPUs on the GPU's own NUMA node, before any
     pinned host buffer is allocated, so that the staging memory of the
@@ -378,12 +389,8 @@ def bind_to_gpu_local_cpus(device_index: int) -> str:
         p = torch.cuda.get_device_properties(device_index)
         dev = Path("/sys/bus/pci/devices") / (
             f"{p.pci_domain_id:04x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0")
-        spec = (dev / "local_cpulist").read_text().strip()
+        cpus = parse_cpulist((dev / "local_cpulist").read_text())
         node = (dev / "numa_node").read_text().strip()
-        cpus: set[int] = set()
-        for part in spec.split(","):
-            lo, _, hi = part.partition("-")
-            cpus.update(range(int(lo), int(hi or lo) + 1))
         cpus &= os.sched_getaffinity(0)
         if not cpus:
             return "unbound (no GPU-local CPU available to this process)"

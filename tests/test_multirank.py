@@ -65,3 +65,11 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["value"] > 0
     assert rec["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_parse_cpulist():
+    """The sysfs CPU lists bench.py binds each rank to."""
+    import bench
+    assert bench.parse_cpulist("0-15\n") == set(range(16))
+    assert bench.parse_cpulist("0-3,8,10-11") == {0, 1, 2, 3, 8, 10, 11}
+    assert bench.parse_cpulist("") == set()
