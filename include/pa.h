@@ -252,23 +252,29 @@ pa_status pa_decode_split_fp8(float *tmp_out, float *max_logits, float *exp_sums
  * pa_decode_step_host -- one whole decode step of one attention layer for a
  * caller whose per-step inputs are in HOST memory (pinned memory makes the
  * copies asynchronous; pageable memory works but the copies then block).
- * Enqueues on `stream`: host->device copies of key and value [S,Hk,D] (one
- * new token per sequence) and slot_mapping [S] int64 into `workspace`, then
- * the cache write (pa_reshape_and_cache) while query [S,H,D], block_tables
- * [S,MB] int32 and context_lens [S] int32 are copied on a library-owned side
- * stream (forked from and joined back to `stream` with events); attention
- * (pa_decode, or pa_decode_split + pa_reduce when partition_size > 0); and the
- * output [S,H,D]: written by the attention kernel straight into out_host when
- * out_host is page-locked memory the device can address, else copied back.
- * Returns without waiting: out_host is valid once the stream has reached this
- * point.  Calls on one stream are ordered; the workspace is reused per call.
+ * Enqueues on `stream`: the cache write (pa_reshape_and_cache) of key and
+ * value [S,Hk,D] (one new token per sequence) at slot_mapping [S] int64,
+ * while query [S,H,D], block_tables [S,MB] int32 and context_lens [S] int32
+ * are copied into `workspace` on a library-owned side stream (forked from and
+ * joined back to `stream` with events).  When key, value and slot_mapping are
+ * all page-locked memory the device can address (16-, 16- and 8-byte
+ * aligned), the cache write reads them there, over the host link; otherwise
+ * they are first copied into `workspace` and the side stream forks after that
+ * copy.  Then attention (pa_decode, or pa_decode_split + pa_reduce when
+ * partition_size > 0); and the output [S,H,D]: written by the attention
+ * kernel straight into out_host when out_host is page-locked memory the
+ * device can address, else copied back.
+ * Returns without waiting: the host inputs must stay unchanged, and out_host
+ * is valid, once the stream has reached this point.  Calls on one stream are
+ * ordered; the workspace is reused per call.
  *   key_cache, value_cache   device caches as for pa_decode (stay resident)
  *   workspace                caller-owned device memory, 256-byte aligned, of
  *                            pa_decode_step_host_workspace_bytes(...) bytes
  * Packed inputs: pass value_host = slot_mapping_host = NULL when value and
  * slot_mapping follow key_host in one host buffer at the workspace's relative
  * offsets (key, value, slot_mapping, each part starting 256-byte aligned after
- * the previous one); the three then go over in one transfer.  Likewise
+ * the previous one); the three then go over in one transfer (or are read in
+ * place).  Likewise
  * block_tables_host = context_lens_host = NULL for query, block_tables,
  * context_lens packed after query_host.  Otherwise every part is copied on
  * its own (parts that merely happen to be adjacent are never merged).

@@ -694,19 +694,37 @@ pa_status pa_decode_step_host(void* out_host, const void* query_host, const void
   const Copy attend_in[3] = {{d_query, query_host, q_bytes},
                              {d_tables, block_tables_host, num_seqs * max_blocks_per_seq * 4},
                              {d_lens, context_lens_host, num_seqs * 4}};
-  // The new rows go first; then (fork) the side stream copies the query and
-  // tables while this stream writes the rows into the caches.  The fork comes
-  // after all earlier work on this stream, so nothing still reads the
-  // workspace the side stream overwrites.
-  if (!copy_in(write_in, 3, 0, s) || cudaEventRecord(fork->fork, s) != cudaSuccess ||
+  // The cache write reads the new rows straight from host memory when all
+  // three parts are page-locked memory the device can address: its reads then
+  // share the link with the side stream's copy of the query and tables, and
+  // nothing waits for a separate copy of the rows.  Otherwise the rows are
+  // copied into the workspace first, and the side stream forks after that copy.
+  const void* src_key = device_view_of_host(const_cast<void*>(key_host));
+  const void* src_value = nullptr;
+  const void* src_slots = nullptr;
+  if (src_key && value_host) {
+    src_value = device_view_of_host(const_cast<void*>(value_host));
+    src_slots = device_view_of_host(const_cast<int64_t*>(slot_mapping_host));
+  } else if (src_key) {  // packed after key_host, at the workspace's offsets
+    src_value = static_cast<const uint8_t*>(src_key) + (l.off[1] - l.off[0]);
+    src_slots = static_cast<const uint8_t*>(src_key) + (l.off[2] - l.off[0]);
+  }
+  const bool read_direct = src_key && src_value && src_slots && aligned16(src_key) &&
+                           aligned16(src_value) &&
+                           (reinterpret_cast<uintptr_t>(src_slots) & 7u) == 0;
+  // The fork comes after all earlier work on this stream, so nothing still
+  // reads the workspace the side stream overwrites.
+  if ((!read_direct && !copy_in(write_in, 3, 0, s)) ||
+      cudaEventRecord(fork->fork, s) != cudaSuccess ||
       cudaStreamWaitEvent(fork->side, fork->fork, 0) != cudaSuccess ||
       !copy_in(attend_in, 3, 3, fork->side) ||
       cudaEventRecord(fork->join, fork->side) != cudaSuccess)
     return PA_ERR_CUDA;
-  pa_status st = pa_reshape_and_cache(d_key, d_value, num_kv_heads * head_dim,
-                                      num_kv_heads * head_dim, key_cache, value_cache, d_slots,
-                                      num_seqs, num_kv_heads, head_dim, num_blocks, block_size,
-                                      dtype, stream);
+  pa_status st = pa_reshape_and_cache(
+      read_direct ? src_key : d_key, read_direct ? src_value : d_value, num_kv_heads * head_dim,
+      num_kv_heads * head_dim, key_cache, value_cache,
+      read_direct ? static_cast<const int64_t*>(src_slots) : d_slots, num_seqs, num_kv_heads,
+      head_dim, num_blocks, block_size, dtype, stream);
   if (st != PA_OK) return st;
   // join, then attend; the output goes straight into out_host when that is
   // page-locked memory the device can address, else through the workspace

@@ -392,6 +392,30 @@ def test_host_step_unpacked_inputs_pageable_output(name, ps, dev, oracle_lib):
     _check_close(step.out, ref, cfg, f"host step {name}, unpacked inputs, pageable output")
 
 
+@pytest.mark.parametrize("pageable", [("key", "value", "slot_mapping"), ("value",)],
+                         ids=["all_rows_pageable", "value_pageable"])
+def test_host_step_pageable_new_rows(pageable, dev, oracle_lib):
+    """pa_decode_step_host when some of the new rows are in pageable memory:
+    the cache write cannot read them from host memory, so all three are copied
+    into the workspace first (with every part pinned it reads them directly)."""
+    from paged_kv_cache_444_b200 import HostStep
+    cfg = SMALL["gqa_small"]
+    batch = workloads.make_batch(cfg, dev)
+    host = HostCopy(batch)
+    ref, kc_ref, _ = oracle_step(oracle_lib, host)
+    step = HostStep(batch.key_cache, batch.value_cache, cfg.num_seqs, cfg.num_heads,
+                    batch.block_tables.shape[1], cfg.scale, 0, cfg.torch_dtype)
+    for name_ in ("query", "key", "value", "slot_mapping", "block_tables", "context_lens"):
+        t = getattr(batch, name_).cpu().clone()
+        setattr(step, name_, t if name_ in pageable else t.pin_memory())
+    step.out.fill_(float("nan"))
+    step.run()
+    torch.cuda.synchronize()
+    pa_check_error()
+    assert np.array_equal(bits(batch.key_cache), kc_ref)
+    _check_close(step.out, ref, cfg, f"host step, pageable {pageable}")
+
+
 @pytest.mark.parametrize("name,ps", [("gqa_small", 0), ("long_small", 64), ("tiny", 0)])
 def test_plan_replays_from_a_cuda_graph(name, ps, dev, oracle_lib):
     """A DecodePlan run eagerly, and the same plan captured once in a CUDA
