@@ -144,13 +144,14 @@ struct Stages { static constexpr int value = D == 64 ? PA_STAGES_D64 : PA_STAGES
 // A power of two, at most kMaxCluster, and no more than the device can
 // co-schedule for this kernel.
 template <class K>
-int pick_cluster(K kernel, int smem_bytes, int64_t max_pages, int* cache) {
+int pick_cluster(K kernel, int smem_bytes, int64_t max_pages, std::atomic<int>* cache) {
   int want = 1;
   while (want < kMaxCluster && static_cast<int64_t>(want) * PA_CLUSTER_TABLE_PAGES < max_pages)
     want *= 2;
   int dev = 0;
   if (want == 1 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
-  if (cache[dev] == 0) {  // largest schedulable cluster size for this kernel on this device
+  int known = cache[dev].load(std::memory_order_relaxed);
+  if (known == 0) {  // largest schedulable cluster size for this kernel on this device
     int best = 1;
     for (int c = kMaxCluster; c > 1; c /= 2) {
       cudaLaunchConfig_t cfg = {};
@@ -171,9 +172,10 @@ int pick_cluster(K kernel, int smem_bytes, int64_t max_pages, int* cache) {
       }
       cudaGetLastError();
     }
-    cache[dev] = best;
+    cache[dev].store(best, std::memory_order_relaxed);  // every thread finds the same value
+    known = best;
   }
-  return want < cache[dev] ? want : cache[dev];
+  return want < known ? want : known;
 }
 
 template <int D, bool BF16, class Warp, int EB = 2>
@@ -183,7 +185,7 @@ pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeAr
   using L = DecodeSmem<D, NST, EB>;
   auto kernel = paged_decode_kernel<D, NST, BF16, Warp, EB>;
   static std::atomic<uint64_t> done{0};
-  static int cluster_cache[kMaxDevices] = {};
+  static std::atomic<int> cluster_cache[kMaxDevices] = {};
   if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
   const bool split = a.tmp_out != nullptr;
   const int c = split ? 1 : pick_cluster(kernel, L::kAlloc, max_pages, cluster_cache);
@@ -872,7 +874,7 @@ pa_status launch_shared_prefix_t(const CUtensorMap& km, const CUtensorMap& vm,
   using L = DecodeSmem<D, NST>;
   auto kernel = shared_prefix_decode_kernel<D, NST, BF16>;
   static std::atomic<uint64_t> done{0};
-  static int cluster_cache[kMaxDevices] = {};
+  static std::atomic<int> cluster_cache[kMaxDevices] = {};
   if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
   // one cluster size for the launch: as large as PA_SHARED_CLUSTER if the
   // device can co-schedule it, and 1 when no item can exceed the threshold
