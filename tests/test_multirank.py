@@ -1,6 +1,6 @@
 """Multi-rank plumbing of bench.py on CPU with the gloo backend, world size 2:
 the max/sum-over-ranks timing reductions, the barrier, and the reference arm
-launched through torch.distributed.run exactly as the driver launches it
+launched through torch.distributed.run as a multi-GPU run is launched
 (rank 0 alone prints one JSON line, the other rank exits 0)."""
 import json
 import os
