@@ -6,11 +6,15 @@
 
 One step = the whole hot path over one seeded synthetic decode batch:
 pa_reshape_and_cache (one new token per sequence), then pa_decode, or
-pa_decode_split + pa_reduce for the long-context workload.  Inputs are
-resident in HBM when the timed region starts; the K/V bytes each step reads
-exceed the 126 MB L2, so no flush is needed between steps.  Multi-GPU runs
-are independent replicas (one batch per GPU, no collective on the data
-path); timing is the max over ranks of the CUDA-event time.
+pa_decode_split + pa_reduce for the long-context workload (the default, the
+largest single-GPU one).  Inputs are resident in HBM when timing starts; the
+K/V bytes each step reads exceed the 126 MB L2, so no flush is needed
+between steps.  Timing: regions of exactly K steps, each bracketed by a
+barrier and a device synchronise on both sides and timed with CUDA events,
+repeated until --min-timed-s is covered; the value uses the median region.
+Each kernel is also timed alone, per launch, with L2 flushed before every
+launch (the roofline figure).  Multi-GPU runs are independent replicas (one
+batch per GPU, no collective on the data path); times are the max over ranks.
 
 Rank 0 prints ONE JSON line.
 """
@@ -33,7 +37,7 @@ sys.path.insert(0, str(ROOT))
 
 from paged_kv_cache_444_b200 import workloads  # noqa: E402
 
-MAIN_CONFIG = "mha_llama2_7b"
+MAIN_CONFIG = "long_context_split"
 METRIC = "paged decode attn achieved HBM GB/s & % of peak; decode tokens/s (1 B200)"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -157,9 +161,82 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-# the step, with CUDA events around each kernel
+# the step, its kernels, and how they are timed
 # ---------------------------------------------------------------------------
+L2_BYTES = 126 * 1024 * 1024
+
+
+class L2Flush:
+    """Writes a buffer of twice the L2 size, so that the next launch starts
+    with none of its inputs in L2.  Runs between timed launches, untimed."""
+
+    def __init__(self, device):
+        self.buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+
+    def __call__(self):
+        self.buf.zero_()
+
+
+def stats_ms(times) -> dict:
+    """Mean, median and p10 / p90 (nearest rank) of a list of times in ms."""
+    xs = sorted(float(t) for t in times)
+    pick = lambda f: xs[min(len(xs) - 1, max(0, int(round(f * (len(xs) - 1)))))]
+    return {"n": len(xs), "mean": statistics.fmean(xs), "median": statistics.median(xs),
+            "p10": pick(0.1), "p90": pick(0.9)}
+
+
+def launch_times(fn, reps: int, warmup: int, flush=None) -> list[float]:
+    """CUDA-event time (ms) of each of `reps` launches of fn() on the current
+    stream (the stream the binding launches on), each bracketed by its own
+    pair of events; with `flush`, L2 is flushed before every launch, outside
+    the events."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for a, b in evs:
+        if flush is not None:
+            flush()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def loop_ms(fn, reps: int, warmup: int) -> float:
+    """Average time (ms) of `reps` back-to-back launches of fn(): events at
+    the two ends only, so consecutive launches overlap as they would in use."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def kernel_stats(fn, nbytes: int, reps: int, warmup: int, flush) -> dict:
+    """One kernel (or fixed group of kernels) timed alone: per-launch times
+    with L2 flushed before each, and the back-to-back average; GB/s from the
+    algorithmic bytes over the mean flushed launch time."""
+    t = stats_ms(launch_times(fn, reps, warmup, flush))
+    b2b = loop_ms(fn, reps, warmup)
+    return {"ms": {k: (round(v, 5) if k != "n" else v) for k, v in t.items()},
+            "ms_back_to_back": round(b2b, 5), "algorithmic_bytes": int(nbytes),
+            "gbs": round(nbytes / (t["mean"] / 1e3) / 1e9, 1),
+            "gbs_median": round(nbytes / (t["median"] / 1e3) / 1e9, 1),
+            "gbs_back_to_back": round(nbytes / (b2b / 1e3) / 1e9, 1)}
+
+
 class Step:
+    """One decode step over a seeded batch: pa_reshape_and_cache, then
+    pa_decode, or pa_decode_split + pa_reduce for the split workload."""
+
     def __init__(self, batch: workloads.DecodeBatch):
         from paged_kv_cache_444_b200 import SplitWorkspace
         self.b = batch
@@ -179,70 +256,78 @@ class Step:
                                batch.context_lens, cfg.scale, out=self.out,
                                partition_size=self.ps, workspace=self.ws)
 
-    def run(self, ev=None):
-        """One step; ev = list of launches+1 CUDA events to record between kernels."""
+    def run(self):
+        self.plan.run()   # validated once; the timed path
+
+    def kernels(self, ctx) -> list:
+        """(name, launch, algorithmic bytes) of each kernel of the step, and of
+        the attention as a whole when it takes two kernels."""
         from paged_kv_cache_444_b200 import (pa_decode, pa_decode_split, pa_reduce,
                                              pa_reshape_and_cache)
-        b, cfg = self.b, self.cfg
-        if not ev:
-            self.plan.run()   # validated once; the timed path
-            return
-        if ev:
-            ev[0].record()
-        pa_reshape_and_cache(b.key, b.value, b.key_cache, b.value_cache, b.slot_mapping)
-        if ev:
-            ev[1].record()
+        b, cfg, w = self.b, self.cfg, self.ws
+        by = workloads.algorithmic_bytes(cfg, ctx)
+        write = lambda: pa_reshape_and_cache(b.key, b.value, b.key_cache, b.value_cache,
+                                             b.slot_mapping)
+        ks = [("pa_reshape_and_cache", write, by["write"])]
         if self.ps:
-            w = self.ws
-            pa_decode_split(w.tmp_out, w.max_logits, w.exp_sums, b.query, b.key_cache,
-                            b.value_cache, b.block_tables, b.context_lens, cfg.scale, self.ps)
-            if ev:
-                ev[2].record()
-            pa_reduce(self.out, w.tmp_out, w.max_logits, w.exp_sums, b.context_lens, self.ps)
-            if ev:
-                ev[3].record()
+            split = lambda: pa_decode_split(w.tmp_out, w.max_logits, w.exp_sums, b.query,
+                                            b.key_cache, b.value_cache, b.block_tables,
+                                            b.context_lens, cfg.scale, self.ps)
+            reduce = lambda: pa_reduce(self.out, w.tmp_out, w.max_logits, w.exp_sums,
+                                       b.context_lens, self.ps)
+
+            def both():
+                split()
+                reduce()
+            parts = sum(-(-int(c) // self.ps) for c in ctx) * cfg.num_heads
+            reduce_bytes = parts * (cfg.head_dim + 2) * 4 + by["out"] + by["context_lens"]
+            ks += [("pa_decode_split", split, attention_kernel_bytes(cfg, ctx, True)),
+                   ("pa_reduce", reduce, reduce_bytes),
+                   ("pa_decode_split+pa_reduce", both, by["attention"])]
         else:
-            pa_decode(self.out, b.query, b.key_cache, b.value_cache, b.block_tables,
-                      b.context_lens, cfg.scale)
-            if ev:
-                ev[2].record()
+            ks.append(("pa_decode", lambda: pa_decode(self.out, b.query, b.key_cache,
+                                                      b.value_cache, b.block_tables,
+                                                      b.context_lens, cfg.scale),
+                       by["attention"]))
+        return ks
 
 
-def time_steps(step: Step, steps: int, warmup: int, world: int, device, clocks=None,
-               kernel_steps: int = 200):
-    """Warm up, then time `steps` steps back to back (CUDA events at the two
-    ends only, so consecutive launches may overlap as they would in use), then
-    time `kernel_steps` more with an event between every two kernels for the
-    per-kernel durations.  Returns (ms per step, [ms per kernel])."""
+def time_regions(run, steps: int, warmup: int, world: int, device, min_total_s: float,
+                 max_regions: int = 400) -> list[float]:
+    """Warm up, then time regions of exactly `steps` back-to-back runs, each
+    bracketed by a barrier and a device synchronise on both sides and timed
+    with CUDA events at its two ends; as many regions as make up min_total_s
+    (at least one).  Returns each region's ms per step, max over ranks."""
     for _ in range(warmup):
-        step.run()
+        run()
     torch.cuda.synchronize()
-    barrier(world, device)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ctx = clocks if clocks is not None else _Null()
-    with ctx:
+
+    def region() -> float:
+        barrier(world, device)
         torch.cuda.synchronize()
-        start.record()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
         for _ in range(steps):
-            step.run()
-        end.record()
+            run()
+        b.record()
         torch.cuda.synchronize()
-    barrier(world, device)
-    ms = start.elapsed_time(end) / steps
-    ks = max(1, min(steps, kernel_steps))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(step.launches + 1)]
-           for _ in range(ks)]
-    for k in range(ks):
-        step.run(evs[k])
-    torch.cuda.synchronize()
-    per_kernel = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / ks
-                  for i in range(step.launches)]
-    return ms, per_kernel
+        barrier(world, device)
+        return a.elapsed_time(b) / steps
+
+    first = max_over_ranks(region(), world, device)
+    n = max(1, min(max_regions, math.ceil(min_total_s * 1e3 / max(1e-6, first * steps))))
+    times = [region() for _ in range(n - 1)]
+    if world > 1 and times:
+        import torch.distributed as dist
+        t = torch.tensor(times, dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        times = t.tolist()
+    return [first] + times
 
 
-def shared_prefix_kernel_ms(batch, warmup: int, reps: int = 100) -> float:
-    """CUDA-event time of pa_decode_shared_prefix on a batch with prefix groups
-    (the same attention as pa_decode, reading each shared page once per group)."""
+def shared_prefix_stats(batch, warmup: int, flush, reps: int = 100) -> dict:
+    """pa_decode_shared_prefix timed alone on a batch with prefix groups (the
+    same attention as pa_decode, reading each shared page once per group)."""
     from paged_kv_cache_444_b200 import pa_decode_shared_prefix
     cfg = batch.cfg
     out = torch.empty_like(batch.query)
@@ -252,48 +337,53 @@ def shared_prefix_kernel_ms(batch, warmup: int, reps: int = 100) -> float:
         pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
                                 batch.block_tables, batch.context_lens, batch.group_starts,
                                 batch.prefix_blocks, cfg.scale, max(sizes))
-    for _ in range(warmup):
-        run()
-    torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(reps):
-        run()
-    end.record()
-    torch.cuda.synchronize()
-    return start.elapsed_time(end) / reps
+    unique = workloads.unique_kv_bytes(cfg, batch.block_tables.cpu().tolist(),
+                                       batch.context_lens.cpu().tolist())
+    by = workloads.algorithmic_bytes(cfg, batch.context_lens.cpu().tolist())
+    nbytes = unique + by["block_table"] + by["query"] + by["out"] + by["context_lens"]
+    return kernel_stats(run, nbytes, reps, warmup, flush)
 
 
-def fp8_decode_ms(batch, warmup: int, reps: int = 100) -> float | None:
-    """CUDA-event time of pa_decode_fp8 on the same batch with its caches held
-    as E4M3 codes (x * 64 quantised by torch, scale 1/64); None where the
-    fp8 path is not built (head_dim != 128) or the batch uses the split path."""
-    from paged_kv_cache_444_b200 import pa_decode_fp8
+def fp8_stats(batch, warmup: int, flush, reps: int = 100) -> dict | None:
+    """pa_decode_fp8 (pa_decode_split_fp8 + pa_reduce for the split workload)
+    timed alone on the same batch with its caches held as E4M3 codes (x * 64
+    quantised by torch, scale 1/64); None where the fp8 path is not built
+    (head_dim != 128).  Algorithmic bytes count K/V at one byte per element."""
+    from paged_kv_cache_444_b200 import (SplitWorkspace, pa_decode_fp8, pa_decode_split_fp8,
+                                         pa_reduce)
     cfg = batch.cfg
-    if cfg.head_dim != 128 or cfg.partition_size:
+    if cfg.head_dim != 128:
         return None
     q8 = lambda t: (t.float() * 64.0).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
     kc, vc = q8(batch.key_cache), q8(batch.value_cache)
     out = torch.empty_like(batch.query)
+    ctx = batch.context_lens.cpu().tolist()
+    by = workloads.algorithmic_bytes(cfg, ctx)
+    nbytes = by["kv"] // 2 + by["block_table"] + by["query"] + by["out"] + by["context_lens"]
+    if cfg.partition_size:
+        ps = cfg.partition_size
+        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, batch.max_partitions,
+                            batch.query.device)
 
-    def run():
-        pa_decode_fp8(out, batch.query, kc, vc, batch.block_tables, batch.context_lens,
-                      cfg.scale, 1.0 / 64, 1.0 / 64)
-    for _ in range(warmup):
-        run()
-    torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(reps):
-        run()
-    end.record()
-    torch.cuda.synchronize()
+        def run():
+            pa_decode_split_fp8(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query, kc, vc,
+                                batch.block_tables, batch.context_lens, cfg.scale, 1.0 / 64,
+                                1.0 / 64, ps)
+            pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, batch.context_lens, ps)
+        kernel = "pa_decode_split_fp8+pa_reduce"
+    else:
+        def run():
+            pa_decode_fp8(out, batch.query, kc, vc, batch.block_tables, batch.context_lens,
+                          cfg.scale, 1.0 / 64, 1.0 / 64)
+        kernel = "pa_decode_fp8"
+    r = kernel_stats(run, nbytes, reps, warmup, flush)
+    r["kernel"] = kernel
     del kc, vc
-    return start.elapsed_time(end) / reps
+    return r
 
 
-def prefill_measure(device, warmup: int, reps: int = 20, peak_tflops: float = 0.0,
-                    peak_kind: str = "") -> dict:
+def prefill_measure(device, warmup: int, reps: int = 100, peak_tflops: float = 0.0,
+                    peak_kind: str = "", flush=None) -> dict:
     """Chunked prefill on a Llama-3-8B-shaped GQA layer: 8 sequences each
     bringing a 512-token chunk at the end of a context drawn U[512, 4096]
     (32/8 heads, d=128, bf16, 16-token blocks).  Compute-bound: reported in
@@ -308,27 +398,24 @@ def prefill_measure(device, warmup: int, reps: int = 20, peak_tflops: float = 0.
     def run():
         pa_prefill(out, query, b.key_cache, b.value_cache, b.block_tables, b.context_lens,
                    starts, cfg.scale, chunk)
-    for _ in range(warmup):
-        run()
-    torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(reps):
-        run()
-    end.record()
-    torch.cuda.synchronize()
-    ms = start.elapsed_time(end) / reps
+    t = stats_ms(launch_times(run, reps, warmup, flush))
+    b2b = loop_ms(run, reps, warmup)
+    ms = t["mean"]
     ctx = b.context_lens.cpu().tolist()
     pairs = sum(sum(c - chunk + i + 1 for i in range(chunk)) for c in ctx)
     flops = 4 * cfg.head_dim * cfg.num_heads * pairs
     tf = flops / (ms / 1e3) / 1e12
     return {"workload": "chunked_prefill_gqa: 8 seqs x 512-token chunks at ctx U[512,4096], "
                         "32/8 heads, d=128, bf16", "kernel": "pa_prefill",
-            "ms": round(ms, 5), "tflops": round(tf, 1),
+            "ms": round(ms, 5), "ms_stats": {k: (round(v, 5) if k != "n" else v)
+                                             for k, v in t.items()},
+            "ms_back_to_back": round(b2b, 5), "tflops": round(tf, 1),
+            "tflops_back_to_back": round(flops / (b2b / 1e3) / 1e12, 1),
             "query_tokens_per_s": round(T / (ms / 1e3), 1),
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak_tflops,
                          "unit": "TFLOP/s", "frac": round(tf / peak_tflops, 4) if peak_tflops else None,
-                         "peak_kind": peak_kind, "algorithmic_flops": flops}}
+                         "peak_kind": peak_kind, "algorithmic_flops": flops,
+                         "timing": "mean of per-launch CUDA-event times, L2 flushed before each"}}
 
 
 def graph_steps(step: Step, steps: int, warmup: int) -> float | None:
@@ -400,28 +487,19 @@ def bind_to_gpu_local_cpus(device_index: int) -> str:
         return f"unbound ({type(e).__name__})"
 
 
-def e2e_steps(step: Step, steps: int, warmup: int, world: int, device):
+def e2e_regions(step: Step, steps: int, warmup: int, world: int, device, min_total_s: float):
     """The same step through the C ABI from host buffers (pa_decode_step_host):
     every step copies its inputs in from pinned host memory, writes the cache,
-    attends, and copies the output back, all inside the timing."""
+    attends, and copies the output back, all inside the timing.  Regions of
+    exactly `steps` steps as for the device-resident step."""
     from paged_kv_cache_444_b200 import HostStep
     b, cfg = step.b, step.cfg
     hs = HostStep(b.key_cache, b.value_cache, cfg.num_seqs, cfg.num_heads,
                   b.block_tables.shape[1], cfg.scale, step.ps, cfg.torch_dtype)
     for n in ("query", "key", "value", "slot_mapping", "block_tables", "context_lens"):
         getattr(hs, n).copy_(getattr(b, n).cpu())
-    for _ in range(warmup):
-        hs.run()
-    torch.cuda.synchronize()
-    barrier(world, device)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(steps):
-        hs.run()
-    end.record()
-    torch.cuda.synchronize()
-    barrier(world, device)
-    return start.elapsed_time(end) / steps, hs.h2d_bytes, hs.d2h_bytes
+    regions = time_regions(hs.run, steps, warmup, world, device, min_total_s)
+    return regions, hs.h2d_bytes, hs.d2h_bytes
 
 
 # ---------------------------------------------------------------------------
@@ -540,10 +618,24 @@ def cpu_baseline(cfg, context_lens, block_tables, batch, budget_s: float = 12.0)
     sub_cfg = cfg.scaled(num_seqs=len(seqs))
     by = workloads.algorithmic_bytes(sub_cfg, sub_ctx)["step"]
     return {"value": round(by / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "seconds": round(secs, 3),
+            "seconds": round(secs, 3), "host": host_description(),
             "sample": f"{len(seqs)} of {cfg.num_seqs} sequences of {cfg.name} "
                       f"({sum(sub_ctx)} context tokens, all {cfg.num_heads} heads): oracle "
                       f"cache write + fp64 decode, single thread"}
+
+
+def host_description() -> dict:
+    """The host the CPU baseline ran on: its CPU model (/proc/cpuinfo), the
+    logical CPUs the OS reports, and how many the oracle used (one)."""
+    model = None
+    try:
+        for line in Path("/proc/cpuinfo").read_text().splitlines():
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"cpu_model": model, "os_cpu_count": os.cpu_count(), "cores_used": 1}
 
 
 # ---------------------------------------------------------------------------
@@ -557,8 +649,9 @@ def run_native(args, world, rank, local):
     from paged_kv_cache_444_b200 import load
     load()
     peak, peak_kind = measured_peak()
+    flush = L2Flush(device)
 
-    def bench_config(name, steps, warmup, clocks=None):
+    def bench_config(name, steps, min_total_s, clocks=None):
         cfg = workloads.CONFIGS[name]
         cfg = cfg.scaled(seed=cfg.seed + 1000 * rank)
         if name == args.config and (args.num_seqs or args.num_blocks):
@@ -568,66 +661,71 @@ def run_native(args, world, rank, local):
                              name=f"{cfg.name}[seqs={args.num_seqs or cfg.num_seqs}]")
         batch = workloads.make_batch(cfg, device)
         step = Step(batch)
-        ms, per_kernel = time_steps(step, steps, warmup, world, device, clocks)
-        ms_max = max_over_ranks(ms, world, device)
-        gms = graph_steps(step, steps, warmup) if args.graph else None
-        shared_ms = shared_prefix_kernel_ms(batch, warmup) if batch.group_starts is not None \
-            else None
-        f8_ms = fp8_decode_ms(batch, warmup) if args.fp8 else None
         ctx = batch.context_lens.cpu().tolist()
         by = workloads.algorithmic_bytes(cfg, ctx)
-        attn_ms = per_kernel[1] + (per_kernel[2] if step.ps else 0.0)
-        kern_ms = per_kernel[1]
-        kern_bytes = attention_kernel_bytes(cfg, ctx, bool(step.ps))
+        with (clocks if clocks is not None else _Null()):
+            regions = time_regions(step.run, steps, args.warmup, world, device, min_total_s)
+        st = stats_ms(regions)
         total_bytes = sum_over_ranks(by["step"], world, device)
+        kernels = {}
+        for kname, fn, nbytes in step.kernels(ctx):
+            k = kernel_stats(fn, nbytes, args.kernel_reps, args.warmup, flush)
+            k["frac_of_peak"] = round(k["gbs"] / peak, 4)
+            kernels[kname] = k
+        attn = "pa_decode_split+pa_reduce" if step.ps else "pa_decode"
         res = {
-            "ms_per_step": ms_max,
-            "value": total_bytes / (ms_max / 1e3) / 1e9,
-            "per_kernel_ms": per_kernel,
-            "attention_ms": attn_ms,
-            "attention_gbs": (by["attention"]) / (attn_ms / 1e3) / 1e9,
-            "kernel_gbs": kern_bytes / (kern_ms / 1e3) / 1e9,
-            "kernel_bytes": kern_bytes,
-            "bytes": by,
-            "tokens_per_s": sum_over_ranks(cfg.num_seqs, world, device) / (ms_max / 1e3),
-            "graph_ms_per_step": gms,
-            "shared_prefix_kernel_ms": shared_ms,
-            "unique_kv_bytes": (workloads.unique_kv_bytes(cfg, batch.block_tables.cpu().tolist(),
-                                                          batch.context_lens.cpu().tolist())
-                                if shared_ms else None),
-            "fp8_ms": f8_ms,
-            "kernel": "pa_decode_split" if step.ps else "pa_decode",
-            "context_tokens": int(sum(ctx)),
+            "regions": regions, "stats": st, "ms_per_step": st["median"],
+            "value": total_bytes / (st["median"] / 1e3) / 1e9,
+            "bytes": by, "kernels": kernels, "attention_kernel": attn,
+            "dominant": "pa_decode_split" if step.ps else "pa_decode",
+            "tokens_per_s": sum_over_ranks(cfg.num_seqs, world, device) / (st["median"] / 1e3),
+            "graph_ms_per_step": graph_steps(step, steps, args.warmup) if args.graph else None,
+            "shared_prefix": (shared_prefix_stats(batch, args.warmup, flush, args.kernel_reps)
+                              if batch.group_starts is not None else None),
+            "fp8": fp8_stats(batch, args.warmup, flush, args.kernel_reps) if args.fp8 else None,
+            "context_tokens": int(sum(ctx)), "name": name,
         }
+        if res["shared_prefix"]:
+            res["shared_prefix"]["frac_of_peak"] = round(res["shared_prefix"]["gbs"] / peak, 4)
+            res["shared_prefix"]["speedup_vs_pa_decode"] = round(
+                kernels["pa_decode"]["ms"]["mean"] / res["shared_prefix"]["ms"]["mean"], 3)
+        if res["fp8"]:
+            res["fp8"]["frac_of_peak"] = round(res["fp8"]["gbs"] / peak, 4)
+            res["fp8"]["speedup_vs_16bit"] = round(
+                kernels[attn]["ms"]["mean"] / res["fp8"]["ms"]["mean"], 3)
         return cfg, batch, step, res
 
     results = {}
     clocks = ClockSampler(local)
-    cfg, batch, step, main = bench_config(args.config, args.steps, args.warmup, clocks)
-    e2e_ms, h2d, d2h = e2e_steps(step, max(3, args.steps // 4), args.warmup, world, device)
-    e2e_ms = max_over_ranks(e2e_ms, world, device)
+    cfg, batch, step, main = bench_config(args.config, args.steps, args.min_timed_s, clocks)
+    e2e_reg, h2d, d2h = e2e_regions(step, args.steps, args.warmup, world, device,
+                                    args.min_timed_s)
+    e2e_st = stats_ms(e2e_reg)
     total_bytes = sum_over_ranks(main["bytes"]["step"], world, device)
     ctx_main = batch.context_lens.cpu().tolist()
     bt_main = batch.block_tables.cpu().tolist()
 
+    results[args.config] = main
     if not args.only_main:
         for name in workloads.CONFIG_ORDER:
             if name == args.config:
-                results[name] = main
                 continue
-            _, b2, s2, r = bench_config(name, args.config_steps, args.warmup)
+            _, b2, s2, r = bench_config(name, args.config_steps, args.config_min_timed_s)
             results[name] = r
             del b2, s2
             torch.cuda.empty_cache()
 
-    kname = "pa_decode_split" if step.ps else "pa_decode"
+    kname = main["dominant"]
+    kmain = main["kernels"][kname]
     roof = {"bound": "hbm", "kernel": kname,
-            "achieved": round(main["kernel_gbs"], 1), "peak": peak, "unit": "GB/s",
-            "frac": round(main["kernel_gbs"] / peak, 4), "peak_kind": peak_kind,
-            "algorithmic_bytes_per_launch": main["kernel_bytes"],
-            "traffic": None}
-    roof["traffic"] = recorded_traffic(args.config, kname, sum(ctx_main))
-
+            "achieved": kmain["gbs"], "peak": peak, "unit": "GB/s",
+            "frac": round(kmain["gbs"] / peak, 4), "peak_kind": peak_kind,
+            "algorithmic_bytes_per_launch": kmain["algorithmic_bytes"],
+            "timing": f"mean of {kmain['ms']['n']} per-launch CUDA-event times of the kernel "
+                      f"alone, L2 flushed before each launch",
+            "launch_ms": kmain["ms"],
+            "traffic": recorded_traffic(args.config, kname, sum(ctx_main))}
+    st = main["stats"]
     line = {
         "metric": METRIC,
         "value": round(main["value"], 2),
@@ -647,52 +745,38 @@ def run_native(args, world, rank, local):
                    "block_size": cfg.block_size, "num_blocks": cfg.num_blocks,
                    "partition_size": cfg.partition_size or None,
                    "context_tokens": int(sum(ctx_main)),
-                   "l2": "inputs larger than L2 (K/V read per step >> 126 MB), no flush",
+                   "l2": "inputs larger than L2 (K/V read per step >> 126 MB), no flush between "
+                         "steps; kernels timed alone are L2-flushed before each launch",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "timing": {"regions": len(main["regions"]), "steps_per_region": args.steps,
+                   "ms_per_step_median": round(st["median"], 5),
+                   "ms_per_step_p10": round(st["p10"], 5), "ms_per_step_p90": round(st["p90"], 5),
+                   "ms_per_step_mean": round(st["mean"], 5),
+                   "first_region_ms_per_step": round(main["regions"][0], 5),
+                   "timed_s": round(sum(main["regions"]) * args.steps / 1e3, 3),
+                   "value_is": "step bytes / median over regions of the region's ms per step"},
         "decode_tokens_per_s": round(main["tokens_per_s"], 1),
         "graph_ms_per_step": (round(main["graph_ms_per_step"], 5)
                               if main["graph_ms_per_step"] else None),
-        "attention_gbs": round(main["attention_gbs"], 1),
-        "per_kernel_ms": {n: round(v, 5) for n, v in zip(
-            ["pa_reshape_and_cache", kname] + (["pa_reduce"] if step.ps else []),
-            main["per_kernel_ms"])},
+        "kernels": main["kernels"],
         "roofline": roof,
-        "gpu_launches": step.launches * args.steps,
-        "e2e": {"value": round(total_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
-                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h,
+        "gpu_launches": step.launches * args.steps * len(main["regions"]),
+        "e2e": {"value": round(total_bytes / (e2e_st["median"] / 1e3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_st["median"], 5),
+                "ms_per_step_p10": round(e2e_st["p10"], 5),
+                "ms_per_step_p90": round(e2e_st["p90"], 5),
+                "steps": args.steps * len(e2e_reg), "regions": len(e2e_reg),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "frac_of_resident_step": round(main["ms_per_step"] / e2e_st["median"], 4),
                 "api": "pa_decode_step_host (C ABI, pinned host buffers in and out)",
                 "host_cpus": host_cpus},
         "clocks": clocks.summary(),
     }
-    if results:
-        line["per_config"] = {
-            n: {"ms_per_step": round(r["ms_per_step"], 5), "step_gbs": round(r["value"], 1),
-                "attention_gbs": round(r["attention_gbs"], 1),
-                "kernel_gbs": round(r["kernel_gbs"], 1),
-                "kernel_frac_of_peak": round(r["kernel_gbs"] / peak, 4),
-                "kernel_traffic": recorded_traffic(n, r["kernel"], r["context_tokens"]),
-                "kernel_algorithmic_bytes": r["kernel_bytes"],
-                "attention_frac_of_peak": round(r["attention_gbs"] / peak, 4),
-                "decode_tokens_per_s": round(r["tokens_per_s"], 1),
-                "graph_ms_per_step": (round(r["graph_ms_per_step"], 5)
-                                      if r["graph_ms_per_step"] else None),
-                "per_kernel_ms": [round(x, 5) for x in r["per_kernel_ms"]],
-                **({"pa_decode_shared_prefix_ms": round(r["shared_prefix_kernel_ms"], 5),
-                    # the shared-prefix kernel reads each shared page once:
-                    # its rate on the unique K/V bytes, against the copy peak
-                    "pa_decode_shared_prefix_unique_gbs": round(
-                        r["unique_kv_bytes"] / (r["shared_prefix_kernel_ms"] / 1e3) / 1e9, 1),
-                    "pa_decode_shared_prefix_unique_frac_of_peak": round(
-                        r["unique_kv_bytes"] / (r["shared_prefix_kernel_ms"] / 1e3) / 1e9 / peak,
-                        4)}
-                   if r["shared_prefix_kernel_ms"] else {}),
-                **(fp8_entry(r, peak) if r["fp8_ms"] else {})}
-            for n, r in results.items()}
+    line["per_config"] = {n: config_entry(r, peak) for n, r in results.items()}
     if args.prefill and not args.only_main:
         tp, tk = measured_tensor_peak()
         line["prefill"] = prefill_measure(device, args.warmup, reps=args.prefill_reps,
-                                          peak_tflops=tp, peak_kind=tk)
+                                          peak_tflops=tp, peak_kind=tk, flush=flush)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, ctx_main, bt_main, batch,
                                             budget_s=args.cpu_budget)
@@ -703,16 +787,31 @@ def run_native(args, world, rank, local):
         dist.destroy_process_group()
 
 
-def fp8_entry(r: dict, peak: float) -> dict:
-    """pa_decode_fp8 on the same batch: time, algorithmic GB/s (K/V at one
-    byte per element) and the speed-up over the 16-bit decode kernel."""
-    by = r["bytes"]
-    fp8_bytes = by["kv"] // 2 + by["block_table"] + by["query"] + by["out"] + by["context_lens"]
-    gbs = fp8_bytes / (r["fp8_ms"] / 1e3) / 1e9
-    return {"pa_decode_fp8": {"ms": round(r["fp8_ms"], 5), "gbs": round(gbs, 1),
-                              "frac_of_peak": round(gbs / peak, 4),
-                              "speedup_vs_16bit_kernel": round(r["per_kernel_ms"][1] /
-                                                               r["fp8_ms"], 3)}}
+def config_entry(r: dict, peak: float) -> dict:
+    """The per-workload summary of the JSON line."""
+    attn = r["kernels"][r["attention_kernel"]]
+    e = {"ms_per_step": round(r["ms_per_step"], 5), "step_gbs": round(r["value"], 1),
+         "ms_per_step_p10": round(r["stats"]["p10"], 5),
+         "ms_per_step_p90": round(r["stats"]["p90"], 5),
+         "attention_kernel": r["attention_kernel"], "attention_gbs": attn["gbs"],
+         "attention_frac_of_peak": round(attn["gbs"] / peak, 4),
+         "kernel": r["dominant"], "kernel_gbs": r["kernels"][r["dominant"]]["gbs"],
+         "kernel_frac_of_peak": r["kernels"][r["dominant"]]["frac_of_peak"],
+         "kernel_traffic": recorded_traffic(r.get("name", ""), r["dominant"],
+                                            r["context_tokens"]),
+         "decode_tokens_per_s": round(r["tokens_per_s"], 1),
+         "graph_ms_per_step": (round(r["graph_ms_per_step"], 5)
+                               if r["graph_ms_per_step"] else None),
+         "kernels": {k: {"ms_mean": v["ms"]["mean"], "ms_median": v["ms"]["median"],
+                         "ms_p10": v["ms"]["p10"], "ms_p90": v["ms"]["p90"],
+                         "ms_back_to_back": v["ms_back_to_back"], "gbs": v["gbs"],
+                         "frac_of_peak": v["frac_of_peak"]}
+                     for k, v in r["kernels"].items()}}
+    if r["shared_prefix"]:
+        e["pa_decode_shared_prefix"] = r["shared_prefix"]
+    if r["fp8"]:
+        e["fp8"] = r["fp8"]
+    return e
 
 
 def recorded_traffic(config: str, kernel: str, context_tokens: int):
@@ -808,12 +907,18 @@ def run_reference(args, world, rank, local):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=20,
+                    help="steps per timed region (each region is exactly this many steps)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--config", default=MAIN_CONFIG, choices=list(workloads.CONFIGS))
-    ap.add_argument("--config-steps", type=int, default=300,
-                    help="timed steps for each of the other workloads")
+    ap.add_argument("--min-timed-s", type=float, default=1.0,
+                    help="regions of --steps steps are repeated until this much is timed")
+    ap.add_argument("--config-steps", type=int, default=20,
+                    help="steps per timed region for each of the other workloads")
+    ap.add_argument("--config-min-timed-s", type=float, default=0.25)
+    ap.add_argument("--kernel-reps", type=int, default=100,
+                    help="launches of each kernel timed alone (L2 flushed before each)")
     ap.add_argument("--only-main", action="store_true", help="skip the per-workload table")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0,
@@ -821,12 +926,12 @@ def main(argv=None):
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="also time the step replayed from a CUDA graph")
     ap.add_argument("--fp8", action=argparse.BooleanOptionalAction, default=True,
-                    help="also time pa_decode_fp8 on each batch (E4M3 copy of its caches)")
+                    help="also time the fp8 decode on each batch (E4M3 copy of its caches)")
     ap.add_argument("--prefill", action=argparse.BooleanOptionalAction, default=True,
                     help="also time pa_prefill on a chunked-prefill GQA layer")
     ap.add_argument("--only-prefill", action="store_true",
                     help="time only pa_prefill (its own JSON object; for profiling captures)")
-    ap.add_argument("--prefill-reps", type=int, default=20)
+    ap.add_argument("--prefill-reps", type=int, default=100)
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="override the workload's batch size (small profiling captures)")
     ap.add_argument("--num-blocks", type=int, default=0,
@@ -845,7 +950,7 @@ def main(argv=None):
         torch.cuda.set_device(device)
         tp, tk = measured_tensor_peak()
         print(json.dumps(prefill_measure(device, args.warmup, reps=args.prefill_reps,
-                                         peak_tflops=tp, peak_kind=tk)))
+                                         peak_tflops=tp, peak_kind=tk, flush=L2Flush(device))))
     else:
         run_native(args, world, rank, local)
 

@@ -614,15 +614,28 @@ const StepFork* step_fork(cudaStream_t s) {
   return &forks.emplace(std::make_pair(dev, s), f).first->second;
 }
 
-// The device address of page-locked host memory the GPU can write directly,
-// or nullptr (pageable memory).
-void* device_view_of_host(void* p) {
-  cudaPointerAttributes attr{};
-  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
-    cudaGetLastError();
-    return nullptr;
-  }
-  return attr.type == cudaMemoryTypeHost ? attr.devicePointer : nullptr;
+// The device address of `bytes` bytes of page-locked host memory at p that
+// the GPU can read and write directly, or nullptr.  Both the first and the
+// last byte must lie in page-locked memory, and the last byte's device
+// address must follow from the first's: a range that runs past the end of
+// its page-locked allocation (into pageable memory or another allocation) is
+// not addressable as one piece and takes the copy path instead.
+void* device_view_of_host(const void* p, int64_t bytes) {
+  if (bytes <= 0) return nullptr;
+  auto view = [](const void* q) -> void* {
+    cudaPointerAttributes attr{};
+    if (cudaPointerGetAttributes(&attr, q) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    return attr.type == cudaMemoryTypeHost ? attr.devicePointer : nullptr;
+  };
+  void* first = view(p);
+  if (!first) return nullptr;
+  const void* last_host = static_cast<const uint8_t*>(p) + (bytes - 1);
+  void* last = view(last_host);
+  if (last != static_cast<void*>(static_cast<uint8_t*>(first) + (bytes - 1))) return nullptr;
+  return first;
 }
 }  // namespace
 
@@ -701,15 +714,21 @@ pa_status pa_decode_step_host(void* out_host, const void* query_host, const void
   // share the link with the side stream's copy of the query and tables, and
   // nothing waits for a separate copy of the rows.  Otherwise the rows are
   // copied into the workspace first, and the side stream forks after that copy.
-  const void* src_key = device_view_of_host(const_cast<void*>(key_host));
+  const void* src_key = nullptr;
   const void* src_value = nullptr;
   const void* src_slots = nullptr;
-  if (src_key && value_host) {
-    src_value = device_view_of_host(const_cast<void*>(value_host));
-    src_slots = device_view_of_host(const_cast<int64_t*>(slot_mapping_host));
-  } else if (src_key) {  // packed after key_host, at the workspace's offsets
-    src_value = static_cast<const uint8_t*>(src_key) + (l.off[1] - l.off[0]);
-    src_slots = static_cast<const uint8_t*>(src_key) + (l.off[2] - l.off[0]);
+  if (value_host) {
+    src_key = device_view_of_host(key_host, kv_bytes);
+    if (src_key) {
+      src_value = device_view_of_host(value_host, kv_bytes);
+      src_slots = device_view_of_host(slot_mapping_host, num_seqs * 8);
+    }
+  } else {  // packed after key_host, at the workspace's offsets: the whole stage
+    src_key = device_view_of_host(key_host, l.off[2] - l.off[0] + num_seqs * 8);
+    if (src_key) {
+      src_value = static_cast<const uint8_t*>(src_key) + (l.off[1] - l.off[0]);
+      src_slots = static_cast<const uint8_t*>(src_key) + (l.off[2] - l.off[0]);
+    }
   }
   const bool read_direct = src_key && src_value && src_slots && aligned16(src_key) &&
                            aligned16(src_value) &&
@@ -731,7 +750,7 @@ pa_status pa_decode_step_host(void* out_host, const void* query_host, const void
   // join, then attend; the output goes straight into out_host when that is
   // page-locked memory the device can address, else through the workspace
   if (cudaStreamWaitEvent(s, fork->join, 0) != cudaSuccess) return PA_ERR_CUDA;
-  void* direct = device_view_of_host(out_host);
+  void* direct = device_view_of_host(out_host, q_bytes);
   if (direct && !aligned16(direct)) direct = nullptr;
   void* d_out = direct ? direct : static_cast<void*>(w + l.off[6]);
   if (partition_size > 0) {

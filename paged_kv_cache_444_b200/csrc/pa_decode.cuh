@@ -359,6 +359,23 @@ __device__ __forceinline__ void merge_and_emit(uint8_t* smem, int nrows, bool sp
 }
 
 // ---------------------------------------------------------------------------
+// After a warp's page loop: true when none of its TMA loads is still in
+// flight.  A loop that ended normally (ok) consumed every page it issued.  One
+// that gave up at page k_stop has issued pages k_stop .. min(k_stop + NST,
+// n_pages) - 1 (at most one per stage) and not consumed them; each is waited
+// for with the bounded wait.  Whole warp.
+// ---------------------------------------------------------------------------
+template <int NST>
+__device__ __forceinline__ bool drain_stages(bool ok, int k_stop, int n_pages, uint32_t bar0) {
+  if (ok) return true;
+  bool landed = true;
+  const int k_end = min(k_stop + NST, n_pages);
+  for (int k = k_stop; k < k_end; ++k)
+    landed &= __all_sync(~0u, mbar_wait_bounded(bar0 + (k % NST) * 8, (k / NST) & 1));
+  return landed;
+}
+
+// ---------------------------------------------------------------------------
 // The kernel: one (sequence, KV head, partition) item per cluster.
 //
 // Launched without a cluster attribute, every CTA is a cluster of one and
@@ -515,6 +532,7 @@ __global__ void __launch_bounds__(kThreads)
 
   // ---- main loop over this warp's pages ----
   bool ok = true;
+  int k_stop = my_pages;  // first page not consumed
   for (int k = 0; k < my_pages; ++k) {
     if (k > 0 && (k & 31) == 0) {
       ++win;
@@ -526,6 +544,7 @@ __global__ void __launch_bounds__(kThreads)
     if (!__all_sync(~0u, mbar_wait_bounded(bar0 + stg * 8, (k / NST) & 1))) {
       if (lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
       ok = false;
+      k_stop = k;
       break;
     }
     const uint32_t kb = stage0 + stg * L::kStageBytes;
@@ -536,8 +555,17 @@ __global__ void __launch_bounds__(kThreads)
     if (k + NST < my_pages) issue(k + NST);
   }
 
-  // ---- merge the four warps (the stage area is reused as the merge buffer) ----
-  __syncthreads();
+  // ---- merge the four warps (the stage area is reused as the merge buffer).
+  // A warp that gave up on a wait still has its loads for pages k_stop ..
+  // k_stop + NST - 1 in flight: wait for them (bounded) first.  If one never
+  // lands, the stage area is left alone and the CTA ends without writing. ----
+  if (!__syncthreads_and(drain_stages<NST>(ok, k_stop, my_pages, bar0))) {
+    if (spread) {  // still meet the cluster's two merge barriers
+      cluster_sync();
+      cluster_sync();
+    }
+    return;
+  }
   float* red_acc = reinterpret_cast<float*>(smem);
   float* red_m = reinterpret_cast<float*>(smem + L::kRedMOffset);
   float* red_l = reinterpret_cast<float*>(smem + L::kRedLOffset);

@@ -273,6 +273,7 @@ __global__ void __launch_bounds__(kThreads)
 
   // ---- main loop ----
   bool ok = true;
+  int k_stop = my_count;  // first page not consumed
   for (int k = 0; k < my_count; ++k) {
     if (k > 0 && (k & 31) == 0) {
       ++win;
@@ -286,6 +287,7 @@ __global__ void __launch_bounds__(kThreads)
     if (!__all_sync(~0u, mbar_wait_bounded(bar0 + stg * 8, (k / NST) & 1))) {
       if (lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
       ok = false;
+      k_stop = k;
       break;
     }
     const int lim0 = (live0 && (member < 0 || member == mem0)) ? ctx0 : 0;
@@ -301,8 +303,15 @@ __global__ void __launch_bounds__(kThreads)
     if (k + NST < my_count) issue(k + NST);
   }
 
-  // ---- merge warps (and the cluster's CTAs) and write the rows ----
-  __syncthreads();
+  // ---- merge warps (and the cluster's CTAs) and write the rows; loads left
+  // in flight by a wait that gave up are drained first (see drain_stages) ----
+  if (!__syncthreads_and(drain_stages<NST>(ok, k_stop, my_count, bar0))) {
+    if (spread) {
+      cluster_sync();
+      cluster_sync();
+    }
+    return;
+  }
   float* red_acc = reinterpret_cast<float*>(smem);
   float* red_m = reinterpret_cast<float*>(smem + L::kRedMOffset);
   float* red_l = reinterpret_cast<float*>(smem + L::kRedLOffset);

@@ -51,3 +51,19 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.fail("GPU test collected but no CUDA device is visible")
     return torch.device("cuda", 0)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Print the full-size parity errors the GPU tests recorded."""
+    try:
+        from parity_helpers import PARITY_REPORT
+    except Exception:
+        return
+    if not PARITY_REPORT:
+        return
+    tr = terminalreporter
+    tr.section("full-size parity: max-abs error vs the fp64 oracle")
+    tr.write_line(f"{'workload':<22}{'kernel':<28}{'vs oracle':>12}{'vs rounded':>12}{'tol':>9}")
+    for r in PARITY_REPORT:
+        tr.write_line(f"{r['workload']:<22}{r['kernel']:<28}{r['max_abs_vs_oracle']:>12.3e}"
+                      f"{r['max_abs_vs_rounded_oracle']:>12.3e}{r['tolerance']:>9.0e}")

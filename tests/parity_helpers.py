@@ -114,3 +114,29 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
 
 def max_err(gpu_out: torch.Tensor, ref: np.ndarray) -> float:
     return float(np.max(np.abs(to_f64(gpu_out) - ref))) if ref.size else 0.0
+
+
+# (workload, kernel, max|gpu - oracle|, max|gpu - round_to_dtype(oracle)|, tolerance)
+# of the full-size checks, printed in pytest's terminal summary and, when
+# PA_PARITY_REPORT names a file, written there as JSON lines.
+PARITY_REPORT: list[dict] = []
+
+
+def report_parity(orc, workload: str, kernel: str, gpu_out: torch.Tensor, ref: np.ndarray,
+                  dtype_code: int, tol: float) -> float:
+    """Record the error of gpu_out against the fp64 oracle and against the
+    oracle rounded to the output dtype (nearest even); returns the first."""
+    import json
+    import os
+    g = to_f64(gpu_out)
+    err = float(np.max(np.abs(g - ref))) if ref.size else 0.0
+    rounded = orc.decode_bits(orc.round_to_dtype(ref, dtype_code), dtype_code)
+    err_r = float(np.max(np.abs(g - rounded))) if ref.size else 0.0
+    row = {"workload": workload, "kernel": kernel, "max_abs_vs_oracle": err,
+           "max_abs_vs_rounded_oracle": err_r, "tolerance": tol, "outputs": int(ref.size)}
+    PARITY_REPORT.append(row)
+    path = os.environ.get("PA_PARITY_REPORT")
+    if path:
+        with open(path, "a", encoding="utf-8") as f:
+            f.write(json.dumps(row) + "\n")
+    return err

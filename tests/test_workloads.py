@@ -65,12 +65,14 @@ def test_shared_prefix_groups_share_exactly_their_prefix():
 
 
 @pytest.mark.parametrize("name", workloads.CONFIG_ORDER)
-def test_written_slot_is_the_newest_position(name):
+def test_written_slot_is_the_newest_position(name, oracle_lib):
+    """The generator's slot of position ctx-1 equals the oracle's slot (whose
+    arithmetic is pinned to the pages' worked example of tokens 1..9)."""
     cfg = C[name]
     ctx, bt, slots = _index_structure(cfg)
     for s in range(cfg.num_seqs):
         pos = int(ctx[s]) - 1
-        assert slots[s] == bt[s, pos // cfg.block_size] * cfg.block_size + pos % cfg.block_size
+        assert slots[s] == oracle_lib.slot(np.ascontiguousarray(bt[s]), pos, cfg.block_size)
 
 
 def test_batches_are_reproducible_bit_for_bit():
