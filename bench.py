@@ -325,30 +325,56 @@ def time_regions(run, steps: int, warmup: int, world: int, device, min_total_s: 
     return [first] + times
 
 
-def shared_prefix_stats(batch, warmup: int, flush, reps: int = 100) -> dict:
-    """pa_decode_shared_prefix timed alone on a batch with prefix groups (the
-    same attention as pa_decode, reading each shared page once per group)."""
-    from paged_kv_cache_444_b200 import pa_decode_shared_prefix
+SHARED_SPLIT_PARTITION = 512  # tokens per partition of pa_decode_shared_prefix_split
+
+
+def shared_prefix_stats(batch, warmup: int, flush, reps: int = 100,
+                        partition_size: int = 0) -> dict:
+    """pa_decode_shared_prefix (or, with a partition size,
+    pa_decode_shared_prefix_split + pa_reduce) timed alone on a batch with
+    prefix groups: the same attention as pa_decode, reading each shared page
+    once per group.  Algorithmic bytes count the unique K/V bytes."""
+    from paged_kv_cache_444_b200 import (SplitWorkspace, pa_decode_shared_prefix,
+                                         pa_decode_shared_prefix_split, pa_reduce)
     cfg = batch.cfg
     out = torch.empty_like(batch.query)
     sizes = (batch.group_starts[1:] - batch.group_starts[:-1]).tolist()
+    if partition_size:
+        P = (batch.block_tables.shape[1] * cfg.block_size + partition_size - 1) // partition_size
+        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, batch.query.device)
 
-    def run():
-        pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
-                                batch.block_tables, batch.context_lens, batch.group_starts,
-                                batch.prefix_blocks, cfg.scale, max(sizes))
+        def run():
+            pa_decode_shared_prefix_split(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query,
+                                          batch.key_cache, batch.value_cache,
+                                          batch.block_tables, batch.context_lens,
+                                          batch.group_starts, batch.prefix_blocks, cfg.scale,
+                                          max(sizes), partition_size)
+            pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, batch.context_lens,
+                      partition_size)
+    else:
+        def run():
+            pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
+                                    batch.block_tables, batch.context_lens, batch.group_starts,
+                                    batch.prefix_blocks, cfg.scale, max(sizes))
     unique = workloads.unique_kv_bytes(cfg, batch.block_tables.cpu().tolist(),
                                        batch.context_lens.cpu().tolist())
     by = workloads.algorithmic_bytes(cfg, batch.context_lens.cpu().tolist())
     nbytes = unique + by["block_table"] + by["query"] + by["out"] + by["context_lens"]
-    return kernel_stats(run, nbytes, reps, warmup, flush)
+    r = kernel_stats(run, nbytes, reps, warmup, flush)
+    r["kernel"] = ("pa_decode_shared_prefix_split+pa_reduce" if partition_size
+                   else "pa_decode_shared_prefix")
+    if partition_size:
+        r["partition_size"] = partition_size
+    return r
 
 
-def fp8_stats(batch, warmup: int, flush, reps: int = 100) -> dict | None:
-    """pa_decode_fp8 (pa_decode_split_fp8 + pa_reduce for the split workload)
-    timed alone on the same batch with its caches held as E4M3 codes (x * 64
-    quantised by torch, scale 1/64); None where the fp8 path is not built
-    (head_dim != 128).  Algorithmic bytes count K/V at one byte per element."""
+def fp8_stats(batch, warmup: int, flush, reps: int = 100,
+              partition_size: int | None = None) -> dict | None:
+    """pa_decode_fp8 (pa_decode_split_fp8 + pa_reduce for the split workload,
+    or when a partition size is given) timed alone on the same batch with its
+    caches held as E4M3 codes (x * 64 quantised by torch, scale 1/64); None
+    where the fp8 path is not built (head_dim != 128).  Algorithmic bytes
+    count K/V at one byte per element."""
     from paged_kv_cache_444_b200 import (SplitWorkspace, pa_decode_fp8, pa_decode_split_fp8,
                                          pa_reduce)
     cfg = batch.cfg
@@ -360,10 +386,10 @@ def fp8_stats(batch, warmup: int, flush, reps: int = 100) -> dict | None:
     ctx = batch.context_lens.cpu().tolist()
     by = workloads.algorithmic_bytes(cfg, ctx)
     nbytes = by["kv"] // 2 + by["block_table"] + by["query"] + by["out"] + by["context_lens"]
-    if cfg.partition_size:
-        ps = cfg.partition_size
-        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, batch.max_partitions,
-                            batch.query.device)
+    ps = cfg.partition_size if partition_size is None else partition_size
+    if ps:
+        P = (batch.block_tables.shape[1] * cfg.block_size + ps - 1) // ps
+        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, batch.query.device)
 
         def run():
             pa_decode_split_fp8(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query, kc, vc,
@@ -378,7 +404,31 @@ def fp8_stats(batch, warmup: int, flush, reps: int = 100) -> dict | None:
         kernel = "pa_decode_fp8"
     r = kernel_stats(run, nbytes, reps, warmup, flush)
     r["kernel"] = kernel
+    if ps:
+        r["partition_size"] = ps
     del kc, vc
+    return r
+
+
+def split_variants(batch, warmup: int, flush, reps: int, fp8: bool) -> dict:
+    """pa_decode_split + pa_reduce (and its fp8 form) with 512-token
+    partitions on a single-pass batch: the same attention cut into
+    equal-sized items."""
+    from paged_kv_cache_444_b200 import SplitWorkspace, pa_decode_split, pa_reduce
+    cfg = batch.cfg
+    ps = 512
+    P = (batch.block_tables.shape[1] * cfg.block_size + ps - 1) // ps
+    ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, batch.query.device)
+    out = torch.empty_like(batch.query)
+
+    def run():
+        pa_decode_split(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query, batch.key_cache,
+                        batch.value_cache, batch.block_tables, batch.context_lens, cfg.scale, ps)
+        pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, batch.context_lens, ps)
+    nbytes = workloads.algorithmic_bytes(cfg, batch.context_lens.cpu().tolist())["attention"]
+    r = {"pa_decode_split+pa_reduce": kernel_stats(run, nbytes, reps, warmup, flush)}
+    if fp8:
+        r["fp8"] = fp8_stats(batch, warmup, flush, reps, partition_size=ps)
     return r
 
 
@@ -682,17 +732,28 @@ def run_native(args, world, rank, local):
             "graph_ms_per_step": graph_steps(step, steps, args.warmup) if args.graph else None,
             "shared_prefix": (shared_prefix_stats(batch, args.warmup, flush, args.kernel_reps)
                               if batch.group_starts is not None else None),
+            "shared_prefix_split": (shared_prefix_stats(batch, args.warmup, flush,
+                                                        args.kernel_reps, SHARED_SPLIT_PARTITION)
+                                    if batch.group_starts is not None else None),
             "fp8": fp8_stats(batch, args.warmup, flush, args.kernel_reps) if args.fp8 else None,
+            # batches of few, unequal items: the split form of each kernel too
+            "split512": (split_variants(batch, args.warmup, flush, args.kernel_reps, args.fp8)
+                         if batch.group_starts is not None else None),
             "context_tokens": int(sum(ctx)), "name": name,
         }
-        if res["shared_prefix"]:
-            res["shared_prefix"]["frac_of_peak"] = round(res["shared_prefix"]["gbs"] / peak, 4)
-            res["shared_prefix"]["speedup_vs_pa_decode"] = round(
-                kernels["pa_decode"]["ms"]["mean"] / res["shared_prefix"]["ms"]["mean"], 3)
+        for key in ("shared_prefix", "shared_prefix_split"):
+            if res[key]:
+                res[key]["frac_of_peak"] = round(res[key]["gbs"] / peak, 4)
+                res[key]["speedup_vs_pa_decode"] = round(
+                    kernels["pa_decode"]["ms"]["mean"] / res[key]["ms"]["mean"], 3)
         if res["fp8"]:
             res["fp8"]["frac_of_peak"] = round(res["fp8"]["gbs"] / peak, 4)
             res["fp8"]["speedup_vs_16bit"] = round(
                 kernels[attn]["ms"]["mean"] / res["fp8"]["ms"]["mean"], 3)
+        if res["split512"]:
+            for v in (res["split512"]["pa_decode_split+pa_reduce"], res["split512"].get("fp8")):
+                if v:
+                    v["frac_of_peak"] = round(v["gbs"] / peak, 4)
         return cfg, batch, step, res
 
     results = {}
@@ -809,8 +870,11 @@ def config_entry(r: dict, peak: float) -> dict:
                      for k, v in r["kernels"].items()}}
     if r["shared_prefix"]:
         e["pa_decode_shared_prefix"] = r["shared_prefix"]
+        e["pa_decode_shared_prefix_split"] = r["shared_prefix_split"]
     if r["fp8"]:
         e["fp8"] = r["fp8"]
+    if r["split512"]:
+        e["split512"] = r["split512"]
     return e
 
 

@@ -17,7 +17,9 @@
  * Conventions shared by every entry point:
  *  - Every buffer argument is a DEVICE pointer owned by the caller.  The
  *    library allocates no memory, never synchronises (except
- *    pa_check_error), and keeps no per-call state.
+ *    pa_check_error), and keeps no per-call state (pa_decode_step_host,
+ *    which takes host buffers, keeps a side stream and two events per
+ *    device and stream; see there).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Work is enqueued asynchronously; the returned status covers argument
  *    validation and launch errors only.
@@ -205,6 +207,36 @@ pa_status pa_decode_shared_prefix(void *out, const void *query, const void *key_
                                   pa_dtype dtype, void *stream);
 
 /*
+ * pa_decode_shared_prefix_split -- the shared-prefix decode cut into the
+ * partitions of pa_decode_split, for batches whose groups differ in size
+ * (the same pages as pa_decode_shared_prefix: "vLLM PagedAttention 原理与源码
+ * 深度解析" §3.3; "读一个真实 serving 系统 · vLLM 架构巡礼" §2).  Writes, for every
+ * sequence s, head h and partition p < ceil(context_lens[s]/partition_size),
+ * the partials pa_decode_split would write (same layouts and meaning), so
+ * pa_reduce merges them into the output.  A partition that reaches into a
+ * group's shared prefix is computed once for a chunk of up to
+ * 16 / (num_heads/num_kv_heads) members, reading each shared page once; a
+ * partition past the prefix is computed for its sequence alone.  Entries of
+ * partitions >= ceil(context_lens[s]/partition_size) are not written.
+ * Arguments as pa_decode_shared_prefix (groups) and pa_decode_split
+ * (partials, partition_size a positive multiple of block_size,
+ * ceil(ctx/partition_size) <= max_partitions).  A sequence outside every
+ * group is skipped and reported (PA_CHECK_GROUP).
+ */
+pa_status pa_decode_shared_prefix_split(float *tmp_out, float *max_logits, float *exp_sums,
+                                        const void *query, const void *key_cache,
+                                        const void *value_cache, const int32_t *block_tables,
+                                        const int32_t *context_lens,
+                                        const int32_t *group_starts,
+                                        const int32_t *prefix_blocks, float scale,
+                                        int64_t num_seqs, int64_t num_groups,
+                                        int64_t max_group_size, int64_t num_heads,
+                                        int64_t num_kv_heads, int64_t head_dim,
+                                        int64_t num_blocks, int64_t block_size,
+                                        int64_t max_blocks_per_seq, int64_t partition_size,
+                                        int64_t max_partitions, pa_dtype dtype, void *stream);
+
+/*
  * FP8 KV cache ("vLLM PagedAttention 原理与源码深度解析" §8.4: --kv-cache-dtype
  * fp8).  The caches hold one byte per element, an OCP E4M3 code c; with one
  * scale per cache tensor, c stands for c * k_scale in the key cache and
@@ -267,6 +299,14 @@ pa_status pa_decode_split_fp8(float *tmp_out, float *max_logits, float *exp_sums
  * Returns without waiting: the host inputs must stay unchanged, and out_host
  * is valid, once the stream has reached this point.  Calls on one stream are
  * ordered; the workspace is reused per call.
+ * State: unlike the other entry points, this one keeps state across calls.
+ * The first call for a (device, stream) pair creates a side stream and two
+ * events (cudaStreamCreateWithFlags, cudaEventCreateWithFlags) and keeps them
+ * in a process-wide table until exit; later calls on that pair reuse them.
+ * It allocates no device memory.
+ * A part is read (or the output written) in place only when its first and
+ * last byte both lie in one page-locked range the device can address; a part
+ * that runs past the end of its page-locked allocation is copied instead.
  *   key_cache, value_cache   device caches as for pa_decode (stay resident)
  *   workspace                caller-owned device memory, 256-byte aligned, of
  *                            pa_decode_step_host_workspace_bytes(...) bytes

@@ -16,8 +16,9 @@ import torch
 
 import oracle as oracle_mod
 from paged_kv_cache_444_b200 import (SplitWorkspace, decode_step, pa_check_error, pa_decode_fp8,
-                                     pa_decode_shared_prefix, pa_decode_split_fp8, pa_reduce,
-                                     pa_reshape_and_cache, workloads)
+                                     pa_decode_shared_prefix, pa_decode_shared_prefix_split,
+                                     pa_decode_split_fp8, pa_reduce, pa_reshape_and_cache,
+                                     workloads)
 from parity_helpers import TOL, bits, ocode, report_parity, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -108,8 +109,10 @@ def test_full_size_workload(name, cuda_device, oracle_lib):
     assert torch.equal(flat_before, flat_after)
 
 
-def test_full_size_shared_prefix_beam(cuda_device, oracle_lib):
-    """pa_decode_shared_prefix on the full beam batch (64 sequences in groups
+@pytest.mark.parametrize("partition_size", [0, 512], ids=["single_pass", "split512"])
+def test_full_size_shared_prefix_beam(partition_size, cuda_device, oracle_lib):
+    """pa_decode_shared_prefix (and pa_decode_shared_prefix_split + pa_reduce
+    with 512-token partitions) on the full beam batch (64 sequences in groups
     of 4 sharing 32 blocks), with the group arrays and max group size the
     benchmark passes, after the step's cache write."""
     cfg = workloads.CONFIGS["shared_prefix_beam"]
@@ -121,24 +124,37 @@ def test_full_size_shared_prefix_beam(cuda_device, oracle_lib):
                          batch.slot_mapping)
     sizes = (batch.group_starts[1:] - batch.group_starts[:-1]).tolist()
     out = torch.full_like(batch.query, float("nan"))
-    pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
-                            batch.block_tables, batch.context_lens, batch.group_starts,
-                            batch.prefix_blocks, cfg.scale, max(sizes))
+    if partition_size:
+        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, batch.max_partitions,
+                            cuda_device)
+        pa_decode_shared_prefix_split(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query,
+                                      batch.key_cache, batch.value_cache, batch.block_tables,
+                                      batch.context_lens, batch.group_starts,
+                                      batch.prefix_blocks, cfg.scale, max(sizes), partition_size)
+        pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, batch.context_lens,
+                  partition_size)
+        kernel = "pa_decode_shared_prefix_split+pa_reduce"
+    else:
+        pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
+                                batch.block_tables, batch.context_lens, batch.group_starts,
+                                batch.prefix_blocks, cfg.scale, max(sizes))
+        kernel = "pa_decode_shared_prefix"
     torch.cuda.synchronize()
     pa_check_error()
     ref, _, _ = _oracle_written(oracle_lib, cfg, snap)
     assert np.isfinite(to_f64(out)).all()
-    err = report_parity(oracle_lib, cfg.name, "pa_decode_shared_prefix", out[seqs], ref,
-                        ocode(cfg), TOL[cfg.dtype])
+    err = report_parity(oracle_lib, cfg.name, kernel, out[seqs], ref, ocode(cfg),
+                        TOL[cfg.dtype])
     assert err <= TOL[cfg.dtype], f"max-abs {err:.3e}"
 
 
-@pytest.mark.parametrize("name", ["mha_llama2_7b", "gqa_llama3_8b", "shared_prefix_beam",
-                                  "long_context_split"])
-def test_full_size_fp8(name, cuda_device, oracle_lib):
-    """pa_decode_fp8 (pa_decode_split_fp8 + pa_reduce for the long-context
-    workload, partition 512) on the E4M3 copies of the full-size caches the
-    benchmark times, after the step's 16-bit write."""
+@pytest.mark.parametrize("name,ps", [("mha_llama2_7b", 0), ("gqa_llama3_8b", 0),
+                                     ("shared_prefix_beam", 0), ("shared_prefix_beam", 512),
+                                     ("long_context_split", 512)])
+def test_full_size_fp8(name, ps, cuda_device, oracle_lib):
+    """pa_decode_fp8, or pa_decode_split_fp8 + pa_reduce with 512-token
+    partitions, on the E4M3 copies of the full-size caches the benchmark
+    times, after the step's 16-bit write."""
     cfg = workloads.CONFIGS[name]
     batch = workloads.make_batch(cfg, cuda_device)
     pa_reshape_and_cache(batch.key, batch.value, batch.key_cache, batch.value_cache,
@@ -147,9 +163,9 @@ def test_full_size_fp8(name, cuda_device, oracle_lib):
     seqs = _sample(batch, 2 if cfg.partition_size else 4)
     snap = _compact(batch, seqs, kc8, vc8)
     out = torch.full_like(batch.query, float("nan"))
-    if cfg.partition_size:
-        ps = cfg.partition_size
-        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, batch.max_partitions,
+    if ps:
+        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim,
+                            (batch.block_tables.shape[1] * cfg.block_size + ps - 1) // ps,
                             cuda_device)
         pa_decode_split_fp8(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query, kc8, vc8,
                             batch.block_tables, batch.context_lens, cfg.scale, FP8_SCALE,

@@ -73,3 +73,17 @@ def test_parse_cpulist():
     assert bench.parse_cpulist("0-15\n") == set(range(16))
     assert bench.parse_cpulist("0-3,8,10-11") == {0, 1, 2, 3, 8, 10, 11}
     assert bench.parse_cpulist("") == set()
+
+
+def test_timing_statistics_and_host_description():
+    """The region / launch statistics the JSON line reports: nearest-rank
+    p10 / p90, median and mean of a known list; the CPU-baseline host record."""
+    sys.path.insert(0, str(ROOT))
+    import bench
+    st = bench.stats_ms([float(x) for x in range(1, 101)])   # 1 .. 100 ms
+    assert st["n"] == 100 and st["mean"] == 50.5 and st["median"] == 50.5
+    assert st["p10"] == 11.0 and st["p90"] == 90.0            # ranks round(0.1 * 99), round(0.9 * 99)
+    one = bench.stats_ms([3.0])
+    assert one["p10"] == one["p90"] == one["median"] == 3.0
+    host = bench.host_description()
+    assert host["os_cpu_count"] == os.cpu_count() and host["cores_used"] == 1
