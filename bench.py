@@ -167,14 +167,17 @@ L2_BYTES = 126 * 1024 * 1024
 
 
 class L2Flush:
-    """Writes a buffer of twice the L2 size, so that the next launch starts
-    with none of its inputs in L2.  Runs between timed launches, untimed."""
+    """Reads a buffer of twice the L2 size, so that the next launch starts
+    with none of its inputs in L2.  Runs between timed launches, untimed.  A
+    read leaves L2 holding clean lines; a write flush would leave ~126 MB of
+    dirty lines whose write-back to HBM lands inside the next timed launch."""
 
     def __init__(self, device):
-        self.buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+        self.buf = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+        self.out = torch.zeros((), dtype=torch.float32, device=device)
 
     def __call__(self):
-        self.buf.zero_()
+        torch.sum(self.buf, dim=0, out=self.out)
 
 
 def stats_ms(times) -> dict:
@@ -921,6 +924,93 @@ def kernel_source_digest(csrc: Path | None = None) -> str:
     return h.hexdigest()[:16]
 
 
+PROFILE_KERNELS = ("pa_reshape_and_cache", "pa_decode", "pa_decode_split", "pa_reduce",
+                   "pa_decode_shared_prefix", "pa_decode_shared_prefix_split", "pa_decode_fp8",
+                   "pa_decode_split_fp8", "pa_prefill")
+
+
+def run_profile(args, local):
+    """Launch one kernel alone, --warmup + --steps times, on the --config
+    workload (pa_prefill: its chunked-prefill layer), for profiler captures:
+    nothing else of the library runs.  Prints the mean CUDA-event time of the
+    --steps launches as a short JSON object (not a bench line)."""
+    from paged_kv_cache_444_b200 import (SplitWorkspace, load, pa_decode_fp8,
+                                         pa_decode_shared_prefix, pa_decode_shared_prefix_split,
+                                         pa_decode_split, pa_decode_split_fp8, pa_prefill,
+                                         pa_reduce)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    load()
+    name = args.profile
+    if name == "pa_prefill":
+        pb = workloads.make_prefill_batch(device=device)
+        b = pb.cache
+
+        out = torch.empty_like(pb.query)
+
+        def run():
+            pa_prefill(out, pb.query, b.key_cache, b.value_cache, b.block_tables,
+                       b.context_lens, pb.query_starts, b.cfg.scale, pb.chunk)
+        cfg = b.cfg
+    else:
+        cfg = workloads.CONFIGS[args.config]
+        if args.num_seqs or args.num_blocks:
+            cfg = cfg.scaled(num_seqs=args.num_seqs or cfg.num_seqs,
+                             num_blocks=args.num_blocks or cfg.num_blocks)
+        b = workloads.make_batch(cfg, device)
+        step = Step(b)
+        ps = cfg.partition_size or SHARED_SPLIT_PARTITION
+        P = (b.block_tables.shape[1] * cfg.block_size + ps - 1) // ps
+        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, device)
+        out = torch.empty_like(b.query)
+        sizes = ((b.group_starts[1:] - b.group_starts[:-1]).tolist()
+                 if b.group_starts is not None else None)
+        if name in ("pa_decode_fp8", "pa_decode_split_fp8"):
+            q8 = lambda t: (t.float() * 64.0).clamp(-448, 448).to(torch.float8_e4m3fn) \
+                .view(torch.uint8)
+            kc8, vc8 = q8(b.key_cache), q8(b.value_cache)
+        if name in ("pa_decode_shared_prefix", "pa_decode_shared_prefix_split") and sizes is None:
+            raise SystemExit(f"--profile {name} needs a workload with prefix groups")
+        step_kernels = dict((n, fn) for n, fn, _ in step.kernels([]))
+        launches = {
+            "pa_reshape_and_cache": step_kernels["pa_reshape_and_cache"],
+            "pa_decode": step_kernels.get("pa_decode"),
+            "pa_decode_split": lambda: pa_decode_split(
+                ws.tmp_out, ws.max_logits, ws.exp_sums, b.query, b.key_cache, b.value_cache,
+                b.block_tables, b.context_lens, cfg.scale, ps),
+            "pa_reduce": lambda: pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums,
+                                           b.context_lens, ps),
+            "pa_decode_shared_prefix": lambda: pa_decode_shared_prefix(
+                out, b.query, b.key_cache, b.value_cache, b.block_tables, b.context_lens,
+                b.group_starts, b.prefix_blocks, cfg.scale, max(sizes)),
+            "pa_decode_shared_prefix_split": lambda: pa_decode_shared_prefix_split(
+                ws.tmp_out, ws.max_logits, ws.exp_sums, b.query, b.key_cache, b.value_cache,
+                b.block_tables, b.context_lens, b.group_starts, b.prefix_blocks, cfg.scale,
+                max(sizes), ps),
+            "pa_decode_fp8": lambda: pa_decode_fp8(
+                out, b.query, kc8, vc8, b.block_tables, b.context_lens, cfg.scale, 1 / 64, 1 / 64),
+            "pa_decode_split_fp8": lambda: pa_decode_split_fp8(
+                ws.tmp_out, ws.max_logits, ws.exp_sums, b.query, kc8, vc8, b.block_tables,
+                b.context_lens, cfg.scale, 1 / 64, 1 / 64, ps),
+        }
+        if name == "pa_decode" and step.ps:
+            raise SystemExit("--profile pa_decode: use a single-pass workload")
+        if name == "pa_reduce":
+            launches["pa_decode_split"]()      # partials for the merge to read
+        run = launches[name]
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        run()
+    e.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": name, "workload": cfg.name, "launches": args.steps,
+                      "ms_per_launch": round(a.elapsed_time(e) / args.steps, 5)}))
+
+
 def run_reference(args, world, rank, local):
     """The oracle (fp64, one CPU thread) as the reference arm: each step is a
     bounded sample of the same workload."""
@@ -996,6 +1086,9 @@ def main(argv=None):
     ap.add_argument("--only-prefill", action="store_true",
                     help="time only pa_prefill (its own JSON object; for profiling captures)")
     ap.add_argument("--prefill-reps", type=int, default=100)
+    ap.add_argument("--profile", choices=PROFILE_KERNELS, default=None,
+                    help="launch only this kernel (--warmup + --steps times) on the --config "
+                         "workload, for profiler captures; prints its mean time, no bench line")
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="override the workload's batch size (small profiling captures)")
     ap.add_argument("--num-blocks", type=int, default=0,
@@ -1008,6 +1101,8 @@ def main(argv=None):
         ap.error("--gpus N > 1 must be launched with torch.distributed.run (one rank per GPU)")
     if args.impl == "reference":
         run_reference(args, world, rank, local)
+    elif args.profile:
+        run_profile(args, local)
     elif args.only_prefill:
         import torch
         device = torch.device("cuda", local)
