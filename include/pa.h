@@ -216,8 +216,11 @@ pa_status pa_decode_shared_prefix(void *out, const void *query, const void *key_
  * pa_reduce merges them into the output.  A partition that reaches into a
  * group's shared prefix is computed once for a chunk of up to
  * 16 / (num_heads/num_kv_heads) members, reading each shared page once; a
- * partition past the prefix is computed for its sequence alone.  Entries of
- * partitions >= ceil(context_lens[s]/partition_size) are not written.
+ * partition past the prefix is computed for its sequence alone (two kernel
+ * launches on `stream`).  Entries of partitions >= ceil(context_lens[s] /
+ * partition_size) are not written, except that a chunk's shared partition
+ * may write an empty partial (max -inf, sum 0) for a member whose context
+ * ends before it, which pa_reduce never reads.
  * Arguments as pa_decode_shared_prefix (groups) and pa_decode_split
  * (partials, partition_size a positive multiple of block_size,
  * ceil(ctx/partition_size) <= max_partitions).  A sequence outside every

@@ -236,6 +236,8 @@ pa_status check_attention_args(const void* query, const void* key_cache, const v
 pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cache,
                      int64_t num_seqs, int64_t head_dim, int64_t num_blocks, pa_dtype dtype,
                      cudaStream_t stream) {
+  a.k_cache = static_cast<const uint8_t*>(key_cache);
+  a.v_cache = static_cast<const uint8_t*>(value_cache);
   CUtensorMap km, vm;
   if (!encode_cache_map(&km, key_cache, dtype, num_blocks, a.num_kv_heads, head_dim) ||
       !encode_cache_map(&vm, value_cache, dtype, num_blocks, a.num_kv_heads, head_dim))
@@ -256,6 +258,8 @@ pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cach
 pa_status run_decode_fp8(DecodeArgs a, const void* key_cache, const void* value_cache,
                          int64_t num_seqs, int64_t num_blocks, pa_dtype dtype,
                          cudaStream_t stream) {
+  a.k_cache = static_cast<const uint8_t*>(key_cache);
+  a.v_cache = static_cast<const uint8_t*>(value_cache);
   CUtensorMap km, vm;
   if (!encode_cache_map(&km, key_cache, dtype, num_blocks, a.num_kv_heads, 128, 1) ||
       !encode_cache_map(&vm, value_cache, dtype, num_blocks, a.num_kv_heads, 128, 1))
@@ -1024,16 +1028,36 @@ extern "C" pa_status pa_decode_shared_prefix_split(
       (reinterpret_cast<uintptr_t>(max_logits) & 3u) ||
       (reinterpret_cast<uintptr_t>(exp_sums) & 3u))
     return PA_ERR_ALIGN;
-  const long long items = num_seqs * num_kv_heads * max_partitions;
-  if (items > INT32_MAX) return PA_ERR_SHAPE;
+  // (1) the partitions that reach into a group's shared prefix: one item per
+  // (group, chunk, KV head, partition), shared pages read once per chunk
+  const long long items = static_cast<long long>(a.num_groups) * a.chunks_per_group *
+                          num_kv_heads * max_partitions;
+  if (items > INT32_MAX || num_seqs * num_kv_heads * max_partitions > INT32_MAX)
+    return PA_ERR_SHAPE;
   a.tmp_out = tmp_out;
   a.max_logits = max_logits;
   a.exp_sums = exp_sums;
   a.partition_pages = static_cast<int>(partition_size / kPage);
   a.max_partitions = static_cast<int>(max_partitions);
   a.longest_first = 0;
-  return shared_prefix_launch(a, key_cache, value_cache, items, head_dim, num_blocks, dtype,
-                              as_stream(stream));
+  cudaStream_t s = as_stream(stream);
+  if ((st = shared_prefix_launch(a, key_cache, value_cache, items, head_dim, num_blocks, dtype,
+                                 s)) != PA_OK)
+    return st;
+  // (2) every other partition, per sequence: pa_decode_split told to skip
+  // the partitions (1) wrote
+  DecodeArgs d = make_args(query, block_tables, context_lens, scale, num_heads, num_kv_heads,
+                           max_blocks_per_seq, num_blocks);
+  d.tmp_out = tmp_out;
+  d.max_logits = max_logits;
+  d.exp_sums = exp_sums;
+  d.partition_size = static_cast<int>(partition_size);
+  d.parts_per_head = static_cast<int>(max_partitions);
+  d.max_partitions = static_cast<int>(max_partitions);
+  d.group_starts = group_starts;
+  d.prefix_blocks = prefix_blocks;
+  d.num_groups = a.num_groups;
+  return run_decode(d, key_cache, value_cache, num_seqs, head_dim, num_blocks, dtype, s);
 }
 // <<< shared-prefix decode
 

@@ -18,13 +18,14 @@
 //
 // Split mode (pa_decode_shared_prefix_split) cuts every sequence into the
 // partitions of pa_decode_split and writes the same partials, which pa_reduce
-// merges.  A partition that reaches into the shared prefix is one work item
-// for the whole chunk of members (the shared pages it covers once, with every
-// row live, then each member's own pages inside the partition); a partition
-// past the prefix is an item of its sequence alone.  Items then hold at most
-// one partition of pages (plus the members' own pages where a partition
-// straddles the end of the prefix), so a batch of unequal groups no longer
-// waits on its largest item.
+// merges.  Here a work item is (group, chunk, KV head, partition) for the
+// partitions that reach into the group's shared prefix: the shared pages the
+// partition covers, once, with every row live, then each member's own pages
+// inside the partition.  The partitions past the prefix are computed per
+// sequence by paged_decode_kernel in split mode, which skips these.  Items
+// then hold at most one partition of pages (plus the members' own pages where
+// a partition straddles the end of the prefix), so a batch of unequal groups
+// no longer waits on its largest item.
 #pragma once
 
 #include "pa_decode.cuh"
@@ -80,10 +81,10 @@ __global__ void __launch_bounds__(kThreads)
   pdl_wait();
 
   // grid slot -> (group, chunk) and KV head; KV heads of one slot are adjacent.
-  // Split mode: grid slot -> (sequence, KV head, partition), partition fastest.
+  // Split mode: grid slot -> (group, chunk, KV head, partition), partition fastest.
   const bool split = a.tmp_out != nullptr;
   int item = blockIdx.x / csize;
-  int part = 0, split_seq = 0;
+  int part = 0;
   if (split) {
     part = item % a.max_partitions;
     item /= a.max_partitions;
@@ -91,18 +92,7 @@ __global__ void __launch_bounds__(kThreads)
   const int kvh = item % a.num_kv_heads;
   int slot = item / a.num_kv_heads;
   const int G = a.group;
-  if (split) {
-    // the group of sequence `slot`: the last g with group_starts[g] <= slot
-    split_seq = slot;
-    int lo = 0, hi = a.num_groups;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (a.group_starts[mid] <= split_seq) lo = mid; else hi = mid;
-    }
-    const int b0 = a.group_starts[lo];
-    const int c = split_seq >= b0 ? (split_seq - b0) / a.members_per_chunk : 0;
-    slot = lo * a.chunks_per_group + min(c, a.chunks_per_group - 1);
-  } else if (a.longest_first) {
+  if (!split && a.longest_first) {
     // rank every (group, chunk) slot by its page count, longest first (ties
     // by index), and take the one whose rank is this grid slot
     const int U = a.num_groups * a.chunks_per_group;
@@ -152,29 +142,21 @@ __global__ void __launch_bounds__(kThreads)
     if (reporter) record_error(kErrGroup, grp);
     s_end = s_begin + a.chunks_per_group * a.members_per_chunk;
   }
-  int first = s_begin + chunk * a.members_per_chunk;
-  int members = min(a.members_per_chunk, s_end - first);
+  const int first = s_begin + chunk * a.members_per_chunk;
+  const int members = min(a.members_per_chunk, s_end - first);
   int P = a.prefix_blocks[grp];
   if (P < 0 || P > a.max_blocks_per_seq) {
     if (reporter) record_error(kErrGroup, grp);
     P = P < 0 ? 0 : a.max_blocks_per_seq;
   }
   // the item's window of table entries [e0, e1): everything, or one partition
+  // (split mode: only partitions that reach into the prefix; the others are
+  // pa_decode_split's, per sequence)
   int e0 = 0, e1 = a.max_blocks_per_seq;
   if (split) {
-    if (split_seq < s_begin || split_seq >= s_end || split_seq < first ||
-        split_seq >= first + members) {
-      if (threadIdx.x == 0 && kvh == 0 && part == 0) record_error(kErrGroup, grp);
-      return;  // a sequence no group holds (or past a clipped group)
-    }
     e0 = part * a.partition_pages;
     e1 = min(e0 + a.partition_pages, a.max_blocks_per_seq);
-    if (e0 < P) {
-      if (split_seq != first) return;  // the chunk's first member owns the shared item
-    } else {
-      first = split_seq;               // past the prefix: this sequence alone
-      members = 1;
-    }
+    if (e0 >= P) return;
   }
   if (members <= 0) return;
   const int nrows = members * G;
