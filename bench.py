@@ -328,46 +328,28 @@ def time_regions(run, steps: int, warmup: int, world: int, device, min_total_s: 
     return [first] + times
 
 
-SHARED_SPLIT_PARTITION = 512  # tokens per partition of pa_decode_shared_prefix_split
+SPLIT_PARTITION = 512  # tokens per partition of the split forms timed on single-pass batches
 
 
-def shared_prefix_stats(batch, warmup: int, flush, reps: int = 100,
-                        partition_size: int = 0) -> dict:
-    """pa_decode_shared_prefix (or, with a partition size,
-    pa_decode_shared_prefix_split + pa_reduce) timed alone on a batch with
-    prefix groups: the same attention as pa_decode, reading each shared page
-    once per group.  Algorithmic bytes count the unique K/V bytes."""
-    from paged_kv_cache_444_b200 import (SplitWorkspace, pa_decode_shared_prefix,
-                                         pa_decode_shared_prefix_split, pa_reduce)
+def shared_prefix_stats(batch, warmup: int, flush, reps: int = 100) -> dict:
+    """pa_decode_shared_prefix timed alone on a batch with prefix groups: the
+    same attention as pa_decode, reading each shared page once per group.
+    Algorithmic bytes count the unique K/V bytes."""
+    from paged_kv_cache_444_b200 import pa_decode_shared_prefix
     cfg = batch.cfg
     out = torch.empty_like(batch.query)
     sizes = (batch.group_starts[1:] - batch.group_starts[:-1]).tolist()
-    if partition_size:
-        P = (batch.block_tables.shape[1] * cfg.block_size + partition_size - 1) // partition_size
-        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, batch.query.device)
 
-        def run():
-            pa_decode_shared_prefix_split(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query,
-                                          batch.key_cache, batch.value_cache,
-                                          batch.block_tables, batch.context_lens,
-                                          batch.group_starts, batch.prefix_blocks, cfg.scale,
-                                          max(sizes), partition_size)
-            pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, batch.context_lens,
-                      partition_size)
-    else:
-        def run():
-            pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
-                                    batch.block_tables, batch.context_lens, batch.group_starts,
-                                    batch.prefix_blocks, cfg.scale, max(sizes))
+    def run():
+        pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
+                                batch.block_tables, batch.context_lens, batch.group_starts,
+                                batch.prefix_blocks, cfg.scale, max(sizes))
     unique = workloads.unique_kv_bytes(cfg, batch.block_tables.cpu().tolist(),
                                        batch.context_lens.cpu().tolist())
     by = workloads.algorithmic_bytes(cfg, batch.context_lens.cpu().tolist())
     nbytes = unique + by["block_table"] + by["query"] + by["out"] + by["context_lens"]
     r = kernel_stats(run, nbytes, reps, warmup, flush)
-    r["kernel"] = ("pa_decode_shared_prefix_split+pa_reduce" if partition_size
-                   else "pa_decode_shared_prefix")
-    if partition_size:
-        r["partition_size"] = partition_size
+    r["kernel"] = "pa_decode_shared_prefix"
     return r
 
 
@@ -419,7 +401,7 @@ def split_variants(batch, warmup: int, flush, reps: int, fp8: bool) -> dict:
     equal-sized items."""
     from paged_kv_cache_444_b200 import SplitWorkspace, pa_decode_split, pa_reduce
     cfg = batch.cfg
-    ps = 512
+    ps = SPLIT_PARTITION
     P = (batch.block_tables.shape[1] * cfg.block_size + ps - 1) // ps
     ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, batch.query.device)
     out = torch.empty_like(batch.query)
@@ -735,16 +717,13 @@ def run_native(args, world, rank, local):
             "graph_ms_per_step": graph_steps(step, steps, args.warmup) if args.graph else None,
             "shared_prefix": (shared_prefix_stats(batch, args.warmup, flush, args.kernel_reps)
                               if batch.group_starts is not None else None),
-            "shared_prefix_split": (shared_prefix_stats(batch, args.warmup, flush,
-                                                        args.kernel_reps, SHARED_SPLIT_PARTITION)
-                                    if batch.group_starts is not None else None),
             "fp8": fp8_stats(batch, args.warmup, flush, args.kernel_reps) if args.fp8 else None,
             # batches of few, unequal items: the split form of each kernel too
             "split512": (split_variants(batch, args.warmup, flush, args.kernel_reps, args.fp8)
                          if batch.group_starts is not None else None),
             "context_tokens": int(sum(ctx)), "name": name,
         }
-        for key in ("shared_prefix", "shared_prefix_split"):
+        for key in ("shared_prefix",):
             if res[key]:
                 res[key]["frac_of_peak"] = round(res[key]["gbs"] / peak, 4)
                 res[key]["speedup_vs_pa_decode"] = round(
@@ -873,7 +852,6 @@ def config_entry(r: dict, peak: float) -> dict:
                      for k, v in r["kernels"].items()}}
     if r["shared_prefix"]:
         e["pa_decode_shared_prefix"] = r["shared_prefix"]
-        e["pa_decode_shared_prefix_split"] = r["shared_prefix_split"]
     if r["fp8"]:
         e["fp8"] = r["fp8"]
     if r["split512"]:
@@ -925,8 +903,7 @@ def kernel_source_digest(csrc: Path | None = None) -> str:
 
 
 PROFILE_KERNELS = ("pa_reshape_and_cache", "pa_decode", "pa_decode_split", "pa_reduce",
-                   "pa_decode_shared_prefix", "pa_decode_shared_prefix_split", "pa_decode_fp8",
-                   "pa_decode_split_fp8", "pa_prefill")
+                   "pa_decode_shared_prefix", "pa_decode_fp8", "pa_decode_split_fp8", "pa_prefill")
 
 
 def run_profile(args, local):
@@ -935,9 +912,8 @@ def run_profile(args, local):
     nothing else of the library runs.  Prints the mean CUDA-event time of the
     --steps launches as a short JSON object (not a bench line)."""
     from paged_kv_cache_444_b200 import (SplitWorkspace, load, pa_decode_fp8,
-                                         pa_decode_shared_prefix, pa_decode_shared_prefix_split,
-                                         pa_decode_split, pa_decode_split_fp8, pa_prefill,
-                                         pa_reduce)
+                                         pa_decode_shared_prefix, pa_decode_split,
+                                         pa_decode_split_fp8, pa_prefill, pa_reduce)
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     load()
@@ -959,7 +935,7 @@ def run_profile(args, local):
                              num_blocks=args.num_blocks or cfg.num_blocks)
         b = workloads.make_batch(cfg, device)
         step = Step(b)
-        ps = cfg.partition_size or SHARED_SPLIT_PARTITION
+        ps = cfg.partition_size or SPLIT_PARTITION
         P = (b.block_tables.shape[1] * cfg.block_size + ps - 1) // ps
         ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, device)
         out = torch.empty_like(b.query)
@@ -969,7 +945,7 @@ def run_profile(args, local):
             q8 = lambda t: (t.float() * 64.0).clamp(-448, 448).to(torch.float8_e4m3fn) \
                 .view(torch.uint8)
             kc8, vc8 = q8(b.key_cache), q8(b.value_cache)
-        if name in ("pa_decode_shared_prefix", "pa_decode_shared_prefix_split") and sizes is None:
+        if name == "pa_decode_shared_prefix" and sizes is None:
             raise SystemExit(f"--profile {name} needs a workload with prefix groups")
         step_kernels = dict((n, fn) for n, fn, _ in step.kernels([]))
         launches = {
@@ -983,10 +959,6 @@ def run_profile(args, local):
             "pa_decode_shared_prefix": lambda: pa_decode_shared_prefix(
                 out, b.query, b.key_cache, b.value_cache, b.block_tables, b.context_lens,
                 b.group_starts, b.prefix_blocks, cfg.scale, max(sizes)),
-            "pa_decode_shared_prefix_split": lambda: pa_decode_shared_prefix_split(
-                ws.tmp_out, ws.max_logits, ws.exp_sums, b.query, b.key_cache, b.value_cache,
-                b.block_tables, b.context_lens, b.group_starts, b.prefix_blocks, cfg.scale,
-                max(sizes), ps),
             "pa_decode_fp8": lambda: pa_decode_fp8(
                 out, b.query, kc8, vc8, b.block_tables, b.context_lens, cfg.scale, 1 / 64, 1 / 64),
             "pa_decode_split_fp8": lambda: pa_decode_split_fp8(

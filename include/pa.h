@@ -69,7 +69,8 @@ enum {
     PA_CHECK_PARTITIONS = 4,    /* ceil(context_lens[s]/partition_size) > max_partitions; index = s */
     PA_CHECK_WAIT_TIMEOUT = 5,  /* a shared-memory barrier wait gave up; index = CTA id */
     PA_CHECK_GROUP = 6,         /* malformed group bounds or prefix length; index = group */
-    PA_CHECK_QUERY = 7          /* prefill: q_len < 0, q_len > context_lens[s] or context too long; index = s */
+    PA_CHECK_QUERY = 7,         /* prefill: q_len < 0, q_len > context_lens[s] or context too long; index = s */
+    PA_CHECK_VALUE = 8          /* prefill, bf16: a V value beyond the fp16 range was clamped to +-65504; index = s */
 };
 
 /* Short English name of a status code (static string, never NULL). */
@@ -207,39 +208,6 @@ pa_status pa_decode_shared_prefix(void *out, const void *query, const void *key_
                                   pa_dtype dtype, void *stream);
 
 /*
- * pa_decode_shared_prefix_split -- the shared-prefix decode cut into the
- * partitions of pa_decode_split, for batches whose groups differ in size
- * (the same pages as pa_decode_shared_prefix: "vLLM PagedAttention 原理与源码
- * 深度解析" §3.3; "读一个真实 serving 系统 · vLLM 架构巡礼" §2).  Writes, for every
- * sequence s, head h and partition p < ceil(context_lens[s]/partition_size),
- * the partials pa_decode_split would write (same layouts and meaning), so
- * pa_reduce merges them into the output.  A partition that reaches into a
- * group's shared prefix is computed once for a chunk of up to
- * 16 / (num_heads/num_kv_heads) members, reading each shared page once; a
- * partition past the prefix is computed for its sequence alone (two kernel
- * launches on `stream`).  Entries of partitions >= ceil(context_lens[s] /
- * partition_size) are not written, except that a chunk's shared partition
- * may write an empty partial (max -inf, sum 0) for a member whose context
- * ends before it, which pa_reduce never reads.
- * Arguments as pa_decode_shared_prefix (groups) and pa_decode_split
- * (partials, partition_size a positive multiple of block_size,
- * ceil(ctx/partition_size) <= max_partitions).  A sequence outside every
- * group is skipped and reported (PA_CHECK_GROUP).
- */
-pa_status pa_decode_shared_prefix_split(float *tmp_out, float *max_logits, float *exp_sums,
-                                        const void *query, const void *key_cache,
-                                        const void *value_cache, const int32_t *block_tables,
-                                        const int32_t *context_lens,
-                                        const int32_t *group_starts,
-                                        const int32_t *prefix_blocks, float scale,
-                                        int64_t num_seqs, int64_t num_groups,
-                                        int64_t max_group_size, int64_t num_heads,
-                                        int64_t num_kv_heads, int64_t head_dim,
-                                        int64_t num_blocks, int64_t block_size,
-                                        int64_t max_blocks_per_seq, int64_t partition_size,
-                                        int64_t max_partitions, pa_dtype dtype, void *stream);
-
-/*
  * FP8 KV cache ("vLLM PagedAttention 原理与源码深度解析" §8.4: --kv-cache-dtype
  * fp8).  The caches hold one byte per element, an OCP E4M3 code c; with one
  * scale per cache tensor, c stands for c * k_scale in the key cache and
@@ -353,8 +321,12 @@ pa_status pa_decode_step_host(void *out_host, const void *query_host, const void
  *                  query_starts[num_seqs] = num_query_tokens
  *   max_query_len  host-side upper bound of every q_len (sizes the grid)
  * Other arguments as pa_decode.  A sequence with q_len > context_lens[s] is
- * skipped and reported (PA_CHECK_QUERY).  fp32 accumulation; P enters the
- * P.V product in the cache dtype (bf16 as a hi + lo pair).
+ * skipped and reported (PA_CHECK_QUERY).  fp32 accumulation.  P enters the
+ * P.V product as fp16 (11 bits).  With bf16 caches each V block is first
+ * rewritten as fp16 in shared memory: exact for every bf16 value below
+ * 65 520 in magnitude (values below 2^-14 lose at most 2^-25 each); a V value
+ * beyond the fp16 range saturates to +-65504 and is reported
+ * (PA_CHECK_VALUE, index = the sequence).
  */
 pa_status pa_prefill(void *out, const void *query, const void *key_cache,
                      const void *value_cache, const int32_t *block_tables,

@@ -11,15 +11,13 @@ from __future__ import annotations
 import torch
 
 from ._lib import (DecodePlan, HostStep, PagedAttentionError, load, pa_check_error, pa_copy_blocks, pa_decode,
-                   pa_decode_fp8, pa_decode_noalloc, pa_decode_shared_prefix,
-                   pa_decode_shared_prefix_split, pa_decode_split,
+                   pa_decode_fp8, pa_decode_noalloc, pa_decode_shared_prefix, pa_decode_split,
                    pa_decode_split_fp8, pa_prefill, pa_reduce, pa_reshape_and_cache,
                    pa_reshape_and_cache_fp8)
 
 __all__ = [
     "PagedAttentionError", "load", "pa_reshape_and_cache", "pa_decode", "pa_decode_split",
     "pa_reduce", "pa_check_error", "pa_decode_noalloc", "pa_decode_shared_prefix",
-    "pa_decode_shared_prefix_split",
     "pa_copy_blocks", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_decode_split_fp8",
     "pa_prefill", "SplitWorkspace", "decode_step", "HostStep", "DecodePlan",
 ]

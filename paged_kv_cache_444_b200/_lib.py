@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_NULL", 2: "PA_ERR_SHAPE", 3: "PA_ERR_DTYP
                 4: "PA_ERR_ALIGN", 5: "PA_ERR_UNSUPPORTED", 6: "PA_ERR_CUDA",
                 7: "PA_ERR_BOUNDS"}
 CHECK_CODES = {1: "slot", 2: "block_id", 3: "context_len", 4: "partitions", 5: "wait_timeout",
-               6: "group", 7: "query"}
+               6: "group", 7: "query", 8: "value"}
 DTYPE_CODES = {torch.float16: 0, torch.bfloat16: 1}
 
 
@@ -60,7 +60,6 @@ SIGNATURES = {
                                _i64, _i64, _i, _p]),
     "pa_decode_shared_prefix": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _f, _i64, _i64, _i64, _i64,
                                      _i64, _i64, _i64, _i64, _i64, _i, _p]),
-    "pa_decode_shared_prefix_split": (_i, [_p] * 10 + [_f] + [_i64] * 11 + [_i, _p]),
     "pa_copy_blocks": (_i, [_p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p]),
     "pa_reshape_and_cache_fp8": (_i, [_p, _p, _i64, _i64, _p, _p, _p, _i64, _i64, _i64, _i64,
                                       _i64, _f, _f, _i, _p]),
@@ -257,36 +256,6 @@ def pa_decode_shared_prefix(out: torch.Tensor, query: torch.Tensor, key_cache: t
         prefix_blocks.data_ptr(), float(scale), S, n_groups, int(max_group_size), H, Hk, D, NB,
         bs, MB, dt, _stream(stream))
     _check(st, "pa_decode_shared_prefix")
-
-
-def pa_decode_shared_prefix_split(tmp_out: torch.Tensor, max_logits: torch.Tensor,
-                                  exp_sums: torch.Tensor, query: torch.Tensor,
-                                  key_cache: torch.Tensor, value_cache: torch.Tensor,
-                                  block_tables: torch.Tensor, context_lens: torch.Tensor,
-                                  group_starts: torch.Tensor, prefix_blocks: torch.Tensor,
-                                  scale: float, max_group_size: int, partition_size: int,
-                                  stream=None) -> None:
-    """pa_decode_shared_prefix cut into pa_decode_split's partitions: writes
-    the partials (tmp_out [S, H, P, D], max_logits / exp_sums [S, H, P] fp32)
-    that pa_reduce merges; shared prefix pages are read once per group chunk."""
-    S, H, D, NB, bs, Hk, MB, dt = _attention_common(query, key_cache, value_cache,
-                                                    block_tables, context_lens)
-    P = max_logits.shape[-1]
-    _need(tmp_out.shape == (S, H, P, D) and tmp_out.dtype == torch.float32
-          and tmp_out.is_contiguous(), "tmp_out must be [S, H, P, D] float32")
-    _need(max_logits.shape == (S, H, P) and exp_sums.shape == (S, H, P) and
-          max_logits.dtype == exp_sums.dtype == torch.float32, "max_logits/exp_sums [S, H, P] f32")
-    n_groups = prefix_blocks.shape[0]
-    _need(group_starts.dtype == torch.int32 and group_starts.shape == (n_groups + 1,),
-          "group_starts must be [num_groups + 1] int32")
-    _need(prefix_blocks.dtype == torch.int32, "prefix_blocks must be int32")
-    st = load().pa_decode_shared_prefix_split(
-        tmp_out.data_ptr(), max_logits.data_ptr(), exp_sums.data_ptr(), query.data_ptr(),
-        key_cache.data_ptr(), value_cache.data_ptr(), block_tables.data_ptr(),
-        context_lens.data_ptr(), group_starts.data_ptr(), prefix_blocks.data_ptr(),
-        float(scale), S, n_groups, int(max_group_size), H, Hk, D, NB, bs, MB,
-        int(partition_size), P, dt, _stream(stream))
-    _check(st, "pa_decode_shared_prefix_split")
 
 
 def pa_copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor,

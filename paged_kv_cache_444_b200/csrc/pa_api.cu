@@ -236,8 +236,6 @@ pa_status check_attention_args(const void* query, const void* key_cache, const v
 pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cache,
                      int64_t num_seqs, int64_t head_dim, int64_t num_blocks, pa_dtype dtype,
                      cudaStream_t stream) {
-  a.k_cache = static_cast<const uint8_t*>(key_cache);
-  a.v_cache = static_cast<const uint8_t*>(value_cache);
   CUtensorMap km, vm;
   if (!encode_cache_map(&km, key_cache, dtype, num_blocks, a.num_kv_heads, head_dim) ||
       !encode_cache_map(&vm, value_cache, dtype, num_blocks, a.num_kv_heads, head_dim))
@@ -258,8 +256,6 @@ pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cach
 pa_status run_decode_fp8(DecodeArgs a, const void* key_cache, const void* value_cache,
                          int64_t num_seqs, int64_t num_blocks, pa_dtype dtype,
                          cudaStream_t stream) {
-  a.k_cache = static_cast<const uint8_t*>(key_cache);
-  a.v_cache = static_cast<const uint8_t*>(value_cache);
   CUtensorMap km, vm;
   if (!encode_cache_map(&km, key_cache, dtype, num_blocks, a.num_kv_heads, 128, 1) ||
       !encode_cache_map(&vm, value_cache, dtype, num_blocks, a.num_kv_heads, 128, 1))
@@ -901,11 +897,10 @@ pa_status launch_shared_prefix_t(const CUtensorMap& km, const CUtensorMap& vm,
   if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
   // one cluster size for the launch: as large as PA_SHARED_CLUSTER if the
   // device can co-schedule it, and 1 when no item can exceed the threshold
-  // (split mode: items are at most a partition, never spread)
   const int64_t max_item_pages =
       static_cast<int64_t>(a.members_per_chunk) * a.max_blocks_per_seq;
   int c = 1;
-  if (!a.tmp_out && max_item_pages > PA_SHARED_CLUSTER_PAGES) {
+  if (max_item_pages > PA_SHARED_CLUSTER_PAGES) {
     c = pick_cluster(kernel, L::kAlloc, static_cast<int64_t>(PA_SHARED_CLUSTER) *
                                             PA_CLUSTER_TABLE_PAGES, cluster_cache);
     if (c > PA_SHARED_CLUSTER) c = PA_SHARED_CLUSTER;
@@ -914,66 +909,6 @@ pa_status launch_shared_prefix_t(const CUtensorMap& km, const CUtensorMap& vm,
   if (items * c > INT32_MAX) return PA_ERR_SHAPE;
   return launch_ex(kernel, static_cast<unsigned>(items * c), kThreads, L::kAlloc, stream, c, km,
                    vm, a);
-}
-
-// Validation and arguments shared by the single-pass and split forms.
-pa_status shared_prefix_setup(const void* query, const void* key_cache, const void* value_cache,
-                              const int32_t* block_tables, const int32_t* context_lens,
-                              const int32_t* group_starts, const int32_t* prefix_blocks,
-                              float scale, int64_t num_seqs, int64_t num_groups,
-                              int64_t max_group_size, int64_t num_heads, int64_t num_kv_heads,
-                              int64_t head_dim, int64_t num_blocks, int64_t block_size,
-                              int64_t max_blocks_per_seq, pa_dtype dtype, SharedPrefixArgs* a,
-                              bool* nothing) {
-  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
-                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
-                                      num_blocks, block_size, max_blocks_per_seq, dtype);
-  if (st != PA_OK) return st;
-  if (num_groups < 0 || max_group_size <= 0) return PA_ERR_SHAPE;
-  *nothing = num_seqs == 0 || num_groups == 0;
-  if (*nothing) return PA_OK;
-  if (!group_starts || !prefix_blocks) return PA_ERR_NULL;
-  if ((reinterpret_cast<uintptr_t>(group_starts) & 3u) ||
-      (reinterpret_cast<uintptr_t>(prefix_blocks) & 3u))
-    return PA_ERR_ALIGN;
-  const int64_t G = num_heads / num_kv_heads;
-  const int64_t per_chunk = 16 / G;                       // G <= 16 checked above
-  const int64_t chunks = (max_group_size + per_chunk - 1) / per_chunk;
-  if (num_groups > INT32_MAX || chunks > INT32_MAX ||
-      num_groups * num_kv_heads * chunks > INT32_MAX)
-    return PA_ERR_SHAPE;
-  *a = SharedPrefixArgs{};
-  a->query = static_cast<const uint16_t*>(query);
-  a->block_tables = block_tables;
-  a->context_lens = context_lens;
-  a->group_starts = group_starts;
-  a->prefix_blocks = prefix_blocks;
-  a->scale_log2 = scale * kLog2e;
-  a->num_seqs = static_cast<int>(num_seqs);
-  a->num_heads = static_cast<int>(num_heads);
-  a->num_kv_heads = static_cast<int>(num_kv_heads);
-  a->group = static_cast<int>(G);
-  a->max_blocks_per_seq = static_cast<int>(max_blocks_per_seq);
-  a->num_blocks = static_cast<int>(num_blocks);
-  a->num_groups = static_cast<int>(num_groups);
-  a->members_per_chunk = static_cast<int>(per_chunk);
-  a->chunks_per_group = static_cast<int>(chunks);
-  return PA_OK;
-}
-
-pa_status shared_prefix_launch(const SharedPrefixArgs& a, const void* key_cache,
-                               const void* value_cache, long long items, int64_t head_dim,
-                               int64_t num_blocks, pa_dtype dtype, cudaStream_t s) {
-  CUtensorMap km, vm;
-  if (!encode_cache_map(&km, key_cache, dtype, num_blocks, a.num_kv_heads, head_dim) ||
-      !encode_cache_map(&vm, value_cache, dtype, num_blocks, a.num_kv_heads, head_dim))
-    return PA_ERR_CUDA;
-  const bool bf16 = dtype == PA_BF16;
-  if (head_dim == 64)
-    return bf16 ? launch_shared_prefix_t<64, true>(km, vm, a, items, s)
-                : launch_shared_prefix_t<64, false>(km, vm, a, items, s);
-  return bf16 ? launch_shared_prefix_t<128, true>(km, vm, a, items, s)
-              : launch_shared_prefix_t<128, false>(km, vm, a, items, s);
 }
 
 }  // namespace
@@ -986,78 +921,50 @@ extern "C" pa_status pa_decode_shared_prefix(void* out, const void* query, const
                                   int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
                                   int64_t block_size, int64_t max_blocks_per_seq, pa_dtype dtype,
                                   void* stream) {
-  SharedPrefixArgs a;
-  bool nothing = false;
-  pa_status st = shared_prefix_setup(query, key_cache, value_cache, block_tables, context_lens,
-                                     group_starts, prefix_blocks, scale, num_seqs, num_groups,
-                                     max_group_size, num_heads, num_kv_heads, head_dim,
-                                     num_blocks, block_size, max_blocks_per_seq, dtype, &a,
-                                     &nothing);
-  if (st != PA_OK || nothing) return st;
-  if (!out) return PA_ERR_NULL;
-  if (!aligned16(out)) return PA_ERR_ALIGN;
-  a.out = static_cast<uint16_t*>(out);
-  const long long items = static_cast<long long>(a.num_groups) * a.num_kv_heads *
-                          a.chunks_per_group;
-  a.longest_first = static_cast<long long>(a.num_groups) * a.chunks_per_group <= kLptMaxSeqs;
-  return shared_prefix_launch(a, key_cache, value_cache, items, head_dim, num_blocks, dtype,
-                              as_stream(stream));
-}
-
-extern "C" pa_status pa_decode_shared_prefix_split(
-    float* tmp_out, float* max_logits, float* exp_sums, const void* query,
-    const void* key_cache, const void* value_cache, const int32_t* block_tables,
-    const int32_t* context_lens, const int32_t* group_starts, const int32_t* prefix_blocks,
-    float scale, int64_t num_seqs, int64_t num_groups, int64_t max_group_size,
-    int64_t num_heads, int64_t num_kv_heads, int64_t head_dim, int64_t num_blocks,
-    int64_t block_size, int64_t max_blocks_per_seq, int64_t partition_size,
-    int64_t max_partitions, pa_dtype dtype, void* stream) {
-  if (partition_size <= 0 || max_partitions <= 0) return PA_ERR_SHAPE;
-  if (partition_size % kPage != 0) return PA_ERR_UNSUPPORTED;
-  if (partition_size > INT32_MAX || max_partitions > INT32_MAX) return PA_ERR_SHAPE;
-  SharedPrefixArgs a;
-  bool nothing = false;
-  pa_status st = shared_prefix_setup(query, key_cache, value_cache, block_tables, context_lens,
-                                     group_starts, prefix_blocks, scale, num_seqs, num_groups,
-                                     max_group_size, num_heads, num_kv_heads, head_dim,
-                                     num_blocks, block_size, max_blocks_per_seq, dtype, &a,
-                                     &nothing);
-  if (st != PA_OK || nothing) return st;
-  if (!tmp_out || !max_logits || !exp_sums) return PA_ERR_NULL;
-  if ((reinterpret_cast<uintptr_t>(tmp_out) & 7u) ||
-      (reinterpret_cast<uintptr_t>(max_logits) & 3u) ||
-      (reinterpret_cast<uintptr_t>(exp_sums) & 3u))
+  pa_status st = check_attention_args(query, key_cache, value_cache, block_tables, context_lens,
+                                      scale, num_seqs, num_heads, num_kv_heads, head_dim,
+                                      num_blocks, block_size, max_blocks_per_seq, dtype);
+  if (st != PA_OK) return st;
+  if (num_groups < 0 || max_group_size <= 0) return PA_ERR_SHAPE;
+  if (num_seqs == 0 || num_groups == 0) return PA_OK;
+  if (!out || !group_starts || !prefix_blocks) return PA_ERR_NULL;
+  if (!aligned16(out) || (reinterpret_cast<uintptr_t>(group_starts) & 3u) ||
+      (reinterpret_cast<uintptr_t>(prefix_blocks) & 3u))
     return PA_ERR_ALIGN;
-  // (1) the partitions that reach into a group's shared prefix: one item per
-  // (group, chunk, KV head, partition), shared pages read once per chunk
-  const long long items = static_cast<long long>(a.num_groups) * a.chunks_per_group *
-                          num_kv_heads * max_partitions;
-  if (items > INT32_MAX || num_seqs * num_kv_heads * max_partitions > INT32_MAX)
-    return PA_ERR_SHAPE;
-  a.tmp_out = tmp_out;
-  a.max_logits = max_logits;
-  a.exp_sums = exp_sums;
-  a.partition_pages = static_cast<int>(partition_size / kPage);
-  a.max_partitions = static_cast<int>(max_partitions);
-  a.longest_first = 0;
+  const int64_t G = num_heads / num_kv_heads;
+  const int64_t per_chunk = 16 / G;                       // G <= 16 checked above
+  const int64_t chunks = (max_group_size + per_chunk - 1) / per_chunk;
+  const int64_t items = num_groups * num_kv_heads * chunks;
+  if (num_groups > INT32_MAX || chunks > INT32_MAX || items > INT32_MAX) return PA_ERR_SHAPE;
+  CUtensorMap km, vm;
+  if (!encode_cache_map(&km, key_cache, dtype, num_blocks, num_kv_heads, head_dim) ||
+      !encode_cache_map(&vm, value_cache, dtype, num_blocks, num_kv_heads, head_dim))
+    return PA_ERR_CUDA;
+  SharedPrefixArgs a{};
+  a.query = static_cast<const uint16_t*>(query);
+  a.out = static_cast<uint16_t*>(out);
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.group_starts = group_starts;
+  a.prefix_blocks = prefix_blocks;
+  a.scale_log2 = scale * kLog2e;
+  a.num_seqs = static_cast<int>(num_seqs);
+  a.num_heads = static_cast<int>(num_heads);
+  a.num_kv_heads = static_cast<int>(num_kv_heads);
+  a.group = static_cast<int>(G);
+  a.max_blocks_per_seq = static_cast<int>(max_blocks_per_seq);
+  a.num_blocks = static_cast<int>(num_blocks);
+  a.num_groups = static_cast<int>(num_groups);
+  a.members_per_chunk = static_cast<int>(per_chunk);
+  a.chunks_per_group = static_cast<int>(chunks);
+  a.longest_first = num_groups * chunks <= kLptMaxSeqs;
   cudaStream_t s = as_stream(stream);
-  if ((st = shared_prefix_launch(a, key_cache, value_cache, items, head_dim, num_blocks, dtype,
-                                 s)) != PA_OK)
-    return st;
-  // (2) every other partition, per sequence: pa_decode_split told to skip
-  // the partitions (1) wrote
-  DecodeArgs d = make_args(query, block_tables, context_lens, scale, num_heads, num_kv_heads,
-                           max_blocks_per_seq, num_blocks);
-  d.tmp_out = tmp_out;
-  d.max_logits = max_logits;
-  d.exp_sums = exp_sums;
-  d.partition_size = static_cast<int>(partition_size);
-  d.parts_per_head = static_cast<int>(max_partitions);
-  d.max_partitions = static_cast<int>(max_partitions);
-  d.group_starts = group_starts;
-  d.prefix_blocks = prefix_blocks;
-  d.num_groups = a.num_groups;
-  return run_decode(d, key_cache, value_cache, num_seqs, head_dim, num_blocks, dtype, s);
+  const bool bf16 = dtype == PA_BF16;
+  if (head_dim == 64)
+    return bf16 ? launch_shared_prefix_t<64, true>(km, vm, a, items, s)
+                : launch_shared_prefix_t<64, false>(km, vm, a, items, s);
+  return bf16 ? launch_shared_prefix_t<128, true>(km, vm, a, items, s)
+              : launch_shared_prefix_t<128, false>(km, vm, a, items, s);
 }
 // <<< shared-prefix decode
 
@@ -1095,7 +1002,8 @@ pa_status launch_prefill_t(const CUtensorMap& qm, const CUtensorMap& km, const C
   auto kernel = paged_prefill_kernel<D, BF16>;
   static std::atomic<uint64_t> done{0};
   if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
-  return launch_ex(kernel, static_cast<unsigned>(grid), kPrefillThreads, L::kAlloc, stream, 1, qm,
+  return launch_ex(kernel, static_cast<unsigned>(grid), PrefillRoles<BF16>::kThreads, L::kAlloc,
+                   stream, 1, qm,
                    km, vm, a);
 }
 

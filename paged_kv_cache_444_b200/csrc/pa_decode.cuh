@@ -64,24 +64,7 @@ struct DecodeArgs {
   int cluster_pages;          // an item with more pages than this is spread over its cluster
   int num_seqs;
   int longest_first;          // order single-pass items by descending context length
-  // split mode, optional: sequences come in groups that share their first
-  // prefix_blocks[g] table entries; partitions that reach into a group's
-  // shared prefix are left to the shared-prefix kernel (null: none skipped)
-  const int32_t* group_starts;  // [num_groups + 1]
-  const int32_t* prefix_blocks; // [num_groups]
-  int num_groups;
-  const uint8_t* k_cache;       // the caches' base addresses (L2 prefetch of later pages)
-  const uint8_t* v_cache;
 };
-
-// Pages of a warp's ring pulled into L2 ahead of their TMA loads (beyond the
-// NST pages in flight into shared memory), per cache element size.
-#ifndef PA_PREFETCH_16
-#define PA_PREFETCH_16 0
-#endif
-#ifndef PA_PREFETCH_FP8
-#define PA_PREFETCH_FP8 0
-#endif
 
 
 template <int D, int NST, int EB = 2>   // EB: bytes per cache element (2, or 1 for fp8)
@@ -376,36 +359,6 @@ __device__ __forceinline__ void merge_and_emit(uint8_t* smem, int nrows, bool sp
 }
 
 // ---------------------------------------------------------------------------
-// Split mode with prefix groups: true when partition `part` of sequence s
-// reaches into the shared prefix of s's group (its first entry lies before
-// the group's prefix_blocks), which the shared-prefix kernel computes once
-// per chunk of members.  A sequence outside every group has no shared prefix.
-// Whole CTA, uniform result; uses the stage area (free at this point).
-// ---------------------------------------------------------------------------
-template <int STAGE_BYTES>
-__device__ __forceinline__ bool partition_in_shared_prefix(const DecodeArgs& a, int s, int part,
-                                                           uint8_t* smem) {
-  const int n = a.num_groups + 1;
-  const int* starts = a.group_starts;
-  if (n * 4 <= STAGE_BYTES) {  // the group bounds into shared memory, one pass
-    int* st = reinterpret_cast<int*>(smem);
-    for (int i = threadIdx.x; i < n; i += kThreads) st[i] = a.group_starts[i];
-    __syncthreads();
-    starts = st;
-  }
-  int lo = 0, hi = a.num_groups;  // the last g with starts[g] <= s
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (starts[mid] <= s) lo = mid; else hi = mid;
-  }
-  const bool member = a.num_groups > 0 && starts[lo] <= s && s < starts[lo + 1];
-  __syncthreads();  // every thread has read the bounds; the stage area is reused next
-  if (!member) return false;
-  const int P = min(max(a.prefix_blocks[lo], 0), a.max_blocks_per_seq);
-  return part * (a.partition_size / kPage) < P;
-}
-
-// ---------------------------------------------------------------------------
 // After a warp's page loop: true when none of its TMA loads is still in
 // flight.  A loop that ended normally (ok) consumed every page it issued.  One
 // that gave up at page k_stop has issued pages k_stop .. min(k_stop + NST,
@@ -504,9 +457,6 @@ __global__ void __launch_bounds__(kThreads)
     t_begin = part * a.partition_size;
     t_end = min(t_begin + a.partition_size, ctx);
     if (t_begin >= t_end) return;  // partition past the end: nothing to write
-    if (a.group_starts != nullptr &&
-        partition_in_shared_prefix<L::kStagesBytes>(a, s, part, smem))
-      return;  // the shared-prefix kernel writes this partition
   } else if (ctx == 0) {
     // empty sequence: zero output rows
     if (crank == 0) {
@@ -571,27 +521,8 @@ __global__ void __launch_bounds__(kThreads)
     }
   };
 
-  // L2 prefetch of page k's K and V rows (whole warp: lanes 0-15 take the 16
-  // K rows, lanes 16-31 the V rows), PF pages beyond the ring, so that their
-  // TMA loads find them in L2.  Ids were range-checked by load_ids.
-  constexpr int PF = EB == 1 ? PA_PREFETCH_FP8 : PA_PREFETCH_16;
-  static_assert(NST + PF <= 32, "prefetched pages must lie within the next id window");
-  auto prefetch = [&](int k) {
-    const int src = ((k >> 5) == win) ? ids_cur : ids_next;
-    const int id = __shfl_sync(0xffffffffu, src, k & 31);
-    if (id >= 0) {
-      const uint8_t* base = lane < 16 ? a.k_cache : a.v_cache;
-      const size_t row = (static_cast<size_t>(id) * kPage + (lane & 15)) * a.num_kv_heads + kvh;
-      prefetch_l2_bulk(base + row * (D * EB), D * EB);
-    }
-  };
-
   const int pre = my_pages < NST ? my_pages : NST;
   for (int k = 0; k < pre; ++k) issue(k);
-  if constexpr (PF > 0) {
-    const int pf_end = min(my_pages, NST + PF);
-    for (int k = NST; k < pf_end; ++k) prefetch(k);
-  }
 
   // ---- this warp's query rows ----
   Warp st;
@@ -622,9 +553,6 @@ __global__ void __launch_bounds__(kThreads)
     st.page(kb, kb + L::kPageBytes, tok0, t_end, a.scale_log2, lane);
     __syncwarp();
     if (k + NST < my_pages) issue(k + NST);
-    if constexpr (PF > 0) {
-      if (k + NST + PF < my_pages) prefetch(k + NST + PF);
-    }
   }
 
   // ---- merge the four warps (the stage area is reused as the merge buffer).

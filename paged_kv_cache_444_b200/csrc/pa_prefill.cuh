@@ -33,7 +33,9 @@
 // 16-bit operand and the final 1/l uses the same reference).  bf16 P enters
 // P V as a hi + lo pair of bf16 products (at least 14 bits of P, split by
 // bit truncation so the conversion unit stays free for 2^x); fp16 P is
-// rounded once and l sums the rounded values.
+// rounded once and l sums the rounded values.  With bf16 caches the default
+// build rewrites each V block as fp16 in shared memory (four converter warps)
+// and takes the fp16 P path instead (PA_PREFILL_V_FP16, below).
 #pragma once
 
 #include "pa_decode.cuh"
@@ -48,6 +50,37 @@ constexpr int kPrefillPages = kPrefillKeys / kPage; // 8 pages per block
 constexpr int kWarpMma = 8;                         // issues every MMA, owns tensor memory
 constexpr int kWarpTma = 9;                         // Q, K and V loads
 constexpr int kPrefillThreads = 10 * 32;            // + two softmax warpgroups (warps 0-7)
+constexpr int kWarpConv = 10;                       // V converters: warps 10-13 (convert mode)
+constexpr unsigned kErrValue = 8;
+
+// bf16 caches: rewrite each landed V block as fp16 in shared memory (warps
+// 10-13, once per block for both tiles), so that P enters P V once, as fp16
+// (11 bits), instead of as a bf16 hi + lo pair.  fp16 holds every bf16 value
+// of magnitude below 65 520 exactly, apart from the tiny ones below 2^-14,
+// which lose at most 2^-25 each; larger values saturate to +-65 504 and are
+// reported (PA_CHECK_VALUE).
+#ifndef PA_PREFILL_V_FP16
+#define PA_PREFILL_V_FP16 1
+#endif
+template <bool BF16>
+struct PrefillRoles {
+  static constexpr bool kConvert = BF16 && PA_PREFILL_V_FP16 != 0;
+  // convert mode: four whole warpgroups (setmaxnreg works per warpgroup):
+  // softmax 0-7, then MMA, TMA, converters 10-13 and two idle warps
+  static constexpr int kThreads = kConvert ? 16 * 32 : kPrefillThreads;
+  static constexpr bool kPHiLo = BF16 && !kConvert;   // P as a bf16 hi + lo pair
+};
+
+// Register split of convert mode: 512 threads launched at 128 registers each
+// (65 536, the whole file); the two softmax warpgroups take 184, the other two
+// give up to 72: 2 x 128 x 184 + 2 x 128 x 72 = 65 536.
+constexpr uint32_t kRegsSoftmax = 184, kRegsOther = 72;
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+}
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+}
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;                      // O_t: columns [128 t, 128 t + D)
 constexpr uint32_t kTmemS = 256;                    // S_t / P_t: [256 + 128 t, +128)
@@ -85,7 +118,8 @@ struct PrefillSmem {
   static constexpr int kBarKEmpty = kBarKFull + 8 * NST;
   static constexpr int kBarVFull = kBarKEmpty + 8 * NST;
   static constexpr int kBarVEmpty = kBarVFull + 8 * NST;
-  static constexpr int kBarS = kBarVEmpty + 8 * NST;   // per tile: S_t(j) (and P_t(j-1) V) done
+  static constexpr int kBarVConv = kBarVEmpty + 8 * NST;  // V block rewritten as fp16 (convert mode)
+  static constexpr int kBarS = kBarVConv + 8 * NST;    // per tile: S_t(j) (and P_t(j-1) V) done
   static constexpr int kBarP = kBarS + 16;             // per tile: P_t(j) written
   static constexpr int kBarO = kBarP + 16;             // every MMA done
   static constexpr int kTmemSlot = kBarO + 8;
@@ -202,11 +236,12 @@ __device__ __forceinline__ bool prefill_unit_of_rank(const LptSeq& q, int max_ke
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(kPrefillThreads, 1)
+__global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap qmap,
                          const __grid_constant__ CUtensorMap kmap,
                          const __grid_constant__ CUtensorMap vmap, const PrefillArgs a) {
   using L = PrefillSmem<D, BF16>;
+  using R = PrefillRoles<BF16>;
   constexpr int NST = L::NST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -303,6 +338,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(sb + L::kBarKEmpty + 8 * i, 1);
       mbar_init(sb + L::kBarVFull + 8 * i, 1);
       mbar_init(sb + L::kBarVEmpty + 8 * i, 1);
+      if constexpr (R::kConvert) mbar_init(sb + L::kBarVConv + 8 * i, 128);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(sb + L::kBarS + 8 * t, 1);
@@ -326,7 +362,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   __syncthreads();
   tmem_fence_after_sync();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlot);
-
+  // the warpgroup index, made visibly warp-uniform for the register split
+  const int wgroup = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x) / 128, 0);
+  if (wgroup >= 2) {
+  // warpgroups 2 and 3: MMA issuer, TMA producer, V converters, idle warps
+  if constexpr (R::kConvert) regs_decrease();
   if (warp == kWarpTma) {
     // ================= TMA producer =================
     if (lane == 0) {
@@ -399,7 +439,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   } else if (warp == kWarpMma) {
     // ================= MMA issuer =================
     constexpr uint32_t kIdS = umma_idesc_f16(BF16, kPrefillRows, kPrefillKeys, false);
-    constexpr uint32_t kIdO = umma_idesc_f16(BF16, kPrefillRows, D, true);
+    constexpr uint32_t kIdO = umma_idesc_f16(R::kPHiLo, kPrefillRows, D, true);
     auto issue_s = [&](int t, int j) {   // S_t(j) = Q_t K_j^T, then report it
       const uint32_t kst = sb + L::kK + (j % NST) * L::kStage;
       const uint32_t qt = sb + L::kQ + t * L::kQTile;
@@ -418,7 +458,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       for (int k = 0; k < pages_here; ++k) {
         const uint64_t bd = umma_desc_sw128(vst + k * 2048, L::kSlab, 1024);
         umma_f16_ts(tmem + kTmemO + 128 * t, pcol + 8 * k, bd, kIdO, (j > 0 || k > 0) ? 1u : 0u);
-        if constexpr (BF16) umma_f16_ts(tmem + kTmemO + 128 * t, pcol + 64 + 8 * k, bd, kIdO, 1u);
+        if constexpr (R::kPHiLo)
+          umma_f16_ts(tmem + kTmemO + 128 * t, pcol + 64 + 8 * k, bd, kIdO, 1u);
       }
     };
     // whole-warp waits; lane 0 issues
@@ -430,6 +471,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int last_page = (ctx - 1) / kPage;
     const int tail_row = ctx % kPage;          // first row past the context in the last page
     auto v_ready = [&](int j) {                // V_j landed; clear its rows past the context
+      if constexpr (R::kConvert)   // the converters rewrote it (and cleared those rows)
+        return wait(sb + L::kBarVConv + 8 * (j % NST), (j / NST) & 1);
       if (!wait(sb + L::kBarVFull + 8 * (j % NST), (j / NST) & 1)) return false;
       const int lp = last_page - j * kPrefillPages;
       if (tail_row != 0 && lp >= 0 && lp < kPrefillPages) {
@@ -486,7 +529,53 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (lane == 0) umma_commit(sb + L::kBarO);
     __syncwarp();
     if (!mbar_wait_bounded(sb + L::kBarO, 0) && lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
-  } else if (warp < 4 || has_b) {
+  } else if (R::kConvert && warp >= kWarpConv && warp < kWarpConv + 4) {
+    // ================= V converters (convert mode) =================
+    // Each landed V block (bf16, 128 keys x D, two or one 128-byte-swizzled
+    // slabs) is rewritten in place as fp16, element for element (the swizzle
+    // moves whole 16-byte chunks, so chunk positions are unchanged), and rows
+    // past the context in the sequence's last page are cleared.
+    const int ct = threadIdx.x - kWarpConv * 32;   // 0 .. 127
+    const int last_page = (ctx - 1) / kPage;
+    const int tail_row = ctx % kPage;
+    uint32_t clipped = 0;
+    for (int j = 0; j < nkb; ++j) {
+      const int st = j % NST;
+      if (!__all_sync(0xffffffffu, wait_or_abort(sb + L::kBarVFull + 8 * st, (j / NST) & 1,
+                                                 abort_flag)))
+        break;
+      const uint32_t vst = sb + L::kV + st * L::kStage;
+      const int lp = last_page - j * kPrefillPages;  // this block's page holding the end, if any
+      for (int c = ct; c < L::kStage / 16; c += 128) {
+        const int row = (c >> 3) & (kPrefillKeys - 1);   // key within the block
+        const uint32_t addr = vst + c * 16;
+        uint32_t w[4];
+        if (tail_row != 0 && (row >> 4) == lp && (row & 15) >= tail_row) {
+          w[0] = w[1] = w[2] = w[3] = 0u;
+        } else {
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr));
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+            uint32_t h;
+            asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(hi), "f"(lo));
+            // no bf16 value is 65 504, so a half of magnitude 65 504 was clipped
+            clipped |= __vcmpeq2(h & 0x7fff7fffu, 0x7bff7bffu);
+            w[i] = h;
+          }
+        }
+        sts128(addr, w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(sb + L::kBarVConv + 8 * st);
+    }
+    if (__any_sync(0xffffffffu, clipped != 0) && lane == 0) record_error(kErrValue, s);
+  }
+  } else {
+  // warpgroups 0 and 1: the softmax of tiles A and B
+  if constexpr (R::kConvert) regs_increase();
+  if (warp < 4 || has_b) {
     // ================= softmax: tile t = warp / 4, row = TMEM lane =================
     const int t = warp >> 2;
     const int row = threadIdx.x & 127;
@@ -504,7 +593,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (!ok) break;
       tmem_fence_after_sync();
       float p[kPrefillKeys];
-      tmem_ld128(t_lane + s_col, p);
+      if constexpr (R::kConvert) tmem_ld128_x32(t_lane + s_col, p);
+      else tmem_ld128(t_lane + s_col, p);
       // keys at or past this row's limit are -inf
       const int kbase = j * kPrefillKeys;
       if (kbase + kPrefillKeys > lim) {
@@ -559,7 +649,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float x0 = p[64 * half + 2 * i], x1 = p[64 * half + 2 * i + 1];
-          if constexpr (BF16) {
+          if constexpr (R::kPHiLo) {
             // hi = the top 16 bits of p (p truncated to bf16, remainder below
             // 2^-7 p), lo = the exact fp32 remainder p - hi >= 0 truncated the
             // same way: P keeps at least 14 significant bits (error < 2^-14 p),
@@ -577,7 +667,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
         }
         tmem_st32u(t_lane + s_col + 32 * half, h);
-        if constexpr (BF16) tmem_st32u(t_lane + s_col + 64 + 32 * half, lo);
+        if constexpr (R::kPHiLo) tmem_st32u(t_lane + s_col + 64 + 32 * half, lo);
       }
       l += ((lsum[0].x + lsum[0].y) + (lsum[1].x + lsum[1].y)) +
            ((lsum[2].x + lsum[2].y) + (lsum[3].x + lsum[3].y));
@@ -617,6 +707,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
     }
+  }
   }
 
   tmem_fence_before_sync();

@@ -15,17 +15,6 @@
 // live (the others see a zero token limit and stay unchanged).  The pages are
 // spread over the CTAs of a cluster and their warps exactly as in
 // paged_decode_kernel, and merged the same way.
-//
-// Split mode (pa_decode_shared_prefix_split) cuts every sequence into the
-// partitions of pa_decode_split and writes the same partials, which pa_reduce
-// merges.  Here a work item is (group, chunk, KV head, partition) for the
-// partitions that reach into the group's shared prefix: the shared pages the
-// partition covers, once, with every row live, then each member's own pages
-// inside the partition.  The partitions past the prefix are computed per
-// sequence by paged_decode_kernel in split mode, which skips these.  Items
-// then hold at most one partition of pages (plus the members' own pages where
-// a partition straddles the end of the prefix), so a batch of unequal groups
-// no longer waits on its largest item.
 #pragma once
 
 #include "pa_decode.cuh"
@@ -53,13 +42,6 @@ struct SharedPrefixArgs {
   int chunks_per_group;           // ceil(max_group_size / members_per_chunk)
   int cluster_pages;              // items with more pages are spread over the cluster
   int longest_first;              // order (group, chunk) slots by descending page count
-  // split mode (tmp_out != null): one grid item per (sequence, KV head,
-  // partition of partition_pages pages); partials as pa_decode_split writes them
-  float* tmp_out;                 // [S, H, max_partitions, D]
-  float* max_logits;              // [S, H, max_partitions]
-  float* exp_sums;                // [S, H, max_partitions]
-  int partition_pages;
-  int max_partitions;
 };
 
 template <int D, int NST, bool BF16>
@@ -80,19 +62,12 @@ __global__ void __launch_bounds__(kThreads)
   pdl_launch_dependents();
   pdl_wait();
 
-  // grid slot -> (group, chunk) and KV head; KV heads of one slot are adjacent.
-  // Split mode: grid slot -> (group, chunk, KV head, partition), partition fastest.
-  const bool split = a.tmp_out != nullptr;
-  int item = blockIdx.x / csize;
-  int part = 0;
-  if (split) {
-    part = item % a.max_partitions;
-    item /= a.max_partitions;
-  }
+  // grid slot -> (group, chunk) and KV head; KV heads of one slot are adjacent
+  const int item = blockIdx.x / csize;
   const int kvh = item % a.num_kv_heads;
   int slot = item / a.num_kv_heads;
   const int G = a.group;
-  if (!split && a.longest_first) {
+  if (a.longest_first) {
     // rank every (group, chunk) slot by its page count, longest first (ties
     // by index), and take the one whose rank is this grid slot
     const int U = a.num_groups * a.chunks_per_group;
@@ -144,22 +119,13 @@ __global__ void __launch_bounds__(kThreads)
   }
   const int first = s_begin + chunk * a.members_per_chunk;
   const int members = min(a.members_per_chunk, s_end - first);
+  if (members <= 0) return;
+  const int nrows = members * G;
   int P = a.prefix_blocks[grp];
   if (P < 0 || P > a.max_blocks_per_seq) {
     if (reporter) record_error(kErrGroup, grp);
     P = P < 0 ? 0 : a.max_blocks_per_seq;
   }
-  // the item's window of table entries [e0, e1): everything, or one partition
-  // (split mode: only partitions that reach into the prefix; the others are
-  // pa_decode_split's, per sequence)
-  int e0 = 0, e1 = a.max_blocks_per_seq;
-  if (split) {
-    e0 = part * a.partition_pages;
-    e1 = min(e0 + a.partition_pages, a.max_blocks_per_seq);
-    if (e0 >= P) return;
-  }
-  if (members <= 0) return;
-  const int nrows = members * G;
 
   // lane j < members describes member j: its sequence, context length, and
   // the pages of its private tail (table entries P .. P+tail-1)
@@ -179,10 +145,8 @@ __global__ void __launch_bounds__(kThreads)
   int most_ctx = my_ctx;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) most_ctx = max(most_ctx, __shfl_xor_sync(~0u, most_ctx, o));
-  // shared entries [e0, e0 + Pn) and member j's own entries [tail0, tail0 + tail_j)
-  const int Pn = max(0, min(min(P, most_pages), e1) - e0);  // shared pages anyone needs
-  const int tail0 = max(P, e0);
-  const int my_tail = lane < members ? max(0, min(my_pages, e1) - tail0) : 0;
+  const int Pn = min(P, most_pages);                 // prefix pages anyone needs
+  const int my_tail = lane < members ? max(0, my_pages - P) : 0;
   int incl = my_tail;                                // inclusive prefix sum of tails
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -192,8 +156,7 @@ __global__ void __launch_bounds__(kThreads)
   const int my_off = Pn + incl - my_tail;            // first virtual page of my tail
   const int n_pages = Pn + __shfl_sync(~0u, incl, 31);
 
-  if (n_pages == 0) {  // no member has a token in the window
-    if (split) return;   // no partial of this partition is ever read
+  if (n_pages == 0) {  // every member has an empty context
     if (crank == 0) {
       for (int i = threadIdx.x; i < nrows * D; i += kThreads) {
         const int r = i / D;
@@ -226,10 +189,10 @@ __global__ void __launch_bounds__(kThreads)
     }
     if (v < Pn) {
       member = -1;
-      entry = e0 + v;
+      entry = v;
     } else {
       member = owner;
-      entry = tail0 + (v - start);
+      entry = P + (v - start);
     }
   };
 
@@ -362,19 +325,10 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   merge_and_emit<D, NST>(smem, nrows, spread, ctas, crank,
-                         [&](int r, int d, float o0, float o1, float big_m, float big_l) {
+                         [&](int r, int d, float o0, float o1, float, float big_l) {
     const size_t hrow = static_cast<size_t>(first + r / G) * a.num_heads + kvh * G + r % G;
-    if (split) {
-      const size_t pidx = hrow * a.max_partitions + part;
-      *reinterpret_cast<float2*>(a.tmp_out + pidx * D + d) = make_float2(o0, o1);
-      if (d == 0) {
-        a.max_logits[pidx] = big_m * kLn2;
-        a.exp_sums[pidx] = big_l;
-      }
-    } else {
-      const float inv = big_l > 0.f ? 1.f / big_l : 0.f;
-      *reinterpret_cast<uint32_t*>(a.out + hrow * D + d) = pack2<BF16>(o0 * inv, o1 * inv);
-    }
+    const float inv = big_l > 0.f ? 1.f / big_l : 0.f;
+    *reinterpret_cast<uint32_t*>(a.out + hrow * D + d) = pack2<BF16>(o0 * inv, o1 * inv);
   });
 }
 

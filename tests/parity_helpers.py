@@ -54,19 +54,16 @@ def gpu_step(batch: workloads.DecodeBatch, write: bool = True, partition_size: i
              max_partitions: int | None = None, shared_prefix: bool = False,
              max_group_size: int | None = None):
     """The CUDA path: pa_reshape_and_cache, then pa_decode, pa_decode_split +
-    pa_reduce, pa_decode_shared_prefix, or (shared_prefix with a partition
-    size) pa_decode_shared_prefix_split + pa_reduce.  Returns (out, partials
-    or None)."""
+    pa_reduce, or pa_decode_shared_prefix.  Returns (out, partials or None)."""
     from paged_kv_cache_444_b200 import (SplitWorkspace, pa_decode, pa_decode_shared_prefix,
-                                         pa_decode_shared_prefix_split, pa_decode_split,
-                                         pa_reduce, pa_reshape_and_cache)
+                                         pa_decode_split, pa_reduce, pa_reshape_and_cache)
     cfg = batch.cfg
     if write:
         pa_reshape_and_cache(batch.key, batch.value, batch.key_cache, batch.value_cache,
                              batch.slot_mapping)
     out = torch.full_like(batch.query, float("nan"))
     parts = None
-    if shared_prefix and not partition_size:
+    if shared_prefix:
         sizes = (batch.group_starts[1:] - batch.group_starts[:-1]).tolist()
         pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
                                 batch.block_tables, batch.context_lens, batch.group_starts,
@@ -78,17 +75,9 @@ def gpu_step(batch: workloads.DecodeBatch, write: bool = True, partition_size: i
         ws.tmp_out.fill_(float("nan"))
         ws.max_logits.fill_(float("nan"))
         ws.exp_sums.fill_(float("nan"))
-        if shared_prefix:
-            sizes = (batch.group_starts[1:] - batch.group_starts[:-1]).tolist()
-            pa_decode_shared_prefix_split(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query,
-                                          batch.key_cache, batch.value_cache,
-                                          batch.block_tables, batch.context_lens,
-                                          batch.group_starts, batch.prefix_blocks, cfg.scale,
-                                          max_group_size or max(sizes), partition_size)
-        else:
-            pa_decode_split(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query,
-                            batch.key_cache, batch.value_cache, batch.block_tables,
-                            batch.context_lens, cfg.scale, partition_size)
+        pa_decode_split(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query,
+                        batch.key_cache, batch.value_cache, batch.block_tables,
+                        batch.context_lens, cfg.scale, partition_size)
         pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, batch.context_lens,
                   partition_size)
         parts = ws

@@ -160,30 +160,6 @@ def test_shared_prefix_validation(lib):
 
 
 @host_only
-def test_shared_prefix_split_validation(lib):
-    f = lib.pa_decode_shared_prefix_split
-    base = [FAKE] * 10 + [0.1, 8]           # partials .. prefix_blocks, scale, num_seqs
-    sizes = [2, 4, 8, 2, 128, 64, 16, 8]    # groups, max size, H, Hk, D, NB, bs, MB
-
-    def call(b=base, sz=sizes, ps=64, P=2):
-        return f(*b, *sz, ps, P, 0, None)
-    assert call(ps=0) == SHAPE                                    # partition size
-    assert call(ps=24) == UNSUP                                   # not a multiple of 16
-    assert call(P=0) == SHAPE                                     # max_partitions
-    assert call(sz=[2, 0] + sizes[2:]) == SHAPE                   # max_group_size 0
-    assert call(sz=[0] + sizes[1:]) == OK                         # no groups: nothing to do
-    b = list(base)
-    b[0] = None
-    assert call(b) == NULL                                        # tmp_out
-    b = list(base)
-    b[8] = None
-    assert call(b) == NULL                                        # group_starts
-    b = list(base)
-    b[1] = FAKE + 2
-    assert call(b) == ALIGN                                       # max_logits
-
-
-@host_only
 def test_copy_blocks_validation(lib):
     f = lib.pa_copy_blocks
     assert f(FAKE, FAKE, FAKE, 0, 64, 16, 2, 128, 2, None) == OK        # no pairs

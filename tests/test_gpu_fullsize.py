@@ -16,9 +16,8 @@ import torch
 
 import oracle as oracle_mod
 from paged_kv_cache_444_b200 import (SplitWorkspace, decode_step, pa_check_error, pa_decode_fp8,
-                                     pa_decode_shared_prefix, pa_decode_shared_prefix_split,
-                                     pa_decode_split_fp8, pa_reduce, pa_reshape_and_cache,
-                                     workloads)
+                                     pa_decode_shared_prefix, pa_decode_split_fp8, pa_reduce,
+                                     pa_reshape_and_cache, workloads)
 from parity_helpers import TOL, bits, ocode, report_parity, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -109,10 +108,8 @@ def test_full_size_workload(name, cuda_device, oracle_lib):
     assert torch.equal(flat_before, flat_after)
 
 
-@pytest.mark.parametrize("partition_size", [0, 512], ids=["single_pass", "split512"])
-def test_full_size_shared_prefix_beam(partition_size, cuda_device, oracle_lib):
-    """pa_decode_shared_prefix (and pa_decode_shared_prefix_split + pa_reduce
-    with 512-token partitions) on the full beam batch (64 sequences in groups
+def test_full_size_shared_prefix_beam(cuda_device, oracle_lib):
+    """pa_decode_shared_prefix on the full beam batch (64 sequences in groups
     of 4 sharing 32 blocks), with the group arrays and max group size the
     benchmark passes, after the step's cache write."""
     cfg = workloads.CONFIGS["shared_prefix_beam"]
@@ -124,21 +121,10 @@ def test_full_size_shared_prefix_beam(partition_size, cuda_device, oracle_lib):
                          batch.slot_mapping)
     sizes = (batch.group_starts[1:] - batch.group_starts[:-1]).tolist()
     out = torch.full_like(batch.query, float("nan"))
-    if partition_size:
-        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, batch.max_partitions,
-                            cuda_device)
-        pa_decode_shared_prefix_split(ws.tmp_out, ws.max_logits, ws.exp_sums, batch.query,
-                                      batch.key_cache, batch.value_cache, batch.block_tables,
-                                      batch.context_lens, batch.group_starts,
-                                      batch.prefix_blocks, cfg.scale, max(sizes), partition_size)
-        pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, batch.context_lens,
-                  partition_size)
-        kernel = "pa_decode_shared_prefix_split+pa_reduce"
-    else:
-        pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
-                                batch.block_tables, batch.context_lens, batch.group_starts,
-                                batch.prefix_blocks, cfg.scale, max(sizes))
-        kernel = "pa_decode_shared_prefix"
+    pa_decode_shared_prefix(out, batch.query, batch.key_cache, batch.value_cache,
+                            batch.block_tables, batch.context_lens, batch.group_starts,
+                            batch.prefix_blocks, cfg.scale, max(sizes))
+    kernel = "pa_decode_shared_prefix"
     torch.cuda.synchronize()
     pa_check_error()
     ref, _, _ = _oracle_written(oracle_lib, cfg, snap)

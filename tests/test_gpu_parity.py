@@ -90,14 +90,12 @@ def test_split_matches_oracle(name, ps, dev, oracle_lib):
     out, ws = gpu_step(batch, partition_size=ps)
     pa_check_error()
     _check_close(out, ref, cfg, f"{name} split {ps}")
-    _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, ps, exact_coverage=True)
+    _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, ps)
 
 
-def _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, ps, exact_coverage):
+def _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, ps):
     """The partial statistics of a split launch against the oracle's
-    partitions.  Every partition p < ceil(ctx/P) must be written; with
-    exact_coverage no other entry may be, else the others may only hold an
-    empty partial (max -inf, sum 0), which the merge never reads."""
+    partitions: exactly the partitions p < ceil(ctx/P) are written."""
     P = ws.max_partitions
     acc, pmax, psum = oracle_lib.decode_partitioned(host.query, kc_ref, vc_ref,
                                                     host.block_tables, host.context_lens,
@@ -107,12 +105,7 @@ def _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, ps, exact_coverag
     gs = ws.exp_sums.cpu().numpy().astype(np.float64)
     ga = ws.tmp_out.cpu().numpy().astype(np.float64)
     valid = ~np.isnan(pmax)
-    if exact_coverage:
-        assert np.array_equal(valid, ~np.isnan(gm)), "partitions written differ from ceil(ctx/P)"
-    else:
-        assert not np.isnan(gm[valid]).any(), "a partition p < ceil(ctx/P) was not written"
-        extra = ~valid & ~np.isnan(gm)
-        assert (gm[extra] == -np.inf).all() and (gs[extra] == 0).all()
+    assert np.array_equal(valid, ~np.isnan(gm)), "partitions written differ from ceil(ctx/P)"
     assert np.max(np.abs(gm[valid] - pmax[valid])) <= 1e-4
     rel = np.abs(gs[valid] - psum[valid]) / psum[valid]
     assert np.max(rel) <= 1e-2
@@ -246,8 +239,7 @@ def test_many_sequences_natural_order(dev, oracle_lib):
 
 NAN_CASES = [(n, m) for n in ("mha_small", "gqa_small", "gqa16_two_rows", "d64_gqa2",
                               "shared_small") for m in ("single", "split64")]
-NAN_CASES += [("shared_small", "shared"),      # the shared-prefix kernels need their groups
-              ("shared_small", "shared_split64")]
+NAN_CASES.append(("shared_small", "shared"))   # the shared-prefix kernel needs its groups
 
 
 @pytest.mark.parametrize("name,mode", NAN_CASES)
@@ -259,8 +251,8 @@ def test_nan_rows_past_context_do_not_leak(name, mode, dev, oracle_lib):
     assert poison_past_context(batch) > 0
     host = HostCopy(batch)
     ref, _, _ = oracle_step(oracle_lib, host)
-    out, _ = gpu_step(batch, partition_size=64 if mode.endswith("split64") else 0,
-                      shared_prefix=mode.startswith("shared"))
+    out, _ = gpu_step(batch, partition_size=64 if mode == "split64" else 0,
+                      shared_prefix=mode == "shared")
     pa_check_error()
     _check_close(out, ref, cfg, f"{name} {mode} with NaN past the context")
 
@@ -319,25 +311,6 @@ def test_shared_prefix_matches_oracle(name, dev, oracle_lib):
     _check_close(out, ref, cfg, f"shared prefix {name}")
     plain, _ = gpu_step(batch, write=False)
     assert np.max(np.abs(to_f64(plain) - to_f64(out))) <= TOL[cfg.dtype]
-
-
-@pytest.mark.parametrize("ps", [16, 64, 512])
-@pytest.mark.parametrize("name", list(SHARED_CASES))
-def test_shared_prefix_split_matches_oracle(name, ps, dev, oracle_lib):
-    """pa_decode_shared_prefix_split + pa_reduce: the merged output and every
-    partial against the oracle, for partitions smaller than, equal to and
-    larger than the shared prefixes (so partitions straddle a prefix's end)."""
-    base, over, starts, prefix = SHARED_CASES[name]
-    cfg = SMALL[base].scaled(**over) if over else SMALL[base]
-    batch = workloads.make_batch(cfg, dev)
-    if starts is not None:
-        batch = _regroup(batch, starts, prefix)
-    host = HostCopy(batch)
-    ref, kc_ref, vc_ref = oracle_step(oracle_lib, host)
-    out, ws = gpu_step(batch, shared_prefix=True, partition_size=ps)
-    pa_check_error()
-    _check_close(out, ref, cfg, f"shared prefix split {name} ps={ps}")
-    _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, ps, exact_coverage=False)
 
 
 def test_shared_prefix_reports_bad_groups(dev):

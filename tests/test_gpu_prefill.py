@@ -157,6 +157,36 @@ def test_prefill_reports_query_longer_than_context(cuda_device):
     assert e.value.detail >> 56 == 7 and e.value.detail & 0xffff == 1
 
 
+def test_prefill_bf16_reports_v_beyond_fp16_range(cuda_device, oracle_lib):
+    """bf16 V blocks are rewritten as fp16 in shared memory for the P V
+    product; a V value beyond the fp16 range saturates to +-65504 and is
+    reported with its sequence (PA_CHECK_VALUE).  The other sequences'
+    outputs still match the oracle."""
+    cfg, b, query, starts, qlens = _case("gqa4_bf16", cuda_device)
+    s_bad = 2
+    blk = int(b.block_tables[s_bad, 3])
+    b.value_cache[blk, 5, 1, 17] = 1.0e5                     # in context (ctx 300)
+    kc = bits(b.key_cache).copy()
+    vc = bits(b.value_cache).copy()
+    assert oracle_lib.reshape_and_cache(bits(b.key), bits(b.value), kc, vc,
+                                        b.slot_mapping.cpu().numpy(), cfg.num_blocks,
+                                        cfg.block_size) == 0
+    ref = oracle_lib.prefill(bits(query), kc, vc, b.block_tables.cpu().numpy(),
+                             b.context_lens.cpu().numpy(), starts.cpu().numpy(), cfg.scale,
+                             ocode(cfg))
+    pa_reshape_and_cache(b.key, b.value, b.key_cache, b.value_cache, b.slot_mapping)
+    out = torch.full_like(query, float("nan"))
+    pa_prefill(out, query, b.key_cache, b.value_cache, b.block_tables, b.context_lens, starts,
+               cfg.scale, max(qlens))
+    with pytest.raises(PagedAttentionError) as e:
+        pa_check_error()
+    assert e.value.detail >> 56 == 8 and e.value.detail & 0xffff == s_bad
+    st = starts.cpu().tolist()
+    keep = [t for i in range(len(qlens)) if i != s_bad for t in range(st[i], st[i + 1])]
+    g = to_f64(out)
+    assert np.max(np.abs(g[keep] - ref[keep])) <= TOL[cfg.dtype]
+
+
 def test_prefill_reports_invalid_sequence_in_fixed_order(cuda_device):
     """Past 256 sequences the units go out in the fixed order; an invalid
     sequence is still skipped and reported, and the others are written."""
