@@ -91,18 +91,41 @@ MUTATIONS = [
 ]
 
 
-@pytest.mark.parametrize("what,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
-def test_pins_catch_planted_mistake(what, old, new, tmp_path: Path):
+def _plant_and_run(what, old, new, workdir: Path):
+    """Compile the oracle with one planted mistake and run the pin suite on it
+    in a child process; returns (returncode, stdout)."""
     src = oracle_mod.SOURCE.read_text(encoding="utf-8")
-    assert old in src, f"mutation anchor no longer in the oracle source: {old!r}"
-    mutant_src = tmp_path / "pa_oracle_mutant.c"
+    if old not in src:
+        return None, f"mutation anchor no longer in the oracle source: {old!r}"
+    workdir.mkdir(parents=True, exist_ok=True)
+    mutant_src = workdir / "pa_oracle_mutant.c"
     mutant_src.write_text(src.replace(old, new), encoding="utf-8")
-    lib = oracle_mod.compile_oracle(mutant_src, tmp_path / "libmutant.so")
+    lib = oracle_mod.compile_oracle(mutant_src, workdir / "libmutant.so")
     code = _RUNNER.format(tests=str(TESTS_DIR), root=str(ROOT), lib=str(lib))
     proc = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
                           timeout=600)
-    if proc.returncode != 0:
+    return proc.returncode, proc.stdout
+
+
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    """Every planted copy built and run at once, one worker per CPU (each is
+    a gcc build and a child process, independent of the others)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    base = tmp_path_factory.mktemp("mutants")
+    with ThreadPoolExecutor(max_workers=max(1, os.cpu_count() or 1)) as pool:
+        futures = {what: pool.submit(_plant_and_run, what, old, new, base / f"m{i}")
+                   for i, (what, old, new) in enumerate(MUTATIONS)}
+        return {what: f.result() for what, f in futures.items()}
+
+
+@pytest.mark.parametrize("what", [m[0] for m in MUTATIONS])
+def test_pins_catch_planted_mistake(what, mutant_results):
+    returncode, out = mutant_results[what]
+    assert returncode is not None, out
+    if returncode != 0:
         return  # the planted mistake crashed the pin suite: caught
-    line = [ln for ln in proc.stdout.splitlines() if ln.startswith("CAUGHT")][-1]
+    line = [ln for ln in out.splitlines() if ln.startswith("CAUGHT")][-1]
     caught = [c for c in line[len("CAUGHT"):].strip().split(",") if c]
     assert caught, f"no pin caught the planted mistake: {what}"
