@@ -130,6 +130,9 @@ pa_status launch_ex(K kernel, unsigned grid, unsigned block, size_t smem, cudaSt
 template <int D>
 struct Stages { static constexpr int value = D == 64 ? PA_STAGES_D64 : PA_STAGES_D128; };
 
+#ifndef PA_SPLIT_PERSISTENT
+#define PA_SPLIT_PERSISTENT 1  // split launches: one wave of CTAs over the items that exist
+#endif
 #ifndef PA_CLUSTER_PAGES
 #define PA_CLUSTER_PAGES 256  // an item with more pages is spread over its cluster
 #endif
@@ -178,16 +181,50 @@ int pick_cluster(K kernel, int smem_bytes, int64_t max_pages, std::atomic<int>* 
   return want < known ? want : known;
 }
 
+// CTAs of `kernel` that fit on the device at once (SMs x resident CTAs per SM),
+// looked up once per device; 0 if the query fails.
+template <class K>
+long long resident_ctas(K kernel, int smem_bytes, std::atomic<long long>* cache) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  long long known = cache[dev].load(std::memory_order_relaxed);
+  if (known == 0) {
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem_bytes) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    known = static_cast<long long>(per_sm) * sms;
+    cache[dev].store(known, std::memory_order_relaxed);
+  }
+  return known;
+}
+
 template <int D, bool BF16, class Warp, int EB = 2>
 pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeArgs a,
                           long long grid, int64_t max_pages, cudaStream_t stream) {
   constexpr int NST = EB == 1 ? PA_STAGES_FP8 : Stages<D>::value;
   using L = DecodeSmem<D, NST, EB>;
-  auto kernel = paged_decode_kernel<D, NST, BF16, Warp, EB>;
-  static std::atomic<uint64_t> done{0};
+  auto kernel = paged_decode_kernel<D, NST, BF16, Warp, EB, false>;
+  auto kernel_persist = paged_decode_kernel<D, NST, BF16, Warp, EB, true>;
+  static std::atomic<uint64_t> done{0}, done_persist{0};
   static std::atomic<int> cluster_cache[kMaxDevices] = {};
-  if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
+  static std::atomic<long long> resident_cache[kMaxDevices] = {};
   const bool split = a.tmp_out != nullptr;
+  if (split && a.persistent) {
+    // one wave of CTAs loops over the items that exist (at most `grid`)
+    if (!ensure_smem(kernel_persist, L::kAlloc, &done_persist)) return PA_ERR_CUDA;
+    const long long resident = resident_ctas(kernel_persist, L::kAlloc, resident_cache);
+    if (resident > 0) {
+      if (grid > resident) grid = resident;
+      return launch_ex(kernel_persist, static_cast<unsigned>(grid), kThreads, L::kAlloc, stream,
+                       1, km, vm, a);
+    }
+    a.persistent = 0;
+  }
+  if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
   const int c = split ? 1 : pick_cluster(kernel, L::kAlloc, max_pages, cluster_cache);
   a.cluster_pages = PA_CLUSTER_PAGES;
   if (grid * c > INT32_MAX) return PA_ERR_SHAPE;
@@ -242,6 +279,9 @@ pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cach
     return PA_ERR_CUDA;
   const long long grid = num_seqs * a.num_kv_heads * static_cast<long long>(a.parts_per_head);
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
+  // split mode, up to kLptMaxSeqs sequences: persistent CTAs over a dense item list
+  a.num_seqs = static_cast<int>(num_seqs);
+  a.persistent = PA_SPLIT_PERSISTENT && a.tmp_out != nullptr && num_seqs <= kLptMaxSeqs;
   const bool bf16 = dtype == PA_BF16;
   const int64_t max_pages = a.max_blocks_per_seq;  // block_size == 16 == one page
   if (head_dim == 64)
@@ -262,6 +302,8 @@ pa_status run_decode_fp8(DecodeArgs a, const void* key_cache, const void* value_
     return PA_ERR_CUDA;
   const long long grid = num_seqs * a.num_kv_heads * static_cast<long long>(a.parts_per_head);
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
+  a.num_seqs = static_cast<int>(num_seqs);
+  a.persistent = PA_SPLIT_PERSISTENT && a.tmp_out != nullptr && num_seqs <= kLptMaxSeqs;
   const int64_t max_pages = a.max_blocks_per_seq;
   if (dtype == PA_BF16) {
     if (a.group <= 8)

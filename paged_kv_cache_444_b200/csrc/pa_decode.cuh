@@ -64,6 +64,7 @@ struct DecodeArgs {
   int cluster_pages;          // an item with more pages than this is spread over its cluster
   int num_seqs;
   int longest_first;          // order single-pass items by descending context length
+  int persistent;             // split mode: CTAs loop over a dense list of the items that exist
 };
 
 
@@ -78,7 +79,11 @@ struct DecodeSmem {
   static constexpr int kRedLOffset = kRedMOffset + kWarps * 16 * 4;
   static constexpr int kPartMOffset = kRedLOffset + kWarps * 16 * 4;
   static constexpr int kPartLOffset = kPartMOffset + 16 * 4;
-  static constexpr int kBytes = kPartLOffset + 16 * 4;
+  // persistent split mode: every sequence's context length and the running
+  // count of partitions before it (outside the stage area: kept across items)
+  static constexpr int kCtxOffset = kPartLOffset + 16 * 4;
+  static constexpr int kCumOffset = kCtxOffset + kLptMaxSeqs * 4;
+  static constexpr int kBytes = kCumOffset + (kLptMaxSeqs + 1) * 4;
   static constexpr int kAlloc = kBytes + 1024;            // + alignment slack
   // the merge buffers reuse the stage area: per-warp rows (kWarps x group x D
   // floats) and, for an item spread over a cluster, this CTA's merged rows
@@ -389,87 +394,40 @@ __device__ __forceinline__ bool drain_stages(bool ok, int k_stop, int n_pages, u
 // takes the same branch and either all of them reach both cluster barriers
 // or none does.
 // ---------------------------------------------------------------------------
-template <int D, int NST, bool BF16, class Warp, int EB = 2>
-__global__ void __launch_bounds__(kThreads)
-    paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
-                        const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
+// ---------------------------------------------------------------------------
+// One (sequence, KV head, partition) item, whole CTA (and, spread, whole
+// cluster): the page loop of every warp, the merge, the output or partials.
+// ctx is the sequence's validated context length.  Returns false when a TMA
+// load never landed after a wait gave up (the stage area is then left alone
+// and the CTA must end).
+// ---------------------------------------------------------------------------
+template <int D, int NST, bool BF16, class Warp, int EB>
+__device__ __forceinline__ bool decode_item(const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                            const DecodeArgs& a, uint8_t* smem, int s, int kvh,
+                                            int part, int ctx, int csize, int crank) {
   using L = DecodeSmem<D, NST, EB>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int csize = static_cast<int>(cluster_nctarank());
-  const int crank = static_cast<int>(cluster_ctarank());
-  prefetch_tensormap(&kmap);
-  prefetch_tensormap(&vmap);
-  pdl_launch_dependents();
-  pdl_wait();  // inputs may come from the previous kernel of the stream
-
-  int item = blockIdx.x / csize;
-  const int part = item % a.parts_per_head;
-  item /= a.parts_per_head;
-  const int kvh = item % a.num_kv_heads;
-  int s = item / a.num_kv_heads;
+  // ---- this item's token range ----
   const int group = a.group;
   const bool split = a.tmp_out != nullptr;
-  const bool reporter = threadIdx.x == 0 && crank == 0 && part == 0 && kvh == 0;
-
-  // ---- longest-first order: grid slot s takes the s-th longest sequence
-  // (ties by index), so that long items start first and short ones fill the
-  // tail.  The rank of every sequence is counted against all others. ----
-  if (a.longest_first) {
-    int* lens = reinterpret_cast<int*>(smem);      // stage area, not in use yet
-    int* chosen = lens + kLptMaxSeqs;
-    const int n4 = (a.num_seqs + 3) >> 2;
-    for (int i = threadIdx.x; i < n4 * 4; i += kThreads)
-      lens[i] = i < a.num_seqs ? max(a.context_lens[i], 0) : -1;  // -1 pads: never counted
-    __syncthreads();
-    const int4* lens4 = reinterpret_cast<const int4*>(lens);
-    for (int t = threadIdx.x; t < a.num_seqs; t += kThreads) {
-      const int lt = lens[t];
-      int rank = 0;
-      for (int j4 = 0; j4 < n4; ++j4) {
-        const int4 v = lens4[j4];
-        const int j = j4 * 4;
-        rank += (v.x > lt) | ((v.x == lt) & (j < t));
-        rank += (v.y > lt) | ((v.y == lt) & (j + 1 < t));
-        rank += (v.z > lt) | ((v.z == lt) & (j + 2 < t));
-        rank += (v.w > lt) | ((v.w == lt) & (j + 3 < t));
-      }
-      if (rank == s) *chosen = t;
-    }
-    __syncthreads();
-    s = *chosen;
-    __syncthreads();  // the stage area is about to be reused
-  }
-
-  // ---- context length and this item's token range ----
-  int ctx = a.context_lens[s];
-  const int cap = a.max_blocks_per_seq * kPage;
-  if (ctx < 0 || ctx > cap) {
-    if (reporter) record_error(kErrContextLen, s);
-    ctx = ctx < 0 ? 0 : cap;
-  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int t_begin = 0, t_end = ctx;
   if (split) {
-    if (reporter && (ctx + a.partition_size - 1) / a.partition_size > a.max_partitions)
-      record_error(kErrPartitions, s);
     t_begin = part * a.partition_size;
     t_end = min(t_begin + a.partition_size, ctx);
-    if (t_begin >= t_end) return;  // partition past the end: nothing to write
+    if (t_begin >= t_end) return true;  // partition past the end: nothing to write
   } else if (ctx == 0) {
     // empty sequence: zero output rows
     if (crank == 0) {
       uint16_t* o = a.out + (static_cast<size_t>(s) * a.num_heads + kvh * group) * D;
       for (int i = threadIdx.x; i < group * D; i += kThreads) o[i] = 0;
     }
-    return;
+    return true;
   }
 
   const int first_page = t_begin / kPage;
   const int n_pages = (t_end - first_page * kPage + kPage - 1) / kPage;
   const bool spread = csize > 1 && n_pages > a.cluster_pages;
-  if (csize > 1 && !spread && crank != 0) return;  // short item: CTA 0 alone
+  if (csize > 1 && !spread && crank != 0) return true;  // short item: CTA 0 alone
   const int ctas = spread ? csize : 1;             // CTAs sharing this item
   const int page0 = (spread ? crank : 0) + ctas * warp;  // this warp's first page
   const int pstride = ctas * kWarps;                      // and its page stride
@@ -564,7 +522,7 @@ __global__ void __launch_bounds__(kThreads)
       cluster_sync();
       cluster_sync();
     }
-    return;
+    return false;
   }
   float* red_acc = reinterpret_cast<float*>(smem);
   float* red_m = reinterpret_cast<float*>(smem + L::kRedMOffset);
@@ -597,6 +555,116 @@ __global__ void __launch_bounds__(kThreads)
       *reinterpret_cast<uint32_t*>(a.out + hrow * D + d) = pack2<BF16>(o0 * inv, o1 * inv);
     }
   });
+  return true;
+}
+
+template <int D, int NST, bool BF16, class Warp, int EB = 2, bool PERSIST = false>
+__global__ void __launch_bounds__(kThreads)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                        const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
+  using L = DecodeSmem<D, NST, EB>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int csize = static_cast<int>(cluster_nctarank());
+  const int crank = static_cast<int>(cluster_ctarank());
+  prefetch_tensormap(&kmap);
+  prefetch_tensormap(&vmap);
+  pdl_launch_dependents();
+  pdl_wait();  // inputs may come from the previous kernel of the stream
+
+  int item = blockIdx.x / csize;
+  const int part = item % a.parts_per_head;
+  item /= a.parts_per_head;
+  const int kvh = item % a.num_kv_heads;
+  int s = item / a.num_kv_heads;
+  const bool split = a.tmp_out != nullptr;
+  const bool reporter = threadIdx.x == 0 && crank == 0 && part == 0 && kvh == 0;
+  const int cap = a.max_blocks_per_seq * kPage;
+
+  // ---- persistent split mode: the items that exist (partition p of
+  // sequence s for p < ceil(ctx_s / partition_size), every KV head), in a
+  // dense order that every CTA derives from the context lengths; CTA b takes
+  // items b, b + gridDim.x, ...  No CTA is launched for a partition past its
+  // sequence's end. ----
+  if constexpr (PERSIST) {
+    int* ctxs = reinterpret_cast<int*>(smem + L::kCtxOffset);
+    int* cum = reinterpret_cast<int*>(smem + L::kCumOffset);
+    for (int i = threadIdx.x; i < a.num_seqs; i += kThreads) {
+      int c = a.context_lens[i];
+      if (c < 0 || c > cap) {
+        if (blockIdx.x == 0) record_error(kErrContextLen, i);
+        c = c < 0 ? 0 : cap;
+      }
+      int np = (c + a.partition_size - 1) / a.partition_size;
+      if (np > a.max_partitions) {
+        if (blockIdx.x == 0) record_error(kErrPartitions, i);
+        np = a.max_partitions;
+      }
+      ctxs[i] = c;
+      cum[i + 1] = np;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {  // running count (at most kLptMaxSeqs sequences)
+      int acc = 0;
+      cum[0] = 0;
+      for (int i = 0; i < a.num_seqs; ++i) cum[i + 1] = (acc += cum[i + 1]);
+    }
+    __syncthreads();
+    const int items = cum[a.num_seqs] * a.num_kv_heads;
+    for (int u = blockIdx.x; u < items; u += gridDim.x) {
+      const int kv = u % a.num_kv_heads, su = u / a.num_kv_heads;
+      int lo = 0, hi = a.num_seqs;  // the sequence with cum[s] <= su < cum[s + 1]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (cum[mid] <= su) lo = mid; else hi = mid;
+      }
+      if (!decode_item<D, NST, BF16, Warp, EB>(kmap, vmap, a, smem, lo, kv, su - cum[lo],
+                                               ctxs[lo], 1, 0))
+        return;
+      __syncthreads();  // the merge buffers (stage area) are free for the next item
+    }
+    return;
+  }
+
+  // ---- longest-first order: grid slot s takes the s-th longest sequence
+  // (ties by index), so that long items start first and short ones fill the
+  // tail.  The rank of every sequence is counted against all others. ----
+  if (a.longest_first) {
+    int* lens = reinterpret_cast<int*>(smem);      // stage area, not in use yet
+    int* chosen = lens + kLptMaxSeqs;
+    const int n4 = (a.num_seqs + 3) >> 2;
+    for (int i = threadIdx.x; i < n4 * 4; i += kThreads)
+      lens[i] = i < a.num_seqs ? max(a.context_lens[i], 0) : -1;  // -1 pads: never counted
+    __syncthreads();
+    const int4* lens4 = reinterpret_cast<const int4*>(lens);
+    for (int t = threadIdx.x; t < a.num_seqs; t += kThreads) {
+      const int lt = lens[t];
+      int rank = 0;
+      for (int j4 = 0; j4 < n4; ++j4) {
+        const int4 v = lens4[j4];
+        const int j = j4 * 4;
+        rank += (v.x > lt) | ((v.x == lt) & (j < t));
+        rank += (v.y > lt) | ((v.y == lt) & (j + 1 < t));
+        rank += (v.z > lt) | ((v.z == lt) & (j + 2 < t));
+        rank += (v.w > lt) | ((v.w == lt) & (j + 3 < t));
+      }
+      if (rank == s) *chosen = t;
+    }
+    __syncthreads();
+    s = *chosen;
+    __syncthreads();  // the stage area is about to be reused
+  }
+
+  // ---- context length ----
+  int ctx = a.context_lens[s];
+  if (ctx < 0 || ctx > cap) {
+    if (reporter) record_error(kErrContextLen, s);
+    ctx = ctx < 0 ? 0 : cap;
+  }
+  if (split && reporter && (ctx + a.partition_size - 1) / a.partition_size > a.max_partitions)
+    record_error(kErrPartitions, s);
+  decode_item<D, NST, BF16, Warp, EB>(kmap, vmap, a, smem, s, kvh, part, ctx, csize, crank);
 }
 
 }  // namespace pa
