@@ -207,8 +207,8 @@ pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeAr
                           long long grid, int64_t max_pages, cudaStream_t stream) {
   constexpr int NST = EB == 1 ? PA_STAGES_FP8 : Stages<D>::value;
   using L = DecodeSmem<D, NST, EB>;
-  auto kernel = paged_decode_kernel<D, NST, BF16, Warp, EB, false>;
-  auto kernel_persist = paged_decode_kernel<D, NST, BF16, Warp, EB, true>;
+  auto kernel = paged_decode_kernel<D, NST, BF16, Warp, EB>;
+  auto kernel_persist = paged_decode_persistent_kernel<D, NST, BF16, Warp, EB>;
   static std::atomic<uint64_t> done{0}, done_persist{0};
   static std::atomic<int> cluster_cache[kMaxDevices] = {};
   static std::atomic<long long> resident_cache[kMaxDevices] = {};

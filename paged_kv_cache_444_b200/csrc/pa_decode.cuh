@@ -371,12 +371,14 @@ __device__ __forceinline__ void merge_and_emit(uint8_t* smem, int nrows, bool sp
 // for with the bounded wait.  Whole warp.
 // ---------------------------------------------------------------------------
 template <int NST>
-__device__ __forceinline__ bool drain_stages(bool ok, int k_stop, int n_pages, uint32_t bar0) {
+__device__ __forceinline__ bool drain_stages(bool ok, int k_stop, int n_pages, uint32_t bar0,
+                                             int kbase = 0) {
   if (ok) return true;
   bool landed = true;
   const int k_end = min(k_stop + NST, n_pages);
   for (int k = k_stop; k < k_end; ++k)
-    landed &= __all_sync(~0u, mbar_wait_bounded(bar0 + (k % NST) * 8, (k / NST) & 1));
+    landed &= __all_sync(~0u, mbar_wait_bounded(bar0 + ((kbase + k) % NST) * 8,
+                                                 ((kbase + k) / NST) & 1));
   return landed;
 }
 
@@ -395,16 +397,33 @@ __device__ __forceinline__ bool drain_stages(bool ok, int k_stop, int n_pages, u
 // or none does.
 // ---------------------------------------------------------------------------
 // ---------------------------------------------------------------------------
+// Each warp's ring of NST stages, one mbarrier per stage.  The barriers are
+// initialised once per CTA; a CTA that takes several items carries each
+// warp's count of pages through the ring (kbase) from item to item, so that
+// page k of an item uses stage (kbase + k) % NST with phase parity
+// ((kbase + k) / NST) & 1.  Whole warp.
+// ---------------------------------------------------------------------------
+template <int NST>
+__device__ __forceinline__ void init_ring(uint32_t bar0, int lane) {
+  if (lane == 0) {
+    for (int i = 0; i < NST; ++i) mbar_init(bar0 + i * 8, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
 // One (sequence, KV head, partition) item, whole CTA (and, spread, whole
 // cluster): the page loop of every warp, the merge, the output or partials.
-// ctx is the sequence's validated context length.  Returns false when a TMA
-// load never landed after a wait gave up (the stage area is then left alone
-// and the CTA must end).
+// ctx is the sequence's validated context length; the warps' rings are
+// initialised and kbase (per warp) counts the pages they already took.
+// Returns false when a wait gave up on this item (after draining what it
+// can): the ring's count is then no longer known, and the CTA must end.
 // ---------------------------------------------------------------------------
 template <int D, int NST, bool BF16, class Warp, int EB>
 __device__ __forceinline__ bool decode_item(const CUtensorMap& kmap, const CUtensorMap& vmap,
                                             const DecodeArgs& a, uint8_t* smem, int s, int kvh,
-                                            int part, int ctx, int csize, int crank) {
+                                            int part, int ctx, int csize, int crank, int& kbase) {
   using L = DecodeSmem<D, NST, EB>;
   // ---- this item's token range ----
   const int group = a.group;
@@ -437,12 +456,6 @@ __device__ __forceinline__ bool decode_item(const CUtensorMap& kmap, const CUten
   const uint32_t stage0 = smem_addr(smem) + warp * NST * L::kStageBytes;
   const uint32_t bar0 = smem_addr(smem + L::kBarOffset) + warp * NST * 8;
 
-  if (lane == 0) {
-    for (int i = 0; i < NST; ++i) mbar_init(bar0 + i * 8, 1);
-    fence_barrier_init();
-  }
-  __syncwarp();
-
   // ---- block ids: lane j holds the id of this warp's page (win*32 + j) ----
   const size_t row_base = static_cast<size_t>(s) * a.max_blocks_per_seq + first_page;
   auto load_ids = [&](int win) -> int {
@@ -464,7 +477,7 @@ __device__ __forceinline__ bool decode_item(const CUtensorMap& kmap, const CUten
     const int src = ((k >> 5) == win) ? ids_cur : ids_next;
     const int id = __shfl_sync(0xffffffffu, src, k & 31);
     if (lane == 0) {
-      const int st = k % NST;
+      const int st = (kbase + k) % NST;
       const uint32_t bar = bar0 + st * 8;
       const uint32_t dk = stage0 + st * L::kStageBytes;
       const uint32_t dv = dk + L::kPageBytes;
@@ -497,9 +510,9 @@ __device__ __forceinline__ bool decode_item(const CUtensorMap& kmap, const CUten
       ids_cur = ids_next;
       ids_next = my_pages > (win + 1) * 32 ? load_ids(win + 1) : -1;
     }
-    const int stg = k % NST;
+    const int stg = (kbase + k) % NST;
     // the whole warp takes the same branch, whatever each lane's wait saw
-    if (!__all_sync(~0u, mbar_wait_bounded(bar0 + stg * 8, (k / NST) & 1))) {
+    if (!__all_sync(~0u, mbar_wait_bounded(bar0 + stg * 8, ((kbase + k) / NST) & 1))) {
       if (lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
       ok = false;
       k_stop = k;
@@ -517,7 +530,7 @@ __device__ __forceinline__ bool decode_item(const CUtensorMap& kmap, const CUten
   // A warp that gave up on a wait still has its loads for pages k_stop ..
   // k_stop + NST - 1 in flight: wait for them (bounded) first.  If one never
   // lands, the stage area is left alone and the CTA ends without writing. ----
-  if (!__syncthreads_and(drain_stages<NST>(ok, k_stop, my_pages, bar0))) {
+  if (!__syncthreads_and(drain_stages<NST>(ok, k_stop, my_pages, bar0, kbase))) {
     if (spread) {  // still meet the cluster's two merge barriers
       cluster_sync();
       cluster_sync();
@@ -555,10 +568,14 @@ __device__ __forceinline__ bool decode_item(const CUtensorMap& kmap, const CUten
       *reinterpret_cast<uint32_t*>(a.out + hrow * D + d) = pack2<BF16>(o0 * inv, o1 * inv);
     }
   });
-  return true;
+  // the merge buffers were written through the generic proxy: order those
+  // writes before a later item's TMA loads into the same stage area
+  fence_proxy_async_smem();
+  kbase += my_pages;
+  return __syncthreads_and(ok);
 }
 
-template <int D, int NST, bool BF16, class Warp, int EB = 2, bool PERSIST = false>
+template <int D, int NST, bool BF16, class Warp, int EB = 2>
 __global__ void __launch_bounds__(kThreads)
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
@@ -581,51 +598,6 @@ __global__ void __launch_bounds__(kThreads)
   const bool split = a.tmp_out != nullptr;
   const bool reporter = threadIdx.x == 0 && crank == 0 && part == 0 && kvh == 0;
   const int cap = a.max_blocks_per_seq * kPage;
-
-  // ---- persistent split mode: the items that exist (partition p of
-  // sequence s for p < ceil(ctx_s / partition_size), every KV head), in a
-  // dense order that every CTA derives from the context lengths; CTA b takes
-  // items b, b + gridDim.x, ...  No CTA is launched for a partition past its
-  // sequence's end. ----
-  if constexpr (PERSIST) {
-    int* ctxs = reinterpret_cast<int*>(smem + L::kCtxOffset);
-    int* cum = reinterpret_cast<int*>(smem + L::kCumOffset);
-    for (int i = threadIdx.x; i < a.num_seqs; i += kThreads) {
-      int c = a.context_lens[i];
-      if (c < 0 || c > cap) {
-        if (blockIdx.x == 0) record_error(kErrContextLen, i);
-        c = c < 0 ? 0 : cap;
-      }
-      int np = (c + a.partition_size - 1) / a.partition_size;
-      if (np > a.max_partitions) {
-        if (blockIdx.x == 0) record_error(kErrPartitions, i);
-        np = a.max_partitions;
-      }
-      ctxs[i] = c;
-      cum[i + 1] = np;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {  // running count (at most kLptMaxSeqs sequences)
-      int acc = 0;
-      cum[0] = 0;
-      for (int i = 0; i < a.num_seqs; ++i) cum[i + 1] = (acc += cum[i + 1]);
-    }
-    __syncthreads();
-    const int items = cum[a.num_seqs] * a.num_kv_heads;
-    for (int u = blockIdx.x; u < items; u += gridDim.x) {
-      const int kv = u % a.num_kv_heads, su = u / a.num_kv_heads;
-      int lo = 0, hi = a.num_seqs;  // the sequence with cum[s] <= su < cum[s + 1]
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (cum[mid] <= su) lo = mid; else hi = mid;
-      }
-      if (!decode_item<D, NST, BF16, Warp, EB>(kmap, vmap, a, smem, lo, kv, su - cum[lo],
-                                               ctxs[lo], 1, 0))
-        return;
-      __syncthreads();  // the merge buffers (stage area) are free for the next item
-    }
-    return;
-  }
 
   // ---- longest-first order: grid slot s takes the s-th longest sequence
   // (ties by index), so that long items start first and short ones fill the
@@ -653,6 +625,7 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
     s = *chosen;
+    fence_proxy_async_smem();  // generic writes to the stage area before TMA writes to it
     __syncthreads();  // the stage area is about to be reused
   }
 
@@ -664,7 +637,79 @@ __global__ void __launch_bounds__(kThreads)
   }
   if (split && reporter && (ctx + a.partition_size - 1) / a.partition_size > a.max_partitions)
     record_error(kErrPartitions, s);
-  decode_item<D, NST, BF16, Warp, EB>(kmap, vmap, a, smem, s, kvh, part, ctx, csize, crank);
+  init_ring<NST>(smem_addr(smem + L::kBarOffset) + (threadIdx.x >> 5) * NST * 8, threadIdx.x & 31);
+  int kbase = 0;
+  decode_item<D, NST, BF16, Warp, EB>(kmap, vmap, a, smem, s, kvh, part, ctx, csize, crank,
+                                      kbase);
+}
+
+
+// ---------------------------------------------------------------------------
+// Split mode, persistent (up to kLptMaxSeqs sequences): the items that exist
+// -- partition p of sequence s for p < ceil(ctx_s / partition_size), every KV
+// head -- in a dense order that every CTA derives from the context lengths.
+// The grid is one wave (SMs x resident CTAs); CTA b takes items b,
+// b + gridDim.x, ..., so no CTA is launched for a partition past its
+// sequence's end.  Each warp's ring runs on from item to item.
+// ---------------------------------------------------------------------------
+template <int D, int NST, bool BF16, class Warp, int EB = 2>
+__global__ void __launch_bounds__(kThreads, 3)  // three CTAs per SM: at most 168 registers
+    paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap kmap,
+                                   const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
+  using L = DecodeSmem<D, NST, EB>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  prefetch_tensormap(&kmap);
+  prefetch_tensormap(&vmap);
+  pdl_launch_dependents();
+  pdl_wait();  // inputs may come from the previous kernel of the stream
+  const int cap = a.max_blocks_per_seq * kPage;
+
+  {
+    int* ctxs = reinterpret_cast<int*>(smem + L::kCtxOffset);
+    int* cum = reinterpret_cast<int*>(smem + L::kCumOffset);
+    for (int i = threadIdx.x; i < a.num_seqs; i += kThreads) {
+      int c = a.context_lens[i];
+      if (c < 0 || c > cap) {
+        if (blockIdx.x == 0) record_error(kErrContextLen, i);
+        c = c < 0 ? 0 : cap;
+      }
+      int np = (c + a.partition_size - 1) / a.partition_size;
+      if (np > a.max_partitions) {
+        if (blockIdx.x == 0) record_error(kErrPartitions, i);
+        np = a.max_partitions;
+      }
+      ctxs[i] = c;
+      cum[i + 1] = np;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {  // running count (at most kLptMaxSeqs sequences)
+      int acc = 0;
+      cum[0] = 0;
+      for (int i = 0; i < a.num_seqs; ++i) cum[i + 1] = (acc += cum[i + 1]);
+    }
+    __syncthreads();
+    const int items = cum[a.num_seqs] * a.num_kv_heads;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    init_ring<NST>(smem_addr(smem + L::kBarOffset) + warp * NST * 8, lane);
+    int kbase = 0;  // this warp's pages through its ring so far
+    for (int u = blockIdx.x; u < items; u += gridDim.x) {
+      const int kv = u % a.num_kv_heads, su = u / a.num_kv_heads;
+      int lo = 0, hi = a.num_seqs;  // the sequence with cum[s] <= su < cum[s + 1]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (cum[mid] <= su) lo = mid; else hi = mid;
+      }
+      // (decode_item ends with a CTA barrier: the merge buffers, in the
+      // stage area, are free for the next item's pages)
+      if (!decode_item<D, NST, BF16, Warp, EB>(kmap, vmap, a, smem, lo, kv, su - cum[lo],
+                                               ctxs[lo], 1, 0, kbase))
+        return;
+    }
+    return;
+  }
+
 }
 
 }  // namespace pa

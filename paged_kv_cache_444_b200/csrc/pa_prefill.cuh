@@ -302,6 +302,7 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
     s = slot[0];
     pair = slot[1];
     kvh = static_cast<int>(blockIdx.x) % a.num_kv_heads;
+    fence_proxy_async_smem();  // generic writes to the stage area before TMA writes to it
     __syncthreads();  // the stage area is about to be reused
     if (s < 0) return;  // more CTAs than units: nothing to do
   } else {

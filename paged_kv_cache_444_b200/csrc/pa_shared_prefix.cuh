@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
     slot = *chosen;
+    fence_proxy_async_smem();  // generic writes to the stage area before TMA writes to it
     __syncthreads();  // the stage area is about to be reused
   }
   const int chunk = slot % a.chunks_per_group;
