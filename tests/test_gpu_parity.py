@@ -114,6 +114,21 @@ def _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, ps):
     assert np.nanmax(np.abs(na - ng)[valid]) <= TOL[cfg.dtype]
 
 
+def test_split_over_full_grid_for_many_sequences(dev, oracle_lib):
+    """More than 256 sequences: the split launch covers every possible
+    partition with its own CTA (the persistent form serves smaller batches);
+    partials and merged output against the oracle."""
+    cfg = SMALL["mha_small"].scaled(num_seqs=300, num_heads=2, num_kv_heads=2, num_blocks=2048,
+                                    ctx=("uniform", 0, 90), seed=23)
+    batch = workloads.make_batch(cfg, dev)
+    host = HostCopy(batch)
+    ref, kc_ref, vc_ref = oracle_step(oracle_lib, host)
+    out, ws = gpu_step(batch, partition_size=32)
+    pa_check_error()
+    _check_close(out, ref, cfg, "split, 300 sequences")
+    _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, 32)
+
+
 def test_split_single_partition_equals_single_pass(dev):
     cfg = SMALL["gqa_small"]
     batch = workloads.make_batch(cfg, dev)
