@@ -131,7 +131,7 @@ template <int D>
 struct Stages { static constexpr int value = D == 64 ? PA_STAGES_D64 : PA_STAGES_D128; };
 
 #ifndef PA_SPLIT_PERSISTENT
-#define PA_SPLIT_PERSISTENT 1  // split launches: one wave of CTAs over the items that exist
+#define PA_SPLIT_PERSISTENT 1  // fp8 split launches: one wave of CTAs over the items that exist
 #endif
 #ifndef PA_CLUSTER_PAGES
 #define PA_CLUSTER_PAGES 256  // an item with more pages is spread over its cluster
@@ -208,21 +208,24 @@ pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeAr
   constexpr int NST = EB == 1 ? PA_STAGES_FP8 : Stages<D>::value;
   using L = DecodeSmem<D, NST, EB>;
   auto kernel = paged_decode_kernel<D, NST, BF16, Warp, EB>;
-  auto kernel_persist = paged_decode_persistent_kernel<D, NST, BF16, Warp, EB>;
-  static std::atomic<uint64_t> done{0}, done_persist{0};
+  static std::atomic<uint64_t> done{0};
   static std::atomic<int> cluster_cache[kMaxDevices] = {};
-  static std::atomic<long long> resident_cache[kMaxDevices] = {};
   const bool split = a.tmp_out != nullptr;
-  if (split && a.persistent) {
-    // one wave of CTAs loops over the items that exist (at most `grid`)
-    if (!ensure_smem(kernel_persist, L::kAlloc, &done_persist)) return PA_ERR_CUDA;
-    const long long resident = resident_ctas(kernel_persist, L::kAlloc, resident_cache);
-    if (resident > 0) {
-      if (grid > resident) grid = resident;
-      return launch_ex(kernel_persist, static_cast<unsigned>(grid), kThreads, L::kAlloc, stream,
-                       1, km, vm, a);
+  if constexpr (EB == 1) {  // the persistent form is built for the fp8 pages only
+    static std::atomic<uint64_t> done_persist{0};
+    static std::atomic<long long> resident_cache[kMaxDevices] = {};
+    auto kernel_persist = paged_decode_persistent_kernel<D, NST, BF16, Warp, EB>;
+    if (split && a.persistent) {
+      // one wave of CTAs loops over the items that exist (at most `grid`)
+      if (!ensure_smem(kernel_persist, L::kAlloc, &done_persist)) return PA_ERR_CUDA;
+      const long long resident = resident_ctas(kernel_persist, L::kAlloc, resident_cache);
+      if (resident > 0) {
+        if (grid > resident) grid = resident;
+        return launch_ex(kernel_persist, static_cast<unsigned>(grid), kThreads, L::kAlloc,
+                         stream, 1, km, vm, a);
+      }
+      a.persistent = 0;
     }
-    a.persistent = 0;
   }
   if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
   const int c = split ? 1 : pick_cluster(kernel, L::kAlloc, max_pages, cluster_cache);
@@ -279,9 +282,10 @@ pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cach
     return PA_ERR_CUDA;
   const long long grid = num_seqs * a.num_kv_heads * static_cast<long long>(a.parts_per_head);
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
-  // split mode, up to kLptMaxSeqs sequences: persistent CTAs over a dense item list
+  // 16-bit split launches keep the grid over every possible partition: the
+  // persistent form measured 2.5-4 % slower on these kernels
   a.num_seqs = static_cast<int>(num_seqs);
-  a.persistent = PA_SPLIT_PERSISTENT && a.tmp_out != nullptr && num_seqs <= kLptMaxSeqs;
+  a.persistent = 0;
   const bool bf16 = dtype == PA_BF16;
   const int64_t max_pages = a.max_blocks_per_seq;  // block_size == 16 == one page
   if (head_dim == 64)
@@ -302,6 +306,9 @@ pa_status run_decode_fp8(DecodeArgs a, const void* key_cache, const void* value_
     return PA_ERR_CUDA;
   const long long grid = num_seqs * a.num_kv_heads * static_cast<long long>(a.parts_per_head);
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
+  // fp8 split launches with up to kLptMaxSeqs sequences: one persistent wave of
+  // CTAs over the partitions that exist (measured 2.5-7 % faster than the
+  // grid over every possible partition; the fp8 items are short)
   a.num_seqs = static_cast<int>(num_seqs);
   a.persistent = PA_SPLIT_PERSISTENT && a.tmp_out != nullptr && num_seqs <= kLptMaxSeqs;
   const int64_t max_pages = a.max_blocks_per_seq;
