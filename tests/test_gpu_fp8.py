@@ -93,6 +93,34 @@ def test_fp8_split_matches_oracle(name, ps, cuda_device, oracle_lib):
     assert err <= TOL[cfg.dtype], f"{name} split {ps}: {err:.3e}"
 
 
+@pytest.mark.parametrize("name,ps", [("ragged_bf16", 16), ("many_seqs_f16", 32)],
+                         ids=["persistent_ragged_with_empty", "full_grid_300_seqs"])
+def test_fp8_split_ragged_and_large_batches(name, ps, cuda_device, oracle_lib):
+    """The fp8 split launch is persistent up to 256 sequences (one wave of CTAs
+    over the partitions that exist, empty sequences contributing none) and a
+    grid over every possible partition beyond; both against the oracle."""
+    cfg = (CASES["ragged_bf16"] if name == "ragged_bf16" else
+           C["mha_llama2_7b"].scaled(num_seqs=300, num_heads=2, num_kv_heads=2, num_blocks=2048,
+                                     ctx=("uniform", 0, 90), seed=56))
+    b, kc, vc = _fp8_batch(cfg, cuda_device)
+    ref, _, _ = _oracle(oracle_lib, b, kc, vc)
+    pa_reshape_and_cache_fp8(b.key, b.value, kc, vc, b.slot_mapping, K_SCALE, V_SCALE)
+    P = (b.block_tables.shape[1] * 16 + ps - 1) // ps
+    ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, cuda_device)
+    out = torch.full_like(b.query, float("nan"))
+    pa_decode_split_fp8(ws.tmp_out, ws.max_logits, ws.exp_sums, b.query, kc, vc, b.block_tables,
+                        b.context_lens, cfg.scale, K_SCALE, V_SCALE, ps)
+    pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, b.context_lens, ps)
+    torch.cuda.synchronize()
+    pa_check_error()
+    g = to_f64(out)
+    assert np.isfinite(g).all()
+    zero = (b.context_lens == 0).cpu().numpy()
+    assert (g[zero] == 0).all()
+    err = np.max(np.abs(g - ref))
+    assert err <= TOL[cfg.dtype], f"{name} split {ps}: {err:.3e}"
+
+
 @pytest.mark.parametrize("split", [0, 64])
 @pytest.mark.parametrize("name", ["mha_f16", "gqa_bf16", "gqa16_bf16"])
 def test_fp8_nan_codes_past_context_do_not_leak(name, split, cuda_device, oracle_lib):
