@@ -1044,16 +1044,39 @@ bool encode_query_map(CUtensorMap* map, const void* query, pa_dtype dtype, int64
   return r == CUDA_SUCCESS;
 }
 
+// Streaming multiprocessors of the current device, looked up once per device
+// (0 if the query fails).
+long long sm_count() {
+  static std::atomic<long long> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  long long known = cache[dev].load(std::memory_order_relaxed);
+  if (known == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    known = sms;
+    cache[dev].store(known, std::memory_order_relaxed);
+  }
+  return known;
+}
+
+// The prefill grid is persistent: one CTA per SM (its shared memory admits
+// no second one), each walking its share of the items.
 template <int D, bool BF16>
 pa_status launch_prefill_t(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
-                           const PrefillArgs& a, long long grid, cudaStream_t stream) {
+                           const PrefillArgs& a, long long items, cudaStream_t stream) {
   using L = PrefillSmem<D, BF16>;
   auto kernel = paged_prefill_kernel<D, BF16>;
   static std::atomic<uint64_t> done{0};
   if (!ensure_smem(kernel, L::kAlloc, &done)) return PA_ERR_CUDA;
+  const long long sms = sm_count();
+  if (sms <= 0) return PA_ERR_CUDA;
+  const long long grid = items < sms ? items : sms;
   return launch_ex(kernel, static_cast<unsigned>(grid), PrefillRoles<BF16>::kThreads, L::kAlloc,
-                   stream, 1, qm,
-                   km, vm, a);
+                   stream, 1, qm, km, vm, a);
 }
 
 
@@ -1079,8 +1102,8 @@ extern "C" pa_status pa_prefill(void* out, const void* query, const void* key_ca
   const int64_t tile = kPrefillRows / G;                  // G <= 16 checked above
   const int64_t tiles = (max_query_len + tile - 1) / tile;
   const int64_t pairs = (tiles + 1) / 2;                  // two query tiles per CTA
-  const long long grid = num_seqs * num_kv_heads * pairs;
-  if (grid > INT32_MAX) return PA_ERR_SHAPE;
+  const long long items = num_seqs * num_kv_heads * pairs;   // (sequence, KV head, tile pair)
+  if (items > INT32_MAX) return PA_ERR_SHAPE;
   CUtensorMap qm, km, vm;
   if (!encode_query_map(&qm, query, dtype, num_query_tokens, num_heads, head_dim, G, tile) ||
       !encode_cache_map(&km, key_cache, dtype, num_blocks, num_kv_heads, head_dim) ||
@@ -1104,9 +1127,9 @@ extern "C" pa_status pa_prefill(void* out, const void* query, const void* key_ca
   cudaStream_t s = as_stream(stream);
   const bool bf16 = dtype == PA_BF16;
   if (head_dim == 64)
-    return bf16 ? launch_prefill_t<64, true>(qm, km, vm, a, grid, s)
-                : launch_prefill_t<64, false>(qm, km, vm, a, grid, s);
-  return bf16 ? launch_prefill_t<128, true>(qm, km, vm, a, grid, s)
-              : launch_prefill_t<128, false>(qm, km, vm, a, grid, s);
+    return bf16 ? launch_prefill_t<64, true>(qm, km, vm, a, items, s)
+                : launch_prefill_t<64, false>(qm, km, vm, a, items, s);
+  return bf16 ? launch_prefill_t<128, true>(qm, km, vm, a, items, s)
+              : launch_prefill_t<128, false>(qm, km, vm, a, items, s);
 }
 // <<< chunked prefill

@@ -52,6 +52,9 @@ constexpr int kWarpTma = 9;                         // Q, K and V loads
 constexpr int kPrefillThreads = 10 * 32;            // + two softmax warpgroups (warps 0-7)
 constexpr int kWarpConv = 10;                       // V converters: warps 10-13 (convert mode)
 constexpr unsigned kErrValue = 8;
+constexpr int kRankMaxSeqs = 256;     // batches ranked longest-first by every CTA: sequences,
+constexpr int kRankMaxUnits = 2048;   // units (sequence, tile pair),
+constexpr int kRankMaxWork = 16384;   // and units x sequences counted
 
 // bf16 caches: rewrite each landed V block as fp16 in shared memory (warps
 // 10-13, once per block for both tiles), so that P enters P V once, as fp16
@@ -122,9 +125,15 @@ struct PrefillSmem {
   static constexpr int kBarS = kBarVConv + 8 * NST;    // per tile: S_t(j) (and P_t(j-1) V) done
   static constexpr int kBarP = kBarS + 16;             // per tile: P_t(j) written
   static constexpr int kBarO = kBarP + 16;             // every MMA done
-  static constexpr int kTmemSlot = kBarO + 8;
+  static constexpr int kBarQFree = kBarO + 8;          // an item's S products done: Q replaceable
+  static constexpr int kBarOFull = kBarQFree + 8;      // per tile: an item's last P V done
+  static constexpr int kBarOFree = kBarOFull + 16;     // per tile: O read by the epilogue
+  static constexpr int kTmemSlot = kBarOFree + 16;
   static constexpr int kAbort = kTmemSlot + 4;
-  static constexpr int kBytes = kAbort + 4;
+  static constexpr int kSched = kAbort + 4;            // unit count and per-warp sums (16 ints)
+  static constexpr int kSeqs = (kSched + 64 + 15) & ~15;   // int4 per sequence while ranking
+  static constexpr int kList = kSeqs + 16 * kRankMaxSeqs;  // unit of each rank
+  static constexpr int kBytes = kList + 4 * kRankMaxUnits;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
@@ -153,14 +162,20 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
-// Longest-first item order.  A unit is (sequence, tile pair); its cost grows
-// with the keys its last query token sees, hist + min(T2 (p + 1), q_len)
-// (hist = context - q_len, T2 = query tokens of a tile pair).  CTAs start in
-// grid order, so handing out units by descending key count (ties by
-// sequence, then pair) starts the long ones first and fills the tail with
-// short ones; the K/V a sequence's pairs share is read again from L2.
+// Work items and their order.  An item is (sequence s, tile pair p, KV head);
+// a unit is (s, p), and item i is unit i / Hk with KV head i % Hk.  The grid
+// is persistent (one CTA per SM, G = gridDim.x): CTA b takes the items
+//   k G + b  (k even)   and   k G + G - 1 - b  (k odd),   k = 0, 1, ...
+// of a list ordered by descending cost, so each CTA gets a mix of long and
+// short items.  A unit's cost grows with the keys its last query token sees,
+// hist + min(T2 (p + 1), q_len) (hist = context - q_len, T2 = query tokens
+// of a tile pair).  For up to kRankMaxSeqs sequences and small unit counts,
+// every CTA ranks the units itself: descending key count, ties by sequence
+// then pair (a sequence's own pairs all differ in key count); each thread
+// counts the units ranked before one unit.  Other batches take the units in
+// a fixed order, the last pairs of every sequence (most keys) first, and skip
+// the pairs a sequence does not have.
 // ---------------------------------------------------------------------------
-constexpr int kLptSeqsPerLane = 8;  // one warp ranks up to 256 sequences
 
 // floor(x / d) for x >= 0 and d >= 2 from a float reciprocal: below 2^24 both
 // are exact floats and the quotient (< 2^23) comes out within 1 of its floor,
@@ -173,66 +188,60 @@ __device__ __forceinline__ int div_floor(int x, int d, float inv_d) {
   return q;
 }
 
-// One sequence as the ranking sees it: hist = context - q_len, its tile
-// pairs, and q_len (-1 marks an invalid sequence, which has no units).
-struct LptSeq {
-  int hist[kLptSeqsPerLane], q_len[kLptSeqsPerLane], pairs[kLptSeqsPerLane];
-};
-
-// Pairs of sequence i whose key count exceeds K.
-__device__ __forceinline__ int pairs_above(const LptSeq& q, int i, int t2, float inv_t2, int K) {
-  if (q.q_len[i] <= 0) return 0;
-  const int x = K - q.hist[i];
-  if (x >= q.q_len[i]) return 0;
-  return x < 0 ? q.pairs[i] : q.pairs[i] - div_floor(x, t2, inv_t2);  // T2 (p + 1) <= x fall short
+// Pairs of a sequence (hist, q_len, pairs) whose key count exceeds K.
+__device__ __forceinline__ int pairs_above_of(int hist, int q_len, int pairs, int t2,
+                                              float inv_t2, int K) {
+  if (q_len <= 0) return 0;
+  const int x = K - hist;
+  if (x >= q_len) return 0;
+  return x < 0 ? pairs : pairs - div_floor(x, t2, inv_t2);  // T2 (p + 1) <= x fall short
 }
 
-// The unit of rank j (0 = most keys), found by one warp: a binary search for
-// its key count K (the least K with at most j units above it), then its place
-// among the units with exactly K keys in (sequence, pair) order.  Returns
-// false when fewer than j + 1 units exist.
-__device__ __forceinline__ bool prefill_unit_of_rank(const LptSeq& q, int max_keys, int t2, int j,
-                                                     int lane, int& s_out, int& p_out) {
-  const float inv_t2 = 1.f / static_cast<float>(t2);
-  auto above = [&](int K) {
-    int c = 0;
-#pragma unroll
-    for (int i = 0; i < kLptSeqsPerLane; ++i) c += pairs_above(q, i, t2, inv_t2, K);
-    return static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)));
-  };
-  if (above(-1) <= j) return false;
-  int lo = -1, hi = max_keys;  // above(lo) > j >= above(hi) = 0
-  while (hi - lo > 1) {
-    const int mid = lo + (hi - lo) / 2;
-    if (above(mid) <= j) hi = mid;
-    else lo = mid;
+// The k-th item of this CTA (snake order), or -1 past the last.
+__device__ __forceinline__ int prefill_item_index(int k, int total) {
+  const long long g = gridDim.x, b = blockIdx.x;
+  const long long i = k * g + ((k & 1) ? g - 1 - b : b);
+  return i < total ? static_cast<int>(i) : -1;
+}
+
+struct PrefillItem {
+  int s, kvh, q0, q_len, ctx, tile_a, n_pages, nkb;
+  bool has_b;
+};
+
+// Item i; false when it has no work (a pair its sequence does not have, or an
+// invalid sequence, reported once when `report`).
+__device__ __forceinline__ bool prefill_item(const PrefillArgs& a, const int* list, bool ranked,
+                                             bool report, int i, PrefillItem& it) {
+  const int r = i / a.num_kv_heads;
+  it.kvh = i - r * a.num_kv_heads;
+  int p;
+  if (ranked) {
+    const int e = list[r];
+    it.s = e & 0xffff;
+    p = e >> 16;
+  } else {
+    const int back = r / a.num_seqs;
+    it.s = r - back * a.num_seqs;
+    p = a.pairs_per_seq - 1 - back;
   }
-  const int K = hi;
-  int t = j - above(K);  // index among the units with exactly K keys
-  bool found = false;
-#pragma unroll
-  for (int i = 0; i < kLptSeqsPerLane; ++i) {
-    const int below = pairs_above(q, i, t2, inv_t2, K - 1);
-    const int e = below - pairs_above(q, i, t2, inv_t2, K);
-    int inc = e;  // inclusive scan over the lanes (sequences i*32 + lane)
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, inc, d);
-      if (lane >= d) inc += v;
-    }
-    const int total = __shfl_sync(0xffffffffu, inc, 31);
-    if (!found && t < total) {
-      const int src = __ffs(__ballot_sync(0xffffffffu, t < inc)) - 1;
-      const int before = __shfl_sync(0xffffffffu, inc - e, src);
-      // the pairs with exactly K keys follow the pairs - below with fewer
-      const int first = __shfl_sync(0xffffffffu, q.pairs[i] - below, src);
-      s_out = i * 32 + src;
-      p_out = first + (t - before);
-      found = true;
-    }
-    if (!found) t -= total;
+  it.q0 = a.query_starts[it.s];
+  it.q_len = a.query_starts[it.s + 1] - it.q0;
+  it.ctx = a.context_lens[it.s];
+  if (it.q0 < 0 || it.q_len < 0 || it.q0 > a.num_tokens - it.q_len || it.q_len > it.ctx ||
+      it.ctx > a.max_blocks_per_seq * kPage) {
+    if (report && it.kvh == 0 && p == 0) record_error(kErrQuery, it.s);
+    return false;
   }
-  return found;
+  it.tile_a = 2 * p * a.tile_tokens;
+  if (it.tile_a >= it.q_len) return false;
+  const int tile_b = it.tile_a + a.tile_tokens;
+  it.has_b = tile_b < it.q_len;
+  const int last_tok = min((it.has_b ? tile_b : it.tile_a) + a.tile_tokens, it.q_len);
+  const int lim_max = it.ctx - it.q_len + last_tok;   // keys the pair's last token sees
+  it.n_pages = (lim_max + kPage - 1) / kPage;
+  it.nkb = (it.n_pages + kPrefillPages - 1) / kPrefillPages;
+  return true;
 }
 
 template <int D, bool BF16>
@@ -256,84 +265,80 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
   pdl_launch_dependents();
   pdl_wait();
 
-  // ---- work item ----
-  const int cap = a.max_blocks_per_seq * kPage;
-  auto seq_valid = [&](int q0, int q_len, int ctx) {
-    return !(q0 < 0 || q_len < 0 || q0 > a.num_tokens - q_len || q_len > ctx || ctx > cap);
-  };
+  // ---- the unit order (every CTA derives the same one) ----
   const int G = a.group;
-  int s, pair, kvh;
-  if (a.num_seqs <= 32 * kLptSeqsPerLane) {
-    // longest first: CTA b takes unit b / Hk, KV head b % Hk
-    int* slot = reinterpret_cast<int*>(smem);  // stage area, not in use yet
-    if (warp == 0) {
-      LptSeq q;
-      int max_keys = 0;
-      const int t2 = 2 * a.tile_tokens;
-#pragma unroll
-      for (int i = 0; i < kLptSeqsPerLane; ++i) {
-        const int t = i * 32 + lane;
-        q.hist[i] = 0;
-        q.q_len[i] = -1;
-        q.pairs[i] = 0;
-        if (t < a.num_seqs) {
-          const int q0 = a.query_starts[t], ql = a.query_starts[t + 1] - q0;
-          const int ctx = a.context_lens[t];
-          if (seq_valid(q0, ql, ctx)) {
-            q.hist[i] = ctx - ql;
-            q.q_len[i] = ql;
-            q.pairs[i] = ql / t2 + (ql % t2 != 0);
-            max_keys = max(max_keys, ctx);
-          } else if (t == static_cast<int>(blockIdx.x)) {
-            record_error(kErrQuery, t);  // each sequence is checked by one CTA
-          }
-        }
-      }
-      max_keys = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(max_keys)));
-      int us = -1, up = 0;
-      const bool found = prefill_unit_of_rank(
-          q, max_keys, t2, static_cast<int>(blockIdx.x) / a.num_kv_heads, lane, us, up);
-      if (lane == 0) {
-        slot[0] = found ? us : -1;
-        slot[1] = up;
+  const int t2 = 2 * a.tile_tokens;
+  int* sched = reinterpret_cast<int*>(smem + L::kSched);   // [0] units, [4 + w] per-warp sums
+  int4* seqs = reinterpret_cast<int4*>(smem + L::kSeqs);   // hist, q_len, pairs, first unit
+  int* list = reinterpret_cast<int*>(smem + L::kList);     // unit of each rank: s | p << 16
+  const bool table = a.num_seqs <= kRankMaxSeqs;
+  bool ranked = false;
+  if (table) {
+    const int t = threadIdx.x;
+    int hist = 0, ql = -1, np = 0;
+    if (t < a.num_seqs) {
+      const int q0 = a.query_starts[t], len = a.query_starts[t + 1] - q0;
+      const int ctx = a.context_lens[t];
+      if (q0 < 0 || len < 0 || q0 > a.num_tokens - len || len > ctx ||
+          ctx > a.max_blocks_per_seq * kPage) {
+        if (t % gridDim.x == blockIdx.x) record_error(kErrQuery, t);  // one CTA reports it
+      } else {
+        hist = ctx - len;
+        ql = len;
+        np = len / t2 + (len % t2 != 0);
       }
     }
+    int first = np;  // inclusive scan over the warp's sequences
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, first, d);
+      if (lane >= d) first += v;
+    }
+    if (lane == 31 && warp < kRankMaxSeqs / 32) sched[4 + warp] = first;
     __syncthreads();
-    s = slot[0];
-    pair = slot[1];
-    kvh = static_cast<int>(blockIdx.x) % a.num_kv_heads;
-    fence_proxy_async_smem();  // generic writes to the stage area before TMA writes to it
-    __syncthreads();  // the stage area is about to be reused
-    if (s < 0) return;  // more CTAs than units: nothing to do
-  } else {
-    // the last tile pairs of every sequence (most keys) first
-    const int per_pair = a.num_seqs * a.num_kv_heads;
-    int item = blockIdx.x;
-    pair = a.pairs_per_seq - 1 - item / per_pair;
-    item %= per_pair;
-    kvh = item % a.num_kv_heads;
-    s = item / a.num_kv_heads;
+    if (t < a.num_seqs) {
+      for (int w = 0; w < warp; ++w) first += sched[4 + w];
+      seqs[t] = make_int4(hist, ql, np, first - np);
+      if (t == a.num_seqs - 1) sched[0] = first;
+    }
+    __syncthreads();
+    const int n_units = sched[0];
+    ranked = n_units <= kRankMaxUnits &&
+             static_cast<long long>(n_units) * a.num_seqs <= kRankMaxWork;
+    if (ranked) {
+      const float inv_t2 = 1.f / static_cast<float>(t2);
+      for (int u = t; u < n_units; u += blockDim.x) {
+        int lo = 0, hi = a.num_seqs;  // the owner: the last sequence whose first unit is <= u
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (seqs[mid].w <= u) lo = mid;
+          else hi = mid;
+        }
+        const int4 me = seqs[lo];
+        const int p = u - me.w;
+        const int K = me.x + min(t2 * (p + 1), me.y);
+        int rank = 0;
+        for (int i = 0; i < a.num_seqs; ++i) {
+          const int4 o = seqs[i];
+          const int gt = pairs_above_of(o.x, o.y, o.z, t2, inv_t2, K);
+          rank += gt;
+          if (i < lo) rank += pairs_above_of(o.x, o.y, o.z, t2, inv_t2, K - 1) - gt;
+        }
+        list[rank] = lo | (p << 16);
+      }
+      __syncthreads();
+    }
   }
-
-  const int q0 = a.query_starts[s];
-  const int q_len = a.query_starts[s + 1] - q0;
-  const int ctx = a.context_lens[s];
-  if (!seq_valid(q0, q_len, ctx)) {
-    if (threadIdx.x == 0 && kvh == 0 && pair == 0) record_error(kErrQuery, s);
-    return;
-  }
-  const int tile_a = 2 * pair * a.tile_tokens, tile_b = tile_a + a.tile_tokens;
-  if (tile_a >= q_len) return;
-  const bool has_b = tile_b < q_len;
-  const int last_tok = min((has_b ? tile_b : tile_a) + a.tile_tokens, q_len);  // exclusive
-  const int lim_max = ctx - q_len + last_tok;      // keys the pair's last token sees
-  const int n_pages = (lim_max + kPage - 1) / kPage;
-  const int nkb = (n_pages + kPrefillPages - 1) / kPrefillPages;
+  const int total = ranked ? sched[0] * a.num_kv_heads
+                           : a.num_seqs * a.num_kv_heads * a.pairs_per_seq;
+  if (prefill_item_index(0, total) < 0) return;   // more CTAs than items
+  const bool report = !table && warp == kWarpTma && lane == 0;
   const int q_rows = a.tile_tokens * G;           // rows a Q box fills
 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
   if (threadIdx.x == 0) {
     mbar_init(sb + L::kBarQ, 1);
+    mbar_init(sb + L::kBarQFree, 1);
     for (int i = 0; i < NST; ++i) {
       mbar_init(sb + L::kBarKFull + 8 * i, 1);
       mbar_init(sb + L::kBarKEmpty + 8 * i, 1);
@@ -344,6 +349,8 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(sb + L::kBarS + 8 * t, 1);
       mbar_init(sb + L::kBarP + 8 * t, 4 * 32);
+      mbar_init(sb + L::kBarOFull + 8 * t, 1);
+      mbar_init(sb + L::kBarOFree + 8 * t, 4 * 32);
     }
     mbar_init(sb + L::kBarO, 1);
     *abort_flag = 0;
@@ -370,79 +377,90 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
   if constexpr (R::kConvert) regs_decrease();
   if (warp == kWarpTma) {
     // ================= TMA producer =================
-    if (lane == 0) {
-      const int tiles = has_b ? 2 : 1;
-      mbar_arrive_expect_tx(sb + L::kBarQ, tiles * L::kSlabs * q_rows * 128);
-      for (int t = 0; t < tiles; ++t) {
-#pragma unroll
-        for (int b = 0; b < L::kSlabs; ++b)
-          tma_load_4d(sb + L::kQ + t * L::kQTile + b * L::kSlab, &qmap, sb + L::kBarQ, 0, b,
-                      kvh * G, q0 + (t == 0 ? tile_a : tile_b));
-      }
-    }
-    const int32_t* bt = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
-    int k_issued = 0, v_issued = 0;
+    // Blocks of K and V go through the rings in one running count g over all
+    // of the CTA's items; Q is replaced once the previous item's S products
+    // are done.
+    int n_q = 0, k_issued = 0, v_issued = 0;
     bool ok = true;
-    for (int j = 0; j < nkb; ++j) {
-      const int st = j % NST;
-      const uint32_t par = ((j / NST) & 1) ^ 1;
-      int id = -1;
-      if (lane < kPrefillPages) {
-        const int pg = j * kPrefillPages + lane;
-        if (pg < n_pages) {
-          id = bt[pg];
-          if (id < 0 || id >= a.num_blocks) {
-            record_error(kErrBlockId, static_cast<long long>(s) * a.max_blocks_per_seq + pg);
-            id = -1;   // a fully out-of-range box: zeros
+    for (int k = 0; ok; ++k) {
+      const int i = prefill_item_index(k, total);
+      if (i < 0) break;
+      PrefillItem it;
+      if (!prefill_item(a, list, ranked, report, i, it)) continue;
+      if (n_q > 0 && !(ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarQFree,
+                                                                  (n_q - 1) & 1, abort_flag))))
+        break;
+      if (lane == 0) {
+        const int tiles = it.has_b ? 2 : 1;
+        mbar_arrive_expect_tx(sb + L::kBarQ, tiles * L::kSlabs * q_rows * 128);
+        for (int t = 0; t < tiles; ++t) {
+#pragma unroll
+          for (int b = 0; b < L::kSlabs; ++b)
+            tma_load_4d(sb + L::kQ + t * L::kQTile + b * L::kSlab, &qmap, sb + L::kBarQ, 0, b,
+                        it.kvh * G, it.q0 + it.tile_a + t * a.tile_tokens);
+        }
+      }
+      ++n_q;
+      const int32_t* bt = a.block_tables + static_cast<size_t>(it.s) * a.max_blocks_per_seq;
+      for (int j = 0; j < it.nkb; ++j) {
+        const int g = k_issued;
+        const int st = g % NST;
+        const uint32_t par = ((g / NST) & 1) ^ 1;
+        int id = -1;
+        if (lane < kPrefillPages) {
+          const int pg = j * kPrefillPages + lane;
+          if (pg < it.n_pages) {
+            id = bt[pg];
+            if (id < 0 || id >= a.num_blocks) {
+              record_error(kErrBlockId, static_cast<long long>(it.s) * a.max_blocks_per_seq + pg);
+              id = -1;   // a fully out-of-range box: zeros
+            }
           }
         }
-      }
-      if (j >= NST) ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarKEmpty + 8 * st, par,
-                                                               abort_flag));
-      if (!ok) break;
-      const uint32_t kst = sb + L::kK + st * L::kStage;
-      if (lane == 0) mbar_arrive_expect_tx(sb + L::kBarKFull + 8 * st, L::kStage);
-#pragma unroll
-      for (int p = 0; p < kPrefillPages; ++p) {
-        const int idp = __shfl_sync(0xffffffffu, id, p);
-        if (lane == 0) {
-#pragma unroll
-          for (int b = 0; b < L::kSlabs; ++b)
-            tma_load_4d(kst + b * L::kSlab + p * 2048, &kmap, sb + L::kBarKFull + 8 * st, 0, b,
-                        kvh, idp * kPage);
-        }
-      }
-      k_issued = j + 1;
-      if (j >= NST) ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarVEmpty + 8 * st, par,
-                                                               abort_flag));
-      if (!ok) break;
-      const uint32_t vst = sb + L::kV + st * L::kStage;
-      if (lane == 0) mbar_arrive_expect_tx(sb + L::kBarVFull + 8 * st, L::kStage);
-#pragma unroll
-      for (int p = 0; p < kPrefillPages; ++p) {
-        const int idp = __shfl_sync(0xffffffffu, id, p);
-        if (lane == 0) {
+        if (g >= NST && !(ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarKEmpty + 8 * st,
+                                                                     par, abort_flag))))
+          break;
+        const uint32_t kst = sb + L::kK + st * L::kStage;
+        if (lane == 0) mbar_arrive_expect_tx(sb + L::kBarKFull + 8 * st, L::kStage);
+        // lane 0 registers the stage's bytes first; then lane p issues page p's boxes, which
+        // measured faster than lane 0 issuing all of them
+        __syncwarp();
+        if (lane < kPrefillPages) {
 #pragma unroll
           for (int b = 0; b < L::kSlabs; ++b)
-            tma_load_4d(vst + b * L::kSlab + p * 2048, &vmap, sb + L::kBarVFull + 8 * st, 0, b,
-                        kvh, idp * kPage);
+            tma_load_4d(kst + b * L::kSlab + lane * 2048, &kmap, sb + L::kBarKFull + 8 * st, 0, b,
+                        it.kvh, id * kPage);
         }
+        k_issued = g + 1;
+        if (g >= NST && !(ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarVEmpty + 8 * st,
+                                                                     par, abort_flag))))
+          break;
+        const uint32_t vst = sb + L::kV + st * L::kStage;
+        if (lane == 0) mbar_arrive_expect_tx(sb + L::kBarVFull + 8 * st, L::kStage);
+        __syncwarp();
+        if (lane < kPrefillPages) {
+#pragma unroll
+          for (int b = 0; b < L::kSlabs; ++b)
+            tma_load_4d(vst + b * L::kSlab + lane * 2048, &vmap, sb + L::kBarVFull + 8 * st, 0, b,
+                        it.kvh, id * kPage);
+        }
+        v_issued = g + 1;
       }
-      v_issued = j + 1;
     }
     // every load issued lands before the CTA can exit (after an abort some were
     // never consumed); in the normal path these phases have long completed
-    if (!mbar_wait_bounded(sb + L::kBarQ, 0) && lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
-    for (int j = max(0, k_issued - NST); j < k_issued; ++j)
-      mbar_wait_bounded(sb + L::kBarKFull + 8 * (j % NST), (j / NST) & 1);
-    for (int j = max(0, v_issued - NST); j < v_issued; ++j)
-      mbar_wait_bounded(sb + L::kBarVFull + 8 * (j % NST), (j / NST) & 1);
+    if (n_q > 0 && !mbar_wait_bounded(sb + L::kBarQ, (n_q - 1) & 1) && lane == 0)
+      record_error(kErrWaitTimeout, blockIdx.x);
+    for (int g = max(0, k_issued - NST); g < k_issued; ++g)
+      mbar_wait_bounded(sb + L::kBarKFull + 8 * (g % NST), (g / NST) & 1);
+    for (int g = max(0, v_issued - NST); g < v_issued; ++g)
+      mbar_wait_bounded(sb + L::kBarVFull + 8 * (g % NST), (g / NST) & 1);
   } else if (warp == kWarpMma) {
     // ================= MMA issuer =================
     constexpr uint32_t kIdS = umma_idesc_f16(BF16, kPrefillRows, kPrefillKeys, false);
     constexpr uint32_t kIdO = umma_idesc_f16(R::kPHiLo, kPrefillRows, D, true);
-    auto issue_s = [&](int t, int j) {   // S_t(j) = Q_t K_j^T, then report it
-      const uint32_t kst = sb + L::kK + (j % NST) * L::kStage;
+    auto issue_s = [&](int t, int g) {   // S_t = Q_t K_g^T, then report it
+      const uint32_t kst = sb + L::kK + (g % NST) * L::kStage;
       const uint32_t qt = sb + L::kQ + t * L::kQTile;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
@@ -452,8 +470,9 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
       }
       umma_commit(sb + L::kBarS + 8 * t);
     };
-    auto issue_pv = [&](int t, int j) {  // O_t += P_t(j) V_j over the block's pages
-      const uint32_t vst = sb + L::kV + (j % NST) * L::kStage;
+    // O_t (+)= P_t V_g over the pages of block j of an item with n_pages pages
+    auto issue_pv = [&](int t, int g, int j, int n_pages) {
+      const uint32_t vst = sb + L::kV + (g % NST) * L::kStage;
       const uint32_t pcol = tmem + kTmemS + 128 * t;  // hi in 64 columns, lo in the next 64
       const int pages_here = min(kPrefillPages, n_pages - j * kPrefillPages);
       for (int k = 0; k < pages_here; ++k) {
@@ -469,15 +488,15 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
       tmem_fence_after_sync();
       return r;
     };
-    const int last_page = (ctx - 1) / kPage;
-    const int tail_row = ctx % kPage;          // first row past the context in the last page
-    auto v_ready = [&](int j) {                // V_j landed; clear its rows past the context
+    // V of running block g (block j of item `it`) landed; rows past the context cleared
+    auto v_ready = [&](int g, int j, const PrefillItem& it) {
       if constexpr (R::kConvert)   // the converters rewrote it (and cleared those rows)
-        return wait(sb + L::kBarVConv + 8 * (j % NST), (j / NST) & 1);
-      if (!wait(sb + L::kBarVFull + 8 * (j % NST), (j / NST) & 1)) return false;
-      const int lp = last_page - j * kPrefillPages;
+        return wait(sb + L::kBarVConv + 8 * (g % NST), (g / NST) & 1);
+      if (!wait(sb + L::kBarVFull + 8 * (g % NST), (g / NST) & 1)) return false;
+      const int lp = (it.ctx - 1) / kPage - j * kPrefillPages;
+      const int tail_row = it.ctx % kPage;     // first row past the context in the last page
       if (tail_row != 0 && lp >= 0 && lp < kPrefillPages) {
-        const uint32_t vst = sb + L::kV + (j % NST) * L::kStage;
+        const uint32_t vst = sb + L::kV + (g % NST) * L::kStage;
         const int chunks = (kPage - tail_row) * 8;
         for (int i = lane; i < chunks * L::kSlabs; i += 32) {
           const int b = i / chunks, c = i % chunks;
@@ -488,45 +507,71 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
       }
       return true;
     };
-    bool ok = wait(sb + L::kBarQ, 0) && wait(sb + L::kBarKFull, 0);
-    if (ok) {
-      if (lane == 0) {
-        issue_s(0, 0);
-        if (has_b) issue_s(1, 0);
-        umma_commit(sb + L::kBarKEmpty);
+    // Per item the issue order is S_A(j), P_B(j-1) V, S_B(j), P_A(j) V, so each
+    // tile's softmax overlaps the other tile's MMAs.  Running counts: g0 blocks
+    // before this item, done[t] S/P rounds and items[t] items of tile t.
+    int n_q = 0, g0 = 0, done[2] = {0, 0}, items[2] = {0, 0};
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int i = prefill_item_index(k, total);
+      if (i < 0) break;
+      PrefillItem it;
+      if (!prefill_item(a, list, ranked, false, i, it)) continue;
+      const bool hb = it.has_b;
+      const int nkb = it.nkb;
+      // before the first P_t V of an item: the epilogue has read O_t of the last one
+      auto o_free = [&](int t) {
+        return items[t] == 0 || wait(sb + L::kBarOFree + 8 * t, (items[t] - 1) & 1);
+      };
+      if (!(ok = wait(sb + L::kBarQ, n_q & 1))) break;
+      ++n_q;
+      for (int j = 0; j < nkb; ++j) {
+        const int g = g0 + j;
+        if (!(ok = wait(sb + L::kBarKFull + 8 * (g % NST), (g / NST) & 1))) break;
+        if (lane == 0) issue_s(0, g);                    // after P_A(j-1) V in issue order
+        __syncwarp();
+        if (j > 0 && hb) {
+          if (!(ok = (j > 1 || o_free(1)) && wait(sb + L::kBarP + 8, (done[1] + j - 1) & 1))) break;
+          if (lane == 0) issue_pv(1, g - 1, j - 1, it.n_pages);
+          __syncwarp();
+        }
+        if (lane == 0) {
+          if (j > 0) umma_commit(sb + L::kBarVEmpty + 8 * ((g - 1) % NST));  // V used by both tiles
+          if (hb) issue_s(1, g);
+          umma_commit(sb + L::kBarKEmpty + 8 * (g % NST));                  // K used by both tiles
+          if (j == nkb - 1) umma_commit(sb + L::kBarQFree);                 // the item's last S
+        }
+        __syncwarp();
+        if (!(ok = (j > 0 || o_free(0)) && v_ready(g, j, it) &&
+                   wait(sb + L::kBarP, (done[0] + j) & 1)))
+          break;
+        if (lane == 0) issue_pv(0, g, j, it.n_pages);
+        __syncwarp();
       }
-      __syncwarp();
-      ok = v_ready(0) && wait(sb + L::kBarP, 0);
-      if (ok && lane == 0) issue_pv(0, 0);
-      __syncwarp();
-    }
-    for (int j = 1; ok && j < nkb; ++j) {
-      const int st = j % NST;
-      if (!(ok = wait(sb + L::kBarKFull + 8 * st, (j / NST) & 1))) break;
-      if (lane == 0) issue_s(0, j);                      // after P_A(j-1) V in issue order
-      __syncwarp();
-      if (has_b) {
-        if (!(ok = wait(sb + L::kBarP + 8, (j - 1) & 1))) break;
-        if (lane == 0) issue_pv(1, j - 1);
+      if (!ok) break;
+      const int gl = g0 + nkb - 1;
+      if (hb) {
+        if (!(ok = (nkb > 1 || o_free(1)) && wait(sb + L::kBarP + 8, (done[1] + nkb - 1) & 1)))
+          break;
+        if (lane == 0) issue_pv(1, gl, nkb - 1, it.n_pages);
         __syncwarp();
       }
       if (lane == 0) {
-        umma_commit(sb + L::kBarVEmpty + 8 * ((j - 1) % NST));   // V_{j-1} used by both tiles
-        if (has_b) issue_s(1, j);
-        umma_commit(sb + L::kBarKEmpty + 8 * st);                 // K_j used by both tiles
+        umma_commit(sb + L::kBarVEmpty + 8 * (gl % NST));
+        umma_commit(sb + L::kBarOFull);
+        if (hb) umma_commit(sb + L::kBarOFull + 8);
       }
       __syncwarp();
-      if (!(ok = v_ready(j) && wait(sb + L::kBarP, j & 1))) break;
-      if (lane == 0) issue_pv(0, j);
-      __syncwarp();
+      g0 += nkb;
+      done[0] += nkb;
+      ++items[0];
+      if (hb) {
+        done[1] += nkb;
+        ++items[1];
+      }
     }
-    if (ok && has_b) {
-      ok = wait(sb + L::kBarP + 8, (nkb - 1) & 1);
-      if (ok && lane == 0) issue_pv(1, nkb - 1);
-      __syncwarp();
-    }
-    // every MMA issued has completed before the epilogue reads O and before
-    // tensor memory is freed (also after an abort)
+    // every MMA issued has completed before tensor memory is freed (also
+    // after an abort)
     if (lane == 0) umma_commit(sb + L::kBarO);
     __syncwarp();
     if (!mbar_wait_bounded(sb + L::kBarO, 0) && lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
@@ -537,60 +582,76 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
     // moves whole 16-byte chunks, so chunk positions are unchanged), and rows
     // past the context in the sequence's last page are cleared.
     const int ct = threadIdx.x - kWarpConv * 32;   // 0 .. 127
-    const int last_page = (ctx - 1) / kPage;
-    const int tail_row = ctx % kPage;
-    uint32_t clipped = 0;
-    for (int j = 0; j < nkb; ++j) {
-      const int st = j % NST;
-      if (!__all_sync(0xffffffffu, wait_or_abort(sb + L::kBarVFull + 8 * st, (j / NST) & 1,
-                                                 abort_flag)))
-        break;
-      const uint32_t vst = sb + L::kV + st * L::kStage;
-      const int lp = last_page - j * kPrefillPages;  // this block's page holding the end, if any
-      for (int c = ct; c < L::kStage / 16; c += 128) {
-        const int row = (c >> 3) & (kPrefillKeys - 1);   // key within the block
-        const uint32_t addr = vst + c * 16;
-        uint32_t w[4];
-        if (tail_row != 0 && (row >> 4) == lp && (row & 15) >= tail_row) {
-          w[0] = w[1] = w[2] = w[3] = 0u;
-        } else {
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr));
+    int g0 = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int i = prefill_item_index(k, total);
+      if (i < 0) break;
+      PrefillItem it;
+      if (!prefill_item(a, list, ranked, false, i, it)) continue;
+      const int last_page = (it.ctx - 1) / kPage;
+      const int tail_row = it.ctx % kPage;
+      uint32_t clipped = 0;
+      for (int j = 0; j < it.nkb; ++j) {
+        const int g = g0 + j, st = g % NST;
+        if (!(ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarVFull + 8 * st,
+                                                         (g / NST) & 1, abort_flag))))
+          break;
+        const uint32_t vst = sb + L::kV + st * L::kStage;
+        const int lp = last_page - j * kPrefillPages;  // this block's page holding the end, if any
+        for (int c = ct; c < L::kStage / 16; c += 128) {
+          const int row = (c >> 3) & (kPrefillKeys - 1);   // key within the block
+          const uint32_t addr = vst + c * 16;
+          uint32_t w[4];
+          if (tail_row != 0 && (row >> 4) == lp && (row & 15) >= tail_row) {
+            w[0] = w[1] = w[2] = w[3] = 0u;
+          } else {
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr));
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
-            uint32_t h;
-            asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(hi), "f"(lo));
-            // no bf16 value is 65 504, so a half of magnitude 65 504 was clipped
-            clipped |= __vcmpeq2(h & 0x7fff7fffu, 0x7bff7bffu);
-            w[i] = h;
+            for (int q = 0; q < 4; ++q) {
+              const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xffff0000u);
+              uint32_t h;
+              asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(hi), "f"(lo));
+              // no bf16 value is 65 504, so a half of magnitude 65 504 was clipped
+              clipped |= __vcmpeq2(h & 0x7fff7fffu, 0x7bff7bffu);
+              w[q] = h;
+            }
           }
+          sts128(addr, w[0], w[1], w[2], w[3]);
         }
-        sts128(addr, w[0], w[1], w[2], w[3]);
+        fence_proxy_async_smem();
+        mbar_arrive(sb + L::kBarVConv + 8 * st);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(sb + L::kBarVConv + 8 * st);
+      if (__any_sync(0xffffffffu, clipped != 0) && lane == 0) record_error(kErrValue, it.s);
+      g0 += it.nkb;
     }
-    if (__any_sync(0xffffffffu, clipped != 0) && lane == 0) record_error(kErrValue, s);
   }
   } else {
   // warpgroups 0 and 1: the softmax of tiles A and B
   if constexpr (R::kConvert) regs_increase();
-  if (warp < 4 || has_b) {
-    // ================= softmax: tile t = warp / 4, row = TMEM lane =================
-    const int t = warp >> 2;
-    const int row = threadIdx.x & 127;
-    const int t_begin = t == 0 ? tile_a : tile_b;
-    const int nrows = (min(t_begin + a.tile_tokens, q_len) - t_begin) * G;
-    const int lim = row < nrows ? ctx - q_len + t_begin + row / G + 1 : 0;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t s_col = kTmemS + 128 * t, o_col = kTmemO + 128 * t;
-    const float sl2 = a.scale_log2;
+  // ================= softmax: tile t = warp / 4, row = TMEM lane =================
+  const int t = warp >> 2;
+  const int row = threadIdx.x & 127;
+  const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+  const uint32_t s_col = kTmemS + 128 * t, o_col = kTmemO + 128 * t;
+  const float sl2 = a.scale_log2;
+  int done = 0, items = 0;   // S/P rounds and items of this tile so far
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int i = prefill_item_index(k, total);
+    if (i < 0) break;
+    PrefillItem it;
+    if (!prefill_item(a, list, ranked, false, i, it)) continue;
+    if (t == 1 && !it.has_b) continue;
+    const int t_begin = it.tile_a + t * a.tile_tokens;
+    const int nrows = (min(t_begin + a.tile_tokens, it.q_len) - t_begin) * G;
+    const int lim = row < nrows ? it.ctx - it.q_len + t_begin + row / G + 1 : 0;
     float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nkb; ++j) {
+    for (int j = 0; j < it.nkb; ++j) {
       // S_t(j) is in, and with it every earlier P_t V: O_t is current
-      ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarS + 8 * t, j & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarS + 8 * t, (done + j) & 1,
+                                                 abort_flag));
       if (!ok) break;
       tmem_fence_after_sync();
       float p[kPrefillKeys];
@@ -612,15 +673,15 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
       }
       float mx8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = p[i];
+      for (int q = 0; q < 8; ++q) mx8[q] = p[q];
       static_assert((kPrefillKeys - 8) % 16 == 8, "the key loop below leaves 8 keys for the tail");
 #pragma unroll
       for (int c = 8; c + 16 <= kPrefillKeys; c += 16) {   // keys 8 .. 119
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], p[c + i], p[c + 8 + i]);
+        for (int q = 0; q < 8; ++q) mx8[q] = fmax3(mx8[q], p[c + q], p[c + 8 + q]);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], p[kPrefillKeys - 8 + i]);   // 120 .. 127
+      for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(mx8[q], p[kPrefillKeys - 8 + q]);   // 120 .. 127
       const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
                              fmaxf(mx8[6], mx8[7])) * mul;
       const float m_new = fmaxf(m_ref, mx);
@@ -643,28 +704,28 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
       // remainder p - hi in column 64 + i (lo)
       float2 lsum[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) lsum[i] = make_float2(0.f, 0.f);
+      for (int q = 0; q < 4; ++q) lsum[q] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t h[32], lo[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x0 = p[64 * half + 2 * i], x1 = p[64 * half + 2 * i + 1];
+        for (int q = 0; q < 32; ++q) {
+          const float x0 = p[64 * half + 2 * q], x1 = p[64 * half + 2 * q + 1];
           if constexpr (R::kPHiLo) {
             // hi = the top 16 bits of p (p truncated to bf16, remainder below
             // 2^-7 p), lo = the exact fp32 remainder p - hi >= 0 truncated the
             // same way: P keeps at least 14 significant bits (error < 2^-14 p),
             // with no rounding arithmetic and no conversion-unit work
             const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
-            h[i] = __byte_perm(b0, b1, 0x7632);
+            h[q] = __byte_perm(b0, b1, 0x7632);
             const float2 r = ffma2(make_float2(__uint_as_float(b0 & 0xffff0000u),
                                                __uint_as_float(b1 & 0xffff0000u)),
                                    make_float2(-1.f, -1.f), make_float2(x0, x1));
-            lo[i] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
-            lsum[i & 3] = ffma2(make_float2(x0, x1), make_float2(1.f, 1.f), lsum[i & 3]);
+            lo[q] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
+            lsum[q & 3] = ffma2(make_float2(x0, x1), make_float2(1.f, 1.f), lsum[q & 3]);
           } else {
-            h[i] = pack2<false>(x0, x1);
-            lsum[i & 3] = ffma2(unpack2<false>(h[i]), make_float2(1.f, 1.f), lsum[i & 3]);
+            h[q] = pack2<false>(x0, x1);
+            lsum[q & 3] = ffma2(unpack2<false>(h[q]), make_float2(1.f, 1.f), lsum[q & 3]);
           }
         }
         tmem_st32u(t_lane + s_col + 32 * half, h);
@@ -678,36 +739,41 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
           float o[32];
           tmem_ld32(t_lane + o_col + 32 * c, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          for (int q = 0; q < 32; ++q) o[q] *= alpha;
           tmem_st32(t_lane + o_col + 32 * c, o);
         }
       }
       tmem_fence_before_sync();
       mbar_arrive(sb + L::kBarP + 8 * t);
     }
-    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarO, 0, abort_flag));
-    if (ok) {
-      tmem_fence_after_sync();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint16_t* o_row = a.out + (static_cast<size_t>(q0 + t_begin + row / G) * a.num_heads +
-                                 kvh * G + row % G) * D;
+    if (!ok) break;
+    done += it.nkb;
+    // the item's last P_t V is done: O_t is final
+    ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarOFull + 8 * t, items & 1, abort_flag));
+    if (!ok) break;
+    tmem_fence_after_sync();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    uint16_t* o_row = a.out + (static_cast<size_t>(it.q0 + t_begin + row / G) * a.num_heads +
+                               it.kvh * G + row % G) * D;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tmem_ld32(t_lane + o_col + 32 * c, o);
-        if (row < nrows) {
+    for (int c = 0; c < D / 32; ++c) {
+      float o[32];
+      tmem_ld32(t_lane + o_col + 32 * c, o);
+      if (row < nrows) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 v;
-            v.x = pack2<BF16>(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
-            v.y = pack2<BF16>(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
-            v.z = pack2<BF16>(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
-            v.w = pack2<BF16>(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
-            *reinterpret_cast<uint4*>(o_row + 32 * c + 8 * q) = v;
-          }
+        for (int q = 0; q < 4; ++q) {
+          uint4 v;
+          v.x = pack2<BF16>(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+          v.y = pack2<BF16>(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+          v.z = pack2<BF16>(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+          v.w = pack2<BF16>(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+          *reinterpret_cast<uint4*>(o_row + 32 * c + 8 * q) = v;
         }
       }
     }
+    tmem_fence_before_sync();
+    mbar_arrive(sb + L::kBarOFree + 8 * t);   // O_t may be overwritten
+    ++items;
   }
   }
 

@@ -46,8 +46,8 @@ def _mixed(seed, n, ctx_hi, q_hi):
     return tuple(ctx), tuple(q)
 
 
-# 40 sequences: the longest-first order ranks units across several 32-sequence
-# chunks, with many equal key counts and empty sequences among them
+# 40 sequences: the longest-first order ranks units with many equal key counts
+# and empty sequences among them
 _ctx, _q = _mixed(444_071, 40, 300, 70)
 CASES["many_seqs_gqa4_bf16"] = (C["gqa_llama3_8b"], dict(num_seqs=40, num_heads=8,
                                                           num_kv_heads=2, num_blocks=1000,
@@ -58,6 +58,15 @@ CASES["fixed_order_300_seqs_f16"] = (C["gqa_llama3_8b"], dict(num_seqs=300, num_
                                                                num_kv_heads=2, dtype="f16",
                                                                num_blocks=1200,
                                                                ctx=("fixed", _ctx), seed=72), _q)
+# few enough sequences to rank, but too many units x sequences to count: the
+# fixed order again, with the sequences checked while the units are counted
+_ctx, _q = _mixed(444_073, 100, 500, 300)
+CASES["fixed_order_100_seqs_bf16"] = (C["gqa_llama3_8b"], dict(num_seqs=100, num_heads=4,
+                                                                num_kv_heads=1, num_blocks=3600,
+                                                                ctx=("fixed", _ctx), seed=73), _q)
+_units = sum(-(-q // (2 * 32)) for q in _q)                # tile pairs of 2 x 32 tokens
+assert _units <= 2048 and _units * 100 > 16384, _units
+
 # scale 1 instead of 1/sqrt(D): peaked rows whose running maximum jumps by more
 # than 2^8 between key blocks, so the output accumulator is rescaled
 SCALE = {"peaky_bf16": 1.0, "peaky_f16": 1.0}
