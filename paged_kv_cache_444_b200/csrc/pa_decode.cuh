@@ -576,7 +576,7 @@ __device__ __forceinline__ bool decode_item(const CUtensorMap& kmap, const CUten
 }
 
 template <int D, int NST, bool BF16, class Warp, int EB = 2>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, EB == 1 ? 3 : 0)  // fp8: three CTAs per SM
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
   using L = DecodeSmem<D, NST, EB>;
