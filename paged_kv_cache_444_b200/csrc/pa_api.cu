@@ -1100,8 +1100,8 @@ extern "C" pa_status pa_prefill(void* out, const void* query, const void* key_ca
   if (num_query_tokens * num_heads > INT32_MAX || max_query_len > INT32_MAX) return PA_ERR_SHAPE;
   const int64_t G = num_heads / num_kv_heads;
   const int64_t tile = kPrefillRows / G;                  // G <= 16 checked above
-  const int64_t tiles = (max_query_len + tile - 1) / tile;
-  const int64_t pairs = (tiles + 1) / 2;                  // two query tiles per CTA
+  const int64_t span = 2 * tile;                          // two query tiles per CTA
+  const int64_t pairs = (max_query_len + span - 1) / span;
   const long long items = num_seqs * num_kv_heads * pairs;   // (sequence, KV head, tile pair)
   if (items > INT32_MAX) return PA_ERR_SHAPE;
   CUtensorMap qm, km, vm;

@@ -197,10 +197,9 @@ __device__ __forceinline__ int pairs_above_of(int hist, int q_len, int pairs, in
   return x < 0 ? pairs : pairs - div_floor(x, t2, inv_t2);  // T2 (p + 1) <= x fall short
 }
 
-// The k-th item of this CTA (snake order), or -1 past the last.
-__device__ __forceinline__ int prefill_item_index(int k, int total) {
-  const long long g = gridDim.x, b = blockIdx.x;
-  const long long i = k * g + ((k & 1) ? g - 1 - b : b);
+// The k-th item of CTA b of g, snake order, or -1 past the last.
+__device__ __forceinline__ int prefill_item_index(int k, int total, int b, int g) {
+  const long long i = static_cast<long long>(k) * g + ((k & 1) ? g - 1 - b : b);
   return i < total ? static_cast<int>(i) : -1;
 }
 
@@ -210,9 +209,10 @@ struct PrefillItem {
 };
 
 // Item i; false when it has no work (a pair its sequence does not have, or an
-// invalid sequence, reported once when `report`).
+// invalid sequence, reported once when `report`).  A tile pair covers `span`
+// query tokens, tile A the first half and tile B the second.
 __device__ __forceinline__ bool prefill_item(const PrefillArgs& a, const int* list, bool ranked,
-                                             bool report, int i, PrefillItem& it) {
+                                             bool report, int i, int span, PrefillItem& it) {
   const int r = i / a.num_kv_heads;
   it.kvh = i - r * a.num_kv_heads;
   int p;
@@ -233,15 +233,209 @@ __device__ __forceinline__ bool prefill_item(const PrefillArgs& a, const int* li
     if (report && it.kvh == 0 && p == 0) record_error(kErrQuery, it.s);
     return false;
   }
-  it.tile_a = 2 * p * a.tile_tokens;
+  it.tile_a = p * span;
   if (it.tile_a >= it.q_len) return false;
-  const int tile_b = it.tile_a + a.tile_tokens;
+  const int half = span / 2;
+  const int tile_b = it.tile_a + half;
   it.has_b = tile_b < it.q_len;
-  const int last_tok = min((it.has_b ? tile_b : it.tile_a) + a.tile_tokens, it.q_len);
+  const int last_tok = min((it.has_b ? tile_b : it.tile_a) + half, it.q_len);
   const int lim_max = it.ctx - it.q_len + last_tok;   // keys the pair's last token sees
   it.n_pages = (lim_max + kPage - 1) / kPage;
   it.nkb = (it.n_pages + kPrefillPages - 1) / kPrefillPages;
   return true;
+}
+
+// One 128-key block of a tile's online softmax, thread = row (tensor-memory
+// lane): S of keys j*128 .. j*128 + 127 (fp32, in p) -> P written over S in
+// tensor memory as 16-bit (for PHiLo, bf16 hi + lo in two column halves),
+// l and the reference maximum m_ref updated, O_t rescaled in tensor memory
+// when m_ref moves.  lim = keys this row sees.
+template <bool PHiLo, int D>
+__device__ __forceinline__ void prefill_softmax_block(float (&p)[kPrefillKeys], int j, int lim,
+                                                      float sl2, float& m_ref, float& l,
+                                                      uint32_t t_lane, uint32_t s_col,
+                                                      uint32_t o_col) {
+  // keys at or past this row's limit are -inf
+  const int kbase = j * kPrefillKeys;
+  if (kbase + kPrefillKeys > lim) {
+#pragma unroll
+    for (int c = 0; c < kPrefillKeys; ++c) p[c] = kbase + c < lim ? p[c] : -INFINITY;
+  }
+  // the block's largest logit in log2 units: for scale > 0 the maximum of
+  // the raw S (three-input max), scaled once; otherwise S is scaled first
+  float mul = sl2;
+  if (!(sl2 > 0.f)) {
+#pragma unroll
+    for (int c = 0; c < kPrefillKeys; ++c) p[c] = p[c] == -INFINITY ? -INFINITY : p[c] * sl2;
+    mul = 1.f;
+  }
+  float mx8[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) mx8[q] = p[q];
+  static_assert((kPrefillKeys - 8) % 16 == 8, "the key loop below leaves 8 keys for the tail");
+#pragma unroll
+  for (int c = 8; c + 16 <= kPrefillKeys; c += 16) {   // keys 8 .. 119
+#pragma unroll
+    for (int q = 0; q < 8; ++q) mx8[q] = fmax3(mx8[q], p[c + q], p[c + 8 + q]);
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(mx8[q], p[kPrefillKeys - 8 + q]);   // 120 .. 127
+  const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                         fmaxf(mx8[6], mx8[7])) * mul;
+  const float m_new = fmaxf(m_ref, mx);
+  const bool need = m_new > m_ref + kRescaleSlack;
+  float alpha = 1.f;
+  if (need) {
+    alpha = ex2(m_ref - m_new);   // 0 when m_ref is still -inf
+    m_ref = m_new;
+  }
+  l *= alpha;
+  const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+  const float2 negm = make_float2(-m_use, -m_use), mul2 = make_float2(mul, mul);
+#pragma unroll
+  for (int c = 0; c < kPrefillKeys; c += 2) {
+    const float2 x = ffma2(make_float2(p[c], p[c + 1]), mul2, negm);   // S * scale - m
+    p[c] = ex2(x.x);
+    p[c + 1] = ex2(x.y);
+  }
+  // P (and l) over S_t: keys 2i, 2i+1 packed in column i (hi); for bf16 the
+  // remainder p - hi in column 64 + i (lo)
+  float2 lsum[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) lsum[q] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t h[32], lo[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      const float x0 = p[64 * half + 2 * q], x1 = p[64 * half + 2 * q + 1];
+      if constexpr (PHiLo) {
+        // hi = the top 16 bits of p (p truncated to bf16, remainder below
+        // 2^-7 p), lo = the exact fp32 remainder p - hi >= 0 truncated the
+        // same way: P keeps at least 14 significant bits (error < 2^-14 p),
+        // with no rounding arithmetic and no conversion-unit work
+        const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
+        h[q] = __byte_perm(b0, b1, 0x7632);
+        const float2 r = ffma2(make_float2(__uint_as_float(b0 & 0xffff0000u),
+                                           __uint_as_float(b1 & 0xffff0000u)),
+                               make_float2(-1.f, -1.f), make_float2(x0, x1));
+        lo[q] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
+        lsum[q & 3] = ffma2(make_float2(x0, x1), make_float2(1.f, 1.f), lsum[q & 3]);
+      } else {
+        h[q] = pack2<false>(x0, x1);
+        lsum[q & 3] = ffma2(unpack2<false>(h[q]), make_float2(1.f, 1.f), lsum[q & 3]);
+      }
+    }
+    tmem_st32u(t_lane + s_col + 32 * half, h);
+    if constexpr (PHiLo) tmem_st32u(t_lane + s_col + 64 + 32 * half, lo);
+  }
+  l += ((lsum[0].x + lsum[0].y) + (lsum[1].x + lsum[1].y)) +
+       ((lsum[2].x + lsum[2].y) + (lsum[3].x + lsum[3].y));
+  if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      float o[32];
+      tmem_ld32(t_lane + o_col + 32 * c, o);
+#pragma unroll
+      for (int q = 0; q < 32; ++q) o[q] *= alpha;
+      tmem_st32(t_lane + o_col + 32 * c, o);
+    }
+  }
+}
+
+// The epilogue of a tile, thread = row: O_t / l from tensor memory as the
+// output dtype, for rows below nrows (row r = token t_begin + r / G, head
+// kvh * G + r % G of the query rows starting at q0).
+template <bool BF16, int D>
+__device__ __forceinline__ void prefill_store_rows(const PrefillArgs& a, uint32_t t_lane,
+                                                   uint32_t o_col, float l, int row, int nrows,
+                                                   int q0, int t_begin, int kvh) {
+  const int G = a.group;
+  tmem_fence_after_sync();
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  uint16_t* o_row = a.out + (static_cast<size_t>(q0 + t_begin + row / G) * a.num_heads +
+                             kvh * G + row % G) * D;
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    float o[32];
+    tmem_ld32(t_lane + o_col + 32 * c, o);
+    if (row < nrows) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 v;
+        v.x = pack2<BF16>(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+        v.y = pack2<BF16>(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+        v.z = pack2<BF16>(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+        v.w = pack2<BF16>(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+        *reinterpret_cast<uint4*>(o_row + 32 * c + 8 * q) = v;
+      }
+    }
+  }
+}
+
+// Ranks the units longest first into `list` (unit of each rank: s | p << 16),
+// the same order in every CTA; every thread of the CTA calls it.  t2 = query
+// tokens per unit.  Returns false (nothing ranked) for batches past the
+// limits, which take the fixed order.  Invalid sequences are reported here.
+__device__ __forceinline__ bool prefill_rank_units(const PrefillArgs& a, int t2, int* sched,
+                                                   int4* seqs, int* list, int warp, int lane) {
+  if (a.num_seqs > kRankMaxSeqs) return false;
+  bool ranked = false;
+  const int t = threadIdx.x;
+  int hist = 0, ql = -1, np = 0;
+  if (t < a.num_seqs) {
+    const int q0 = a.query_starts[t], len = a.query_starts[t + 1] - q0;
+    const int ctx = a.context_lens[t];
+    if (q0 < 0 || len < 0 || q0 > a.num_tokens - len || len > ctx ||
+        ctx > a.max_blocks_per_seq * kPage) {
+      if (t % gridDim.x == blockIdx.x) record_error(kErrQuery, t);  // one CTA reports it
+    } else {
+      hist = ctx - len;
+      ql = len;
+      np = len / t2 + (len % t2 != 0);
+    }
+  }
+  int first = np;  // inclusive scan over the warp's sequences
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, first, d);
+    if (lane >= d) first += v;
+  }
+  if (lane == 31 && warp < kRankMaxSeqs / 32) sched[4 + warp] = first;
+  __syncthreads();
+  if (t < a.num_seqs) {
+    for (int w = 0; w < warp; ++w) first += sched[4 + w];
+    seqs[t] = make_int4(hist, ql, np, first - np);
+    if (t == a.num_seqs - 1) sched[0] = first;
+  }
+  __syncthreads();
+  const int n_units = sched[0];
+  ranked = n_units <= kRankMaxUnits &&
+           static_cast<long long>(n_units) * a.num_seqs <= kRankMaxWork;
+  if (ranked) {
+    const float inv_t2 = 1.f / static_cast<float>(t2);
+    for (int u = t; u < n_units; u += blockDim.x) {
+      int lo = 0, hi = a.num_seqs;  // the owner: the last sequence whose first unit is <= u
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (seqs[mid].w <= u) lo = mid;
+        else hi = mid;
+      }
+      const int4 me = seqs[lo];
+      const int p = u - me.w;
+      const int K = me.x + min(t2 * (p + 1), me.y);
+      int rank = 0;
+      for (int i = 0; i < a.num_seqs; ++i) {
+        const int4 o = seqs[i];
+        const int gt = pairs_above_of(o.x, o.y, o.z, t2, inv_t2, K);
+        rank += gt;
+        if (i < lo) rank += pairs_above_of(o.x, o.y, o.z, t2, inv_t2, K - 1) - gt;
+      }
+      list[rank] = lo | (p << 16);
+    }
+    __syncthreads();
+  }
+  return ranked;
 }
 
 template <int D, bool BF16>
@@ -272,66 +466,10 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
   int4* seqs = reinterpret_cast<int4*>(smem + L::kSeqs);   // hist, q_len, pairs, first unit
   int* list = reinterpret_cast<int*>(smem + L::kList);     // unit of each rank: s | p << 16
   const bool table = a.num_seqs <= kRankMaxSeqs;
-  bool ranked = false;
-  if (table) {
-    const int t = threadIdx.x;
-    int hist = 0, ql = -1, np = 0;
-    if (t < a.num_seqs) {
-      const int q0 = a.query_starts[t], len = a.query_starts[t + 1] - q0;
-      const int ctx = a.context_lens[t];
-      if (q0 < 0 || len < 0 || q0 > a.num_tokens - len || len > ctx ||
-          ctx > a.max_blocks_per_seq * kPage) {
-        if (t % gridDim.x == blockIdx.x) record_error(kErrQuery, t);  // one CTA reports it
-      } else {
-        hist = ctx - len;
-        ql = len;
-        np = len / t2 + (len % t2 != 0);
-      }
-    }
-    int first = np;  // inclusive scan over the warp's sequences
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, first, d);
-      if (lane >= d) first += v;
-    }
-    if (lane == 31 && warp < kRankMaxSeqs / 32) sched[4 + warp] = first;
-    __syncthreads();
-    if (t < a.num_seqs) {
-      for (int w = 0; w < warp; ++w) first += sched[4 + w];
-      seqs[t] = make_int4(hist, ql, np, first - np);
-      if (t == a.num_seqs - 1) sched[0] = first;
-    }
-    __syncthreads();
-    const int n_units = sched[0];
-    ranked = n_units <= kRankMaxUnits &&
-             static_cast<long long>(n_units) * a.num_seqs <= kRankMaxWork;
-    if (ranked) {
-      const float inv_t2 = 1.f / static_cast<float>(t2);
-      for (int u = t; u < n_units; u += blockDim.x) {
-        int lo = 0, hi = a.num_seqs;  // the owner: the last sequence whose first unit is <= u
-        while (hi - lo > 1) {
-          const int mid = (lo + hi) >> 1;
-          if (seqs[mid].w <= u) lo = mid;
-          else hi = mid;
-        }
-        const int4 me = seqs[lo];
-        const int p = u - me.w;
-        const int K = me.x + min(t2 * (p + 1), me.y);
-        int rank = 0;
-        for (int i = 0; i < a.num_seqs; ++i) {
-          const int4 o = seqs[i];
-          const int gt = pairs_above_of(o.x, o.y, o.z, t2, inv_t2, K);
-          rank += gt;
-          if (i < lo) rank += pairs_above_of(o.x, o.y, o.z, t2, inv_t2, K - 1) - gt;
-        }
-        list[rank] = lo | (p << 16);
-      }
-      __syncthreads();
-    }
-  }
+  const bool ranked = prefill_rank_units(a, t2, sched, seqs, list, warp, lane);
   const int total = ranked ? sched[0] * a.num_kv_heads
                            : a.num_seqs * a.num_kv_heads * a.pairs_per_seq;
-  if (prefill_item_index(0, total) < 0) return;   // more CTAs than items
+  if (prefill_item_index(0, total, blockIdx.x, gridDim.x) < 0) return;   // more CTAs than items
   const bool report = !table && warp == kWarpTma && lane == 0;
   const int q_rows = a.tile_tokens * G;           // rows a Q box fills
 
@@ -383,10 +521,10 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
     int n_q = 0, k_issued = 0, v_issued = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int i = prefill_item_index(k, total);
+      const int i = prefill_item_index(k, total, blockIdx.x, gridDim.x);
       if (i < 0) break;
       PrefillItem it;
-      if (!prefill_item(a, list, ranked, report, i, it)) continue;
+      if (!prefill_item(a, list, ranked, report, i, t2, it)) continue;
       if (n_q > 0 && !(ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarQFree,
                                                                   (n_q - 1) & 1, abort_flag))))
         break;
@@ -513,10 +651,10 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
     int n_q = 0, g0 = 0, done[2] = {0, 0}, items[2] = {0, 0};
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int i = prefill_item_index(k, total);
+      const int i = prefill_item_index(k, total, blockIdx.x, gridDim.x);
       if (i < 0) break;
       PrefillItem it;
-      if (!prefill_item(a, list, ranked, false, i, it)) continue;
+      if (!prefill_item(a, list, ranked, false, i, t2, it)) continue;
       const bool hb = it.has_b;
       const int nkb = it.nkb;
       // before the first P_t V of an item: the epilogue has read O_t of the last one
@@ -585,10 +723,10 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
     int g0 = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int i = prefill_item_index(k, total);
+      const int i = prefill_item_index(k, total, blockIdx.x, gridDim.x);
       if (i < 0) break;
       PrefillItem it;
-      if (!prefill_item(a, list, ranked, false, i, it)) continue;
+      if (!prefill_item(a, list, ranked, false, i, t2, it)) continue;
       const int last_page = (it.ctx - 1) / kPage;
       const int tail_row = it.ctx % kPage;
       uint32_t clipped = 0;
@@ -639,10 +777,10 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
   int done = 0, items = 0;   // S/P rounds and items of this tile so far
   bool ok = true;
   for (int k = 0; ok; ++k) {
-    const int i = prefill_item_index(k, total);
+    const int i = prefill_item_index(k, total, blockIdx.x, gridDim.x);
     if (i < 0) break;
     PrefillItem it;
-    if (!prefill_item(a, list, ranked, false, i, it)) continue;
+    if (!prefill_item(a, list, ranked, false, i, t2, it)) continue;
     if (t == 1 && !it.has_b) continue;
     const int t_begin = it.tile_a + t * a.tile_tokens;
     const int nrows = (min(t_begin + a.tile_tokens, it.q_len) - t_begin) * G;
@@ -657,92 +795,7 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
       float p[kPrefillKeys];
       if constexpr (R::kConvert) tmem_ld128_x32(t_lane + s_col, p);
       else tmem_ld128(t_lane + s_col, p);
-      // keys at or past this row's limit are -inf
-      const int kbase = j * kPrefillKeys;
-      if (kbase + kPrefillKeys > lim) {
-#pragma unroll
-        for (int c = 0; c < kPrefillKeys; ++c) p[c] = kbase + c < lim ? p[c] : -INFINITY;
-      }
-      // the block's largest logit in log2 units: for scale > 0 the maximum of
-      // the raw S (three-input max), scaled once; otherwise S is scaled first
-      float mul = sl2;
-      if (!(sl2 > 0.f)) {
-#pragma unroll
-        for (int c = 0; c < kPrefillKeys; ++c) p[c] = p[c] == -INFINITY ? -INFINITY : p[c] * sl2;
-        mul = 1.f;
-      }
-      float mx8[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) mx8[q] = p[q];
-      static_assert((kPrefillKeys - 8) % 16 == 8, "the key loop below leaves 8 keys for the tail");
-#pragma unroll
-      for (int c = 8; c + 16 <= kPrefillKeys; c += 16) {   // keys 8 .. 119
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mx8[q] = fmax3(mx8[q], p[c + q], p[c + 8 + q]);
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(mx8[q], p[kPrefillKeys - 8 + q]);   // 120 .. 127
-      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                             fmaxf(mx8[6], mx8[7])) * mul;
-      const float m_new = fmaxf(m_ref, mx);
-      const bool need = m_new > m_ref + kRescaleSlack;
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2(m_ref - m_new);   // 0 when m_ref is still -inf
-        m_ref = m_new;
-      }
-      l *= alpha;
-      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-      const float2 negm = make_float2(-m_use, -m_use), mul2 = make_float2(mul, mul);
-#pragma unroll
-      for (int c = 0; c < kPrefillKeys; c += 2) {
-        const float2 x = ffma2(make_float2(p[c], p[c + 1]), mul2, negm);   // S * scale - m
-        p[c] = ex2(x.x);
-        p[c + 1] = ex2(x.y);
-      }
-      // P (and l) over S_t: keys 2i, 2i+1 packed in column i (hi); for bf16 the
-      // remainder p - hi in column 64 + i (lo)
-      float2 lsum[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) lsum[q] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t h[32], lo[32];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const float x0 = p[64 * half + 2 * q], x1 = p[64 * half + 2 * q + 1];
-          if constexpr (R::kPHiLo) {
-            // hi = the top 16 bits of p (p truncated to bf16, remainder below
-            // 2^-7 p), lo = the exact fp32 remainder p - hi >= 0 truncated the
-            // same way: P keeps at least 14 significant bits (error < 2^-14 p),
-            // with no rounding arithmetic and no conversion-unit work
-            const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
-            h[q] = __byte_perm(b0, b1, 0x7632);
-            const float2 r = ffma2(make_float2(__uint_as_float(b0 & 0xffff0000u),
-                                               __uint_as_float(b1 & 0xffff0000u)),
-                                   make_float2(-1.f, -1.f), make_float2(x0, x1));
-            lo[q] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
-            lsum[q & 3] = ffma2(make_float2(x0, x1), make_float2(1.f, 1.f), lsum[q & 3]);
-          } else {
-            h[q] = pack2<false>(x0, x1);
-            lsum[q & 3] = ffma2(unpack2<false>(h[q]), make_float2(1.f, 1.f), lsum[q & 3]);
-          }
-        }
-        tmem_st32u(t_lane + s_col + 32 * half, h);
-        if constexpr (R::kPHiLo) tmem_st32u(t_lane + s_col + 64 + 32 * half, lo);
-      }
-      l += ((lsum[0].x + lsum[0].y) + (lsum[1].x + lsum[1].y)) +
-           ((lsum[2].x + lsum[2].y) + (lsum[3].x + lsum[3].y));
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          float o[32];
-          tmem_ld32(t_lane + o_col + 32 * c, o);
-#pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] *= alpha;
-          tmem_st32(t_lane + o_col + 32 * c, o);
-        }
-      }
+      prefill_softmax_block<R::kPHiLo, D>(p, j, lim, sl2, m_ref, l, t_lane, s_col, o_col);
       tmem_fence_before_sync();
       mbar_arrive(sb + L::kBarP + 8 * t);
     }
@@ -751,26 +804,7 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
     // the item's last P_t V is done: O_t is final
     ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarOFull + 8 * t, items & 1, abort_flag));
     if (!ok) break;
-    tmem_fence_after_sync();
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    uint16_t* o_row = a.out + (static_cast<size_t>(it.q0 + t_begin + row / G) * a.num_heads +
-                               it.kvh * G + row % G) * D;
-#pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
-      float o[32];
-      tmem_ld32(t_lane + o_col + 32 * c, o);
-      if (row < nrows) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 v;
-          v.x = pack2<BF16>(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
-          v.y = pack2<BF16>(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
-          v.z = pack2<BF16>(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
-          v.w = pack2<BF16>(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
-          *reinterpret_cast<uint4*>(o_row + 32 * c + 8 * q) = v;
-        }
-      }
-    }
+    prefill_store_rows<BF16, D>(a, t_lane, o_col, l, row, nrows, it.q0, t_begin, it.kvh);
     tmem_fence_before_sync();
     mbar_arrive(sb + L::kBarOFree + 8 * t);   // O_t may be overwritten
     ++items;
