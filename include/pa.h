@@ -319,7 +319,8 @@ pa_status pa_decode_step_host(void *out_host, const void *query_host, const void
  *   query, out     [num_query_tokens, num_heads, head_dim], rows grouped by sequence
  *   query_starts   [num_seqs + 1] int32, query_starts[0] = 0, nondecreasing,
  *                  query_starts[num_seqs] = num_query_tokens
- *   max_query_len  host-side upper bound of every q_len (sizes the grid)
+ *   max_query_len  host-side upper bound of every q_len (bounds the work list; the
+ *                  grid is persistent, at most one CTA per SM)
  * Other arguments as pa_decode.  A sequence with q_len > context_lens[s] is
  * skipped and reported (PA_CHECK_QUERY).  fp32 accumulation.  P enters the
  * P.V product as fp16 (11 bits).  With bf16 caches each V block is first
