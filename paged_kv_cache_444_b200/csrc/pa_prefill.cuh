@@ -23,7 +23,15 @@
 // thread run in issue order: S_t(j+1) may overwrite P_t(j) as soon as it is
 // issued after the P V that reads it, and the commit that reports S_t(j+1)
 // also reports that P V done (the softmax may then rescale O_t).  Another warp
-// loads Q once and the K and V pages with TMA through rings of NST stages.
+// loads each item's Q and the K and V pages with TMA through rings of NST
+// stages.
+//
+// The grid is persistent, one CTA per SM: each CTA walks its share of the
+// items (ordered longest first, see below) with every ring and phase running
+// on from item to item, and hands items over with three barriers (Q free: the
+// item's S products are done; O full / O free per tile: its last P V is done,
+// its epilogue has read O), so an item's epilogue and Q load overlap the
+// neighbouring item's products.
 //
 // The causal mask is a per-row key limit (pos + 1) applied to S; blocks past
 // the pair's last key are never loaded, and V rows past the context are
