@@ -346,6 +346,16 @@ pa_status pa_prefill(void *out, const void *query, const void *key_cache,
 pa_status pa_check_error(void *stream, int64_t *detail);
 
 /*
+ * pa_selftest_wait_timeout -- the failure path of every kernel's shared-memory
+ * barrier waits, exercised on purpose: one CTA waits on an mbarrier that
+ * nothing completes, with the kernels' own bounded wait (2 s of %globaltimer),
+ * then records PA_CHECK_WAIT_TIMEOUT (index 0) and returns.  No memory is
+ * touched and the device context stays usable; pa_check_error then reports
+ * the timeout.  Asynchronous on `stream` like every launch.
+ */
+pa_status pa_selftest_wait_timeout(void *stream);
+
+/*
  * pa_decode_noalloc -- the long-context decode of pa_decode_split followed by
  * pa_reduce, for callers that cannot allocate device memory when they call.
  * The pages have no counterpart of this entry point: it exists for

@@ -13,13 +13,14 @@ import torch
 from ._lib import (DecodePlan, HostStep, PagedAttentionError, load, pa_check_error, pa_copy_blocks, pa_decode,
                    pa_decode_fp8, pa_decode_noalloc, pa_decode_shared_prefix, pa_decode_split,
                    pa_decode_split_fp8, pa_prefill, pa_reduce, pa_reshape_and_cache,
-                   pa_reshape_and_cache_fp8)
+                   pa_reshape_and_cache_fp8, pa_selftest_wait_timeout)
 
 __all__ = [
     "PagedAttentionError", "load", "pa_reshape_and_cache", "pa_decode", "pa_decode_split",
     "pa_reduce", "pa_check_error", "pa_decode_noalloc", "pa_decode_shared_prefix",
     "pa_copy_blocks", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_decode_split_fp8",
-    "pa_prefill", "SplitWorkspace", "decode_step", "HostStep", "DecodePlan",
+    "pa_prefill", "pa_selftest_wait_timeout", "SplitWorkspace", "decode_step", "HostStep",
+    "DecodePlan",
 ]
 
 

@@ -56,6 +56,7 @@ SIGNATURES = {
                              _i64, _i64, _i64, _i64, _i, _p]),
     "pa_reduce": (_i, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i, _p]),
     "pa_check_error": (_i, [_p, ctypes.POINTER(_i64)]),
+    "pa_selftest_wait_timeout": (_i, [_p]),
     "pa_decode_noalloc": (_i, [_p, _p, _p, _p, _p, _p, _f, _i64, _i64, _i64, _i64, _i64, _i64,
                                _i64, _i64, _i, _p]),
     "pa_decode_shared_prefix": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _f, _i64, _i64, _i64, _i64,
@@ -502,6 +503,13 @@ def pa_check_error(stream=None) -> int:
     if st != PA_OK:
         raise PagedAttentionError(st, "pa_check_error", int(detail.value))
     return 0
+
+
+def pa_selftest_wait_timeout(stream=None) -> None:
+    """Run the bounded-wait failure path on purpose: a kernel waits (2 s) on a
+    barrier nothing completes and records PA_CHECK_WAIT_TIMEOUT, which the
+    next pa_check_error reports."""
+    _check(load().pa_selftest_wait_timeout(_stream(stream)), "pa_selftest_wait_timeout")
 
 
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024

@@ -845,6 +845,29 @@ pa_status pa_check_error(void* stream, int64_t* detail) {
 }
 
 }  // extern "C"
+// >>> self-test of the bounded barrier wait (pa_selftest_wait_timeout): one
+// CTA waits, with the kernels' own bounded wait, on an mbarrier that nothing
+// completes, and records the timeout the way every kernel does.
+namespace {
+__global__ void wait_timeout_selftest_kernel() {
+  __shared__ alignas(8) uint64_t bar;
+  const uint32_t b = pa::smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    pa::mbar_init(b, 1);   // one arrival completes phase 0; none is made
+    pa::fence_barrier_init();
+  }
+  __syncthreads();
+  const bool landed = pa::mbar_wait_bounded(b, 0);
+  if (!__all_sync(0xffffffffu, landed) && threadIdx.x == 0)
+    pa::record_error(pa::kErrWaitTimeout, blockIdx.x);
+}
+}  // namespace
+
+extern "C" pa_status pa_selftest_wait_timeout(void* stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>();
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+// <<< self-test of the bounded barrier wait
 
 // >>> no-allocation entry point (pa_decode_noalloc): split decode + merge
 // with the partition scratch in a fixed device array of this file (declared

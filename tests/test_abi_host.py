@@ -135,6 +135,7 @@ def test_valid_call_without_gpu_reports_cuda_error(lib):
     assert _decode(lib) == CUDA
     detail = ctypes.c_int64(0)
     assert lib.pa_check_error(None, ctypes.byref(detail)) == CUDA
+    assert lib.pa_selftest_wait_timeout(None) == CUDA
 
 
 def test_binding_raises_without_library(tmp_path):

@@ -539,3 +539,26 @@ def test_empty_batch_is_a_no_op(dev):
     pa_decode(out, b.query[:0], b.key_cache, b.value_cache, b.block_tables[:0],
               b.context_lens[:0], cfg.scale)
     torch.cuda.synchronize()
+
+
+def test_bounded_wait_gives_up_and_context_stays_usable(dev, oracle_lib):
+    """The failure path of every kernel's barrier waits, taken on purpose: a
+    kernel waits on a barrier that nothing completes, gives up after the
+    bounded wait, records PA_CHECK_WAIT_TIMEOUT and returns.  pa_check_error
+    reports it once, and a decode launched afterwards in the same context
+    still matches the oracle."""
+    from paged_kv_cache_444_b200 import pa_selftest_wait_timeout
+    pa_check_error()                                  # start from a clean error word
+    pa_selftest_wait_timeout()
+    with pytest.raises(PagedAttentionError) as e:
+        pa_check_error()
+    assert e.value.detail >> 56 == 5                  # PA_CHECK_WAIT_TIMEOUT
+    assert pa_check_error() == 0                      # reported once, then cleared
+    cfg = SMALL["gqa_small"]
+    batch = workloads.make_batch(cfg, dev)
+    host = HostCopy(batch)
+    ref, kc_ref, _ = oracle_step(oracle_lib, host)
+    out, _ = gpu_step(batch)
+    pa_check_error()
+    assert np.array_equal(bits(batch.key_cache), kc_ref)
+    _check_close(out, ref, cfg, "decode after a barrier timeout")
