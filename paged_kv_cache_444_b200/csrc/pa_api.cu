@@ -1146,7 +1146,6 @@ extern "C" pa_status pa_prefill(void* out, const void* query, const void* key_ca
   a.max_blocks_per_seq = static_cast<int>(max_blocks_per_seq);
   a.num_blocks = static_cast<int>(num_blocks);
   a.tile_tokens = static_cast<int>(tile);
-  a.pairs_per_seq = static_cast<int>(pairs);
   cudaStream_t s = as_stream(stream);
   const bool bf16 = dtype == PA_BF16;
   if (head_dim == 64)

@@ -111,7 +111,6 @@ struct PrefillArgs {
   int max_blocks_per_seq;
   int num_blocks;
   int tile_tokens;              // query tokens per tile (128 / group, rounded down)
-  int pairs_per_seq;            // ceil(ceil(max_query_len / tile_tokens) / 2)
 };
 
 template <int D, bool BF16>
@@ -138,8 +137,8 @@ struct PrefillSmem {
   static constexpr int kBarOFree = kBarOFull + 16;     // per tile: O read by the epilogue
   static constexpr int kTmemSlot = kBarOFree + 16;
   static constexpr int kAbort = kTmemSlot + 4;
-  static constexpr int kSched = kAbort + 4;            // unit count and per-warp sums (16 ints)
-  static constexpr int kSeqs = (kSched + 64 + 15) & ~15;   // int4 per sequence while ranking
+  static constexpr int kSched = kAbort + 4;            // unit count and per-warp sums (32 ints)
+  static constexpr int kSeqs = (kSched + 128 + 15) & ~15;  // int4 per sequence while ranking
   static constexpr int kList = kSeqs + 16 * kRankMaxSeqs;  // unit of each rank
   static constexpr int kBytes = kList + 4 * kRankMaxUnits;
   static constexpr int kAlloc = kBytes + 1024;
@@ -180,9 +179,8 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
 // of a tile pair).  For up to kRankMaxSeqs sequences and small unit counts,
 // every CTA ranks the units itself: descending key count, ties by sequence
 // then pair (a sequence's own pairs all differ in key count); each thread
-// counts the units ranked before one unit.  Other batches take the units in
-// a fixed order, the last pairs of every sequence (most keys) first, and skip
-// the pairs a sequence does not have.
+// counts the units ranked before one unit.  Other batches take the units
+// sequence-major, only those that exist (prefill_order_units).
 // ---------------------------------------------------------------------------
 
 // floor(x / d) for x >= 0 and d >= 2 from a float reciprocal: below 2^24 both
@@ -216,31 +214,59 @@ struct PrefillItem {
   bool has_b;
 };
 
-// Item i; false when it has no work (a pair its sequence does not have, or an
-// invalid sequence, reported once when `report`).  A tile pair covers `span`
-// query tokens, tile A the first half and tile B the second.
+// Tile pairs (units) of sequence s: ceil(q_len / span), or -1 for an invalid
+// sequence (outside the query rows, longer than its context, or a context
+// past the block table), which has none.
+__device__ __forceinline__ int prefill_units_of(const PrefillArgs& a, int s, int span) {
+  const int q0 = a.query_starts[s], len = a.query_starts[s + 1] - q0;
+  const int ctx = a.context_lens[s];
+  if (q0 < 0 || len < 0 || q0 > a.num_tokens - len || len > ctx ||
+      ctx > a.max_blocks_per_seq * kPage)
+    return -1;
+  return len / span + (len % span != 0);
+}
+
+// Item i (unit i / Hk, KV head i % Hk); false when it has no work.  The unit
+// comes from the ranked list, or, sequence-major, from the per-thread chunk
+// sums (`list`, see prefill_order_units).  A tile pair covers `span` query
+// tokens, tile A the first half and tile B the second.
 __device__ __forceinline__ bool prefill_item(const PrefillArgs& a, const int* list, bool ranked,
-                                             bool report, int i, int span, PrefillItem& it) {
-  const int r = i / a.num_kv_heads;
-  it.kvh = i - r * a.num_kv_heads;
+                                             int i, int span, PrefillItem& it) {
+  const int u = i / a.num_kv_heads;
+  it.kvh = i - u * a.num_kv_heads;
   int p;
   if (ranked) {
-    const int e = list[r];
+    const int e = list[u];
     it.s = e & 0xffff;
     p = e >> 16;
   } else {
-    const int back = r / a.num_seqs;
-    it.s = r - back * a.num_seqs;
-    p = a.pairs_per_seq - 1 - back;
+    // the chunk holding u: the last one whose first unit is <= u; then its
+    // sequences one by one
+    const int n = static_cast<int>(blockDim.x);
+    const int chunk = (a.num_seqs + n - 1) / n;
+    int lo = 0, hi = n;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (list[mid] <= u) lo = mid;
+      else hi = mid;
+    }
+    int first = list[lo], s = lo * chunk;
+    const int s_end = min(a.num_seqs, s + chunk);
+    for (; s < s_end; ++s) {
+      const int units = max(0, prefill_units_of(a, s, span));
+      if (u < first + units) break;
+      first += units;
+    }
+    if (s >= s_end) return false;   // not reached: u is below the unit count
+    it.s = s;
+    p = u - first;
   }
   it.q0 = a.query_starts[it.s];
   it.q_len = a.query_starts[it.s + 1] - it.q0;
   it.ctx = a.context_lens[it.s];
   if (it.q0 < 0 || it.q_len < 0 || it.q0 > a.num_tokens - it.q_len || it.q_len > it.ctx ||
-      it.ctx > a.max_blocks_per_seq * kPage) {
-    if (report && it.kvh == 0 && p == 0) record_error(kErrQuery, it.s);
-    return false;
-  }
+      it.ctx > a.max_blocks_per_seq * kPage)
+    return false;                   // not reached: an invalid sequence has no units
   it.tile_a = p * span;
   if (it.tile_a >= it.q_len) return false;
   const int half = span / 2;
@@ -381,69 +407,103 @@ __device__ __forceinline__ void prefill_store_rows(const PrefillArgs& a, uint32_
   }
 }
 
-// Ranks the units longest first into `list` (unit of each rank: s | p << 16),
-// the same order in every CTA; every thread of the CTA calls it.  t2 = query
-// tokens per unit.  Returns false (nothing ranked) for batches past the
-// limits, which take the fixed order.  Invalid sequences are reported here.
-__device__ __forceinline__ bool prefill_rank_units(const PrefillArgs& a, int t2, int* sched,
-                                                   int4* seqs, int* list, int warp, int lane) {
-  if (a.num_seqs > kRankMaxSeqs) return false;
-  bool ranked = false;
+// The unit order, the same in every CTA; every thread of the CTA calls it and
+// gets the number of units.  t2 = query tokens per unit.  Invalid sequences
+// have no units and are reported here (each by one CTA).
+//  - Up to kRankMaxSeqs sequences and small unit counts (`ranked`): list[rank]
+//    = s | p << 16, longest first.
+//  - Otherwise sequence-major: thread t takes a chunk of ceil(S / blockDim)
+//    sequences and list[t] = the first unit of its chunk (prefix sums), so
+//    only units that exist are walked (prefill_item finds one by a binary
+//    search over the chunks and a scan of one chunk).
+__device__ __forceinline__ int prefill_order_units(const PrefillArgs& a, int t2, int* sched,
+                                                   int4* seqs, int* list, int warp, int lane,
+                                                   bool& ranked) {
   const int t = threadIdx.x;
-  int hist = 0, ql = -1, np = 0;
-  if (t < a.num_seqs) {
-    const int q0 = a.query_starts[t], len = a.query_starts[t + 1] - q0;
-    const int ctx = a.context_lens[t];
-    if (q0 < 0 || len < 0 || q0 > a.num_tokens - len || len > ctx ||
-        ctx > a.max_blocks_per_seq * kPage) {
-      if (t % gridDim.x == blockIdx.x) record_error(kErrQuery, t);  // one CTA reports it
-    } else {
-      hist = ctx - len;
-      ql = len;
-      np = len / t2 + (len % t2 != 0);
+  const bool table = a.num_seqs <= kRankMaxSeqs;
+  ranked = false;
+  if (table) {
+    int hist = 0, ql = -1, np = 0;
+    if (t < a.num_seqs) {
+      const int q0 = a.query_starts[t], len = a.query_starts[t + 1] - q0;
+      const int ctx = a.context_lens[t];
+      if (q0 < 0 || len < 0 || q0 > a.num_tokens - len || len > ctx ||
+          ctx > a.max_blocks_per_seq * kPage) {
+        if (t % gridDim.x == blockIdx.x) record_error(kErrQuery, t);  // one CTA reports it
+      } else {
+        hist = ctx - len;
+        ql = len;
+        np = len / t2 + (len % t2 != 0);
+      }
+    }
+    int first = np;  // inclusive scan over the warp's sequences
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, first, d);
+      if (lane >= d) first += v;
+    }
+    if (lane == 31) sched[4 + warp] = first;
+    __syncthreads();
+    if (t < a.num_seqs) {
+      for (int w = 0; w < warp; ++w) first += sched[4 + w];
+      seqs[t] = make_int4(hist, ql, np, first - np);
+      if (t == a.num_seqs - 1) sched[0] = first;
+    }
+    __syncthreads();
+    const int n_units = sched[0];
+    ranked = n_units <= kRankMaxUnits &&
+             static_cast<long long>(n_units) * a.num_seqs <= kRankMaxWork;
+    if (ranked) {
+      const float inv_t2 = 1.f / static_cast<float>(t2);
+      for (int u = t; u < n_units; u += blockDim.x) {
+        int lo = 0, hi = a.num_seqs;  // the owner: the last sequence whose first unit is <= u
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (seqs[mid].w <= u) lo = mid;
+          else hi = mid;
+        }
+        const int4 me = seqs[lo];
+        const int p = u - me.w;
+        const int K = me.x + min(t2 * (p + 1), me.y);
+        int rank = 0;
+        for (int i = 0; i < a.num_seqs; ++i) {
+          const int4 o = seqs[i];
+          const int gt = pairs_above_of(o.x, o.y, o.z, t2, inv_t2, K);
+          rank += gt;
+          if (i < lo) rank += pairs_above_of(o.x, o.y, o.z, t2, inv_t2, K - 1) - gt;
+        }
+        list[rank] = lo | (p << 16);
+      }
+      __syncthreads();
+      return n_units;
     }
   }
-  int first = np;  // inclusive scan over the warp's sequences
+  // sequence-major: this thread's chunk of sequences and its unit count
+  const int n = static_cast<int>(blockDim.x);
+  const int chunk = (a.num_seqs + n - 1) / n;
+  int mine = 0;
+  for (int s = t * chunk; s < min(a.num_seqs, (t + 1) * chunk); ++s) {
+    const int units = prefill_units_of(a, s, t2);
+    if (units < 0) {
+      if (!table && s % gridDim.x == blockIdx.x) record_error(kErrQuery, s);  // one CTA reports it
+    } else {
+      mine += units;
+    }
+  }
+  int first = mine;  // inclusive scan over the warp
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, first, d);
     if (lane >= d) first += v;
   }
-  if (lane == 31 && warp < kRankMaxSeqs / 32) sched[4 + warp] = first;
+  __syncthreads();   // sched and list are reused from the ranked form
+  if (lane == 31) sched[4 + warp] = first;
   __syncthreads();
-  if (t < a.num_seqs) {
-    for (int w = 0; w < warp; ++w) first += sched[4 + w];
-    seqs[t] = make_int4(hist, ql, np, first - np);
-    if (t == a.num_seqs - 1) sched[0] = first;
-  }
+  for (int w = 0; w < warp; ++w) first += sched[4 + w];
+  list[t] = first - mine;
+  if (t == n - 1) sched[0] = first;
   __syncthreads();
-  const int n_units = sched[0];
-  ranked = n_units <= kRankMaxUnits &&
-           static_cast<long long>(n_units) * a.num_seqs <= kRankMaxWork;
-  if (ranked) {
-    const float inv_t2 = 1.f / static_cast<float>(t2);
-    for (int u = t; u < n_units; u += blockDim.x) {
-      int lo = 0, hi = a.num_seqs;  // the owner: the last sequence whose first unit is <= u
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (seqs[mid].w <= u) lo = mid;
-        else hi = mid;
-      }
-      const int4 me = seqs[lo];
-      const int p = u - me.w;
-      const int K = me.x + min(t2 * (p + 1), me.y);
-      int rank = 0;
-      for (int i = 0; i < a.num_seqs; ++i) {
-        const int4 o = seqs[i];
-        const int gt = pairs_above_of(o.x, o.y, o.z, t2, inv_t2, K);
-        rank += gt;
-        if (i < lo) rank += pairs_above_of(o.x, o.y, o.z, t2, inv_t2, K - 1) - gt;
-      }
-      list[rank] = lo | (p << 16);
-    }
-    __syncthreads();
-  }
-  return ranked;
+  return sched[0];
 }
 
 template <int D, bool BF16>
@@ -473,12 +533,10 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
   int* sched = reinterpret_cast<int*>(smem + L::kSched);   // [0] units, [4 + w] per-warp sums
   int4* seqs = reinterpret_cast<int4*>(smem + L::kSeqs);   // hist, q_len, pairs, first unit
   int* list = reinterpret_cast<int*>(smem + L::kList);     // unit of each rank: s | p << 16
-  const bool table = a.num_seqs <= kRankMaxSeqs;
-  const bool ranked = prefill_rank_units(a, t2, sched, seqs, list, warp, lane);
-  const int total = ranked ? sched[0] * a.num_kv_heads
-                           : a.num_seqs * a.num_kv_heads * a.pairs_per_seq;
+  bool ranked;
+  const int total = prefill_order_units(a, t2, sched, seqs, list, warp, lane, ranked) *
+                    a.num_kv_heads;
   if (prefill_item_index(0, total, blockIdx.x, gridDim.x) < 0) return;   // more CTAs than items
-  const bool report = !table && warp == kWarpTma && lane == 0;
   const int q_rows = a.tile_tokens * G;           // rows a Q box fills
 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
@@ -532,7 +590,7 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
       const int i = prefill_item_index(k, total, blockIdx.x, gridDim.x);
       if (i < 0) break;
       PrefillItem it;
-      if (!prefill_item(a, list, ranked, report, i, t2, it)) continue;
+      if (!prefill_item(a, list, ranked, i, t2, it)) continue;
       if (n_q > 0 && !(ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarQFree,
                                                                   (n_q - 1) & 1, abort_flag))))
         break;
@@ -662,7 +720,7 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
       const int i = prefill_item_index(k, total, blockIdx.x, gridDim.x);
       if (i < 0) break;
       PrefillItem it;
-      if (!prefill_item(a, list, ranked, false, i, t2, it)) continue;
+      if (!prefill_item(a, list, ranked, i, t2, it)) continue;
       const bool hb = it.has_b;
       const int nkb = it.nkb;
       // before the first P_t V of an item: the epilogue has read O_t of the last one
@@ -734,7 +792,7 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
       const int i = prefill_item_index(k, total, blockIdx.x, gridDim.x);
       if (i < 0) break;
       PrefillItem it;
-      if (!prefill_item(a, list, ranked, false, i, t2, it)) continue;
+      if (!prefill_item(a, list, ranked, i, t2, it)) continue;
       const int last_page = (it.ctx - 1) / kPage;
       const int tail_row = it.ctx % kPage;
       uint32_t clipped = 0;
@@ -788,7 +846,7 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
     const int i = prefill_item_index(k, total, blockIdx.x, gridDim.x);
     if (i < 0) break;
     PrefillItem it;
-    if (!prefill_item(a, list, ranked, false, i, t2, it)) continue;
+    if (!prefill_item(a, list, ranked, i, t2, it)) continue;
     if (t == 1 && !it.has_b) continue;
     const int t_begin = it.tile_a + t * a.tile_tokens;
     const int nrows = (min(t_begin + a.tile_tokens, it.q_len) - t_begin) * G;

@@ -67,6 +67,21 @@ CASES["fixed_order_100_seqs_bf16"] = (C["gqa_llama3_8b"], dict(num_seqs=100, num
 _units = sum(-(-q // (2 * 32)) for q in _q)                # tile pairs of 2 x 32 tokens
 assert _units <= 2048 and _units * 100 > 16384, _units
 
+# a step that mixes decodes with long chunks: 700 sequences (two per thread's
+# chunk in the sequence-major order), nearly all bringing one query token, four
+# bringing hundreds; the long ones set max_query_len, so most (sequence, pair)
+# slots are empty and only the units that exist are walked
+_rng = np.random.default_rng(444_074)
+_ctx = [int(c) for c in _rng.integers(1, 300, 700)]
+_q = [1] * 700
+for _i, _n in ((3, 900), (256, 513), (511, 700), (699, 64)):
+    _ctx[_i] = _n + int(_rng.integers(0, 400))
+    _q[_i] = _n
+CASES["mixed_700_seqs_bf16"] = (C["gqa_llama3_8b"], dict(num_seqs=700, num_heads=8,
+                                                          num_kv_heads=2, num_blocks=9000,
+                                                          ctx=("fixed", tuple(_ctx)), seed=74),
+                                 tuple(_q))
+
 # scale 1 instead of 1/sqrt(D): peaked rows whose running maximum jumps by more
 # than 2^8 between key blocks, so the output accumulator is rescaled
 SCALE = {"peaky_bf16": 1.0, "peaky_f16": 1.0}
