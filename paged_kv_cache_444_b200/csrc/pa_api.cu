@@ -130,6 +130,9 @@ pa_status launch_ex(K kernel, unsigned grid, unsigned block, size_t smem, cudaSt
 template <int D>
 struct Stages { static constexpr int value = D == 64 ? PA_STAGES_D64 : PA_STAGES_D128; };
 
+// 16-bit split launches go persistent past this many waves of resident CTAs
+constexpr long long kPersistWaves = 64;
+
 #ifndef PA_SPLIT_PERSISTENT
 #define PA_SPLIT_PERSISTENT 1  // fp8 split launches: one wave of CTAs over the items that exist
 #endif
@@ -211,15 +214,18 @@ pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeAr
   static std::atomic<uint64_t> done{0};
   static std::atomic<int> cluster_cache[kMaxDevices] = {};
   const bool split = a.tmp_out != nullptr;
-  if constexpr (EB == 1) {  // the persistent form is built for the fp8 pages only
+  {
     static std::atomic<uint64_t> done_persist{0};
     static std::atomic<long long> resident_cache[kMaxDevices] = {};
     auto kernel_persist = paged_decode_persistent_kernel<D, NST, BF16, Warp, EB>;
     if (split && a.persistent) {
-      // one wave of CTAs loops over the items that exist (at most `grid`)
+      // one wave of CTAs loops over the items that exist (at most `grid`):
+      // always for the fp8 pages; for 16-bit pages only when the grid over
+      // every possible partition would run past kPersistWaves waves (a long
+      // table, where most of those CTAs would find their partition empty)
       if (!ensure_smem(kernel_persist, L::kAlloc, &done_persist)) return PA_ERR_CUDA;
       const long long resident = resident_ctas(kernel_persist, L::kAlloc, resident_cache);
-      if (resident > 0) {
+      if (resident > 0 && (EB == 1 || grid > kPersistWaves * resident)) {
         if (grid > resident) grid = resident;
         return launch_ex(kernel_persist, static_cast<unsigned>(grid), kThreads, L::kAlloc,
                          stream, 1, km, vm, a);
@@ -282,10 +288,12 @@ pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cach
     return PA_ERR_CUDA;
   const long long grid = num_seqs * a.num_kv_heads * static_cast<long long>(a.parts_per_head);
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
-  // 16-bit split launches keep the grid over every possible partition: the
-  // persistent form measured 2.5-4 % slower on these kernels
+  // 16-bit split launches keep the grid over every possible partition unless
+  // it runs past kPersistWaves waves: the persistent form measured 3-4 %
+  // slower on full tables, and 3.3x faster on a skewed one (one 128K-token
+  // sequence among 255 of 1K, 524 288 possible partitions)
   a.num_seqs = static_cast<int>(num_seqs);
-  a.persistent = 0;
+  a.persistent = PA_SPLIT_PERSISTENT && a.tmp_out != nullptr && num_seqs <= kLptMaxSeqs;
   const bool bf16 = dtype == PA_BF16;
   const int64_t max_pages = a.max_blocks_per_seq;  // block_size == 16 == one page
   if (head_dim == 64)

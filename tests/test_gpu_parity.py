@@ -562,3 +562,23 @@ def test_bounded_wait_gives_up_and_context_stays_usable(dev, oracle_lib):
     pa_check_error()
     assert np.array_equal(bits(batch.key_cache), kc_ref)
     _check_close(out, ref, cfg, "decode after a barrier timeout")
+
+
+def test_split_persistent_on_a_long_skewed_table(dev, oracle_lib):
+    """A 16-bit split launch whose grid over every possible partition would run
+    past 64 waves of resident CTAs takes the persistent form, over only the
+    partitions that exist: 256 sequences, one of 4096 tokens among 255 of
+    0-79, 32-token partitions (a full grid of 256 x 2 x 128 CTAs, 147 waves of
+    the 444 resident).  Partials and merged output against the oracle."""
+    rng = np.random.default_rng(444_091)
+    ctx = [4096] + [int(c) for c in rng.integers(0, 80, 255)]
+    cfg = SMALL["gqa_small"].scaled(num_seqs=256, num_heads=8, num_kv_heads=2, num_blocks=2048,
+                                    ctx=("fixed", tuple(ctx)), seed=91)
+    batch = workloads.make_batch(cfg, dev)
+    assert cfg.num_seqs * cfg.num_kv_heads * (batch.block_tables.shape[1] * 16 // 32) > 128 * 444
+    host = HostCopy(batch)
+    ref, kc_ref, vc_ref = oracle_step(oracle_lib, host)
+    out, ws = gpu_step(batch, partition_size=32)
+    pa_check_error()
+    _check_close(out, ref, cfg, "split, persistent, skewed table")
+    _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, 32)
