@@ -293,7 +293,7 @@ pa_status run_decode(DecodeArgs a, const void* key_cache, const void* value_cach
   // slower on full tables, and 3.3x faster on a skewed one (one 128K-token
   // sequence among 255 of 1K, 524 288 possible partitions)
   a.num_seqs = static_cast<int>(num_seqs);
-  a.persistent = PA_SPLIT_PERSISTENT && a.tmp_out != nullptr && num_seqs <= kLptMaxSeqs;
+  a.persistent = PA_SPLIT_PERSISTENT && a.tmp_out != nullptr;
   const bool bf16 = dtype == PA_BF16;
   const int64_t max_pages = a.max_blocks_per_seq;  // block_size == 16 == one page
   if (head_dim == 64)
@@ -314,11 +314,11 @@ pa_status run_decode_fp8(DecodeArgs a, const void* key_cache, const void* value_
     return PA_ERR_CUDA;
   const long long grid = num_seqs * a.num_kv_heads * static_cast<long long>(a.parts_per_head);
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
-  // fp8 split launches with up to kLptMaxSeqs sequences: one persistent wave of
-  // CTAs over the partitions that exist (measured 2.5-7 % faster than the
-  // grid over every possible partition; the fp8 items are short)
+  // fp8 split launches: one persistent wave of CTAs over the partitions that
+  // exist (measured 2.5-7 % faster than the grid over every possible
+  // partition; the fp8 items are short)
   a.num_seqs = static_cast<int>(num_seqs);
-  a.persistent = PA_SPLIT_PERSISTENT && a.tmp_out != nullptr && num_seqs <= kLptMaxSeqs;
+  a.persistent = PA_SPLIT_PERSISTENT && a.tmp_out != nullptr;
   const int64_t max_pages = a.max_blocks_per_seq;
   if (dtype == PA_BF16) {
     if (a.group <= 8)

@@ -79,18 +79,21 @@ struct DecodeSmem {
   static constexpr int kRedLOffset = kRedMOffset + kWarps * 16 * 4;
   static constexpr int kPartMOffset = kRedLOffset + kWarps * 16 * 4;
   static constexpr int kPartLOffset = kPartMOffset + 16 * 4;
-  // persistent split mode: every sequence's context length and the running
-  // count of partitions before it (outside the stage area: kept across items)
-  static constexpr int kCtxOffset = kPartLOffset + 16 * 4;
-  static constexpr int kCumOffset = kCtxOffset + kLptMaxSeqs * 4;
-  static constexpr int kBytes = kCumOffset + (kLptMaxSeqs + 1) * 4;
+  // persistent split mode (outside the stage area: kept across items): up to
+  // kLptMaxSeqs sequences, every context and the partitions before each
+  // sequence; beyond, the partitions before each thread's chunk of
+  // sequences and per-warp sums
+  static constexpr int kSeqOffset = kPartLOffset + 16 * 4;
+  static constexpr int kSeqBytes = (2 * kLptMaxSeqs + 1) * 4 > (kThreads + 1 + kWarps) * 4
+                                       ? (2 * kLptMaxSeqs + 1) * 4
+                                       : (kThreads + 1 + kWarps) * 4;
+  static constexpr int kBytes = kSeqOffset + kSeqBytes;
   static constexpr int kAlloc = kBytes + 1024;            // + alignment slack
   // the merge buffers reuse the stage area: per-warp rows (kWarps x group x D
   // floats) and, for an item spread over a cluster, this CTA's merged rows
   static constexpr int kPartAccOffset = kWarps * 16 * D * 4;
   static_assert(kPartAccOffset + 16 * D * 4 <= kStagesBytes, "merge buffers must fit in the stages");
   static_assert((D * EB) % 128 == 0, "a cache row must be a whole number of 128-byte boxes");
-  static_assert((kLptMaxSeqs + 1) * 4 <= kStagesBytes, "length table must fit in the stages");
 };
 
 // Address of 16-byte chunk `c` (0 .. D/8-1) of row `r` in a swizzled page.
@@ -645,13 +648,38 @@ __global__ void __launch_bounds__(kThreads, EB == 1 ? 3 : 0)  // fp8: three CTAs
 
 
 // ---------------------------------------------------------------------------
-// Split mode, persistent (up to kLptMaxSeqs sequences): the items that exist
-// -- partition p of sequence s for p < ceil(ctx_s / partition_size), every KV
-// head -- in a dense order that every CTA derives from the context lengths.
-// The grid is one wave (SMs x resident CTAs); CTA b takes items b,
-// b + gridDim.x, ..., so no CTA is launched for a partition past its
-// sequence's end.  Each warp's ring runs on from item to item.
+// Split mode, persistent: the items that exist -- partition p of sequence s
+// for p < ceil(ctx_s / partition_size), every KV head -- in a dense order that
+// every CTA derives from the context lengths.  Up to kLptMaxSeqs sequences
+// every context and the partitions before each sequence sit in shared
+// memory, and an item's sequence is a binary search away.  Beyond, thread t
+// counts the partitions of a chunk of ceil(S / kThreads) sequences, a block
+// scan gives each chunk's first partition, and an item's sequence is found by
+// a binary search over the chunks and a scan of one chunk.  The grid is one
+// wave (SMs x resident CTAs); CTA b takes items b, b + gridDim.x, ..., so no
+// CTA is launched for a partition past its sequence's end.  Each warp's ring
+// runs on from item to item.
 // ---------------------------------------------------------------------------
+
+// Partitions of sequence s (clamped as the kernels clamp: a context outside
+// [0, cap] to the range, a count past max_partitions to it), its clamped
+// context in ctx; the clamps are reported when `report`.
+__device__ __forceinline__ int split_partitions(const DecodeArgs& a, int s, int cap, bool report,
+                                                int& ctx) {
+  int c = a.context_lens[s];
+  if (c < 0 || c > cap) {
+    if (report) record_error(kErrContextLen, s);
+    c = c < 0 ? 0 : cap;
+  }
+  int np = (c + a.partition_size - 1) / a.partition_size;
+  if (np > a.max_partitions) {
+    if (report) record_error(kErrPartitions, s);
+    np = a.max_partitions;
+  }
+  ctx = c;
+  return np;
+}
+
 template <int D, int NST, bool BF16, class Warp, int EB = 2>
 __global__ void __launch_bounds__(kThreads, 3)  // three CTAs per SM: at most 168 registers
     paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -665,51 +693,82 @@ __global__ void __launch_bounds__(kThreads, 3)  // three CTAs per SM: at most 16
   pdl_launch_dependents();
   pdl_wait();  // inputs may come from the previous kernel of the stream
   const int cap = a.max_blocks_per_seq * kPage;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  {
-    int* ctxs = reinterpret_cast<int*>(smem + L::kCtxOffset);
-    int* cum = reinterpret_cast<int*>(smem + L::kCumOffset);
-    for (int i = threadIdx.x; i < a.num_seqs; i += kThreads) {
-      int c = a.context_lens[i];
-      if (c < 0 || c > cap) {
-        if (blockIdx.x == 0) record_error(kErrContextLen, i);
-        c = c < 0 ? 0 : cap;
-      }
-      int np = (c + a.partition_size - 1) / a.partition_size;
-      if (np > a.max_partitions) {
-        if (blockIdx.x == 0) record_error(kErrPartitions, i);
-        np = a.max_partitions;
-      }
-      ctxs[i] = c;
-      cum[i + 1] = np;
-    }
+  const bool small = a.num_seqs <= kLptMaxSeqs;
+  int* ctxs = reinterpret_cast<int*>(smem + L::kSeqOffset);   // small: [S] contexts
+  int* cum = ctxs + kLptMaxSeqs;                              // small: [S + 1] partitions before
+  int* chunk_first = ctxs;                                    // else: [kThreads + 1]
+  int* warp_sum = ctxs + kThreads + 1;                        // else: [kWarps]
+  const int chunk = (a.num_seqs + kThreads - 1) / kThreads;
+  const int t = threadIdx.x;
+  int total;
+  if (small) {
+    for (int s = t; s < a.num_seqs; s += kThreads)
+      cum[s + 1] = split_partitions(a, s, cap, blockIdx.x == 0, ctxs[s]);   // one CTA reports
     __syncthreads();
-    if (threadIdx.x == 0) {  // running count (at most kLptMaxSeqs sequences)
+    if (t == 0) {  // running count
       int acc = 0;
       cum[0] = 0;
-      for (int i = 0; i < a.num_seqs; ++i) cum[i + 1] = (acc += cum[i + 1]);
+      for (int s = 0; s < a.num_seqs; ++s) cum[s + 1] = (acc += cum[s + 1]);
     }
     __syncthreads();
-    const int items = cum[a.num_seqs] * a.num_kv_heads;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    init_ring<NST>(smem_addr(smem + L::kBarOffset) + warp * NST * 8, lane);
-    int kbase = 0;  // this warp's pages through its ring so far
-    for (int u = blockIdx.x; u < items; u += gridDim.x) {
-      const int kv = u % a.num_kv_heads, su = u / a.num_kv_heads;
+    total = cum[a.num_seqs];
+  } else {
+    int mine = 0;
+    for (int s = t * chunk; s < min(a.num_seqs, (t + 1) * chunk); ++s) {
+      int c;
+      mine += split_partitions(a, s, cap, blockIdx.x == 0, c);   // one CTA reports
+    }
+    int incl = mine;  // block scan of the chunk counts
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    for (int w = 0; w < warp; ++w) incl += warp_sum[w];
+    chunk_first[t] = incl - mine;
+    if (t == kThreads - 1) chunk_first[kThreads] = incl;
+    __syncthreads();
+    total = chunk_first[kThreads];
+  }
+  const int items = total * a.num_kv_heads;
+  init_ring<NST>(smem_addr(smem + L::kBarOffset) + warp * NST * 8, lane);
+  int kbase = 0;  // this warp's pages through its ring so far
+  for (int u = blockIdx.x; u < items; u += gridDim.x) {
+    const int kv = u % a.num_kv_heads, su = u / a.num_kv_heads;
+    int s, first, ctx = 0;
+    if (small) {
       int lo = 0, hi = a.num_seqs;  // the sequence with cum[s] <= su < cum[s + 1]
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
         if (cum[mid] <= su) lo = mid; else hi = mid;
       }
-      // (decode_item ends with a CTA barrier: the merge buffers, in the
-      // stage area, are free for the next item's pages)
-      if (!decode_item<D, NST, BF16, Warp, EB>(kmap, vmap, a, smem, lo, kv, su - cum[lo],
-                                               ctxs[lo], 1, 0, kbase))
-        return;
+      s = lo;
+      first = cum[lo];
+      ctx = ctxs[lo];
+    } else {
+      int lo = 0, hi = kThreads;  // the chunk: the last one whose first partition is <= su
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (chunk_first[mid] <= su) lo = mid; else hi = mid;
+      }
+      first = chunk_first[lo];
+      s = lo * chunk;
+      for (const int s_end = min(a.num_seqs, s + chunk); s < s_end; ++s) {
+        const int np = split_partitions(a, s, cap, false, ctx);
+        if (su < first + np) break;
+        first += np;
+      }
     }
-    return;
+    // (decode_item ends with a CTA barrier: the merge buffers, in the stage
+    // area, are free for the next item's pages)
+    if (!decode_item<D, NST, BF16, Warp, EB>(kmap, vmap, a, smem, s, kv, su - first, ctx, 1, 0,
+                                             kbase))
+      return;
   }
-
 }
 
 }  // namespace pa

@@ -96,9 +96,10 @@ def test_fp8_split_matches_oracle(name, ps, cuda_device, oracle_lib):
 @pytest.mark.parametrize("name,ps", [("ragged_bf16", 16), ("many_seqs_f16", 32)],
                          ids=["persistent_ragged_with_empty", "full_grid_300_seqs"])
 def test_fp8_split_ragged_and_large_batches(name, ps, cuda_device, oracle_lib):
-    """The fp8 split launch is persistent up to 256 sequences (one wave of CTAs
-    over the partitions that exist, empty sequences contributing none) and a
-    grid over every possible partition beyond; both against the oracle."""
+    """The fp8 split launch is persistent (one wave of CTAs over the
+    partitions that exist, empty sequences contributing none), on a ragged
+    batch and on 300 sequences (chunks of three per thread); both against the
+    oracle."""
     cfg = (CASES["ragged_bf16"] if name == "ragged_bf16" else
            C["mha_llama2_7b"].scaled(num_seqs=300, num_heads=2, num_kv_heads=2, num_blocks=2048,
                                      ctx=("uniform", 0, 90), seed=56))

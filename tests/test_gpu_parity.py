@@ -115,8 +115,8 @@ def _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, ps):
 
 
 def test_split_over_full_grid_for_many_sequences(dev, oracle_lib):
-    """More than 256 sequences: the split launch covers every possible
-    partition with its own CTA (the persistent form serves smaller batches);
+    """300 sequences on a short table: the grid over every possible partition
+    stays far below 64 waves, so the split launch gives each its own CTA;
     partials and merged output against the oracle."""
     cfg = SMALL["mha_small"].scaled(num_seqs=300, num_heads=2, num_kv_heads=2, num_blocks=2048,
                                     ctx=("uniform", 0, 90), seed=23)
@@ -567,12 +567,14 @@ def test_bounded_wait_gives_up_and_context_stays_usable(dev, oracle_lib):
 def test_split_persistent_on_a_long_skewed_table(dev, oracle_lib):
     """A 16-bit split launch whose grid over every possible partition would run
     past 64 waves of resident CTAs takes the persistent form, over only the
-    partitions that exist: 256 sequences, one of 4096 tokens among 255 of
-    0-79, 32-token partitions (a full grid of 256 x 2 x 128 CTAs, 147 waves of
-    the 444 resident).  Partials and merged output against the oracle."""
+    partitions that exist: 300 sequences (chunks of three per thread), one of
+    4096 tokens among 299 of 0-79, 32-token partitions (a full grid of
+    300 x 2 x 128 CTAs, 173 waves of the 444 resident).  Partials and merged
+    output against the oracle."""
     rng = np.random.default_rng(444_091)
-    ctx = [4096] + [int(c) for c in rng.integers(0, 80, 255)]
-    cfg = SMALL["gqa_small"].scaled(num_seqs=256, num_heads=8, num_kv_heads=2, num_blocks=2048,
+    ctx = [int(c) for c in rng.integers(0, 80, 300)]
+    ctx[137] = 4096
+    cfg = SMALL["gqa_small"].scaled(num_seqs=300, num_heads=8, num_kv_heads=2, num_blocks=2048,
                                     ctx=("fixed", tuple(ctx)), seed=91)
     batch = workloads.make_batch(cfg, dev)
     assert cfg.num_seqs * cfg.num_kv_heads * (batch.block_tables.shape[1] * 16 // 32) > 128 * 444
