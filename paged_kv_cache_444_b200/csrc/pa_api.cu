@@ -83,13 +83,13 @@ bool ensure_smem(K kernel, int bytes, std::atomic<uint64_t>* done_mask) {
   return true;
 }
 
-// Launch with programmatic stream serialisation (the kernel may start while
-// the previous kernel of the stream drains; every kernel here waits for it
-// with griddepcontrol.wait before reading inputs) and, if cluster > 1, as
-// clusters of `cluster` CTAs along x.
+// Launch as clusters of `cluster` CTAs along x when cluster > 1; a plain
+// launch otherwise, with programmatic stream serialisation if `programmatic`
+// (the kernel may start while the previous kernel of the stream drains; every
+// kernel here waits for it with griddepcontrol.wait before reading inputs).
 template <class K, class... Args>
-pa_status launch_ex(K kernel, unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
-                    int cluster, Args... args) {
+pa_status launch_cfg(K kernel, unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                     int cluster, bool programmatic, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(block, 1, 1);
@@ -103,7 +103,7 @@ pa_status launch_ex(K kernel, unsigned grid, unsigned block, size_t smem, cudaSt
     attrs[n].val.clusterDim.y = 1;
     attrs[n].val.clusterDim.z = 1;
     ++n;
-  } else {
+  } else if (programmatic) {
     attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attrs[n].val.programmaticStreamSerializationAllowed = 1;
     ++n;
@@ -117,6 +117,12 @@ pa_status launch_ex(K kernel, unsigned grid, unsigned block, size_t smem, cudaSt
   return PA_OK;
 }
 
+template <class K, class... Args>
+pa_status launch_ex(K kernel, unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                    int cluster, Args... args) {
+  return launch_cfg(kernel, grid, block, smem, stream, cluster, true, args...);
+}
+
 // Pipeline depth per head_dim: stages of (K page + V page) per warp.
 #ifndef PA_STAGES_D128
 #define PA_STAGES_D128 2
@@ -126,6 +132,9 @@ pa_status launch_ex(K kernel, unsigned grid, unsigned block, size_t smem, cudaSt
 #endif
 #ifndef PA_STAGES_FP8
 #define PA_STAGES_FP8 4  // fp8 pages are half the bytes: twice the stages in the same space
+#endif
+#ifndef PA_STAGES_FP8_T
+#define PA_STAGES_FP8_T 3  // transposed fp8 page step: four CTAs per SM share the space
 #endif
 template <int D>
 struct Stages { static constexpr int value = D == 64 ? PA_STAGES_D64 : PA_STAGES_D128; };
@@ -205,10 +214,10 @@ long long resident_ctas(K kernel, int smem_bytes, std::atomic<long long>* cache)
   return known;
 }
 
-template <int D, bool BF16, class Warp, int EB = 2>
+template <int D, bool BF16, class Warp, int EB = 2,
+          int NST = (EB == 1 ? PA_STAGES_FP8 : Stages<D>::value)>
 pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeArgs a,
                           long long grid, int64_t max_pages, cudaStream_t stream) {
-  constexpr int NST = EB == 1 ? PA_STAGES_FP8 : Stages<D>::value;
   using L = DecodeSmem<D, NST, EB>;
   auto kernel = paged_decode_kernel<D, NST, BF16, Warp, EB>;
   static std::atomic<uint64_t> done{0};
@@ -227,8 +236,12 @@ pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeAr
       const long long resident = resident_ctas(kernel_persist, L::kAlloc, resident_cache);
       if (resident > 0 && (EB == 1 || grid > kPersistWaves * resident)) {
         if (grid > resident) grid = resident;
-        return launch_ex(kernel_persist, static_cast<unsigned>(grid), kThreads, L::kAlloc,
-                         stream, 1, km, vm, a);
+        // in stream order, not programmatically: a persistent grid wants all
+        // its CTAs resident together, and an early launch lets its first CTAs
+        // take the slots the previous kernel leaves while the rest wait (the
+        // fp8 long-context split + reduce, back to back: 324 us, against 245)
+        return launch_cfg(kernel_persist, static_cast<unsigned>(grid), kThreads, L::kAlloc,
+                          stream, 1, false, km, vm, a);
       }
       a.persistent = 0;
     }
@@ -322,14 +335,14 @@ pa_status run_decode_fp8(DecodeArgs a, const void* key_cache, const void* value_
   const int64_t max_pages = a.max_blocks_per_seq;
   if (dtype == PA_BF16) {
     if (a.group <= 8)
-      return launch_decode_t<128, true, MmaFp8Warp<128, true, false>, 1>(km, vm, a, grid,
-                                                                        max_pages, stream);
+      return launch_decode_t<128, true, MmaFp8WarpT<128, true>, 1, PA_STAGES_FP8_T>(
+          km, vm, a, grid, max_pages, stream);
     return launch_decode_t<128, true, MmaFp8Warp<128, true, true>, 1>(km, vm, a, grid, max_pages,
                                                                      stream);
   }
   if (a.group <= 8)
-    return launch_decode_t<128, false, MmaFp8Warp<128, false, false>, 1>(km, vm, a, grid,
-                                                                        max_pages, stream);
+    return launch_decode_t<128, false, MmaFp8WarpT<128, false>, 1, PA_STAGES_FP8_T>(
+        km, vm, a, grid, max_pages, stream);
   return launch_decode_t<128, false, MmaFp8Warp<128, false, true>, 1>(km, vm, a, grid, max_pages,
                                                                      stream);
 }

@@ -109,6 +109,7 @@ template <int D, bool BF16, bool TWO_ROWS>
 struct MmaWarp {
   static constexpr int KSTEPS = D / 16;  // k-steps of 16 over head_dim
   static constexpr int NTILES = D / 8;   // 8-wide n-tiles of the output
+  static constexpr int kMinBlocks = 0;   // single pass: no register cap
   uint32_t qa[KSTEPS][4];                // Q as mma A fragments (rows = query heads of the group)
   float acc[NTILES][4];                  // O fragments (rows r0 / r1)
   float m[2], l[2];                      // running max (log2 domain) and lane-partial sums
@@ -579,7 +580,7 @@ __device__ __forceinline__ bool decode_item(const CUtensorMap& kmap, const CUten
 }
 
 template <int D, int NST, bool BF16, class Warp, int EB = 2>
-__global__ void __launch_bounds__(kThreads, EB == 1 ? 3 : 0)  // fp8: three CTAs per SM
+__global__ void __launch_bounds__(kThreads, Warp::kMinBlocks)
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
   using L = DecodeSmem<D, NST, EB>;
@@ -681,7 +682,8 @@ __device__ __forceinline__ int split_partitions(const DecodeArgs& a, int s, int 
 }
 
 template <int D, int NST, bool BF16, class Warp, int EB = 2>
-__global__ void __launch_bounds__(kThreads, 3)  // three CTAs per SM: at most 168 registers
+// at least three CTAs per SM (at most 168 registers), more where the page step allows
+__global__ void __launch_bounds__(kThreads, Warp::kMinBlocks > 3 ? Warp::kMinBlocks : 3)
     paged_decode_persistent_kernel(const __grid_constant__ CUtensorMap kmap,
                                    const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
   using L = DecodeSmem<D, NST, EB>;

@@ -7,10 +7,15 @@
 // per page and tensor, so a page of one head is 2 KB instead of 4 KB.  The
 // query stays 16-bit; k_scale is folded into the logit scale and v_scale into
 // the output, so the page steps below work on the raw codes:
-//  - MmaFp8Warp (every group size, one query head per KV head included: fp16
-//    mma on a 16-row tile whose rows are the group's heads; for one head the
-//    tensor cores take the products off the issue path, measured 7 % faster
-//    than packed fp32 FMA on CUDA cores): the page is read with the same b16 ldmatrix as
+//  - MmaFp8WarpT (groups of up to 8 query heads, one included): both
+//    products transposed, so that the page's tokens and the head's dims fill
+//    the mma's 16 rows and the query heads its 8 columns.  Half the mma and
+//    accumulators of MmaFp8Warp; 122 registers, four CTAs per SM.
+//  - MmaFp8Warp (groups of 9 to 16: fp16 mma on a 16-row tile whose rows are
+//    the group's heads; the same tile served every group size before the
+//    transposed step, and for one head the tensor cores took the products
+//    off the issue path, measured 7 % faster than packed fp32 FMA on CUDA
+//    cores): the page is read with the same b16 ldmatrix as
 //    the 16-bit path, which hands each lane 4 consecutive codes of a row
 //    where the 16-bit fragment layout expects 2 + 2 codes 8 apart.  Inside
 //    one 16-element k-step that is a fixed permutation of the head dims, so
@@ -26,7 +31,8 @@
 namespace pa {
 
 // ---------------------------------------------------------------------------
-// Tensor-core path (every group size, 1..16), head_dim 128.
+// Tensor-core path with a 16-row query tile (groups of 9 to 16), head_dim 128.
+// Its query prescale and pow2 serve the transposed step below too.
 //
 // Both products run as fp16 mma whatever the query dtype: E4M3 -> fp16 is one
 // exact conversion, and P in fp16 keeps 11 bits.  A bf16 (or fp16) query row
@@ -38,6 +44,7 @@ namespace pa {
 template <int D, bool BF16, bool TWO_ROWS>
 struct MmaFp8Warp {
   static_assert(D == 128, "fp8 tensor-core path is built for head_dim 128");
+  static constexpr int kMinBlocks = 3;  // three CTAs per SM: at most 168 registers
   static constexpr int KSTEPS = D / 16;
   static constexpr int NTILES = D / 8;
   uint32_t qa[KSTEPS][4];   // fp16 Q fragments, head dims permuted as the fp8 K fragments
@@ -219,6 +226,191 @@ struct MmaFp8Warp {
         if (tig == 0) {
           red_m[r1] = m[1];
           red_l[r1] = l1;
+        }
+      }
+    }
+  }
+};
+
+// Four E4M3 codes -> two half2 (codes 0, 1 -> lo; codes 2, 3 -> hi), exactly.
+__device__ __forceinline__ void e4m3x4_to_h2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
+}
+
+// Transpose of an 8 x 8 matrix of 16-bit elements held in the mma fragment
+// layout (lane l: row l / 4, elements 2(l % 4) and 2(l % 4) + 1).  Whole warp.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core path for groups of up to 8 query heads: both products
+// transposed, S^T = K Q^T and O^T = V^T P^T.  The page's 16 tokens (first
+// product) and 16-dim slices of the head (second) are the M = 16 rows of the
+// mma, the group's query heads its N = 8 columns.  Against the 16-row query
+// tile of MmaFp8Warp this halves the mma per page (8 + 8 instead of 16 + 16)
+// and the accumulator registers: a small group no longer carries 8 or more
+// padding rows.
+//  - K: the b16 ldmatrix hands lane (g, t) codes 4t .. 4t+3 of token g (and
+//    g + 8) in a 16-dim chunk.  The k-step takes dims 4t, 4t+1 at positions
+//    2t, 2t+1 and dims 4t+2, 4t+3 at 2t+8, 2t+9; Q's B fragment is then the
+//    same four consecutive dims of query row g.
+//  - P: the S^T accumulator holds (token g or g + 8; query rows 2t, 2t+1),
+//    and the B operand of the second product wants (tokens 2t, 2t+1; row g):
+//    one movmatrix transpose per 8 tokens, after the fp16 packing.
+//  - V: the transposed ldmatrix hands lane (g, t) tokens 2t, 2t+1 of dims
+//    2g, 2g+1 of a chunk; one byte permute over two chunks gathers the
+//    even-dim (or odd-dim) codes of two m-tile rows.  M-tile 2c holds the even
+//    dims of chunks 2c, 2c+1 (row g: dim 32c + 2g; row g + 8: dim 32c + 16 +
+//    2g), m-tile 2c + 1 the odd dims; publish puts them back in order.
+// ---------------------------------------------------------------------------
+template <int D, bool BF16>
+struct MmaFp8WarpT {
+  static_assert(D == 128, "fp8 tensor-core path is built for head_dim 128");
+  static constexpr int kMinBlocks = 4;  // CTAs per SM the register budget is built for
+  static constexpr int KSTEPS = D / 16;
+  static constexpr int MTILES = D / 16;
+  uint32_t qb[KSTEPS][2];  // fp16 Q^T fragments of query row lane / 4
+  float acc[MTILES][4];    // O^T: (m-tile row g, query row 2t | 2t+1), (row g + 8, ...)
+  float m[2], l[2];        // query rows 2t, 2t+1: running max (log2), lane-partial sum
+  float rs[2];             // 2^-s of query rows 2t, 2t+1 (undo the query prescale)
+
+  __device__ __forceinline__ void init(const uint16_t* q_group, int group, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    float4 v[KSTEPS];
+    float mx = 0.f;
+    const uint16_t* qrow = q_group + g * D;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      const uint2 w = g < group ? *reinterpret_cast<const uint2*>(qrow + kk * 16 + 4 * t)
+                                : make_uint2(0u, 0u);
+      const float2 x = unpack2<BF16>(w.x), y = unpack2<BF16>(w.y);
+      v[kk] = make_float4(x.x, x.y, y.x, y.y);
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(y.x), fabsf(y.y))));
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const int s = MmaFp8Warp<D, BF16, false>::prescale_exp(mx);
+    const float f = MmaFp8Warp<D, BF16, false>::pow2(s);
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      qb[kk][0] = pack2<false>(v[kk].x * f, v[kk].y * f);
+      qb[kk][1] = pack2<false>(v[kk].z * f, v[kk].w * f);
+    }
+    // the exponents of query rows 2t and 2t + 1 sit in lanes 8t and 8t + 4
+    const int s0 = __shfl_sync(0xffffffffu, s, 8 * t), s1 = __shfl_sync(0xffffffffu, s, 8 * t + 4);
+    rs[0] = MmaFp8Warp<D, BF16, false>::pow2(-s0);
+    rs[1] = MmaFp8Warp<D, BF16, false>::pow2(-s1);
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.f;
+  }
+
+  __device__ __forceinline__ void page(uint32_t kbase, uint32_t vbase, int tok0, int t_end,
+                                       float scale_log2, int lane) {
+    const int g = lane >> 2;
+    const int mtok = ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int mchk = lane >> 4;
+    // ---- S^T = K Q^T: one x4 ldmatrix covers two k-steps (two accumulator chains) ----
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kp = 0; kp < KSTEPS / 2; ++kp) {
+      const int c = 2 * kp + mchk;
+      uint32_t r0, r1, r2, r3;  // (tok 0-7, chunk 2kp) (8-15, 2kp) (0-7, 2kp+1) (8-15, 2kp+1)
+      ldsm_x4(kbase + mtok * 128 + ((c ^ (mtok & 7)) << 4), r0, r1, r2, r3);
+      uint32_t a[4], b[4];
+      e4m3x4_to_h2x2(r0, a[0], a[2]);
+      e4m3x4_to_h2x2(r1, a[1], a[3]);
+      e4m3x4_to_h2x2(r2, b[0], b[2]);
+      e4m3x4_to_h2x2(r3, b[1], b[3]);
+      mma_16816<false>(s0, a, qb[2 * kp][0], qb[2 * kp][1]);
+      mma_16816<false>(s1, b, qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
+    }
+    // ---- scale (with each row's 2^-s), mask, row maxima over the 16 tokens ----
+    const float sl0 = scale_log2 * rs[0], sl1 = scale_log2 * rs[1];
+    const int lim = t_end - tok0;
+    const bool lo_live = g < lim, hi_live = g + 8 < lim;
+    const float x0 = lo_live ? (s0[0] + s1[0]) * sl0 : -INFINITY;  // token g, row 2t
+    const float x1 = lo_live ? (s0[1] + s1[1]) * sl1 : -INFINITY;  // token g, row 2t+1
+    const float x2 = hi_live ? (s0[2] + s1[2]) * sl0 : -INFINITY;  // token g+8, row 2t
+    const float x3 = hi_live ? (s0[3] + s1[3]) * sl1 : -INFINITY;  // token g+8, row 2t+1
+    // lanes of equal t hold the same two rows; each reduces one of them over
+    // the 8 lanes and the other comes back from the neighbour of opposite g parity
+    const bool odd = g & 1;
+    float keep = odd ? fmaxf(x1, x3) : fmaxf(x0, x2);
+    const float send = odd ? fmaxf(x0, x2) : fmaxf(x1, x3);
+    keep = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+    keep = fmaxf(keep, __shfl_xor_sync(0xffffffffu, keep, 8));
+    keep = fmaxf(keep, __shfl_xor_sync(0xffffffffu, keep, 16));
+    const float other = __shfl_xor_sync(0xffffffffu, keep, 4);
+    const float mn0 = fmaxf(m[0], odd ? other : keep);
+    const float mn1 = fmaxf(m[1], odd ? keep : other);
+    const float al0 = ex2(m[0] - mn0), al1 = ex2(m[1] - mn1);
+    m[0] = mn0;
+    m[1] = mn1;
+    // ---- P in fp16, l sums the same rounded values, then P^T as a B operand ----
+    const uint32_t p_lo = pack2<false>(ex2(x0 - mn0), ex2(x1 - mn1));  // token g
+    const uint32_t p_hi = pack2<false>(ex2(x2 - mn0), ex2(x3 - mn1));  // token g + 8
+    {
+      const float2 u = unpack2<false>(p_lo), w = unpack2<false>(p_hi);
+      l[0] = l[0] * al0 + (u.x + w.x);
+      l[1] = l[1] * al1 + (u.y + w.y);
+    }
+    const uint32_t pb0 = movmatrix_trans(p_lo);  // tokens 2t, 2t+1 of query row g
+    const uint32_t pb1 = movmatrix_trans(p_hi);  // tokens 2t+8, 2t+9
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+      acc[i][0] *= al0;
+      acc[i][1] *= al1;
+      acc[i][2] *= al0;
+      acc[i][3] *= al1;
+    }
+    // ---- O^T += V^T P^T: one transposed x4 ldmatrix covers two 16-dim chunks ----
+#pragma unroll
+    for (int cp = 0; cp < D / 32; ++cp) {
+      const int c = 2 * cp + mchk;
+      uint32_t r0, r1, r2, r3;  // (tok 0-7, chunk 2cp) (8-15, 2cp) (0-7, 2cp+1) (8-15, 2cp+1)
+      ldsm_x4_trans(vbase + mtok * 128 + ((c ^ (mtok & 7)) << 4), r0, r1, r2, r3);
+      uint32_t ae[4], ao[4];  // rows g (chunk 2cp) and g + 8 (chunk 2cp+1); tokens 2t.. | 2t+8..
+      e4m3x4_to_h2x2(__byte_perm(r0, r2, 0x6420), ae[0], ae[1]);
+      e4m3x4_to_h2x2(__byte_perm(r1, r3, 0x6420), ae[2], ae[3]);
+      e4m3x4_to_h2x2(__byte_perm(r0, r2, 0x7531), ao[0], ao[1]);
+      e4m3x4_to_h2x2(__byte_perm(r1, r3, 0x7531), ao[2], ao[3]);
+      mma_16816<false>(acc[2 * cp], ae, pb0, pb1);
+      mma_16816<false>(acc[2 * cp + 1], ao, pb0, pb1);
+    }
+  }
+
+  // Query rows < group into the merge buffers, head dims in order.
+  __device__ __forceinline__ void publish(float* red_acc, float* red_m, float* red_l, int group,
+                                          int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    float l0 = l[0], l1 = l[1];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = 2 * t + h;
+      if (row < group) {
+#pragma unroll
+        for (int cp = 0; cp < D / 32; ++cp) {
+          float* o = red_acc + row * D + cp * 32 + 2 * g;
+          *reinterpret_cast<float2*>(o) = make_float2(acc[2 * cp][h], acc[2 * cp + 1][h]);
+          *reinterpret_cast<float2*>(o + 16) =
+              make_float2(acc[2 * cp][2 + h], acc[2 * cp + 1][2 + h]);
+        }
+        if (g == 0) {
+          red_m[row] = m[h];
+          red_l[row] = h ? l1 : l0;
         }
       }
     }

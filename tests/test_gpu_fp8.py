@@ -32,6 +32,12 @@ CASES = {
     "ragged_bf16": C["gqa_llama3_8b"].scaled(num_seqs=8, num_blocks=100,
                                              ctx=("fixed", (0, 1, 15, 16, 17, 31, 32, 33)),
                                              seed=55),
+    # the transposed page step at its widest group (all 8 mma columns live)
+    # and at an odd one (3 heads: the second row of some lanes is padding)
+    "gqa8_f16": C["mha_llama2_7b"].scaled(num_seqs=5, num_heads=16, num_kv_heads=2,
+                                          num_blocks=300, ctx=("uniform", 1, 800), seed=56),
+    "gqa3_bf16": C["gqa_llama3_8b"].scaled(num_seqs=5, num_heads=12, num_kv_heads=4,
+                                           num_blocks=300, ctx=("uniform", 1, 800), seed=57),
 }
 
 
@@ -74,7 +80,7 @@ def test_fp8_write_and_decode_match_oracle(name, cuda_device, oracle_lib):
     assert err <= TOL[cfg.dtype], f"{name}: {err:.3e}"
 
 
-@pytest.mark.parametrize("name", ["gqa_bf16", "mha_f16"])
+@pytest.mark.parametrize("name", ["gqa_bf16", "mha_f16", "gqa8_f16", "gqa3_bf16"])
 @pytest.mark.parametrize("ps", [16, 256])
 def test_fp8_split_matches_oracle(name, ps, cuda_device, oracle_lib):
     cfg = CASES[name]
@@ -123,7 +129,7 @@ def test_fp8_split_ragged_and_large_batches(name, ps, cuda_device, oracle_lib):
 
 
 @pytest.mark.parametrize("split", [0, 64])
-@pytest.mark.parametrize("name", ["mha_f16", "gqa_bf16", "gqa16_bf16"])
+@pytest.mark.parametrize("name", ["mha_f16", "gqa_bf16", "gqa16_bf16", "gqa8_f16"])
 def test_fp8_nan_codes_past_context_do_not_leak(name, split, cuda_device, oracle_lib):
     """E4M3 NaN codes (0x7f) in the never-written rows past each context."""
     cfg = CASES[name]
@@ -148,7 +154,7 @@ def test_fp8_nan_codes_past_context_do_not_leak(name, split, cuda_device, oracle
     assert np.max(np.abs(g - ref)) <= TOL[cfg.dtype]
 
 
-@pytest.mark.parametrize("name", ["mha_f16", "gqa_bf16"])
+@pytest.mark.parametrize("name", ["mha_f16", "gqa_bf16", "gqa3_bf16"])
 def test_fp8_context_len_one_is_exact(name, cuda_device):
     # p = 1, and code * 2^-5 is exact in fp32 and in the 16-bit output
     cfg = CASES[name]
