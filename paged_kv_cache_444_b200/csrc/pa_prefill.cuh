@@ -42,7 +42,7 @@
 // P V as a hi + lo pair of bf16 products (at least 14 bits of P, split by
 // bit truncation so the conversion unit stays free for 2^x); fp16 P is
 // rounded once and l sums the rounded values.  With bf16 caches the default
-// build rewrites each V block as fp16 in shared memory (four converter warps)
+// build rewrites each V block as fp16 in shared memory (six converter warps)
 // and takes the fp16 P path instead (PA_PREFILL_V_FP16, below).
 #pragma once
 
@@ -58,7 +58,8 @@ constexpr int kPrefillPages = kPrefillKeys / kPage; // 8 pages per block
 constexpr int kWarpMma = 8;                         // issues every MMA, owns tensor memory
 constexpr int kWarpTma = 9;                         // Q, K and V loads
 constexpr int kPrefillThreads = 10 * 32;            // + two softmax warpgroups (warps 0-7)
-constexpr int kWarpConv = 10;                       // V converters: warps 10-13 (convert mode)
+constexpr int kWarpConv = 10;                       // V converters: warps 10-15 (convert mode)
+constexpr int kConvWarps = 6;
 constexpr unsigned kErrValue = 8;
 constexpr int kRankMaxSeqs = 256;     // batches ranked longest-first by every CTA: sequences,
 constexpr int kRankMaxUnits = 2048;   // units (sequence, tile pair),
@@ -77,7 +78,7 @@ template <bool BF16>
 struct PrefillRoles {
   static constexpr bool kConvert = BF16 && PA_PREFILL_V_FP16 != 0;
   // convert mode: four whole warpgroups (setmaxnreg works per warpgroup):
-  // softmax 0-7, then MMA, TMA, converters 10-13 and two idle warps
+  // softmax 0-7, then MMA, TMA and converters 10-15
   static constexpr int kThreads = kConvert ? 16 * 32 : kPrefillThreads;
   static constexpr bool kPHiLo = BF16 && !kConvert;   // P as a bf16 hi + lo pair
 };
@@ -548,7 +549,7 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
       mbar_init(sb + L::kBarKEmpty + 8 * i, 1);
       mbar_init(sb + L::kBarVFull + 8 * i, 1);
       mbar_init(sb + L::kBarVEmpty + 8 * i, 1);
-      if constexpr (R::kConvert) mbar_init(sb + L::kBarVConv + 8 * i, 128);
+      if constexpr (R::kConvert) mbar_init(sb + L::kBarVConv + 8 * i, kConvWarps * 32);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(sb + L::kBarS + 8 * t, 1);
@@ -577,7 +578,7 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
   // the warpgroup index, made visibly warp-uniform for the register split
   const int wgroup = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x) / 128, 0);
   if (wgroup >= 2) {
-  // warpgroups 2 and 3: MMA issuer, TMA producer, V converters, idle warps
+  // warpgroups 2 and 3: MMA issuer, TMA producer, V converters
   if constexpr (R::kConvert) regs_decrease();
   if (warp == kWarpTma) {
     // ================= TMA producer =================
@@ -779,13 +780,13 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
     if (lane == 0) umma_commit(sb + L::kBarO);
     __syncwarp();
     if (!mbar_wait_bounded(sb + L::kBarO, 0) && lane == 0) record_error(kErrWaitTimeout, blockIdx.x);
-  } else if (R::kConvert && warp >= kWarpConv && warp < kWarpConv + 4) {
+  } else if (R::kConvert && warp >= kWarpConv && warp < kWarpConv + kConvWarps) {
     // ================= V converters (convert mode) =================
     // Each landed V block (bf16, 128 keys x D, two or one 128-byte-swizzled
     // slabs) is rewritten in place as fp16, element for element (the swizzle
     // moves whole 16-byte chunks, so chunk positions are unchanged), and rows
     // past the context in the sequence's last page are cleared.
-    const int ct = threadIdx.x - kWarpConv * 32;   // 0 .. 127
+    const int ct = threadIdx.x - kWarpConv * 32;   // 0 .. kConvWarps * 32 - 1
     int g0 = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
@@ -795,7 +796,7 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
       if (!prefill_item(a, list, ranked, i, t2, it)) continue;
       const int last_page = (it.ctx - 1) / kPage;
       const int tail_row = it.ctx % kPage;
-      uint32_t clipped = 0;
+      uint32_t hmax = 0;   // per-half maximum of |fp16| written
       for (int j = 0; j < it.nkb; ++j) {
         const int g = g0 + j, st = g % NST;
         if (!(ok = __all_sync(0xffffffffu, wait_or_abort(sb + L::kBarVFull + 8 * st,
@@ -803,11 +804,12 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
           break;
         const uint32_t vst = sb + L::kV + st * L::kStage;
         const int lp = last_page - j * kPrefillPages;  // this block's page holding the end, if any
-        for (int c = ct; c < L::kStage / 16; c += 128) {
+        const bool tail_block = tail_row != 0 && lp >= 0 && lp < kPrefillPages;
+        for (int c = ct; c < L::kStage / 16; c += kConvWarps * 32) {
           const int row = (c >> 3) & (kPrefillKeys - 1);   // key within the block
           const uint32_t addr = vst + c * 16;
           uint32_t w[4];
-          if (tail_row != 0 && (row >> 4) == lp && (row & 15) >= tail_row) {
+          if (tail_block && (row >> 4) == lp && (row & 15) >= tail_row) {
             w[0] = w[1] = w[2] = w[3] = 0u;
           } else {
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -817,8 +819,7 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
               const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xffff0000u);
               uint32_t h;
               asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(hi), "f"(lo));
-              // no bf16 value is 65 504, so a half of magnitude 65 504 was clipped
-              clipped |= __vcmpeq2(h & 0x7fff7fffu, 0x7bff7bffu);
+              hmax = __vmaxu2(hmax, h & 0x7fff7fffu);
               w[q] = h;
             }
           }
@@ -827,7 +828,9 @@ __global__ void __launch_bounds__(PrefillRoles<BF16>::kThreads, 1)
         fence_proxy_async_smem();
         mbar_arrive(sb + L::kBarVConv + 8 * st);
       }
-      if (__any_sync(0xffffffffu, clipped != 0) && lane == 0) record_error(kErrValue, it.s);
+      // no bf16 value is 65 504, so a half of magnitude 65 504 was clipped
+      if (__any_sync(0xffffffffu, __vcmpeq2(hmax, 0x7bff7bffu) != 0) && lane == 0)
+        record_error(kErrValue, it.s);
       g0 += it.nkb;
     }
   }
