@@ -203,3 +203,34 @@ def test_fp8_full_size_gqa_sampled(cuda_device, oracle_lib):
     assert np.array_equal(kc.index_select(0, ids).cpu().numpy(), kh)
     err = np.max(np.abs(to_f64(out[seqs]) - ref))
     assert err <= TOL["bf16"], err
+
+
+@pytest.mark.parametrize("name,ctx", [
+    # a block table wide enough (> 512 pages) that single-pass fp8 decode
+    # runs in thread-block clusters: items over 256 pages are spread over the
+    # CTAs of their cluster and merged through distributed shared memory,
+    # shorter ones stay on one CTA
+    ("gqa_bf16", (1, 40, 4097, 5000, 17000)),   # transposed page step, group 4
+    ("mha_f16", (4300, 1, 8200)),               # transposed page step, one head
+    ("gqa16_bf16", (17, 9000, 4200)),           # 16-row tile, group 16
+])
+def test_fp8_cluster_spread_items_match_oracle(name, ctx, cuda_device, oracle_lib):
+    base = CASES[name]
+    need = sum((c + 15) // 16 for c in ctx)
+    cfg = base.scaled(num_seqs=len(ctx), ctx=("fixed", ctx), num_blocks=need + 64)
+    b, kc, vc = _fp8_batch(cfg, cuda_device)
+    width = 1100  # table columns past each sequence's pages are never read
+    pad = torch.full((cfg.num_seqs, width - b.block_tables.shape[1]), -1, dtype=torch.int32,
+                     device=cuda_device)
+    b.block_tables = torch.cat([b.block_tables, pad], dim=1).contiguous()
+    ref, _, _ = _oracle(oracle_lib, b, kc, vc)
+    pa_reshape_and_cache_fp8(b.key, b.value, kc, vc, b.slot_mapping, K_SCALE, V_SCALE)
+    out = torch.full_like(b.query, float("nan"))
+    pa_decode_fp8(out, b.query, kc, vc, b.block_tables, b.context_lens, cfg.scale, K_SCALE,
+                  V_SCALE)
+    torch.cuda.synchronize()
+    pa_check_error()
+    g = to_f64(out)
+    assert np.isfinite(g).all()
+    err = np.max(np.abs(g - ref))
+    assert err <= TOL[cfg.dtype], f"{name} spread: {err:.3e}"
