@@ -258,7 +258,7 @@ template <int D, bool BF16>
 pa_status launch_decode_d(const CUtensorMap& km, const CUtensorMap& vm, const DecodeArgs& a,
                           long long grid, int64_t max_pages, cudaStream_t stream) {
   if (a.group <= 8)
-    return launch_decode_t<D, BF16, MmaWarp<D, BF16, false>>(km, vm, a, grid, max_pages, stream);
+    return launch_decode_t<D, BF16, MmaWarpT<D, BF16>>(km, vm, a, grid, max_pages, stream);
   return launch_decode_t<D, BF16, MmaWarp<D, BF16, true>>(km, vm, a, grid, max_pages, stream);
 }
 

@@ -23,13 +23,15 @@
 // window of 32 ids held one per lane (a second window is prefetched).
 //
 // Math.  fp32 throughout.  The G query heads of a KV head (1 for MHA, up to
-// 16 for GQA) form a small dense contraction: S = Q K^T and O += P V run as
-// mma.sync m16n8k16 with fp32 accumulators (Q rows padded to 16, P in the
-// cache dtype for the second product, bf16 as a hi + lo pair).  For one head
-// the tile has a single live row: the tensor cores take the products off the
-// issue path, which measured faster than packed fp32 FMA on the CUDA cores.
-// The softmax is online, in base 2 with scale*log2(e) folded into the logits,
-// with warp-shuffle max reductions.
+// 16 for GQA) form a small dense contraction on mma.sync m16n8k16 with fp32
+// accumulators (P in the cache dtype for the second product, bf16 as a hi +
+// lo pair).  Groups of up to 8 heads run both products transposed (MmaWarpT:
+// S^T = K Q^T, O^T = V^T P^T, tokens and head dims as the mma's 16 rows, the
+// heads as its 8 columns); groups of 9 to 16 run a 16-row query tile
+// (MmaWarp), which the shared-prefix kernel also uses.  Even for one head the
+// tensor cores take the products off the issue path, which measured faster
+// than packed fp32 FMA on the CUDA cores.  The softmax is online, in base 2
+// with scale*log2(e) folded into the logits, with warp-shuffle max reductions.
 #pragma once
 
 #include "pa_device.cuh"
@@ -103,7 +105,8 @@ __device__ __forceinline__ uint32_t page_chunk(uint32_t base, int r, int c) {
 }
 
 // ---------------------------------------------------------------------------
-// Per-warp state and page step (tensor cores, every group size)
+// Per-warp state and page step with a 16-row query tile (groups of 9 to 16,
+// and the shared-prefix kernel's member rows)
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool TWO_ROWS>
 struct MmaWarp {
@@ -280,6 +283,132 @@ struct MmaWarp {
         if (tig == 0) {
           red_m[r1] = m[1];
           red_l[r1] = l1;
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Page step with both products transposed, for groups of up to 8 query heads:
+// S^T = K Q^T and O^T = V^T P^T, with the page's 16 tokens (first product)
+// and 16-dim slices of the head (second) as the mma's M = 16 rows and the
+// group's query heads as its N = 8 columns.  K comes in as A fragments
+// through the plain ldmatrix, V^T through the transposed one, and the S^T
+// accumulator (token, query row) becomes the B operand of the second product
+// by one movmatrix transpose per 8 tokens.  bf16 P goes in as a hi + lo pair.
+// ---------------------------------------------------------------------------
+template <int D, bool BF16>
+struct MmaWarpT {
+  static constexpr int kMinBlocks = 0;
+  static constexpr int KSTEPS = D / 16;
+  static constexpr int MTILES = D / 16;
+  uint32_t qb[KSTEPS][2];  // Q^T B fragments of query row lane / 4
+  float acc[MTILES][4];    // O^T: (dim 16c + g, rows 2t, 2t+1), (dim 16c + 8 + g, ...)
+  float m[2], l[2];        // query rows 2t, 2t+1
+
+  __device__ __forceinline__ void init(const uint16_t* q_group, int group, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t* q = reinterpret_cast<const uint32_t*>(q_group + g * D);
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      qb[kk][0] = g < group ? q[(kk * 16 + 2 * t) >> 1] : 0u;
+      qb[kk][1] = g < group ? q[(kk * 16 + 8 + 2 * t) >> 1] : 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.f;
+  }
+
+  __device__ __forceinline__ void page(uint32_t kbase, uint32_t vbase, int tok0, int t_end,
+                                       float scale_log2, int lane) {
+    const int g = lane >> 2;
+    // ---- S^T = K Q^T ----
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+    const int ktok = (lane & 7) + ((lane >> 3) & 1) * 8;
+    const int kchk = lane >> 4;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      uint32_t a[4];  // (tok 0-7, chunk 2kk) (8-15, 2kk) (0-7, 2kk+1) (8-15, 2kk+1)
+      ldsm_x4(page_chunk<D>(kbase, ktok, 2 * kk + kchk), a[0], a[1], a[2], a[3]);
+      if (kk & 1) mma_16816<BF16>(s1, a, qb[kk][0], qb[kk][1]);
+      else        mma_16816<BF16>(s0, a, qb[kk][0], qb[kk][1]);
+    }
+    const int lim = t_end - tok0;
+    const bool lo_live = g < lim, hi_live = g + 8 < lim;
+    const float x0 = lo_live ? (s0[0] + s1[0]) * scale_log2 : -INFINITY;  // token g, row 2t
+    const float x1 = lo_live ? (s0[1] + s1[1]) * scale_log2 : -INFINITY;  // token g, row 2t+1
+    const float x2 = hi_live ? (s0[2] + s1[2]) * scale_log2 : -INFINITY;  // token g+8, row 2t
+    const float x3 = hi_live ? (s0[3] + s1[3]) * scale_log2 : -INFINITY;
+    const bool odd = g & 1;
+    float keep = odd ? fmaxf(x1, x3) : fmaxf(x0, x2);
+    const float send = odd ? fmaxf(x0, x2) : fmaxf(x1, x3);
+    keep = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+    keep = fmaxf(keep, __shfl_xor_sync(0xffffffffu, keep, 8));
+    keep = fmaxf(keep, __shfl_xor_sync(0xffffffffu, keep, 16));
+    const float other = __shfl_xor_sync(0xffffffffu, keep, 4);
+    const float mn0 = fmaxf(m[0], odd ? other : keep);
+    const float mn1 = fmaxf(m[1], odd ? keep : other);
+    const float al0 = ex2(m[0] - mn0), al1 = ex2(m[1] - mn1);
+    m[0] = mn0;
+    m[1] = mn1;
+    const float p0 = ex2(x0 - mn0), p1 = ex2(x1 - mn1), p2 = ex2(x2 - mn0), p3 = ex2(x3 - mn1);
+    const uint32_t h_lo = pack2<BF16>(p0, p1), h_hi = pack2<BF16>(p2, p3);
+    uint32_t pb[4];
+    pb[0] = movmatrix_trans(h_lo);
+    pb[1] = movmatrix_trans(h_hi);
+    if constexpr (BF16) {
+      const float2 u = unpack2<true>(h_lo), w = unpack2<true>(h_hi);
+      pb[2] = movmatrix_trans(pack2<true>(p0 - u.x, p1 - u.y));
+      pb[3] = movmatrix_trans(pack2<true>(p2 - w.x, p3 - w.y));
+      l[0] = l[0] * al0 + (p0 + p2);
+      l[1] = l[1] * al1 + (p1 + p3);
+    } else {
+      const float2 u = unpack2<false>(h_lo), w = unpack2<false>(h_hi);
+      l[0] = l[0] * al0 + (u.x + w.x);
+      l[1] = l[1] * al1 + (u.y + w.y);
+    }
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+      acc[i][0] *= al0;
+      acc[i][1] *= al1;
+      acc[i][2] *= al0;
+      acc[i][3] *= al1;
+    }
+    // ---- O^T += V^T P^T ----
+    const int vtok = (lane & 7) + (lane >> 4) * 8;
+    const int vchk = (lane >> 3) & 1;
+#pragma unroll
+    for (int c = 0; c < MTILES; ++c) {
+      uint32_t a[4];  // (tok 0-7, chunk 2c) (0-7, 2c+1) (8-15, 2c) (8-15, 2c+1), transposed
+      ldsm_x4_trans(page_chunk<D>(vbase, vtok, 2 * c + vchk), a[0], a[1], a[2], a[3]);
+      mma_16816<BF16>(acc[c], a, pb[0], pb[1]);
+      if constexpr (BF16) mma_16816<BF16>(acc[c], a, pb[2], pb[3]);
+    }
+  }
+
+  __device__ __forceinline__ void publish(float* red_acc, float* red_m, float* red_l, int group,
+                                          int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    float l0 = l[0], l1 = l[1];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = 2 * t + h;
+      if (row < group) {
+#pragma unroll
+        for (int c = 0; c < MTILES; ++c) {
+          red_acc[row * D + 16 * c + g] = acc[c][h];
+          red_acc[row * D + 16 * c + 8 + g] = acc[c][2 + h];
+        }
+        if (g == 0) {
+          red_m[row] = m[h];
+          red_l[row] = h ? l1 : l0;
         }
       }
     }

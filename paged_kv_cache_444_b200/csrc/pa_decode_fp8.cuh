@@ -240,13 +240,6 @@ __device__ __forceinline__ void e4m3x4_to_h2x2(uint32_t x, uint32_t& lo, uint32_
       : "r"(x));
 }
 
-// Transpose of an 8 x 8 matrix of 16-bit elements held in the mma fragment
-// layout (lane l: row l / 4, elements 2(l % 4) and 2(l % 4) + 1).  Whole warp.
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
 
 // ---------------------------------------------------------------------------
 // Tensor-core path for groups of up to 8 query heads: both products

@@ -149,6 +149,14 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
                : "r"(addr));
 }
 
+// Transpose of an 8 x 8 matrix of 16-bit elements held in the mma fragment
+// layout (lane l: row l / 4, elements 2(l % 4) and 2(l % 4) + 1).  Whole warp.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------------------
 // mma.sync m16n8k16, fp32 accumulate, A row-major / B column-major.
 // ---------------------------------------------------------------------------
