@@ -886,9 +886,11 @@ OFF_DECODE_PATH = ("pa_prefill.cuh", "pa_umma.cuh", "pa_shared_prefix.cuh", "pa_
 
 
 def kernel_source_digest(csrc: Path | None = None) -> str:
-    """Hash of the decode path's sources: every csrc file but those off the
+    """Hash of the decode path's code: every csrc file but those off the
     path, with the marked host-side regions of pa_api.cu that serve other
-    kernels ("// >>> ..." to "// <<< ...") left out."""
+    kernels ("// >>> ..." to "// <<< ...") left out, then comments, trailing
+    blanks and empty lines removed, so that an edit of comments alone keeps
+    the hash (and the traffic captured for the code)."""
     import hashlib
     import re
     h = hashlib.sha256()
@@ -898,7 +900,11 @@ def kernel_source_digest(csrc: Path | None = None) -> str:
         data = p.read_bytes()
         if p.name == "pa_api.cu":
             data = re.sub(rb"\n// >>> .*?\n// <<< [^\n]*", b"", data, flags=re.S)
-        h.update(data)
+        data = re.sub(rb"/\*.*?\*/", b"", data, flags=re.S)
+        data = re.sub(rb"//[^\n]*", b"", data)
+        data = re.sub(rb"[ \t]+\n", b"\n", data)
+        data = re.sub(rb"\n\s*\n", b"\n", data)
+        h.update(p.name.encode() + b"\0" + data)
     return h.hexdigest()[:16]
 
 

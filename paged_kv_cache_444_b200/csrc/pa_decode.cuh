@@ -335,12 +335,16 @@ struct MmaWarpT {
       if (kk & 1) mma_16816<BF16>(s1, a, qb[kk][0], qb[kk][1]);
       else        mma_16816<BF16>(s0, a, qb[kk][0], qb[kk][1]);
     }
+    // ---- scale, mask the tail, row maxima over the page's 16 tokens ----
     const int lim = t_end - tok0;
     const bool lo_live = g < lim, hi_live = g + 8 < lim;
     const float x0 = lo_live ? (s0[0] + s1[0]) * scale_log2 : -INFINITY;  // token g, row 2t
     const float x1 = lo_live ? (s0[1] + s1[1]) * scale_log2 : -INFINITY;  // token g, row 2t+1
     const float x2 = hi_live ? (s0[2] + s1[2]) * scale_log2 : -INFINITY;  // token g+8, row 2t
     const float x3 = hi_live ? (s0[3] + s1[3]) * scale_log2 : -INFINITY;
+    // lanes of equal t hold the same two rows; each reduces one of them over
+    // the 8 lanes and the other comes back from the neighbour of opposite g
+    // parity (token 0 of the page is always live, so the maxima are finite)
     const bool odd = g & 1;
     float keep = odd ? fmaxf(x1, x3) : fmaxf(x0, x2);
     const float send = odd ? fmaxf(x0, x2) : fmaxf(x1, x3);
@@ -353,6 +357,9 @@ struct MmaWarpT {
     const float al0 = ex2(m[0] - mn0), al1 = ex2(m[1] - mn1);
     m[0] = mn0;
     m[1] = mn1;
+    // ---- P in the cache dtype as the B operand of the second product: fp16 P
+    // once (l sums the rounded values), bf16 P as a hi + lo pair (l sums the
+    // fp32 p) ----
     const float p0 = ex2(x0 - mn0), p1 = ex2(x1 - mn1), p2 = ex2(x2 - mn0), p3 = ex2(x3 - mn1);
     const uint32_t h_lo = pack2<BF16>(p0, p1), h_hi = pack2<BF16>(p2, p3);
     uint32_t pb[4];
