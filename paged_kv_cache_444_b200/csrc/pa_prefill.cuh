@@ -41,7 +41,7 @@
 // 16-bit operand and the final 1/l uses the same reference).  bf16 P enters
 // P V as a hi + lo pair of bf16 products (at least 14 bits of P, split by
 // bit truncation so the conversion unit stays free for 2^x); fp16 P is
-// rounded once and l sums the rounded values.  With bf16 caches the default
+// rounded once and l sums the fp32 p.  With bf16 caches the default
 // build rewrites each V block as fp16 in shared memory (six converter warps)
 // and takes the fp16 P path instead (PA_PREFILL_V_FP16, below).
 #pragma once
@@ -357,8 +357,10 @@ __device__ __forceinline__ void prefill_softmax_block(float (&p)[kPrefillKeys], 
         lo[q] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
         lsum[q & 3] = ffma2(make_float2(x0, x1), make_float2(1.f, 1.f), lsum[q & 3]);
       } else {
+        // l sums the fp32 p (P.V takes them rounded to fp16: O / l is off
+        // by at most 2^-11 relative, summed over keys with random signs)
         h[q] = pack2<false>(x0, x1);
-        lsum[q & 3] = ffma2(unpack2<false>(h[q]), make_float2(1.f, 1.f), lsum[q & 3]);
+        lsum[q & 3] = ffma2(make_float2(x0, x1), make_float2(1.f, 1.f), lsum[q & 3]);
       }
     }
     tmem_st32u(t_lane + s_col + 32 * half, h);
