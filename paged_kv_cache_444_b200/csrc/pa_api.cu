@@ -259,7 +259,7 @@ pa_status launch_decode_d(const CUtensorMap& km, const CUtensorMap& vm, const De
                           long long grid, int64_t max_pages, cudaStream_t stream) {
   if (a.group <= 8)
     return launch_decode_t<D, BF16, MmaWarpT<D, BF16>>(km, vm, a, grid, max_pages, stream);
-  return launch_decode_t<D, BF16, MmaWarp<D, BF16, true>>(km, vm, a, grid, max_pages, stream);
+  return launch_decode_t<D, BF16, MmaWarp<D, BF16>>(km, vm, a, grid, max_pages, stream);
 }
 
 // Shared validation of the attention arguments (host only, no CUDA calls).
@@ -337,13 +337,13 @@ pa_status run_decode_fp8(DecodeArgs a, const void* key_cache, const void* value_
     if (a.group <= 8)
       return launch_decode_t<128, true, MmaFp8WarpT<128, true>, 1, PA_STAGES_FP8_T>(
           km, vm, a, grid, max_pages, stream);
-    return launch_decode_t<128, true, MmaFp8Warp<128, true, true>, 1>(km, vm, a, grid, max_pages,
+    return launch_decode_t<128, true, MmaFp8Warp<128, true>, 1>(km, vm, a, grid, max_pages,
                                                                      stream);
   }
   if (a.group <= 8)
     return launch_decode_t<128, false, MmaFp8WarpT<128, false>, 1, PA_STAGES_FP8_T>(
         km, vm, a, grid, max_pages, stream);
-  return launch_decode_t<128, false, MmaFp8Warp<128, false, true>, 1>(km, vm, a, grid, max_pages,
+  return launch_decode_t<128, false, MmaFp8Warp<128, false>, 1>(km, vm, a, grid, max_pages,
                                                                      stream);
 }
 // <<< fp8 KV cache launch

@@ -108,7 +108,7 @@ __device__ __forceinline__ uint32_t page_chunk(uint32_t base, int r, int c) {
 // Per-warp state and page step with a 16-row query tile (groups of 9 to 16,
 // and the shared-prefix kernel's member rows)
 // ---------------------------------------------------------------------------
-template <int D, bool BF16, bool TWO_ROWS>
+template <int D, bool BF16>
 struct MmaWarp {
   static constexpr int KSTEPS = D / 16;  // k-steps of 16 over head_dim
   static constexpr int NTILES = D / 8;   // 8-wide n-tiles of the output
@@ -125,9 +125,9 @@ struct MmaWarp {
       const uint32_t* q0 = reinterpret_cast<const uint32_t*>(q_group + r0 * D);
       const uint32_t* q1 = reinterpret_cast<const uint32_t*>(q_group + r1 * D);
       qa[kk][0] = r0 < group ? q0[klo >> 1] : 0u;
-      qa[kk][1] = (TWO_ROWS && r1 < group) ? q1[klo >> 1] : 0u;
+      qa[kk][1] = r1 < group ? q1[klo >> 1] : 0u;
       qa[kk][2] = r0 < group ? q0[khi >> 1] : 0u;
-      qa[kk][3] = (TWO_ROWS && r1 < group) ? q1[khi >> 1] : 0u;
+      qa[kk][3] = r1 < group ? q1[khi >> 1] : 0u;
     }
 #pragma unroll
     for (int n = 0; n < NTILES; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
@@ -173,21 +173,16 @@ struct MmaWarp {
     }
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
     // reference max: the running max, or 0 while a row has seen no token
     // (then every exponent below is of -inf and gives 0, never NaN)
-    const float mn0r = fmaxf(m[0], mx0);
+    const float mn0r = fmaxf(m[0], mx0), mn1r = fmaxf(m[1], mx1);
     const float mn0 = mn0r == -INFINITY ? 0.f : mn0r;
-    const float al0 = ex2(m[0] - mn0);
+    const float mn1 = mn1r == -INFINITY ? 0.f : mn1r;
+    const float al0 = ex2(m[0] - mn0), al1 = ex2(m[1] - mn1);
     m[0] = mn0r;
-    float mn1 = 0.f, al1 = 1.f;
-    if constexpr (TWO_ROWS) {
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float mn1r = fmaxf(m[1], mx1);
-      mn1 = mn1r == -INFINITY ? 0.f : mn1r;
-      al1 = ex2(m[1] - mn1);
-      m[1] = mn1r;
-    }
+    m[1] = mn1r;
     // ---- P = 2^(x - m) as the A operand of P V.  bf16 keeps 8 mantissa
     // bits, so P goes in as a hi + lo pair of bf16 (about 16 bits, two mma
     // per tile) and l sums the unrounded fp32 p; fp16 (11 bits) goes in once
@@ -195,47 +190,35 @@ struct MmaWarp {
     float p0[4], p1[4];
     p0[0] = ex2(sc[0][0] - mn0); p0[1] = ex2(sc[0][1] - mn0);
     p0[2] = ex2(sc[1][0] - mn0); p0[3] = ex2(sc[1][1] - mn0);
-    if constexpr (TWO_ROWS) {
-      p1[0] = ex2(sc[0][2] - mn1); p1[1] = ex2(sc[0][3] - mn1);
-      p1[2] = ex2(sc[1][2] - mn1); p1[3] = ex2(sc[1][3] - mn1);
-    } else {
-      p1[0] = p1[1] = p1[2] = p1[3] = 0.f;
-    }
+    p1[0] = ex2(sc[0][2] - mn1); p1[1] = ex2(sc[0][3] - mn1);
+    p1[2] = ex2(sc[1][2] - mn1); p1[3] = ex2(sc[1][3] - mn1);
     uint32_t pa[4], pl[4];
     pa[0] = pack2<BF16>(p0[0], p0[1]);
     pa[2] = pack2<BF16>(p0[2], p0[3]);
-    pa[1] = TWO_ROWS ? pack2<BF16>(p1[0], p1[1]) : 0u;
-    pa[3] = TWO_ROWS ? pack2<BF16>(p1[2], p1[3]) : 0u;
+    pa[1] = pack2<BF16>(p1[0], p1[1]);
+    pa[3] = pack2<BF16>(p1[2], p1[3]);
     if constexpr (BF16) {
       const float2 h0 = unpack2<BF16>(pa[0]), h2 = unpack2<BF16>(pa[2]);
+      const float2 h1 = unpack2<BF16>(pa[1]), h3 = unpack2<BF16>(pa[3]);
       pl[0] = pack2<BF16>(p0[0] - h0.x, p0[1] - h0.y);
       pl[2] = pack2<BF16>(p0[2] - h2.x, p0[3] - h2.y);
-      if constexpr (TWO_ROWS) {
-        const float2 h1 = unpack2<BF16>(pa[1]), h3 = unpack2<BF16>(pa[3]);
-        pl[1] = pack2<BF16>(p1[0] - h1.x, p1[1] - h1.y);
-        pl[3] = pack2<BF16>(p1[2] - h3.x, p1[3] - h3.y);
-      } else {
-        pl[1] = pl[3] = 0u;
-      }
+      pl[1] = pack2<BF16>(p1[0] - h1.x, p1[1] - h1.y);
+      pl[3] = pack2<BF16>(p1[2] - h3.x, p1[3] - h3.y);
       l[0] = l[0] * al0 + ((p0[0] + p0[1]) + (p0[2] + p0[3]));
-      if constexpr (TWO_ROWS) l[1] = l[1] * al1 + ((p1[0] + p1[1]) + (p1[2] + p1[3]));
+      l[1] = l[1] * al1 + ((p1[0] + p1[1]) + (p1[2] + p1[3]));
     } else {
       const float2 u = unpack2<BF16>(pa[0]), v = unpack2<BF16>(pa[2]);
+      const float2 w = unpack2<BF16>(pa[1]), z = unpack2<BF16>(pa[3]);
       l[0] = l[0] * al0 + ((u.x + u.y) + (v.x + v.y));
-      if constexpr (TWO_ROWS) {
-        const float2 w = unpack2<BF16>(pa[1]), z = unpack2<BF16>(pa[3]);
-        l[1] = l[1] * al1 + ((w.x + w.y) + (z.x + z.y));
-      }
+      l[1] = l[1] * al1 + ((w.x + w.y) + (z.x + z.y));
     }
     // ---- rescale O, then O += P V ----
 #pragma unroll
     for (int n = 0; n < NTILES; ++n) {
       acc[n][0] *= al0;
       acc[n][1] *= al0;
-      if constexpr (TWO_ROWS) {
-        acc[n][2] *= al1;
-        acc[n][3] *= al1;
-      }
+      acc[n][2] *= al1;
+      acc[n][3] *= al1;
     }
     const int vtok = ((lane >> 3) & 1) * 8 + (lane & 7);
     const int vchk = lane >> 4;
@@ -256,14 +239,11 @@ struct MmaWarp {
   __device__ __forceinline__ void publish(float* red_acc, float* red_m, float* red_l, int group,
                                           int lane) {
     const int r0 = lane >> 2, r1 = r0 + 8, tig = lane & 3;
-    float l0 = l[0];
+    float l0 = l[0], l1 = l[1];
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    float l1 = l[1];
-    if constexpr (TWO_ROWS) {
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    }
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
     if (r0 < group) {
 #pragma unroll
       for (int n = 0; n < NTILES; ++n)
@@ -274,16 +254,14 @@ struct MmaWarp {
         red_l[r0] = l0;
       }
     }
-    if constexpr (TWO_ROWS) {
-      if (r1 < group) {
+    if (r1 < group) {
 #pragma unroll
-        for (int n = 0; n < NTILES; ++n)
-          *reinterpret_cast<float2*>(red_acc + r1 * D + n * 8 + tig * 2) =
-              make_float2(acc[n][2], acc[n][3]);
-        if (tig == 0) {
-          red_m[r1] = m[1];
-          red_l[r1] = l1;
-        }
+      for (int n = 0; n < NTILES; ++n)
+        *reinterpret_cast<float2*>(red_acc + r1 * D + n * 8 + tig * 2) =
+            make_float2(acc[n][2], acc[n][3]);
+      if (tig == 0) {
+        red_m[r1] = m[1];
+        red_l[r1] = l1;
       }
     }
   }

@@ -32,7 +32,6 @@ namespace pa {
 
 // ---------------------------------------------------------------------------
 // Tensor-core path with a 16-row query tile (groups of 9 to 16), head_dim 128.
-// Its query prescale and pow2 serve the transposed step below too.
 //
 // Both products run as fp16 mma whatever the query dtype: E4M3 -> fp16 is one
 // exact conversion, and P in fp16 keeps 11 bits.  A bf16 (or fp16) query row
@@ -41,7 +40,18 @@ namespace pa {
 // the row's logit scale.  Only elements more than 2^27 below the row's
 // largest can lose bits, and they cannot move a logit.
 // ---------------------------------------------------------------------------
-template <int D, bool BF16, bool TWO_ROWS>
+// 2^e as a float, e in [-126, 127].
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+
+// The s for which 2^s brings a row whose largest |element| is mx into
+// [2^13, 2^14) (0 for an all-zero row).
+__device__ __forceinline__ int query_prescale_exp(float mx) {
+  if (!(mx > 0.f)) return 0;
+  const int e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 127;  // floor(log2 mx)
+  return max(-100, min(100, 13 - e));
+}
+
+template <int D, bool BF16>
 struct MmaFp8Warp {
   static_assert(D == 128, "fp8 tensor-core path is built for head_dim 128");
   static constexpr int kMinBlocks = 3;  // three CTAs per SM: at most 168 registers
@@ -51,17 +61,6 @@ struct MmaFp8Warp {
   float acc[NTILES][4];     // n-tile 2c: even dims of 16-dim chunk c; 2c+1: odd dims
   float m[2], l[2];
   float rs[2];              // 2^-s of rows r0, r1 (undo the query prescale)
-
-  __device__ __forceinline__ static float pow2(int e) {
-    return __int_as_float((e + 127) << 23);  // e in [-126, 127]
-  }
-
-  // 2^s that brings a row whose largest |element| is mx into [2^13, 2^14)
-  __device__ __forceinline__ static int prescale_exp(float mx) {
-    if (!(mx > 0.f)) return 0;
-    const int e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 127;  // floor(log2 mx)
-    return max(-100, min(100, 13 - e));
-  }
 
   __device__ __forceinline__ void init(const uint16_t* q_group, int group, int lane) {
     const int r0 = lane >> 2, r1 = r0 + 8, tig = lane & 3;
@@ -76,8 +75,8 @@ struct MmaFp8Warp {
       const uint32_t* q1 = reinterpret_cast<const uint32_t*>(q_group + r1 * D);
       v0[kk][0] = unpack2<BF16>(r0 < group ? q0[d0 >> 1] : 0u);
       v0[kk][1] = unpack2<BF16>(r0 < group ? q0[(d0 >> 1) + 1] : 0u);
-      v1[kk][0] = unpack2<BF16>((TWO_ROWS && r1 < group) ? q1[d0 >> 1] : 0u);
-      v1[kk][1] = unpack2<BF16>((TWO_ROWS && r1 < group) ? q1[(d0 >> 1) + 1] : 0u);
+      v1[kk][0] = unpack2<BF16>(r1 < group ? q1[d0 >> 1] : 0u);
+      v1[kk][1] = unpack2<BF16>(r1 < group ? q1[(d0 >> 1) + 1] : 0u);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         mx0 = fmaxf(mx0, fmaxf(fabsf(v0[kk][h].x), fabsf(v0[kk][h].y)));
@@ -88,10 +87,10 @@ struct MmaFp8Warp {
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const int s0 = prescale_exp(mx0), s1 = prescale_exp(mx1);
-    const float f0 = pow2(s0), f1 = pow2(s1);
-    rs[0] = pow2(-s0);
-    rs[1] = pow2(-s1);
+    const int s0 = query_prescale_exp(mx0), s1 = query_prescale_exp(mx1);
+    const float f0 = pow2i(s0), f1 = pow2i(s1);
+    rs[0] = pow2i(-s0);
+    rs[1] = pow2i(-s1);
 #pragma unroll
     for (int kk = 0; kk < KSTEPS; ++kk) {
       qa[kk][0] = pack2<false>(v0[kk][0].x * f0, v0[kk][0].y * f0);
@@ -139,41 +138,31 @@ struct MmaFp8Warp {
     }
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    const float mn0 = fmaxf(m[0], mx0);
-    const float al0 = ex2(m[0] - mn0);
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    // token 0 of the page is always live, so both maxima are finite
+    const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+    const float al0 = ex2(m[0] - mn0), al1 = ex2(m[1] - mn1);
     m[0] = mn0;
-    float mn1 = 0.f, al1 = 1.f;
-    if constexpr (TWO_ROWS) {
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      mn1 = fmaxf(m[1], mx1);
-      al1 = ex2(m[1] - mn1);
-      m[1] = mn1;
-    }
+    m[1] = mn1;
     // ---- P in fp16; l sums the same rounded values ----
     uint32_t pa[4];
     pa[0] = pack2<false>(ex2(sc[0][0] - mn0), ex2(sc[0][1] - mn0));
     pa[2] = pack2<false>(ex2(sc[1][0] - mn0), ex2(sc[1][1] - mn0));
+    pa[1] = pack2<false>(ex2(sc[0][2] - mn1), ex2(sc[0][3] - mn1));
+    pa[3] = pack2<false>(ex2(sc[1][2] - mn1), ex2(sc[1][3] - mn1));
     {
       const float2 u = unpack2<false>(pa[0]), v = unpack2<false>(pa[2]);
+      const float2 w = unpack2<false>(pa[1]), z = unpack2<false>(pa[3]);
       l[0] = l[0] * al0 + ((u.x + u.y) + (v.x + v.y));
-    }
-    if constexpr (TWO_ROWS) {
-      pa[1] = pack2<false>(ex2(sc[0][2] - mn1), ex2(sc[0][3] - mn1));
-      pa[3] = pack2<false>(ex2(sc[1][2] - mn1), ex2(sc[1][3] - mn1));
-      const float2 u = unpack2<false>(pa[1]), v = unpack2<false>(pa[3]);
-      l[1] = l[1] * al1 + ((u.x + u.y) + (v.x + v.y));
-    } else {
-      pa[1] = pa[3] = 0u;
+      l[1] = l[1] * al1 + ((w.x + w.y) + (z.x + z.y));
     }
 #pragma unroll
     for (int n = 0; n < NTILES; ++n) {
       acc[n][0] *= al0;
       acc[n][1] *= al0;
-      if constexpr (TWO_ROWS) {
-        acc[n][2] *= al1;
-        acc[n][3] *= al1;
-      }
+      acc[n][2] *= al1;
+      acc[n][3] *= al1;
     }
     // ---- O += P V: one transposed x4 ldmatrix covers two 16-dim chunks.  Each
     // register holds codes [t0: d, d+1][t1: d, d+1] (t0 = 2*tig, d = 2*(lane/4));
@@ -199,14 +188,11 @@ struct MmaFp8Warp {
   __device__ __forceinline__ void publish(float* red_acc, float* red_m, float* red_l, int group,
                                           int lane) {
     const int r0 = lane >> 2, r1 = r0 + 8, tig = lane & 3;
-    float l0 = l[0];
+    float l0 = l[0], l1 = l[1];
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    float l1 = l[1];
-    if constexpr (TWO_ROWS) {
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    }
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
     if (r0 < group) {
 #pragma unroll
       for (int c = 0; c < D / 16; ++c)
@@ -217,16 +203,14 @@ struct MmaFp8Warp {
         red_l[r0] = l0;
       }
     }
-    if constexpr (TWO_ROWS) {
-      if (r1 < group) {
+    if (r1 < group) {
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c)
-          *reinterpret_cast<float4*>(red_acc + r1 * D + c * 16 + tig * 4) =
-              make_float4(acc[2 * c][2], acc[2 * c + 1][2], acc[2 * c][3], acc[2 * c + 1][3]);
-        if (tig == 0) {
-          red_m[r1] = m[1];
-          red_l[r1] = l1;
-        }
+      for (int c = 0; c < D / 16; ++c)
+        *reinterpret_cast<float4*>(red_acc + r1 * D + c * 16 + tig * 4) =
+            make_float4(acc[2 * c][2], acc[2 * c + 1][2], acc[2 * c][3], acc[2 * c + 1][3]);
+      if (tig == 0) {
+        red_m[r1] = m[1];
+        red_l[r1] = l1;
       }
     }
   }
@@ -288,8 +272,8 @@ struct MmaFp8WarpT {
     }
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const int s = MmaFp8Warp<D, BF16, false>::prescale_exp(mx);
-    const float f = MmaFp8Warp<D, BF16, false>::pow2(s);
+    const int s = query_prescale_exp(mx);
+    const float f = pow2i(s);
 #pragma unroll
     for (int kk = 0; kk < KSTEPS; ++kk) {
       qb[kk][0] = pack2<false>(v[kk].x * f, v[kk].y * f);
@@ -297,8 +281,8 @@ struct MmaFp8WarpT {
     }
     // the exponents of query rows 2t and 2t + 1 sit in lanes 8t and 8t + 4
     const int s0 = __shfl_sync(0xffffffffu, s, 8 * t), s1 = __shfl_sync(0xffffffffu, s, 8 * t + 4);
-    rs[0] = MmaFp8Warp<D, BF16, false>::pow2(-s0);
-    rs[1] = MmaFp8Warp<D, BF16, false>::pow2(-s1);
+    rs[0] = pow2i(-s0);
+    rs[1] = pow2i(-s1);
 #pragma unroll
     for (int i = 0; i < MTILES; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
     m[0] = m[1] = -INFINITY;

@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kThreads)
                                 const __grid_constant__ CUtensorMap vmap,
                                 const SharedPrefixArgs a) {
   using L = DecodeSmem<D, NST>;
-  using Warp = MmaWarp<D, BF16, true>;
+  using Warp = MmaWarp<D, BF16>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
