@@ -140,3 +140,32 @@ def report_parity(orc, workload: str, kernel: str, gpu_out: torch.Tensor, ref: n
         with open(path, "a", encoding="utf-8") as f:
             f.write(json.dumps(row) + "\n")
     return err
+
+
+# E4M3 caches for the fp8 tests: one scale per cache tensor
+K_SCALE, V_SCALE = 1.0 / 64, 1.0 / 32
+
+
+def fp8_batch(cfg: workloads.DecodeConfig, dev):
+    """A seeded batch whose caches are also held as E4M3 codes (torch's
+    float8_e4m3fn cast of x / scale, saturated to +-448)."""
+    b = workloads.make_batch(cfg, dev)
+    q8 = lambda t, s: (t.float() * (1.0 / s)).clamp(-448, 448).to(torch.float8_e4m3fn) \
+        .view(torch.uint8)
+    kc = q8(b.key_cache, K_SCALE).contiguous()
+    vc = q8(b.value_cache, V_SCALE).contiguous()
+    return b, kc, vc
+
+
+def fp8_oracle(orc, b: workloads.DecodeBatch, kc: torch.Tensor, vc: torch.Tensor):
+    """Oracle quantising write (on host copies of the E4M3 caches) then the
+    oracle's fp8 decode; returns (out float64, key codes after, value codes after)."""
+    cfg = b.cfg
+    kh = kc.cpu().numpy().copy()
+    vh = vc.cpu().numpy().copy()
+    assert orc.reshape_and_cache_fp8(bits(b.key), bits(b.value), kh, vh,
+                                     b.slot_mapping.cpu().numpy(), cfg.num_blocks,
+                                     cfg.block_size, K_SCALE, V_SCALE, ocode(cfg)) == 0
+    ref = orc.decode_fp8(bits(b.query), kh, vh, b.block_tables.cpu().numpy(),
+                         b.context_lens.cpu().numpy(), cfg.scale, K_SCALE, V_SCALE, ocode(cfg))
+    return ref, kh, vh

@@ -14,11 +14,11 @@ import oracle as oracle_mod
 from paged_kv_cache_444_b200 import (SplitWorkspace, pa_check_error, pa_decode_fp8,
                                      pa_decode_split_fp8, pa_reduce, pa_reshape_and_cache_fp8,
                                      workloads)
-from parity_helpers import TOL, bits, ocode, poison_past_context, to_f64
+from parity_helpers import (K_SCALE, V_SCALE, TOL, bits, fp8_batch as _fp8_batch,
+                            fp8_oracle as _oracle, ocode, poison_past_context, to_f64)
 
 pytestmark = pytest.mark.gpu
 
-K_SCALE, V_SCALE = 1.0 / 64, 1.0 / 32
 C = workloads.CONFIGS
 CASES = {
     "mha_f16": C["mha_llama2_7b"].scaled(num_seqs=5, num_heads=4, num_kv_heads=4, num_blocks=256,
@@ -39,27 +39,6 @@ CASES = {
     "gqa3_bf16": C["gqa_llama3_8b"].scaled(num_seqs=5, num_heads=12, num_kv_heads=4,
                                            num_blocks=300, ctx=("uniform", 1, 800), seed=57),
 }
-
-
-def _fp8_batch(cfg, dev):
-    b = workloads.make_batch(cfg, dev)
-    q8 = lambda t, s: (t.float() * (1.0 / s)).clamp(-448, 448).to(torch.float8_e4m3fn) \
-        .view(torch.uint8)
-    kc = q8(b.key_cache, K_SCALE).contiguous()
-    vc = q8(b.value_cache, V_SCALE).contiguous()
-    return b, kc, vc
-
-
-def _oracle(orc, b, kc, vc):
-    cfg = b.cfg
-    kh = kc.cpu().numpy().copy()
-    vh = vc.cpu().numpy().copy()
-    assert orc.reshape_and_cache_fp8(bits(b.key), bits(b.value), kh, vh,
-                                     b.slot_mapping.cpu().numpy(), cfg.num_blocks,
-                                     cfg.block_size, K_SCALE, V_SCALE, ocode(cfg)) == 0
-    ref = orc.decode_fp8(bits(b.query), kh, vh, b.block_tables.cpu().numpy(),
-                         b.context_lens.cpu().numpy(), cfg.scale, K_SCALE, V_SCALE, ocode(cfg))
-    return ref, kh, vh
 
 
 @pytest.mark.parametrize("name", list(CASES))

@@ -12,8 +12,8 @@ import torch
 from paged_kv_cache_444_b200 import (SplitWorkspace, pa_check_error, pa_decode_fp8,
                                      pa_decode_split_fp8, pa_reduce, pa_reshape_and_cache_fp8,
                                      workloads)
-from parity_helpers import TOL, HostCopy, gpu_step, oracle_step, to_f64
-from test_gpu_fp8 import K_SCALE, V_SCALE, _fp8_batch, _oracle
+from parity_helpers import (K_SCALE, V_SCALE, TOL, HostCopy, fp8_batch, fp8_oracle, gpu_step,
+                            oracle_step, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -56,8 +56,8 @@ def test_sweep_16bit_matches_oracle(i, cuda_device, oracle_lib):
 @pytest.mark.parametrize("i", range(10))
 def test_sweep_fp8_matches_oracle(i, cuda_device, oracle_lib):
     cfg, ps = _layout(100 + i, head_dims=(128,))
-    b, kc, vc = _fp8_batch(cfg, cuda_device)
-    ref, _, _ = _oracle(oracle_lib, b, kc, vc)
+    b, kc, vc = fp8_batch(cfg, cuda_device)
+    ref, _, _ = fp8_oracle(oracle_lib, b, kc, vc)
     pa_reshape_and_cache_fp8(b.key, b.value, kc, vc, b.slot_mapping, K_SCALE, V_SCALE)
     out = torch.full_like(b.query, float("nan"))
     if ps:
