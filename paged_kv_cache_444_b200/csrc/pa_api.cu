@@ -152,7 +152,7 @@ constexpr long long kPersistWaves = 64;
 #define PA_CLUSTER_TABLE_PAGES 512  // clusters only when a table can hold more pages
 #endif
 #ifndef PA_CLUSTER_FILL_PAGES
-#define PA_CLUSTER_FILL_PAGES 64  // fewer items than resident CTAs: spread items longer than this
+#define PA_CLUSTER_FILL_PAGES 32  // fewer items than resident CTAs: spread items longer than this
 #endif
 
 // Cluster size for a single-pass launch.  Clusters are used only when the
@@ -257,7 +257,7 @@ pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeAr
     // fewer items than CTAs resident at once leave slots idle: the items
     // longer than PA_CLUSTER_FILL_PAGES are spread over CTA pairs so that
     // they use them (the fp8 beam batch, 512 items on 592 slots: the longest
-    // items bound the launch, 47.2 -> 41.1 us)
+    // items bound the launch, 47.1 -> 39.0 us)
     static std::atomic<long long> fill_resident[kMaxDevices] = {};
     const long long resident = resident_ctas(kernel, L::kAlloc, fill_resident);
     if (resident > 0 && grid < resident) {
