@@ -152,15 +152,15 @@ constexpr long long kPersistWaves = 64;
 #define PA_CLUSTER_TABLE_PAGES 512  // clusters only when a table can hold more pages
 #endif
 #ifndef PA_CLUSTER_FILL_PAGES
-#define PA_CLUSTER_FILL_PAGES 32  // fewer items than resident CTAs: spread items longer than this
+#define PA_CLUSTER_FILL_PAGES 32  // pairs fit in the resident slots: spread items longer than this
 #endif
 
 // Cluster size for a single-pass launch.  Clusters are used only when the
 // block table admits very long sequences (more than PA_CLUSTER_TABLE_PAGES
 // pages): then every item longer than PA_CLUSTER_PAGES pages is spread so that
 // the longest possible one gives each CTA about PA_CLUSTER_TABLE_PAGES pages.
-// (launch_decode_t also asks for pairs when the grid leaves resident CTA slots
-// idle.)  A power of two, at most kMaxCluster, and no more than the device can
+// (launch_decode_t also asks for pairs when twice the grid fits in the
+// resident CTA slots.)  A power of two, at most kMaxCluster, and no more than the device can
 // co-schedule for this kernel.
 template <class K>
 int pick_cluster(K kernel, int smem_bytes, int64_t max_pages, std::atomic<int>* cache) {
@@ -254,13 +254,14 @@ pa_status launch_decode_t(const CUtensorMap& km, const CUtensorMap& vm, DecodeAr
   int c = split ? 1 : pick_cluster(kernel, L::kAlloc, max_pages, cluster_cache);
   a.cluster_pages = PA_CLUSTER_PAGES;
   if (!split && c == 1 && max_pages > PA_CLUSTER_FILL_PAGES) {
-    // fewer items than CTAs resident at once leave slots idle: the items
-    // longer than PA_CLUSTER_FILL_PAGES are spread over CTA pairs so that
-    // they use them (the fp8 beam batch, 512 items on 592 slots: the longest
-    // items bound the launch, 47.1 -> 39.0 us)
+    // a grid whose CTA pairs all fit in the resident slots leaves half of
+    // them idle: the items longer than PA_CLUSTER_FILL_PAGES are spread over
+    // pairs so that they use them (32 fp8 sequences x 8 KV heads on 592
+    // slots: 51.2 -> 40.6 us).  With more items some pairs would wait for a
+    // second wave, which measured up to 39 % slower on uniform batches
     static std::atomic<long long> fill_resident[kMaxDevices] = {};
     const long long resident = resident_ctas(kernel, L::kAlloc, fill_resident);
-    if (resident > 0 && grid < resident) {
+    if (resident > 0 && 2 * grid <= resident) {
       c = pick_cluster(kernel, L::kAlloc, 2 * static_cast<int64_t>(PA_CLUSTER_TABLE_PAGES),
                        cluster_cache);
       a.cluster_pages = PA_CLUSTER_FILL_PAGES;
