@@ -281,9 +281,11 @@ struct MmaWarpT {
   static constexpr int kMinBlocks = 0;
   static constexpr int KSTEPS = D / 16;
   static constexpr int MTILES = D / 16;
+  static constexpr float kSlack = 8.f;  // log2 units the reference max may trail by
   uint32_t qb[KSTEPS][2];  // Q^T B fragments of query row lane / 4
   float acc[MTILES][4];    // O^T: (dim 16c + g, rows 2t, 2t+1), (dim 16c + 8 + g, ...)
-  float m[2], l[2];        // query rows 2t, 2t+1
+  float m[2], l[2];        // query rows 2t, 2t+1: reference max (log2), lane-partial sum
+  float mt[2];             // and their true running max
 
   __device__ __forceinline__ void init(const uint16_t* q_group, int group, int lane) {
     const int g = lane >> 2, t = lane & 3;
@@ -295,7 +297,7 @@ struct MmaWarpT {
     }
 #pragma unroll
     for (int i = 0; i < MTILES; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    m[0] = m[1] = -INFINITY;
+    m[0] = m[1] = mt[0] = mt[1] = -INFINITY;
     l[0] = l[1] = 0.f;
   }
 
@@ -330,15 +332,29 @@ struct MmaWarpT {
     keep = fmaxf(keep, __shfl_xor_sync(0xffffffffu, keep, 8));
     keep = fmaxf(keep, __shfl_xor_sync(0xffffffffu, keep, 16));
     const float other = __shfl_xor_sync(0xffffffffu, keep, 4);
-    const float mn0 = fmaxf(m[0], odd ? other : keep);
-    const float mn1 = fmaxf(m[1], odd ? keep : other);
-    const float al0 = ex2(m[0] - mn0), al1 = ex2(m[1] - mn1);
-    m[0] = mn0;
-    m[1] = mn1;
+    mt[0] = fmaxf(mt[0], odd ? other : keep);
+    mt[1] = fmaxf(mt[1], odd ? keep : other);
+    // The reference max m trails the true one by at most 2^kSlack, so P stays
+    // at most 2^8; O and l are rescaled only when some row of the warp
+    // outgrows that, a branch the whole warp takes.
+    if (__any_sync(0xffffffffu, (mt[0] > m[0] + kSlack) | (mt[1] > m[1] + kSlack))) {
+      const float al0 = ex2(m[0] - mt[0]), al1 = ex2(m[1] - mt[1]);
+      m[0] = mt[0];
+      m[1] = mt[1];
+      l[0] *= al0;
+      l[1] *= al1;
+#pragma unroll
+      for (int i = 0; i < MTILES; ++i) {
+        acc[i][0] *= al0;
+        acc[i][1] *= al1;
+        acc[i][2] *= al0;
+        acc[i][3] *= al1;
+      }
+    }
     // ---- P in the cache dtype as the B operand of the second product: fp16 P
     // once (l sums the rounded values), bf16 P as a hi + lo pair (l sums the
     // fp32 p) ----
-    const float p0 = ex2(x0 - mn0), p1 = ex2(x1 - mn1), p2 = ex2(x2 - mn0), p3 = ex2(x3 - mn1);
+    const float p0 = ex2(x0 - m[0]), p1 = ex2(x1 - m[1]), p2 = ex2(x2 - m[0]), p3 = ex2(x3 - m[1]);
     const uint32_t h_lo = pack2<BF16>(p0, p1), h_hi = pack2<BF16>(p2, p3);
     uint32_t pb[4];
     pb[0] = movmatrix_trans(h_lo);
@@ -347,19 +363,12 @@ struct MmaWarpT {
       const float2 u = unpack2<true>(h_lo), w = unpack2<true>(h_hi);
       pb[2] = movmatrix_trans(pack2<true>(p0 - u.x, p1 - u.y));
       pb[3] = movmatrix_trans(pack2<true>(p2 - w.x, p3 - w.y));
-      l[0] = l[0] * al0 + (p0 + p2);
-      l[1] = l[1] * al1 + (p1 + p3);
+      l[0] += p0 + p2;
+      l[1] += p1 + p3;
     } else {
       const float2 u = unpack2<false>(h_lo), w = unpack2<false>(h_hi);
-      l[0] = l[0] * al0 + (u.x + w.x);
-      l[1] = l[1] * al1 + (u.y + w.y);
-    }
-#pragma unroll
-    for (int i = 0; i < MTILES; ++i) {
-      acc[i][0] *= al0;
-      acc[i][1] *= al1;
-      acc[i][2] *= al0;
-      acc[i][3] *= al1;
+      l[0] += u.x + w.x;
+      l[1] += u.y + w.y;
     }
     // ---- O^T += V^T P^T ----
     const int vtok = (lane & 7) + (lane >> 4) * 8;
@@ -373,10 +382,14 @@ struct MmaWarpT {
     }
   }
 
+  // The partials are restated against the true max (a factor <= 1).
   __device__ __forceinline__ void publish(float* red_acc, float* red_m, float* red_l, int group,
                                           int lane) {
     const int g = lane >> 2, t = lane & 3;
-    float l0 = l[0], l1 = l[1];
+    float f[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) f[h] = mt[h] > -INFINITY ? ex2(m[h] - mt[h]) : 1.f;
+    float l0 = l[0] * f[0], l1 = l[1] * f[1];
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -388,11 +401,11 @@ struct MmaWarpT {
       if (row < group) {
 #pragma unroll
         for (int c = 0; c < MTILES; ++c) {
-          red_acc[row * D + 16 * c + g] = acc[c][h];
-          red_acc[row * D + 16 * c + 8 + g] = acc[c][2 + h];
+          red_acc[row * D + 16 * c + g] = acc[c][h] * f[h];
+          red_acc[row * D + 16 * c + 8 + g] = acc[c][2 + h] * f[h];
         }
         if (g == 0) {
-          red_m[row] = m[h];
+          red_m[row] = mt[h];
           red_l[row] = h ? l1 : l0;
         }
       }

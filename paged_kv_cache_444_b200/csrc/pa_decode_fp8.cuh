@@ -252,9 +252,11 @@ struct MmaFp8WarpT {
   static constexpr int kMinBlocks = 4;  // CTAs per SM the register budget is built for
   static constexpr int KSTEPS = D / 16;
   static constexpr int MTILES = D / 16;
+  static constexpr float kSlack = 8.f;  // log2 units the reference max may trail by
   uint32_t qb[KSTEPS][2];  // fp16 Q^T fragments of query row lane / 4
   float acc[MTILES][4];    // O^T: (m-tile row g, query row 2t | 2t+1), (row g + 8, ...)
-  float m[2], l[2];        // query rows 2t, 2t+1: running max (log2), lane-partial sum
+  float m[2], l[2];        // query rows 2t, 2t+1: reference max (log2), lane-partial sum
+  float mt[2];             // and their true running max
   float rs[2];             // 2^-s of query rows 2t, 2t+1 (undo the query prescale)
 
   __device__ __forceinline__ void init(const uint16_t* q_group, int group, int lane) {
@@ -285,7 +287,7 @@ struct MmaFp8WarpT {
     rs[1] = pow2i(-s1);
 #pragma unroll
     for (int i = 0; i < MTILES; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    m[0] = m[1] = -INFINITY;
+    m[0] = m[1] = mt[0] = mt[1] = -INFINITY;
     l[0] = l[1] = 0.f;
   }
 
@@ -326,28 +328,35 @@ struct MmaFp8WarpT {
     keep = fmaxf(keep, __shfl_xor_sync(0xffffffffu, keep, 8));
     keep = fmaxf(keep, __shfl_xor_sync(0xffffffffu, keep, 16));
     const float other = __shfl_xor_sync(0xffffffffu, keep, 4);
-    const float mn0 = fmaxf(m[0], odd ? other : keep);
-    const float mn1 = fmaxf(m[1], odd ? keep : other);
-    const float al0 = ex2(m[0] - mn0), al1 = ex2(m[1] - mn1);
-    m[0] = mn0;
-    m[1] = mn1;
+    mt[0] = fmaxf(mt[0], odd ? other : keep);
+    mt[1] = fmaxf(mt[1], odd ? keep : other);
+    // The reference max m trails the true one by at most 2^kSlack, so P stays
+    // at most 2^8 (exact in fp16 up to its 11 bits); O and l are rescaled only
+    // when some row of the warp outgrows that, a branch the whole warp takes.
+    if (__any_sync(0xffffffffu, (mt[0] > m[0] + kSlack) | (mt[1] > m[1] + kSlack))) {
+      const float al0 = ex2(m[0] - mt[0]), al1 = ex2(m[1] - mt[1]);
+      m[0] = mt[0];
+      m[1] = mt[1];
+      l[0] *= al0;
+      l[1] *= al1;
+#pragma unroll
+      for (int i = 0; i < MTILES; ++i) {
+        acc[i][0] *= al0;
+        acc[i][1] *= al1;
+        acc[i][2] *= al0;
+        acc[i][3] *= al1;
+      }
+    }
     // ---- P in fp16, l sums the same rounded values, then P^T as a B operand ----
-    const uint32_t p_lo = pack2<false>(ex2(x0 - mn0), ex2(x1 - mn1));  // token g
-    const uint32_t p_hi = pack2<false>(ex2(x2 - mn0), ex2(x3 - mn1));  // token g + 8
+    const uint32_t p_lo = pack2<false>(ex2(x0 - m[0]), ex2(x1 - m[1]));  // token g
+    const uint32_t p_hi = pack2<false>(ex2(x2 - m[0]), ex2(x3 - m[1]));  // token g + 8
     {
       const float2 u = unpack2<false>(p_lo), w = unpack2<false>(p_hi);
-      l[0] = l[0] * al0 + (u.x + w.x);
-      l[1] = l[1] * al1 + (u.y + w.y);
+      l[0] += u.x + w.x;
+      l[1] += u.y + w.y;
     }
     const uint32_t pb0 = movmatrix_trans(p_lo);  // tokens 2t, 2t+1 of query row g
     const uint32_t pb1 = movmatrix_trans(p_hi);  // tokens 2t+8, 2t+9
-#pragma unroll
-    for (int i = 0; i < MTILES; ++i) {
-      acc[i][0] *= al0;
-      acc[i][1] *= al1;
-      acc[i][2] *= al0;
-      acc[i][3] *= al1;
-    }
     // ---- O^T += V^T P^T: one transposed x4 ldmatrix covers two 16-dim chunks ----
 #pragma unroll
     for (int cp = 0; cp < D / 32; ++cp) {
@@ -365,10 +374,14 @@ struct MmaFp8WarpT {
   }
 
   // Query rows < group into the merge buffers, head dims in order.
+  // The partials are restated against the true max (a factor <= 1).
   __device__ __forceinline__ void publish(float* red_acc, float* red_m, float* red_l, int group,
                                           int lane) {
     const int g = lane >> 2, t = lane & 3;
-    float l0 = l[0], l1 = l[1];
+    float f[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) f[h] = mt[h] > -INFINITY ? ex2(m[h] - mt[h]) : 1.f;
+    float l0 = l[0] * f[0], l1 = l[1] * f[1];
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -381,12 +394,13 @@ struct MmaFp8WarpT {
 #pragma unroll
         for (int cp = 0; cp < D / 32; ++cp) {
           float* o = red_acc + row * D + cp * 32 + 2 * g;
-          *reinterpret_cast<float2*>(o) = make_float2(acc[2 * cp][h], acc[2 * cp + 1][h]);
+          *reinterpret_cast<float2*>(o) =
+              make_float2(acc[2 * cp][h] * f[h], acc[2 * cp + 1][h] * f[h]);
           *reinterpret_cast<float2*>(o + 16) =
-              make_float2(acc[2 * cp][2 + h], acc[2 * cp + 1][2 + h]);
+              make_float2(acc[2 * cp][2 + h] * f[h], acc[2 * cp + 1][2 + h] * f[h]);
         }
         if (g == 0) {
-          red_m[row] = m[h];
+          red_m[row] = mt[h];
           red_l[row] = h ? l1 : l0;
         }
       }
