@@ -732,25 +732,28 @@ __global__ void __launch_bounds__(kThreads, Warp::kMinBlocks)
 
   // ---- longest-first order: grid slot s takes the s-th longest sequence
   // (ties by index), so that long items start first and short ones fill the
-  // tail.  The rank of every sequence is counted against all others. ----
+  // tail.  The rank of every sequence is counted against all others, on keys
+  // (length << 8 | 255 - index) that order both at once. ----
   if (a.longest_first) {
-    int* lens = reinterpret_cast<int*>(smem);      // stage area, not in use yet
-    int* chosen = lens + kLptMaxSeqs;
+    unsigned* keys = reinterpret_cast<unsigned*>(smem);  // stage area, not in use yet
+    int* chosen = reinterpret_cast<int*>(keys + kLptMaxSeqs);
     const int n4 = (a.num_seqs + 3) >> 2;
-    for (int i = threadIdx.x; i < n4 * 4; i += kThreads)
-      lens[i] = i < a.num_seqs ? max(a.context_lens[i], 0) : -1;  // -1 pads: never counted
+    const unsigned lcap = static_cast<unsigned>(min(cap, (1 << 24) - 1));
+    for (int i = threadIdx.x; i < n4 * 4; i += kThreads) {
+      unsigned key = 0u;  // pads: below every sequence's key, never counted
+      if (i < a.num_seqs)
+        key = (min(static_cast<unsigned>(max(a.context_lens[i], 0)), lcap) << 8) |
+              static_cast<unsigned>(255 - i);
+      keys[i] = key;
+    }
     __syncthreads();
-    const int4* lens4 = reinterpret_cast<const int4*>(lens);
+    const uint4* keys4 = reinterpret_cast<const uint4*>(keys);
     for (int t = threadIdx.x; t < a.num_seqs; t += kThreads) {
-      const int lt = lens[t];
+      const unsigned kt = keys[t];
       int rank = 0;
       for (int j4 = 0; j4 < n4; ++j4) {
-        const int4 v = lens4[j4];
-        const int j = j4 * 4;
-        rank += (v.x > lt) | ((v.x == lt) & (j < t));
-        rank += (v.y > lt) | ((v.y == lt) & (j + 1 < t));
-        rank += (v.z > lt) | ((v.z == lt) & (j + 2 < t));
-        rank += (v.w > lt) | ((v.w == lt) & (j + 3 < t));
+        const uint4 v = keys4[j4];
+        rank += (v.x > kt) + (v.y > kt) + (v.z > kt) + (v.w > kt);
       }
       if (rank == s) *chosen = t;
     }
