@@ -31,7 +31,10 @@
 // (MmaWarp), which the shared-prefix kernel also uses.  Even for one head the
 // tensor cores take the products off the issue path, which measured faster
 // than packed fp32 FMA on the CUDA cores.  The softmax is online, in base 2
-// with scale*log2(e) folded into the logits, with warp-shuffle max reductions.
+// with scale*log2(e) folded into the logits, with warp-shuffle max reductions;
+// in the transposed steps the reference max may trail the true one by 2^8, so
+// O is rescaled only when a row outgrows that, and the partials are restated
+// against the true max at the end.
 #pragma once
 
 #include "pa_device.cuh"
