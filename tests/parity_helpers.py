@@ -146,10 +146,50 @@ def report_parity(orc, workload: str, kernel: str, gpu_out: torch.Tensor, ref: n
 K_SCALE, V_SCALE = 1.0 / 64, 1.0 / 32
 
 
-def fp8_batch(cfg: workloads.DecodeConfig, dev):
+def grow_logits(batch: workloads.DecodeBatch, step: float = 7.0, every: int = 64,
+                max_steps: int = 1 << 30) -> float:
+    """Rewrite the key cache so that, for every sequence and KV head, the
+    logit of the group's first query head climbs by about `step` (natural
+    units; 7 is 10 log2 units) every `every` tokens: key row j becomes a
+    quarter of its random self plus c_j times that query's unit vector, with
+    c_j * |q| * scale = step * min(j // every, max_steps) (a cap keeps E4M3
+    codes of the rows below saturation).  The running maximum then jumps
+    past any slack of 2^8 several times along each sequence.  Block tables
+    must not share blocks between sequences.  Returns the largest climb
+    (natural units) seen by one (sequence, head)."""
+    cfg = batch.cfg
+    G = cfg.num_heads // cfg.num_kv_heads
+    kc = batch.key_cache.float()
+    bt = batch.block_tables.cpu()
+    cl = batch.context_lens.cpu().tolist()
+    dev = kc.device
+    top = 0.0
+    for s, n in enumerate(cl):
+        if n <= 0:
+            continue
+        j = torch.arange(n)
+        blocks = bt[s, j // cfg.block_size].to(dev)
+        rows = (j % cfg.block_size).to(dev)
+        for h in range(cfg.num_kv_heads):
+            q = batch.query[s, h * G].float()
+            qn = float(q.norm())
+            if qn == 0.0:
+                continue
+            k = torch.clamp(j // every, max=max_steps).to(torch.float32)
+            c = (step * k / (qn * cfg.scale)).to(dev)
+            kc[blocks, rows, h] = 0.25 * kc[blocks, rows, h] + c[:, None] * (q / qn)[None, :]
+            top = max(top, step * min((n - 1) // every, max_steps))
+    batch.key_cache.copy_(kc.to(batch.key_cache.dtype))
+    return top
+
+
+def fp8_batch(cfg: workloads.DecodeConfig, dev, prepare=None):
     """A seeded batch whose caches are also held as E4M3 codes (torch's
-    float8_e4m3fn cast of x / scale, saturated to +-448)."""
+    float8_e4m3fn cast of x / scale, saturated to +-448).  `prepare(batch)`,
+    if given, edits the 16-bit batch before the codes are taken."""
     b = workloads.make_batch(cfg, dev)
+    if prepare is not None:
+        prepare(b)
     q8 = lambda t, s: (t.float() * (1.0 / s)).clamp(-448, 448).to(torch.float8_e4m3fn) \
         .view(torch.uint8)
     kc = q8(b.key_cache, K_SCALE).contiguous()

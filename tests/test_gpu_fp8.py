@@ -15,7 +15,8 @@ from paged_kv_cache_444_b200 import (SplitWorkspace, pa_check_error, pa_decode_f
                                      pa_decode_split_fp8, pa_reduce, pa_reshape_and_cache_fp8,
                                      workloads)
 from parity_helpers import (K_SCALE, V_SCALE, TOL, bits, fp8_batch as _fp8_batch,
-                            fp8_oracle as _oracle, ocode, poison_past_context, to_f64)
+                            fp8_oracle as _oracle, grow_logits, ocode, poison_past_context,
+                            to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +58,37 @@ def test_fp8_write_and_decode_match_oracle(name, cuda_device, oracle_lib):
     assert np.isfinite(g).all()
     err = np.max(np.abs(g - ref))
     assert err <= TOL[cfg.dtype], f"{name}: {err:.3e}"
+
+
+@pytest.mark.parametrize("ps", [0, 256])
+@pytest.mark.parametrize("name", ["mha_f16", "gqa_bf16", "gqa8_f16", "gqa16_bf16"])
+def test_fp8_growing_logits_force_the_rescale(name, ps, cuda_device, oracle_lib):
+    """Logits that climb by about 10 log2 units every 4 pages (three climbs,
+    which keeps the key codes below saturation): the page step rescales O and
+    l mid-sequence and restates its partials against the true maximum."""
+    cfg = CASES[name]
+    top = []
+    b, kc, vc = _fp8_batch(cfg, cuda_device,
+                           prepare=lambda bb: top.append(grow_logits(bb, max_steps=3)))
+    assert top[0] >= 14.0
+    ref, _, _ = _oracle(oracle_lib, b, kc, vc)
+    pa_reshape_and_cache_fp8(b.key, b.value, kc, vc, b.slot_mapping, K_SCALE, V_SCALE)
+    out = torch.full_like(b.query, float("nan"))
+    if ps:
+        P = (b.block_tables.shape[1] * 16 + ps - 1) // ps
+        ws = SplitWorkspace(cfg.num_seqs, cfg.num_heads, cfg.head_dim, P, cuda_device)
+        pa_decode_split_fp8(ws.tmp_out, ws.max_logits, ws.exp_sums, b.query, kc, vc,
+                            b.block_tables, b.context_lens, cfg.scale, K_SCALE, V_SCALE, ps)
+        pa_reduce(out, ws.tmp_out, ws.max_logits, ws.exp_sums, b.context_lens, ps)
+    else:
+        pa_decode_fp8(out, b.query, kc, vc, b.block_tables, b.context_lens, cfg.scale, K_SCALE,
+                      V_SCALE)
+    torch.cuda.synchronize()
+    pa_check_error()
+    g = to_f64(out)
+    assert np.isfinite(g).all()
+    err = np.max(np.abs(g - ref))
+    assert err <= TOL[cfg.dtype], f"{name} growing logits, split {ps}: {err:.3e}"
 
 
 @pytest.mark.parametrize("name", ["gqa_bf16", "mha_f16", "gqa8_f16", "gqa3_bf16"])

@@ -7,7 +7,7 @@ import pytest
 import torch
 
 from paged_kv_cache_444_b200 import PagedAttentionError, pa_check_error, workloads
-from parity_helpers import (TOL, HostCopy, bits, gpu_step, max_err, oracle_step,
+from parity_helpers import (TOL, HostCopy, bits, gpu_step, grow_logits, max_err, oracle_step,
                             poison_past_context, to_f64)
 
 pytestmark = pytest.mark.gpu
@@ -112,6 +112,25 @@ def _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, ps):
     na = acc / psum[..., None]
     ng = ga / gs[..., None]
     assert np.nanmax(np.abs(na - ng)[valid]) <= TOL[cfg.dtype]
+
+
+@pytest.mark.parametrize("ps", [0, 256])
+@pytest.mark.parametrize("name", ["mha_small", "gqa_small", "gqa8", "mha_bf16", "gqa16_two_rows"])
+def test_growing_logits_force_the_rescale(name, ps, dev, oracle_lib):
+    """Logits that climb by about 10 log2 units every 4 pages: the running
+    maximum outgrows the page step's slack again and again, so O and l are
+    rescaled mid-sequence and the published partials are restated against
+    the true maximum.  Output (and the split's partials) against the oracle."""
+    cfg = SMALL[name]
+    batch = workloads.make_batch(cfg, dev)
+    assert grow_logits(batch) >= 14.0  # at least two climbs past the slack
+    host = HostCopy(batch)
+    ref, kc_ref, vc_ref = oracle_step(oracle_lib, host)
+    out, ws = gpu_step(batch, partition_size=ps)
+    pa_check_error()
+    _check_close(out, ref, cfg, f"{name} growing logits, split {ps}")
+    if ps:
+        _check_partials(oracle_lib, host, kc_ref, vc_ref, cfg, ws, ps)
 
 
 def test_split_over_full_grid_for_many_sequences(dev, oracle_lib):
