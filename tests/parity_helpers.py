@@ -154,9 +154,10 @@ def grow_logits(batch: workloads.DecodeBatch, step: float = 7.0, every: int = 64
     quarter of its random self plus c_j times that query's unit vector, with
     c_j * |q| * scale = step * min(j // every, max_steps) (a cap keeps E4M3
     codes of the rows below saturation).  The running maximum then jumps
-    past any slack of 2^8 several times along each sequence.  Block tables
-    must not share blocks between sequences.  Returns the largest climb
-    (natural units) seen by one (sequence, head)."""
+    past any slack of 2^8 several times along each sequence.  A block that
+    several sequences share keeps the last one's rewrite (the cache stays one
+    consistent input for both sides).  Returns the largest climb (natural
+    units) planned for one (sequence, head)."""
     cfg = batch.cfg
     G = cfg.num_heads // cfg.num_kv_heads
     kc = batch.key_cache.float()

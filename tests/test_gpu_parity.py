@@ -330,6 +330,25 @@ SHARED_CASES = {
 }
 
 
+@pytest.mark.parametrize("name", ["beam4_gqa4", "gqa8_chunked", "long_prefix_spread"])
+def test_shared_prefix_growing_logits(name, dev, oracle_lib):
+    """The shared-prefix kernel with key rows whose logits climb by about 10
+    log2 units every 4 pages (members sharing a prefix block keep the last
+    member's rewrite of it): its page step rescales O mid-sequence, on shared
+    and private pages.  Against the oracle."""
+    base, over, starts, prefix = SHARED_CASES[name]
+    cfg = SMALL[base].scaled(**over) if over else SMALL[base]
+    batch = workloads.make_batch(cfg, dev)
+    if starts is not None:
+        batch = _regroup(batch, starts, prefix)
+    assert grow_logits(batch) >= 14.0
+    host = HostCopy(batch)
+    ref, _, _ = oracle_step(oracle_lib, host)
+    out, _ = gpu_step(batch, shared_prefix=True)
+    pa_check_error()
+    _check_close(out, ref, cfg, f"{name} shared prefix, growing logits")
+
+
 @pytest.mark.parametrize("name", list(SHARED_CASES))
 def test_shared_prefix_matches_oracle(name, dev, oracle_lib):
     base, over, starts, prefix = SHARED_CASES[name]
